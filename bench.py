@@ -1,0 +1,386 @@
+"""Benchmark: layer-streamed NF4 LoRA linears, fwd + bwd, on the Llama-3.1-8B
+shaped stack (32 layers x 7 projections, T = 2048 tokens, r = 16, alpha = 32,
+NF4 base streamed from pinned host RAM through a 2-slot VRAM pool).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = forward over layers 0..31 then backward over 31..0, every
+projection through lora_linear_fwd / lora_linear_bwd of the C ABI, base
+weights streamed by the layer pool.  Prints ONE JSON line (rank 0).
+
+--impl reference times the CPU oracle (fp64, host cores) on a bounded sample
+of the same workload and prints the same metric.  With N > 1 every rank runs
+an independent replica (weak scaling; the method has no exchange step).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "train tok/s, 8B-shape NF4 LoRA fwd+bwd; % of bf16 tensor-core peak"
+UNIT = "tok/s"
+WORKLOAD = "8b"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sms, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sms.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sms:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        loaded = [v for v in sms if mx is None or v >= 0.3 * mx] or sms
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sms)}
+
+
+def _dist():
+    n = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return n, rank, local
+
+
+# ----------------------------------------------------------------- ours ---
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from layer_streamed_nf4_b200 import lsnf4, synth
+    from layer_streamed_nf4_b200.stack import Stack
+
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+    cfg = synth.STACKS[WORKLOAD]
+    T = args.tokens or cfg.tokens
+    L = args.layers or cfg.layers
+    stream = torch.cuda.Stream()
+    peaks = _peaks()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    results = {}
+    kernel = None
+    pool_stats = None
+    clocks = None
+    st_main = Stack(cfg, layers=L, tokens=T, mode="streamed", n_slots=args.slots, seed=synth.SEED + rank,
+                    stream=stream)
+    modes = ["streamed"] + [m for m in ("no_h2d", "resident") if m in args.modes]
+    for mode in modes:
+        st = st_main if mode == "streamed" else st_main.with_mode(mode)
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                st.step()
+        stream.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        if mode == "streamed":
+            lsnf4.timing_enable(True)
+            ps0 = st.pool_stats()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        sampler = ClockSampler(local) if mode == "streamed" else None
+        if sampler:
+            sampler.__enter__()
+        with torch.cuda.stream(stream):
+            t0.record(stream)
+            for _ in range(args.steps):
+                st.step()
+            t1.record(stream)
+        t1.synchronize()
+        if sampler:
+            sampler.__exit__()
+            clocks = sampler.summary()
+        torch.cuda.synchronize()
+        barrier()
+        ms = t0.elapsed_time(t1) / args.steps
+        ms = max_over_ranks(ms)
+        results[mode] = ms
+        if mode == "streamed":
+            kernel = lsnf4.timing_read()
+            lsnf4.timing_enable(False)
+            ps1 = st.pool_stats()
+            pool_stats = {k: ps1[k] - ps0[k] for k in ps1}
+        st.check_status()
+        if st is not st_main:
+            st.close()
+
+    # End to end through the public API with host buffers: every step copies
+    # its input hidden states (layer-0 projection inputs) from pinned host
+    # memory and reads the step's result (layer-0 input gradients) back.
+    e2e = None
+    if not args.no_e2e:
+        st = st_main
+        ins = [st.x[0, pi] for pi in range(len(st.proj))]
+        outs = [st.dX[0, pi] for pi in range(len(st.proj))]
+        h_in = [torch.empty_like(t, device="cpu").pin_memory() for t in ins]
+        h_out = [torch.empty_like(t, device="cpu").pin_memory() for t in outs]
+        for h, t in zip(h_in, ins):
+            h.copy_(t)
+        bi = sum(t.numel() * t.element_size() for t in ins)
+        bo = sum(t.numel() * t.element_size() for t in outs)
+        torch.cuda.synchronize()
+        barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        ps0 = st.pool_stats() or {"bytes_copied": 0}
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.steps):
+                for h, t in zip(h_in, ins):
+                    t.copy_(h, non_blocking=True)
+                st.step()
+                for h, t in zip(h_out, outs):
+                    h.copy_(t, non_blocking=True)
+            e1.record(stream)
+        e1.synchronize()
+        barrier()
+        ems = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+        ps = st.pool_stats() or {"bytes_copied": 0}
+        e2e = {"value": world * T / (ems / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": int(bi + (ps["bytes_copied"] - ps0["bytes_copied"]) / max(args.steps, 1)),
+               "d2h_bytes_per_step": int(bo), "ms_per_step": ems}
+
+    st_main.check_status()
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        st_main.close()
+        return
+
+    ms = results["streamed"]
+    flop_step = st_main.flop_per_step()
+    value = world * T / (ms / 1e3)
+
+    g = {k: kernel[k] for k in ("gemm_fwd", "gemm_bwd")}
+    g_ms = sum(v["ms"] for v in g.values())
+    g_flop = sum(v["work"] for v in g.values())
+    g_launch = sum(v["launches"] for v in g.values())
+    achieved = g_flop / (g_ms / 1e3) / 1e12 if g_ms > 0 else 0.0
+    peak = peaks["bf16_tflops_sustained"]
+    launches = sum(v["kernels"] for v in kernel.values())
+    step_kernel_ms = sum(v["ms"] for v in kernel.values()) / args.steps
+    dq = kernel["dequant"]
+    h2d_gbs = (pool_stats["bytes_copied"] / (pool_stats["copy_ms"] / 1e3) / 1e9
+               if pool_stats and pool_stats["copy_ms"] > 0 else None)
+    extra_modes = {m: {"ms_per_step": results[m], "tok_s": world * T / (results[m] / 1e3),
+                       "pct_bf16_peak": 100 * flop_step / (results[m] / 1e3) / 1e12 / peaks["bf16_tflops"]}
+                   for m in results}
+    traffic = _traffic_from_profile()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{cfg.name} NF4 LoRA stack: {L} layers x 7 projections (q,k,v,o,gate,up,down), "
+                               f"T={T} tokens (batch 1 x seq {T}), r={cfg.rank}, alpha={cfg.alpha:g}, "
+                               f"base NF4 blk-64 + double quant streamed from pinned host RAM, "
+                               f"{args.slots}-slot VRAM pool",
+                   "tokens": T, "layers": L, "rank": cfg.rank, "pool_slots": args.slots, "base": cfg.base,
+                   "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (per step ~11 GB of activations, ~3.6 GB of streamed weights)"},
+        "pct_bf16_peak": 100 * flop_step / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+        "flop_per_step": flop_step,
+        "modes": extra_modes,
+        "roofline": {"bound": "tensor", "kernel": "lsn_gemm_kernel (fwd y and bwd dX GEMMs)",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"{peaks['source']} bf16_tflops_sustained (kernel timed inside a long step)",
+                     "frac_of_burst": achieved / peaks["bf16_tflops"],
+                     "launches": g_launch, "flop_per_launch": g_flop / max(g_launch, 1),
+                     "ms_per_launch": g_ms / max(g_launch, 1),
+                     "traffic": traffic},
+        "kernels": {k: {"launches": v["launches"], "ms_per_step": v["ms"] / args.steps,
+                        "share_of_kernel_time": v["ms"] / max(sum(x["ms"] for x in kernel.values()), 1e-9)}
+                    for k, v in kernel.items() if v["launches"]},
+        "dequant_share_of_step": dq["ms"] / args.steps / ms,
+        "pool": {"h2d_gbs": h2d_gbs, "bytes_per_step": pool_stats["bytes_copied"] / args.steps if pool_stats else 0,
+                 "copies_per_step": pool_stats["copies"] / args.steps if pool_stats else 0,
+                 "exposed_copy_ms": ms - results["no_h2d"] if "no_h2d" in results else None},
+        "step_kernel_ms": step_kernel_ms,
+        "peak_mem_gb": torch.cuda.max_memory_allocated() / 1e9,
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        rows = max(args.cpu_rows, os.cpu_count() or 1)
+        line["cpu_baseline"] = cpu_baseline(args, sample_rows=rows, budget_s=args.cpu_budget)
+    st_main.close()
+    print(json.dumps(line))
+
+
+def _traffic_from_profile():
+    """DRAM bytes per GEMM launch from the committed ncu summary, if it records one for this kernel build."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d.get("gemm_dram_bytes_per_launch")
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------ reference ---
+
+def cpu_baseline(args, sample_rows: int, budget_s: float):
+    """The oracle (fp64, plain loops, OpenMP over rows) on a bounded sample: `sample_rows` token rows through
+    the seven projections of one 8B-shaped layer, fwd + bwd.  Step time per token is scaled by the layer count
+    (derived, arithmetic)."""
+    import numpy as np
+
+    import oracle
+    from layer_streamed_nf4_b200 import synth
+    cfg = synth.STACKS[WORKLOAD]
+    L = cfg.layers
+    cores = os.cpu_count() or 1
+    # Inputs: a few rows of the same distributions; weights NF4 via the oracle.
+    t_total = 0.0
+    rows_done = 0
+    cases = []
+    for pi, (name, K, N) in enumerate(cfg.projections):
+        c = synth.linear_case(sample_rows, K, N, cfg.rank, cfg.alpha, seed=synth.SEED, layer=0, proj=pi)
+        q = oracle.nf4_quantize(c.W)
+        Wb = oracle.nf4_dequant(q["packed"], q["absmax_q"], q["s2"], q["offset"], c.W.size).reshape(N, K)
+        cases.append((c, Wb))
+    t0 = time.perf_counter()
+    for c, Wb in cases:
+        oracle.lora_fwd(c.x, Wb, c.A, c.B, c.scale)
+        oracle.lora_bwd_dx(c.dY, Wb, c.A, c.B, c.scale)
+        oracle.lora_bwd_dadb(c.x, c.dY, c.A, c.B, c.scale)
+        if time.perf_counter() - t0 > budget_s:
+            break
+    t_total = time.perf_counter() - t0
+    rows_done = sample_rows
+    s_per_token_step = t_total / rows_done * L
+    return {"value": 1.0 / s_per_token_step, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{rows_done} token rows through the 7 projections of one {cfg.name} layer (fwd+bwd, "
+                      f"fp64 oracle, OpenMP); per-step time = layer time x {L} layers (derived, arithmetic)",
+            "seconds": t_total}
+
+
+def run_reference(args):
+    world, rank, _ = _dist()
+    if rank != 0:
+        return
+    from layer_streamed_nf4_b200 import synth
+    cfg = synth.STACKS[WORKLOAD]
+    vals = []
+    for i in range(args.warmup + args.steps):
+        cb = cpu_baseline(args, sample_rows=args.ref_rows, budget_s=1e9)
+        if i >= args.warmup:
+            vals.append(cb)
+    v = statistics.median(c["value"] for c in vals)
+    s_step = sum(c["seconds"] for c in vals) / len(vals)
+    line = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": s_step * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": f"{cfg.name} NF4 LoRA stack (oracle sample)", "tokens": cfg.tokens,
+                       "layers": cfg.layers, "rank": cfg.rank},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": vals[0]["cores"], "kind": "oracle",
+                             "sample": vals[0]["sample"]},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--tokens", type=int, default=0, help="override T (default: the workload's 2048)")
+    ap.add_argument("--layers", type=int, default=0, help="override the layer count (default 32)")
+    ap.add_argument("--slots", type=int, default=2)
+    ap.add_argument("--modes", default="no_h2d,resident", help="extra modes timed after the streamed one")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=32)
+    ap.add_argument("--cpu-budget", type=float, default=60.0)
+    ap.add_argument("--ref-rows", type=int, default=4)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

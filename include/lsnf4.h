@@ -1,0 +1,291 @@
+/*
+ * lsnf4.h -- C ABI of liblsnf4.so: layer-streamed NF4 LoRA linears on B200 (sm_100a).
+ *
+ * The method ("Exact Layer Streaming: LoRA Fine-Tuning of an 8B Model on a 4 GB
+ * Laptop GPU", abstract) keeps a frozen base model -- NF4 or bf16 -- in host
+ * RAM, streams its decoder layers through a small pool of pre-allocated VRAM
+ * buffers on a separate copy stream, and trains LoRA adapters on top.  This
+ * library is its per-layer hot path:
+ *
+ *   nf4_quantize / nf4_dequant  the 4-bit base format and its double-quantised
+ *                               constants ("Can You Fine-Tune a 27B Model on a
+ *                               Laptop? (I Did the Math)", 2:19-2:29);
+ *   lora_linear_fwd / _bwd      y = x W^T + s (x A^T) B^T and its gradients
+ *                               for x, A, B (same video, 1:36-1:58);
+ *   layer_pool_*                the VRAM layer pool fed from pinned host RAM,
+ *                               prefetching the next layer on a side stream
+ *                               (same video, 7:11-7:42; the sourcefeed article
+ *                               "An 8B Fine-Tune Now Fits in 4 GB of VRAM",
+ *                               section "The trick is that frozen weights are
+ *                               just data").
+ *
+ * Conventions (all entry points):
+ *  - Every call returns an lsn_status.  Argument errors are detected before
+ *    anything is enqueued; lsn_last_error() then holds a message.  CUDA
+ *    launch errors are reported as LSN_ERR_CUDA by the call that launched;
+ *    asynchronous faults surface at the caller's next synchronisation.
+ *  - Compute calls are asynchronous on the stream passed in; no call
+ *    synchronises the device unless its comment says so.
+ *  - All tensor pointers are DEVICE pointers owned by the caller, row-major and
+ *    contiguous, unless stated otherwise.  bf16 tensors are passed as uint16_t
+ *    bit patterns.  Pointers passed to a compute call must stay valid until
+ *    the work enqueued on the stream has finished.
+ *  - Every tensor pointer must be 16-byte aligned (the tensor-memory-access
+ *    unit reads rows in 16-byte units).
+ *  - Results are deterministic: the same inputs and shapes give the same bits,
+ *    independent of pointers, streams or what ran before.
+ */
+#ifndef LSNF4_H
+#define LSNF4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream handle (cudaStream_t); NULL means the legacy default stream. */
+typedef struct CUstream_st* lsn_stream_t;
+
+typedef enum {
+    LSN_OK = 0,
+    LSN_ERR_INVALID_ARG = 1, /* bad shape, null or misaligned pointer, unpinned host memory */
+    LSN_ERR_CUDA = 2,        /* a CUDA runtime/driver call failed */
+    LSN_ERR_NO_MEMORY = 3,   /* device or host allocation failed */
+    LSN_ERR_TIMEOUT = 4,     /* a bounded wait ran out */
+    LSN_ERR_UNSUPPORTED = 5, /* no sm_100 device, or a shape outside the supported set */
+    LSN_ERR_STATE = 6        /* call out of order (e.g. pool has no free slot) */
+} lsn_status;
+
+/* Thread-local message describing the last failure of this thread; never NULL. */
+const char* lsn_last_error(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int lsn_version(void);
+
+/* ------------------------------------------------------------- NF4 codec --
+ *
+ * Format (the pages name NF4 and a second quantisation pass over its
+ * constants but print neither; this follows QLoRA's construction, the paper
+ * the sourcefeed article links):
+ *  - levels: 16 fp32 values, index 0 = -1, index 7 = 0, index 15 = +1; the
+ *    normalised N(0,1) quantiles of 7 negative and 8 positive equal steps up to
+ *    p_max = 1 - (1/32 + 1/30)/2;
+ *  - first level: blocks of 64 consecutive elements of the row-major weight
+ *    (cols % 64 == 0, so a block never crosses a row); code = nearest level
+ *    of w / absmax (smallest exact distance, lower index on a tie), computed in
+ *    fp32; an all-zero block codes to index 7;
+ *  - packing: byte j = (code[2j] << 4) | code[2j+1];
+ *  - second level: offset = mean of all block absmax values (fp64 sums:
+ *    sequential within each group of 256 blocks, then over groups in order;
+ *    divided by the block count, rounded to fp32); per group of 256 blocks,
+ *    s2 = max |fp32(absmax - offset)| and each block stores the 8-bit index of
+ *    the nearest entry of the table k/127 (k = -127..127 at index k+127) to
+ *    fp32((absmax - offset) / s2); s2 == 0 stores index 127;
+ *  - dequantisation: absmax_hat = fp32(fp32(table[code8] * s2) + offset),
+ *    w = bf16_rne(fp32(level[code4] * absmax_hat)), no fused multiply-add.
+ */
+
+/* Copies the 16 fp32 NF4 levels into out[16] (host memory). */
+void lsn_nf4_codebook(float out[16]);
+/* Copies the 256-entry fp32 second-level table into out[256] (host memory). */
+void lsn_dq_codebook(float out[256]);
+
+/* A quantised weight of rows x cols (N x K), cols % 64 == 0.  All pointers are
+ * caller-owned device memory:
+ *   packed     [rows*cols/2]      uint8, two 4-bit codes per byte
+ *   absmax_q   [rows*cols/64]     uint8 second-level codes
+ *   absmax_s2  [ceil(nblk/256)]   fp32 per group of 256 blocks
+ *   offset     [1]                fp32 (device, so quantisation never syncs) */
+typedef struct {
+    int64_t rows, cols;
+    uint8_t* packed;
+    uint8_t* absmax_q;
+    float* absmax_s2;
+    float* offset;
+} lsn_nf4_weight;
+
+/* Byte sizes of the four arrays of an rows x cols NF4 weight. */
+size_t lsn_nf4_packed_bytes(int64_t rows, int64_t cols);
+size_t lsn_nf4_absmax_bytes(int64_t rows, int64_t cols);
+size_t lsn_nf4_s2_bytes(int64_t rows, int64_t cols);
+/* Total bytes of the four arrays when each starts on a 1 KiB boundary (the
+ * layout used for a layer blob, see lsn_nf4_blob_layout). */
+size_t lsn_nf4_blob_bytes(int64_t rows, int64_t cols);
+/* Offsets of packed, absmax_q, absmax_s2 and offset inside such a blob
+ * (out[4], bytes from the blob start, each a multiple of 1024). */
+void lsn_nf4_blob_layout(int64_t rows, int64_t cols, size_t out[4]);
+
+/* Workspace bytes nf4_quantize needs for an rows x cols weight. */
+size_t lsn_nf4_quantize_ws_bytes(int64_t rows, int64_t cols);
+
+/* Quantise an fp32 weight W [rows, cols] (device) into *out.
+ * ws: device scratch of at least lsn_nf4_quantize_ws_bytes(rows, cols).
+ * Bit-exact with the format above.  A non-finite input element makes the
+ * result undefined (the host does not scan W); rows*cols == 0 is a no-op. */
+lsn_status nf4_quantize(const float* W, const lsn_nf4_weight* out, void* ws, size_t ws_bytes,
+                        lsn_stream_t stream);
+
+/* Dequantise *w into bf16 W_out [rows, cols] (device).  HBM-bound. */
+lsn_status nf4_dequant(const lsn_nf4_weight* w, uint16_t* W_out, lsn_stream_t stream);
+
+/* ------------------------------------------------------------ LoRA linear --
+ *
+ * y  = x W^T + s (x A^T) B^T                        (forward)
+ * dX = dY W + s (dY B) A                            (input gradient)
+ * dA = s (dY B)^T x,   dB = s dY^T (x A^T)          (adapter gradients, fp32)
+ * x [T,K], W [N,K] (rows = N out features, cols = K in features), A [r,K],
+ * B [N,r], y and dY [T,N], dX [T,K], dA [r,K], dB [N,r]; s = scale
+ * (alpha / r).  The base W is frozen: there is no gradient for it.
+ *
+ * Shapes supported: K % 64 == 0, N % 64 == 0, 1 <= r <= 64 with r % 8 == 0,
+ * T >= 0 (T == 0 is a no-op; any T, including a ragged last tile).
+ * Precision: bf16 operands, fp32 accumulation in tensor memory; s*(x A^T) and
+ * s*(dY B) enter the tensor-core contraction rounded to bf16; y and dX are
+ * written as bf16; dA and dB are accumulated in fp32 in a fixed order.
+ */
+typedef enum { LSN_BASE_NF4 = 0, LSN_BASE_BF16 = 1 } lsn_base_kind;
+
+typedef struct {
+    int kind;            /* lsn_base_kind */
+    int64_t rows, cols;  /* N, K */
+    lsn_nf4_weight nf4;  /* used when kind == LSN_BASE_NF4 (its rows/cols must match) */
+    const uint16_t* bf16;/* used when kind == LSN_BASE_BF16: bf16 W [rows, cols] */
+} lsn_base;
+
+/* Workspace bytes lora_linear_fwd / lora_linear_bwd need (the larger of the two). */
+size_t lsn_lora_ws_bytes(int64_t T, int64_t K, int64_t N, int r, int kind);
+
+/* Forward.  y may not alias x.  ws: device scratch of lsn_lora_ws_bytes bytes,
+ * not touched by anyone else until the enqueued work finishes. */
+lsn_status lora_linear_fwd(const lsn_base* W, const uint16_t* x, int64_t T, const uint16_t* A,
+                           const uint16_t* B, int r, float scale, uint16_t* y, void* ws,
+                           size_t ws_bytes, lsn_stream_t stream);
+
+/* Backward.  dX may be NULL (input gradient not wanted).  accumulate != 0 adds
+ * into dA and dB (gradient accumulation), otherwise they are overwritten. */
+lsn_status lora_linear_bwd(const lsn_base* W, const uint16_t* x, const uint16_t* dY, int64_t T,
+                           const uint16_t* A, const uint16_t* B, int r, float scale, uint16_t* dX,
+                           float* dA, float* dB, int accumulate, void* ws, size_t ws_bytes,
+                           lsn_stream_t stream);
+
+/* Synchronise `stream`, then read the status word at the start of a LoRA
+ * workspace: LSN_ERR_TIMEOUT if a tensor-core kernel gave up on a bounded
+ * wait since the last check (the word is then cleared), LSN_OK otherwise.
+ * The workspace must have been zero-filled once when it was allocated. */
+lsn_status lsn_ws_status(void* ws, lsn_stream_t stream);
+
+/* ------------------------------------------------------- kernel timing --
+ *
+ * Optional per-launch timing of the library's own kernels: while enabled,
+ * every launch is bracketed by two CUDA events on the stream it runs on, and
+ * lsn_timing_read sums the event-measured device time per kernel kind with
+ * the algorithmic work of each launch (flops for the GEMMs, bytes for the
+ * memory-bound kernels).  Recording adds two event records per launch.
+ */
+typedef enum {
+    LSN_K_GEMM_FWD = 0,   /* y = x W^T + s u B^T                 (flop) */
+    LSN_K_GEMM_BWD = 1,   /* dX = dY W + s g A                   (flop) */
+    LSN_K_DEQUANT = 2,    /* NF4 -> bf16                         (bytes) */
+    LSN_K_LORA_DOWN = 3,  /* u = x A^T, g = dY B                 (bytes) */
+    LSN_K_LORA_TGRAD = 4, /* dA, dB token reductions             (bytes) */
+    LSN_K_QUANTIZE = 5,   /* fp32 -> NF4                         (bytes) */
+    LSN_K_COUNT = 6
+} lsn_kernel_kind;
+
+typedef struct {
+    uint64_t launches[LSN_K_COUNT];  /* timed launch groups (one per library call site) */
+    uint64_t kernels[LSN_K_COUNT];   /* CUDA kernels inside those groups */
+    double ms[LSN_K_COUNT];          /* summed device time */
+    double work[LSN_K_COUNT];        /* summed algorithmic flop or bytes */
+} lsn_kernel_timing;
+
+/* Start (on != 0, clearing previous records) or stop recording.  At most
+ * 65536 launches are kept; later ones are counted but not timed. */
+lsn_status lsn_timing_enable(int on);
+/* Wait for the recorded events, return the sums and clear the records. */
+lsn_status lsn_timing_read(lsn_kernel_timing* out);
+
+/* ------------------------------------------------------------ layer pool --
+ *
+ * n_slots VRAM buffers of slot_bytes each, allocated once at creation; the
+ * pool copies registered host blobs (one per layer) into slots on its own copy
+ * stream and orders copy and compute with events:
+ *   ready[slot]     recorded on the copy stream after a layer's copy;
+ *   released[slot]  recorded on the compute stream by layer_pool_release.
+ * A copy into a slot always waits for that slot's released event, so a slot is
+ * never overwritten while compute may still read it.  Forward sweeps prefetch
+ * layer i+1 while layer i computes, backward sweeps layer i-1; with 2 slots a
+ * fwd+bwd step reads 2L-2 layers (each layer twice, minus the two still
+ * resident at the turn).
+ */
+typedef struct lsn_pool lsn_pool;
+
+typedef struct {
+    uint64_t copies;          /* host-to-device layer copies enqueued */
+    uint64_t bytes_copied;    /* their bytes */
+    uint64_t hits;            /* acquire/prefetch found the layer already resident */
+    uint64_t misses;          /* acquire had to start the copy itself */
+    double copy_ms;           /* summed device time of completed copies (events) */
+} lsn_pool_stats;
+
+/* Create a pool on `device` (the device is made current for the calls).
+ * Slots are 1 KiB aligned.  Fails with LSN_ERR_NO_MEMORY if the slots do not fit. */
+lsn_status layer_pool_create(int n_slots, size_t slot_bytes, int device, lsn_pool** out);
+
+/* Register the host blob of `layer` (0 <= layer < 65536).  host_pinned must be
+ * page-locked (cudaHostAlloc / cudaHostRegister) -- pageable memory is
+ * rejected -- and stay alive and unchanged until layer_pool_destroy;
+ * bytes <= slot_bytes.  Re-registering a layer replaces its blob and drops
+ * any resident copy. */
+lsn_status layer_pool_register(lsn_pool* pool, int layer, const void* host_pinned, size_t bytes);
+
+/* Start copying `layer` into a free slot (no-op if resident or in flight).
+ * Takes the least recently released slot that is neither acquired nor holding
+ * a prefetched, not yet acquired layer; LSN_ERR_STATE if there is none. */
+lsn_status layer_pool_prefetch(lsn_pool* pool, int layer);
+
+/* Make `compute` wait until `layer` is in VRAM (copying it first if needed)
+ * and return its slot address in *dev_ptr.  The slot stays valid for kernels
+ * enqueued on `compute` until layer_pool_release. */
+lsn_status layer_pool_acquire(lsn_pool* pool, int layer, lsn_stream_t compute, void** dev_ptr);
+
+/* Record released[slot] on `compute`: the slot may be reused once the work
+ * enqueued on `compute` before this call has finished. */
+lsn_status layer_pool_release(lsn_pool* pool, int layer, lsn_stream_t compute);
+
+/* Host-side bounded wait for every enqueued copy; LSN_ERR_TIMEOUT after
+ * timeout_ms milliseconds (the copies keep running). */
+lsn_status layer_pool_wait_idle(lsn_pool* pool, int timeout_ms);
+
+/* Counters since creation or the last reset. */
+lsn_status layer_pool_stats(lsn_pool* pool, lsn_pool_stats* out);
+
+/* Forget which layers are resident (slots are refilled on the next acquire)
+ * and zero the counters.  Waits for the pool's copies first (bounded, 10 s). */
+lsn_status layer_pool_reset(lsn_pool* pool);
+
+/* Test hooks that plant host-side faults (no GPU fault is ever produced):
+ *   LSN_POOL_FAULT_NONE         normal operation;
+ *   LSN_POOL_FAULT_STALE_SLOT   a copy into a slot that already held a layer
+ *                               is skipped: the slot is relabelled but keeps
+ *                               the previous layer's bytes -- the aliasing
+ *                               defect the bit-exactness gate must catch
+ *                               ("Exact Layer Streaming", abstract);
+ *   LSN_POOL_FAULT_COPY_ERROR   the next copy fails with LSN_ERR_CUDA before
+ *                               anything is enqueued. */
+typedef enum {
+    LSN_POOL_FAULT_NONE = 0,
+    LSN_POOL_FAULT_STALE_SLOT = 1,
+    LSN_POOL_FAULT_COPY_ERROR = 2
+} lsn_pool_fault;
+lsn_status layer_pool_inject_fault(lsn_pool* pool, int fault);
+
+/* Free the slots, events and the copy stream (waits for pending copies). */
+void layer_pool_destroy(lsn_pool* pool);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LSNF4_H */

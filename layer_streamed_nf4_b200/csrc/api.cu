@@ -1,0 +1,304 @@
+// The C entry points of liblsnf4.so (declared in include/lsnf4.h): argument
+// checks, workspace carving and the launch sequence of each call.
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+#include "timing.cuh"
+
+namespace lsn {
+
+// Defined in codec.cu, gemm.cu and lora_small.cu.
+size_t quantize_ws_bytes(int64_t rows, int64_t cols);
+lsn_status launch_quantize(const float* W, const lsn_nf4_weight* out, void* ws, size_t ws_bytes, cudaStream_t st);
+lsn_status launch_dequant(const lsn_nf4_weight* w, uint16_t* out, cudaStream_t st);
+lsn_status launch_gemm(const uint16_t* A, int64_t lda, const uint16_t* B, int64_t ldb, bool b_mn, const uint16_t* LA,
+                       const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D, int64_t ldd,
+                       int* err, cudaStream_t st);
+lsn_status launch_lora_down(const uint16_t* X, const uint16_t* W, bool w_rk, int64_t T, int64_t Kd, int r,
+                            float scale, float* u32, uint16_t* u16, cudaStream_t st);
+lsn_status launch_lora_tgrad(const float* G, const uint16_t* X, bool out_rk, int64_t T, int64_t Kd, int r,
+                             float scale, int accumulate, float* out, float* partial, cudaStream_t st);
+size_t tgrad_ws_bytes(int64_t T, int64_t Kd, int r);
+int tgrad_splits(int64_t T, int64_t Kd);
+
+namespace {
+thread_local std::string g_last_error = "no error";
+}
+
+lsn_status fail(lsn_status st, const std::string& msg) {
+    g_last_error = msg;
+    return st;
+}
+
+lsn_status fail_cuda(cudaError_t e, const char* what) {
+    g_last_error = std::string(what) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")";
+    return LSN_ERR_CUDA;
+}
+
+int sm_count() {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static int cache[64] = {0};
+    if (dev < 0 || dev >= 64) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+bool device_is_sm100() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    return major == 10 && minor == 0;
+}
+
+}  // namespace lsn
+
+using namespace lsn;
+
+namespace {
+
+lsn_status check_device() {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail_cuda(e, "cudaGetDevice");
+    if (!device_is_sm100()) return fail(LSN_ERR_UNSUPPORTED, "liblsnf4 is built for sm_100a (B200) only");
+    return LSN_OK;
+}
+
+lsn_status check_nf4(const lsn_nf4_weight* w, const char* who) {
+    const std::string f(who);
+    LSN_CHECK_ARG(w != nullptr, f + ": weight is NULL");
+    LSN_CHECK_ARG(w->rows >= 0 && w->cols >= 0, f + ": negative shape");
+    LSN_CHECK_ARG(w->cols % 64 == 0, f + ": cols must be a multiple of 64");
+    if (w->rows * w->cols == 0) return LSN_OK;
+    LSN_CHECK_ARG(w->packed && w->absmax_q && w->absmax_s2 && w->offset, f + ": NULL array in the NF4 weight");
+    LSN_CHECK_ARG(aligned16(w->packed), f + ": packed must be 16-byte aligned");
+    LSN_CHECK_ARG((reinterpret_cast<uintptr_t>(w->absmax_s2) & 3) == 0 && (reinterpret_cast<uintptr_t>(w->offset) & 3) == 0,
+                  f + ": absmax_s2/offset must be 4-byte aligned");
+    return LSN_OK;
+}
+
+// Workspace layout of the LoRA calls (each region 256-byte aligned):
+//   [0, 256)  status word of the GEMM kernels (must be zero-filled once)
+//   u32  fp32 [T, r]     x A^T
+//   g32  fp32 [T, r]     dY B
+//   s16  bf16 [T, r]     bf16(s u) or bf16(s g)
+//   part fp32 partials of the token reductions
+//   w16  bf16 [N, K]     dequantised base (NF4 base only)
+struct LoraWs {
+    int* err;
+    float* u32;
+    float* g32;
+    uint16_t* s16;
+    float* part;
+    uint16_t* w16;
+    size_t total;
+};
+
+LoraWs carve(void* ws, int64_t T, int64_t K, int64_t N, int r, int kind) {
+    LoraWs w;
+    size_t off = 0;
+    char* b = reinterpret_cast<char*>(ws);
+    auto take = [&](size_t bytes) { char* p = b ? b + off : nullptr; off += round_up(bytes, 256); return p; };
+    w.err = reinterpret_cast<int*>(take(256));
+    w.u32 = reinterpret_cast<float*>(take((size_t)T * r * 4));
+    w.g32 = reinterpret_cast<float*>(take((size_t)T * r * 4));
+    w.s16 = reinterpret_cast<uint16_t*>(take((size_t)T * r * 2));
+    const size_t pa = tgrad_ws_bytes(T, K, r), pb = tgrad_ws_bytes(T, N, r);
+    w.part = reinterpret_cast<float*>(take(pa > pb ? pa : pb));
+    w.w16 = reinterpret_cast<uint16_t*>(take(kind == LSN_BASE_NF4 ? (size_t)N * K * 2 : 0));
+    w.total = off;
+    return w;
+}
+
+lsn_status check_lora(const lsn_base* W, const uint16_t* x, int64_t T, const uint16_t* A, const uint16_t* B, int r,
+                      void* ws, size_t ws_bytes, const char* who) {
+    const std::string f(who);
+    LSN_CHECK_ARG(W != nullptr, f + ": base is NULL");
+    LSN_CHECK_ARG(W->kind == LSN_BASE_NF4 || W->kind == LSN_BASE_BF16, f + ": unknown base kind");
+    LSN_CHECK_ARG(T >= 0, f + ": T must be >= 0");
+    LSN_CHECK_ARG(W->rows > 0 && W->cols > 0, f + ": empty base weight");
+    LSN_CHECK_ARG(W->rows % 64 == 0 && W->cols % 64 == 0, f + ": N and K must be multiples of 64");
+    LSN_CHECK_ARG(W->rows <= (int64_t)1 << 30 && W->cols <= (int64_t)1 << 30 && T <= (int64_t)1 << 30,
+                  f + ": dimension too large");
+    LSN_CHECK_ARG(r >= 8 && r <= 64 && r % 8 == 0, f + ": rank must be a multiple of 8 in [8, 64]");
+    if (W->kind == LSN_BASE_NF4) {
+        lsn_status s = check_nf4(&W->nf4, who);
+        if (s != LSN_OK) return s;
+        LSN_CHECK_ARG(W->nf4.rows == W->rows && W->nf4.cols == W->cols, f + ": NF4 weight shape differs from the base shape");
+    } else {
+        LSN_CHECK_ARG(W->bf16 != nullptr && aligned16(W->bf16), f + ": bf16 base must be a 16-byte aligned pointer");
+    }
+    LSN_CHECK_ARG((x || T == 0) && A && B, f + ": NULL tensor");
+    LSN_CHECK_ARG(aligned16(x) && aligned16(A) && aligned16(B), f + ": tensors must be 16-byte aligned");
+    LSN_CHECK_ARG(ws != nullptr && aligned16(ws), f + ": workspace must be a 16-byte aligned device pointer");
+    const size_t need = carve(nullptr, T, W->cols, W->rows, r, W->kind).total;
+    LSN_CHECK_ARG(ws_bytes >= need, f + ": workspace too small (need " + std::to_string(need) + " bytes)");
+    return LSN_OK;
+}
+
+double dequant_bytes(int64_t N, int64_t K) {
+    const double n = (double)N * (double)K;
+    return n / 2.0 + n / 64.0 + 4.0 * (double)((N * K / 64 + 255) / 256) + 4.0 + 2.0 * n;
+}
+
+lsn_status timed_dequant(const lsn_nf4_weight* w, uint16_t* out, cudaStream_t st) {
+    TimingScope ts(LSN_K_DEQUANT, dequant_bytes(w->rows, w->cols), st);
+    return launch_dequant(w, out, st);
+}
+
+lsn_status timed_down(const uint16_t* X, const uint16_t* W, bool w_rk, int64_t T, int64_t Kd, int r, float scale,
+                      float* u32, uint16_t* u16, cudaStream_t st) {
+    const double bytes = 2.0 * T * Kd + 2.0 * r * Kd + (u32 ? 4.0 * T * r : 0.0) + (u16 ? 2.0 * T * r : 0.0);
+    TimingScope ts(LSN_K_LORA_DOWN, bytes, st);
+    return launch_lora_down(X, W, w_rk, T, Kd, r, scale, u32, u16, st);
+}
+
+lsn_status timed_tgrad(const float* G, const uint16_t* X, bool out_rk, int64_t T, int64_t Kd, int r, float scale,
+                       int accumulate, float* out, float* partial, cudaStream_t st) {
+    const double bytes = 2.0 * T * Kd + 4.0 * T * r + 4.0 * r * Kd * (accumulate ? 2.0 : 1.0);
+    TimingScope ts(LSN_K_LORA_TGRAD, bytes, st, tgrad_splits(T, Kd) > 1 ? 2 : 1);
+    return launch_lora_tgrad(G, X, out_rk, T, Kd, r, scale, accumulate, out, partial, st);
+}
+
+lsn_status timed_gemm(int kind, const uint16_t* A, int64_t lda, const uint16_t* B, int64_t ldb, bool b_mn,
+                      const uint16_t* LA, const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D,
+                      int64_t ldd, int* err, cudaStream_t st) {
+    TimingScope ts(kind, 2.0 * M * N * (double)(Kc + r), st);
+    return launch_gemm(A, lda, B, ldb, b_mn, LA, LB, r, M, N, Kc, D, ldd, err, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* lsn_last_error(void) { return g_last_error.c_str(); }
+
+int lsn_version(void) { return 100; }
+
+void lsn_nf4_codebook(float out[16]) { std::memcpy(out, nf4_tables().level, sizeof(float) * 16); }
+
+void lsn_dq_codebook(float out[256]) { std::memcpy(out, nf4_tables().dq, sizeof(float) * 256); }
+
+size_t lsn_nf4_packed_bytes(int64_t rows, int64_t cols) { return (size_t)(rows * cols / 2); }
+size_t lsn_nf4_absmax_bytes(int64_t rows, int64_t cols) { return (size_t)(rows * cols / 64); }
+size_t lsn_nf4_s2_bytes(int64_t rows, int64_t cols) { return (size_t)((rows * cols / 64 + 255) / 256) * 4; }
+
+void lsn_nf4_blob_layout(int64_t rows, int64_t cols, size_t out[4]) {
+    size_t off = 0;
+    out[0] = off;
+    off += round_up(lsn_nf4_packed_bytes(rows, cols), 1024);
+    out[1] = off;
+    off += round_up(lsn_nf4_absmax_bytes(rows, cols), 1024);
+    out[2] = off;
+    off += round_up(lsn_nf4_s2_bytes(rows, cols), 1024);
+    out[3] = off;
+}
+
+size_t lsn_nf4_blob_bytes(int64_t rows, int64_t cols) {
+    size_t o[4];
+    lsn_nf4_blob_layout(rows, cols, o);
+    return o[3] + 1024;
+}
+
+size_t lsn_nf4_quantize_ws_bytes(int64_t rows, int64_t cols) { return quantize_ws_bytes(rows, cols); }
+
+lsn_status nf4_quantize(const float* W, const lsn_nf4_weight* out, void* ws, size_t ws_bytes, lsn_stream_t stream) {
+    lsn_status s = check_nf4(out, "nf4_quantize");
+    if (s != LSN_OK) return s;
+    if (out->rows * out->cols == 0) return LSN_OK;
+    LSN_CHECK_ARG(W != nullptr && aligned16(W), "nf4_quantize: W must be a 16-byte aligned device pointer");
+    LSN_CHECK_ARG(ws != nullptr && aligned16(ws), "nf4_quantize: workspace must be 16-byte aligned");
+    LSN_CHECK_ARG(ws_bytes >= quantize_ws_bytes(out->rows, out->cols), "nf4_quantize: workspace too small");
+    if ((s = check_device()) != LSN_OK) return s;
+    const double numel = (double)out->rows * (double)out->cols;
+    TimingScope ts(LSN_K_QUANTIZE, numel * 4.0 + numel / 2.0 + numel / 64.0 * 6.0, reinterpret_cast<cudaStream_t>(stream),
+                   4);
+    return launch_quantize(W, out, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+lsn_status nf4_dequant(const lsn_nf4_weight* w, uint16_t* W_out, lsn_stream_t stream) {
+    lsn_status s = check_nf4(w, "nf4_dequant");
+    if (s != LSN_OK) return s;
+    if (w->rows * w->cols == 0) return LSN_OK;
+    LSN_CHECK_ARG(W_out != nullptr && aligned16(W_out), "nf4_dequant: output must be a 16-byte aligned device pointer");
+    if ((s = check_device()) != LSN_OK) return s;
+    return timed_dequant(w, W_out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t lsn_lora_ws_bytes(int64_t T, int64_t K, int64_t N, int r, int kind) {
+    return carve(nullptr, T, K, N, r, kind).total;
+}
+
+lsn_status lora_linear_fwd(const lsn_base* W, const uint16_t* x, int64_t T, const uint16_t* A, const uint16_t* B, int r,
+                           float scale, uint16_t* y, void* ws, size_t ws_bytes, lsn_stream_t stream) {
+    lsn_status s = check_lora(W, x, T, A, B, r, ws, ws_bytes, "lora_linear_fwd");
+    if (s != LSN_OK) return s;
+    LSN_CHECK_ARG((y != nullptr || T == 0) && aligned16(y), "lora_linear_fwd: y must be a 16-byte aligned device pointer");
+    if (T == 0) return LSN_OK;
+    if ((s = check_device()) != LSN_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t N = W->rows, K = W->cols;
+    LoraWs w = carve(ws, T, K, N, r, W->kind);
+    if ((s = timed_down(x, A, true, T, K, r, scale, nullptr, w.s16, st)) != LSN_OK) return s;
+    const uint16_t* Wb = W->bf16;
+    if (W->kind == LSN_BASE_NF4) {
+        if ((s = timed_dequant(&W->nf4, w.w16, st)) != LSN_OK) return s;
+        Wb = w.w16;
+    }
+    return timed_gemm(LSN_K_GEMM_FWD, x, K, Wb, K, false, w.s16, B, r, T, N, K, y, N, w.err, st);
+}
+
+lsn_status lora_linear_bwd(const lsn_base* W, const uint16_t* x, const uint16_t* dY, int64_t T, const uint16_t* A,
+                           const uint16_t* B, int r, float scale, uint16_t* dX, float* dA, float* dB, int accumulate,
+                           void* ws, size_t ws_bytes, lsn_stream_t stream) {
+    lsn_status s = check_lora(W, x, T, A, B, r, ws, ws_bytes, "lora_linear_bwd");
+    if (s != LSN_OK) return s;
+    LSN_CHECK_ARG((dY != nullptr || T == 0) && aligned16(dY), "lora_linear_bwd: dY must be a 16-byte aligned device pointer");
+    LSN_CHECK_ARG(dA && dB && aligned16(dA) && aligned16(dB), "lora_linear_bwd: dA/dB must be 16-byte aligned device pointers");
+    LSN_CHECK_ARG(dX == nullptr || aligned16(dX), "lora_linear_bwd: dX must be 16-byte aligned");
+    if ((s = check_device()) != LSN_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t N = W->rows, K = W->cols;
+    LoraWs w = carve(ws, T, K, N, r, W->kind);
+    if (T > 0) {
+        if ((s = timed_down(dY, B, false, T, N, r, scale, w.g32, w.s16, st)) != LSN_OK) return s;
+        if ((s = timed_down(x, A, true, T, K, r, scale, w.u32, nullptr, st)) != LSN_OK) return s;
+        if (dX) {
+            const uint16_t* Wb = W->bf16;
+            if (W->kind == LSN_BASE_NF4) {
+                if ((s = timed_dequant(&W->nf4, w.w16, st)) != LSN_OK) return s;
+                Wb = w.w16;
+            }
+            if ((s = timed_gemm(LSN_K_GEMM_BWD, dY, N, Wb, K, true, w.s16, A, r, T, K, N, dX, K, w.err, st)) != LSN_OK)
+                return s;
+        }
+    }
+    // With T == 0 the reductions write zeros (or leave accumulators unchanged).
+    if ((s = timed_tgrad(w.g32, x, true, T, K, r, scale, accumulate, dA, w.part, st)) != LSN_OK) return s;
+    return timed_tgrad(w.u32, dY, false, T, N, r, scale, accumulate, dB, w.part, st);
+}
+
+lsn_status lsn_ws_status(void* ws, lsn_stream_t stream) {
+    LSN_CHECK_ARG(ws != nullptr, "lsn_ws_status: workspace is NULL");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int h = 0;
+    LSN_CUDA_TRY(cudaMemcpyAsync(&h, ws, sizeof(int), cudaMemcpyDeviceToHost, st));
+    LSN_CUDA_TRY(cudaStreamSynchronize(st));
+    if (h != 0) {
+        LSN_CUDA_TRY(cudaMemsetAsync(ws, 0, sizeof(int), st));
+        LSN_CUDA_TRY(cudaStreamSynchronize(st));
+        return fail(LSN_ERR_TIMEOUT, "a tensor-core kernel gave up waiting (code " + std::to_string(h) + ")");
+    }
+    return LSN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,294 @@
+// NF4 codec: quantisation with double-quantised absmax constants, and the
+// standalone dequantisation kernel.
+//
+// Format ("Can You Fine-Tune a 27B Model on a Laptop? (I Did the Math)",
+// 2:19-2:29, names a 4-bit format for bell-curve weights and a second
+// quantisation of its constants; the construction followed is QLoRA's, the
+// paper linked by "An 8B Fine-Tune Now Fits in 4 GB of VRAM"):
+//   levels      normal quantiles, 7 negative, 0, 8 positive, scaled to [-1, 1]
+//   level code  nearest level of w / absmax over blocks of 64, ties lower
+//   packing     byte j = code[2j] << 4 | code[2j+1]
+//   constants   8-bit codes of (absmax - mean) / s2 on the table k/127, one
+//               fp32 s2 per 256 blocks, one fp32 mean per tensor
+//   dequant     w = bf16(level[q] * (table[c] * s2 + mean)), each op rounded
+//
+// Every rounding-sensitive operation uses an explicit IEEE intrinsic
+// (__fdiv_rn, __fsub_rn, __fmul_rn, __fadd_rn) so the compiler can neither
+// contract nor approximate it.
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace lsn {
+
+// ------------------------------------------------------------ host tables --
+
+namespace {
+
+double std_normal_cdf(double x) { return 0.5 * std::erfc(-x / std::sqrt(2.0)); }
+
+// Quantile of N(0,1) for p in [1/2, 1): bisection on the CDF (bracket [0, 9])
+// until the bracket stops shrinking, then two Newton steps on the upper tail
+// 1 - Phi(x) = erfc(x / sqrt 2) / 2, which libm evaluates with full relative
+// accuracy.
+double std_normal_quantile_upper(double p) {
+    if (p == 0.5) return 0.0;
+    double lo = 0.0, hi = 9.0;
+    for (int it = 0; it < 2000; ++it) {
+        const double mid = 0.5 * (lo + hi);
+        if (mid <= lo || mid >= hi) break;
+        if (std_normal_cdf(mid) < p) lo = mid; else hi = mid;
+    }
+    double x = 0.5 * (lo + hi);
+    const double tail = 1.0 - p;
+    for (int it = 0; it < 2; ++it) {
+        const double f = 0.5 * std::erfc(x / std::sqrt(2.0)) - tail;      // decreasing in x
+        const double dens = std::exp(-0.5 * x * x) / std::sqrt(2.0 * M_PI);
+        x += f / dens;
+    }
+    return x;
+}
+
+// Largest fp32 value that is <= the exact midpoint of two fp32 levels: an
+// fp32 v has its nearest level at index <= i exactly when v <= thr[i]
+// (ties go to the lower index).
+float threshold_below(float a, float b) {
+    const double mid = ((double)a + (double)b) * 0.5;   // exact: two fp32 summands
+    float t = (float)mid;
+    if ((double)t > mid) t = std::nextafter(t, -INFINITY);
+    return t;
+}
+
+Nf4Tables build_tables() {
+    Nf4Tables t;
+    const double p_max = 1.0 - 0.5 * (1.0 / 32.0 + 1.0 / 30.0);
+    double lv[16];
+    int n = 0;
+    for (int j = 7; j >= 1; --j) lv[n++] = -std_normal_quantile_upper(0.5 + (p_max - 0.5) * j / 7.0);
+    lv[n++] = 0.0;
+    for (int j = 1; j <= 8; ++j) lv[n++] = std_normal_quantile_upper(0.5 + (p_max - 0.5) * j / 8.0);
+    double mx = 0.0;
+    for (double v : lv) mx = std::fmax(mx, std::fabs(v));
+    for (int i = 0; i < 16; ++i) t.level[i] = (float)(lv[i] / mx);
+    for (int i = 0; i < 15; ++i) t.thr[i] = threshold_below(t.level[i], t.level[i + 1]);
+    for (int k = -127; k <= 127; ++k) t.dq[k + 127] = (float)((double)k / 127.0);
+    t.dq[255] = 0.0f;
+    for (int i = 0; i < 254; ++i) t.dq_thr[i] = threshold_below(t.dq[i], t.dq[i + 1]);
+    return t;
+}
+
+}  // namespace
+
+const Nf4Tables& nf4_tables() {
+    static Nf4Tables tables = build_tables();
+    return tables;
+}
+
+// ---------------------------------------------------------------- kernels --
+
+struct LevelParams { float level[16]; float thr[15]; };
+struct DqParams { float dq[256]; float thr[254]; };
+
+// Pass 1: one warp per block of 64 elements.  Lane l owns elements 2l, 2l+1:
+// absmax by a warp max, codes by counting thresholds below w / absmax, one
+// packed byte per lane (32 contiguous bytes per block).
+__global__ void __launch_bounds__(256) nf4_level_codes_kernel(const float2* __restrict__ W, int64_t nblk,
+                                                               uint8_t* __restrict__ packed,
+                                                               float* __restrict__ absmax, LevelParams P) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t b = warp0; b < nblk; b += nwarps) {
+        const float2 w = W[b * 32 + lane];
+        float a = fmaxf(fabsf(w.x), fabsf(w.y));
+        #pragma unroll
+        for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+        uint32_t q0 = 7, q1 = 7;
+        if (a > 0.0f) {
+            const float v0 = __fdiv_rn(w.x, a), v1 = __fdiv_rn(w.y, a);
+            q0 = 0; q1 = 0;
+            #pragma unroll
+            for (int i = 0; i < 15; ++i) { q0 += (v0 > P.thr[i]); q1 += (v1 > P.thr[i]); }
+        }
+        packed[b * 32 + lane] = (uint8_t)((q0 << 4) | q1);
+        if (lane == 0) absmax[b] = a;
+    }
+}
+
+// Pass 2: one thread per group of 256 blocks, sequential fp64 sum.
+__global__ void dq_group_sum_kernel(const float* __restrict__ absmax, int64_t nblk, int64_t ngrp,
+                                    double* __restrict__ partial) {
+    const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (g >= ngrp) return;
+    const int64_t b1 = (g * 256 + 256 < nblk) ? g * 256 + 256 : nblk;
+    double s = 0.0;
+    for (int64_t b = g * 256; b < b1; ++b) s = __dadd_rn(s, (double)absmax[b]);
+    partial[g] = s;
+}
+
+// Pass 3: one thread: sum of the group partials in group order, mean, fp32.
+__global__ void dq_offset_kernel(const double* __restrict__ partial, int64_t ngrp, int64_t nblk,
+                                 float* __restrict__ offset) {
+    if (blockIdx.x != 0 || threadIdx.x != 0) return;
+    double s = 0.0;
+    for (int64_t g = 0; g < ngrp; ++g) s = __dadd_rn(s, partial[g]);
+    *offset = __double2float_rn(__ddiv_rn(s, (double)nblk));
+}
+
+// Pass 4: one warp per group: s2 = max |absmax - offset|, then the 8-bit
+// code of each block by binary search over the 254 thresholds.
+__global__ void __launch_bounds__(256) dq_codes_kernel(const float* __restrict__ absmax, int64_t nblk,
+                                                        int64_t ngrp, const float* __restrict__ offset,
+                                                        uint8_t* __restrict__ absmax_q, float* __restrict__ s2,
+                                                        DqParams P) {
+    __shared__ float thr[256];
+    for (int i = threadIdx.x; i < 254; i += blockDim.x) thr[i] = P.thr[i];
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const float off = *offset;
+    for (int64_t g = warp0; g < ngrp; g += nwarps) {
+        float c[8];
+        float m = 0.0f;
+        #pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int64_t b = g * 256 + i * 32 + lane;
+            c[i] = (b < nblk) ? __fsub_rn(absmax[b], off) : 0.0f;
+            m = fmaxf(m, fabsf(c[i]));
+        }
+        #pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) s2[g] = m;
+        #pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int64_t b = g * 256 + i * 32 + lane;
+            if (b >= nblk) continue;
+            uint32_t code = 127;
+            if (m > 0.0f) {
+                const float v = __fdiv_rn(c[i], m);
+                int lo = 0, hi = 254;                 // count of thresholds strictly below v
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if (thr[mid] < v) lo = mid + 1; else hi = mid;
+                }
+                code = (uint32_t)lo;
+            }
+            absmax_q[b] = (uint8_t)code;
+        }
+    }
+}
+
+// Standalone dequantisation: each thread turns one 32-bit word of packed
+// codes (8 weights, always inside one 64-block) into 8 bf16 = one 16-byte
+// store.  Loads are 4 bytes per lane (128 B per warp), stores 16 bytes per
+// lane (512 B per warp), both contiguous across the warp.
+struct DequantParams { float level[16]; float dq[256]; };
+
+__global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint32_t* __restrict__ packed,
+                                                           const uint8_t* __restrict__ absmax_q,
+                                                           const float* __restrict__ s2,
+                                                           const float* __restrict__ offset, int64_t nwords,
+                                                           uint4* __restrict__ out, DequantParams P) {
+    __shared__ float lv[16];
+    __shared__ float dq[256];
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) dq[i] = P.dq[i];
+    if (threadIdx.x < 16) lv[threadIdx.x] = P.level[threadIdx.x];
+    __syncthreads();
+    const float off = *offset;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    // Four independent words in flight per thread.
+    for (; w + 3 * stride < nwords; w += 4 * stride) {
+        uint32_t p[4];
+        float ah[4];
+        #pragma unroll
+        for (int u = 0; u < 4; ++u) p[u] = __ldg(packed + w + u * stride);
+        #pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int64_t b = (w + u * stride) >> 3;
+            ah[u] = __fadd_rn(__fmul_rn(dq[__ldg(absmax_q + b)], __ldg(s2 + (b >> 8))), off);
+        }
+        #pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            uint32_t r[4];
+            #pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t byte = (p[u] >> (8 * j)) & 0xffu;
+                r[j] = pack_bf16x2(__fmul_rn(lv[byte >> 4], ah[u]), __fmul_rn(lv[byte & 15u], ah[u]));
+            }
+            out[w + u * stride] = make_uint4(r[0], r[1], r[2], r[3]);
+        }
+    }
+    for (; w < nwords; w += stride) {
+        const uint32_t p = __ldg(packed + w);
+        const int64_t b = w >> 3;
+        const float a = __fadd_rn(__fmul_rn(dq[__ldg(absmax_q + b)], __ldg(s2 + (b >> 8))), off);
+        uint32_t r[4];
+        #pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t byte = (p >> (8 * j)) & 0xffu;
+            r[j] = pack_bf16x2(__fmul_rn(lv[byte >> 4], a), __fmul_rn(lv[byte & 15u], a));
+        }
+        out[w] = make_uint4(r[0], r[1], r[2], r[3]);
+    }
+}
+
+// ------------------------------------------------------------ launchers ---
+
+size_t quantize_ws_bytes(int64_t rows, int64_t cols) {
+    const int64_t nblk = rows * cols / 64;
+    const int64_t ngrp = (nblk + 255) / 256;
+    return round_up((size_t)nblk * sizeof(float), 256) + (size_t)ngrp * sizeof(double);
+}
+
+static int grid_for(int64_t work_items, int per_block, int waves_cap) {
+    int64_t g = (work_items + per_block - 1) / per_block;
+    const int64_t cap = (int64_t)sm_count() * waves_cap;
+    if (g > cap) g = cap;
+    if (g < 1) g = 1;
+    return (int)g;
+}
+
+lsn_status launch_quantize(const float* W, const lsn_nf4_weight* out, void* ws, size_t ws_bytes,
+                           cudaStream_t st) {
+    const int64_t numel = out->rows * out->cols;
+    const int64_t nblk = numel / 64;
+    const int64_t ngrp = (nblk + 255) / 256;
+    const Nf4Tables& T = nf4_tables();
+    float* absmax = reinterpret_cast<float*>(ws);
+    double* partial = reinterpret_cast<double*>(reinterpret_cast<char*>(ws) + round_up((size_t)nblk * 4, 256));
+    LevelParams lp;
+    std::memcpy(lp.level, T.level, sizeof(lp.level));
+    std::memcpy(lp.thr, T.thr, sizeof(lp.thr));
+    nf4_level_codes_kernel<<<grid_for(nblk, 8, 16), 256, 0, st>>>(reinterpret_cast<const float2*>(W), nblk,
+                                                                  out->packed, absmax, lp);
+    dq_group_sum_kernel<<<(int)ceil_div(ngrp, 128), 128, 0, st>>>(absmax, nblk, ngrp, partial);
+    dq_offset_kernel<<<1, 32, 0, st>>>(partial, ngrp, nblk, out->offset);
+    DqParams dp;
+    std::memcpy(dp.dq, T.dq, sizeof(dp.dq));
+    std::memcpy(dp.thr, T.dq_thr, sizeof(dp.thr));
+    dq_codes_kernel<<<grid_for(ngrp, 8, 16), 256, 0, st>>>(absmax, nblk, ngrp, out->offset, out->absmax_q,
+                                                          out->absmax_s2, dp);
+    LSN_CUDA_TRY(cudaGetLastError());
+    (void)ws_bytes;
+    return LSN_OK;
+}
+
+lsn_status launch_dequant(const lsn_nf4_weight* w, uint16_t* out, cudaStream_t st) {
+    const int64_t nwords = w->rows * w->cols / 8;
+    const Nf4Tables& T = nf4_tables();
+    DequantParams P;
+    std::memcpy(P.level, T.level, sizeof(P.level));
+    std::memcpy(P.dq, T.dq, sizeof(P.dq));
+    // Enough threads for four words each on every SM, several blocks per SM.
+    const int grid = grid_for(ceil_div(nwords, 4), 256, 8);
+    nf4_dequant_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint32_t*>(w->packed), w->absmax_q,
+                                             w->absmax_s2, w->offset, nwords, reinterpret_cast<uint4*>(out), P);
+    LSN_CUDA_TRY(cudaGetLastError());
+    return LSN_OK;
+}
+
+}  // namespace lsn

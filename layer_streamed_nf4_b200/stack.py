@@ -1,0 +1,213 @@
+"""The layer loop of a training step over a stack of frozen-base LoRA linears.
+
+"Can You Fine-Tune a 27B Model on a Laptop? (I Did the Math)", 7:11-7:42: the
+frozen base lives in system RAM, each decoder layer is copied into a small
+VRAM buffer on a separate stream while the previous one computes, and every
+layer is read twice per step (forward, then backward).  This module drives
+that loop through the C ABI: per step a forward sweep over layers 0..L-1
+(acquire i, prefetch i+1, seven lora_linear_fwd calls, release i) and a
+backward sweep over L-1..0 (acquire i, prefetch i-1, seven lora_linear_bwd
+calls, release i).  All compute and all copies are library calls; this file
+only sequences them and owns the (synthetic) tensors.
+
+Modes with identical kernels and launch shapes, for the bit-exactness gate
+("Exact Layer Streaming", abstract: streamed compared with a resident run of
+the same numerics):
+  resident  every layer blob copied once into one device buffer;
+  streamed  layer blobs in pinned host RAM, n_slots VRAM slots (default 2);
+  no_h2d    a pool with one slot per layer, pre-filled before timing.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+from . import lsnf4, synth
+
+
+def _round_up(a: int, b: int) -> int:
+    return (a + b - 1) // b * b
+
+
+@dataclass
+class ProjLayout:
+    name: str
+    K: int
+    N: int
+    offset: int      # byte offset of this projection in the layer blob
+    nbytes: int
+
+
+class Stack:
+    def __init__(self, cfg: synth.StackConfig, layers: int | None = None, tokens: int | None = None,
+                 mode: str = "streamed", n_slots: int = 2, seed: int = synth.SEED, keep_outputs: bool = False,
+                 distinct_activations: bool = True, device: int = 0, stream: torch.cuda.Stream | None = None):
+        assert mode in ("resident", "streamed", "no_h2d")
+        self.cfg, self.mode, self.seed = cfg, mode, seed
+        self.L = layers if layers is not None else cfg.layers
+        self.T = tokens if tokens is not None else cfg.tokens
+        self.r, self.scale = cfg.rank, cfg.alpha / cfg.rank
+        self.nf4 = cfg.base == "nf4"
+        self.kind = lsnf4.LSN_BASE_NF4 if self.nf4 else lsnf4.LSN_BASE_BF16
+        self.dev = torch.device("cuda", device)
+        self.stream = stream if stream is not None else torch.cuda.current_stream(self.dev)
+        self.keep_outputs = keep_outputs
+        off = 0
+        self.proj: list[ProjLayout] = []
+        for name, K, N in cfg.projections:
+            nb = lsnf4.nf4_blob_bytes(N, K) if self.nf4 else _round_up(N * K * 2, 1024)
+            self.proj.append(ProjLayout(name, K, N, off, nb))
+            off += nb
+        self.layer_bytes = off
+        self.pool = None
+        self.host = None
+        self.resident = None
+        self._build_weights()
+        self._build_tensors(distinct_activations)
+        self._setup_mode(n_slots)
+
+    # ------------------------------------------------------------ set-up --
+
+    def _build_weights(self):
+        """W ~ N(0, 0.02) per projection, quantised on the device, stored per layer in pinned host RAM."""
+        self.host = torch.empty((self.L, self.layer_bytes), dtype=torch.uint8, pin_memory=True)
+        dblob = torch.zeros(self.layer_bytes, dtype=torch.uint8, device=self.dev)
+        maxnk = max(p.N * p.K for p in self.proj)
+        qws_bytes = lsnf4.nf4_quantize_ws_bytes(1, maxnk) if self.nf4 else 0
+        qws = torch.zeros(max(qws_bytes, 16), dtype=torch.uint8, device=self.dev)
+        with torch.cuda.stream(self.stream):
+            for l in range(self.L):
+                for pi, p in enumerate(self.proj):
+                    W = synth.device_normal((p.N, p.K), 0.02, self.seed, l, pi, synth.T_W, device=self.dev)
+                    addr = dblob.data_ptr() + p.offset
+                    if self.nf4:
+                        w = lsnf4.nf4_weight_in_blob(p.N, p.K, addr)
+                        lsnf4.nf4_quantize(W, w, qws, qws_bytes, self.stream)
+                    else:
+                        dst = dblob[p.offset:p.offset + p.N * p.K * 2].view(torch.bfloat16)
+                        dst.copy_(W.reshape(-1).to(torch.bfloat16))
+                    del W
+                self.host[l].copy_(dblob, non_blocking=False)
+        self.stream.synchronize()
+
+    def _build_tensors(self, distinct: bool):
+        T, r, dev = self.T, self.r, self.dev
+        self.x, self.dY, self.A, self.B, self.dA, self.dB = {}, {}, {}, {}, {}, {}
+        for l in range(self.L):
+            for pi, p in enumerate(self.proj):
+                la = l if distinct else 0
+                self.x[l, pi] = synth.device_normal((T, p.K), 1.0, self.seed, la, pi, synth.T_X, device=dev,
+                                                    dtype=torch.bfloat16) if (distinct or l == 0) else self.x[0, pi]
+                self.dY[l, pi] = synth.device_normal((T, p.N), 1.0, self.seed, la, pi, synth.T_DY, device=dev,
+                                                     dtype=torch.bfloat16) if (distinct or l == 0) else self.dY[0, pi]
+                self.A[l, pi] = synth.device_uniform((r, p.K), 1.0 / p.K ** 0.5, self.seed, l, pi, synth.T_A,
+                                                     device=dev, dtype=torch.bfloat16)
+                self.B[l, pi] = synth.device_normal((p.N, r), 0.01, self.seed, l, pi, synth.T_B, device=dev,
+                                                    dtype=torch.bfloat16)
+                self.dA[l, pi] = torch.zeros((r, p.K), dtype=torch.float32, device=dev)
+                self.dB[l, pi] = torch.zeros((p.N, r), dtype=torch.float32, device=dev)
+        nl = self.L if self.keep_outputs else 1
+        self.y = {(l, pi): torch.empty((T, p.N), dtype=torch.bfloat16, device=dev)
+                  for l in range(nl) for pi, p in enumerate(self.proj)}
+        self.dX = {(l, pi): torch.empty((T, p.K), dtype=torch.bfloat16, device=dev)
+                   for l in range(nl) for pi, p in enumerate(self.proj)}
+        self.ws_bytes = max(lsnf4.lora_ws_bytes(T, p.K, p.N, r, self.kind) for p in self.proj)
+        self.ws = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=dev)
+        torch.cuda.synchronize(dev)
+
+    def _setup_mode(self, n_slots: int):
+        if self.mode == "resident":
+            self.resident = self.host.to(self.dev)
+            return
+        slots = self.L if self.mode == "no_h2d" else n_slots
+        self.pool = lsnf4.layer_pool_create(slots, self.layer_bytes, self.dev.index or 0)
+        for l in range(self.L):
+            lsnf4.layer_pool_register(self.pool, l, self.host[l].data_ptr(), self.layer_bytes)
+        if self.mode == "no_h2d":
+            for l in range(self.L):
+                lsnf4.layer_pool_prefetch(self.pool, l)
+            lsnf4.layer_pool_wait_idle(self.pool, 600000)
+
+    def with_mode(self, mode: str, n_slots: int = 2) -> "Stack":
+        """A stack sharing this one's host blobs and tensors, run in another mode."""
+        import copy
+        assert mode in ("resident", "streamed", "no_h2d")
+        other = copy.copy(self)
+        other.mode, other.pool, other.resident = mode, None, None
+        other._setup_mode(n_slots)
+        return other
+
+    def close(self):
+        if self.pool is not None:
+            lsnf4.layer_pool_destroy(self.pool)
+            self.pool = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # ------------------------------------------------------------ layers --
+
+    def _acquire(self, l: int) -> int:
+        if self.mode == "resident":
+            return self.resident[l].data_ptr()
+        return lsnf4.layer_pool_acquire(self.pool, l, self.stream)
+
+    def _prefetch(self, l: int):
+        if self.mode != "resident" and 0 <= l < self.L:
+            lsnf4.layer_pool_prefetch(self.pool, l)
+
+    def _release(self, l: int):
+        if self.mode != "resident":
+            lsnf4.layer_pool_release(self.pool, l, self.stream)
+
+    def _base(self, addr: int, p: ProjLayout):
+        if self.nf4:
+            return lsnf4.base_nf4(lsnf4.nf4_weight_in_blob(p.N, p.K, addr + p.offset))
+        return lsnf4.base_bf16(addr + p.offset, p.N, p.K)
+
+    def _out(self, d, l, pi):
+        return d[(l if self.keep_outputs else 0), pi]
+
+    def forward(self):
+        s = self.stream
+        for l in range(self.L):
+            addr = self._acquire(l)
+            self._prefetch(l + 1)
+            for pi, p in enumerate(self.proj):
+                lsnf4.lora_linear_fwd(self._base(addr, p), self.x[l, pi], self.T, self.A[l, pi], self.B[l, pi],
+                                      self.r, self.scale, self._out(self.y, l, pi), self.ws, self.ws_bytes, s)
+            self._release(l)
+
+    def backward(self, accumulate: bool = False):
+        s = self.stream
+        for l in reversed(range(self.L)):
+            addr = self._acquire(l)
+            self._prefetch(l - 1)
+            for pi in reversed(range(len(self.proj))):
+                p = self.proj[pi]
+                lsnf4.lora_linear_bwd(self._base(addr, p), self.x[l, pi], self.dY[l, pi], self.T, self.A[l, pi],
+                                      self.B[l, pi], self.r, self.scale, self._out(self.dX, l, pi), self.dA[l, pi],
+                                      self.dB[l, pi], accumulate, self.ws, self.ws_bytes, s)
+            self._release(l)
+
+    def step(self, accumulate: bool = False):
+        self.forward()
+        self.backward(accumulate)
+
+    # ------------------------------------------------------------ facts ---
+
+    def flop_per_step(self) -> float:
+        return float(self.cfg.flop_per_token_per_layer()) * self.T * self.L
+
+    def h2d_bytes_per_layer(self) -> int:
+        return self.layer_bytes
+
+    def pool_stats(self) -> dict | None:
+        return lsnf4.layer_pool_stats(self.pool) if self.pool is not None else None
+
+    def check_status(self):
+        lsnf4.ws_status(self.ws, self.stream)

@@ -1,0 +1,110 @@
+"""CPU checks of the C-ABI library: it loads, exports every symbol the header
+declares, and its host-side logic (tables, sizes, argument checks) is right.
+No call here launches GPU work."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from layer_streamed_nf4_b200 import build
+    build.build()
+    from layer_streamed_nf4_b200 import lsnf4
+    return lsnf4
+
+
+def _header_functions():
+    src = open(os.path.join(ROOT, "include", "lsnf4.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = set()
+    for m in re.finditer(r"^\s*(?:const\s+)?[\w\s\*]+?\b(\w+)\s*\(", src, flags=re.M):
+        name = m.group(1)
+        if name not in ("defined",):
+            names.add(name)
+    return names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    declared = _header_functions()
+    assert len(declared) >= 25, declared
+    so = ctypes.CDLL(lib.lib_path())
+    missing = [n for n in sorted(declared) if not hasattr(so, n)]
+    assert not missing, missing
+    assert set(lib.EXPORTS) == declared
+
+
+def test_codebook_matches_oracle_bitwise(lib, orc):
+    got = np.array(lib.nf4_codebook(), np.float32)
+    assert np.array_equal(got.view(np.uint32), orc.nf4_codebook().view(np.uint32))
+    dq = np.array(lib.dq_codebook(), np.float32)
+    assert np.array_equal(dq.view(np.uint32), orc.dq_table().view(np.uint32))
+
+
+def test_sizes_and_blob_layout(lib):
+    rows, cols = 14336, 4096
+    assert lib.nf4_packed_bytes(rows, cols) == rows * cols // 2
+    assert lib.nf4_absmax_bytes(rows, cols) == rows * cols // 64
+    assert lib.nf4_s2_bytes(rows, cols) == 4 * ((rows * cols // 64 + 255) // 256)
+    o = lib.nf4_blob_layout(rows, cols)
+    assert all(v % 1024 == 0 for v in o)
+    assert o[0] == 0 and o[1] >= rows * cols // 2 and o[2] - o[1] >= rows * cols // 64
+    assert lib.nf4_blob_bytes(rows, cols) == o[3] + 1024
+    # workspace grows with the problem and covers the dequantised base for NF4
+    small = lib.lora_ws_bytes(256, 512, 512, 8, lib.LSN_BASE_BF16)
+    big = lib.lora_ws_bytes(256, 512, 512, 8, lib.LSN_BASE_NF4)
+    assert big >= small + 512 * 512 * 2
+
+
+@pytest.mark.parametrize("r", [0, 4, 7, 72])
+def test_bad_rank_is_rejected_before_any_launch(lib, r):
+    W = lib.base_bf16(1 << 20, 512, 512)
+    with pytest.raises(lib.LsnError) as e:
+        lib.lora_linear_fwd(W, 1 << 20, 16, 1 << 20, 1 << 20, r, 2.0, 1 << 20, 1 << 20, 1 << 30, stream=0)
+    assert e.value.status == lib.LSN_ERR_INVALID_ARG
+
+
+def test_bad_shapes_and_pointers_are_rejected(lib):
+    W = lib.base_bf16(1 << 20, 500, 512)                       # N not a multiple of 64
+    with pytest.raises(lib.LsnError) as e:
+        lib.lora_linear_fwd(W, 1 << 20, 16, 1 << 20, 1 << 20, 8, 2.0, 1 << 20, 1 << 20, 1 << 30, stream=0)
+    assert e.value.status == lib.LSN_ERR_INVALID_ARG
+    W = lib.base_bf16(1 << 20, 512, 512)
+    with pytest.raises(lib.LsnError) as e:                     # misaligned x
+        lib.lora_linear_fwd(W, (1 << 20) + 2, 16, 1 << 20, 1 << 20, 8, 2.0, 1 << 20, 1 << 20, 1 << 30, stream=0)
+    assert e.value.status == lib.LSN_ERR_INVALID_ARG
+    with pytest.raises(lib.LsnError) as e:                     # workspace too small
+        lib.lora_linear_fwd(W, 1 << 20, 16, 1 << 20, 1 << 20, 8, 2.0, 1 << 20, 1 << 20, 64, stream=0)
+    assert e.value.status == lib.LSN_ERR_INVALID_ARG
+    w = lib.make_nf4_weight(64, 100, 1 << 20, 1 << 20, 1 << 20, 1 << 20)   # cols % 64 != 0
+    with pytest.raises(lib.LsnError) as e:
+        lib.nf4_dequant(w, 1 << 20, stream=0)
+    assert e.value.status == lib.LSN_ERR_INVALID_ARG
+    w = lib.make_nf4_weight(64, 128, None, 1 << 20, 1 << 20, 1 << 20)       # NULL packed
+    with pytest.raises(lib.LsnError) as e:
+        lib.nf4_dequant(w, 1 << 20, stream=0)
+    assert e.value.status == lib.LSN_ERR_INVALID_ARG
+
+
+def test_empty_weight_is_a_no_op(lib):
+    w = lib.make_nf4_weight(0, 64, None, None, None, None)
+    lib.nf4_dequant(w, None, stream=0)
+
+
+def test_pool_rejects_bad_arguments(lib):
+    with pytest.raises(lib.LsnError) as e:
+        lib.layer_pool_create(0, 1024, 0)
+    assert e.value.status == lib.LSN_ERR_INVALID_ARG
+    with pytest.raises(lib.LsnError) as e:
+        lib.layer_pool_create(2, 0, 0)
+    assert e.value.status == lib.LSN_ERR_INVALID_ARG
+
+
+def test_last_error_is_never_null(lib):
+    assert isinstance(lib.last_error(), str)
+    assert lib.version() >= 100

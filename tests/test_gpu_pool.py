@@ -1,0 +1,135 @@
+"""The layer pool and the bit-exactness gate.
+
+"Exact Layer Streaming" (abstract) gates streaming on bit-exactness against a
+resident run of the same numerics, forward and backward as two separate
+claims, and reports an aliasing defect that left the forward exact while the
+gradients were wrong on most layers above ~165 MiB per NF4 layer (the Soup
+benchmarks README, protocol notes).  Here: streamed == resident with
+torch.equal for every y and dX of every projection and every dA/dB of every
+layer, on stacks of each workload shape (the 72B-shaped layer is ~432 MiB),
+plus a planted aliasing fault that the gate must catch, and host-side fault
+injection."""
+import pytest
+
+from layer_streamed_nf4_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import torch
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from layer_streamed_nf4_b200 import lsnf4
+    return lsnf4
+
+
+def _run(cfg, layers, tokens, mode, fault=None, steps=1):
+    import torch
+    from layer_streamed_nf4_b200 import lsnf4
+    from layer_streamed_nf4_b200.stack import Stack
+    st = Stack(cfg, layers=layers, tokens=tokens, mode=mode, keep_outputs=True)
+    if fault is not None:
+        lsnf4.layer_pool_inject_fault(st.pool, fault)
+    for _ in range(steps):
+        st.step()
+    torch.cuda.synchronize()
+    st.check_status()
+    return st
+
+
+def _compare(a, b):
+    """(forward equal?, backward equal?, list of layers whose dA/dB differ)."""
+    import torch
+    fwd = all(torch.equal(a.y[k], b.y[k]) for k in a.y)
+    bad = sorted({l for (l, pi) in a.dA if not (torch.equal(a.dA[l, pi], b.dA[l, pi]) and
+                                                torch.equal(a.dB[l, pi], b.dB[l, pi]))})
+    bwd = not bad and all(torch.equal(a.dX[k], b.dX[k]) for k in a.dX)
+    return fwd, bwd, bad
+
+
+@pytest.mark.parametrize("name,layers,tokens", [("0.5b", 24, 512), ("3b", 4, 1024), ("8b", 4, 2048), ("72b", 3, 1024)])
+def test_streamed_equals_resident(lib, name, layers, tokens):
+    cfg = synth.STACKS[name]
+    res = _run(cfg, layers, tokens, "resident")
+    stm = _run(cfg, layers, tokens, "streamed", steps=2)
+    fwd, bwd, bad = _compare(stm, res)
+    assert fwd, f"{name}: streamed forward differs from resident"
+    # two streamed steps without accumulation: gradients are those of one step
+    assert bwd, f"{name}: streamed backward differs from resident on layers {bad}"
+    s = stm.pool_stats()
+    assert s["copies"] == (2 * layers - 2) + (2 * layers - 4), s   # first step 2L-2, steady state 2L-4
+    stm.close()
+
+
+def test_no_h2d_equals_resident(lib):
+    cfg = synth.STACKS["8b"]
+    res = _run(cfg, 3, 512, "resident")
+    pre = _run(cfg, 3, 512, "no_h2d")
+    fwd, bwd, bad = _compare(pre, res)
+    assert fwd and bwd, bad
+
+
+def test_planted_aliasing_is_caught(lib):
+    """A pool that hands back a stale slot (the aliasing defect) must fail the gate."""
+    cfg = synth.STACKS["8b"]
+    res = _run(cfg, 4, 256, "resident")
+    bad_run = _run(cfg, 4, 256, "streamed", fault=lib.LSN_POOL_FAULT_STALE_SLOT)
+    fwd, bwd, bad = _compare(bad_run, res)
+    assert not (fwd and bwd), "the bit-exactness gate missed a planted aliasing fault"
+
+
+def test_injected_copy_failure_then_reset(lib):
+    import torch
+    from layer_streamed_nf4_b200.stack import Stack
+    cfg = synth.STACKS["8b"]
+    st = Stack(cfg, layers=3, tokens=256, mode="streamed", keep_outputs=True)
+    lib.layer_pool_inject_fault(st.pool, lib.LSN_POOL_FAULT_COPY_ERROR)
+    with pytest.raises(lib.LsnError) as e:
+        st.step()
+    assert e.value.status == lib.LSN_ERR_CUDA
+    torch.cuda.synchronize()
+    lib.layer_pool_reset(st.pool)
+    st.step()
+    torch.cuda.synchronize()
+    res = _run(cfg, 3, 256, "resident")
+    fwd, bwd, bad = _compare(st, res)
+    assert fwd and bwd, bad
+    st.close()
+
+
+def test_pool_rules(lib):
+    import torch
+    n = 1 << 20
+    host = torch.empty(n, dtype=torch.uint8, pin_memory=True)
+    host2 = torch.empty(n, dtype=torch.uint8, pin_memory=True)
+    host.fill_(1)
+    host2.fill_(2)
+    pool = lib.layer_pool_create(1, n, 0)
+    try:
+        with pytest.raises(lib.LsnError) as e:                       # pageable memory is refused
+            pageable = torch.empty(n, dtype=torch.uint8)
+            lib.layer_pool_register(pool, 0, pageable.data_ptr(), n)
+        assert e.value.status == lib.LSN_ERR_INVALID_ARG
+        with pytest.raises(lib.LsnError) as e:                       # larger than a slot
+            lib.layer_pool_register(pool, 0, host.data_ptr(), n + 1)
+        assert e.value.status == lib.LSN_ERR_INVALID_ARG
+        lib.layer_pool_register(pool, 0, host.data_ptr(), n)
+        lib.layer_pool_register(pool, 1, host2.data_ptr(), n)
+        s = torch.cuda.current_stream()
+        p0 = lib.layer_pool_acquire(pool, 0, s)
+        with pytest.raises(lib.LsnError) as e:                       # the only slot is in use
+            lib.layer_pool_prefetch(pool, 1)
+        assert e.value.status == lib.LSN_ERR_STATE
+        lib.layer_pool_release(pool, 0, s)
+        with pytest.raises(lib.LsnError) as e:                       # release of a layer not held
+            lib.layer_pool_release(pool, 0, s)
+        assert e.value.status == lib.LSN_ERR_STATE
+        p1 = lib.layer_pool_acquire(pool, 1, s)
+        assert p1 == p0                                              # same slot, reused after release
+        lib.layer_pool_release(pool, 1, s)
+        lib.layer_pool_wait_idle(pool, 10000)
+        st = lib.layer_pool_stats(pool)
+        assert st["copies"] == 2 and st["bytes_copied"] == 2 * n and st["misses"] == 2
+    finally:
+        lib.layer_pool_destroy(pool)
