@@ -127,6 +127,30 @@ size_t lsn_nf4_quantize_ws_bytes(int64_t rows, int64_t cols);
 lsn_status nf4_quantize(const float* W, const lsn_nf4_weight* out, void* ws, size_t ws_bytes,
                         lsn_stream_t stream);
 
+/* Largest rows*cols nf4_quantize_noalloc accepts (2^26 elements). */
+#define LSN_NF4_NOALLOC_MAX_ELEMS 67108864LL
+
+/* nf4_quantize without a caller workspace and without allocating anything.
+ * (The pages have no counterpart: this exists for callers of the library.)
+ *
+ * For callers that cannot provide device memory when they quantise -- a host
+ * whose allocator has reserved all device memory up front, a loop that must
+ * not pay for cudaMalloc's implicit synchronisation, a plug-in without an
+ * allocator.  The scratch it needs lives in a fixed array inside this
+ * library's device image: 4 MiB + 32 KiB per device, present on every device
+ * that loads the library until the process exits.  Limit: rows*cols <=
+ * LSN_NF4_NOALLOC_MAX_ELEMS; larger weights are rejected with
+ * LSN_ERR_INVALID_ARG before anything is enqueued.  Results are bit-identical
+ * to nf4_quantize.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls share the one array: calls whose work overlaps on the
+ * GPU (different streams without ordering between them) race and corrupt
+ * each other's results -- order them on one stream or with events.  It calls
+ * no cudaMalloc, cudaFree or allocating library routine. */
+lsn_status nf4_quantize_noalloc(const float* W, const lsn_nf4_weight* out, lsn_stream_t stream);
+
 /* Dequantise *w into bf16 W_out [rows, cols] (device).  HBM-bound. */
 lsn_status nf4_dequant(const lsn_nf4_weight* w, uint16_t* W_out, lsn_stream_t stream);
 

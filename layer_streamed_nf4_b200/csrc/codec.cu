@@ -292,3 +292,78 @@ lsn_status launch_dequant(const lsn_nf4_weight* w, uint16_t* out, cudaStream_t s
 }
 
 }  // namespace lsn
+
+// ------------------------------------------------- allocation-free variant --
+//
+// nf4_quantize needs scratch memory (one fp32 absmax per 64-block and one
+// fp64 partial sum per group of 256 blocks) and takes it from the caller.
+// Some callers cannot hand out device memory at the moment they quantise: a
+// host whose allocator has reserved all device memory up front and allows no
+// other allocation, a latency-critical loop that must not pay for
+// cudaMalloc's implicit device synchronisation, or a plug-in that has no
+// allocator at all.  nf4_quantize_noalloc serves them with a fixed scratch
+// array that lives in this library's device image: it is allocated by the
+// CUDA runtime when the library's module is loaded on a device and stays
+// there until the process exits.
+
+namespace lsn {
+namespace {
+
+constexpr int64_t kNoAllocMaxElems = (int64_t)1 << 26;               // 67,108,864 weight elements
+constexpr int64_t kNoAllocMaxBlocks = kNoAllocMaxElems / 64;         // 1,048,576 absmax values
+constexpr int64_t kNoAllocMaxGroups = kNoAllocMaxBlocks / 256;       // 4,096 partial sums
+constexpr size_t kNoAllocScratchBytes =
+    (size_t)kNoAllocMaxBlocks * sizeof(float) + (size_t)kNoAllocMaxGroups * sizeof(double);
+
+// Shared by every call on a device; holds whatever the last call left.  The
+// quantisation passes write every absmax and partial they later read, so
+// nothing in it has to start at zero.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {nullptr};
+
+// Device address of the scratch array on the current device.  The host-side
+// name g_noalloc_scratch is only a stand-in for the symbol, never a device
+// address, so it is resolved once per device with cudaGetSymbolAddress.
+lsn_status noalloc_scratch(void** out) {
+    int dev = 0;
+    LSN_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return fail(LSN_ERR_UNSUPPORTED, "nf4_quantize_noalloc: device index too large");
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return fail_cuda(e, "nf4_quantize_noalloc: cudaGetSymbolAddress(scratch)");
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return LSN_OK;
+}
+
+}  // namespace
+
+}  // namespace lsn
+
+extern "C" lsn_status nf4_quantize_noalloc(const float* W, const lsn_nf4_weight* out, lsn_stream_t stream) {
+    using namespace lsn;
+    LSN_CHECK_ARG(out != nullptr, "nf4_quantize_noalloc: weight is NULL");
+    LSN_CHECK_ARG(out->rows >= 0 && out->cols >= 0, "nf4_quantize_noalloc: negative shape");
+    LSN_CHECK_ARG(out->cols % 64 == 0, "nf4_quantize_noalloc: cols must be a multiple of 64");
+    const int64_t numel = out->rows * out->cols;
+    if (numel == 0) return LSN_OK;
+    LSN_CHECK_ARG(numel <= kNoAllocMaxElems,
+                  "nf4_quantize_noalloc: rows*cols = " + std::to_string(numel) + " exceeds the fixed scratch limit of " +
+                      std::to_string(kNoAllocMaxElems) + " elements; use nf4_quantize with a caller workspace");
+    LSN_CHECK_ARG(W != nullptr && aligned16(W), "nf4_quantize_noalloc: W must be a 16-byte aligned device pointer");
+    LSN_CHECK_ARG(out->packed && out->absmax_q && out->absmax_s2 && out->offset,
+                  "nf4_quantize_noalloc: NULL array in the NF4 weight");
+    LSN_CHECK_ARG(aligned16(out->packed), "nf4_quantize_noalloc: packed must be 16-byte aligned");
+    if (!device_is_sm100()) return fail(LSN_ERR_UNSUPPORTED, "liblsnf4 is built for sm_100a (B200) only");
+    void* scratch = nullptr;
+    lsn_status s = noalloc_scratch(&scratch);
+    if (s != LSN_OK) return s;
+    return launch_quantize(W, out, scratch, kNoAllocScratchBytes, reinterpret_cast<cudaStream_t>(stream));
+}
+

@@ -39,6 +39,7 @@ EXPORTS = (
     "layer_pool_create", "layer_pool_register", "layer_pool_prefetch", "layer_pool_acquire",
     "layer_pool_release", "layer_pool_wait_idle", "layer_pool_stats", "layer_pool_reset",
     "layer_pool_inject_fault", "layer_pool_destroy", "lsn_timing_enable", "lsn_timing_read",
+    "nf4_quantize_noalloc",
 )
 
 
@@ -91,6 +92,7 @@ for _n in ("lsn_nf4_packed_bytes", "lsn_nf4_absmax_bytes", "lsn_nf4_s2_bytes", "
 _sig("lsn_nf4_blob_layout", None, [_i64, _i64, ctypes.POINTER(_sz)])
 _sig("nf4_quantize", _i, [_vp, ctypes.POINTER(NF4Weight), _vp, _sz, _vp])
 _sig("nf4_dequant", _i, [ctypes.POINTER(NF4Weight), _vp, _vp])
+_sig("nf4_quantize_noalloc", _i, [_vp, ctypes.POINTER(NF4Weight), _vp])
 _sig("lsn_lora_ws_bytes", _sz, [_i64, _i64, _i64, _i, _i])
 _sig("lora_linear_fwd", _i, [ctypes.POINTER(Base), _vp, _i64, _vp, _vp, _i, ctypes.c_float, _vp, _vp, _sz, _vp])
 _sig("lora_linear_bwd", _i, [ctypes.POINTER(Base), _vp, _vp, _i64, _vp, _vp, _i, ctypes.c_float, _vp, _vp, _vp, _i,
@@ -183,6 +185,14 @@ def nf4_weight_in_blob(rows, cols, base_addr: int) -> NF4Weight:
 
 def nf4_quantize(W, out: NF4Weight, ws, ws_bytes: int, stream=None):
     _check(_lib.nf4_quantize(_ptr(W), ctypes.byref(out), _ptr(ws), ws_bytes, _stream(stream)), "nf4_quantize")
+
+
+def nf4_quantize_noalloc(W, out: NF4Weight, stream=None):
+    """nf4_quantize with the library's fixed scratch array instead of a workspace (see lsnf4.h)."""
+    _check(_lib.nf4_quantize_noalloc(_ptr(W), ctypes.byref(out), _stream(stream)), "nf4_quantize_noalloc")
+
+
+NF4_NOALLOC_MAX_ELEMS = 1 << 26
 
 
 def nf4_dequant(w: NF4Weight, W_out, stream=None):
