@@ -369,6 +369,56 @@ def run_reference(args):
     print(json.dumps(line))
 
 
+def run_case(args):
+    """One projection of the 8B-shaped stack, lora_linear_fwd + lora_linear_bwd, NF4 base, repeated: the small,
+    self-contained launch sequence used for focused profiles (prints its own JSON line)."""
+    import torch
+    from layer_streamed_nf4_b200 import lsnf4, synth
+    cfg = synth.STACKS[WORKLOAD]
+    proj = {name: (pi, K, N) for pi, (name, K, N) in enumerate(cfg.projections)}
+    pi, K, N = proj[args.case]
+    T, r = args.tokens or cfg.tokens, cfg.rank
+    scale = cfg.alpha / r
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    W = synth.device_normal((N, K), 0.02, synth.SEED, 0, pi, synth.T_W, device=dev)
+    blob = torch.zeros(lsnf4.nf4_blob_bytes(N, K), dtype=torch.uint8, device=dev)
+    w = lsnf4.nf4_weight_in_blob(N, K, blob.data_ptr())
+    qws = torch.zeros(lsnf4.nf4_quantize_ws_bytes(N, K), dtype=torch.uint8, device=dev)
+    lsnf4.nf4_quantize(W, w, qws, qws.numel())
+    del W, qws
+    base = lsnf4.base_nf4(w)
+    x = synth.device_normal((T, K), 1.0, synth.SEED, 0, pi, synth.T_X, device=dev, dtype=torch.bfloat16)
+    dY = synth.device_normal((T, N), 1.0, synth.SEED, 0, pi, synth.T_DY, device=dev, dtype=torch.bfloat16)
+    A = synth.device_uniform((r, K), 1.0 / K ** 0.5, synth.SEED, 0, pi, synth.T_A, device=dev, dtype=torch.bfloat16)
+    B = synth.device_normal((N, r), 0.01, synth.SEED, 0, pi, synth.T_B, device=dev, dtype=torch.bfloat16)
+    y = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
+    dX = torch.empty((T, K), dtype=torch.bfloat16, device=dev)
+    dA = torch.zeros((r, K), dtype=torch.float32, device=dev)
+    dB = torch.zeros((N, r), dtype=torch.float32, device=dev)
+    nbytes = lsnf4.lora_ws_bytes(T, K, N, r, lsnf4.LSN_BASE_NF4)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+
+    def one():
+        lsnf4.lora_linear_fwd(base, x, T, A, B, r, scale, y, ws, nbytes)
+        lsnf4.lora_linear_bwd(base, x, dY, T, A, B, r, scale, dX, dA, dB, False, ws, nbytes)
+
+    for _ in range(args.warmup):
+        one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        one()
+    e1.record()
+    e1.synchronize()
+    lsnf4.ws_status(ws)
+    ms = e0.elapsed_time(e1) / args.steps
+    flop = 2.0 * T * N * (K + r) + 2.0 * T * K * (N + r)
+    print(json.dumps({"case": args.case, "T": T, "K": K, "N": N, "r": r, "ms_fwd_bwd": ms,
+                      "gemm_tflops_if_all_time_were_gemm": flop / (ms / 1e3) / 1e12}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -384,10 +434,13 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=32)
     ap.add_argument("--cpu-budget", type=float, default=60.0)
     ap.add_argument("--ref-rows", type=int, default=4)
+    ap.add_argument("--case", default="", help="profile one 8B projection (q,k,v,o,gate,up,down) instead of the stack")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
         run_reference(args)
+    elif args.case:
+        run_case(args)
     else:
         run_ours(args)
 

@@ -17,7 +17,8 @@ lsn_status launch_gemm(const uint16_t* A, int64_t lda, const uint16_t* B, int64_
                        const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D, int64_t ldd,
                        int* err, cudaStream_t st);
 lsn_status launch_lora_down(const uint16_t* X, const uint16_t* W, bool w_rk, int64_t T, int64_t Kd, int r,
-                            float scale, float* u32, uint16_t* u16, cudaStream_t st);
+                            float scale, float* u32, uint16_t* u16, uint16_t* wt, float* partial, cudaStream_t st);
+size_t down_ws_bytes(int64_t T, int64_t Kd, int r);
 lsn_status launch_lora_tgrad(const float* G, const uint16_t* X, bool out_rk, int64_t T, int64_t Kd, int r,
                              float scale, int accumulate, float* out, float* partial, cudaStream_t st);
 size_t tgrad_ws_bytes(int64_t T, int64_t Kd, int r);
@@ -91,13 +92,16 @@ lsn_status check_nf4(const lsn_nf4_weight* w, const char* who) {
 //   u32  fp32 [T, r]     x A^T
 //   g32  fp32 [T, r]     dY B
 //   s16  bf16 [T, r]     bf16(s u) or bf16(s g)
-//   part fp32 partials of the token reductions
+//   bt   bf16 [r, N]     B transposed for the backward's g = dY B
+//   part fp32 split partials (down projections and token reductions, used
+//        one after the other on the stream)
 //   w16  bf16 [N, K]     dequantised base (NF4 base only)
 struct LoraWs {
     int* err;
     float* u32;
     float* g32;
     uint16_t* s16;
+    uint16_t* bt;
     float* part;
     uint16_t* w16;
     size_t total;
@@ -112,8 +116,10 @@ LoraWs carve(void* ws, int64_t T, int64_t K, int64_t N, int r, int kind) {
     w.u32 = reinterpret_cast<float*>(take((size_t)T * r * 4));
     w.g32 = reinterpret_cast<float*>(take((size_t)T * r * 4));
     w.s16 = reinterpret_cast<uint16_t*>(take((size_t)T * r * 2));
-    const size_t pa = tgrad_ws_bytes(T, K, r), pb = tgrad_ws_bytes(T, N, r);
-    w.part = reinterpret_cast<float*>(take(pa > pb ? pa : pb));
+    w.bt = reinterpret_cast<uint16_t*>(take((size_t)N * r * 2));
+    size_t part = tgrad_ws_bytes(T, K, r);
+    for (size_t v : {tgrad_ws_bytes(T, N, r), down_ws_bytes(T, K, r), down_ws_bytes(T, N, r)}) part = v > part ? v : part;
+    w.part = reinterpret_cast<float*>(take(part));
     w.w16 = reinterpret_cast<uint16_t*>(take(kind == LSN_BASE_NF4 ? (size_t)N * K * 2 : 0));
     w.total = off;
     return w;
@@ -156,16 +162,17 @@ lsn_status timed_dequant(const lsn_nf4_weight* w, uint16_t* out, cudaStream_t st
 }
 
 lsn_status timed_down(const uint16_t* X, const uint16_t* W, bool w_rk, int64_t T, int64_t Kd, int r, float scale,
-                      float* u32, uint16_t* u16, cudaStream_t st) {
+                      float* u32, uint16_t* u16, const LoraWs& w, cudaStream_t st) {
     const double bytes = 2.0 * T * Kd + 2.0 * r * Kd + (u32 ? 4.0 * T * r : 0.0) + (u16 ? 2.0 * T * r : 0.0);
-    TimingScope ts(LSN_K_LORA_DOWN, bytes, st);
-    return launch_lora_down(X, W, w_rk, T, Kd, r, scale, u32, u16, st);
+    const int kernels = 1 + (w_rk ? 0 : 1) + (down_ws_bytes(T, Kd, r) > 0 ? 1 : 0);
+    TimingScope ts(LSN_K_LORA_DOWN, bytes, st, kernels);
+    return launch_lora_down(X, W, w_rk, T, Kd, r, scale, u32, u16, w.bt, w.part, st);
 }
 
 lsn_status timed_tgrad(const float* G, const uint16_t* X, bool out_rk, int64_t T, int64_t Kd, int r, float scale,
                        int accumulate, float* out, float* partial, cudaStream_t st) {
     const double bytes = 2.0 * T * Kd + 4.0 * T * r + 4.0 * r * Kd * (accumulate ? 2.0 : 1.0);
-    TimingScope ts(LSN_K_LORA_TGRAD, bytes, st, tgrad_splits(T, Kd) > 1 ? 2 : 1);
+    TimingScope ts(LSN_K_LORA_TGRAD, bytes, st, (r + 15) / 16 + (tgrad_splits(T, Kd) > 1 ? 1 : 0));
     return launch_lora_tgrad(G, X, out_rk, T, Kd, r, scale, accumulate, out, partial, st);
 }
 
@@ -248,7 +255,7 @@ lsn_status lora_linear_fwd(const lsn_base* W, const uint16_t* x, int64_t T, cons
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int64_t N = W->rows, K = W->cols;
     LoraWs w = carve(ws, T, K, N, r, W->kind);
-    if ((s = timed_down(x, A, true, T, K, r, scale, nullptr, w.s16, st)) != LSN_OK) return s;
+    if ((s = timed_down(x, A, true, T, K, r, scale, nullptr, w.s16, w, st)) != LSN_OK) return s;
     const uint16_t* Wb = W->bf16;
     if (W->kind == LSN_BASE_NF4) {
         if ((s = timed_dequant(&W->nf4, w.w16, st)) != LSN_OK) return s;
@@ -270,8 +277,8 @@ lsn_status lora_linear_bwd(const lsn_base* W, const uint16_t* x, const uint16_t*
     const int64_t N = W->rows, K = W->cols;
     LoraWs w = carve(ws, T, K, N, r, W->kind);
     if (T > 0) {
-        if ((s = timed_down(dY, B, false, T, N, r, scale, w.g32, w.s16, st)) != LSN_OK) return s;
-        if ((s = timed_down(x, A, true, T, K, r, scale, w.u32, nullptr, st)) != LSN_OK) return s;
+        if ((s = timed_down(dY, B, false, T, N, r, scale, w.g32, w.s16, w, st)) != LSN_OK) return s;
+        if ((s = timed_down(x, A, true, T, K, r, scale, w.u32, nullptr, w, st)) != LSN_OK) return s;
         if (dX) {
             const uint16_t* Wb = W->bf16;
             if (W->kind == LSN_BASE_NF4) {

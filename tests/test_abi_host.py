@@ -105,6 +105,15 @@ def test_pool_rejects_bad_arguments(lib):
     assert e.value.status == lib.LSN_ERR_INVALID_ARG
 
 
+@pytest.mark.parametrize("T", [0, 1, 63, 64, 2048, 100000])
+@pytest.mark.parametrize("K,N", [(64, 64), (896, 4864), (4096, 1024), (14336, 4096)])
+def test_workspace_sizes_for_edge_shapes(lib, T, K, N):
+    for r in (8, 16, 64):
+        for kind in (lib.LSN_BASE_NF4, lib.LSN_BASE_BF16):
+            n = lib.lora_ws_bytes(T, K, N, r, kind)
+            assert n >= 256 + (N * K * 2 if kind == lib.LSN_BASE_NF4 else 0)
+
+
 def test_last_error_is_never_null(lib):
     assert isinstance(lib.last_error(), str)
     assert lib.version() >= 100
