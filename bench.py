@@ -138,6 +138,7 @@ def run_ours(args):
         return float(t.item())
 
     results = {}
+    host_issue = {}
     kernel = None
     pool_stats = None
     clocks = None
@@ -161,10 +162,13 @@ def run_ours(args):
             sampler.__enter__()
         with torch.cuda.stream(stream):
             t0.record(stream)
+            h0 = time.perf_counter()
             for _ in range(args.steps):
                 st.step()
+            host_ms = (time.perf_counter() - h0) * 1e3 / args.steps
             t1.record(stream)
         t1.synchronize()
+        host_issue[mode] = host_ms
         if sampler:
             sampler.__exit__()
             clocks = sampler.summary()
@@ -251,7 +255,8 @@ def run_ours(args):
     dq = kernel["dequant"]
     h2d_gbs = (pool_stats["bytes_copied"] / (pool_stats["copy_ms"] / 1e3) / 1e9
                if pool_stats and pool_stats["copy_ms"] > 0 else None)
-    extra_modes = {m: {"ms_per_step": results[m], "tok_s": world * T / (results[m] / 1e3),
+    extra_modes = {m: {"ms_per_step": results[m], "host_issue_ms_per_step": host_issue.get(m),
+                       "tok_s": world * T / (results[m] / 1e3),
                        "pct_bf16_peak": 100 * flop_step / (results[m] / 1e3) / 1e12 / peaks["bf16_tflops"]}
                    for m in results}
     traffic = _traffic_from_profile()

@@ -17,10 +17,11 @@ lsn_status launch_gemm(const uint16_t* A, int64_t lda, const uint16_t* B, int64_
                        const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D, int64_t ldd,
                        int* err, cudaStream_t st);
 lsn_status launch_lora_down(const uint16_t* X, const uint16_t* W, bool w_rk, int64_t T, int64_t Kd, int r,
-                            float scale, float* u32, uint16_t* u16, uint16_t* wt, float* partial, cudaStream_t st);
+                            float scale, float* u32, uint16_t* u16, float* partial, int* counters, cudaStream_t st);
 size_t down_ws_bytes(int64_t T, int64_t Kd, int r);
 lsn_status launch_lora_tgrad(const float* G, const uint16_t* X, bool out_rk, int64_t T, int64_t Kd, int r,
-                             float scale, int accumulate, float* out, float* partial, cudaStream_t st);
+                             float scale, int accumulate, float* out, float* partial, int* counters, cudaStream_t st);
+size_t split_counter_count(int64_t T, int64_t K, int64_t N);
 size_t tgrad_ws_bytes(int64_t T, int64_t Kd, int r);
 int tgrad_splits(int64_t T, int64_t Kd);
 
@@ -88,20 +89,22 @@ lsn_status check_nf4(const lsn_nf4_weight* w, const char* who) {
 }
 
 // Workspace layout of the LoRA calls (each region 256-byte aligned):
-//   [0, 256)  status word of the GEMM kernels (must be zero-filled once)
+//   [0, 256)  status word of the GEMM kernels
+//   cnt  int32           tickets of the split reductions (self-resetting)
 //   u32  fp32 [T, r]     x A^T
 //   g32  fp32 [T, r]     dY B
 //   s16  bf16 [T, r]     bf16(s u) or bf16(s g)
-//   bt   bf16 [r, N]     B transposed for the backward's g = dY B
 //   part fp32 split partials (down projections and token reductions, used
 //        one after the other on the stream)
 //   w16  bf16 [N, K]     dequantised base (NF4 base only)
+// The status word and the tickets must be zero when the workspace is first
+// used: fill the workspace with zeros once, when it is allocated.
 struct LoraWs {
     int* err;
+    int* cnt;
     float* u32;
     float* g32;
     uint16_t* s16;
-    uint16_t* bt;
     float* part;
     uint16_t* w16;
     size_t total;
@@ -113,10 +116,10 @@ LoraWs carve(void* ws, int64_t T, int64_t K, int64_t N, int r, int kind) {
     char* b = reinterpret_cast<char*>(ws);
     auto take = [&](size_t bytes) { char* p = b ? b + off : nullptr; off += round_up(bytes, 256); return p; };
     w.err = reinterpret_cast<int*>(take(256));
+    w.cnt = reinterpret_cast<int*>(take(split_counter_count(T, K, N) * sizeof(int)));
     w.u32 = reinterpret_cast<float*>(take((size_t)T * r * 4));
     w.g32 = reinterpret_cast<float*>(take((size_t)T * r * 4));
     w.s16 = reinterpret_cast<uint16_t*>(take((size_t)T * r * 2));
-    w.bt = reinterpret_cast<uint16_t*>(take((size_t)N * r * 2));
     size_t part = tgrad_ws_bytes(T, K, r);
     for (size_t v : {tgrad_ws_bytes(T, N, r), down_ws_bytes(T, K, r), down_ws_bytes(T, N, r)}) part = v > part ? v : part;
     w.part = reinterpret_cast<float*>(take(part));
@@ -164,16 +167,15 @@ lsn_status timed_dequant(const lsn_nf4_weight* w, uint16_t* out, cudaStream_t st
 lsn_status timed_down(const uint16_t* X, const uint16_t* W, bool w_rk, int64_t T, int64_t Kd, int r, float scale,
                       float* u32, uint16_t* u16, const LoraWs& w, cudaStream_t st) {
     const double bytes = 2.0 * T * Kd + 2.0 * r * Kd + (u32 ? 4.0 * T * r : 0.0) + (u16 ? 2.0 * T * r : 0.0);
-    const int kernels = 1 + (w_rk ? 0 : 1) + (down_ws_bytes(T, Kd, r) > 0 ? 1 : 0);
-    TimingScope ts(LSN_K_LORA_DOWN, bytes, st, kernels);
-    return launch_lora_down(X, W, w_rk, T, Kd, r, scale, u32, u16, w.bt, w.part, st);
+    TimingScope ts(LSN_K_LORA_DOWN, bytes, st, 1);
+    return launch_lora_down(X, W, w_rk, T, Kd, r, scale, u32, u16, w.part, w.cnt, st);
 }
 
 lsn_status timed_tgrad(const float* G, const uint16_t* X, bool out_rk, int64_t T, int64_t Kd, int r, float scale,
-                       int accumulate, float* out, float* partial, cudaStream_t st) {
+                       int accumulate, float* out, const LoraWs& w, cudaStream_t st) {
     const double bytes = 2.0 * T * Kd + 4.0 * T * r + 4.0 * r * Kd * (accumulate ? 2.0 : 1.0);
-    TimingScope ts(LSN_K_LORA_TGRAD, bytes, st, (r + 15) / 16 + (tgrad_splits(T, Kd) > 1 ? 1 : 0));
-    return launch_lora_tgrad(G, X, out_rk, T, Kd, r, scale, accumulate, out, partial, st);
+    TimingScope ts(LSN_K_LORA_TGRAD, bytes, st, 1);
+    return launch_lora_tgrad(G, X, out_rk, T, Kd, r, scale, accumulate, out, w.part, w.cnt, st);
 }
 
 lsn_status timed_gemm(int kind, const uint16_t* A, int64_t lda, const uint16_t* B, int64_t ldb, bool b_mn,
@@ -290,8 +292,8 @@ lsn_status lora_linear_bwd(const lsn_base* W, const uint16_t* x, const uint16_t*
         }
     }
     // With T == 0 the reductions write zeros (or leave accumulators unchanged).
-    if ((s = timed_tgrad(w.g32, x, true, T, K, r, scale, accumulate, dA, w.part, st)) != LSN_OK) return s;
-    return timed_tgrad(w.u32, dY, false, T, N, r, scale, accumulate, dB, w.part, st);
+    if ((s = timed_tgrad(w.g32, x, true, T, K, r, scale, accumulate, dA, w, st)) != LSN_OK) return s;
+    return timed_tgrad(w.u32, dY, false, T, N, r, scale, accumulate, dB, w, st);
 }
 
 lsn_status lsn_ws_status(void* ws, lsn_stream_t stream) {

@@ -14,21 +14,7 @@ namespace lsn {
 
 namespace {
 
-// ----------------------------------------------------------- down proj ---
-//
-// out[t, j] = sum_k X[t, k] * W[j, k] for j < r (W row-major [r, Kd]; the
-// backward's B [N, r] is first transposed into that layout).  A CTA owns 64
-// token rows and one split of the K range; 64-wide K chunks of X and W are
-// staged in shared memory by cp.async through a 4-stage ring (rows padded to
-// 144 bytes so ldmatrix is conflict-free), and each warp multiplies its 16
-// rows with W on the warp-level tensor-core instruction (mma.sync m16n8k16,
-// bf16 in, fp32 accumulate): the inputs are exact bf16 values, so this is the
-// exact product rounded only by fp32 accumulation.  The big contractions use
-// tcgen05; this skinny one is bound by the HBM read of X.
-constexpr int kDnWarps = 4;
-constexpr int kDnRows = 16 * kDnWarps;       // token rows per CTA
-constexpr int kDnStages = 4;
-constexpr int kDnPitch = 72;                 // bf16 per staged row (64 + 8 padding)
+// ------------------------------------------------------------- helpers ---
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                uint32_t b0, uint32_t b1) {
@@ -39,8 +25,13 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ void ldmatrix_x4(uint32_t saddr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+__device__ __forceinline__ void ldsm_x4(uint32_t saddr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(saddr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t saddr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                  : "r"(saddr));
 }
@@ -53,17 +44,66 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-template <int NT>   // NT n-tiles of 8 rank columns: r = 8 * NT
+// Two bf16 values packed low/high into one register.
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) { return pack_bf16x2(lo, hi); }
+
+// Deterministic split reduction: every CTA of a group writes its partial, then
+// the CTA that finishes last (a ticket from an integer counter) adds the
+// partials in split order.  The counter is reset for the next launch.  Returns
+// true (in every thread) in the last CTA, after a fence that makes the other
+// CTAs' partials visible.
+__device__ __forceinline__ bool last_in_group(int* counter, int nsplit) {
+    __shared__ int ticket;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        ticket = atomicAdd(counter, 1);
+        if (ticket == nsplit - 1) atomicExch(counter, 0);
+    }
+    __syncthreads();
+    const bool last = ticket == nsplit - 1;
+    if (last) __threadfence();
+    return last;
+}
+
+// ----------------------------------------------------------- down proj ---
+//
+// out[t, j] = sum_k X[t, k] * Wt(j, k) for j < r, with W given either as
+// A [r, Kd] (u = x A^T) or as B [Kd, r] (g = dY B).  A CTA owns 64 token rows
+// and one split of the K range; 64-wide K chunks of X and W are staged in
+// shared memory by cp.async through a 4-stage ring (rows padded so ldmatrix
+// is conflict-free), and each warp multiplies its 16 rows with W on the
+// warp-level tensor-core instruction (mma.sync m16n8k16, bf16 in, fp32
+// accumulate; the inputs are exact bf16 values).  W in the B layout is read
+// with ldmatrix.trans, so no transposed copy is made.  The big contractions
+// use tcgen05; this skinny one is bound by the HBM read of X.
+constexpr int kDnWarps = 4;
+constexpr int kDnRows = 16 * kDnWarps;       // token rows per CTA
+constexpr int kDnStages = 4;
+constexpr int kDnPitch = 72;                 // bf16 per staged X row (64 + 8 padding)
+
+template <int NT, bool B_KR>
+struct DownSmem {
+    static constexpr int R = 8 * NT;
+    static constexpr int NP = (NT + 1) / 2;                       // n-tile pairs
+    static constexpr int WROWS = B_KR ? 64 : 16 * NP;             // staged W rows
+    static constexpr int WPITCH = B_KR ? 16 * NP + 8 : kDnPitch;  // bf16 per staged W row
+    static constexpr size_t X_BYTES = sizeof(uint16_t) * kDnStages * kDnRows * kDnPitch;
+    static constexpr size_t W_BYTES = sizeof(uint16_t) * kDnStages * WROWS * WPITCH;
+    static constexpr size_t BYTES = X_BYTES + W_BYTES;
+};
+
+template <int NT, bool B_KR>
 __global__ void __launch_bounds__(128) lora_down_kernel(const uint16_t* __restrict__ X, const uint16_t* __restrict__ W,
-                                                        int64_t T, int64_t Kd, int chunks_per_split, float scale,
-                                                        float* __restrict__ u32, uint16_t* __restrict__ u16,
-                                                        float* __restrict__ partial) {
-    constexpr int R = 8 * NT;
-    constexpr int NP = (NT + 1) / 2;          // n-tile pairs (W rows padded to 16 * NP with zeros)
-    constexpr int WR = 16 * NP;
+                                                        int64_t T, int64_t Kd, int chunks_per_split, int nsplit,
+                                                        float scale, float* __restrict__ u32,
+                                                        uint16_t* __restrict__ u16, float* __restrict__ partial,
+                                                        int* __restrict__ counters) {
+    using L = DownSmem<NT, B_KR>;
+    constexpr int R = L::R, NP = L::NP, WROWS = L::WROWS, WPITCH = L::WPITCH;
     extern __shared__ __align__(16) uint8_t dn_smem[];
     auto xs = reinterpret_cast<uint16_t (*)[kDnRows][kDnPitch]>(dn_smem);
-    auto ws = reinterpret_cast<uint16_t (*)[WR][kDnPitch]>(dn_smem + sizeof(uint16_t) * kDnStages * kDnRows * kDnPitch);
+    auto ws = reinterpret_cast<uint16_t (*)[WROWS][WPITCH]>(dn_smem + L::X_BYTES);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t row_base = (int64_t)blockIdx.x * kDnRows;
     const int64_t nchunks = Kd / 64;
@@ -72,21 +112,25 @@ __global__ void __launch_bounds__(128) lora_down_kernel(const uint16_t* __restri
     const int64_t nc = c_end > c_begin ? c_end - c_begin : 0;
 
     auto load = [&](int stage, int64_t c) {
-        // X: 64 rows x 128 bytes = 512 pieces of 16 bytes, 4 per thread.
         #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 4; ++i) {                     // X: 64 rows x 8 pieces of 16 bytes
             const int p = tid + i * 128, row = p >> 3, piece = p & 7;
             const int64_t t = row_base + row;
             const bool ok = t < T;
-            const uint16_t* src = X + (ok ? t : 0) * Kd + c * 64 + piece * 8;
-            cp_async16(smem_u32(&xs[stage][row][piece * 8]), src, ok ? 16u : 0u);
+            cp_async16(smem_u32(&xs[stage][row][piece * 8]), X + (ok ? t : 0) * Kd + c * 64 + piece * 8, ok ? 16u : 0u);
         }
-        // W: WR rows x 128 bytes; rows >= R are zero.
-        for (int p = tid; p < WR * 8; p += 128) {
-            const int row = p >> 3, piece = p & 7;
-            const bool ok = row < R;
-            const uint16_t* src = W + (int64_t)(ok ? row : 0) * Kd + c * 64 + piece * 8;
-            cp_async16(smem_u32(&ws[stage][row][piece * 8]), src, ok ? 16u : 0u);
+        if (B_KR) {                                       // W = B [Kd, r]: 64 rows x r/8 pieces
+            for (int p = tid; p < 64 * NT; p += 128) {
+                const int row = p / NT, piece = p % NT;
+                cp_async16(smem_u32(&ws[stage][row][piece * 8]), W + (c * 64 + row) * (int64_t)R + piece * 8, 16u);
+            }
+        } else {                                          // W = A [r, Kd]: WROWS rows x 8 pieces
+            for (int p = tid; p < WROWS * 8; p += 128) {
+                const int row = p >> 3, piece = p & 7;
+                const bool ok = row < R;
+                cp_async16(smem_u32(&ws[stage][row][piece * 8]), W + (int64_t)(ok ? row : 0) * Kd + c * 64 + piece * 8,
+                           ok ? 16u : 0u);
+            }
         }
     };
 
@@ -99,11 +143,14 @@ __global__ void __launch_bounds__(128) lora_down_kernel(const uint16_t* __restri
         if (s < nc) load(s, c_begin + s);
         cp_async_commit();
     }
-    // ldmatrix row addresses: A (16 rows of the warp, 16 columns), B (16 W rows, 16 columns).
+    // ldmatrix lane addresses (matrix i = lanes 8i..8i+7):
+    //   X (A operand): rows warp*16 + {0-7, 8-15, 0-7, 8-15}, columns {0, 0, 8, 8}
+    //   A [r, Kd]:     W rows {0-7, 0-7, 8-15, 8-15} of the pair, columns {0, 8, 0, 8}
+    //   B [Kd, r]:     K rows {0-7, 8-15, 0-7, 8-15}, rank columns {0, 0, 8, 8}, transposed
     const int a_row = warp * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
     const int a_col = 8 * (lane >> 4);
-    const int b_row = (lane & 7) + 8 * (lane >> 4);
-    const int b_col = 8 * ((lane >> 3) & 1);
+    const int w_row = B_KR ? (lane & 7) + 8 * ((lane >> 3) & 1) : (lane & 7) + 8 * (lane >> 4);
+    const int w_col = B_KR ? 8 * (lane >> 4) : 8 * ((lane >> 3) & 1);
     for (int64_t i = 0; i < nc; ++i) {
         cp_async_wait<kDnStages - 2>();
         __syncthreads();
@@ -111,17 +158,17 @@ __global__ void __launch_bounds__(128) lora_down_kernel(const uint16_t* __restri
         #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
             uint32_t a0, a1, a2, a3;
-            ldmatrix_x4(smem_u32(&xs[st][a_row][ks * 16 + a_col]), a0, a1, a2, a3);
+            ldsm_x4(smem_u32(&xs[st][a_row][ks * 16 + a_col]), a0, a1, a2, a3);
             #pragma unroll
             for (int p = 0; p < NP; ++p) {
                 uint32_t b00, b01, b10, b11;
-                ldmatrix_x4(smem_u32(&ws[st][p * 16 + b_row][ks * 16 + b_col]), b00, b01, b10, b11);
+                if (B_KR) ldsm_x4_t(smem_u32(&ws[st][ks * 16 + w_row][p * 16 + w_col]), b00, b01, b10, b11);
+                else      ldsm_x4(smem_u32(&ws[st][p * 16 + w_row][ks * 16 + w_col]), b00, b01, b10, b11);
                 mma_bf16_16816(acc[2 * p], a0, a1, a2, a3, b00, b01);
                 mma_bf16_16816(acc[2 * p + 1], a0, a1, a2, a3, b10, b11);
             }
         }
-        // Refill the stage consumed one iteration ago (all warps are past it).
-        const int64_t nxt = i + kDnStages - 1;
+        const int64_t nxt = i + kDnStages - 1;            // refill the stage consumed last iteration
         if (nxt < nc) load((int)(nxt % kDnStages), c_begin + nxt);
         cp_async_commit();
     }
@@ -131,135 +178,137 @@ __global__ void __launch_bounds__(128) lora_down_kernel(const uint16_t* __restri
     const int g = lane >> 2, q = lane & 3;
     const int64_t row0 = row_base + warp * 16 + g, row1 = row0 + 8;
     const bool ok0 = row0 < T, ok1 = row1 < T;
+    auto emit = [&](int64_t row, int j, float v) {
+        if (u32) u32[row * R + j] = v;
+        if (u16) u16[row * R + j] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(scale, v)));
+    };
+    if (nsplit == 1) {
+        #pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const int j = n * 8 + 2 * q;
+            if (ok0) { emit(row0, j, acc[n][0]); emit(row0, j + 1, acc[n][1]); }
+            if (ok1) { emit(row1, j, acc[n][2]); emit(row1, j + 1, acc[n][3]); }
+        }
+        return;
+    }
+    float* pp = partial + (int64_t)blockIdx.y * T * R;
     #pragma unroll
     for (int n = 0; n < NT; ++n) {
         const int j = n * 8 + 2 * q;
-        if (partial != nullptr) {
-            float* pp = partial + (int64_t)blockIdx.y * T * R;
-            if (ok0) { pp[row0 * R + j] = acc[n][0]; pp[row0 * R + j + 1] = acc[n][1]; }
-            if (ok1) { pp[row1 * R + j] = acc[n][2]; pp[row1 * R + j + 1] = acc[n][3]; }
-        } else {
-            if (ok0) {
-                if (u32) { u32[row0 * R + j] = acc[n][0]; u32[row0 * R + j + 1] = acc[n][1]; }
-                if (u16) {
-                    u16[row0 * R + j] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(scale, acc[n][0])));
-                    u16[row0 * R + j + 1] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(scale, acc[n][1])));
-                }
-            }
-            if (ok1) {
-                if (u32) { u32[row1 * R + j] = acc[n][2]; u32[row1 * R + j + 1] = acc[n][3]; }
-                if (u16) {
-                    u16[row1 * R + j] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(scale, acc[n][2])));
-                    u16[row1 * R + j + 1] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(scale, acc[n][3])));
-                }
-            }
-        }
+        if (ok0) { pp[row0 * R + j] = acc[n][0]; pp[row0 * R + j + 1] = acc[n][1]; }
+        if (ok1) { pp[row1 * R + j] = acc[n][2]; pp[row1 * R + j + 1] = acc[n][3]; }
     }
-}
-
-// Sum the K-split partials of the down projection in split order.
-__global__ void lora_down_finish(const float* __restrict__ partial, int64_t n, int nsplit, float scale,
-                                 float* __restrict__ u32, uint16_t* __restrict__ u16) {
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= n) return;
-    float s = 0.0f;
-    for (int k = 0; k < nsplit; ++k) s += partial[(int64_t)k * n + i];
-    if (u32) u32[i] = s;
-    if (u16) u16[i] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(scale, s)));
-}
-
-// B [N, r] -> Bt [r, N] (bf16), so the backward's g = dY B uses the same
-// down-projection kernel as u = x A^T.
-__global__ void transpose_nr_kernel(const uint16_t* __restrict__ B, int64_t N, int r, uint16_t* __restrict__ Bt) {
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= N * r) return;
-    const int64_t n = i / r, j = i % r;
-    Bt[j * N + n] = B[i];
+    if (!last_in_group(counters + blockIdx.x, nsplit)) return;
+    for (int idx = tid; idx < kDnRows * R; idx += 128) {
+        const int64_t row = row_base + idx / R;
+        const int j = idx % R;
+        if (row >= T) continue;
+        float sum = 0.0f;
+        for (int sp = 0; sp < nsplit; ++sp) sum += __ldcg(partial + ((int64_t)sp * T + row) * R + j);
+        emit(row, j, sum);
+    }
 }
 
 // -------------------------------------------------------- token reduce ---
 //
-// R[j, k] = sum_{t in split} G[t, j] * X[t, k].  A CTA owns 128 columns k
-// (lane l owns k0 + 4l .. 4l+3) and one split of the tokens, staged 32
-// tokens at a time (X tile 32 x 128 bf16, G tile 32 x NJ fp32) by cp.async
-// through a 4-stage ring; its four warps take tokens w, w+4, ... of each tile
-// and keep NJ x 4 fp32 accumulators per lane (register-resident: all indices
-// are compile-time constants), reading G rows as broadcast 16-byte loads.
-// The four warp partials are added in warp order.  With one split the result
-// is finished here (scale, optional accumulate); otherwise partial
-// [split][r][Kd] is written and summed in split order by lora_tgrad_finish.
+// R[j, k] = sum_{t in split} G[t, j] * X[t, k] (dA with G = g, X = x; dB with
+// G = u, X = dY).  On the warp-level tensor-core instruction with M = k, N = j
+// and the tokens as the contraction: X tiles [32 t x 128 k] are staged by
+// cp.async (4 stages) and read transposed with ldmatrix.trans; G is fp32, so
+// each element enters as two bf16 MMAs, hi = bf16(G) and lo = bf16(G - hi),
+// which leaves a relative error below 2^-17 per product before fp32
+// accumulation.  A CTA owns 128 columns k (warp w: k0+32w .. +31) and one
+// token split; splits are combined by the last CTA of each column tile in
+// split order.
 constexpr int kTgCols = 128;
-constexpr int kTgWarps = 4;
-constexpr int kTgTok = 32;          // tokens per staged tile
+constexpr int kTgTok = 32;          // tokens per staged tile (two MMA k-steps)
 constexpr int kTgStages = 4;
+constexpr int kTgXPitch = kTgCols + 8;
 
-template <int NJ, bool OUT_RK>
+template <int NT>
+struct TgSmem {
+    static constexpr int GPITCH = 8 * NT + 4;
+    static constexpr size_t X_BYTES = sizeof(uint16_t) * kTgStages * kTgTok * kTgXPitch;
+    static constexpr size_t G_BYTES = sizeof(float) * kTgStages * kTgTok * GPITCH;
+    static constexpr size_t BYTES = X_BYTES + G_BYTES;
+};
+
+template <int NT, bool OUT_RK>
 __global__ void __launch_bounds__(128) lora_tgrad_kernel(const float* __restrict__ G, const uint16_t* __restrict__ X,
-                                                         int64_t T, int64_t Kd, int r, int j0, int64_t per_split,
-                                                         int nsplit, float scale, int accumulate,
-                                                         float* __restrict__ out, float* __restrict__ partial) {
-    // Dynamic shared memory: the staging ring, later reused for the warp
-    // partials (red) once every copy has landed.
+                                                         int64_t T, int64_t Kd, int64_t per_split, int nsplit,
+                                                         float scale, int accumulate, float* __restrict__ out,
+                                                         float* __restrict__ partial, int* __restrict__ counters) {
+    using L = TgSmem<NT>;
+    constexpr int R = 8 * NT, GPITCH = L::GPITCH;
     extern __shared__ __align__(16) uint8_t tg_smem[];
-    auto xs = reinterpret_cast<uint16_t (*)[kTgTok][kTgCols]>(tg_smem);
-    auto gs = reinterpret_cast<float (*)[kTgTok][NJ]>(tg_smem + sizeof(uint16_t) * kTgStages * kTgTok * kTgCols);
-    auto red = reinterpret_cast<float (*)[NJ][kTgCols + 4]>(tg_smem);
+    auto xs = reinterpret_cast<uint16_t (*)[kTgTok][kTgXPitch]>(tg_smem);
+    auto gs = reinterpret_cast<float (*)[kTgTok][GPITCH]>(tg_smem + L::X_BYTES);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t k0 = (int64_t)blockIdx.x * kTgCols;
-    const int split = blockIdx.y;
-    const int64_t tb = split * per_split;
+    const int64_t tb = (int64_t)blockIdx.y * per_split;
     const int64_t te = (tb + per_split < T) ? tb + per_split : T;
     const int64_t ntiles = te > tb ? (te - tb + kTgTok - 1) / kTgTok : 0;
 
     auto load = [&](int stage, int64_t tile) {
         const int64_t t0 = tb + tile * kTgTok;
-        // X: 32 rows x 256 bytes = 512 pieces, 4 per thread.
         #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 4; ++i) {                     // X: 32 rows x 16 pieces of 16 bytes
             const int p = tid + i * 128, row = p >> 4, piece = p & 15;
             const int64_t t = t0 + row, k = k0 + piece * 8;
             const bool ok = t < te && k < Kd;
-            const uint16_t* src = X + (ok ? t : 0) * Kd + (ok ? k : 0);
-            cp_async16(smem_u32(&xs[stage][row][piece * 8]), src, ok ? 16u : 0u);
+            cp_async16(smem_u32(&xs[stage][row][piece * 8]), X + (ok ? t : 0) * Kd + (ok ? k : 0), ok ? 16u : 0u);
         }
-        // G: 32 rows x NJ floats (NJ/4 pieces per row).
-        for (int p = tid; p < kTgTok * (NJ / 4); p += 128) {
-            const int row = p / (NJ / 4), piece = p % (NJ / 4);
+        for (int p = tid; p < kTgTok * (R / 4); p += 128) {   // G: 32 rows x R/4 pieces
+            const int row = p / (R / 4), piece = p % (R / 4);
             const int64_t t = t0 + row;
-            const bool ok = t < te && j0 + piece * 4 < r;
-            const float* src = G + (ok ? t : 0) * r + (ok ? j0 + piece * 4 : 0);
-            cp_async16(smem_u32(&gs[stage][row][piece * 4]), src, ok ? 16u : 0u);
+            const bool ok = t < te;
+            cp_async16(smem_u32(&gs[stage][row][piece * 4]), G + (ok ? t : 0) * R + piece * 4, ok ? 16u : 0u);
         }
     };
 
-    float acc[NJ][4];
+    float acc[2][NT][4];
     #pragma unroll
-    for (int j = 0; j < NJ; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
+    for (int m = 0; m < 2; ++m)
+        #pragma unroll
+        for (int n = 0; n < NT; ++n) acc[m][n][0] = acc[m][n][1] = acc[m][n][2] = acc[m][n][3] = 0.0f;
 
     #pragma unroll
     for (int s = 0; s < kTgStages - 1; ++s) {
         if (s < ntiles) load(s, s);
         cp_async_commit();
     }
+    // A = X^T read transposed: matrix i = lanes 8i..8i+7 covers tokens
+    // {0-7, 0-7, 8-15, 8-15} and columns {0, 8, 0, 8} of a 16 x 16 block.
+    const int a_t = (lane & 7) + 8 * (lane >> 4);
+    const int a_k = 8 * ((lane >> 3) & 1);
+    const int g = lane >> 2, q = lane & 3;
     for (int64_t i = 0; i < ntiles; ++i) {
         cp_async_wait<kTgStages - 2>();
         __syncthreads();
         const int st = (int)(i % kTgStages);
-        #pragma unroll 2
-        for (int tt = warp; tt < kTgTok; tt += kTgWarps) {
-            const uint2 xp = *reinterpret_cast<const uint2*>(&xs[st][tt][4 * lane]);
-            const float x0 = __uint_as_float(xp.x << 16), x1 = __uint_as_float(xp.x & 0xffff0000u);
-            const float x2 = __uint_as_float(xp.y << 16), x3 = __uint_as_float(xp.y & 0xffff0000u);
+        #pragma unroll
+        for (int kk = 0; kk < kTgTok / 16; ++kk) {
+            uint32_t bh[NT][2], bl[NT][2];
             #pragma unroll
-            for (int j4 = 0; j4 < NJ; j4 += 4) {
-                const float4 gv = *reinterpret_cast<const float4*>(&gs[st][tt][j4]);
-                const float gg[4] = {gv.x, gv.y, gv.z, gv.w};
+            for (int n = 0; n < NT; ++n) {
                 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    acc[j4 + u][0] = fmaf(gg[u], x0, acc[j4 + u][0]);
-                    acc[j4 + u][1] = fmaf(gg[u], x1, acc[j4 + u][1]);
-                    acc[j4 + u][2] = fmaf(gg[u], x2, acc[j4 + u][2]);
-                    acc[j4 + u][3] = fmaf(gg[u], x3, acc[j4 + u][3]);
+                for (int h = 0; h < 2; ++h) {
+                    const float v0 = gs[st][kk * 16 + 8 * h + 2 * q][8 * n + g];
+                    const float v1 = gs[st][kk * 16 + 8 * h + 2 * q + 1][8 * n + g];
+                    const float h0 = __bfloat162float(__float2bfloat16_rn(v0));
+                    const float h1 = __bfloat162float(__float2bfloat16_rn(v1));
+                    bh[n][h] = pack2(h0, h1);
+                    bl[n][h] = pack2(__fsub_rn(v0, h0), __fsub_rn(v1, h1));
+                }
+            }
+            #pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4_t(smem_u32(&xs[st][kk * 16 + a_t][warp * 32 + m * 16 + a_k]), a0, a1, a2, a3);
+                #pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                    mma_bf16_16816(acc[m][n], a0, a1, a2, a3, bh[n][0], bh[n][1]);
+                    mma_bf16_16816(acc[m][n], a0, a1, a2, a3, bl[n][0], bl[n][1]);
                 }
             }
         }
@@ -268,78 +317,106 @@ __global__ void __launch_bounds__(128) lora_tgrad_kernel(const float* __restrict
         cp_async_commit();
     }
     cp_async_wait<0>();
-    __syncthreads();                          // staging ring is dead from here on
+
+    // acc[m][n] = { (k = base+g, j = 8n+2q), (k, j+1), (k+8, j), (k+8, j+1) }, base = k0 + 32 warp + 16 m
+    auto out_index = [&](int64_t k, int j) -> int64_t { return OUT_RK ? (int64_t)j * Kd + k : k * R + j; };
+    auto finish = [&](int64_t k, int j, float v) {
+        const int64_t o = out_index(k, j);
+        const float w = __fmul_rn(scale, v);
+        out[o] = accumulate ? __fadd_rn(out[o], w) : w;
+    };
+    if (nsplit == 1) {
+        #pragma unroll
+        for (int m = 0; m < 2; ++m)
+            #pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                const int64_t k = k0 + warp * 32 + m * 16 + g;
+                const int j = 8 * n + 2 * q;
+                if (k < Kd) { finish(k, j, acc[m][n][0]); finish(k, j + 1, acc[m][n][1]); }
+                if (k + 8 < Kd) { finish(k + 8, j, acc[m][n][2]); finish(k + 8, j + 1, acc[m][n][3]); }
+            }
+        return;
+    }
+    float* pp = partial + (int64_t)blockIdx.y * R * Kd;      // partial [split][j][k]
     #pragma unroll
-    for (int j = 0; j < NJ; ++j)
+    for (int m = 0; m < 2; ++m)
         #pragma unroll
-        for (int c = 0; c < 4; ++c) red[warp][j][4 * lane + c] = acc[j][c];
-    __syncthreads();
-    const int nj = (r - j0 < NJ) ? (r - j0) : NJ;
-    for (int idx = tid; idx < nj * kTgCols; idx += blockDim.x) {
-        const int j = idx / kTgCols, c = idx % kTgCols;
-        const int64_t k = k0 + c;
-        if (k >= Kd) continue;
-        float s = 0.0f;
-        #pragma unroll
-        for (int w = 0; w < kTgWarps; ++w) s += red[w][j][c];
-        if (nsplit == 1) {
-            const int64_t o = OUT_RK ? (int64_t)(j0 + j) * Kd + k : k * r + (j0 + j);
-            const float v = __fmul_rn(scale, s);
-            out[o] = accumulate ? __fadd_rn(out[o], v) : v;
-        } else {
-            partial[((int64_t)split * r + (j0 + j)) * Kd + k] = s;
+        for (int n = 0; n < NT; ++n) {
+            const int64_t k = k0 + warp * 32 + m * 16 + g;
+            const int j = 8 * n + 2 * q;
+            if (k < Kd) { pp[(int64_t)j * Kd + k] = acc[m][n][0]; pp[(int64_t)(j + 1) * Kd + k] = acc[m][n][1]; }
+            if (k + 8 < Kd) { pp[(int64_t)j * Kd + k + 8] = acc[m][n][2]; pp[(int64_t)(j + 1) * Kd + k + 8] = acc[m][n][3]; }
         }
+    if (!last_in_group(counters + blockIdx.x, nsplit)) return;
+    for (int idx = tid; idx < R * kTgCols; idx += 128) {
+        const int j = idx / kTgCols;
+        const int64_t k = k0 + idx % kTgCols;
+        if (k >= Kd) continue;
+        float sum = 0.0f;
+        for (int sp = 0; sp < nsplit; ++sp) sum += __ldcg(partial + ((int64_t)sp * R + j) * Kd + k);
+        finish(k, j, sum);
     }
 }
 
-template <bool OUT_RK>
-__global__ void lora_tgrad_finish(const float* __restrict__ partial, int64_t Kd, int r, int nsplit, float scale,
-                                  int accumulate, float* __restrict__ out) {
-    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (idx >= (int64_t)r * Kd) return;
-    const int64_t j = idx / Kd, k = idx % Kd;
-    float s = 0.0f;
-    for (int sp = 0; sp < nsplit; ++sp) s += partial[(int64_t)sp * r * Kd + idx];
-    const int64_t o = OUT_RK ? idx : k * r + j;
-    const float v = __fmul_rn(scale, s);
-    out[o] = accumulate ? __fadd_rn(out[o], v) : v;
-}
-
-template <int NT>
-constexpr size_t down_smem_bytes() {
-    return sizeof(uint16_t) * kDnStages * (kDnRows + 16 * ((NT + 1) / 2)) * kDnPitch;
-}
-
-template <int NJ>
-constexpr size_t tgrad_smem_bytes() {
-    const size_t ring = sizeof(uint16_t) * kTgStages * kTgTok * kTgCols + sizeof(float) * kTgStages * kTgTok * NJ;
-    const size_t red = sizeof(float) * kTgWarps * NJ * (kTgCols + 4);
-    return ring > red ? ring : red;
-}
-
-// Opt a kernel into its dynamic shared-memory size once.
 template <typename K>
 cudaError_t allow_smem(K kernel, size_t bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-template <int NT>
+template <int NT, bool B_KR>
 lsn_status launch_down_nt(dim3 grid, cudaStream_t st, const uint16_t* X, const uint16_t* W, int64_t T, int64_t Kd,
-                          int cps, float scale, float* u32, uint16_t* u16, float* part) {
-    static const cudaError_t attr = allow_smem(lora_down_kernel<NT>, down_smem_bytes<NT>());
+                          int cps, int ns, float scale, float* u32, uint16_t* u16, float* part, int* counters) {
+    constexpr size_t bytes = DownSmem<NT, B_KR>::BYTES;
+    static const cudaError_t attr = allow_smem(lora_down_kernel<NT, B_KR>, bytes);
     if (attr != cudaSuccess) return fail_cuda(attr, "cudaFuncSetAttribute(lora_down smem)");
-    lora_down_kernel<NT><<<grid, 128, down_smem_bytes<NT>(), st>>>(X, W, T, Kd, cps, scale, u32, u16, part);
+    lora_down_kernel<NT, B_KR><<<grid, 128, bytes, st>>>(X, W, T, Kd, cps, ns, scale, u32, u16, part, counters);
     return LSN_OK;
 }
 
-template <int NJ, bool OUT_RK>
-lsn_status launch_tgrad_nj(dim3 grid, cudaStream_t st, const float* G, const uint16_t* X, int64_t T, int64_t Kd, int r,
-                           int j0, int64_t per, int ns, float scale, int accumulate, float* out, float* partial) {
-    static const cudaError_t attr = allow_smem(lora_tgrad_kernel<NJ, OUT_RK>, tgrad_smem_bytes<NJ>());
+template <int NT, bool OUT_RK>
+lsn_status launch_tgrad_nt(dim3 grid, cudaStream_t st, const float* G, const uint16_t* X, int64_t T, int64_t Kd,
+                           int64_t per, int ns, float scale, int accumulate, float* out, float* partial,
+                           int* counters) {
+    constexpr size_t bytes = TgSmem<NT>::BYTES;
+    static const cudaError_t attr = allow_smem(lora_tgrad_kernel<NT, OUT_RK>, bytes);
     if (attr != cudaSuccess) return fail_cuda(attr, "cudaFuncSetAttribute(lora_tgrad smem)");
-    lora_tgrad_kernel<NJ, OUT_RK><<<grid, 128, tgrad_smem_bytes<NJ>(), st>>>(G, X, T, Kd, r, j0, per, ns, scale,
-                                                                             accumulate, out, partial);
+    lora_tgrad_kernel<NT, OUT_RK><<<grid, 128, bytes, st>>>(G, X, T, Kd, per, ns, scale, accumulate, out, partial,
+                                                            counters);
     return LSN_OK;
+}
+
+template <bool B_KR>
+lsn_status dispatch_down(int r, dim3 grid, cudaStream_t st, const uint16_t* X, const uint16_t* W, int64_t T,
+                         int64_t Kd, int cps, int ns, float scale, float* u32, uint16_t* u16, float* part,
+                         int* counters) {
+    switch (r / 8) {
+        case 1: return launch_down_nt<1, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16, part, counters);
+        case 2: return launch_down_nt<2, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16, part, counters);
+        case 3: return launch_down_nt<3, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16, part, counters);
+        case 4: return launch_down_nt<4, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16, part, counters);
+        case 5: return launch_down_nt<5, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16, part, counters);
+        case 6: return launch_down_nt<6, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16, part, counters);
+        case 7: return launch_down_nt<7, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16, part, counters);
+        case 8: return launch_down_nt<8, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16, part, counters);
+        default: return fail(LSN_ERR_INVALID_ARG, "rank must be a multiple of 8 in [8, 64]");
+    }
+}
+
+template <bool OUT_RK>
+lsn_status dispatch_tgrad(int r, dim3 grid, cudaStream_t st, const float* G, const uint16_t* X, int64_t T, int64_t Kd,
+                          int64_t per, int ns, float scale, int accumulate, float* out, float* partial,
+                          int* counters) {
+    switch (r / 8) {
+        case 1: return launch_tgrad_nt<1, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out, partial, counters);
+        case 2: return launch_tgrad_nt<2, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out, partial, counters);
+        case 3: return launch_tgrad_nt<3, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out, partial, counters);
+        case 4: return launch_tgrad_nt<4, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out, partial, counters);
+        case 5: return launch_tgrad_nt<5, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out, partial, counters);
+        case 6: return launch_tgrad_nt<6, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out, partial, counters);
+        case 7: return launch_tgrad_nt<7, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out, partial, counters);
+        case 8: return launch_tgrad_nt<8, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out, partial, counters);
+        default: return fail(LSN_ERR_INVALID_ARG, "rank must be a multiple of 8 in [8, 64]");
+    }
 }
 
 }  // namespace
@@ -366,12 +443,12 @@ size_t down_ws_bytes(int64_t T, int64_t Kd, int r) {
     return s > 1 ? (size_t)s * T * r * sizeof(float) : 0;
 }
 
-// Token splits of a reduction: about two 128-thread CTAs per SM of a 148-SM
+// Token splits of a reduction: about four 128-thread CTAs per SM of a 148-SM
 // part, at least 128 tokens per split.
 int tgrad_splits(int64_t T, int64_t Kd) {
     const int64_t tiles = (Kd + kTgCols - 1) / kTgCols;
     if (tiles <= 0 || T <= 0) return 1;
-    int64_t s = (296 + tiles - 1) / tiles;
+    int64_t s = (592 + tiles - 1) / tiles;
     const int64_t by_t = (T + 127) / 128;
     if (s > by_t) s = by_t;
     if (s > 64) s = 64;
@@ -384,65 +461,36 @@ size_t tgrad_ws_bytes(int64_t T, int64_t Kd, int r) {
     return s > 1 ? (size_t)s * r * Kd * sizeof(float) : 0;
 }
 
-// X [T, Kd] times W: w_rk ? W is A [r, Kd] : W is B [Kd, r] (transposed into
-// `wt` [r, Kd] first).  `partial` must hold down_ws_bytes(T, Kd, r).
+// Integer tickets of the split reductions (one per row block or column tile).
+size_t split_counter_count(int64_t T, int64_t K, int64_t N) {
+    const int64_t a = (T + kDnRows - 1) / kDnRows;
+    const int64_t b = ((K > N ? K : N) + kTgCols - 1) / kTgCols;
+    return (size_t)(a > b ? a : b);
+}
+
+// X [T, Kd] times W: w_rk ? W is A [r, Kd] : W is B [Kd, r].
 lsn_status launch_lora_down(const uint16_t* X, const uint16_t* W, bool w_rk, int64_t T, int64_t Kd, int r,
-                            float scale, float* u32, uint16_t* u16, uint16_t* wt, float* partial, cudaStream_t st) {
+                            float scale, float* u32, uint16_t* u16, float* partial, int* counters, cudaStream_t st) {
     if (T == 0) return LSN_OK;
-    if (!w_rk) {
-        const int64_t n = Kd * r;
-        transpose_nr_kernel<<<(int)ceil_div(n, 256), 256, 0, st>>>(W, Kd, r, wt);
-        W = wt;
-    }
     const int ns = down_splits(T, Kd);
     const int64_t chunks = Kd / 64;
     const int cps = (int)((chunks + ns - 1) / ns);
     dim3 grid((unsigned)((T + kDnRows - 1) / kDnRows), (unsigned)ns);
-    float* part = ns > 1 ? partial : nullptr;
-    lsn_status ls;
-    switch (r / 8) {
-        case 1: ls = launch_down_nt<1>(grid, st, X, W, T, Kd, cps, scale, u32, u16, part); break;
-        case 2: ls = launch_down_nt<2>(grid, st, X, W, T, Kd, cps, scale, u32, u16, part); break;
-        case 3: ls = launch_down_nt<3>(grid, st, X, W, T, Kd, cps, scale, u32, u16, part); break;
-        case 4: ls = launch_down_nt<4>(grid, st, X, W, T, Kd, cps, scale, u32, u16, part); break;
-        case 5: ls = launch_down_nt<5>(grid, st, X, W, T, Kd, cps, scale, u32, u16, part); break;
-        case 6: ls = launch_down_nt<6>(grid, st, X, W, T, Kd, cps, scale, u32, u16, part); break;
-        case 7: ls = launch_down_nt<7>(grid, st, X, W, T, Kd, cps, scale, u32, u16, part); break;
-        case 8: ls = launch_down_nt<8>(grid, st, X, W, T, Kd, cps, scale, u32, u16, part); break;
-        default: return fail(LSN_ERR_INVALID_ARG, "rank must be a multiple of 8 in [8, 64]");
-    }
+    lsn_status ls = w_rk ? dispatch_down<false>(r, grid, st, X, W, T, Kd, cps, ns, scale, u32, u16, partial, counters)
+                         : dispatch_down<true>(r, grid, st, X, W, T, Kd, cps, ns, scale, u32, u16, partial, counters);
     if (ls != LSN_OK) return ls;
-    if (ns > 1) {
-        const int64_t n = T * r;
-        lora_down_finish<<<(int)ceil_div(n, 256), 256, 0, st>>>(partial, n, ns, scale, u32, u16);
-    }
     LSN_CUDA_TRY(cudaGetLastError());
     return LSN_OK;
 }
 
 lsn_status launch_lora_tgrad(const float* G, const uint16_t* X, bool out_rk, int64_t T, int64_t Kd, int r,
-                             float scale, int accumulate, float* out, float* partial, cudaStream_t st) {
+                             float scale, int accumulate, float* out, float* partial, int* counters, cudaStream_t st) {
     const int ns = tgrad_splits(T, Kd);
-    const int64_t per = ((T + ns - 1) / ns + 15) / 16 * 16;
+    const int64_t per = ((T + ns - 1) / ns + kTgTok - 1) / kTgTok * kTgTok;
     dim3 grid((unsigned)((Kd + kTgCols - 1) / kTgCols), (unsigned)ns);
-    for (int j0 = 0; j0 < r; j0 += 16) {
-        const bool wide = r - j0 > 8;
-        lsn_status ls;
-        if (out_rk)
-            ls = wide ? launch_tgrad_nj<16, true>(grid, st, G, X, T, Kd, r, j0, per, ns, scale, accumulate, out, partial)
-                      : launch_tgrad_nj<8, true>(grid, st, G, X, T, Kd, r, j0, per, ns, scale, accumulate, out, partial);
-        else
-            ls = wide ? launch_tgrad_nj<16, false>(grid, st, G, X, T, Kd, r, j0, per, ns, scale, accumulate, out, partial)
-                      : launch_tgrad_nj<8, false>(grid, st, G, X, T, Kd, r, j0, per, ns, scale, accumulate, out, partial);
-        if (ls != LSN_OK) return ls;
-    }
-    if (ns > 1) {
-        const int64_t n = (int64_t)r * Kd;
-        if (out_rk)
-            lora_tgrad_finish<true><<<(int)ceil_div(n, 256), 256, 0, st>>>(partial, Kd, r, ns, scale, accumulate, out);
-        else
-            lora_tgrad_finish<false><<<(int)ceil_div(n, 256), 256, 0, st>>>(partial, Kd, r, ns, scale, accumulate, out);
-    }
+    lsn_status ls = out_rk ? dispatch_tgrad<true>(r, grid, st, G, X, T, Kd, per, ns, scale, accumulate, out, partial, counters)
+                           : dispatch_tgrad<false>(r, grid, st, G, X, T, Kd, per, ns, scale, accumulate, out, partial, counters);
+    if (ls != LSN_OK) return ls;
     LSN_CUDA_TRY(cudaGetLastError());
     return LSN_OK;
 }

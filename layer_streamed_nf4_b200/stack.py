@@ -19,6 +19,7 @@ the same numerics):
 """
 from __future__ import annotations
 
+import ctypes
 from dataclasses import dataclass
 
 import torch
@@ -63,6 +64,7 @@ class Stack:
         self.pool = None
         self.host = None
         self.resident = None
+        self._calls = {}
         self._build_weights()
         self._build_tensors(distinct_activations)
         self._setup_mode(n_slots)
@@ -134,7 +136,7 @@ class Stack:
         import copy
         assert mode in ("resident", "streamed", "no_h2d")
         other = copy.copy(self)
-        other.mode, other.pool, other.resident = mode, None, None
+        other.mode, other.pool, other.resident, other._calls = mode, None, None, {}
         other._setup_mode(n_slots)
         return other
 
@@ -172,26 +174,54 @@ class Stack:
     def _out(self, d, l, pi):
         return d[(l if self.keep_outputs else 0), pi]
 
+    # The per-call arguments depend only on (slot address, layer, projection),
+    # so they are marshalled once and the C entry points are called directly.
+
+    def _fwd_args(self, addr: int, l: int, pi: int):
+        key = ("f", addr, l, pi)
+        a = self._calls.get(key)
+        if a is None:
+            p = self.proj[pi]
+            base = self._base(addr, p)
+            a = (ctypes.byref(base), self.x[l, pi].data_ptr(), self.T, self.A[l, pi].data_ptr(),
+                 self.B[l, pi].data_ptr(), self.r, self.scale, self._out(self.y, l, pi).data_ptr(),
+                 self.ws.data_ptr(), self.ws_bytes, self.stream.cuda_stream, base)
+            self._calls[key] = a
+        return a
+
+    def _bwd_args(self, addr: int, l: int, pi: int, accumulate: bool):
+        key = ("b", addr, l, pi, accumulate)
+        a = self._calls.get(key)
+        if a is None:
+            p = self.proj[pi]
+            base = self._base(addr, p)
+            a = (ctypes.byref(base), self.x[l, pi].data_ptr(), self.dY[l, pi].data_ptr(), self.T,
+                 self.A[l, pi].data_ptr(), self.B[l, pi].data_ptr(), self.r, self.scale,
+                 self._out(self.dX, l, pi).data_ptr(), self.dA[l, pi].data_ptr(), self.dB[l, pi].data_ptr(),
+                 int(accumulate), self.ws.data_ptr(), self.ws_bytes, self.stream.cuda_stream, base)
+            self._calls[key] = a
+        return a
+
     def forward(self):
-        s = self.stream
+        fwd = lsnf4._lib.lora_linear_fwd
         for l in range(self.L):
             addr = self._acquire(l)
             self._prefetch(l + 1)
-            for pi, p in enumerate(self.proj):
-                lsnf4.lora_linear_fwd(self._base(addr, p), self.x[l, pi], self.T, self.A[l, pi], self.B[l, pi],
-                                      self.r, self.scale, self._out(self.y, l, pi), self.ws, self.ws_bytes, s)
+            for pi in range(len(self.proj)):
+                st = fwd(*self._fwd_args(addr, l, pi)[:-1])
+                if st:
+                    lsnf4._check(st, "lora_linear_fwd")
             self._release(l)
 
     def backward(self, accumulate: bool = False):
-        s = self.stream
+        bwd = lsnf4._lib.lora_linear_bwd
         for l in reversed(range(self.L)):
             addr = self._acquire(l)
             self._prefetch(l - 1)
             for pi in reversed(range(len(self.proj))):
-                p = self.proj[pi]
-                lsnf4.lora_linear_bwd(self._base(addr, p), self.x[l, pi], self.dY[l, pi], self.T, self.A[l, pi],
-                                      self.B[l, pi], self.r, self.scale, self._out(self.dX, l, pi), self.dA[l, pi],
-                                      self.dB[l, pi], accumulate, self.ws, self.ws_bytes, s)
+                st = bwd(*self._bwd_args(addr, l, pi, accumulate)[:-1])
+                if st:
+                    lsnf4._check(st, "lora_linear_bwd")
             self._release(l)
 
     def step(self, accumulate: bool = False):
