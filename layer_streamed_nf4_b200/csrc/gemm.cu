@@ -40,17 +40,34 @@ struct GemmArgs {
 
 namespace {
 
-constexpr int BM = 128, BK = 64, STAGES = 4;
+// Tile geometry.  A stage holds a 128-wide slice of the contraction as two
+// 64-wide sub-tiles per operand (each one 128-byte-swizzle atom wide), so one
+// full/empty barrier round trip feeds eight K=16 MMAs: with four, the
+// handshake between producer and MMA issuer kept the tensor pipe measurably
+// idle.
+constexpr int BM = 128;          // rows of A per CTA
+constexpr int BK = 128;          // contraction per stage
+constexpr int SUB = 64;          // contraction per sub-tile (one swizzle atom)
+constexpr int STAGES = 3;
 
-template <int BN, bool B_MN>
+// PAIR = false: one CTA per SM, tile 128 x BN.
+// PAIR = true : a CTA pair (cluster of 2) issues the 2-SM MMA, tile 256 x BN,
+//               each CTA staging its 128 rows of A and BN/2 rows of B.
+template <bool PAIR, int BN, bool B_MN>
 struct Cfg {
-    static constexpr int A_BYTES = BM * BK * 2;
-    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int B_ROWS = PAIR ? BN / 2 : BN;     // B rows (N extent) staged per CTA
+    static constexpr int A_SUB = BM * SUB * 2;             // bytes of one A sub-tile
+    static constexpr int A_BYTES = 2 * A_SUB;
+    static constexpr int B_SUB = B_ROWS * SUB * 2;         // K-major: bytes of one B sub-tile
+    static constexpr int B_BYTES = 2 * B_SUB;              // MN-major: B_ROWS/64 atom columns of 128 x 64
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int BAR_BYTES = 256;
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
-    static constexpr uint32_t IDESC = idesc_bf16(BM, BN, 0, B_MN ? 1 : 0);
+    static constexpr uint32_t IDESC = idesc_bf16(PAIR ? 2 * BM : BM, BN, 0, B_MN ? 1 : 0);
     static constexpr uint32_t TMEM_COLS = 2 * BN;
+    static constexpr int TILE_M = PAIR ? 2 * BM : BM;
+    static constexpr uint32_t TX_BYTES = (PAIR ? 2 : 1) * STAGE_BYTES;
+    static constexpr uint32_t ACC_EMPTY_ARRIVALS = (PAIR ? 2 : 1) * 4;
 };
 
 __device__ __forceinline__ void raise_error(volatile int* abort_flag, int* err, int code) {
@@ -58,12 +75,12 @@ __device__ __forceinline__ void raise_error(volatile int* abort_flag, int* err, 
     if (err) atomicExch(err, code);
 }
 
-template <int BN, bool B_MN>
+template <bool PAIR, int BN, bool B_MN>
 __global__ void __launch_bounds__(192, 1)
     lsn_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmLA, const __grid_constant__ CUtensorMap tmLB,
                     const GemmArgs p) {
-    using C = Cfg<BN, B_MN>;
+    using C = Cfg<PAIR, BN, B_MN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
@@ -76,14 +93,19 @@ __global__ void __launch_bounds__(192, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int num_m = (p.M + BM - 1) / BM;
+    uint32_t rank = 0;
+    if constexpr (PAIR) rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+    const int nunits = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+    const int num_m = (p.M + C::TILE_M - 1) / C::TILE_M;
     const int num_n = (p.N + BN - 1) / BN;
     const int num_tiles = num_m * num_n;
     const int nkb = p.num_kb + (p.lora_k16 > 0 ? 1 : 0);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-        for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 128); }
+        for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], C::ACC_EMPTY_ARRIVALS); }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -92,9 +114,13 @@ __global__ void __launch_bounds__(192, 1)
         tma_prefetch_desc(&tmA); tma_prefetch_desc(&tmB);
         if (p.lora_k16 > 0) { tma_prefetch_desc(&tmLA); tma_prefetch_desc(&tmLB); }
     }
-    if (warp == 1) { tmem_alloc(tmem_holder, C::TMEM_COLS); tmem_relinquish(); }
+    if (warp == 1) {
+        if constexpr (PAIR) { tmem_alloc_pair(tmem_holder, C::TMEM_COLS); tmem_relinquish_pair(); }
+        else                { tmem_alloc(tmem_holder, C::TMEM_COLS); tmem_relinquish(); }
+    }
     tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) cluster_sync_all();   // both CTAs' barriers initialised before any remote use
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
@@ -103,44 +129,47 @@ __global__ void __launch_bounds__(192, 1)
             // ---------------------------------------------------- producer --
             int stage = 0;
             uint32_t phase = 0;
-            int issued_parity[STAGES];
-            for (int s = 0; s < STAGES; ++s) issued_parity[s] = -1;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            for (int tile = unit; tile < num_tiles && ok; tile += nunits) {
                 const int mb = tile % num_m, nb = tile / num_m;
+                const int m_row = mb * C::TILE_M + (int)rank * BM;
+                const int n_off = nb * BN + (int)rank * C::B_ROWS;
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
                     uint8_t* sA = smem + stage * C::STAGE_BYTES;
                     uint8_t* sB = sA + C::A_BYTES;
-                    mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-                    issued_parity[stage] = (int)phase;
+                    uint32_t fbar = smem_u32(&full[stage]);
+                    if constexpr (PAIR) fbar = mapa_shared(fbar, 0);
+                    if (leader) mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
+                    auto load = [&](void* dst, const CUtensorMap* m, int x, int y) {
+                        if constexpr (PAIR) tma_load_2d_pair(dst, m, x, y, fbar);
+                        else                tma_load_2d(dst, m, x, y, &full[stage]);
+                    };
                     const bool lora = kb >= p.num_kb;
                     const CUtensorMap* ma = lora ? &tmLA : &tmA;
                     const CUtensorMap* mbp = lora ? &tmLB : &tmB;
                     const int kc = lora ? 0 : kb * BK;
-                    tma_load_2d(sA, ma, kc, mb * BM, &full[stage]);
+                    load(sA, ma, kc, m_row);
+                    load(sA + C::A_SUB, ma, kc + SUB, m_row);
                     if (!B_MN) {
-                        tma_load_2d(sB, mbp, kc, nb * BN, &full[stage]);
+                        load(sB, mbp, kc, n_off);
+                        load(sB + C::B_SUB, mbp, kc + SUB, n_off);
                     } else {
                         #pragma unroll
-                        for (int a = 0; a < BN / 64; ++a)
-                            tma_load_2d(sB + a * (64 * 128), mbp, nb * BN + a * 64, kc, &full[stage]);
+                        for (int a = 0; a < C::B_ROWS / 64; ++a) load(sB + a * (BK * 128), mbp, n_off + a * 64, kc);
                     }
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
             }
             if (!ok) raise_error(abort_flag, p.err, 1);
-            // Let every copy this CTA issued land before the CTA can exit.
-            for (int s = 0; s < STAGES; ++s)
-                if (issued_parity[s] >= 0) mbar_wait(&full[s], (uint32_t)issued_parity[s], nullptr);
         }
     } else if (warp == 1) {
-        if (lane == 0) {
+        if (lane == 0 && leader) {
             // -------------------------------------------------- MMA issuer --
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+            for (int tile = unit; tile < num_tiles && ok; tile += nunits) {
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
@@ -151,22 +180,27 @@ __global__ void __launch_bounds__(192, 1)
                     const uint32_t b0 = a0 + C::A_BYTES;
                     const int nk = (kb < p.num_kb) ? BK / 16 : p.lora_k16;
                     for (int k = 0; k < nk; ++k) {
-                        const uint64_t ad = smem_desc_sw128(a0 + k * 32, 16, 1024);
-                        const uint64_t bd = B_MN ? smem_desc_sw128(b0 + k * 2048, 64 * 128, 1024)
-                                                 : smem_desc_sw128(b0 + k * 32, 16, 1024);
-                        umma_bf16(d_tmem, ad, bd, C::IDESC, (kb | k) ? 1u : 0u);
+                        const int j = k >> 2, kk = k & 3;       // sub-tile, step inside it
+                        const uint64_t ad = smem_desc_sw128(a0 + j * C::A_SUB + kk * 32, 16, 1024);
+                        const uint64_t bd = B_MN ? smem_desc_sw128(b0 + k * 2048, BK * 128, 1024)
+                                                 : smem_desc_sw128(b0 + j * C::B_SUB + kk * 32, 16, 1024);
+                        if constexpr (PAIR) umma_bf16_pair(d_tmem, ad, bd, C::IDESC, (kb | k) ? 1u : 0u);
+                        else                umma_bf16(d_tmem, ad, bd, C::IDESC, (kb | k) ? 1u : 0u);
                     }
-                    umma_commit(&empty[stage]);
+                    if constexpr (PAIR) umma_commit_pair(&empty[stage]);
+                    else                umma_commit(&empty[stage]);
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
                 if (!ok) break;
-                umma_commit(&acc_full[acc]);
+                if constexpr (PAIR) umma_commit_pair(&acc_full[acc]);
+                else                umma_commit(&acc_full[acc]);
                 acc ^= 1;
                 if (acc == 0) acc_phase ^= 1;
             }
             if (!ok) raise_error(abort_flag, p.err, 2);
-            // Every MMA issued by this thread completes before TMEM is freed.
-            umma_commit(drain);
+            // Every MMA issued here completes before TMEM is freed.
+            if constexpr (PAIR) umma_commit_pair(drain);
+            else                umma_commit(drain);
             mbar_wait(drain, 0, nullptr);
         }
     } else {
@@ -174,12 +208,12 @@ __global__ void __launch_bounds__(192, 1)
         const int q = warp & 3;                    // TMEM lanes 32q .. 32q+31
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+        for (int tile = unit; tile < num_tiles; tile += nunits) {
             const int mb = tile % num_m, nb = tile / num_m;
             const bool got = mbar_wait(&acc_full[acc], acc_phase, abort_flag);
             if (!__all_sync(0xffffffffu, got)) { if (lane == 0) raise_error(abort_flag, p.err, 3); break; }
             tc_fence_after();
-            const int row = mb * BM + q * 32 + lane;
+            const int row = mb * C::TILE_M + (int)rank * BM + q * 32 + lane;
             #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 const int col = nb * BN + c * 32;
@@ -201,7 +235,11 @@ __global__ void __launch_bounds__(192, 1)
                 }
             }
             tc_fence_before();
-            mbar_arrive(&acc_empty[acc]);
+            __syncwarp();
+            if (lane == 0) {
+                if constexpr (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[acc]), 0));
+                else                mbar_arrive(&acc_empty[acc]);
+            }
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1;
         }
@@ -209,9 +247,11 @@ __global__ void __launch_bounds__(192, 1)
     __syncwarp();
     tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) cluster_sync_all();   // no CTA leaves while its peer may still touch its memory
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, C::TMEM_COLS);
+        if constexpr (PAIR) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+        else                tmem_dealloc(tmem_base, C::TMEM_COLS);
     }
 }
 
@@ -251,30 +291,46 @@ lsn_status make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t out
     return LSN_OK;
 }
 
-template <int BN, bool B_MN>
+template <bool PAIR, int BN, bool B_MN>
 lsn_status launch_cfg(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& la, const CUtensorMap& lb,
                       const GemmArgs& args, cudaStream_t st) {
-    using C = Cfg<BN, B_MN>;
+    using C = Cfg<PAIR, BN, B_MN>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(lsn_gemm_kernel<BN, B_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        attr_err = cudaFuncSetAttribute(lsn_gemm_kernel<PAIR, BN, B_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         C::SMEM_BYTES);
     });
     if (attr_err != cudaSuccess) return fail_cuda(attr_err, "cudaFuncSetAttribute(gemm smem)");
-    const int tiles = ((args.M + BM - 1) / BM) * ((args.N + BN - 1) / BN);
-    const int grid = tiles < sm_count() ? tiles : sm_count();
-    lsn_gemm_kernel<BN, B_MN><<<grid, 192, C::SMEM_BYTES, st>>>(a, b, la, lb, args);
-    LSN_CUDA_TRY(cudaGetLastError());
+    const int tiles = ((args.M + C::TILE_M - 1) / C::TILE_M) * ((args.N + BN - 1) / BN);
+    const int units = PAIR ? sm_count() / 2 : sm_count();
+    const int grid = (PAIR ? 2 : 1) * (tiles < units ? tiles : units);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(192);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    if (PAIR) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    LSN_CUDA_TRY(cudaLaunchKernelEx(&cfg, lsn_gemm_kernel<PAIR, BN, B_MN>, a, b, la, lb, args));
     return LSN_OK;
 }
 
 }  // namespace
 
-// N-tile width from the shape alone: 256 unless that leaves SMs idle.
-int gemm_bn(int64_t M, int64_t N) {
-    const int64_t tiles256 = ((M + BM - 1) / BM) * ((N + 255) / 256);
-    return (tiles256 >= 148) ? 256 : 128;
+// Kernel choice from the shape alone: the 2-SM kernel (256 x 256 tiles on
+// CTA pairs) when it has at least one full wave of pairs on a 148-SM part,
+// else the 1-SM kernel with 128 x 128 tiles.
+bool gemm_use_pairs(int64_t M, int64_t N) {
+    const int64_t pair_tiles = ((M + 255) / 256) * ((N + 255) / 256);
+    return pair_tiles >= 74;
 }
 
 // D = A . op(B) + LA . op(LB).
@@ -285,38 +341,34 @@ int gemm_bn(int64_t M, int64_t N) {
 lsn_status launch_gemm(const uint16_t* A, int64_t lda, const uint16_t* B, int64_t ldb, bool b_mn, const uint16_t* LA,
                        const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D, int64_t ldd,
                        int* err, cudaStream_t st) {
-    const int bn = gemm_bn(M, N);
+    const bool pair = gemm_use_pairs(M, N);
+    const int b_rows = pair ? 128 : 128;           // B rows staged per CTA: BN/2 = 128 (pair) or BN = 128
     CUtensorMap ma, mb, mla, mlb;
     lsn_status s;
-    if ((s = make_map(&ma, A, Kc, M, lda, 64, BM)) != LSN_OK) return s;
+    if ((s = make_map(&ma, A, Kc, M, lda, SUB, BM)) != LSN_OK) return s;
     if (!b_mn) {
-        if ((s = make_map(&mb, B, Kc, N, ldb, 64, bn)) != LSN_OK) return s;
+        if ((s = make_map(&mb, B, Kc, N, ldb, SUB, b_rows)) != LSN_OK) return s;
     } else {
-        if ((s = make_map(&mb, B, N, Kc, ldb, 64, 64)) != LSN_OK) return s;
+        if ((s = make_map(&mb, B, N, Kc, ldb, 64, BK)) != LSN_OK) return s;
     }
-    if (r > 0) {
-        if ((s = make_map(&mla, LA, r, M, r, 64, BM)) != LSN_OK) return s;
-        if (!b_mn) {
-            if ((s = make_map(&mlb, LB, r, N, r, 64, bn)) != LSN_OK) return s;
-        } else {
-            if ((s = make_map(&mlb, LB, N, r, N, 64, 64)) != LSN_OK) return s;
-        }
+    if ((s = make_map(&mla, LA, r, M, r, SUB, BM)) != LSN_OK) return s;
+    if (!b_mn) {
+        if ((s = make_map(&mlb, LB, r, N, r, SUB, b_rows)) != LSN_OK) return s;
     } else {
-        mla = ma;
-        mlb = mb;
+        if ((s = make_map(&mlb, LB, N, r, N, 64, BK)) != LSN_OK) return s;
     }
     GemmArgs args;
     args.M = (int)M;
     args.N = (int)N;
-    args.num_kb = (int)(Kc / BK);
+    args.num_kb = (int)((Kc + BK - 1) / BK);
     args.lora_k16 = (r + 15) / 16;
     args.D = D;
     args.ldd = ldd;
     args.err = err;
-    if (bn == 256) return b_mn ? launch_cfg<256, true>(ma, mb, mla, mlb, args, st)
-                               : launch_cfg<256, false>(ma, mb, mla, mlb, args, st);
-    return b_mn ? launch_cfg<128, true>(ma, mb, mla, mlb, args, st)
-                : launch_cfg<128, false>(ma, mb, mla, mlb, args, st);
+    if (pair) return b_mn ? launch_cfg<true, 256, true>(ma, mb, mla, mlb, args, st)
+                          : launch_cfg<true, 256, false>(ma, mb, mla, mlb, args, st);
+    return b_mn ? launch_cfg<false, 128, true>(ma, mb, mla, mlb, args, st)
+                : launch_cfg<false, 128, false>(ma, mb, mla, mlb, args, st);
 }
 
 }  // namespace lsn

@@ -101,6 +101,14 @@ def test_ragged_and_small_shapes(lib, orc, T, K, N, r):
     _full_parity(lib, orc, c, "nf4")
 
 
+@pytest.mark.parametrize("T,K,N", [(300, 256, 9472), (300, 9472, 256)])
+def test_pair_kernel_with_ragged_rows(lib, orc, T, K, N):
+    """Shapes with >= 74 pair tiles run the 2-SM kernel (forward for the first,
+    input gradient for the second), here with a ragged last 256-row tile."""
+    c = synth.linear_case(T, K, N, 16, 32.0, seed=T + K)
+    _full_parity(lib, orc, c, "nf4")
+
+
 def test_b_zero_gives_the_base_product(lib, orc):
     c = synth.linear_case(160, 256, 320, 16, 32.0, seed=3)
     c.B[:] = 0
