@@ -234,6 +234,19 @@ lsn_status lsn_timing_enable(int on);
 /* Wait for the recorded events, return the sums and clear the records. */
 lsn_status lsn_timing_read(lsn_kernel_timing* out);
 
+/* ------------------------------------------------------------- options --
+ *
+ * Process-wide switches between equivalent implementations (same results bit
+ * for bit; only speed differs).
+ *   LSN_OPT_FUSED_NF4  1: NF4 weights on the 2-SM GEMM are converted to bf16
+ *                      inside the GEMM by converter warps (no bf16 copy of W);
+ *                      0 (default): nf4_dequant into the workspace, then the
+ *                      bf16 GEMM.  Narrow shapes always use the latter.
+ */
+typedef enum { LSN_OPT_FUSED_NF4 = 1 } lsn_option;
+lsn_status lsn_set_option(int option, int value);
+int lsn_get_option(int option);
+
 /* ------------------------------------------------------------ layer pool --
  *
  * n_slots VRAM buffers of slot_bytes each, allocated once at creation; the

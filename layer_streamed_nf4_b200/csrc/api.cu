@@ -1,6 +1,7 @@
 // The C entry points of liblsnf4.so (declared in include/lsnf4.h): argument
 // checks, workspace carving and the launch sequence of each call.
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <string>
 
@@ -23,10 +24,15 @@ lsn_status launch_lora_tgrad(const float* G, const uint16_t* X, bool out_rk, int
                              float scale, int accumulate, float* out, float* partial, int* counters, cudaStream_t st);
 size_t split_counter_count(int64_t T, int64_t K, int64_t N);
 size_t tgrad_ws_bytes(int64_t T, int64_t Kd, int r);
+lsn_status launch_gemm_nf4(const uint16_t* A, int64_t lda, const lsn_nf4_weight* w, bool b_mn, const uint16_t* LA,
+                           const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D, int64_t ldd,
+                           int* err, cudaStream_t st);
+bool gemm_use_pairs(int64_t M, int64_t N);
 int tgrad_splits(int64_t T, int64_t Kd);
 
 namespace {
 thread_local std::string g_last_error = "no error";
+std::atomic<int> g_fused_nf4{0};
 }
 
 lsn_status fail(lsn_status st, const std::string& msg) {
@@ -258,6 +264,11 @@ lsn_status lora_linear_fwd(const lsn_base* W, const uint16_t* x, int64_t T, cons
     const int64_t N = W->rows, K = W->cols;
     LoraWs w = carve(ws, T, K, N, r, W->kind);
     if ((s = timed_down(x, A, true, T, K, r, scale, nullptr, w.s16, w, st)) != LSN_OK) return s;
+    if (W->kind == LSN_BASE_NF4 && g_fused_nf4.load() && gemm_use_pairs(T, N)) {
+        // NF4 converted inside the GEMM (no bf16 copy of W).
+        TimingScope ts(LSN_K_GEMM_FWD, 2.0 * T * N * (double)(K + r), st);
+        return launch_gemm_nf4(x, K, &W->nf4, false, w.s16, B, r, T, N, K, y, N, w.err, st);
+    }
     const uint16_t* Wb = W->bf16;
     if (W->kind == LSN_BASE_NF4) {
         if ((s = timed_dequant(&W->nf4, w.w16, st)) != LSN_OK) return s;
@@ -281,7 +292,10 @@ lsn_status lora_linear_bwd(const lsn_base* W, const uint16_t* x, const uint16_t*
     if (T > 0) {
         if ((s = timed_down(dY, B, false, T, N, r, scale, w.g32, w.s16, w, st)) != LSN_OK) return s;
         if ((s = timed_down(x, A, true, T, K, r, scale, w.u32, nullptr, w, st)) != LSN_OK) return s;
-        if (dX) {
+        if (dX && W->kind == LSN_BASE_NF4 && g_fused_nf4.load() && gemm_use_pairs(T, K)) {
+            TimingScope ts(LSN_K_GEMM_BWD, 2.0 * T * K * (double)(N + r), st);
+            if ((s = launch_gemm_nf4(dY, N, &W->nf4, true, w.s16, A, r, T, K, N, dX, K, w.err, st)) != LSN_OK) return s;
+        } else if (dX) {
             const uint16_t* Wb = W->bf16;
             if (W->kind == LSN_BASE_NF4) {
                 if ((s = timed_dequant(&W->nf4, w.w16, st)) != LSN_OK) return s;
@@ -295,6 +309,16 @@ lsn_status lora_linear_bwd(const lsn_base* W, const uint16_t* x, const uint16_t*
     if ((s = timed_tgrad(w.g32, x, true, T, K, r, scale, accumulate, dA, w, st)) != LSN_OK) return s;
     return timed_tgrad(w.u32, dY, false, T, N, r, scale, accumulate, dB, w, st);
 }
+
+lsn_status lsn_set_option(int option, int value) {
+    if (option == LSN_OPT_FUSED_NF4) {
+        g_fused_nf4.store(value != 0 ? 1 : 0);
+        return LSN_OK;
+    }
+    return fail(LSN_ERR_INVALID_ARG, "lsn_set_option: unknown option");
+}
+
+int lsn_get_option(int option) { return option == LSN_OPT_FUSED_NF4 ? g_fused_nf4.load() : -1; }
 
 lsn_status lsn_ws_status(void* ws, lsn_stream_t stream) {
     LSN_CHECK_ARG(ws != nullptr, "lsn_ws_status: workspace is NULL");

@@ -31,11 +31,18 @@ namespace lsn {
 
 struct GemmArgs {
     int M, N;            // output rows (tokens) and columns
-    int num_kb;          // 64-wide contraction blocks of the base term
+    int num_kb;          // 128-wide contraction blocks of the base term
     int lora_k16;        // K=16 MMAs of the LoRA term (0: none)
     uint16_t* D;         // bf16 output, row-major
     int64_t ldd;         // elements
     int* err;            // device error flag (set on a timed-out wait)
+    // NF4 base converted in the kernel (fused variant only):
+    const uint8_t* absmax_q;   // [wrows * wcols / 64] second-level codes
+    const float* absmax_s2;    // [ceil(nblk / 256)]
+    const float* absmax_off;   // [1]
+    int wrows, wcols;          // W is [wrows, wcols] row-major (N_out x K_in)
+    float level[16];           // NF4 levels
+    float dq[256];             // second-level table
 };
 
 namespace {
@@ -49,25 +56,32 @@ constexpr int BM = 128;          // rows of A per CTA
 constexpr int BK = 128;          // contraction per stage
 constexpr int SUB = 64;          // contraction per sub-tile (one swizzle atom)
 constexpr int STAGES = 3;
+constexpr int CONV_WARPS = 8;    // NF4 converter warps (fused variant)
 
 // PAIR = false: one CTA per SM, tile 128 x BN.
 // PAIR = true : a CTA pair (cluster of 2) issues the 2-SM MMA, tile 256 x BN,
 //               each CTA staging its 128 rows of A and BN/2 rows of B.
-template <bool PAIR, int BN, bool B_MN>
+// NF4  = true : B is the NF4 weight, converted to bf16 in shared memory by
+//               converter warps from a TMA-staged packed tile (PAIR only).
+template <bool PAIR, int BN, bool B_MN, bool NF4 = false>
 struct Cfg {
     static constexpr int B_ROWS = PAIR ? BN / 2 : BN;     // B rows (N extent) staged per CTA
     static constexpr int A_SUB = BM * SUB * 2;             // bytes of one A sub-tile
     static constexpr int A_BYTES = 2 * A_SUB;
     static constexpr int B_SUB = B_ROWS * SUB * 2;         // K-major: bytes of one B sub-tile
     static constexpr int B_BYTES = 2 * B_SUB;              // MN-major: B_ROWS/64 atom columns of 128 x 64
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int P_BYTES = NF4 ? 128 * 64 : 0;     // packed NF4 tile: 128 rows x 64 bytes
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + P_BYTES;
     static constexpr int BAR_BYTES = 256;
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+    static constexpr int DQ_BYTES = NF4 ? 1024 : 0;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + DQ_BYTES + 1024;
     static constexpr uint32_t IDESC = idesc_bf16(PAIR ? 2 * BM : BM, BN, 0, B_MN ? 1 : 0);
     static constexpr uint32_t TMEM_COLS = 2 * BN;
     static constexpr int TILE_M = PAIR ? 2 * BM : BM;
-    static constexpr uint32_t TX_BYTES = (PAIR ? 2 : 1) * STAGE_BYTES;
     static constexpr uint32_t ACC_EMPTY_ARRIVALS = (PAIR ? 2 : 1) * 4;
+    static constexpr uint32_t READY_ARRIVALS = (PAIR ? 2 : 1) * CONV_WARPS;
+    static constexpr int THREADS = 192 + (NF4 ? 32 * CONV_WARPS : 0);
+    static_assert(!NF4 || (PAIR && B_ROWS == 128), "the fused NF4 path runs on the pair kernel");
 };
 
 __device__ __forceinline__ void raise_error(volatile int* abort_flag, int* err, int code) {
@@ -75,22 +89,48 @@ __device__ __forceinline__ void raise_error(volatile int* abort_flag, int* err, 
     if (err) atomicExch(err, code);
 }
 
-template <bool PAIR, int BN, bool B_MN>
-__global__ void __launch_bounds__(192, 1)
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// Eight NF4 codes (one 32-bit word of the packed layout: byte j holds element
+// 2j in its high nibble and 2j+1 in its low nibble) to eight bf16 values, by
+// byte permutes on the block's 16-entry table of scaled values: lo[t]/hi[t]
+// hold the low/high bytes of table entries 4t..4t+3.  A selector nibble below
+// 8 picks a byte; the top bit of each code chooses between the tables of
+// entries 0-7 and 8-15 (a byte mask built with prmt's sign-replicate mode).
+__device__ __forceinline__ uint4 nf4x8_to_bf16(uint32_t p, const uint32_t (&lo)[4], const uint32_t (&hi)[4]) {
+    const uint32_t a = p << 4;
+    const uint32_t s0 = p & 0x7777u, s1 = (p >> 16) & 0x7777u;
+    const uint32_t m0 = prmt(a, p, 0xD9C8u), m1 = prmt(a, p, 0xFBEAu);
+    const uint32_t l0 = (prmt(lo[0], lo[1], s0) & ~m0) | (prmt(lo[2], lo[3], s0) & m0);
+    const uint32_t h0 = (prmt(hi[0], hi[1], s0) & ~m0) | (prmt(hi[2], hi[3], s0) & m0);
+    const uint32_t l1 = (prmt(lo[0], lo[1], s1) & ~m1) | (prmt(lo[2], lo[3], s1) & m1);
+    const uint32_t h1 = (prmt(hi[0], hi[1], s1) & ~m1) | (prmt(hi[2], hi[3], s1) & m1);
+    // l0/h0 bytes are elements (1, 0, 3, 2); interleave into bf16 pairs in element order.
+    return make_uint4(prmt(l0, h0, 0x4051u), prmt(l0, h0, 0x6273u), prmt(l1, h1, 0x4051u), prmt(l1, h1, 0x6273u));
+}
+
+template <bool PAIR, int BN, bool B_MN, bool NF4>
+__global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN, NF4>::THREADS, 1)
     lsn_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmLA, const __grid_constant__ CUtensorMap tmLB,
-                    const GemmArgs p) {
-    using C = Cfg<PAIR, BN, B_MN>;
+                    const __grid_constant__ GemmArgs p) {
+    using C = Cfg<PAIR, BN, B_MN, NF4>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
-    uint64_t* full = bars;
-    uint64_t* empty = bars + STAGES;
-    uint64_t* acc_full = bars + 2 * STAGES;
+    uint64_t* full = bars;                    // TMA landed (bf16 path: A and B; NF4: this CTA's A + packed)
+    uint64_t* empty = bars + STAGES;          // MMAs done reading the stage
+    uint64_t* ready = bars + 2 * STAGES;      // NF4: converted B written (counted on the leader)
+    uint64_t* acc_full = bars + 3 * STAGES;
     uint64_t* acc_empty = acc_full + 2;
     uint64_t* drain = acc_empty + 2;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    float* dq_s = reinterpret_cast<float*>(smem + STAGES * C::STAGE_BYTES + C::BAR_BYTES);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint32_t rank = 0;
@@ -104,11 +144,18 @@ __global__ void __launch_bounds__(192, 1)
     const int nkb = p.num_kb + (p.lora_k16 > 0 ? 1 : 0);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+            mbar_init(&ready[s], C::READY_ARRIVALS);
+        }
         for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], C::ACC_EMPTY_ARRIVALS); }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
+    }
+    if constexpr (NF4) {
+        for (int i = threadIdx.x; i < 256; i += blockDim.x) dq_s[i] = p.dq[i];
     }
     if (warp == 0 && lane == 0) {
         tma_prefetch_desc(&tmA); tma_prefetch_desc(&tmB);
@@ -138,25 +185,48 @@ __global__ void __launch_bounds__(192, 1)
                     if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
                     uint8_t* sA = smem + stage * C::STAGE_BYTES;
                     uint8_t* sB = sA + C::A_BYTES;
-                    uint32_t fbar = smem_u32(&full[stage]);
-                    if constexpr (PAIR) fbar = mapa_shared(fbar, 0);
-                    if (leader) mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
-                    auto load = [&](void* dst, const CUtensorMap* m, int x, int y) {
-                        if constexpr (PAIR) tma_load_2d_pair(dst, m, x, y, fbar);
-                        else                tma_load_2d(dst, m, x, y, &full[stage]);
-                    };
+                    uint8_t* sP = sB + C::B_BYTES;
                     const bool lora = kb >= p.num_kb;
                     const CUtensorMap* ma = lora ? &tmLA : &tmA;
                     const CUtensorMap* mbp = lora ? &tmLB : &tmB;
                     const int kc = lora ? 0 : kb * BK;
-                    load(sA, ma, kc, m_row);
-                    load(sA + C::A_SUB, ma, kc + SUB, m_row);
-                    if (!B_MN) {
-                        load(sB, mbp, kc, n_off);
-                        load(sB + C::B_SUB, mbp, kc + SUB, n_off);
+                    if constexpr (NF4) {
+                        // Each CTA counts its own bytes on its own barrier; the
+                        // converters release the stage to the MMA.
+                        mbar_arrive_expect_tx(&full[stage], C::A_BYTES + (lora ? C::B_BYTES : C::P_BYTES));
+                        tma_load_2d(sA, ma, kc, m_row, &full[stage]);
+                        tma_load_2d(sA + C::A_SUB, ma, kc + SUB, m_row, &full[stage]);
+                        if (lora) {
+                            if (!B_MN) {
+                                tma_load_2d(sB, mbp, 0, n_off, &full[stage]);
+                                tma_load_2d(sB + C::B_SUB, mbp, SUB, n_off, &full[stage]);
+                            } else {
+                                #pragma unroll
+                                for (int a = 0; a < C::B_ROWS / 64; ++a)
+                                    tma_load_2d(sB + a * (BK * 128), mbp, n_off + a * 64, 0, &full[stage]);
+                            }
+                        } else {
+                            // packed bytes: fwd rows n_off.., bytes kb*64..; bwd rows kb*128.., bytes n_off/2..
+                            if (!B_MN) tma_load_2d(sP, &tmB, kb * 64, n_off, &full[stage]);
+                            else       tma_load_2d(sP, &tmB, n_off / 2, kb * BK, &full[stage]);
+                        }
                     } else {
-                        #pragma unroll
-                        for (int a = 0; a < C::B_ROWS / 64; ++a) load(sB + a * (BK * 128), mbp, n_off + a * 64, kc);
+                        uint32_t fbar = smem_u32(&full[stage]);
+                        if constexpr (PAIR) fbar = mapa_shared(fbar, 0);
+                        if (leader) mbar_arrive_expect_tx(&full[stage], (PAIR ? 2 : 1) * (C::A_BYTES + C::B_BYTES));
+                        auto load = [&](void* dst, const CUtensorMap* m, int x, int y) {
+                            if constexpr (PAIR) tma_load_2d_pair(dst, m, x, y, fbar);
+                            else                tma_load_2d(dst, m, x, y, &full[stage]);
+                        };
+                        load(sA, ma, kc, m_row);
+                        load(sA + C::A_SUB, ma, kc + SUB, m_row);
+                        if (!B_MN) {
+                            load(sB, mbp, kc, n_off);
+                            load(sB + C::B_SUB, mbp, kc + SUB, n_off);
+                        } else {
+                            #pragma unroll
+                            for (int a = 0; a < C::B_ROWS / 64; ++a) load(sB + a * (BK * 128), mbp, n_off + a * 64, kc);
+                        }
                     }
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
@@ -174,7 +244,9 @@ __global__ void __launch_bounds__(192, 1)
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
                 for (int kb = 0; kb < nkb; ++kb) {
-                    if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+                    const bool got = NF4 ? mbar_wait_cluster(&ready[stage], phase, abort_flag)
+                                         : mbar_wait(&full[stage], phase, abort_flag);
+                    if (!got) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(smem + stage * C::STAGE_BYTES);
                     const uint32_t b0 = a0 + C::A_BYTES;
@@ -203,7 +275,7 @@ __global__ void __launch_bounds__(192, 1)
             else                umma_commit(drain);
             mbar_wait(drain, 0, nullptr);
         }
-    } else {
+    } else if (warp < 6) {
         // -------------------------------------------------------- epilogue --
         const int q = warp & 3;                    // TMEM lanes 32q .. 32q+31
         int acc = 0;
@@ -243,6 +315,92 @@ __global__ void __launch_bounds__(192, 1)
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1;
         }
+    } else if constexpr (NF4) {
+        // ------------------------------------------------------- converters --
+        // Thread t of the 256 converters owns one (row, 64-block) of the
+        // CTA's 128 x 128 B tile per stage: row = t % 128, block = t / 128.
+        // Rows are B rows (forward: W rows n; backward: the contraction rows n
+        // of W read MN-major); the block is 64 consecutive W columns.  In both
+        // majors the 64 bf16 go to one 128-byte row of a 128-byte-swizzled
+        // atom: block b's atom at b * 16 KB, row at (row/8)*1024 + (row%8)*128.
+        const int t = threadIdx.x - 192;
+        const int row = t & 127, blk = t >> 7;
+        const int64_t nblk_row = p.wcols / 64;          // 64-blocks per W row
+        const float off = *p.absmax_off;
+        // The unit's second-level code and s2 are fetched two k-blocks ahead,
+        // so their global-load latency overlaps earlier conversions.
+        struct Meta { uint32_t code; float s2; bool ok; };
+        auto fetch = [&](int tl, int k) -> Meta {
+            Meta m{0u, 0.0f, false};
+            if (tl >= num_tiles || k >= p.num_kb) return m;
+            const int n_off = (tl / num_m) * BN + (int)rank * C::B_ROWS;
+            const int64_t wr = B_MN ? (int64_t)k * BK + row : (int64_t)n_off + row;
+            const int64_t wb = B_MN ? (int64_t)(n_off / 64) + blk : (int64_t)k * 2 + blk;
+            if (wr < p.wrows && wb < nblk_row) {
+                const int64_t bi = wr * nblk_row + wb;
+                m.code = __ldg(p.absmax_q + bi);
+                m.s2 = __ldg(p.absmax_s2 + (bi >> 8));
+                m.ok = true;
+            }
+            return m;
+        };
+        int ft = unit, fk = 0;
+        auto step = [&]() { if (++fk == nkb) { fk = 0; ft += nunits; } };
+        Meta m0 = fetch(ft, fk);
+        step();
+        Meta m1 = fetch(ft, fk);
+        step();
+        int stage = 0;
+        uint32_t phase = 0;
+        bool bad = false;
+        for (int tile = unit; tile < num_tiles && !bad; tile += nunits) {
+            for (int kb = 0; kb < nkb; ++kb) {
+                const Meta cur = m0;
+                m0 = m1;
+                m1 = fetch(ft, fk);
+                step();
+                const bool got = mbar_wait(&full[stage], phase, abort_flag);
+                if (!__all_sync(0xffffffffu, got)) { if (lane == 0) raise_error(abort_flag, p.err, 4); bad = true; break; }
+                if (kb < p.num_kb) {
+                    uint8_t* sB = smem + stage * C::STAGE_BYTES + C::A_BYTES;
+                    const uint8_t* sP = sB + C::B_BYTES;
+                    uint8_t* dst = sB + blk * (BK * 128) + (row >> 3) * 1024 + (row & 7) * 128;
+                    if (cur.ok) {
+                        const float ah = __fadd_rn(__fmul_rn(dq_s[cur.code], cur.s2), off);
+                        // Scaled table: entry q = bf16(level[q] * absmax_hat), packed in pairs.
+                        uint32_t e[8];
+                        #pragma unroll
+                        for (int i = 0; i < 8; ++i) e[i] = pack_bf16x2(__fmul_rn(p.level[2 * i], ah), __fmul_rn(p.level[2 * i + 1], ah));
+                        uint32_t lo[4], hi[4];
+                        #pragma unroll
+                        for (int i = 0; i < 4; ++i) { lo[i] = prmt(e[2 * i], e[2 * i + 1], 0x6420u); hi[i] = prmt(e[2 * i], e[2 * i + 1], 0x7531u); }
+                        // Packed tile row: 64 bytes, 64-byte swizzle (16-byte chunk c stored at c ^ ((row >> 1) & 3)).
+                        const uint8_t* prow = sP + row * 64;
+                        #pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int ch = (2 * blk + h) ^ ((row >> 1) & 3);
+                            const uint4 pk = *reinterpret_cast<const uint4*>(prow + ch * 16);
+                            const uint32_t w[4] = {pk.x, pk.y, pk.z, pk.w};
+                            #pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const int c = h * 4 + i;                 // 8-element chunk of the 64
+                                *reinterpret_cast<uint4*>(dst + ((c ^ (row & 7)) << 4)) = nf4x8_to_bf16(w[i], lo, hi);
+                            }
+                        }
+                    } else {
+                        #pragma unroll
+                        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(dst + (c << 4)) = make_uint4(0, 0, 0, 0);
+                    }
+                    fence_proxy_async_smem();
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    if constexpr (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&ready[stage]), 0));
+                    else                mbar_arrive(&ready[stage]);
+                }
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            }
+        }
     }
     __syncwarp();
     tc_fence_before();
@@ -277,29 +435,34 @@ EncodeTiledFn encode_fn() {
 // A 2-D bf16 tensor [outer, inner] with row stride `stride_elems`, read in
 // boxes of box_inner (64 = 128 bytes, the swizzle span) x box_outer rows.
 lsn_status make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, int64_t stride_elems,
-                    int box_inner, int box_outer) {
+                    int box_inner, int box_outer, bool bytes = false) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return fail(LSN_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    const int esize = bytes ? 1 : 2;
     cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
-    cuuint64_t strides[1] = {(cuuint64_t)stride_elems * 2};
+    cuuint64_t strides[1] = {(cuuint64_t)stride_elems * esize};
     cuuint32_t box[2] = {(cuuint32_t)box_inner, (cuuint32_t)box_outer};
     cuuint32_t es[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    // bf16 operand tiles use the 128-byte swizzle the MMA descriptors expect;
+    // packed NF4 tiles (64-byte rows) use the 64-byte swizzle, which keeps the
+    // converters' 16-byte reads free of bank conflicts.
+    CUresult r = fn(m, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+                    dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    bytes ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(LSN_ERR_CUDA, "cuTensorMapEncodeTiled failed (code " + std::to_string((int)r) + ")");
     return LSN_OK;
 }
 
-template <bool PAIR, int BN, bool B_MN>
+template <bool PAIR, int BN, bool B_MN, bool NF4 = false>
 lsn_status launch_cfg(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& la, const CUtensorMap& lb,
                       const GemmArgs& args, cudaStream_t st) {
-    using C = Cfg<PAIR, BN, B_MN>;
+    using C = Cfg<PAIR, BN, B_MN, NF4>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(lsn_gemm_kernel<PAIR, BN, B_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        C::SMEM_BYTES);
+        attr_err = cudaFuncSetAttribute(lsn_gemm_kernel<PAIR, BN, B_MN, NF4>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     });
     if (attr_err != cudaSuccess) return fail_cuda(attr_err, "cudaFuncSetAttribute(gemm smem)");
     const int tiles = ((args.M + C::TILE_M - 1) / C::TILE_M) * ((args.N + BN - 1) / BN);
@@ -307,7 +470,7 @@ lsn_status launch_cfg(const CUtensorMap& a, const CUtensorMap& b, const CUtensor
     const int grid = (PAIR ? 2 : 1) * (tiles < units ? tiles : units);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(192);
+    cfg.blockDim = dim3(C::THREADS);
     cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -319,7 +482,7 @@ lsn_status launch_cfg(const CUtensorMap& a, const CUtensorMap& b, const CUtensor
         cfg.attrs = attr;
         cfg.numAttrs = 1;
     }
-    LSN_CUDA_TRY(cudaLaunchKernelEx(&cfg, lsn_gemm_kernel<PAIR, BN, B_MN>, a, b, la, lb, args));
+    LSN_CUDA_TRY(cudaLaunchKernelEx(&cfg, lsn_gemm_kernel<PAIR, BN, B_MN, NF4>, a, b, la, lb, args));
     return LSN_OK;
 }
 
@@ -331,6 +494,45 @@ lsn_status launch_cfg(const CUtensorMap& a, const CUtensorMap& b, const CUtensor
 bool gemm_use_pairs(int64_t M, int64_t N) {
     const int64_t pair_tiles = ((M + 255) / 256) * ((N + 255) / 256);
     return pair_tiles >= 74;
+}
+
+// The fused NF4 variant: B is the NF4 weight w (W [wrows, wcols] row-major;
+// forward: N = wrows, Kc = wcols; backward: N = wcols, Kc = wrows).  Runs on
+// the pair kernel only; returns LSN_ERR_UNSUPPORTED for shapes that do not use
+// it so the caller can fall back to dequantise + bf16 GEMM.
+lsn_status launch_gemm_nf4(const uint16_t* A, int64_t lda, const lsn_nf4_weight* w, bool b_mn, const uint16_t* LA,
+                           const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D, int64_t ldd,
+                           int* err, cudaStream_t st) {
+    if (!gemm_use_pairs(M, N)) return LSN_ERR_UNSUPPORTED;
+    const Nf4Tables& T = nf4_tables();
+    CUtensorMap ma, mp, mla, mlb;
+    lsn_status s;
+    if ((s = make_map(&ma, A, Kc, M, lda, SUB, BM)) != LSN_OK) return s;
+    // packed [wrows, wcols/2] bytes, boxes of 64 bytes x 128 rows
+    if ((s = make_map(&mp, w->packed, w->cols / 2, w->rows, w->cols / 2, 64, 128, true)) != LSN_OK) return s;
+    if ((s = make_map(&mla, LA, r, M, r, SUB, BM)) != LSN_OK) return s;
+    if (!b_mn) {
+        if ((s = make_map(&mlb, LB, r, N, r, SUB, 128)) != LSN_OK) return s;
+    } else {
+        if ((s = make_map(&mlb, LB, N, r, N, 64, BK)) != LSN_OK) return s;
+    }
+    GemmArgs args{};
+    args.M = (int)M;
+    args.N = (int)N;
+    args.num_kb = (int)((Kc + BK - 1) / BK);
+    args.lora_k16 = (r + 15) / 16;
+    args.D = D;
+    args.ldd = ldd;
+    args.err = err;
+    args.absmax_q = w->absmax_q;
+    args.absmax_s2 = w->absmax_s2;
+    args.absmax_off = w->offset;
+    args.wrows = (int)w->rows;
+    args.wcols = (int)w->cols;
+    std::memcpy(args.level, T.level, sizeof(args.level));
+    std::memcpy(args.dq, T.dq, sizeof(args.dq));
+    return b_mn ? launch_cfg<true, 256, true, true>(ma, mp, mla, mlb, args, st)
+                : launch_cfg<true, 256, false, true>(ma, mp, mla, mlb, args, st);
 }
 
 // D = A . op(B) + LA . op(LB).
@@ -357,7 +559,7 @@ lsn_status launch_gemm(const uint16_t* A, int64_t lda, const uint16_t* B, int64_
     } else {
         if ((s = make_map(&mlb, LB, N, r, N, 64, BK)) != LSN_OK) return s;
     }
-    GemmArgs args;
+    GemmArgs args{};
     args.M = (int)M;
     args.N = (int)N;
     args.num_kb = (int)((Kc + BK - 1) / BK);

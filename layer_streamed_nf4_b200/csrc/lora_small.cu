@@ -47,23 +47,16 @@ __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_gr
 // Two bf16 values packed low/high into one register.
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) { return pack_bf16x2(lo, hi); }
 
-// Deterministic split reduction: every CTA of a group writes its partial, then
-// the CTA that finishes last (a ticket from an integer counter) adds the
-// partials in split order.  The counter is reset for the next launch.  Returns
-// true (in every thread) in the last CTA, after a fence that makes the other
-// CTAs' partials visible.
-__device__ __forceinline__ bool last_in_group(int* counter, int nsplit) {
-    __shared__ int ticket;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        ticket = atomicAdd(counter, 1);
-        if (ticket == nsplit - 1) atomicExch(counter, 0);
-    }
-    __syncthreads();
-    const bool last = ticket == nsplit - 1;
-    if (last) __threadfence();
-    return last;
+// Split reductions inside a thread-block cluster: the CTAs of one output tile
+// (one per K- or token-split, cluster rank = split index) each leave their
+// partial tile in shared memory; after a cluster barrier, CTA y adds slice y
+// of the tile over ranks 0, 1, ..., S-1 in that order, reading the other
+// CTAs' shared memory directly (DSMEM).  The order depends on the shape only.
+__device__ __forceinline__ float ld_dsmem_f32(const float* local_ptr, uint32_t rank) {
+    float v;
+    const uint32_t a = mapa_shared(smem_u32(local_ptr), rank);
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+    return v;
 }
 
 // ----------------------------------------------------------- down proj ---
@@ -90,15 +83,16 @@ struct DownSmem {
     static constexpr int WPITCH = B_KR ? 16 * NP + 8 : kDnPitch;  // bf16 per staged W row
     static constexpr size_t X_BYTES = sizeof(uint16_t) * kDnStages * kDnRows * kDnPitch;
     static constexpr size_t W_BYTES = sizeof(uint16_t) * kDnStages * WROWS * WPITCH;
-    static constexpr size_t BYTES = X_BYTES + W_BYTES;
+    static constexpr size_t RING = X_BYTES + W_BYTES;
+    static constexpr size_t RED = sizeof(float) * kDnRows * R;
+    static constexpr size_t BYTES = RING > RED ? RING : RED;
 };
 
 template <int NT, bool B_KR>
 __global__ void __launch_bounds__(128) lora_down_kernel(const uint16_t* __restrict__ X, const uint16_t* __restrict__ W,
                                                         int64_t T, int64_t Kd, int chunks_per_split, int nsplit,
                                                         float scale, float* __restrict__ u32,
-                                                        uint16_t* __restrict__ u16, float* __restrict__ partial,
-                                                        int* __restrict__ counters) {
+                                                        uint16_t* __restrict__ u16) {
     using L = DownSmem<NT, B_KR>;
     constexpr int R = L::R, NP = L::NP, WROWS = L::WROWS, WPITCH = L::WPITCH;
     extern __shared__ __align__(16) uint8_t dn_smem[];
@@ -191,22 +185,28 @@ __global__ void __launch_bounds__(128) lora_down_kernel(const uint16_t* __restri
         }
         return;
     }
-    float* pp = partial + (int64_t)blockIdx.y * T * R;
+    // Partial tile [64 rows][R] in shared memory (the staging ring is dead).
+    __syncthreads();
+    float* red = reinterpret_cast<float*>(dn_smem);
     #pragma unroll
     for (int n = 0; n < NT; ++n) {
-        const int j = n * 8 + 2 * q;
-        if (ok0) { pp[row0 * R + j] = acc[n][0]; pp[row0 * R + j + 1] = acc[n][1]; }
-        if (ok1) { pp[row1 * R + j] = acc[n][2]; pp[row1 * R + j + 1] = acc[n][3]; }
+        const int j = n * 8 + 2 * q, rl = warp * 16 + g;
+        red[rl * R + j] = acc[n][0];
+        red[rl * R + j + 1] = acc[n][1];
+        red[(rl + 8) * R + j] = acc[n][2];
+        red[(rl + 8) * R + j + 1] = acc[n][3];
     }
-    if (!last_in_group(counters + blockIdx.x, nsplit)) return;
-    for (int idx = tid; idx < kDnRows * R; idx += 128) {
-        const int64_t row = row_base + idx / R;
-        const int j = idx % R;
-        if (row >= T) continue;
+    cluster_sync_all();
+    const int rank = (int)cluster_ctarank();
+    constexpr int V = kDnRows * R;
+    const int per = (V + nsplit - 1) / nsplit;
+    for (int v = rank * per + tid; v < (rank + 1) * per && v < V; v += 128) {
+        const int64_t row = row_base + v / R;
         float sum = 0.0f;
-        for (int sp = 0; sp < nsplit; ++sp) sum += __ldcg(partial + ((int64_t)sp * T + row) * R + j);
-        emit(row, j, sum);
+        for (int sp = 0; sp < nsplit; ++sp) sum += ld_dsmem_f32(red + v, (uint32_t)sp);
+        if (row < T) emit(row, v % R, sum);
     }
+    cluster_sync_all();                 // partials stay readable until every CTA is done
 }
 
 // -------------------------------------------------------- token reduce ---
@@ -230,14 +230,15 @@ struct TgSmem {
     static constexpr int GPITCH = 8 * NT + 4;
     static constexpr size_t X_BYTES = sizeof(uint16_t) * kTgStages * kTgTok * kTgXPitch;
     static constexpr size_t G_BYTES = sizeof(float) * kTgStages * kTgTok * GPITCH;
-    static constexpr size_t BYTES = X_BYTES + G_BYTES;
+    static constexpr size_t RING = X_BYTES + G_BYTES;
+    static constexpr size_t RED = sizeof(float) * 8 * NT * kTgCols;
+    static constexpr size_t BYTES = RING > RED ? RING : RED;
 };
 
 template <int NT, bool OUT_RK>
 __global__ void __launch_bounds__(128) lora_tgrad_kernel(const float* __restrict__ G, const uint16_t* __restrict__ X,
                                                          int64_t T, int64_t Kd, int64_t per_split, int nsplit,
-                                                         float scale, int accumulate, float* __restrict__ out,
-                                                         float* __restrict__ partial, int* __restrict__ counters) {
+                                                         float scale, int accumulate, float* __restrict__ out) {
     using L = TgSmem<NT>;
     constexpr int R = 8 * NT, GPITCH = L::GPITCH;
     extern __shared__ __align__(16) uint8_t tg_smem[];
@@ -337,25 +338,31 @@ __global__ void __launch_bounds__(128) lora_tgrad_kernel(const float* __restrict
             }
         return;
     }
-    float* pp = partial + (int64_t)blockIdx.y * R * Kd;      // partial [split][j][k]
+    // Partial tile [R][128 columns] in shared memory (the staging ring is dead).
+    __syncthreads();
+    float* red = reinterpret_cast<float*>(tg_smem);
     #pragma unroll
     for (int m = 0; m < 2; ++m)
         #pragma unroll
         for (int n = 0; n < NT; ++n) {
-            const int64_t k = k0 + warp * 32 + m * 16 + g;
+            const int c = warp * 32 + m * 16 + g;
             const int j = 8 * n + 2 * q;
-            if (k < Kd) { pp[(int64_t)j * Kd + k] = acc[m][n][0]; pp[(int64_t)(j + 1) * Kd + k] = acc[m][n][1]; }
-            if (k + 8 < Kd) { pp[(int64_t)j * Kd + k + 8] = acc[m][n][2]; pp[(int64_t)(j + 1) * Kd + k + 8] = acc[m][n][3]; }
+            red[j * kTgCols + c] = acc[m][n][0];
+            red[(j + 1) * kTgCols + c] = acc[m][n][1];
+            red[j * kTgCols + c + 8] = acc[m][n][2];
+            red[(j + 1) * kTgCols + c + 8] = acc[m][n][3];
         }
-    if (!last_in_group(counters + blockIdx.x, nsplit)) return;
-    for (int idx = tid; idx < R * kTgCols; idx += 128) {
-        const int j = idx / kTgCols;
-        const int64_t k = k0 + idx % kTgCols;
-        if (k >= Kd) continue;
+    cluster_sync_all();
+    const int rank = (int)cluster_ctarank();
+    constexpr int V = R * kTgCols;
+    const int per = (V + nsplit - 1) / nsplit;
+    for (int v = rank * per + tid; v < (rank + 1) * per && v < V; v += 128) {
+        const int64_t k = k0 + v % kTgCols;
         float sum = 0.0f;
-        for (int sp = 0; sp < nsplit; ++sp) sum += __ldcg(partial + ((int64_t)sp * R + j) * Kd + k);
-        finish(k, j, sum);
+        for (int sp = 0; sp < nsplit; ++sp) sum += ld_dsmem_f32(red + v, (uint32_t)sp);
+        if (k < Kd) finish(k, v / kTgCols, sum);
     }
+    cluster_sync_all();
 }
 
 template <typename K>
@@ -363,58 +370,75 @@ cudaError_t allow_smem(K kernel, size_t bytes) {
     return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
+// Launch with the splits of one output tile as one cluster along y.
+template <typename Kern, typename... Args>
+cudaError_t launch_split(Kern kernel, dim3 grid, size_t smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    if (grid.y > 1) {
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 1;
+        attr[0].val.clusterDim.y = grid.y;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 template <int NT, bool B_KR>
 lsn_status launch_down_nt(dim3 grid, cudaStream_t st, const uint16_t* X, const uint16_t* W, int64_t T, int64_t Kd,
-                          int cps, int ns, float scale, float* u32, uint16_t* u16, float* part, int* counters) {
+                          int cps, int ns, float scale, float* u32, uint16_t* u16) {
     constexpr size_t bytes = DownSmem<NT, B_KR>::BYTES;
     static const cudaError_t attr = allow_smem(lora_down_kernel<NT, B_KR>, bytes);
     if (attr != cudaSuccess) return fail_cuda(attr, "cudaFuncSetAttribute(lora_down smem)");
-    lora_down_kernel<NT, B_KR><<<grid, 128, bytes, st>>>(X, W, T, Kd, cps, ns, scale, u32, u16, part, counters);
+    LSN_CUDA_TRY(launch_split(lora_down_kernel<NT, B_KR>, grid, bytes, st, X, W, T, Kd, cps, ns, scale, u32, u16));
     return LSN_OK;
 }
 
 template <int NT, bool OUT_RK>
 lsn_status launch_tgrad_nt(dim3 grid, cudaStream_t st, const float* G, const uint16_t* X, int64_t T, int64_t Kd,
-                           int64_t per, int ns, float scale, int accumulate, float* out, float* partial,
-                           int* counters) {
+                           int64_t per, int ns, float scale, int accumulate, float* out) {
     constexpr size_t bytes = TgSmem<NT>::BYTES;
     static const cudaError_t attr = allow_smem(lora_tgrad_kernel<NT, OUT_RK>, bytes);
     if (attr != cudaSuccess) return fail_cuda(attr, "cudaFuncSetAttribute(lora_tgrad smem)");
-    lora_tgrad_kernel<NT, OUT_RK><<<grid, 128, bytes, st>>>(G, X, T, Kd, per, ns, scale, accumulate, out, partial,
-                                                            counters);
+    LSN_CUDA_TRY(launch_split(lora_tgrad_kernel<NT, OUT_RK>, grid, bytes, st, G, X, T, Kd, per, ns, scale, accumulate,
+                              out));
     return LSN_OK;
 }
 
 template <bool B_KR>
 lsn_status dispatch_down(int r, dim3 grid, cudaStream_t st, const uint16_t* X, const uint16_t* W, int64_t T,
-                         int64_t Kd, int cps, int ns, float scale, float* u32, uint16_t* u16, float* part,
-                         int* counters) {
+                         int64_t Kd, int cps, int ns, float scale, float* u32, uint16_t* u16) {
     switch (r / 8) {
-        case 1: return launch_down_nt<1, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16, part, counters);
-        case 2: return launch_down_nt<2, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16, part, counters);
-        case 3: return launch_down_nt<3, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16, part, counters);
-        case 4: return launch_down_nt<4, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16, part, counters);
-        case 5: return launch_down_nt<5, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16, part, counters);
-        case 6: return launch_down_nt<6, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16, part, counters);
-        case 7: return launch_down_nt<7, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16, part, counters);
-        case 8: return launch_down_nt<8, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16, part, counters);
+        case 1: return launch_down_nt<1, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16);
+        case 2: return launch_down_nt<2, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16);
+        case 3: return launch_down_nt<3, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16);
+        case 4: return launch_down_nt<4, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16);
+        case 5: return launch_down_nt<5, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16);
+        case 6: return launch_down_nt<6, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16);
+        case 7: return launch_down_nt<7, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16);
+        case 8: return launch_down_nt<8, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16);
         default: return fail(LSN_ERR_INVALID_ARG, "rank must be a multiple of 8 in [8, 64]");
     }
 }
 
 template <bool OUT_RK>
 lsn_status dispatch_tgrad(int r, dim3 grid, cudaStream_t st, const float* G, const uint16_t* X, int64_t T, int64_t Kd,
-                          int64_t per, int ns, float scale, int accumulate, float* out, float* partial,
-                          int* counters) {
+                          int64_t per, int ns, float scale, int accumulate, float* out) {
     switch (r / 8) {
-        case 1: return launch_tgrad_nt<1, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out, partial, counters);
-        case 2: return launch_tgrad_nt<2, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out, partial, counters);
-        case 3: return launch_tgrad_nt<3, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out, partial, counters);
-        case 4: return launch_tgrad_nt<4, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out, partial, counters);
-        case 5: return launch_tgrad_nt<5, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out, partial, counters);
-        case 6: return launch_tgrad_nt<6, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out, partial, counters);
-        case 7: return launch_tgrad_nt<7, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out, partial, counters);
-        case 8: return launch_tgrad_nt<8, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out, partial, counters);
+        case 1: return launch_tgrad_nt<1, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out);
+        case 2: return launch_tgrad_nt<2, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out);
+        case 3: return launch_tgrad_nt<3, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out);
+        case 4: return launch_tgrad_nt<4, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out);
+        case 5: return launch_tgrad_nt<5, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out);
+        case 6: return launch_tgrad_nt<6, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out);
+        case 7: return launch_tgrad_nt<7, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out);
+        case 8: return launch_tgrad_nt<8, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out);
         default: return fail(LSN_ERR_INVALID_ARG, "rank must be a multiple of 8 in [8, 64]");
     }
 }
@@ -425,74 +449,59 @@ lsn_status dispatch_tgrad(int r, dim3 grid, cudaStream_t st, const float* G, con
 // Split counts depend on the shape only (never on the device or pointers), so
 // a given shape always sums in the same order.
 
-// K-splits of the down projection: about four 128-thread CTAs per SM of a
-// 148-SM part, at least eight 64-wide chunks per split.
+// K-splits of the down projection: up to 8 (one cluster), aiming at about
+// four 128-thread CTAs per SM of a 148-SM part, at least four 64-wide chunks
+// per split.
 int down_splits(int64_t T, int64_t Kd) {
     const int64_t row_blocks = (T + kDnRows - 1) / kDnRows;
     if (row_blocks <= 0 || Kd < 64) return 1;
     const int64_t chunks = Kd / 64;
     int64_t s = (592 + row_blocks - 1) / row_blocks;
-    const int64_t cap = chunks / 8 > 0 ? chunks / 8 : 1;
+    const int64_t cap = chunks / 4 > 0 ? chunks / 4 : 1;
     if (s > cap) s = cap;
+    if (s > 8) s = 8;
     if (s < 1) s = 1;
     return (int)s;
 }
 
-size_t down_ws_bytes(int64_t T, int64_t Kd, int r) {
-    const int s = down_splits(T, Kd);
-    return s > 1 ? (size_t)s * T * r * sizeof(float) : 0;
-}
+size_t down_ws_bytes(int64_t, int64_t, int) { return 0; }
 
-// Token splits of a reduction: about four 128-thread CTAs per SM of a 148-SM
-// part, at least 128 tokens per split.
+// Token splits of a reduction: up to 8 (one cluster), aiming at about four
+// 128-thread CTAs per SM, at least 64 tokens per split.
 int tgrad_splits(int64_t T, int64_t Kd) {
     const int64_t tiles = (Kd + kTgCols - 1) / kTgCols;
     if (tiles <= 0 || T <= 0) return 1;
     int64_t s = (592 + tiles - 1) / tiles;
-    const int64_t by_t = (T + 127) / 128;
+    const int64_t by_t = (T + 63) / 64;
     if (s > by_t) s = by_t;
-    if (s > 64) s = 64;
+    if (s > 8) s = 8;
     if (s < 1) s = 1;
     return (int)s;
 }
 
-size_t tgrad_ws_bytes(int64_t T, int64_t Kd, int r) {
-    const int s = tgrad_splits(T, Kd);
-    return s > 1 ? (size_t)s * r * Kd * sizeof(float) : 0;
-}
+size_t tgrad_ws_bytes(int64_t, int64_t, int) { return 0; }
 
-// Integer tickets of the split reductions (one per row block or column tile).
-size_t split_counter_count(int64_t T, int64_t K, int64_t N) {
-    const int64_t a = (T + kDnRows - 1) / kDnRows;
-    const int64_t b = ((K > N ? K : N) + kTgCols - 1) / kTgCols;
-    return (size_t)(a > b ? a : b);
-}
+size_t split_counter_count(int64_t, int64_t, int64_t) { return 0; }
 
 // X [T, Kd] times W: w_rk ? W is A [r, Kd] : W is B [Kd, r].
 lsn_status launch_lora_down(const uint16_t* X, const uint16_t* W, bool w_rk, int64_t T, int64_t Kd, int r,
-                            float scale, float* u32, uint16_t* u16, float* partial, int* counters, cudaStream_t st) {
+                            float scale, float* u32, uint16_t* u16, float*, int*, cudaStream_t st) {
     if (T == 0) return LSN_OK;
     const int ns = down_splits(T, Kd);
     const int64_t chunks = Kd / 64;
     const int cps = (int)((chunks + ns - 1) / ns);
     dim3 grid((unsigned)((T + kDnRows - 1) / kDnRows), (unsigned)ns);
-    lsn_status ls = w_rk ? dispatch_down<false>(r, grid, st, X, W, T, Kd, cps, ns, scale, u32, u16, partial, counters)
-                         : dispatch_down<true>(r, grid, st, X, W, T, Kd, cps, ns, scale, u32, u16, partial, counters);
-    if (ls != LSN_OK) return ls;
-    LSN_CUDA_TRY(cudaGetLastError());
-    return LSN_OK;
+    return w_rk ? dispatch_down<false>(r, grid, st, X, W, T, Kd, cps, ns, scale, u32, u16)
+                : dispatch_down<true>(r, grid, st, X, W, T, Kd, cps, ns, scale, u32, u16);
 }
 
 lsn_status launch_lora_tgrad(const float* G, const uint16_t* X, bool out_rk, int64_t T, int64_t Kd, int r,
-                             float scale, int accumulate, float* out, float* partial, int* counters, cudaStream_t st) {
+                             float scale, int accumulate, float* out, float*, int*, cudaStream_t st) {
     const int ns = tgrad_splits(T, Kd);
     const int64_t per = ((T + ns - 1) / ns + kTgTok - 1) / kTgTok * kTgTok;
     dim3 grid((unsigned)((Kd + kTgCols - 1) / kTgCols), (unsigned)ns);
-    lsn_status ls = out_rk ? dispatch_tgrad<true>(r, grid, st, G, X, T, Kd, per, ns, scale, accumulate, out, partial, counters)
-                           : dispatch_tgrad<false>(r, grid, st, G, X, T, Kd, per, ns, scale, accumulate, out, partial, counters);
-    if (ls != LSN_OK) return ls;
-    LSN_CUDA_TRY(cudaGetLastError());
-    return LSN_OK;
+    return out_rk ? dispatch_tgrad<true>(r, grid, st, G, X, T, Kd, per, ns, scale, accumulate, out)
+                  : dispatch_tgrad<false>(r, grid, st, G, X, T, Kd, per, ns, scale, accumulate, out);
 }
 
 }  // namespace lsn

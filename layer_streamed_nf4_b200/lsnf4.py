@@ -26,6 +26,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 LSN_OK, LSN_ERR_INVALID_ARG, LSN_ERR_CUDA, LSN_ERR_NO_MEMORY, LSN_ERR_TIMEOUT, LSN_ERR_UNSUPPORTED, LSN_ERR_STATE = range(7)
 LSN_BASE_NF4, LSN_BASE_BF16 = 0, 1
 LSN_POOL_FAULT_NONE, LSN_POOL_FAULT_STALE_SLOT, LSN_POOL_FAULT_COPY_ERROR = 0, 1, 2
+LSN_OPT_FUSED_NF4 = 1
 
 STATUS_NAMES = {0: "LSN_OK", 1: "LSN_ERR_INVALID_ARG", 2: "LSN_ERR_CUDA", 3: "LSN_ERR_NO_MEMORY",
                 4: "LSN_ERR_TIMEOUT", 5: "LSN_ERR_UNSUPPORTED", 6: "LSN_ERR_STATE"}
@@ -39,7 +40,7 @@ EXPORTS = (
     "layer_pool_create", "layer_pool_register", "layer_pool_prefetch", "layer_pool_acquire",
     "layer_pool_release", "layer_pool_wait_idle", "layer_pool_stats", "layer_pool_reset",
     "layer_pool_inject_fault", "layer_pool_destroy", "lsn_timing_enable", "lsn_timing_read",
-    "nf4_quantize_noalloc",
+    "nf4_quantize_noalloc", "lsn_set_option", "lsn_get_option",
 )
 
 
@@ -98,6 +99,8 @@ _sig("lora_linear_fwd", _i, [ctypes.POINTER(Base), _vp, _i64, _vp, _vp, _i, ctyp
 _sig("lora_linear_bwd", _i, [ctypes.POINTER(Base), _vp, _vp, _i64, _vp, _vp, _i, ctypes.c_float, _vp, _vp, _vp, _i,
                              _vp, _sz, _vp])
 _sig("lsn_ws_status", _i, [_vp, _vp])
+_sig("lsn_set_option", _i, [_i, _i])
+_sig("lsn_get_option", _i, [_i])
 _sig("lsn_timing_enable", _i, [_i])
 _sig("lsn_timing_read", _i, [ctypes.POINTER(KernelTiming)])
 _sig("layer_pool_create", _i, [_i, _sz, _i, ctypes.POINTER(_vp)])
@@ -227,6 +230,16 @@ def lora_linear_bwd(W: Base, x, dY, T: int, A, B, r: int, scale: float, dX, dA, 
 
 def ws_status(ws, stream=None):
     _check(_lib.lsn_ws_status(_ptr(ws), _stream(stream)), "lsn_ws_status")
+
+
+# -------------------------------------------------------------- options ---
+
+def set_option(option: int, value: int):
+    _check(_lib.lsn_set_option(option, int(value)), "lsn_set_option")
+
+
+def get_option(option: int) -> int:
+    return int(_lib.lsn_get_option(option))
 
 
 # -------------------------------------------------------- kernel timing ---

@@ -109,6 +109,36 @@ def test_pair_kernel_with_ragged_rows(lib, orc, T, K, N):
     _full_parity(lib, orc, c, "nf4")
 
 
+@pytest.mark.parametrize("T,K,N", [(512, 4096, 9536), (300, 9536, 4096)])
+def test_fused_nf4_equals_bf16_base_of_its_dequant(lib, T, K, N):
+    """The NF4 weight converted inside the GEMM gives exactly the bits of the same
+    GEMM run on nf4_dequant's bf16 weight (same values, same MMA order).  The
+    shapes put one direction on the fused pair kernel, with a partial last
+    N tile and, for K % 128 == 64, a half-empty last contraction stage."""
+    import torch
+    lib.set_option(lib.LSN_OPT_FUSED_NF4, 1)
+    c = synth.linear_case(T, K, N, 16, 32.0, seed=T + N)
+    Lq = Linear(lib, c, "nf4")
+    Wd = torch.empty((N, K), dtype=torch.bfloat16, device="cuda")
+    lib.nf4_dequant(Lq.nf4.w, Wd)
+    Lb = Linear(lib, c, "bf16")
+    Lb.Wb = Wd
+    Lb.base = lib.base_bf16(Wd, N, K)
+    try:
+        a = (Lq.fwd(), *Lq.bwd())
+    finally:
+        lib.set_option(lib.LSN_OPT_FUSED_NF4, 0)
+    b = (Lb.fwd(), *Lb.bwd())
+    c2 = (Lq.fwd(), *Lq.bwd())                      # default path: dequantise + bf16 GEMM
+    torch.cuda.synchronize()
+    Lq.status()
+    Lb.status()
+    for name, u, v in zip(("y", "dX", "dA", "dB"), c2, b):
+        assert torch.equal(u, v), "unfused " + name
+    for name, u, v in zip(("y", "dX", "dA", "dB"), a, b):
+        assert torch.equal(u, v), name
+
+
 def test_b_zero_gives_the_base_product(lib, orc):
     c = synth.linear_case(160, 256, 320, 16, 32.0, seed=3)
     c.B[:] = 0

@@ -48,8 +48,17 @@ def _compare(a, b):
     return fwd, bwd, bad
 
 
-@pytest.mark.parametrize("name,layers,tokens", [("0.5b", 24, 512), ("3b", 4, 1024), ("8b", 4, 2048), ("72b", 3, 1024)])
-def test_streamed_equals_resident(lib, name, layers, tokens):
+@pytest.mark.parametrize("name,layers,tokens,fused", [("0.5b", 24, 512, 0), ("3b", 4, 1024, 0), ("8b", 4, 2048, 0),
+                                                     ("8b", 3, 2048, 1), ("72b", 3, 1024, 0)])
+def test_streamed_equals_resident(lib, name, layers, tokens, fused):
+    lib.set_option(lib.LSN_OPT_FUSED_NF4, fused)
+    try:
+        _streamed_equals_resident(lib, name, layers, tokens)
+    finally:
+        lib.set_option(lib.LSN_OPT_FUSED_NF4, 0)
+
+
+def _streamed_equals_resident(lib, name, layers, tokens):
     cfg = synth.STACKS[name]
     res = _run(cfg, layers, tokens, "resident")
     stm = _run(cfg, layers, tokens, "streamed", steps=2)
