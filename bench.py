@@ -143,10 +143,16 @@ def run_ours(args):
     pool_stats = None
     clocks = None
     st_main = Stack(cfg, layers=L, tokens=T, mode="streamed", n_slots=args.slots, seed=synth.SEED + rank,
-                    stream=stream)
-    modes = ["streamed"] + [m for m in ("no_h2d", "resident") if m in args.modes]
+                    stream=stream, lanes=args.lanes)
+    wanted = args.modes.split(",")
+    modes = ["streamed"] + [m for m in ("no_h2d", "resident", "serial") if m in wanted]
     for mode in modes:
-        st = st_main if mode == "streamed" else st_main.with_mode(mode)
+        if mode == "streamed":
+            st = st_main
+        elif mode == "serial":          # no_h2d with every call on the compute stream
+            st = st_main.with_mode("no_h2d", lanes=1)
+        else:
+            st = st_main.with_mode(mode)
         with torch.cuda.stream(stream):
             for _ in range(args.warmup):
                 st.step()
@@ -183,15 +189,22 @@ def run_ours(args):
             # Second timed region, same steps, every library launch bracketed
             # by CUDA events on its stream: per-kernel device time and work.
             # (The events cost host time, so the step time above is taken
-            # without them.)
+            # without them.)  It runs with one lane, so that no launch waits
+            # for SMs held by another lane's kernel inside its events.
+            st_k = st.with_mode("streamed", n_slots=args.slots, lanes=1)
+            with torch.cuda.stream(stream):
+                st_k.step()
+            stream.synchronize()
             barrier()
             lsnf4.timing_enable(True)
             with torch.cuda.stream(stream):
                 for _ in range(args.steps):
-                    st.step()
+                    st_k.step()
             stream.synchronize()
             kernel = lsnf4.timing_read()
             lsnf4.timing_enable(False)
+            st_k.check_status()
+            st_k.close()
             barrier()
         st.check_status()
         if st is not st_main:
@@ -270,6 +283,8 @@ def run_ours(args):
                                f"{args.slots}-slot VRAM pool",
                    "tokens": T, "layers": L, "rank": cfg.rank, "pool_slots": args.slots, "base": cfg.base,
                    "parallelism": f"replicas x{world}",
+                   "lanes": args.lanes,
+                   "nf4_conversion": "inside the GEMM" if args.fused_nf4 else "nf4_dequant then bf16 GEMM",
                    "l2": "inputs larger than L2 (per step ~11 GB of activations, ~3.6 GB of streamed weights)"},
         "pct_bf16_peak": 100 * flop_step / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
         "flop_per_step": flop_step,
@@ -433,15 +448,20 @@ def main():
     ap.add_argument("--tokens", type=int, default=0, help="override T (default: the workload's 2048)")
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (default 32)")
     ap.add_argument("--slots", type=int, default=2)
-    ap.add_argument("--modes", default="no_h2d,resident", help="extra modes timed after the streamed one")
+    ap.add_argument("--modes", default="no_h2d,resident,serial", help="extra modes timed after the streamed one")
+    ap.add_argument("--lanes", type=int, default=2, help="streams the seven projections of a layer are spread over")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=32)
     ap.add_argument("--cpu-budget", type=float, default=60.0)
     ap.add_argument("--ref-rows", type=int, default=4)
+    ap.add_argument("--fused-nf4", action="store_true", help="convert NF4 inside the GEMM (no bf16 copy of W)")
     ap.add_argument("--case", default="", help="profile one 8B projection (q,k,v,o,gate,up,down) instead of the stack")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.fused_nf4 and args.impl == "ours":
+        from layer_streamed_nf4_b200 import lsnf4
+        lsnf4.set_option(lsnf4.LSN_OPT_FUSED_NF4, 1)
     if args.impl == "reference":
         run_reference(args)
     elif args.case:

@@ -43,6 +43,8 @@ struct GemmArgs {
     int wrows, wcols;          // W is [wrows, wcols] row-major (N_out x K_in)
     float level[16];           // NF4 levels
     float dq[256];             // second-level table
+    const uint16_t* lora_b;    // LoRA operand of the last K-block (fwd: B [N, r]; bwd: A [r, N])
+    int lora_r;
 };
 
 namespace {
@@ -413,6 +415,336 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN, NF4>::THREADS, 1)
     }
 }
 
+// ------------------------------------------------ fused NF4 pair kernel ---
+//
+// The pair GEMM with the NF4 weight as B, converted in shared memory.  Three
+// rings advance in lockstep, one slot per 128-wide K-block, each with its own
+// barriers so that no stage waits on a chain of the others' latencies:
+//   A ring   TMA of this CTA's 128 A rows (counted on the leader), released
+//            by the MMA (multicast commit);
+//   P ring   TMA of this CTA's packed NF4 tile (128 rows x 64 bytes, 64-byte
+//            swizzle), issued by its own producer warp and released by the
+//            converters as soon as they have read it;
+//   B ring   the converted bf16 tile (128-byte swizzle, the MMA operand),
+//            written by 8 converter warps, released by the MMA.
+// The LoRA K-block's B (B_lora or A_lora) is copied into the B ring by the
+// same converters, so every ring has the same slot sequence.
+template <bool B_MN>
+struct CfgN {
+    static constexpr int BN = 256;
+    static constexpr int A_SUB = BM * SUB * 2;      // 16 KB
+    static constexpr int A_BYTES = 2 * A_SUB;       // 32 KB
+    static constexpr int B_BYTES = 128 * BK * 2;    // 32 KB: 128 B rows x 128 contraction
+    static constexpr int P_BYTES = 128 * 64;        // 8 KB packed
+    static constexpr int RING_A = STAGES * A_BYTES;
+    static constexpr int RING_B = STAGES * B_BYTES;
+    static constexpr int RING_P = STAGES * P_BYTES;
+    static constexpr int BAR_BYTES = 256;
+    static constexpr int SMEM_BYTES = RING_A + RING_B + RING_P + BAR_BYTES + 1024 + 1024;
+    static constexpr uint32_t IDESC = idesc_bf16(2 * BM, BN, 0, B_MN ? 1 : 0);
+    static constexpr uint32_t TMEM_COLS = 2 * BN;
+    static constexpr int THREADS = 192 + 32 * CONV_WARPS + 32;   // + converters + packed producer
+};
+
+template <bool B_MN>
+__global__ void __launch_bounds__(CfgN<B_MN>::THREADS, 1)
+    lsn_gemm_nf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmP,
+                        const __grid_constant__ CUtensorMap tmLA, const __grid_constant__ GemmArgs p) {
+    using C = CfgN<B_MN>;
+    constexpr int BN = C::BN;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* ringA = smem;
+    uint8_t* ringB = smem + C::RING_A;
+    uint8_t* ringP = ringB + C::RING_B;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(ringP + C::RING_P);
+    uint64_t* fullA = bars;
+    uint64_t* emptyA = fullA + STAGES;
+    uint64_t* fullP = emptyA + STAGES;
+    uint64_t* emptyP = fullP + STAGES;
+    uint64_t* readyB = emptyP + STAGES;
+    uint64_t* emptyB = readyB + STAGES;
+    uint64_t* acc_full = emptyB + STAGES;
+    uint64_t* acc_empty = acc_full + 2;
+    uint64_t* drain = acc_empty + 2;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    float* dq_s = reinterpret_cast<float*>(ringP + C::RING_P + C::BAR_BYTES);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int unit = (int)(blockIdx.x >> 1), nunits = (int)(gridDim.x >> 1);
+    const int num_m = (p.M + 2 * BM - 1) / (2 * BM);
+    const int num_n = (p.N + BN - 1) / BN;
+    const int num_tiles = num_m * num_n;
+    const int nkb = p.num_kb + (p.lora_k16 > 0 ? 1 : 0);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&fullA[s], 1);
+            mbar_init(&emptyA[s], 1);
+            mbar_init(&fullP[s], 1);
+            mbar_init(&emptyP[s], CONV_WARPS);
+            mbar_init(&readyB[s], 2 * CONV_WARPS);
+            mbar_init(&emptyB[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 8); }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) dq_s[i] = p.dq[i];
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA); tma_prefetch_desc(&tmP); tma_prefetch_desc(&tmLA);
+    }
+    if (warp == 1) { tmem_alloc_pair(tmem_holder, C::TMEM_COLS); tmem_relinquish_pair(); }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+    const int conv_first_warp = 6, ppro_warp = 6 + CONV_WARPS;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // -------------------------------------------------- A producer --
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = unit; tile < num_tiles && ok; tile += nunits) {
+                const int m_row = (tile % num_m) * 2 * BM + (int)rank * BM;
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(&emptyA[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+                    uint8_t* sA = ringA + stage * C::A_BYTES;
+                    const uint32_t fbar = mapa_shared(smem_u32(&fullA[stage]), 0);
+                    if (leader) mbar_arrive_expect_tx(&fullA[stage], 2 * C::A_BYTES);
+                    const bool lora = kb >= p.num_kb;
+                    const CUtensorMap* ma = lora ? &tmLA : &tmA;
+                    const int kc = lora ? 0 : kb * BK;
+                    tma_load_2d_pair(sA, ma, kc, m_row, fbar);
+                    tma_load_2d_pair(sA + C::A_SUB, ma, kc + SUB, m_row, fbar);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (!ok) raise_error(abort_flag, p.err, 1);
+        }
+    } else if (warp == ppro_warp) {
+        if (lane == 0) {
+            // --------------------------------------------- packed producer --
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = unit; tile < num_tiles && ok; tile += nunits) {
+                const int n_off = (tile / num_m) * BN + (int)rank * 128;
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(&emptyP[stage], phase ^ 1, abort_flag)) { ok = false; break; }
+                    const bool lora = kb >= p.num_kb;
+                    mbar_arrive_expect_tx(&fullP[stage], lora ? 0u : (uint32_t)C::P_BYTES);
+                    if (!lora) {
+                        uint8_t* sP = ringP + stage * C::P_BYTES;
+                        if (!B_MN) tma_load_2d(sP, &tmP, kb * 64, n_off, &fullP[stage]);
+                        else       tma_load_2d(sP, &tmP, n_off / 2, kb * BK, &fullP[stage]);
+                    }
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (!ok) raise_error(abort_flag, p.err, 5);
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // -------------------------------------------------- MMA issuer --
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true;
+            for (int tile = unit; tile < num_tiles && ok; tile += nunits) {
+                if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!mbar_wait(&fullA[stage], phase, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait_cluster(&readyB[stage], phase, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(ringA + stage * C::A_BYTES);
+                    const uint32_t b0 = smem_u32(ringB + stage * C::B_BYTES);
+                    const int nk = (kb < p.num_kb) ? BK / 16 : p.lora_k16;
+                    for (int k = 0; k < nk; ++k) {
+                        const int j = k >> 2, kk = k & 3;
+                        const uint64_t ad = smem_desc_sw128(a0 + j * C::A_SUB + kk * 32, 16, 1024);
+                        const uint64_t bd = B_MN ? smem_desc_sw128(b0 + k * 2048, BK * 128, 1024)
+                                                 : smem_desc_sw128(b0 + j * (BK * 128) + kk * 32, 16, 1024);
+                        umma_bf16_pair(d_tmem, ad, bd, C::IDESC, (kb | k) ? 1u : 0u);
+                    }
+                    umma_commit_pair(&emptyA[stage]);
+                    umma_commit_pair(&emptyB[stage]);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+                if (!ok) break;
+                umma_commit_pair(&acc_full[acc]);
+                acc ^= 1;
+                if (acc == 0) acc_phase ^= 1;
+            }
+            if (!ok) raise_error(abort_flag, p.err, 2);
+            umma_commit_pair(drain);
+            mbar_wait(drain, 0, nullptr);
+        }
+    } else if (warp < conv_first_warp) {
+        // -------------------------------------------------------- epilogue --
+        const int q = warp & 3;
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int tile = unit; tile < num_tiles; tile += nunits) {
+            const int mb = tile % num_m, nb = tile / num_m;
+            const bool got = mbar_wait(&acc_full[acc], acc_phase, abort_flag);
+            if (!__all_sync(0xffffffffu, got)) { if (lane == 0) raise_error(abort_flag, p.err, 3); break; }
+            tc_fence_after();
+            const int row = mb * 2 * BM + (int)rank * BM + q * 32 + lane;
+            #pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                const int col = nb * BN + c * 32;
+                if (col >= p.N) break;
+                uint32_t v[32];
+                tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c * 32), v);
+                tmem_ld_wait();
+                if (row < p.M) {
+                    uint4* dst = reinterpret_cast<uint4*>(p.D + (int64_t)row * p.ldd + col);
+                    #pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        uint4 o;
+                        o.x = pack_bf16x2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
+                        o.y = pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
+                        o.z = pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
+                        o.w = pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
+                        dst[i] = o;
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[acc]), 0));
+            acc ^= 1;
+            if (acc == 0) acc_phase ^= 1;
+        }
+    } else {
+        // ------------------------------------------------------- converters --
+        // Thread t owns one (row, 64-block) of the CTA's 128 x 128 B tile per
+        // K-block: row = t % 128 (a B row: forward W row n; backward the
+        // contraction row n of W), block = t / 128 (64 consecutive W
+        // columns).  Its 64 bf16 land in one 128-byte row of a 128-byte
+        // swizzled atom: block b's atom at b * 16 KB, row at (row/8)*1024 +
+        // (row%8)*128, 16-byte chunk c at position c ^ (row % 8).
+        const int t = threadIdx.x - 32 * conv_first_warp;
+        const int row = t & 127, blk = t >> 7;
+        const int64_t nblk_row = p.wcols / 64;
+        const float off = *p.absmax_off;
+        struct Meta { uint32_t code; float s2; bool ok; };
+        auto fetch = [&](int tl, int k) -> Meta {
+            Meta m{0u, 0.0f, false};
+            if (tl >= num_tiles || k >= p.num_kb) return m;
+            const int n_off = (tl / num_m) * BN + (int)rank * 128;
+            const int64_t wr = B_MN ? (int64_t)k * BK + row : (int64_t)n_off + row;
+            const int64_t wb = B_MN ? (int64_t)(n_off / 64) + blk : (int64_t)k * 2 + blk;
+            if (wr < p.wrows && wb < nblk_row) {
+                const int64_t bi = wr * nblk_row + wb;
+                m.code = __ldg(p.absmax_q + bi);
+                m.s2 = __ldg(p.absmax_s2 + (bi >> 8));
+                m.ok = true;
+            }
+            return m;
+        };
+        int ft = unit, fk = 0;
+        auto step = [&]() { if (++fk == nkb) { fk = 0; ft += nunits; } };
+        Meta m0 = fetch(ft, fk);
+        step();
+        Meta m1 = fetch(ft, fk);
+        step();
+        int stage = 0;
+        uint32_t phase = 0;
+        bool bad = false;
+        for (int tile = unit; tile < num_tiles && !bad; tile += nunits) {
+            const int n_off = (tile / num_m) * BN + (int)rank * 128;
+            for (int kb = 0; kb < nkb; ++kb) {
+                const Meta cur = m0;
+                m0 = m1;
+                m1 = fetch(ft, fk);
+                step();
+                const bool got = mbar_wait(&fullP[stage], phase, abort_flag) &&
+                                 mbar_wait(&emptyB[stage], phase ^ 1, abort_flag);
+                if (!__all_sync(0xffffffffu, got)) { if (lane == 0) raise_error(abort_flag, p.err, 4); bad = true; break; }
+                uint8_t* dst = ringB + stage * C::B_BYTES + blk * (BK * 128) + (row >> 3) * 1024 + (row & 7) * 128;
+                if (kb < p.num_kb) {
+                    if (cur.ok) {
+                        const float ah = __fadd_rn(__fmul_rn(dq_s[cur.code], cur.s2), off);
+                        uint32_t e[8];
+                        #pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            e[i] = pack_bf16x2(__fmul_rn(p.level[2 * i], ah), __fmul_rn(p.level[2 * i + 1], ah));
+                        uint32_t lo[4], hi[4];
+                        #pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            lo[i] = prmt(e[2 * i], e[2 * i + 1], 0x6420u);
+                            hi[i] = prmt(e[2 * i], e[2 * i + 1], 0x7531u);
+                        }
+                        const uint8_t* prow = ringP + stage * C::P_BYTES + row * 64;
+                        uint4 pk[2];
+                        #pragma unroll
+                        for (int h = 0; h < 2; ++h)
+                            pk[h] = *reinterpret_cast<const uint4*>(prow + (((2 * blk + h) ^ ((row >> 1) & 3)) << 4));
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&emptyP[stage]);   // packed slot read: release it early
+                        #pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const uint32_t w[4] = {pk[h].x, pk[h].y, pk[h].z, pk[h].w};
+                            #pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const int c = h * 4 + i;
+                                *reinterpret_cast<uint4*>(dst + ((c ^ (row & 7)) << 4)) = nf4x8_to_bf16(w[i], lo, hi);
+                            }
+                        }
+                    } else {
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&emptyP[stage]);
+                        #pragma unroll
+                        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(dst + (c << 4)) = make_uint4(0, 0, 0, 0);
+                    }
+                } else {
+                    // LoRA K-block: copy the bf16 LoRA operand (zero-padded).
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&emptyP[stage]);
+                    int64_t src_row = -1, col0 = 0;
+                    int ncols = 0, ld = 0;
+                    if (!B_MN) {            // B_lora [N, r]: row n, columns 0..r-1 (block 0 only)
+                        const int64_t n = (int64_t)n_off + row;
+                        if (blk == 0 && n < p.N) { src_row = n; col0 = 0; ncols = p.lora_r; ld = p.lora_r; }
+                    } else {                // A_lora [r, N]: row j, columns n_off + 64 blk ..
+                        const int64_t c0 = (int64_t)n_off + 64 * blk;
+                        if (row < p.lora_r && c0 < p.N) { src_row = row; col0 = c0; ncols = 64; ld = p.N; }
+                    }
+                    #pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        uint4 v = make_uint4(0, 0, 0, 0);
+                        if (src_row >= 0 && c * 8 < ncols)
+                            v = __ldg(reinterpret_cast<const uint4*>(p.lora_b + src_row * ld + col0) + c);
+                        *reinterpret_cast<uint4*>(dst + ((c ^ (row & 7)) << 4)) = v;
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&readyB[stage]), 0));
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            }
+        }
+    }
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    }
+}
+
 // --------------------------------------------------------- tensor maps ---
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -505,17 +837,12 @@ lsn_status launch_gemm_nf4(const uint16_t* A, int64_t lda, const lsn_nf4_weight*
                            int* err, cudaStream_t st) {
     if (!gemm_use_pairs(M, N)) return LSN_ERR_UNSUPPORTED;
     const Nf4Tables& T = nf4_tables();
-    CUtensorMap ma, mp, mla, mlb;
+    CUtensorMap ma, mp, mla;
     lsn_status s;
     if ((s = make_map(&ma, A, Kc, M, lda, SUB, BM)) != LSN_OK) return s;
     // packed [wrows, wcols/2] bytes, boxes of 64 bytes x 128 rows
     if ((s = make_map(&mp, w->packed, w->cols / 2, w->rows, w->cols / 2, 64, 128, true)) != LSN_OK) return s;
     if ((s = make_map(&mla, LA, r, M, r, SUB, BM)) != LSN_OK) return s;
-    if (!b_mn) {
-        if ((s = make_map(&mlb, LB, r, N, r, SUB, 128)) != LSN_OK) return s;
-    } else {
-        if ((s = make_map(&mlb, LB, N, r, N, 64, BK)) != LSN_OK) return s;
-    }
     GemmArgs args{};
     args.M = (int)M;
     args.N = (int)N;
@@ -531,8 +858,39 @@ lsn_status launch_gemm_nf4(const uint16_t* A, int64_t lda, const lsn_nf4_weight*
     args.wcols = (int)w->cols;
     std::memcpy(args.level, T.level, sizeof(args.level));
     std::memcpy(args.dq, T.dq, sizeof(args.dq));
-    return b_mn ? launch_cfg<true, 256, true, true>(ma, mp, mla, mlb, args, st)
-                : launch_cfg<true, 256, false, true>(ma, mp, mla, mlb, args, st);
+    args.lora_b = LB;
+    args.lora_r = r;
+    auto launch = [&](auto kernel, int smem_bytes, int threads) -> lsn_status {
+        const int tiles = ((args.M + 255) / 256) * ((args.N + 255) / 256);
+        const int units = sm_count() / 2;
+        const int grid = 2 * (tiles < units ? tiles : units);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)grid);
+        cfg.blockDim = dim3((unsigned)threads);
+        cfg.dynamicSmemBytes = smem_bytes;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        LSN_CUDA_TRY(cudaLaunchKernelEx(&cfg, kernel, ma, mp, mla, args));
+        return LSN_OK;
+    };
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+        attr_err = cudaFuncSetAttribute(lsn_gemm_nf4_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        CfgN<false>::SMEM_BYTES);
+        if (attr_err == cudaSuccess)
+            attr_err = cudaFuncSetAttribute(lsn_gemm_nf4_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            CfgN<true>::SMEM_BYTES);
+    });
+    if (attr_err != cudaSuccess) return fail_cuda(attr_err, "cudaFuncSetAttribute(gemm nf4 smem)");
+    return b_mn ? launch(lsn_gemm_nf4_kernel<true>, CfgN<true>::SMEM_BYTES, CfgN<true>::THREADS)
+                : launch(lsn_gemm_nf4_kernel<false>, CfgN<false>::SMEM_BYTES, CfgN<false>::THREADS);
 }
 
 // D = A . op(B) + LA . op(LB).

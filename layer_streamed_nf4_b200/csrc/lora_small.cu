@@ -64,28 +64,47 @@ __device__ __forceinline__ float ld_dsmem_f32(const float* local_ptr, uint32_t r
 // out[t, j] = sum_k X[t, k] * Wt(j, k) for j < r, with W given either as
 // A [r, Kd] (u = x A^T) or as B [Kd, r] (g = dY B).  A CTA owns 64 token rows
 // and one split of the K range; 64-wide K chunks of X and W are staged in
-// shared memory by cp.async through a 4-stage ring (rows padded so ldmatrix
-// is conflict-free), and each warp multiplies its 16 rows with W on the
+// shared memory by cp.async through a 3-stage ring (16-byte chunks XOR-
+// swizzled by row, so ldmatrix is conflict-free without padding), and each warp multiplies its 16 rows with W on the
 // warp-level tensor-core instruction (mma.sync m16n8k16, bf16 in, fp32
 // accumulate; the inputs are exact bf16 values).  W in the B layout is read
 // with ldmatrix.trans, so no transposed copy is made.  The big contractions
 // use tcgen05; this skinny one is bound by the HBM read of X.
+//
+// At r = 16 the ring takes 30 KB, small enough for one CTA to share an SM
+// with a running GEMM CTA (about 194 KB), so the side work of one
+// projection can proceed underneath another projection's GEMM when the
+// caller issues them on two streams.
 constexpr int kDnWarps = 4;
 constexpr int kDnRows = 16 * kDnWarps;       // token rows per CTA
-constexpr int kDnStages = 4;
-constexpr int kDnPitch = 72;                 // bf16 per staged X row (64 + 8 padding)
+constexpr int kDnStages = 3;
+
+// Offset (in bf16) of element (row, col) of a staged tile whose rows hold
+// `pitch` bf16, with the 16-byte chunk index XOR-ed by `swz`.
+__device__ __forceinline__ int swz_off(int row, int col, int pitch, int swz) {
+    return row * pitch + (((col >> 3) ^ swz) << 3) + (col & 7);
+}
 
 template <int NT, bool B_KR>
 struct DownSmem {
     static constexpr int R = 8 * NT;
     static constexpr int NP = (NT + 1) / 2;                       // n-tile pairs
     static constexpr int WROWS = B_KR ? 64 : 16 * NP;             // staged W rows
-    static constexpr int WPITCH = B_KR ? 16 * NP + 8 : kDnPitch;  // bf16 per staged W row
-    static constexpr size_t X_BYTES = sizeof(uint16_t) * kDnStages * kDnRows * kDnPitch;
-    static constexpr size_t W_BYTES = sizeof(uint16_t) * kDnStages * WROWS * WPITCH;
+    // B [Kd, r] rows hold 16*NP rank columns: 32, 64 or 128 bytes, swizzled
+    // so eight consecutive rows hit distinct banks; 96-byte rows are padded.
+    static constexpr int WPITCH = B_KR ? (NP == 3 ? 16 * NP + 8 : 16 * NP) : 64;
+    static constexpr int X_TILE = kDnRows * 64;                   // bf16 per X stage
+    static constexpr int W_TILE = WROWS * WPITCH;                 // bf16 per W stage
+    static constexpr size_t X_BYTES = sizeof(uint16_t) * kDnStages * X_TILE;
+    static constexpr size_t W_BYTES = sizeof(uint16_t) * kDnStages * W_TILE;
     static constexpr size_t RING = X_BYTES + W_BYTES;
     static constexpr size_t RED = sizeof(float) * kDnRows * R;
     static constexpr size_t BYTES = RING > RED ? RING : RED;
+    // chunk swizzle of a staged W row
+    __device__ static __forceinline__ int wswz(int row) {
+        if (!B_KR) return row & 7;
+        return NP == 1 ? (row >> 2) & 1 : NP == 2 ? (row >> 1) & 3 : NP == 4 ? row & 7 : 0;
+    }
 };
 
 template <int NT, bool B_KR>
@@ -95,9 +114,13 @@ __global__ void __launch_bounds__(128) lora_down_kernel(const uint16_t* __restri
                                                         uint16_t* __restrict__ u16) {
     using L = DownSmem<NT, B_KR>;
     constexpr int R = L::R, NP = L::NP, WROWS = L::WROWS, WPITCH = L::WPITCH;
-    extern __shared__ __align__(16) uint8_t dn_smem[];
-    auto xs = reinterpret_cast<uint16_t (*)[kDnRows][kDnPitch]>(dn_smem);
-    auto ws = reinterpret_cast<uint16_t (*)[WROWS][WPITCH]>(dn_smem + L::X_BYTES);
+    extern __shared__ __align__(128) uint8_t dn_smem[];
+    uint16_t* xs = reinterpret_cast<uint16_t*>(dn_smem);                 // [stage][64 rows][64], swizzled
+    uint16_t* ws = reinterpret_cast<uint16_t*>(dn_smem + L::X_BYTES);    // [stage][WROWS][WPITCH]
+    auto xa = [&](int st, int row, int col) { return smem_u32(xs + st * L::X_TILE + swz_off(row, col, 64, row & 7)); };
+    auto wa = [&](int st, int row, int col) {
+        return smem_u32(ws + st * L::W_TILE + swz_off(row, col, WPITCH, L::wswz(row)));
+    };
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t row_base = (int64_t)blockIdx.x * kDnRows;
     const int64_t nchunks = Kd / 64;
@@ -111,18 +134,18 @@ __global__ void __launch_bounds__(128) lora_down_kernel(const uint16_t* __restri
             const int p = tid + i * 128, row = p >> 3, piece = p & 7;
             const int64_t t = row_base + row;
             const bool ok = t < T;
-            cp_async16(smem_u32(&xs[stage][row][piece * 8]), X + (ok ? t : 0) * Kd + c * 64 + piece * 8, ok ? 16u : 0u);
+            cp_async16(xa(stage, row, piece * 8), X + (ok ? t : 0) * Kd + c * 64 + piece * 8, ok ? 16u : 0u);
         }
         if (B_KR) {                                       // W = B [Kd, r]: 64 rows x r/8 pieces
             for (int p = tid; p < 64 * NT; p += 128) {
                 const int row = p / NT, piece = p % NT;
-                cp_async16(smem_u32(&ws[stage][row][piece * 8]), W + (c * 64 + row) * (int64_t)R + piece * 8, 16u);
+                cp_async16(wa(stage, row, piece * 8), W + (c * 64 + row) * (int64_t)R + piece * 8, 16u);
             }
         } else {                                          // W = A [r, Kd]: WROWS rows x 8 pieces
             for (int p = tid; p < WROWS * 8; p += 128) {
                 const int row = p >> 3, piece = p & 7;
                 const bool ok = row < R;
-                cp_async16(smem_u32(&ws[stage][row][piece * 8]), W + (int64_t)(ok ? row : 0) * Kd + c * 64 + piece * 8,
+                cp_async16(wa(stage, row, piece * 8), W + (int64_t)(ok ? row : 0) * Kd + c * 64 + piece * 8,
                            ok ? 16u : 0u);
             }
         }
@@ -147,24 +170,24 @@ __global__ void __launch_bounds__(128) lora_down_kernel(const uint16_t* __restri
     const int w_col = B_KR ? 8 * (lane >> 4) : 8 * ((lane >> 3) & 1);
     for (int64_t i = 0; i < nc; ++i) {
         cp_async_wait<kDnStages - 2>();
-        __syncthreads();
+        __syncthreads();                                  // chunk i landed; chunk i-1's stage is free
+        const int64_t nxt = i + kDnStages - 1;            // refill it before computing on chunk i
+        if (nxt < nc) load((int)(nxt % kDnStages), c_begin + nxt);
+        cp_async_commit();
         const int st = (int)(i % kDnStages);
         #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
             uint32_t a0, a1, a2, a3;
-            ldsm_x4(smem_u32(&xs[st][a_row][ks * 16 + a_col]), a0, a1, a2, a3);
+            ldsm_x4(xa(st, a_row, ks * 16 + a_col), a0, a1, a2, a3);
             #pragma unroll
             for (int p = 0; p < NP; ++p) {
                 uint32_t b00, b01, b10, b11;
-                if (B_KR) ldsm_x4_t(smem_u32(&ws[st][ks * 16 + w_row][p * 16 + w_col]), b00, b01, b10, b11);
-                else      ldsm_x4(smem_u32(&ws[st][p * 16 + w_row][ks * 16 + w_col]), b00, b01, b10, b11);
+                if (B_KR) ldsm_x4_t(wa(st, ks * 16 + w_row, p * 16 + w_col), b00, b01, b10, b11);
+                else      ldsm_x4(wa(st, p * 16 + w_row, ks * 16 + w_col), b00, b01, b10, b11);
                 mma_bf16_16816(acc[2 * p], a0, a1, a2, a3, b00, b01);
                 mma_bf16_16816(acc[2 * p + 1], a0, a1, a2, a3, b10, b11);
             }
         }
-        const int64_t nxt = i + kDnStages - 1;            // refill the stage consumed last iteration
-        if (nxt < nc) load((int)(nxt % kDnStages), c_begin + nxt);
-        cp_async_commit();
     }
     cp_async_wait<0>();
 
@@ -214,21 +237,23 @@ __global__ void __launch_bounds__(128) lora_down_kernel(const uint16_t* __restri
 // R[j, k] = sum_{t in split} G[t, j] * X[t, k] (dA with G = g, X = x; dB with
 // G = u, X = dY).  On the warp-level tensor-core instruction with M = k, N = j
 // and the tokens as the contraction: X tiles [32 t x 128 k] are staged by
-// cp.async (4 stages) and read transposed with ldmatrix.trans; G is fp32, so
+// cp.async (3 stages, 16-byte chunks XOR-swizzled by token row) and read
+// transposed with ldmatrix.trans; G is fp32, so
 // each element enters as two bf16 MMAs, hi = bf16(G) and lo = bf16(G - hi),
 // which leaves a relative error below 2^-17 per product before fp32
 // accumulation.  A CTA owns 128 columns k (warp w: k0+32w .. +31) and one
-// token split; splits are combined by the last CTA of each column tile in
-// split order.
+// token split; the splits of a column tile form one thread-block cluster and
+// are added in split order through distributed shared memory.  At r = 16 the
+// ring takes 31.5 KB, small enough to share an SM with a running GEMM CTA.
 constexpr int kTgCols = 128;
 constexpr int kTgTok = 32;          // tokens per staged tile (two MMA k-steps)
-constexpr int kTgStages = 4;
-constexpr int kTgXPitch = kTgCols + 8;
+constexpr int kTgStages = 3;
 
 template <int NT>
 struct TgSmem {
     static constexpr int GPITCH = 8 * NT + 4;
-    static constexpr size_t X_BYTES = sizeof(uint16_t) * kTgStages * kTgTok * kTgXPitch;
+    static constexpr int X_TILE = kTgTok * kTgCols;                // bf16 per X stage
+    static constexpr size_t X_BYTES = sizeof(uint16_t) * kTgStages * X_TILE;
     static constexpr size_t G_BYTES = sizeof(float) * kTgStages * kTgTok * GPITCH;
     static constexpr size_t RING = X_BYTES + G_BYTES;
     static constexpr size_t RED = sizeof(float) * 8 * NT * kTgCols;
@@ -241,8 +266,11 @@ __global__ void __launch_bounds__(128) lora_tgrad_kernel(const float* __restrict
                                                          float scale, int accumulate, float* __restrict__ out) {
     using L = TgSmem<NT>;
     constexpr int R = 8 * NT, GPITCH = L::GPITCH;
-    extern __shared__ __align__(16) uint8_t tg_smem[];
-    auto xs = reinterpret_cast<uint16_t (*)[kTgTok][kTgXPitch]>(tg_smem);
+    extern __shared__ __align__(128) uint8_t tg_smem[];
+    uint16_t* xs = reinterpret_cast<uint16_t*>(tg_smem);                 // [stage][32 tokens][128], swizzled
+    auto xa = [&](int st, int row, int col) {
+        return smem_u32(xs + st * L::X_TILE + swz_off(row, col, kTgCols, row & 7));
+    };
     auto gs = reinterpret_cast<float (*)[kTgTok][GPITCH]>(tg_smem + L::X_BYTES);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t k0 = (int64_t)blockIdx.x * kTgCols;
@@ -257,7 +285,7 @@ __global__ void __launch_bounds__(128) lora_tgrad_kernel(const float* __restrict
             const int p = tid + i * 128, row = p >> 4, piece = p & 15;
             const int64_t t = t0 + row, k = k0 + piece * 8;
             const bool ok = t < te && k < Kd;
-            cp_async16(smem_u32(&xs[stage][row][piece * 8]), X + (ok ? t : 0) * Kd + (ok ? k : 0), ok ? 16u : 0u);
+            cp_async16(xa(stage, row, piece * 8), X + (ok ? t : 0) * Kd + (ok ? k : 0), ok ? 16u : 0u);
         }
         for (int p = tid; p < kTgTok * (R / 4); p += 128) {   // G: 32 rows x R/4 pieces
             const int row = p / (R / 4), piece = p % (R / 4);
@@ -285,7 +313,10 @@ __global__ void __launch_bounds__(128) lora_tgrad_kernel(const float* __restrict
     const int g = lane >> 2, q = lane & 3;
     for (int64_t i = 0; i < ntiles; ++i) {
         cp_async_wait<kTgStages - 2>();
-        __syncthreads();
+        __syncthreads();                                  // tile i landed; tile i-1's stage is free
+        const int64_t nxt = i + kTgStages - 1;            // refill it before computing on tile i
+        if (nxt < ntiles) load((int)(nxt % kTgStages), nxt);
+        cp_async_commit();
         const int st = (int)(i % kTgStages);
         #pragma unroll
         for (int kk = 0; kk < kTgTok / 16; ++kk) {
@@ -305,7 +336,7 @@ __global__ void __launch_bounds__(128) lora_tgrad_kernel(const float* __restrict
             #pragma unroll
             for (int m = 0; m < 2; ++m) {
                 uint32_t a0, a1, a2, a3;
-                ldsm_x4_t(smem_u32(&xs[st][kk * 16 + a_t][warp * 32 + m * 16 + a_k]), a0, a1, a2, a3);
+                ldsm_x4_t(xa(st, kk * 16 + a_t, warp * 32 + m * 16 + a_k), a0, a1, a2, a3);
                 #pragma unroll
                 for (int n = 0; n < NT; ++n) {
                     mma_bf16_16816(acc[m][n], a0, a1, a2, a3, bh[n][0], bh[n][1]);
@@ -313,9 +344,6 @@ __global__ void __launch_bounds__(128) lora_tgrad_kernel(const float* __restrict
                 }
             }
         }
-        const int64_t nxt = i + kTgStages - 1;
-        if (nxt < ntiles) load((int)(nxt % kTgStages), nxt);
-        cp_async_commit();
     }
     cp_async_wait<0>();
 
@@ -367,7 +395,11 @@ __global__ void __launch_bounds__(128) lora_tgrad_kernel(const float* __restrict
 
 template <typename K>
 cudaError_t allow_smem(K kernel, size_t bytes) {
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    // Prefer the largest shared-memory carveout, the one a GEMM CTA runs
+    // with, so these CTAs can be placed beside it.
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    return e;
 }
 
 // Launch with the splits of one output tile as one cluster along y.

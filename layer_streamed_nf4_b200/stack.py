@@ -10,6 +10,16 @@ backward sweep over L-1..0 (acquire i, prefetch i-1, seven lora_linear_bwd
 calls, release i).  All compute and all copies are library calls; this file
 only sequences them and owns the (synthetic) tensors.
 
+Lanes: the seven projections of a layer are independent calls, so they are
+issued round-robin on `lanes` streams (default 2), each with its own
+workspace.  The side kernels and the dequantisation of one projection then
+run underneath another projection's GEMM on the SMs' spare shared memory
+and issue slots.  The lanes fork from the compute stream after the layer's
+acquire and join it before the layer's release, so the pool's ordering
+(release event on the compute stream) is unchanged.  Each call's arithmetic
+is independent of the lane it runs on, so results are bitwise the same for
+any lane count.
+
 Modes with identical kernels and launch shapes, for the bit-exactness gate
 ("Exact Layer Streaming", abstract: streamed compared with a resident run of
 the same numerics):
@@ -43,7 +53,8 @@ class ProjLayout:
 class Stack:
     def __init__(self, cfg: synth.StackConfig, layers: int | None = None, tokens: int | None = None,
                  mode: str = "streamed", n_slots: int = 2, seed: int = synth.SEED, keep_outputs: bool = False,
-                 distinct_activations: bool = True, device: int = 0, stream: torch.cuda.Stream | None = None):
+                 distinct_activations: bool = True, device: int = 0, stream: torch.cuda.Stream | None = None,
+                 lanes: int = 2):
         assert mode in ("resident", "streamed", "no_h2d")
         self.cfg, self.mode, self.seed = cfg, mode, seed
         self.L = layers if layers is not None else cfg.layers
@@ -54,6 +65,11 @@ class Stack:
         self.dev = torch.device("cuda", device)
         self.stream = stream if stream is not None else torch.cuda.current_stream(self.dev)
         self.keep_outputs = keep_outputs
+        assert lanes >= 1
+        self.n_lanes = lanes
+        self.lanes = [self.stream] + [torch.cuda.Stream(self.dev) for _ in range(lanes - 1)]
+        self._fork = [torch.cuda.Event() for _ in range(lanes)]
+        self._join = [torch.cuda.Event() for _ in range(lanes)]
         off = 0
         self.proj: list[ProjLayout] = []
         for name, K, N in cfg.projections:
@@ -115,7 +131,7 @@ class Stack:
         self.dX = {(l, pi): torch.empty((T, p.K), dtype=torch.bfloat16, device=dev)
                    for l in range(nl) for pi, p in enumerate(self.proj)}
         self.ws_bytes = max(lsnf4.lora_ws_bytes(T, p.K, p.N, r, self.kind) for p in self.proj)
-        self.ws = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=dev)
+        self.ws = [torch.zeros(self.ws_bytes, dtype=torch.uint8, device=dev) for _ in range(self.n_lanes)]
         torch.cuda.synchronize(dev)
 
     def _setup_mode(self, n_slots: int):
@@ -131,12 +147,19 @@ class Stack:
                 lsnf4.layer_pool_prefetch(self.pool, l)
             lsnf4.layer_pool_wait_idle(self.pool, 600000)
 
-    def with_mode(self, mode: str, n_slots: int = 2) -> "Stack":
-        """A stack sharing this one's host blobs and tensors, run in another mode."""
+    def with_mode(self, mode: str, n_slots: int = 2, lanes: int | None = None) -> "Stack":
+        """A stack sharing this one's host blobs and tensors, run in another mode
+        (and, if given, another lane count)."""
         import copy
         assert mode in ("resident", "streamed", "no_h2d")
         other = copy.copy(self)
         other.mode, other.pool, other.resident, other._calls = mode, None, None, {}
+        if lanes is not None and lanes != self.n_lanes:
+            other.n_lanes = lanes
+            other.lanes = [self.stream] + [torch.cuda.Stream(self.dev) for _ in range(lanes - 1)]
+            other._fork = [torch.cuda.Event() for _ in range(lanes)]
+            other._join = [torch.cuda.Event() for _ in range(lanes)]
+            other.ws = [torch.zeros(self.ws_bytes, dtype=torch.uint8, device=self.dev) for _ in range(lanes)]
         other._setup_mode(n_slots)
         return other
 
@@ -174,6 +197,19 @@ class Stack:
     def _out(self, d, l, pi):
         return d[(l if self.keep_outputs else 0), pi]
 
+    def _fork_lanes(self):
+        """Lanes 1.. start after what the compute stream has issued (the acquire)."""
+        if self.n_lanes > 1:
+            self._fork[0].record(self.stream)
+            for ln in self.lanes[1:]:
+                ln.wait_event(self._fork[0])
+
+    def _join_lanes(self):
+        """The compute stream continues after every lane's work on the layer."""
+        for i, ln in enumerate(self.lanes[1:], 1):
+            self._join[i].record(ln)
+            self.stream.wait_event(self._join[i])
+
     # The per-call arguments depend only on (slot address, layer, projection),
     # so they are marshalled once and the C entry points are called directly.
 
@@ -183,9 +219,10 @@ class Stack:
         if a is None:
             p = self.proj[pi]
             base = self._base(addr, p)
+            lane = pi % self.n_lanes
             a = (ctypes.byref(base), self.x[l, pi].data_ptr(), self.T, self.A[l, pi].data_ptr(),
                  self.B[l, pi].data_ptr(), self.r, self.scale, self._out(self.y, l, pi).data_ptr(),
-                 self.ws.data_ptr(), self.ws_bytes, self.stream.cuda_stream, base)
+                 self.ws[lane].data_ptr(), self.ws_bytes, self.lanes[lane].cuda_stream, base)
             self._calls[key] = a
         return a
 
@@ -195,10 +232,11 @@ class Stack:
         if a is None:
             p = self.proj[pi]
             base = self._base(addr, p)
+            lane = (len(self.proj) - 1 - pi) % self.n_lanes
             a = (ctypes.byref(base), self.x[l, pi].data_ptr(), self.dY[l, pi].data_ptr(), self.T,
                  self.A[l, pi].data_ptr(), self.B[l, pi].data_ptr(), self.r, self.scale,
                  self._out(self.dX, l, pi).data_ptr(), self.dA[l, pi].data_ptr(), self.dB[l, pi].data_ptr(),
-                 int(accumulate), self.ws.data_ptr(), self.ws_bytes, self.stream.cuda_stream, base)
+                 int(accumulate), self.ws[lane].data_ptr(), self.ws_bytes, self.lanes[lane].cuda_stream, base)
             self._calls[key] = a
         return a
 
@@ -207,10 +245,12 @@ class Stack:
         for l in range(self.L):
             addr = self._acquire(l)
             self._prefetch(l + 1)
+            self._fork_lanes()
             for pi in range(len(self.proj)):
                 st = fwd(*self._fwd_args(addr, l, pi)[:-1])
                 if st:
                     lsnf4._check(st, "lora_linear_fwd")
+            self._join_lanes()
             self._release(l)
 
     def backward(self, accumulate: bool = False):
@@ -218,10 +258,12 @@ class Stack:
         for l in reversed(range(self.L)):
             addr = self._acquire(l)
             self._prefetch(l - 1)
+            self._fork_lanes()
             for pi in reversed(range(len(self.proj))):
                 st = bwd(*self._bwd_args(addr, l, pi, accumulate)[:-1])
                 if st:
                     lsnf4._check(st, "lora_linear_bwd")
+            self._join_lanes()
             self._release(l)
 
     def step(self, accumulate: bool = False):
@@ -240,4 +282,5 @@ class Stack:
         return lsnf4.layer_pool_stats(self.pool) if self.pool is not None else None
 
     def check_status(self):
-        lsnf4.ws_status(self.ws, self.stream)
+        for ws, ln in zip(self.ws, self.lanes):
+            lsnf4.ws_status(ws, ln)

@@ -24,11 +24,11 @@ def lib():
     return lsnf4
 
 
-def _run(cfg, layers, tokens, mode, fault=None, steps=1):
+def _run(cfg, layers, tokens, mode, fault=None, steps=1, lanes=2):
     import torch
     from layer_streamed_nf4_b200 import lsnf4
     from layer_streamed_nf4_b200.stack import Stack
-    st = Stack(cfg, layers=layers, tokens=tokens, mode=mode, keep_outputs=True)
+    st = Stack(cfg, layers=layers, tokens=tokens, mode=mode, keep_outputs=True, lanes=lanes)
     if fault is not None:
         lsnf4.layer_pool_inject_fault(st.pool, fault)
     for _ in range(steps):
@@ -60,8 +60,8 @@ def test_streamed_equals_resident(lib, name, layers, tokens, fused):
 
 def _streamed_equals_resident(lib, name, layers, tokens):
     cfg = synth.STACKS[name]
-    res = _run(cfg, layers, tokens, "resident")
-    stm = _run(cfg, layers, tokens, "streamed", steps=2)
+    res = _run(cfg, layers, tokens, "resident", lanes=1)     # every call on one stream
+    stm = _run(cfg, layers, tokens, "streamed", steps=2)     # projections spread over two streams
     fwd, bwd, bad = _compare(stm, res)
     assert fwd, f"{name}: streamed forward differs from resident"
     # two streamed steps without accumulation: gradients are those of one step
@@ -69,6 +69,19 @@ def _streamed_equals_resident(lib, name, layers, tokens):
     s = stm.pool_stats()
     assert s["copies"] == (2 * layers - 2) + (2 * layers - 4), s   # first step 2L-2, steady state 2L-4
     stm.close()
+
+
+@pytest.mark.parametrize("name,layers,tokens", [("0.5b", 4, 512), ("8b", 2, 1024)])
+def test_lane_count_does_not_change_results(lib, name, layers, tokens):
+    """The projections of a layer issued on 1, 2 or 3 streams give the same bits."""
+    cfg = synth.STACKS[name]
+    one = _run(cfg, layers, tokens, "no_h2d", lanes=1)
+    for lanes in (2, 3):
+        many = _run(cfg, layers, tokens, "no_h2d", lanes=lanes)
+        fwd, bwd, bad = _compare(many, one)
+        assert fwd and bwd, (lanes, bad)
+        many.close()
+    one.close()
 
 
 def test_no_h2d_equals_resident(lib):
