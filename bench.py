@@ -143,14 +143,18 @@ def run_ours(args):
     pool_stats = None
     clocks = None
     st_main = Stack(cfg, layers=L, tokens=T, mode="streamed", n_slots=args.slots, seed=synth.SEED + rank,
-                    stream=stream, lanes=args.lanes)
-    wanted = args.modes.split(",")
-    modes = ["streamed"] + [m for m in ("no_h2d", "resident", "serial") if m in wanted]
+                    stream=stream, lanes=args.lanes, api=args.api)
+    wanted = [m for m in args.modes.split(",") if m]
+    modes = ["streamed"] + [m for m in wanted if m in ("no_h2d", "resident", "proj") or m.startswith("streamed_T")]
+    mode_tokens = {m: T for m in modes}
     for mode in modes:
         if mode == "streamed":
             st = st_main
-        elif mode == "serial":          # no_h2d with every call on the compute stream
-            st = st_main.with_mode("no_h2d", lanes=1)
+        elif mode == "proj":            # no_h2d through the per-projection calls on two lanes
+            st = st_main.with_mode("no_h2d", lanes=2, api="proj")
+        elif mode.startswith("streamed_T"):   # the same stream of weights under a larger batch
+            mode_tokens[mode] = int(mode[len("streamed_T"):])
+            st = st_main.with_tokens(mode_tokens[mode], "streamed", n_slots=args.slots)
         else:
             st = st_main.with_mode(mode)
         with torch.cuda.stream(stream):
@@ -192,23 +196,30 @@ def run_ours(args):
             # without them.)  It runs with one lane, so that no launch waits
             # for SMs held by another lane's kernel inside its events.
             st_k = st.with_mode("streamed", n_slots=args.slots, lanes=1)
-            with torch.cuda.stream(stream):
-                st_k.step()
-            stream.synchronize()
-            barrier()
-            lsnf4.timing_enable(True)
-            with torch.cuda.stream(stream):
-                for _ in range(args.steps):
+            lanes_opt = lsnf4.get_option(lsnf4.LSN_OPT_LAYER_LANES)
+            lsnf4.set_option(lsnf4.LSN_OPT_LAYER_LANES, 1)
+            try:
+                with torch.cuda.stream(stream):
                     st_k.step()
-            stream.synchronize()
-            kernel = lsnf4.timing_read()
-            lsnf4.timing_enable(False)
+                stream.synchronize()
+                barrier()
+                lsnf4.timing_enable(True)
+                with torch.cuda.stream(stream):
+                    for _ in range(args.steps):
+                        st_k.step()
+                stream.synchronize()
+                kernel = lsnf4.timing_read()
+                lsnf4.timing_enable(False)
+            finally:
+                lsnf4.set_option(lsnf4.LSN_OPT_LAYER_LANES, lanes_opt)
             st_k.check_status()
             st_k.close()
             barrier()
         st.check_status()
         if st is not st_main:
             st.close()
+            st = None
+            torch.cuda.empty_cache()
 
     # End to end through the public API with host buffers: every step copies
     # its input hidden states (layer-0 projection inputs) from pinned host
@@ -269,8 +280,10 @@ def run_ours(args):
     h2d_gbs = (pool_stats["bytes_copied"] / (pool_stats["copy_ms"] / 1e3) / 1e9
                if pool_stats and pool_stats["copy_ms"] > 0 else None)
     extra_modes = {m: {"ms_per_step": results[m], "host_issue_ms_per_step": host_issue.get(m),
-                       "tok_s": world * T / (results[m] / 1e3),
-                       "pct_bf16_peak": 100 * flop_step / (results[m] / 1e3) / 1e12 / peaks["bf16_tflops"]}
+                       "tokens": mode_tokens[m],
+                       "tok_s": world * mode_tokens[m] / (results[m] / 1e3),
+                       "pct_bf16_peak": 100 * flop_step * mode_tokens[m] / T / (results[m] / 1e3) / 1e12
+                       / peaks["bf16_tflops"]}
                    for m in results}
     traffic = _traffic_from_profile()
     line = {
@@ -283,7 +296,8 @@ def run_ours(args):
                                f"{args.slots}-slot VRAM pool",
                    "tokens": T, "layers": L, "rank": cfg.rank, "pool_slots": args.slots, "base": cfg.base,
                    "parallelism": f"replicas x{world}",
-                   "lanes": args.lanes,
+                   "api": args.api,
+                   "lanes": args.lanes if args.api == "proj" else 1,
                    "nf4_conversion": "inside the GEMM" if args.fused_nf4 else "nf4_dequant then bf16 GEMM",
                    "l2": "inputs larger than L2 (per step ~11 GB of activations, ~3.6 GB of streamed weights)"},
         "pct_bf16_peak": 100 * flop_step / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
@@ -448,7 +462,10 @@ def main():
     ap.add_argument("--tokens", type=int, default=0, help="override T (default: the workload's 2048)")
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (default 32)")
     ap.add_argument("--slots", type=int, default=2)
-    ap.add_argument("--modes", default="no_h2d,resident,serial", help="extra modes timed after the streamed one")
+    ap.add_argument("--modes", default="no_h2d,resident,proj,streamed_T8192",
+                    help="extra modes timed after the streamed one (streamed_T<n>: streamed with n tokens)")
+    ap.add_argument("--api", choices=["layer", "proj"], default="layer",
+                    help="one library call per layer, or one per projection")
     ap.add_argument("--lanes", type=int, default=2, help="streams the seven projections of a layer are spread over")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

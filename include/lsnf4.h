@@ -197,6 +197,56 @@ lsn_status lora_linear_bwd(const lsn_base* W, const uint16_t* x, const uint16_t*
                            float* dA, float* dB, int accumulate, void* ws, size_t ws_bytes,
                            lsn_stream_t stream);
 
+/* ------------------------------------------------------- whole layer ---
+ *
+ * The LoRA linears of one decoder layer (q, k, v, o, gate, up, down, or any
+ * n <= LSN_LAYER_MAX_PROJ) in one call, in the order the layer loop meets
+ * them while the layer sits in its pool slot ("Can You Fine-Tune a 27B Model
+ * on a Laptop? (I Did the Math)", 7:11-7:42).  Every projection's outputs are
+ * bit for bit those of lora_linear_fwd / lora_linear_bwd on the same inputs;
+ * only the launches differ: the NF4 dequantisation of all projections is one
+ * kernel, their rank-r down projections one kernel, their dA/dB token
+ * reductions one kernel.  The forward can keep u = x A^T, the low-rank
+ * activation a LoRA layer saves for its backward pass, so the backward does
+ * not read x again to rebuild it.
+ *
+ * p is a HOST array of n descriptors, read during the call only; the
+ * pointers inside are device pointers that must stay valid until the
+ * enqueued work has finished.  Projections may have different K and N but
+ * share T, r and scale.  The outputs of different projections may not
+ * overlap each other or any input.
+ */
+#define LSN_LAYER_MAX_PROJ 16
+
+typedef struct {
+    lsn_base W;          /* frozen base [N, K] */
+    const uint16_t* x;   /* [T, K] input */
+    const uint16_t* A;   /* [r, K] */
+    const uint16_t* B;   /* [N, r] */
+    uint16_t* y;         /* forward: output [T, N]; unused by the backward */
+    const uint16_t* dY;  /* backward: output gradient [T, N]; unused by the forward */
+    uint16_t* dX;        /* backward: input gradient [T, K], or NULL */
+    float* dA;           /* backward: [r, K] fp32 */
+    float* dB;           /* backward: [N, r] fp32 */
+    float* u;            /* fp32 [T, r] = x A^T, or NULL.  Forward: written when non-NULL.
+                            Backward: read when non-NULL (it must hold what the forward
+                            wrote for the same x and A), recomputed when NULL. */
+} lsn_lora_proj;
+
+/* Workspace bytes of lora_layer_fwd / lora_layer_bwd for these projections
+ * (the larger of the two; 0 when an argument is invalid).  Like the
+ * single-linear workspace it must be zero-filled once when allocated.  With
+ * NF4 bases it holds the dequantised bf16 copy of every projection. */
+size_t lsn_layer_ws_bytes(int n, const lsn_lora_proj* p, int64_t T, int r);
+
+/* Forward of n projections: y_i = x_i W_i^T + s (x_i A_i^T) B_i^T. */
+lsn_status lora_layer_fwd(int n, const lsn_lora_proj* p, int64_t T, int r, float scale, void* ws,
+                          size_t ws_bytes, lsn_stream_t stream);
+
+/* Backward of n projections: dX_i, dA_i, dB_i as lora_linear_bwd. */
+lsn_status lora_layer_bwd(int n, const lsn_lora_proj* p, int64_t T, int r, float scale, int accumulate,
+                          void* ws, size_t ws_bytes, lsn_stream_t stream);
+
 /* Synchronise `stream`, then read the status word at the start of a LoRA
  * workspace: LSN_ERR_TIMEOUT if a tensor-core kernel gave up on a bounded
  * wait since the last check (the word is then cleared), LSN_OK otherwise.
@@ -242,8 +292,15 @@ lsn_status lsn_timing_read(lsn_kernel_timing* out);
  *                      inside the GEMM by converter warps (no bf16 copy of W);
  *                      0 (default): nf4_dequant into the workspace, then the
  *                      bf16 GEMM.  Narrow shapes always use the latter.
+ *   LSN_OPT_LAYER_LANES 2 (default): lora_layer_fwd / _bwd spread the work
+ *                      of different projections that does not depend on each
+ *                      other (their GEMMs; the backward's token reductions)
+ *                      over the caller's stream and a library-owned second
+ *                      stream of the same device, which forks from the
+ *                      caller's stream and joins it again within the call;
+ *                      1: everything on the caller's stream.
  */
-typedef enum { LSN_OPT_FUSED_NF4 = 1 } lsn_option;
+typedef enum { LSN_OPT_FUSED_NF4 = 1, LSN_OPT_LAYER_LANES = 2 } lsn_option;
 lsn_status lsn_set_option(int option, int value);
 int lsn_get_option(int option);
 

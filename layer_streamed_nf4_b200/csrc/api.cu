@@ -6,33 +6,16 @@
 #include <string>
 
 #include "common.cuh"
+#include "launch.cuh"
 #include "timing.cuh"
 
 namespace lsn {
 
-// Defined in codec.cu, gemm.cu and lora_small.cu.
-size_t quantize_ws_bytes(int64_t rows, int64_t cols);
-lsn_status launch_quantize(const float* W, const lsn_nf4_weight* out, void* ws, size_t ws_bytes, cudaStream_t st);
-lsn_status launch_dequant(const lsn_nf4_weight* w, uint16_t* out, cudaStream_t st);
-lsn_status launch_gemm(const uint16_t* A, int64_t lda, const uint16_t* B, int64_t ldb, bool b_mn, const uint16_t* LA,
-                       const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D, int64_t ldd,
-                       int* err, cudaStream_t st);
-lsn_status launch_lora_down(const uint16_t* X, const uint16_t* W, bool w_rk, int64_t T, int64_t Kd, int r,
-                            float scale, float* u32, uint16_t* u16, float* partial, int* counters, cudaStream_t st);
-size_t down_ws_bytes(int64_t T, int64_t Kd, int r);
-lsn_status launch_lora_tgrad(const float* G, const uint16_t* X, bool out_rk, int64_t T, int64_t Kd, int r,
-                             float scale, int accumulate, float* out, float* partial, int* counters, cudaStream_t st);
-size_t split_counter_count(int64_t T, int64_t K, int64_t N);
-size_t tgrad_ws_bytes(int64_t T, int64_t Kd, int r);
-lsn_status launch_gemm_nf4(const uint16_t* A, int64_t lda, const lsn_nf4_weight* w, bool b_mn, const uint16_t* LA,
-                           const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D, int64_t ldd,
-                           int* err, cudaStream_t st);
-bool gemm_use_pairs(int64_t M, int64_t N);
-int tgrad_splits(int64_t T, int64_t Kd);
 
 namespace {
 thread_local std::string g_last_error = "no error";
 std::atomic<int> g_fused_nf4{0};
+std::atomic<int> g_layer_lanes{2};
 }
 
 lsn_status fail(lsn_status st, const std::string& msg) {
@@ -134,9 +117,8 @@ LoraWs carve(void* ws, int64_t T, int64_t K, int64_t N, int r, int kind) {
     return w;
 }
 
-lsn_status check_lora(const lsn_base* W, const uint16_t* x, int64_t T, const uint16_t* A, const uint16_t* B, int r,
-                      void* ws, size_t ws_bytes, const char* who) {
-    const std::string f(who);
+lsn_status check_proj(const lsn_base* W, const uint16_t* x, int64_t T, const uint16_t* A, const uint16_t* B, int r,
+                      const std::string& f) {
     LSN_CHECK_ARG(W != nullptr, f + ": base is NULL");
     LSN_CHECK_ARG(W->kind == LSN_BASE_NF4 || W->kind == LSN_BASE_BF16, f + ": unknown base kind");
     LSN_CHECK_ARG(T >= 0, f + ": T must be >= 0");
@@ -146,7 +128,7 @@ lsn_status check_lora(const lsn_base* W, const uint16_t* x, int64_t T, const uin
                   f + ": dimension too large");
     LSN_CHECK_ARG(r >= 8 && r <= 64 && r % 8 == 0, f + ": rank must be a multiple of 8 in [8, 64]");
     if (W->kind == LSN_BASE_NF4) {
-        lsn_status s = check_nf4(&W->nf4, who);
+        lsn_status s = check_nf4(&W->nf4, f.c_str());
         if (s != LSN_OK) return s;
         LSN_CHECK_ARG(W->nf4.rows == W->rows && W->nf4.cols == W->cols, f + ": NF4 weight shape differs from the base shape");
     } else {
@@ -154,6 +136,14 @@ lsn_status check_lora(const lsn_base* W, const uint16_t* x, int64_t T, const uin
     }
     LSN_CHECK_ARG((x || T == 0) && A && B, f + ": NULL tensor");
     LSN_CHECK_ARG(aligned16(x) && aligned16(A) && aligned16(B), f + ": tensors must be 16-byte aligned");
+    return LSN_OK;
+}
+
+lsn_status check_lora(const lsn_base* W, const uint16_t* x, int64_t T, const uint16_t* A, const uint16_t* B, int r,
+                      void* ws, size_t ws_bytes, const char* who) {
+    const std::string f(who);
+    lsn_status s = check_proj(W, x, T, A, B, r, f);
+    if (s != LSN_OK) return s;
     LSN_CHECK_ARG(ws != nullptr && aligned16(ws), f + ": workspace must be a 16-byte aligned device pointer");
     const size_t need = carve(nullptr, T, W->cols, W->rows, r, W->kind).total;
     LSN_CHECK_ARG(ws_bytes >= need, f + ": workspace too small (need " + std::to_string(need) + " bytes)");
@@ -164,6 +154,152 @@ double dequant_bytes(int64_t N, int64_t K) {
     const double n = (double)N * (double)K;
     return n / 2.0 + n / 64.0 + 4.0 * (double)((N * K / 64 + 255) / 256) + 4.0 + 2.0 * n;
 }
+
+// Workspace of the layer calls: the status word, then per projection i
+//   s16 bf16 [T, r]  bf16(s u_i) (forward) or bf16(s g_i) (backward)
+//   g32 fp32 [T, r]  dY_i B_i
+//   u32 fp32 [T, r]  x_i A_i^T when the caller keeps no u
+//   w16 bf16 [N, K]  dequantised base (NF4 bases only)
+struct LayerWs {
+    int* err;
+    uint16_t* s16[LSN_LAYER_MAX_PROJ];
+    float* g32[LSN_LAYER_MAX_PROJ];
+    float* u32[LSN_LAYER_MAX_PROJ];
+    uint16_t* w16[LSN_LAYER_MAX_PROJ];
+    size_t total;
+};
+
+LayerWs carve_layer(void* ws, int n, const lsn_lora_proj* p, int64_t T, int r) {
+    LayerWs w{};
+    size_t off = 0;
+    char* b = reinterpret_cast<char*>(ws);
+    auto take = [&](size_t bytes) { char* q = b ? b + off : nullptr; off += round_up(bytes, 256); return q; };
+    w.err = reinterpret_cast<int*>(take(256));
+    for (int i = 0; i < n; ++i) {
+        w.s16[i] = reinterpret_cast<uint16_t*>(take((size_t)T * r * 2));
+        w.g32[i] = reinterpret_cast<float*>(take((size_t)T * r * 4));
+        w.u32[i] = reinterpret_cast<float*>(take((size_t)T * r * 4));
+        const bool nf4 = p[i].W.kind == LSN_BASE_NF4;
+        w.w16[i] = reinterpret_cast<uint16_t*>(take(nf4 ? (size_t)p[i].W.rows * p[i].W.cols * 2 : 0));
+    }
+    w.total = off;
+    return w;
+}
+
+lsn_status check_layer(int n, const lsn_lora_proj* p, int64_t T, int r, void* ws, size_t ws_bytes, bool bwd,
+                       const char* who) {
+    const std::string f(who);
+    LSN_CHECK_ARG(n >= 1 && n <= LSN_LAYER_MAX_PROJ, f + ": n must be in [1, LSN_LAYER_MAX_PROJ]");
+    LSN_CHECK_ARG(p != nullptr, f + ": projection array is NULL");
+    for (int i = 0; i < n; ++i) {
+        const std::string fi = f + ": projection " + std::to_string(i);
+        lsn_status s = check_proj(&p[i].W, p[i].x, T, p[i].A, p[i].B, r, fi);
+        if (s != LSN_OK) return s;
+        LSN_CHECK_ARG(aligned16(p[i].u), fi + ": u must be 16-byte aligned");
+        if (!bwd) {
+            LSN_CHECK_ARG((p[i].y != nullptr || T == 0) && aligned16(p[i].y), fi + ": y must be a 16-byte aligned device pointer");
+        } else {
+            LSN_CHECK_ARG((p[i].dY != nullptr || T == 0) && aligned16(p[i].dY), fi + ": dY must be a 16-byte aligned device pointer");
+            LSN_CHECK_ARG(p[i].dA && p[i].dB && aligned16(p[i].dA) && aligned16(p[i].dB),
+                          fi + ": dA/dB must be 16-byte aligned device pointers");
+            LSN_CHECK_ARG(aligned16(p[i].dX), fi + ": dX must be 16-byte aligned");
+        }
+    }
+    LSN_CHECK_ARG(ws != nullptr && aligned16(ws), f + ": workspace must be a 16-byte aligned device pointer");
+    const size_t need = carve_layer(nullptr, n, p, T, r).total;
+    LSN_CHECK_ARG(ws_bytes >= need, f + ": workspace too small (need " + std::to_string(need) + " bytes)");
+    return LSN_OK;
+}
+
+bool fused_here(const lsn_base& W, int64_t M, int64_t N) {
+    return W.kind == LSN_BASE_NF4 && g_fused_nf4.load() && gemm_use_pairs(M, N);
+}
+
+// Dequantise the NF4 bases of the listed projections into their workspace copies, one launch.
+lsn_status layer_dequant(int n, const lsn_lora_proj* p, const bool* want, const LayerWs& w, cudaStream_t st) {
+    const lsn_nf4_weight* ws[LSN_LAYER_MAX_PROJ];
+    uint16_t* outs[LSN_LAYER_MAX_PROJ];
+    int m = 0;
+    double bytes = 0.0;
+    for (int i = 0; i < n; ++i) {
+        if (!want[i]) continue;
+        ws[m] = &p[i].W.nf4;
+        outs[m++] = w.w16[i];
+        bytes += dequant_bytes(p[i].W.rows, p[i].W.cols);
+    }
+    if (m == 0) return LSN_OK;
+    TimingScope ts(LSN_K_DEQUANT, bytes, st);
+    return launch_dequant_batch(m, ws, outs, st);
+}
+
+lsn_status timed_down_batch(int n, const DownSpec* d, bool w_rk, int r, cudaStream_t st) {
+    if (n == 0) return LSN_OK;
+    double bytes = 0.0;
+    for (int i = 0; i < n; ++i)
+        bytes += 2.0 * d[i].T * d[i].Kd + 2.0 * r * d[i].Kd + (d[i].u32 ? 4.0 * d[i].T * r : 0.0) +
+                 (d[i].u16 ? 2.0 * d[i].T * r : 0.0);
+    TimingScope ts(LSN_K_LORA_DOWN, bytes, st, 1);
+    return launch_lora_down_batch(n, d, w_rk, r, st);
+}
+
+lsn_status timed_tgrad_batch(int n, const TgSpec* d, int r, cudaStream_t st) {
+    if (n == 0) return LSN_OK;
+    double bytes = 0.0;
+    for (int i = 0; i < n; ++i)
+        bytes += 2.0 * d[i].T * d[i].Kd + 4.0 * d[i].T * r + 4.0 * r * d[i].Kd * (d[i].accumulate ? 2.0 : 1.0);
+    TimingScope ts(LSN_K_LORA_TGRAD, bytes, st, 1);
+    return launch_lora_tgrad_batch(n, d, r, st);
+}
+
+// The second stream of the layer calls (one per device, created on first
+// use).  A call forks it from the caller's stream with an event, enqueues
+// independent work on both, and makes the caller's stream wait for it again
+// before returning.  The enqueue sequence of a call runs under `mu`, so calls
+// from several host threads cannot interleave their fork/join events.
+struct SideLane {
+    cudaStream_t side = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+std::mutex g_side_mu;
+SideLane g_side[64];
+
+class LaneScope {
+  public:
+    // Forks the side stream from `st` when two lanes are wanted; otherwise
+    // (or if the stream cannot be made) side() is `st` itself.
+    LaneScope(cudaStream_t st, bool want) : st_(st), lk_(g_side_mu) {
+        int dev = 0;
+        if (!want || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return;
+        SideLane& L = g_side[dev];
+        if (!L.side) {
+            if (cudaStreamCreateWithFlags(&L.side, cudaStreamNonBlocking) != cudaSuccess ||
+                cudaEventCreateWithFlags(&L.fork, cudaEventDisableTiming) != cudaSuccess ||
+                cudaEventCreateWithFlags(&L.join, cudaEventDisableTiming) != cudaSuccess) {
+                L = SideLane{};
+                return;
+            }
+        }
+        if (cudaEventRecord(L.fork, st) != cudaSuccess || cudaStreamWaitEvent(L.side, L.fork, 0) != cudaSuccess) return;
+        lane_ = &L;
+    }
+    cudaStream_t main() const { return st_; }
+    cudaStream_t side() const { return lane_ ? lane_->side : st_; }
+    // Join: the caller's stream waits for everything enqueued on the side stream.
+    lsn_status join() {
+        if (!lane_) return LSN_OK;
+        SideLane* L = lane_;
+        lane_ = nullptr;
+        LSN_CUDA_TRY(cudaEventRecord(L->join, L->side));
+        LSN_CUDA_TRY(cudaStreamWaitEvent(st_, L->join, 0));
+        return LSN_OK;
+    }
+    ~LaneScope() { join(); }
+
+  private:
+    cudaStream_t st_;
+    std::lock_guard<std::mutex> lk_;
+    SideLane* lane_ = nullptr;
+};
 
 lsn_status timed_dequant(const lsn_nf4_weight* w, uint16_t* out, cudaStream_t st) {
     TimingScope ts(LSN_K_DEQUANT, dequant_bytes(w->rows, w->cols), st);
@@ -310,7 +446,103 @@ lsn_status lora_linear_bwd(const lsn_base* W, const uint16_t* x, const uint16_t*
     return timed_tgrad(w.u32, dY, false, T, N, r, scale, accumulate, dB, w, st);
 }
 
+size_t lsn_layer_ws_bytes(int n, const lsn_lora_proj* p, int64_t T, int r) {
+    if (n < 1 || n > LSN_LAYER_MAX_PROJ || p == nullptr || T < 0 || r < 8 || r > 64 || r % 8 != 0) return 0;
+    for (int i = 0; i < n; ++i)
+        if (p[i].W.rows < 0 || p[i].W.cols < 0) return 0;
+    return carve_layer(nullptr, n, p, T, r).total;
+}
+
+lsn_status lora_layer_fwd(int n, const lsn_lora_proj* p, int64_t T, int r, float scale, void* ws, size_t ws_bytes,
+                          lsn_stream_t stream) {
+    lsn_status s = check_layer(n, p, T, r, ws, ws_bytes, false, "lora_layer_fwd");
+    if (s != LSN_OK) return s;
+    if (T == 0) return LSN_OK;
+    if ((s = check_device()) != LSN_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const LayerWs w = carve_layer(ws, n, p, T, r);
+    bool deq[LSN_LAYER_MAX_PROJ];
+    DownSpec dn[LSN_LAYER_MAX_PROJ];
+    for (int i = 0; i < n; ++i) {
+        deq[i] = p[i].W.kind == LSN_BASE_NF4 && !fused_here(p[i].W, T, p[i].W.rows);
+        dn[i] = DownSpec{p[i].x, p[i].A, p[i].u, w.s16[i], T, p[i].W.cols, scale};
+    }
+    if ((s = layer_dequant(n, p, deq, w, st)) != LSN_OK) return s;
+    if ((s = timed_down_batch(n, dn, true, r, st)) != LSN_OK) return s;
+    // The GEMMs of the projections are independent: alternate them over two lanes.
+    LaneScope lanes(st, n > 1 && g_layer_lanes.load() == 2);
+    for (int i = 0; i < n; ++i) {
+        const int64_t N = p[i].W.rows, K = p[i].W.cols;
+        const cudaStream_t gs = (i & 1) ? lanes.side() : lanes.main();
+        if (fused_here(p[i].W, T, N)) {
+            TimingScope ts(LSN_K_GEMM_FWD, 2.0 * T * N * (double)(K + r), gs);
+            s = launch_gemm_nf4(p[i].x, K, &p[i].W.nf4, false, w.s16[i], p[i].B, r, T, N, K, p[i].y, N, w.err, gs);
+        } else {
+            const uint16_t* Wb = p[i].W.kind == LSN_BASE_NF4 ? w.w16[i] : p[i].W.bf16;
+            s = timed_gemm(LSN_K_GEMM_FWD, p[i].x, K, Wb, K, false, w.s16[i], p[i].B, r, T, N, K, p[i].y, N, w.err, gs);
+        }
+        if (s != LSN_OK) return s;
+    }
+    return lanes.join();
+}
+
+lsn_status lora_layer_bwd(int n, const lsn_lora_proj* p, int64_t T, int r, float scale, int accumulate, void* ws,
+                          size_t ws_bytes, lsn_stream_t stream) {
+    lsn_status s = check_layer(n, p, T, r, ws, ws_bytes, true, "lora_layer_bwd");
+    if (s != LSN_OK) return s;
+    if ((s = check_device()) != LSN_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const LayerWs w = carve_layer(ws, n, p, T, r);
+    if (T > 0) {
+        bool deq[LSN_LAYER_MAX_PROJ];
+        DownSpec dg[LSN_LAYER_MAX_PROJ], du[LSN_LAYER_MAX_PROJ];
+        int nu = 0;
+        for (int i = 0; i < n; ++i) {
+            const int64_t N = p[i].W.rows, K = p[i].W.cols;
+            deq[i] = p[i].dX && p[i].W.kind == LSN_BASE_NF4 && !fused_here(p[i].W, T, K);
+            dg[i] = DownSpec{p[i].dY, p[i].B, w.g32[i], w.s16[i], T, N, scale};
+            if (!p[i].u) du[nu++] = DownSpec{p[i].x, p[i].A, w.u32[i], nullptr, T, K, scale};
+        }
+        if ((s = layer_dequant(n, p, deq, w, st)) != LSN_OK) return s;
+        if ((s = timed_down_batch(n, dg, false, r, st)) != LSN_OK) return s;
+        if ((s = timed_down_batch(nu, du, true, r, st)) != LSN_OK) return s;
+    }
+    // dA and dB of every projection in one launch (with T == 0: zeros, or the
+    // accumulators left as they are).  They need only g and u, so with two
+    // lanes they run on the side stream beside the input-gradient GEMMs.
+    TgSpec tg[2 * LSN_LAYER_MAX_PROJ];
+    for (int i = 0; i < n; ++i) {
+        const int64_t N = p[i].W.rows, K = p[i].W.cols;
+        tg[2 * i] = TgSpec{w.g32[i], p[i].x, p[i].dA, T, K, true, accumulate, scale};
+        tg[2 * i + 1] = TgSpec{p[i].u ? p[i].u : w.u32[i], p[i].dY, p[i].dB, T, N, false, accumulate, scale};
+    }
+    LaneScope lanes(st, T > 0 && g_layer_lanes.load() == 2);
+    if ((s = timed_tgrad_batch(2 * n, tg, r, lanes.side())) != LSN_OK) return s;
+    if (T > 0) {
+        for (int i = 0, j = 0; i < n; ++i) {
+            if (!p[i].dX) continue;
+            const int64_t N = p[i].W.rows, K = p[i].W.cols;
+            const cudaStream_t gs = (j++ & 1) ? lanes.side() : lanes.main();
+            if (fused_here(p[i].W, T, K)) {
+                TimingScope ts(LSN_K_GEMM_BWD, 2.0 * T * K * (double)(N + r), gs);
+                s = launch_gemm_nf4(p[i].dY, N, &p[i].W.nf4, true, w.s16[i], p[i].A, r, T, K, N, p[i].dX, K, w.err, gs);
+            } else {
+                const uint16_t* Wb = p[i].W.kind == LSN_BASE_NF4 ? w.w16[i] : p[i].W.bf16;
+                s = timed_gemm(LSN_K_GEMM_BWD, p[i].dY, N, Wb, K, true, w.s16[i], p[i].A, r, T, K, N, p[i].dX, K,
+                               w.err, gs);
+            }
+            if (s != LSN_OK) return s;
+        }
+    }
+    return lanes.join();
+}
+
 lsn_status lsn_set_option(int option, int value) {
+    if (option == LSN_OPT_LAYER_LANES) {
+        LSN_CHECK_ARG(value == 1 || value == 2, "lsn_set_option: LSN_OPT_LAYER_LANES takes 1 or 2");
+        g_layer_lanes.store(value);
+        return LSN_OK;
+    }
     if (option == LSN_OPT_FUSED_NF4) {
         g_fused_nf4.store(value != 0 ? 1 : 0);
         return LSN_OK;
@@ -318,7 +550,11 @@ lsn_status lsn_set_option(int option, int value) {
     return fail(LSN_ERR_INVALID_ARG, "lsn_set_option: unknown option");
 }
 
-int lsn_get_option(int option) { return option == LSN_OPT_FUSED_NF4 ? g_fused_nf4.load() : -1; }
+int lsn_get_option(int option) {
+    if (option == LSN_OPT_FUSED_NF4) return g_fused_nf4.load();
+    if (option == LSN_OPT_LAYER_LANES) return g_layer_lanes.load();
+    return -1;
+}
 
 lsn_status lsn_ws_status(void* ws, lsn_stream_t stream) {
     LSN_CHECK_ARG(ws != nullptr, "lsn_ws_status: workspace is NULL");

@@ -20,6 +20,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "launch.cuh"
 
 namespace lsn {
 
@@ -187,52 +188,80 @@ __global__ void __launch_bounds__(256) dq_codes_kernel(const float* __restrict__
 // lane (512 B per warp), both contiguous across the warp.
 struct DequantParams { float level[16]; float dq[256]; };
 
-__global__ void __launch_bounds__(256) nf4_dequant_kernel(const uint32_t* __restrict__ packed,
-                                                           const uint8_t* __restrict__ absmax_q,
-                                                           const float* __restrict__ s2,
-                                                           const float* __restrict__ offset, int64_t nwords,
-                                                           uint4* __restrict__ out, DequantParams P) {
+// One NF4 weight of a dequantisation batch, counted in 16-byte vectors of
+// packed codes (32 elements, half of a 64-element absmax block).
+struct DqItem {
+    const uint4* packed;
+    const uint8_t* absmax_q;
+    const float* s2;
+    const float* offset;
+    uint4* out;          // bf16 output, 64 bytes per vector
+    int64_t nvec;
+    int64_t first;       // first blockIdx.x of the item
+};
+constexpr int kDqMax = 16;
+constexpr int kDqThreads = 256;
+constexpr int kDqUnroll = 4;                       // vectors per thread
+constexpr int kDqVecPerBlock = kDqThreads * kDqUnroll;
+struct DqBatch {
+    int n;
+    DqItem it[kDqMax];
+};
+
+// Standalone dequantisation of a batch of weights: each thread reads 128-bit
+// words of packed codes (coalesced across the warp, four words in flight),
+// looks up the 16 levels in shared memory, scales them by the block's
+// reconstructed absmax and writes 64 bytes of bf16.  A block covers 1024
+// consecutive vectors of one weight.
+__global__ void __launch_bounds__(kDqThreads) nf4_dequant_kernel(const __grid_constant__ DqBatch bt,
+                                                                 const __grid_constant__ DequantParams P) {
     __shared__ float lv[16];
     __shared__ float dq[256];
     for (int i = threadIdx.x; i < 256; i += blockDim.x) dq[i] = P.dq[i];
     if (threadIdx.x < 16) lv[threadIdx.x] = P.level[threadIdx.x];
-    __syncthreads();
-    const float off = *offset;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    // Four independent words in flight per thread.
-    for (; w + 3 * stride < nwords; w += 4 * stride) {
-        uint32_t p[4];
-        float ah[4];
+    int ii = 0;
+    while (ii + 1 < bt.n && (int64_t)blockIdx.x >= bt.it[ii + 1].first) ++ii;
+    const DqItem& it = bt.it[ii];
+    const uint4* __restrict__ packed = it.packed;
+    const uint8_t* __restrict__ absmax_q = it.absmax_q;
+    const float* __restrict__ s2 = it.s2;
+    uint4* __restrict__ out = it.out;
+    const float off = *it.offset;
+    const int64_t v0 = ((int64_t)blockIdx.x - it.first) * kDqVecPerBlock + threadIdx.x;
+    uint4 p[kDqUnroll];
+    float ah[kDqUnroll];
+    #pragma unroll
+    for (int u = 0; u < kDqUnroll; ++u) {
+        const int64_t v = v0 + u * kDqThreads;
+        p[u] = v < it.nvec ? __ldg(packed + v) : make_uint4(0, 0, 0, 0);
+    }
+    uint32_t code[kDqUnroll];
+    float sc[kDqUnroll];
+    #pragma unroll
+    for (int u = 0; u < kDqUnroll; ++u) {
+        const int64_t v = v0 + u * kDqThreads;
+        const int64_t b = (v < it.nvec ? v : 0) >> 1;   // absmax block of the vector
+        code[u] = __ldg(absmax_q + b);
+        sc[u] = __ldg(s2 + (b >> 8));
+    }
+    __syncthreads();                                     // level and code tables are in shared memory
+    #pragma unroll
+    for (int u = 0; u < kDqUnroll; ++u) ah[u] = __fadd_rn(__fmul_rn(dq[code[u]], sc[u]), off);
+    #pragma unroll
+    for (int u = 0; u < kDqUnroll; ++u) {
+        const int64_t v = v0 + u * kDqThreads;
+        if (v >= it.nvec) break;
+        const uint32_t w[4] = {p[u].x, p[u].y, p[u].z, p[u].w};
         #pragma unroll
-        for (int u = 0; u < 4; ++u) p[u] = __ldg(packed + w + u * stride);
-        #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int64_t b = (w + u * stride) >> 3;
-            ah[u] = __fadd_rn(__fmul_rn(dq[__ldg(absmax_q + b)], __ldg(s2 + (b >> 8))), off);
-        }
-        #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int h = 0; h < 4; ++h) {
             uint32_t r[4];
             #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const uint32_t byte = (p[u] >> (8 * j)) & 0xffu;
+                const uint32_t byte = (w[h] >> (8 * j)) & 0xffu;
                 r[j] = pack_bf16x2(__fmul_rn(lv[byte >> 4], ah[u]), __fmul_rn(lv[byte & 15u], ah[u]));
             }
-            out[w + u * stride] = make_uint4(r[0], r[1], r[2], r[3]);
+            out[v * 4 + h] = make_uint4(r[0], r[1], r[2], r[3]);
         }
-    }
-    for (; w < nwords; w += stride) {
-        const uint32_t p = __ldg(packed + w);
-        const int64_t b = w >> 3;
-        const float a = __fadd_rn(__fmul_rn(dq[__ldg(absmax_q + b)], __ldg(s2 + (b >> 8))), off);
-        uint32_t r[4];
-        #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const uint32_t byte = (p >> (8 * j)) & 0xffu;
-            r[j] = pack_bf16x2(__fmul_rn(lv[byte >> 4], a), __fmul_rn(lv[byte & 15u], a));
-        }
-        out[w] = make_uint4(r[0], r[1], r[2], r[3]);
     }
 }
 
@@ -277,18 +306,43 @@ lsn_status launch_quantize(const float* W, const lsn_nf4_weight* out, void* ws, 
     return LSN_OK;
 }
 
-lsn_status launch_dequant(const lsn_nf4_weight* w, uint16_t* out, cudaStream_t st) {
-    const int64_t nwords = w->rows * w->cols / 8;
+lsn_status launch_dequant_batch(int n, const lsn_nf4_weight* const* w, uint16_t* const* out, cudaStream_t st) {
     const Nf4Tables& T = nf4_tables();
     DequantParams P;
     std::memcpy(P.level, T.level, sizeof(P.level));
     std::memcpy(P.dq, T.dq, sizeof(P.dq));
-    // Enough threads for four words each on every SM, several blocks per SM.
-    const int grid = grid_for(ceil_div(nwords, 4), 256, 8);
-    nf4_dequant_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint32_t*>(w->packed), w->absmax_q,
-                                             w->absmax_s2, w->offset, nwords, reinterpret_cast<uint4*>(out), P);
-    LSN_CUDA_TRY(cudaGetLastError());
-    return LSN_OK;
+    DqBatch bt{};
+    int64_t blocks = 0;
+    auto flush = [&]() -> lsn_status {
+        if (bt.n == 0) return LSN_OK;
+        nf4_dequant_kernel<<<(unsigned)blocks, kDqThreads, 0, st>>>(bt, P);
+        LSN_CUDA_TRY(cudaGetLastError());
+        bt = DqBatch{};
+        blocks = 0;
+        return LSN_OK;
+    };
+    for (int i = 0; i < n; ++i) {
+        const int64_t nvec = w[i]->rows * w[i]->cols / 32;
+        if (nvec == 0) continue;
+        if (bt.n == kDqMax) {
+            const lsn_status s = flush();
+            if (s != LSN_OK) return s;
+        }
+        DqItem& it = bt.it[bt.n++];
+        it.packed = reinterpret_cast<const uint4*>(w[i]->packed);
+        it.absmax_q = w[i]->absmax_q;
+        it.s2 = w[i]->absmax_s2;
+        it.offset = w[i]->offset;
+        it.out = reinterpret_cast<uint4*>(out[i]);
+        it.nvec = nvec;
+        it.first = blocks;
+        blocks += ceil_div(nvec, (int64_t)kDqVecPerBlock);
+    }
+    return flush();
+}
+
+lsn_status launch_dequant(const lsn_nf4_weight* w, uint16_t* out, cudaStream_t st) {
+    return launch_dequant_batch(1, &w, &out, st);
 }
 
 }  // namespace lsn

@@ -1,0 +1,59 @@
+// Host-side launchers of the library's kernels (defined in codec.cu, gemm.cu
+// and lora_small.cu), called by the C entry points in api.cu.
+#pragma once
+
+#include "common.cuh"
+
+namespace lsn {
+
+// One rank-r down projection: out[t, j] = sum_k X[t, k] W(j, k) for j < r,
+// W either A [r, Kd] or B [Kd, r]; written as fp32 (u32) and/or as
+// bf16(scale * out) (u16), either may be NULL.
+struct DownSpec {
+    const uint16_t* X;
+    const uint16_t* W;
+    float* u32;
+    uint16_t* u16;
+    int64_t T, Kd;
+    float scale;
+};
+
+// One token reduction: R[j, k] = sum_t G[t, j] X[t, k], written (or, with
+// accumulate, added) as scale * R into out, [r, Kd] when out_rk else [Kd, r].
+struct TgSpec {
+    const float* G;
+    const uint16_t* X;
+    float* out;
+    int64_t T, Kd;
+    bool out_rk;
+    int accumulate;
+    float scale;
+};
+
+size_t quantize_ws_bytes(int64_t rows, int64_t cols);
+lsn_status launch_quantize(const float* W, const lsn_nf4_weight* out, void* ws, size_t ws_bytes, cudaStream_t st);
+lsn_status launch_dequant(const lsn_nf4_weight* w, uint16_t* out, cudaStream_t st);
+// Several NF4 weights dequantised by one launch (at most 16 per launch; more take several).
+lsn_status launch_dequant_batch(int n, const lsn_nf4_weight* const* w, uint16_t* const* out, cudaStream_t st);
+
+lsn_status launch_gemm(const uint16_t* A, int64_t lda, const uint16_t* B, int64_t ldb, bool b_mn, const uint16_t* LA,
+                       const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D, int64_t ldd,
+                       int* err, cudaStream_t st);
+lsn_status launch_gemm_nf4(const uint16_t* A, int64_t lda, const lsn_nf4_weight* w, bool b_mn, const uint16_t* LA,
+                           const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D, int64_t ldd,
+                           int* err, cudaStream_t st);
+bool gemm_use_pairs(int64_t M, int64_t N);
+
+lsn_status launch_lora_down(const uint16_t* X, const uint16_t* W, bool w_rk, int64_t T, int64_t Kd, int r,
+                            float scale, float* u32, uint16_t* u16, float* partial, int* counters, cudaStream_t st);
+lsn_status launch_lora_down_batch(int n, const DownSpec* specs, bool w_rk, int r, cudaStream_t st);
+lsn_status launch_lora_tgrad(const float* G, const uint16_t* X, bool out_rk, int64_t T, int64_t Kd, int r,
+                             float scale, int accumulate, float* out, float* partial, int* counters, cudaStream_t st);
+lsn_status launch_lora_tgrad_batch(int n, const TgSpec* specs, int r, cudaStream_t st);
+size_t down_ws_bytes(int64_t T, int64_t Kd, int r);
+size_t tgrad_ws_bytes(int64_t T, int64_t Kd, int r);
+size_t split_counter_count(int64_t T, int64_t K, int64_t N);
+int down_splits(int64_t T, int64_t Kd);
+int tgrad_splits(int64_t T, int64_t Kd);
+
+}  // namespace lsn

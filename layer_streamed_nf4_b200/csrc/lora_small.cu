@@ -9,6 +9,7 @@
 // HBM read of the activation (x or dY); every sum runs in a fixed order that
 // depends on the shape only, so results are bitwise reproducible.
 #include "common.cuh"
+#include "launch.cuh"
 
 namespace lsn {
 
@@ -65,9 +66,10 @@ __device__ __forceinline__ float ld_dsmem_f32(const float* local_ptr, uint32_t r
 // A [r, Kd] (u = x A^T) or as B [Kd, r] (g = dY B).  A CTA owns 64 token rows
 // and one split of the K range; 64-wide K chunks of X and W are staged in
 // shared memory by cp.async through a 3-stage ring (16-byte chunks XOR-
-// swizzled by row, so ldmatrix is conflict-free without padding), and each warp multiplies its 16 rows with W on the
-// warp-level tensor-core instruction (mma.sync m16n8k16, bf16 in, fp32
-// accumulate; the inputs are exact bf16 values).  W in the B layout is read
+// swizzled by row, so ldmatrix is conflict-free without padding), and each
+// warp multiplies its 16 rows with W on the warp-level tensor-core
+// instruction (mma.sync m16n8k16, bf16 in, fp32 accumulate; the inputs are
+// exact bf16 values).  W in the B layout is read
 // with ldmatrix.trans, so no transposed copy is made.  The big contractions
 // use tcgen05; this skinny one is bound by the HBM read of X.
 //
@@ -75,9 +77,31 @@ __device__ __forceinline__ float ld_dsmem_f32(const float* local_ptr, uint32_t r
 // with a running GEMM CTA (about 194 KB), so the side work of one
 // projection can proceed underneath another projection's GEMM when the
 // caller issues them on two streams.
+//
+// One launch serves a batch of up to kMaxProbs problems of the same rank and
+// W layout (the projections of a layer): blockIdx.x runs over the row blocks
+// of all problems, blockIdx.y is the split, and a problem with fewer splits
+// than the launch leaves its extra CTAs without work.  Each problem keeps
+// the split count and summation order it has when launched alone.
 constexpr int kDnWarps = 4;
 constexpr int kDnRows = 16 * kDnWarps;       // token rows per CTA
 constexpr int kDnStages = 3;
+constexpr int kMaxProbs = 16;
+
+struct DownProb {
+    const uint16_t* X;   // [T, Kd]
+    const uint16_t* W;   // A [r, Kd] or B [Kd, r]
+    float* u32;          // [T, r] fp32, or NULL
+    uint16_t* u16;       // [T, r] bf16(scale * .), or NULL
+    int64_t T, Kd;
+    int cps, ns;         // 64-wide K chunks per split, splits
+    int first;           // first blockIdx.x of the problem
+    float scale;
+};
+struct DownBatch {
+    int n;
+    DownProb p[kMaxProbs];
+};
 
 // Offset (in bf16) of element (row, col) of a staged tile whose rows hold
 // `pitch` bf16, with the 16-byte chunk index XOR-ed by `swz`.
@@ -108,11 +132,18 @@ struct DownSmem {
 };
 
 template <int NT, bool B_KR>
-__global__ void __launch_bounds__(128) lora_down_kernel(const uint16_t* __restrict__ X, const uint16_t* __restrict__ W,
-                                                        int64_t T, int64_t Kd, int chunks_per_split, int nsplit,
-                                                        float scale, float* __restrict__ u32,
-                                                        uint16_t* __restrict__ u16) {
+__global__ void __launch_bounds__(128) lora_down_kernel(const __grid_constant__ DownBatch bt) {
     using L = DownSmem<NT, B_KR>;
+    int pi = 0;
+    while (pi + 1 < bt.n && (int)blockIdx.x >= bt.p[pi + 1].first) ++pi;
+    const DownProb& pb = bt.p[pi];
+    const uint16_t* __restrict__ X = pb.X;
+    const uint16_t* __restrict__ W = pb.W;
+    float* __restrict__ u32 = pb.u32;
+    uint16_t* __restrict__ u16 = pb.u16;
+    const int64_t T = pb.T, Kd = pb.Kd;
+    const int chunks_per_split = pb.cps, nsplit = pb.ns;
+    const float scale = pb.scale;
     constexpr int R = L::R, NP = L::NP, WROWS = L::WROWS, WPITCH = L::WPITCH;
     extern __shared__ __align__(128) uint8_t dn_smem[];
     uint16_t* xs = reinterpret_cast<uint16_t*>(dn_smem);                 // [stage][64 rows][64], swizzled
@@ -122,7 +153,7 @@ __global__ void __launch_bounds__(128) lora_down_kernel(const uint16_t* __restri
         return smem_u32(ws + st * L::W_TILE + swz_off(row, col, WPITCH, L::wswz(row)));
     };
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t row_base = (int64_t)blockIdx.x * kDnRows;
+    const int64_t row_base = (int64_t)((int)blockIdx.x - pb.first) * kDnRows;
     const int64_t nchunks = Kd / 64;
     const int64_t c_begin = (int64_t)blockIdx.y * chunks_per_split;
     const int64_t c_end = (c_begin + chunks_per_split < nchunks) ? c_begin + chunks_per_split : nchunks;
@@ -199,7 +230,8 @@ __global__ void __launch_bounds__(128) lora_down_kernel(const uint16_t* __restri
         if (u32) u32[row * R + j] = v;
         if (u16) u16[row * R + j] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(scale, v)));
     };
-    if (nsplit == 1) {
+    if (nsplit == 1) {                  // every CTA of the cluster takes this branch
+        if (blockIdx.y != 0) return;
         #pragma unroll
         for (int n = 0; n < NT; ++n) {
             const int j = n * 8 + 2 * q;
@@ -245,9 +277,26 @@ __global__ void __launch_bounds__(128) lora_down_kernel(const uint16_t* __restri
 // token split; the splits of a column tile form one thread-block cluster and
 // are added in split order through distributed shared memory.  At r = 16 the
 // ring takes 31.5 KB, small enough to share an SM with a running GEMM CTA.
+// Batched like the down projection: blockIdx.x runs over the column tiles of
+// all problems (dA and dB of several projections), blockIdx.y is the token
+// split.
 constexpr int kTgCols = 128;
 constexpr int kTgTok = 32;          // tokens per staged tile (two MMA k-steps)
 constexpr int kTgStages = 3;
+
+struct TgProb {
+    const float* G;      // [T, r] fp32
+    const uint16_t* X;   // [T, Kd]
+    float* out;          // [r, Kd] when out_rk, else [Kd, r]
+    int64_t T, Kd, per;  // tokens, columns, tokens per split
+    int ns, first;       // splits, first blockIdx.x of the problem
+    int out_rk, accumulate;
+    float scale;
+};
+struct TgBatch {
+    int n;
+    TgProb p[kMaxProbs];
+};
 
 template <int NT>
 struct TgSmem {
@@ -260,11 +309,19 @@ struct TgSmem {
     static constexpr size_t BYTES = RING > RED ? RING : RED;
 };
 
-template <int NT, bool OUT_RK>
-__global__ void __launch_bounds__(128) lora_tgrad_kernel(const float* __restrict__ G, const uint16_t* __restrict__ X,
-                                                         int64_t T, int64_t Kd, int64_t per_split, int nsplit,
-                                                         float scale, int accumulate, float* __restrict__ out) {
+template <int NT>
+__global__ void __launch_bounds__(128) lora_tgrad_kernel(const __grid_constant__ TgBatch bt) {
     using L = TgSmem<NT>;
+    int pi = 0;
+    while (pi + 1 < bt.n && (int)blockIdx.x >= bt.p[pi + 1].first) ++pi;
+    const TgProb& pb = bt.p[pi];
+    const float* __restrict__ G = pb.G;
+    const uint16_t* __restrict__ X = pb.X;
+    float* __restrict__ out = pb.out;
+    const int64_t T = pb.T, Kd = pb.Kd, per_split = pb.per;
+    const int nsplit = pb.ns, accumulate = pb.accumulate;
+    const bool out_rk = pb.out_rk != 0;
+    const float scale = pb.scale;
     constexpr int R = 8 * NT, GPITCH = L::GPITCH;
     extern __shared__ __align__(128) uint8_t tg_smem[];
     uint16_t* xs = reinterpret_cast<uint16_t*>(tg_smem);                 // [stage][32 tokens][128], swizzled
@@ -273,7 +330,7 @@ __global__ void __launch_bounds__(128) lora_tgrad_kernel(const float* __restrict
     };
     auto gs = reinterpret_cast<float (*)[kTgTok][GPITCH]>(tg_smem + L::X_BYTES);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t k0 = (int64_t)blockIdx.x * kTgCols;
+    const int64_t k0 = (int64_t)((int)blockIdx.x - pb.first) * kTgCols;
     const int64_t tb = (int64_t)blockIdx.y * per_split;
     const int64_t te = (tb + per_split < T) ? tb + per_split : T;
     const int64_t ntiles = te > tb ? (te - tb + kTgTok - 1) / kTgTok : 0;
@@ -348,13 +405,14 @@ __global__ void __launch_bounds__(128) lora_tgrad_kernel(const float* __restrict
     cp_async_wait<0>();
 
     // acc[m][n] = { (k = base+g, j = 8n+2q), (k, j+1), (k+8, j), (k+8, j+1) }, base = k0 + 32 warp + 16 m
-    auto out_index = [&](int64_t k, int j) -> int64_t { return OUT_RK ? (int64_t)j * Kd + k : k * R + j; };
+    auto out_index = [&](int64_t k, int j) -> int64_t { return out_rk ? (int64_t)j * Kd + k : k * R + j; };
     auto finish = [&](int64_t k, int j, float v) {
         const int64_t o = out_index(k, j);
         const float w = __fmul_rn(scale, v);
         out[o] = accumulate ? __fadd_rn(out[o], w) : w;
     };
-    if (nsplit == 1) {
+    if (nsplit == 1) {                  // every CTA of the cluster takes this branch
+        if (blockIdx.y != 0) return;
         #pragma unroll
         for (int m = 0; m < 2; ++m)
             #pragma unroll
@@ -423,54 +481,48 @@ cudaError_t launch_split(Kern kernel, dim3 grid, size_t smem, cudaStream_t st, A
 }
 
 template <int NT, bool B_KR>
-lsn_status launch_down_nt(dim3 grid, cudaStream_t st, const uint16_t* X, const uint16_t* W, int64_t T, int64_t Kd,
-                          int cps, int ns, float scale, float* u32, uint16_t* u16) {
+lsn_status launch_down_nt(dim3 grid, cudaStream_t st, const DownBatch& bt) {
     constexpr size_t bytes = DownSmem<NT, B_KR>::BYTES;
     static const cudaError_t attr = allow_smem(lora_down_kernel<NT, B_KR>, bytes);
     if (attr != cudaSuccess) return fail_cuda(attr, "cudaFuncSetAttribute(lora_down smem)");
-    LSN_CUDA_TRY(launch_split(lora_down_kernel<NT, B_KR>, grid, bytes, st, X, W, T, Kd, cps, ns, scale, u32, u16));
+    LSN_CUDA_TRY(launch_split(lora_down_kernel<NT, B_KR>, grid, bytes, st, bt));
     return LSN_OK;
 }
 
-template <int NT, bool OUT_RK>
-lsn_status launch_tgrad_nt(dim3 grid, cudaStream_t st, const float* G, const uint16_t* X, int64_t T, int64_t Kd,
-                           int64_t per, int ns, float scale, int accumulate, float* out) {
+template <int NT>
+lsn_status launch_tgrad_nt(dim3 grid, cudaStream_t st, const TgBatch& bt) {
     constexpr size_t bytes = TgSmem<NT>::BYTES;
-    static const cudaError_t attr = allow_smem(lora_tgrad_kernel<NT, OUT_RK>, bytes);
+    static const cudaError_t attr = allow_smem(lora_tgrad_kernel<NT>, bytes);
     if (attr != cudaSuccess) return fail_cuda(attr, "cudaFuncSetAttribute(lora_tgrad smem)");
-    LSN_CUDA_TRY(launch_split(lora_tgrad_kernel<NT, OUT_RK>, grid, bytes, st, G, X, T, Kd, per, ns, scale, accumulate,
-                              out));
+    LSN_CUDA_TRY(launch_split(lora_tgrad_kernel<NT>, grid, bytes, st, bt));
     return LSN_OK;
 }
 
 template <bool B_KR>
-lsn_status dispatch_down(int r, dim3 grid, cudaStream_t st, const uint16_t* X, const uint16_t* W, int64_t T,
-                         int64_t Kd, int cps, int ns, float scale, float* u32, uint16_t* u16) {
+lsn_status dispatch_down(int r, dim3 grid, cudaStream_t st, const DownBatch& bt) {
     switch (r / 8) {
-        case 1: return launch_down_nt<1, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16);
-        case 2: return launch_down_nt<2, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16);
-        case 3: return launch_down_nt<3, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16);
-        case 4: return launch_down_nt<4, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16);
-        case 5: return launch_down_nt<5, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16);
-        case 6: return launch_down_nt<6, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16);
-        case 7: return launch_down_nt<7, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16);
-        case 8: return launch_down_nt<8, B_KR>(grid, st, X, W, T, Kd, cps, ns, scale, u32, u16);
+        case 1: return launch_down_nt<1, B_KR>(grid, st, bt);
+        case 2: return launch_down_nt<2, B_KR>(grid, st, bt);
+        case 3: return launch_down_nt<3, B_KR>(grid, st, bt);
+        case 4: return launch_down_nt<4, B_KR>(grid, st, bt);
+        case 5: return launch_down_nt<5, B_KR>(grid, st, bt);
+        case 6: return launch_down_nt<6, B_KR>(grid, st, bt);
+        case 7: return launch_down_nt<7, B_KR>(grid, st, bt);
+        case 8: return launch_down_nt<8, B_KR>(grid, st, bt);
         default: return fail(LSN_ERR_INVALID_ARG, "rank must be a multiple of 8 in [8, 64]");
     }
 }
 
-template <bool OUT_RK>
-lsn_status dispatch_tgrad(int r, dim3 grid, cudaStream_t st, const float* G, const uint16_t* X, int64_t T, int64_t Kd,
-                          int64_t per, int ns, float scale, int accumulate, float* out) {
+lsn_status dispatch_tgrad(int r, dim3 grid, cudaStream_t st, const TgBatch& bt) {
     switch (r / 8) {
-        case 1: return launch_tgrad_nt<1, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out);
-        case 2: return launch_tgrad_nt<2, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out);
-        case 3: return launch_tgrad_nt<3, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out);
-        case 4: return launch_tgrad_nt<4, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out);
-        case 5: return launch_tgrad_nt<5, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out);
-        case 6: return launch_tgrad_nt<6, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out);
-        case 7: return launch_tgrad_nt<7, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out);
-        case 8: return launch_tgrad_nt<8, OUT_RK>(grid, st, G, X, T, Kd, per, ns, scale, accumulate, out);
+        case 1: return launch_tgrad_nt<1>(grid, st, bt);
+        case 2: return launch_tgrad_nt<2>(grid, st, bt);
+        case 3: return launch_tgrad_nt<3>(grid, st, bt);
+        case 4: return launch_tgrad_nt<4>(grid, st, bt);
+        case 5: return launch_tgrad_nt<5>(grid, st, bt);
+        case 6: return launch_tgrad_nt<6>(grid, st, bt);
+        case 7: return launch_tgrad_nt<7>(grid, st, bt);
+        case 8: return launch_tgrad_nt<8>(grid, st, bt);
         default: return fail(LSN_ERR_INVALID_ARG, "rank must be a multiple of 8 in [8, 64]");
     }
 }
@@ -515,25 +567,93 @@ size_t tgrad_ws_bytes(int64_t, int64_t, int) { return 0; }
 
 size_t split_counter_count(int64_t, int64_t, int64_t) { return 0; }
 
+// Down projections of a batch of problems, all with W in the same layout
+// (w_rk: A [r, Kd]; otherwise B [Kd, r]) and the same rank.  Problems with
+// T == 0 are skipped; more than kMaxProbs problems take several launches.
+lsn_status launch_lora_down_batch(int n, const DownSpec* specs, bool w_rk, int r, cudaStream_t st) {
+    DownBatch bt{};
+    int blocks = 0, smax = 1;
+    auto flush = [&]() -> lsn_status {
+        if (bt.n == 0) return LSN_OK;
+        dim3 grid((unsigned)blocks, (unsigned)smax);
+        const lsn_status s = w_rk ? dispatch_down<false>(r, grid, st, bt) : dispatch_down<true>(r, grid, st, bt);
+        bt = DownBatch{};
+        blocks = 0;
+        smax = 1;
+        return s;
+    };
+    for (int i = 0; i < n; ++i) {
+        const DownSpec& d = specs[i];
+        if (d.T == 0) continue;
+        if (bt.n == kMaxProbs) {
+            const lsn_status s = flush();
+            if (s != LSN_OK) return s;
+        }
+        DownProb& pb = bt.p[bt.n++];
+        pb.X = d.X;
+        pb.W = d.W;
+        pb.u32 = d.u32;
+        pb.u16 = d.u16;
+        pb.T = d.T;
+        pb.Kd = d.Kd;
+        pb.ns = down_splits(d.T, d.Kd);
+        pb.cps = (int)((d.Kd / 64 + pb.ns - 1) / pb.ns);
+        pb.first = blocks;
+        pb.scale = d.scale;
+        blocks += (int)((d.T + kDnRows - 1) / kDnRows);
+        smax = pb.ns > smax ? pb.ns : smax;
+    }
+    return flush();
+}
+
+// Token reductions of a batch of problems of the same rank.
+lsn_status launch_lora_tgrad_batch(int n, const TgSpec* specs, int r, cudaStream_t st) {
+    TgBatch bt{};
+    int blocks = 0, smax = 1;
+    auto flush = [&]() -> lsn_status {
+        if (bt.n == 0) return LSN_OK;
+        const lsn_status s = dispatch_tgrad(r, dim3((unsigned)blocks, (unsigned)smax), st, bt);
+        bt = TgBatch{};
+        blocks = 0;
+        smax = 1;
+        return s;
+    };
+    for (int i = 0; i < n; ++i) {
+        const TgSpec& d = specs[i];
+        if (d.Kd == 0) continue;
+        if (bt.n == kMaxProbs) {
+            const lsn_status s = flush();
+            if (s != LSN_OK) return s;
+        }
+        TgProb& pb = bt.p[bt.n++];
+        pb.G = d.G;
+        pb.X = d.X;
+        pb.out = d.out;
+        pb.T = d.T;
+        pb.Kd = d.Kd;
+        pb.ns = tgrad_splits(d.T, d.Kd);
+        pb.per = ((d.T + pb.ns - 1) / pb.ns + kTgTok - 1) / kTgTok * kTgTok;
+        pb.first = blocks;
+        pb.out_rk = d.out_rk ? 1 : 0;
+        pb.accumulate = d.accumulate;
+        pb.scale = d.scale;
+        blocks += (int)((d.Kd + kTgCols - 1) / kTgCols);
+        smax = pb.ns > smax ? pb.ns : smax;
+    }
+    return flush();
+}
+
 // X [T, Kd] times W: w_rk ? W is A [r, Kd] : W is B [Kd, r].
 lsn_status launch_lora_down(const uint16_t* X, const uint16_t* W, bool w_rk, int64_t T, int64_t Kd, int r,
                             float scale, float* u32, uint16_t* u16, float*, int*, cudaStream_t st) {
-    if (T == 0) return LSN_OK;
-    const int ns = down_splits(T, Kd);
-    const int64_t chunks = Kd / 64;
-    const int cps = (int)((chunks + ns - 1) / ns);
-    dim3 grid((unsigned)((T + kDnRows - 1) / kDnRows), (unsigned)ns);
-    return w_rk ? dispatch_down<false>(r, grid, st, X, W, T, Kd, cps, ns, scale, u32, u16)
-                : dispatch_down<true>(r, grid, st, X, W, T, Kd, cps, ns, scale, u32, u16);
+    const DownSpec d{X, W, u32, u16, T, Kd, scale};
+    return launch_lora_down_batch(1, &d, w_rk, r, st);
 }
 
 lsn_status launch_lora_tgrad(const float* G, const uint16_t* X, bool out_rk, int64_t T, int64_t Kd, int r,
                              float scale, int accumulate, float* out, float*, int*, cudaStream_t st) {
-    const int ns = tgrad_splits(T, Kd);
-    const int64_t per = ((T + ns - 1) / ns + kTgTok - 1) / kTgTok * kTgTok;
-    dim3 grid((unsigned)((Kd + kTgCols - 1) / kTgCols), (unsigned)ns);
-    return out_rk ? dispatch_tgrad<true>(r, grid, st, G, X, T, Kd, per, ns, scale, accumulate, out)
-                  : dispatch_tgrad<false>(r, grid, st, G, X, T, Kd, per, ns, scale, accumulate, out);
+    const TgSpec d{G, X, out, T, Kd, out_rk, accumulate, scale};
+    return launch_lora_tgrad_batch(1, &d, r, st);
 }
 
 }  // namespace lsn

@@ -27,6 +27,7 @@ LSN_OK, LSN_ERR_INVALID_ARG, LSN_ERR_CUDA, LSN_ERR_NO_MEMORY, LSN_ERR_TIMEOUT, L
 LSN_BASE_NF4, LSN_BASE_BF16 = 0, 1
 LSN_POOL_FAULT_NONE, LSN_POOL_FAULT_STALE_SLOT, LSN_POOL_FAULT_COPY_ERROR = 0, 1, 2
 LSN_OPT_FUSED_NF4 = 1
+LSN_OPT_LAYER_LANES = 2
 
 STATUS_NAMES = {0: "LSN_OK", 1: "LSN_ERR_INVALID_ARG", 2: "LSN_ERR_CUDA", 3: "LSN_ERR_NO_MEMORY",
                 4: "LSN_ERR_TIMEOUT", 5: "LSN_ERR_UNSUPPORTED", 6: "LSN_ERR_STATE"}
@@ -41,6 +42,7 @@ EXPORTS = (
     "layer_pool_release", "layer_pool_wait_idle", "layer_pool_stats", "layer_pool_reset",
     "layer_pool_inject_fault", "layer_pool_destroy", "lsn_timing_enable", "lsn_timing_read",
     "nf4_quantize_noalloc", "lsn_set_option", "lsn_get_option",
+    "lsn_layer_ws_bytes", "lora_layer_fwd", "lora_layer_bwd",
 )
 
 
@@ -59,6 +61,15 @@ class Base(ctypes.Structure):
     _fields_ = [("kind", ctypes.c_int), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
                 ("nf4", NF4Weight), ("bf16", ctypes.c_void_p)]
 
+
+class LoraProj(ctypes.Structure):
+    """One projection of a layer call (lsn_lora_proj)."""
+    _fields_ = [("W", Base), ("x", ctypes.c_void_p), ("A", ctypes.c_void_p), ("B", ctypes.c_void_p),
+                ("y", ctypes.c_void_p), ("dY", ctypes.c_void_p), ("dX", ctypes.c_void_p), ("dA", ctypes.c_void_p),
+                ("dB", ctypes.c_void_p), ("u", ctypes.c_void_p)]
+
+
+LSN_LAYER_MAX_PROJ = 16
 
 KERNEL_KINDS = ("gemm_fwd", "gemm_bwd", "dequant", "lora_down", "lora_tgrad", "quantize")
 
@@ -99,6 +110,9 @@ _sig("lora_linear_fwd", _i, [ctypes.POINTER(Base), _vp, _i64, _vp, _vp, _i, ctyp
 _sig("lora_linear_bwd", _i, [ctypes.POINTER(Base), _vp, _vp, _i64, _vp, _vp, _i, ctypes.c_float, _vp, _vp, _vp, _i,
                              _vp, _sz, _vp])
 _sig("lsn_ws_status", _i, [_vp, _vp])
+_sig("lsn_layer_ws_bytes", _sz, [_i, ctypes.POINTER(LoraProj), _i64, _i])
+_sig("lora_layer_fwd", _i, [_i, ctypes.POINTER(LoraProj), _i64, _i, ctypes.c_float, _vp, _sz, _vp])
+_sig("lora_layer_bwd", _i, [_i, ctypes.POINTER(LoraProj), _i64, _i, ctypes.c_float, _i, _vp, _sz, _vp])
 _sig("lsn_set_option", _i, [_i, _i])
 _sig("lsn_get_option", _i, [_i])
 _sig("lsn_timing_enable", _i, [_i])
@@ -226,6 +240,32 @@ def lora_linear_bwd(W: Base, x, dY, T: int, A, B, r: int, scale: float, dX, dA, 
     _check(_lib.lora_linear_bwd(ctypes.byref(W), _ptr(x), _ptr(dY), T, _ptr(A), _ptr(B), r, scale, _ptr(dX),
                                 _ptr(dA), _ptr(dB), int(bool(accumulate)), _ptr(ws), ws_bytes, _stream(stream)),
            "lora_linear_bwd")
+
+
+# ------------------------------------------------------------ whole layer ---
+
+def lora_proj(W: Base, x, A, B, y=None, dY=None, dX=None, dA=None, dB=None, u=None) -> LoraProj:
+    return LoraProj(W, _ptr(x), _ptr(A), _ptr(B), _ptr(y), _ptr(dY), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(u))
+
+
+def proj_array(projs) -> ctypes.Array:
+    return (LoraProj * len(projs))(*projs)
+
+
+def layer_ws_bytes(projs, T: int, r: int) -> int:
+    arr = projs if isinstance(projs, ctypes.Array) else proj_array(projs)
+    return _lib.lsn_layer_ws_bytes(len(arr), arr, T, r)
+
+
+def lora_layer_fwd(projs, T: int, r: int, scale: float, ws, ws_bytes: int, stream=None):
+    arr = projs if isinstance(projs, ctypes.Array) else proj_array(projs)
+    _check(_lib.lora_layer_fwd(len(arr), arr, T, r, scale, _ptr(ws), ws_bytes, _stream(stream)), "lora_layer_fwd")
+
+
+def lora_layer_bwd(projs, T: int, r: int, scale: float, accumulate: bool, ws, ws_bytes: int, stream=None):
+    arr = projs if isinstance(projs, ctypes.Array) else proj_array(projs)
+    _check(_lib.lora_layer_bwd(len(arr), arr, T, r, scale, int(bool(accumulate)), _ptr(ws), ws_bytes,
+                               _stream(stream)), "lora_layer_bwd")
 
 
 def ws_status(ws, stream=None):

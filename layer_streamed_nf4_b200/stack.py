@@ -10,7 +10,15 @@ backward sweep over L-1..0 (acquire i, prefetch i-1, seven lora_linear_bwd
 calls, release i).  All compute and all copies are library calls; this file
 only sequences them and owns the (synthetic) tensors.
 
-Lanes: the seven projections of a layer are independent calls, so they are
+Two ways to drive a layer (api=...):
+  "layer"  one lora_layer_fwd / lora_layer_bwd call per layer and sweep: the
+           library launches the seven projections together (one dequant, one
+           down-projection and one token-reduction kernel for all of them) and
+           the forward keeps u = x A^T for the backward;
+  "proj"   seven lora_linear_fwd / lora_linear_bwd calls per layer and sweep.
+Both give the same bits.
+
+Lanes ("proj" only): the seven projections of a layer are independent calls, so they are
 issued round-robin on `lanes` streams (default 2), each with its own
 workspace.  The side kernels and the dequantisation of one projection then
 run underneath another projection's GEMM on the SMs' spare shared memory
@@ -54,8 +62,10 @@ class Stack:
     def __init__(self, cfg: synth.StackConfig, layers: int | None = None, tokens: int | None = None,
                  mode: str = "streamed", n_slots: int = 2, seed: int = synth.SEED, keep_outputs: bool = False,
                  distinct_activations: bool = True, device: int = 0, stream: torch.cuda.Stream | None = None,
-                 lanes: int = 2):
+                 lanes: int = 2, api: str = "layer"):
         assert mode in ("resident", "streamed", "no_h2d")
+        assert api in ("layer", "proj")
+        self.api = api
         self.cfg, self.mode, self.seed = cfg, mode, seed
         self.L = layers if layers is not None else cfg.layers
         self.T = tokens if tokens is not None else cfg.tokens
@@ -66,6 +76,7 @@ class Stack:
         self.stream = stream if stream is not None else torch.cuda.current_stream(self.dev)
         self.keep_outputs = keep_outputs
         assert lanes >= 1
+        lanes = lanes if api == "proj" else 1
         self.n_lanes = lanes
         self.lanes = [self.stream] + [torch.cuda.Stream(self.dev) for _ in range(lanes - 1)]
         self._fork = [torch.cuda.Event() for _ in range(lanes)]
@@ -81,6 +92,7 @@ class Stack:
         self.host = None
         self.resident = None
         self._calls = {}
+        self._distinct = distinct_activations
         self._build_weights()
         self._build_tensors(distinct_activations)
         self._setup_mode(n_slots)
@@ -130,7 +142,13 @@ class Stack:
                   for l in range(nl) for pi, p in enumerate(self.proj)}
         self.dX = {(l, pi): torch.empty((T, p.K), dtype=torch.bfloat16, device=dev)
                    for l in range(nl) for pi, p in enumerate(self.proj)}
-        self.ws_bytes = max(lsnf4.lora_ws_bytes(T, p.K, p.N, r, self.kind) for p in self.proj)
+        if self.api == "layer":
+            # u = x A^T kept from the forward for the backward, per (layer, projection)
+            self.u = {(l, pi): torch.zeros((T, r), dtype=torch.float32, device=dev)
+                      for l in range(self.L) for pi in range(len(self.proj))}
+            self.ws_bytes = lsnf4.layer_ws_bytes(self._layer_projs(0, 0), T, r)
+        else:
+            self.ws_bytes = max(lsnf4.lora_ws_bytes(T, p.K, p.N, r, self.kind) for p in self.proj)
         self.ws = [torch.zeros(self.ws_bytes, dtype=torch.uint8, device=dev) for _ in range(self.n_lanes)]
         torch.cuda.synchronize(dev)
 
@@ -147,19 +165,42 @@ class Stack:
                 lsnf4.layer_pool_prefetch(self.pool, l)
             lsnf4.layer_pool_wait_idle(self.pool, 600000)
 
-    def with_mode(self, mode: str, n_slots: int = 2, lanes: int | None = None) -> "Stack":
+    def with_mode(self, mode: str, n_slots: int = 2, lanes: int | None = None, api: str | None = None) -> "Stack":
         """A stack sharing this one's host blobs and tensors, run in another mode
         (and, if given, another lane count)."""
         import copy
         assert mode in ("resident", "streamed", "no_h2d")
         other = copy.copy(self)
         other.mode, other.pool, other.resident, other._calls = mode, None, None, {}
-        if lanes is not None and lanes != self.n_lanes:
+        if api is not None and api != self.api:
+            assert api == "proj" or hasattr(self, "u"), "a stack built for the per-projection calls keeps no u"
+            other.api = api
+            if api == "layer":
+                other.ws_bytes = lsnf4.layer_ws_bytes(self._layer_projs(0, 0), self.T, self.r)
+            else:
+                other.ws_bytes = max(lsnf4.lora_ws_bytes(self.T, p.K, p.N, self.r, self.kind) for p in self.proj)
+            other.n_lanes = lanes if (lanes is not None and api == "proj") else 1
+            other.lanes = [self.stream] + [torch.cuda.Stream(self.dev) for _ in range(other.n_lanes - 1)]
+            other._fork = [torch.cuda.Event() for _ in range(other.n_lanes)]
+            other._join = [torch.cuda.Event() for _ in range(other.n_lanes)]
+            other.ws = [torch.zeros(other.ws_bytes, dtype=torch.uint8, device=self.dev) for _ in range(other.n_lanes)]
+        elif lanes is not None and lanes != self.n_lanes and self.api == "proj":
             other.n_lanes = lanes
             other.lanes = [self.stream] + [torch.cuda.Stream(self.dev) for _ in range(lanes - 1)]
             other._fork = [torch.cuda.Event() for _ in range(lanes)]
             other._join = [torch.cuda.Event() for _ in range(lanes)]
             other.ws = [torch.zeros(self.ws_bytes, dtype=torch.uint8, device=self.dev) for _ in range(lanes)]
+        other._setup_mode(n_slots)
+        return other
+
+    def with_tokens(self, tokens: int, mode: str = "streamed", n_slots: int = 2) -> "Stack":
+        """A stack sharing this one's host blobs (the frozen base) and adapters' seeds, with its own
+        activations for `tokens` tokens (a larger batch streams the same weights)."""
+        import copy
+        other = copy.copy(self)
+        other.T, other.mode = tokens, mode
+        other.pool, other.resident, other._calls = None, None, {}
+        other._build_tensors(self._distinct)
         other._setup_mode(n_slots)
         return other
 
@@ -240,7 +281,46 @@ class Stack:
             self._calls[key] = a
         return a
 
+    def _layer_projs(self, addr: int, l: int):
+        """The lsn_lora_proj array of layer l whose blob sits at addr (cached: it depends on nothing else)."""
+        key = ("L", addr, l)
+        a = self._calls.get(key)
+        if a is None:
+            projs = [lsnf4.lora_proj(self._base(addr, p), self.x[l, pi], self.A[l, pi], self.B[l, pi],
+                                     y=self._out(self.y, l, pi), dY=self.dY[l, pi], dX=self._out(self.dX, l, pi),
+                                     dA=self.dA[l, pi], dB=self.dB[l, pi],
+                                     u=self.u[l, pi] if hasattr(self, "u") else None)
+                     for pi, p in enumerate(self.proj)]
+            a = lsnf4.proj_array(projs)
+            if addr:
+                self._calls[key] = a
+        return a
+
+    def _forward_layers(self):
+        fwd = lsnf4._lib.lora_layer_fwd
+        n, ws, nb, sp = len(self.proj), self.ws[0].data_ptr(), self.ws_bytes, self.stream.cuda_stream
+        for l in range(self.L):
+            addr = self._acquire(l)
+            self._prefetch(l + 1)
+            st = fwd(n, self._layer_projs(addr, l), self.T, self.r, self.scale, ws, nb, sp)
+            if st:
+                lsnf4._check(st, "lora_layer_fwd")
+            self._release(l)
+
+    def _backward_layers(self, accumulate: bool):
+        bwd = lsnf4._lib.lora_layer_bwd
+        n, ws, nb, sp = len(self.proj), self.ws[0].data_ptr(), self.ws_bytes, self.stream.cuda_stream
+        for l in reversed(range(self.L)):
+            addr = self._acquire(l)
+            self._prefetch(l - 1)
+            st = bwd(n, self._layer_projs(addr, l), self.T, self.r, self.scale, int(accumulate), ws, nb, sp)
+            if st:
+                lsnf4._check(st, "lora_layer_bwd")
+            self._release(l)
+
     def forward(self):
+        if self.api == "layer":
+            return self._forward_layers()
         fwd = lsnf4._lib.lora_linear_fwd
         for l in range(self.L):
             addr = self._acquire(l)
@@ -254,6 +334,8 @@ class Stack:
             self._release(l)
 
     def backward(self, accumulate: bool = False):
+        if self.api == "layer":
+            return self._backward_layers(accumulate)
         bwd = lsnf4._lib.lora_linear_bwd
         for l in reversed(range(self.L)):
             addr = self._acquire(l)

@@ -117,3 +117,76 @@ def test_workspace_sizes_for_edge_shapes(lib, T, K, N):
 def test_last_error_is_never_null(lib):
     assert isinstance(lib.last_error(), str)
     assert lib.version() >= 100
+
+
+def test_struct_layouts_match_the_header(lib, tmp_path):
+    """ctypes' view of the ABI structs equals the C compiler's (sizes and field offsets)."""
+    import ctypes
+    import subprocess
+    src = tmp_path / "layout.c"
+    src.write_text(
+        '#include <stdio.h>\n#include <stddef.h>\n#include "lsnf4.h"\n'
+        "int main(void) {\n"
+        '  printf("%zu %zu %zu %zu %zu %zu\\n", sizeof(lsn_nf4_weight), sizeof(lsn_base), sizeof(lsn_lora_proj),\n'
+        "         offsetof(lsn_base, nf4), offsetof(lsn_lora_proj, x), offsetof(lsn_lora_proj, u));\n"
+        "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
+    want = [ctypes.sizeof(lib.NF4Weight), ctypes.sizeof(lib.Base), ctypes.sizeof(lib.LoraProj),
+            lib.Base.nf4.offset, lib.LoraProj.x.offset, lib.LoraProj.u.offset]
+    assert got == want
+
+
+def _fake_projs(lib, shapes, kind):
+    projs = []
+    for K, N in shapes:
+        if kind == lib.LSN_BASE_NF4:
+            base = lib.base_nf4(lib.make_nf4_weight(N, K, 1 << 20, 1 << 20, 1 << 20, 1 << 20))
+        else:
+            base = lib.base_bf16(1 << 20, N, K)
+        projs.append(lib.lora_proj(base, 1 << 20, 1 << 20, 1 << 20, y=1 << 20, dY=1 << 20, dX=1 << 20, dA=1 << 20,
+                                   dB=1 << 20))
+    return projs
+
+
+def test_layer_workspace_sizes(lib):
+    shapes = [(4096, 4096), (4096, 1024), (4096, 1024), (4096, 4096), (4096, 14336), (4096, 14336), (14336, 4096)]
+    nf4 = lib.layer_ws_bytes(_fake_projs(lib, shapes, lib.LSN_BASE_NF4), 2048, 16)
+    bf = lib.layer_ws_bytes(_fake_projs(lib, shapes, lib.LSN_BASE_BF16), 2048, 16)
+    assert nf4 - bf == sum(K * N * 2 for K, N in shapes)         # the dequantised copies
+    assert bf >= 256 + 7 * 2048 * 16 * (2 + 4 + 4)
+    assert lib.layer_ws_bytes(_fake_projs(lib, shapes, lib.LSN_BASE_BF16), 2048, 12) == 0    # bad rank
+    assert lib.layer_ws_bytes(_fake_projs(lib, shapes * 3, lib.LSN_BASE_BF16), 2048, 16) == 0  # n > 16
+
+
+def test_layer_calls_reject_bad_arguments(lib):
+    projs = _fake_projs(lib, [(256, 256), (256, 64)], lib.LSN_BASE_BF16)
+    need = lib.layer_ws_bytes(projs, 128, 8)
+    with pytest.raises(lib.LsnError) as e:                        # workspace too small
+        lib.lora_layer_fwd(projs, 128, 8, 2.0, 1 << 20, need - 1, stream=0)
+    assert e.value.status == lib.LSN_ERR_INVALID_ARG
+    bad = _fake_projs(lib, [(256, 256), (256, 100)], lib.LSN_BASE_BF16)   # N % 64 != 0
+    with pytest.raises(lib.LsnError) as e:
+        lib.lora_layer_bwd(bad, 128, 8, 2.0, False, 1 << 20, 1 << 30, stream=0)
+    assert e.value.status == lib.LSN_ERR_INVALID_ARG
+    mis = _fake_projs(lib, [(256, 256)], lib.LSN_BASE_BF16)
+    mis[0].u = (1 << 20) + 4                                       # misaligned u
+    with pytest.raises(lib.LsnError) as e:
+        lib.lora_layer_fwd(mis, 128, 8, 2.0, 1 << 20, 1 << 30, stream=0)
+    assert e.value.status == lib.LSN_ERR_INVALID_ARG
+    with pytest.raises(lib.LsnError) as e:                        # empty projection list
+        lib.lora_layer_fwd(lib.proj_array([]), 128, 8, 2.0, 1 << 20, 1 << 30, stream=0)
+    assert e.value.status == lib.LSN_ERR_INVALID_ARG
+
+
+def test_options(lib):
+    assert lib.get_option(lib.LSN_OPT_LAYER_LANES) == 2
+    with pytest.raises(lib.LsnError) as e:
+        lib.set_option(lib.LSN_OPT_LAYER_LANES, 3)
+    assert e.value.status == lib.LSN_ERR_INVALID_ARG
+    lib.set_option(lib.LSN_OPT_LAYER_LANES, 1)
+    assert lib.get_option(lib.LSN_OPT_LAYER_LANES) == 1
+    lib.set_option(lib.LSN_OPT_LAYER_LANES, 2)
+    assert lib.get_option(lib.LSN_OPT_FUSED_NF4) == 0
+    assert lib.get_option(12345) == -1

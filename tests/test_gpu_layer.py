@@ -1,0 +1,174 @@
+"""The whole-layer calls (lora_layer_fwd / lora_layer_bwd) through the C ABI.
+
+They launch the projections of a decoder layer together (one dequantisation
+kernel, one down-projection kernel, one token-reduction kernel for all of
+them) and can carry u = x A^T from the forward to the backward.  Each
+projection's results must be bit for bit those of the single-linear calls
+on the same inputs, and within the oracle tolerances."""
+import numpy as np
+import pytest
+
+from layer_streamed_nf4_b200 import synth
+from tests.helpers import DeviceNF4, assert_close, bf16_tensor_to_f64, bits_to_device_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import torch
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from layer_streamed_nf4_b200 import lsnf4
+    return lsnf4
+
+
+class Layer:
+    """Device tensors of n projections sharing T and r (seeded like the stacks)."""
+
+    def __init__(self, lib, shapes, T, r, kind, seed=5):
+        import torch
+        self.lib, self.T, self.r, self.kind = lib, T, r, kind
+        self.scale = 2.0
+        dev = torch.device("cuda")
+        self.p = []
+        for pi, (K, N) in enumerate(shapes):
+            # host inputs from the shared seeded generator; the oracle sees these, never device results
+            c = synth.linear_case(T, K, N, r, self.scale * r, seed=seed * 100 + pi)
+            d = {"K": K, "N": N, "case": c}
+            if kind == "nf4":
+                d["nf4"] = DeviceNF4(N, K).quantize(c.W)
+                d["base"] = lib.base_nf4(d["nf4"].w)
+            else:
+                d["Wb"] = bits_to_device_bf16(synth.to_bf16_bits(c.W))
+                d["base"] = lib.base_bf16(d["Wb"], N, K)
+            for k in ("x", "dY", "A", "B"):
+                d[k] = bits_to_device_bf16(getattr(c, k)) if getattr(c, k).size else \
+                    torch.empty(getattr(c, k).shape, dtype=torch.bfloat16, device=dev)
+            self.p.append(d)
+
+    def outputs(self):
+        import torch
+        out = []
+        for d in self.p:
+            out.append({"y": torch.empty((self.T, d["N"]), dtype=torch.bfloat16, device="cuda"),
+                        "dX": torch.empty((self.T, d["K"]), dtype=torch.bfloat16, device="cuda"),
+                        "dA": torch.zeros((self.r, d["K"]), dtype=torch.float32, device="cuda"),
+                        "dB": torch.zeros((d["N"], self.r), dtype=torch.float32, device="cuda"),
+                        "u": torch.zeros((self.T, self.r), dtype=torch.float32, device="cuda")})
+        return out
+
+    def single(self, accumulate=False, out=None):
+        import torch
+        lib = self.lib
+        out = out or self.outputs()
+        k = lib.LSN_BASE_NF4 if self.kind == "nf4" else lib.LSN_BASE_BF16
+        for d, o in zip(self.p, out):
+            n = lib.lora_ws_bytes(self.T, d["K"], d["N"], self.r, k)
+            ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
+            lib.lora_linear_fwd(d["base"], d["x"], self.T, d["A"], d["B"], self.r, self.scale, o["y"], ws, n)
+            lib.lora_linear_bwd(d["base"], d["x"], d["dY"], self.T, d["A"], d["B"], self.r, self.scale, o["dX"],
+                                o["dA"], o["dB"], accumulate, ws, n)
+            torch.cuda.synchronize()
+            lib.ws_status(ws)
+        return out
+
+    def layer(self, keep_u=True, accumulate=False, out=None):
+        import torch
+        lib = self.lib
+        out = out or self.outputs()
+        projs = [lib.lora_proj(d["base"], d["x"], d["A"], d["B"], y=o["y"], dY=d["dY"], dX=o["dX"], dA=o["dA"],
+                               dB=o["dB"], u=o["u"] if keep_u else None) for d, o in zip(self.p, out)]
+        arr = lib.proj_array(projs)
+        n = lib.layer_ws_bytes(arr, self.T, self.r)
+        ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
+        lib.lora_layer_fwd(arr, self.T, self.r, self.scale, ws, n)
+        lib.lora_layer_bwd(arr, self.T, self.r, self.scale, accumulate, ws, n)
+        torch.cuda.synchronize()
+        lib.ws_status(ws)
+        return out
+
+
+SHAPES_8B = [(4096, 4096), (4096, 1024), (4096, 1024), (4096, 4096), (4096, 14336), (4096, 14336), (14336, 4096)]
+SMALL = [(256, 256), (256, 64), (256, 128), (256, 256), (256, 512), (256, 512), (512, 256)]
+
+
+def _equal(a, b, names=("y", "dX", "dA", "dB")):
+    import torch
+    for i, (u, v) in enumerate(zip(a, b)):
+        for k in names:
+            assert torch.equal(u[k], v[k]), f"projection {i}: {k} differs"
+
+
+@pytest.mark.parametrize("shapes,T,kind", [(SMALL, 300, "nf4"), (SMALL, 77, "bf16"), (SHAPES_8B, 2048, "nf4")])
+def test_layer_equals_single_calls(lib, shapes, T, kind):
+    L = Layer(lib, shapes, T, 16, kind)
+    ref = L.single()
+    _equal(L.layer(keep_u=True), ref)
+    _equal(L.layer(keep_u=False), ref)
+
+
+def test_kept_u_is_x_times_a_transposed(lib, orc):
+    """The u the forward keeps equals the oracle's x A^T (fp32 accumulation of exact bf16 products)."""
+    L = Layer(lib, SMALL[:3], 130, 16, "nf4")
+    out = L.layer(keep_u=True)
+    for d, o in zip(L.p, out):
+        c = d["case"]
+        x = synth.bf16_bits_to_f32(c.x).astype(np.float64)
+        A = synth.bf16_bits_to_f32(c.A).astype(np.float64)
+        assert_close(o["u"].cpu().numpy(), x @ A.T, "u")
+
+
+def test_layer_accumulates_like_single_calls(lib):
+    import torch
+    L = Layer(lib, SMALL, 200, 8, "nf4")
+    a = L.single()
+    a = L.single(accumulate=True, out=a)
+    b = L.layer()
+    b = L.layer(accumulate=True, out=b)
+    _equal(a, b, ("dA", "dB"))
+    assert all(float(o["dA"].abs().sum()) > 0 for o in b)
+
+
+def test_layer_against_oracle(lib, orc):
+    """One small layer checked directly against the fp64 oracle."""
+    L = Layer(lib, SMALL[:2], 96, 16, "nf4", seed=9)
+    out = L.layer()
+    for d, o in zip(L.p, out):
+        c = d["case"]
+        q = orc.nf4_quantize(c.W)                  # the oracle quantises the fp32 weight itself
+        Wb = orc.nf4_dequant(q["packed"], q["absmax_q"], q["s2"], q["offset"], c.W.size).reshape(c.W.shape)
+        x, dY, A, B = c.x, c.dY, c.A, c.B
+        assert_close(bf16_tensor_to_f64(o["y"]), orc.lora_fwd(x, Wb, A, B, L.scale), "y")
+        assert_close(bf16_tensor_to_f64(o["dX"]), orc.lora_bwd_dx(dY, Wb, A, B, L.scale), "dX")
+        rA, rB = orc.lora_bwd_dadb(x, dY, A, B, L.scale)
+        assert_close(o["dA"].cpu().numpy(), rA, "dA")
+        assert_close(o["dB"].cpu().numpy(), rB, "dB")
+
+
+def test_layer_with_fused_nf4_equals_unfused(lib):
+    lib.set_option(lib.LSN_OPT_FUSED_NF4, 1)
+    try:
+        L = Layer(lib, [(4096, 9536), (9536, 4096), (4096, 1024)], 512, 16, "nf4")
+        a = L.layer()
+    finally:
+        lib.set_option(lib.LSN_OPT_FUSED_NF4, 0)
+    _equal(a, L.layer())
+
+
+def test_layer_zero_tokens(lib):
+    import torch
+    L = Layer(lib, SMALL[:2], 0, 16, "nf4")
+    out = L.layer()
+    assert all(float(o["dA"].abs().sum()) == 0.0 and float(o["dB"].abs().sum()) == 0.0 for o in out)
+
+
+def test_layer_lanes_option_gives_the_same_bits(lib):
+    L = Layer(lib, SMALL, 257, 16, "nf4", seed=3)
+    a = L.layer()                                     # default: two lanes
+    lib.set_option(lib.LSN_OPT_LAYER_LANES, 1)
+    try:
+        b = L.layer()
+    finally:
+        lib.set_option(lib.LSN_OPT_LAYER_LANES, 2)
+    _equal(a, b)
+    _equal(a, L.single())

@@ -24,11 +24,11 @@ def lib():
     return lsnf4
 
 
-def _run(cfg, layers, tokens, mode, fault=None, steps=1, lanes=2):
+def _run(cfg, layers, tokens, mode, fault=None, steps=1, lanes=2, api="layer"):
     import torch
     from layer_streamed_nf4_b200 import lsnf4
     from layer_streamed_nf4_b200.stack import Stack
-    st = Stack(cfg, layers=layers, tokens=tokens, mode=mode, keep_outputs=True, lanes=lanes)
+    st = Stack(cfg, layers=layers, tokens=tokens, mode=mode, keep_outputs=True, lanes=lanes, api=api)
     if fault is not None:
         lsnf4.layer_pool_inject_fault(st.pool, fault)
     for _ in range(steps):
@@ -60,8 +60,8 @@ def test_streamed_equals_resident(lib, name, layers, tokens, fused):
 
 def _streamed_equals_resident(lib, name, layers, tokens):
     cfg = synth.STACKS[name]
-    res = _run(cfg, layers, tokens, "resident", lanes=1)     # every call on one stream
-    stm = _run(cfg, layers, tokens, "streamed", steps=2)     # projections spread over two streams
+    res = _run(cfg, layers, tokens, "resident", lanes=1, api="proj")   # per-projection calls on one stream
+    stm = _run(cfg, layers, tokens, "streamed", steps=2)              # whole-layer calls
     fwd, bwd, bad = _compare(stm, res)
     assert fwd, f"{name}: streamed forward differs from resident"
     # two streamed steps without accumulation: gradients are those of one step
@@ -73,11 +73,15 @@ def _streamed_equals_resident(lib, name, layers, tokens):
 
 @pytest.mark.parametrize("name,layers,tokens", [("0.5b", 4, 512), ("8b", 2, 1024)])
 def test_lane_count_does_not_change_results(lib, name, layers, tokens):
-    """The projections of a layer issued on 1, 2 or 3 streams give the same bits."""
+    """The projections of a layer issued on 1, 2 or 3 streams, or as one layer call, give the same bits."""
     cfg = synth.STACKS[name]
-    one = _run(cfg, layers, tokens, "no_h2d", lanes=1)
+    one = _run(cfg, layers, tokens, "no_h2d", lanes=1, api="proj")
+    whole = _run(cfg, layers, tokens, "no_h2d", api="layer")
+    fwd, bwd, bad = _compare(whole, one)
+    assert fwd and bwd, ("layer call", bad)
+    whole.close()
     for lanes in (2, 3):
-        many = _run(cfg, layers, tokens, "no_h2d", lanes=lanes)
+        many = _run(cfg, layers, tokens, "no_h2d", lanes=lanes, api="proj")
         fwd, bwd, bad = _compare(many, one)
         assert fwd and bwd, (lanes, bad)
         many.close()
