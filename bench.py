@@ -299,6 +299,7 @@ def run_ours(args):
                    "api": args.api,
                    "lanes": args.lanes if args.api == "proj" else 1,
                    "nf4_conversion": "inside the GEMM" if args.fused_nf4 else "nf4_dequant then bf16 GEMM",
+                   "programmatic_dependent_launch": not args.no_pdl,
                    "l2": "inputs larger than L2 (per step ~11 GB of activations, ~3.6 GB of streamed weights)"},
         "pct_bf16_peak": 100 * flop_step / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
         "flop_per_step": flop_step,
@@ -473,12 +474,16 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=60.0)
     ap.add_argument("--ref-rows", type=int, default=4)
     ap.add_argument("--fused-nf4", action="store_true", help="convert NF4 inside the GEMM (no bf16 copy of W)")
+    ap.add_argument("--no-pdl", action="store_true", help="ordinary launches instead of programmatic dependent ones")
     ap.add_argument("--case", default="", help="profile one 8B projection (q,k,v,o,gate,up,down) instead of the stack")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
-    if args.fused_nf4 and args.impl == "ours":
+    if args.impl == "ours" and (args.fused_nf4 or args.no_pdl):
         from layer_streamed_nf4_b200 import lsnf4
-        lsnf4.set_option(lsnf4.LSN_OPT_FUSED_NF4, 1)
+        if args.fused_nf4:
+            lsnf4.set_option(lsnf4.LSN_OPT_FUSED_NF4, 1)
+        if args.no_pdl:
+            lsnf4.set_option(lsnf4.LSN_OPT_PDL, 0)
     if args.impl == "reference":
         run_reference(args)
     elif args.case:

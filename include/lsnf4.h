@@ -299,8 +299,15 @@ lsn_status lsn_timing_read(lsn_kernel_timing* out);
  *                      stream of the same device, which forks from the
  *                      caller's stream and joins it again within the call;
  *                      1: everything on the caller's stream.
+ *   LSN_OPT_PDL        1 (default): the hot-path kernels are launched with
+ *                      programmatic dependent launch, so each kernel's set-up
+ *                      (barriers, tensor memory, tensor-map prefetch) overlaps
+ *                      the tail of the kernel before it on the same stream;
+ *                      every kernel still waits for its predecessor to finish
+ *                      before it reads or writes global memory.  0: ordinary
+ *                      stream-ordered launches.
  */
-typedef enum { LSN_OPT_FUSED_NF4 = 1, LSN_OPT_LAYER_LANES = 2 } lsn_option;
+typedef enum { LSN_OPT_FUSED_NF4 = 1, LSN_OPT_LAYER_LANES = 2, LSN_OPT_PDL = 3 } lsn_option;
 lsn_status lsn_set_option(int option, int value);
 int lsn_get_option(int option);
 

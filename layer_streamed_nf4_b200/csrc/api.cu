@@ -16,6 +16,7 @@ namespace {
 thread_local std::string g_last_error = "no error";
 std::atomic<int> g_fused_nf4{0};
 std::atomic<int> g_layer_lanes{2};
+std::atomic<int> g_pdl{1};
 }
 
 lsn_status fail(lsn_status st, const std::string& msg) {
@@ -27,6 +28,8 @@ lsn_status fail_cuda(cudaError_t e, const char* what) {
     g_last_error = std::string(what) + ": " + cudaGetErrorName(e) + " (" + cudaGetErrorString(e) + ")";
     return LSN_ERR_CUDA;
 }
+
+bool pdl_enabled() { return g_pdl.load() != 0; }
 
 int sm_count() {
     int dev = 0;
@@ -538,6 +541,10 @@ lsn_status lora_layer_bwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
 }
 
 lsn_status lsn_set_option(int option, int value) {
+    if (option == LSN_OPT_PDL) {
+        g_pdl.store(value != 0 ? 1 : 0);
+        return LSN_OK;
+    }
     if (option == LSN_OPT_LAYER_LANES) {
         LSN_CHECK_ARG(value == 1 || value == 2, "lsn_set_option: LSN_OPT_LAYER_LANES takes 1 or 2");
         g_layer_lanes.store(value);
@@ -553,6 +560,7 @@ lsn_status lsn_set_option(int option, int value) {
 int lsn_get_option(int option) {
     if (option == LSN_OPT_FUSED_NF4) return g_fused_nf4.load();
     if (option == LSN_OPT_LAYER_LANES) return g_layer_lanes.load();
+    if (option == LSN_OPT_PDL) return g_pdl.load();
     return -1;
 }
 

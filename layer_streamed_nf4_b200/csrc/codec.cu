@@ -208,20 +208,21 @@ struct DqBatch {
     DqItem it[kDqMax];
 };
 
-// Standalone dequantisation of a batch of weights: each thread reads 128-bit
-// words of packed codes (coalesced across the warp, four words in flight),
-// looks up the 16 levels in shared memory, scales them by the block's
-// reconstructed absmax and writes 64 bytes of bf16.  A block covers 1024
-// consecutive vectors of one weight.
+// Standalone dequantisation of a batch of weights: each thread reads four
+// 128-bit words of packed codes (coalesced across the warp, all four in
+// flight at once), builds the block's 16 scaled levels bf16(level *
+// absmax_hat) in registers and maps the 32 codes of a word onto them with
+// byte permutes (no shared-memory lookup per element), writing 64 bytes of
+// bf16 per word.  A block covers 1024 consecutive words of one weight.
 __global__ void __launch_bounds__(kDqThreads) nf4_dequant_kernel(const __grid_constant__ DqBatch bt,
                                                                  const __grid_constant__ DequantParams P) {
-    __shared__ float lv[16];
     __shared__ float dq[256];
     for (int i = threadIdx.x; i < 256; i += blockDim.x) dq[i] = P.dq[i];
-    if (threadIdx.x < 16) lv[threadIdx.x] = P.level[threadIdx.x];
     int ii = 0;
     while (ii + 1 < bt.n && (int64_t)blockIdx.x >= bt.it[ii + 1].first) ++ii;
     const DqItem& it = bt.it[ii];
+    pdl_launch_dependents();
+    pdl_wait();
     const uint4* __restrict__ packed = it.packed;
     const uint8_t* __restrict__ absmax_q = it.absmax_q;
     const float* __restrict__ s2 = it.s2;
@@ -229,39 +230,29 @@ __global__ void __launch_bounds__(kDqThreads) nf4_dequant_kernel(const __grid_co
     const float off = *it.offset;
     const int64_t v0 = ((int64_t)blockIdx.x - it.first) * kDqVecPerBlock + threadIdx.x;
     uint4 p[kDqUnroll];
-    float ah[kDqUnroll];
-    #pragma unroll
-    for (int u = 0; u < kDqUnroll; ++u) {
-        const int64_t v = v0 + u * kDqThreads;
-        p[u] = v < it.nvec ? __ldg(packed + v) : make_uint4(0, 0, 0, 0);
-    }
     uint32_t code[kDqUnroll];
     float sc[kDqUnroll];
     #pragma unroll
     for (int u = 0; u < kDqUnroll; ++u) {
         const int64_t v = v0 + u * kDqThreads;
-        const int64_t b = (v < it.nvec ? v : 0) >> 1;   // absmax block of the vector
+        const bool ok = v < it.nvec;
+        const int64_t b = (ok ? v : 0) >> 1;             // absmax block of the vector
+        p[u] = ok ? __ldg(packed + v) : make_uint4(0, 0, 0, 0);
         code[u] = __ldg(absmax_q + b);
         sc[u] = __ldg(s2 + (b >> 8));
     }
-    __syncthreads();                                     // level and code tables are in shared memory
-    #pragma unroll
-    for (int u = 0; u < kDqUnroll; ++u) ah[u] = __fadd_rn(__fmul_rn(dq[code[u]], sc[u]), off);
+    __syncthreads();                                     // the code table is in shared memory
     #pragma unroll
     for (int u = 0; u < kDqUnroll; ++u) {
         const int64_t v = v0 + u * kDqThreads;
         if (v >= it.nvec) break;
-        const uint32_t w[4] = {p[u].x, p[u].y, p[u].z, p[u].w};
-        #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-            uint32_t r[4];
-            #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const uint32_t byte = (w[h] >> (8 * j)) & 0xffu;
-                r[j] = pack_bf16x2(__fmul_rn(lv[byte >> 4], ah[u]), __fmul_rn(lv[byte & 15u], ah[u]));
-            }
-            out[v * 4 + h] = make_uint4(r[0], r[1], r[2], r[3]);
-        }
+        const float ah = __fadd_rn(__fmul_rn(dq[code[u]], sc[u]), off);
+        uint32_t lo[4], hi[4];
+        nf4_scaled_table(P.level, ah, lo, hi);
+        out[v * 4 + 0] = nf4x8_to_bf16(p[u].x, lo, hi);
+        out[v * 4 + 1] = nf4x8_to_bf16(p[u].y, lo, hi);
+        out[v * 4 + 2] = nf4x8_to_bf16(p[u].z, lo, hi);
+        out[v * 4 + 3] = nf4x8_to_bf16(p[u].w, lo, hi);
     }
 }
 
@@ -315,8 +306,14 @@ lsn_status launch_dequant_batch(int n, const lsn_nf4_weight* const* w, uint16_t*
     int64_t blocks = 0;
     auto flush = [&]() -> lsn_status {
         if (bt.n == 0) return LSN_OK;
-        nf4_dequant_kernel<<<(unsigned)blocks, kDqThreads, 0, st>>>(bt, P);
-        LSN_CUDA_TRY(cudaGetLastError());
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)blocks);
+        cfg.blockDim = dim3(kDqThreads);
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        cfg.attrs = attr;
+        cfg.numAttrs = pdl_attr(&attr[0]);
+        LSN_CUDA_TRY(cudaLaunchKernelEx(&cfg, nf4_dequant_kernel, bt, P));
         bt = DqBatch{};
         blocks = 0;
         return LSN_OK;

@@ -137,6 +137,15 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
     }
 }
 
+// Programmatic dependent launch.  pdl_launch_dependents lets the next kernel
+// on the stream be scheduled while this grid still runs (its CTAs occupy SMs
+// as this grid's CTAs leave and run their own set-up); pdl_wait blocks until
+// the grid this one depends on has finished and its memory writes are
+// visible.  Every kernel launched with the attribute calls pdl_wait before
+// its first global-memory access.  Both are no-ops for an ordinary launch.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -289,6 +298,43 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
     return r;
+}
+
+// ------------------------------------------------------------ NF4 unpack ---
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// Eight NF4 codes (one 32-bit word of the packed layout: byte j holds element
+// 2j in its high nibble and 2j+1 in its low nibble) to eight bf16 values, by
+// byte permutes on the block's 16-entry table of scaled values: lo[t]/hi[t]
+// hold the low/high bytes of table entries 4t..4t+3.  A selector nibble below
+// 8 picks a byte; the top bit of each code chooses between the tables of
+// entries 0-7 and 8-15 (a byte mask built with prmt's sign-replicate mode).
+__device__ __forceinline__ uint4 nf4x8_to_bf16(uint32_t p, const uint32_t (&lo)[4], const uint32_t (&hi)[4]) {
+    const uint32_t a = p << 4;
+    const uint32_t s0 = p & 0x7777u, s1 = (p >> 16) & 0x7777u;
+    const uint32_t m0 = prmt(a, p, 0xD9C8u), m1 = prmt(a, p, 0xFBEAu);
+    const uint32_t l0 = (prmt(lo[0], lo[1], s0) & ~m0) | (prmt(lo[2], lo[3], s0) & m0);
+    const uint32_t h0 = (prmt(hi[0], hi[1], s0) & ~m0) | (prmt(hi[2], hi[3], s0) & m0);
+    const uint32_t l1 = (prmt(lo[0], lo[1], s1) & ~m1) | (prmt(lo[2], lo[3], s1) & m1);
+    const uint32_t h1 = (prmt(hi[0], hi[1], s1) & ~m1) | (prmt(hi[2], hi[3], s1) & m1);
+    // l0/h0 bytes are elements (1, 0, 3, 2); interleave into bf16 pairs in element order.
+    return make_uint4(prmt(l0, h0, 0x4051u), prmt(l0, h0, 0x6273u), prmt(l1, h1, 0x4051u), prmt(l1, h1, 0x6273u));
+}
+
+__device__ __forceinline__ void nf4_scaled_table(const float* level, float ah, uint32_t (&lo)[4], uint32_t (&hi)[4]) {
+    uint32_t e[8];
+    #pragma unroll
+    for (int i = 0; i < 8; ++i) e[i] = pack_bf16x2(__fmul_rn(level[2 * i], ah), __fmul_rn(level[2 * i + 1], ah));
+    #pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        lo[i] = prmt(e[2 * i], e[2 * i + 1], 0x6420u);
+        hi[i] = prmt(e[2 * i], e[2 * i + 1], 0x7531u);
+    }
 }
 
 }  // namespace lsn

@@ -26,6 +26,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "launch.cuh"
 
 namespace lsn {
 
@@ -91,30 +92,6 @@ __device__ __forceinline__ void raise_error(volatile int* abort_flag, int* err, 
     if (err) atomicExch(err, code);
 }
 
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-    uint32_t d;
-    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-    return d;
-}
-
-// Eight NF4 codes (one 32-bit word of the packed layout: byte j holds element
-// 2j in its high nibble and 2j+1 in its low nibble) to eight bf16 values, by
-// byte permutes on the block's 16-entry table of scaled values: lo[t]/hi[t]
-// hold the low/high bytes of table entries 4t..4t+3.  A selector nibble below
-// 8 picks a byte; the top bit of each code chooses between the tables of
-// entries 0-7 and 8-15 (a byte mask built with prmt's sign-replicate mode).
-__device__ __forceinline__ uint4 nf4x8_to_bf16(uint32_t p, const uint32_t (&lo)[4], const uint32_t (&hi)[4]) {
-    const uint32_t a = p << 4;
-    const uint32_t s0 = p & 0x7777u, s1 = (p >> 16) & 0x7777u;
-    const uint32_t m0 = prmt(a, p, 0xD9C8u), m1 = prmt(a, p, 0xFBEAu);
-    const uint32_t l0 = (prmt(lo[0], lo[1], s0) & ~m0) | (prmt(lo[2], lo[3], s0) & m0);
-    const uint32_t h0 = (prmt(hi[0], hi[1], s0) & ~m0) | (prmt(hi[2], hi[3], s0) & m0);
-    const uint32_t l1 = (prmt(lo[0], lo[1], s1) & ~m1) | (prmt(lo[2], lo[3], s1) & m1);
-    const uint32_t h1 = (prmt(hi[0], hi[1], s1) & ~m1) | (prmt(hi[2], hi[3], s1) & m1);
-    // l0/h0 bytes are elements (1, 0, 3, 2); interleave into bf16 pairs in element order.
-    return make_uint4(prmt(l0, h0, 0x4051u), prmt(l0, h0, 0x6273u), prmt(l1, h1, 0x4051u), prmt(l1, h1, 0x6273u));
-}
-
 template <bool PAIR, int BN, bool B_MN, bool NF4>
 __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN, NF4>::THREADS, 1)
     lsn_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -172,6 +149,8 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN, NF4>::THREADS, 1)
     if constexpr (PAIR) cluster_sync_all();   // both CTAs' barriers initialised before any remote use
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
+    pdl_launch_dependents();
+    pdl_wait();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -504,6 +483,8 @@ __global__ void __launch_bounds__(CfgN<B_MN>::THREADS, 1)
     cluster_sync_all();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
+    pdl_launch_dependents();
+    pdl_wait();
     const int conv_first_warp = 6, ppro_warp = 6 + CONV_WARPS;
 
     if (warp == 0) {
@@ -805,15 +786,18 @@ lsn_status launch_cfg(const CUtensorMap& a, const CUtensorMap& b, const CUtensor
     cfg.blockDim = dim3(C::THREADS);
     cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
+    int na = 0;
     if (PAIR) {
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 2;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = 2;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
     }
+    na += pdl_attr(&attr[na]);
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
     LSN_CUDA_TRY(cudaLaunchKernelEx(&cfg, lsn_gemm_kernel<PAIR, BN, B_MN, NF4>, a, b, la, lb, args));
     return LSN_OK;
 }
@@ -869,13 +853,13 @@ lsn_status launch_gemm_nf4(const uint16_t* A, int64_t lda, const lsn_nf4_weight*
         cfg.blockDim = dim3((unsigned)threads);
         cfg.dynamicSmemBytes = smem_bytes;
         cfg.stream = st;
-        cudaLaunchAttribute attr[1];
+        cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 2;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = 1 + pdl_attr(&attr[1]);
         LSN_CUDA_TRY(cudaLaunchKernelEx(&cfg, kernel, ma, mp, mla, args));
         return LSN_OK;
     };

@@ -30,6 +30,17 @@ struct TgSpec {
     float scale;
 };
 
+// Launch attribute of the hot-path kernels: programmatic dependent launch
+// when enabled (LSN_OPT_PDL), so a kernel's set-up overlaps the tail of the
+// kernel before it on the stream.  Returns the number of attributes written (0 or 1).
+bool pdl_enabled();
+inline int pdl_attr(cudaLaunchAttribute* a) {
+    if (!pdl_enabled()) return 0;
+    a->id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a->val.programmaticStreamSerializationAllowed = 1;
+    return 1;
+}
+
 size_t quantize_ws_bytes(int64_t rows, int64_t cols);
 lsn_status launch_quantize(const float* W, const lsn_nf4_weight* out, void* ws, size_t ws_bytes, cudaStream_t st);
 lsn_status launch_dequant(const lsn_nf4_weight* w, uint16_t* out, cudaStream_t st);

@@ -144,6 +144,8 @@ __global__ void __launch_bounds__(128) lora_down_kernel(const __grid_constant__ 
     const int64_t T = pb.T, Kd = pb.Kd;
     const int chunks_per_split = pb.cps, nsplit = pb.ns;
     const float scale = pb.scale;
+    pdl_launch_dependents();
+    pdl_wait();
     constexpr int R = L::R, NP = L::NP, WROWS = L::WROWS, WPITCH = L::WPITCH;
     extern __shared__ __align__(128) uint8_t dn_smem[];
     uint16_t* xs = reinterpret_cast<uint16_t*>(dn_smem);                 // [stage][64 rows][64], swizzled
@@ -322,6 +324,8 @@ __global__ void __launch_bounds__(128) lora_tgrad_kernel(const __grid_constant__
     const int nsplit = pb.ns, accumulate = pb.accumulate;
     const bool out_rk = pb.out_rk != 0;
     const float scale = pb.scale;
+    pdl_launch_dependents();
+    pdl_wait();
     constexpr int R = 8 * NT, GPITCH = L::GPITCH;
     extern __shared__ __align__(128) uint8_t tg_smem[];
     uint16_t* xs = reinterpret_cast<uint16_t*>(tg_smem);                 // [stage][32 tokens][128], swizzled
@@ -468,15 +472,18 @@ cudaError_t launch_split(Kern kernel, dim3 grid, size_t smem, cudaStream_t st, A
     cfg.blockDim = dim3(128);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
+    int na = 0;
     if (grid.y > 1) {
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = 1;
-        attr[0].val.clusterDim.y = grid.y;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = 1;
+        attr[na].val.clusterDim.y = grid.y;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
     }
+    na += pdl_attr(&attr[na]);
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
     return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 

@@ -189,4 +189,8 @@ def test_options(lib):
     assert lib.get_option(lib.LSN_OPT_LAYER_LANES) == 1
     lib.set_option(lib.LSN_OPT_LAYER_LANES, 2)
     assert lib.get_option(lib.LSN_OPT_FUSED_NF4) == 0
+    assert lib.get_option(lib.LSN_OPT_PDL) == 1
+    lib.set_option(lib.LSN_OPT_PDL, 0)
+    assert lib.get_option(lib.LSN_OPT_PDL) == 0
+    lib.set_option(lib.LSN_OPT_PDL, 1)
     assert lib.get_option(12345) == -1

@@ -172,3 +172,16 @@ def test_layer_lanes_option_gives_the_same_bits(lib):
         lib.set_option(lib.LSN_OPT_LAYER_LANES, 2)
     _equal(a, b)
     _equal(a, L.single())
+
+
+def test_dependent_launch_option_gives_the_same_bits(lib):
+    L = Layer(lib, SMALL, 190, 16, "nf4", seed=4)
+    a = L.layer()
+    lib.set_option(lib.LSN_OPT_PDL, 0)
+    try:
+        b = L.layer()
+        c = L.single()
+    finally:
+        lib.set_option(lib.LSN_OPT_PDL, 1)
+    _equal(a, b)
+    _equal(a, c)
