@@ -145,9 +145,17 @@ def run_ours(args):
     st_main = Stack(cfg, layers=L, tokens=T, mode="streamed", n_slots=args.slots, seed=synth.SEED + rank,
                     stream=stream, lanes=args.lanes, api=args.api)
     wanted = [m for m in args.modes.split(",") if m]
-    modes = ["streamed"] + [m for m in wanted if m in ("no_h2d", "resident", "proj") or m.startswith("streamed_T")]
+    modes = ["streamed"] + [m for m in wanted
+                            if m in ("no_h2d", "resident", "proj", "dpo", "recompute") or m.startswith("streamed_T")]
     mode_tokens = {m: T for m in modes}
+    mode_copies = {}
+    # Extra work of the step variants: the reference forward of preference
+    # training (base term only) and the recomputed forward of checkpointing.
+    base_flop = 2.0 * sum(K * N for _, K, N in cfg.projections) * T * L
+    fwd_flop = base_flop + 2.0 * cfg.rank * sum(K + N for _, K, N in cfg.projections) * T * L
+    mode_kwargs = {"dpo": {"reference": True}, "recompute": {"recompute": True}}
     for mode in modes:
+        kw = mode_kwargs.get(mode, {})
         if mode == "streamed":
             st = st_main
         elif mode == "proj":            # no_h2d through the per-projection calls on two lanes
@@ -155,16 +163,19 @@ def run_ours(args):
         elif mode.startswith("streamed_T"):   # the same stream of weights under a larger batch
             mode_tokens[mode] = int(mode[len("streamed_T"):])
             st = st_main.with_tokens(mode_tokens[mode], "streamed", n_slots=args.slots)
+        elif mode in ("dpo", "recompute"):    # step variants over the same streamed pool
+            st = st_main.with_mode("streamed", n_slots=args.slots)
         else:
             st = st_main.with_mode(mode)
         with torch.cuda.stream(stream):
             for _ in range(args.warmup):
-                st.step()
+                st.step(**kw)
         stream.synchronize()
         barrier()
         torch.cuda.synchronize()
+        ps0_mode = st.pool_stats()
         if mode == "streamed":
-            ps0 = st.pool_stats()
+            ps0 = ps0_mode
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         sampler = ClockSampler(local) if mode == "streamed" else None
@@ -174,7 +185,7 @@ def run_ours(args):
             t0.record(stream)
             h0 = time.perf_counter()
             for _ in range(args.steps):
-                st.step()
+                st.step(**kw)
             host_ms = (time.perf_counter() - h0) * 1e3 / args.steps
             t1.record(stream)
         t1.synchronize()
@@ -187,6 +198,9 @@ def run_ours(args):
         ms = t0.elapsed_time(t1) / args.steps
         ms = max_over_ranks(ms)
         results[mode] = ms
+        ps1_mode = st.pool_stats()
+        if ps0_mode and ps1_mode:
+            mode_copies[mode] = (ps1_mode["copies"] - ps0_mode["copies"]) / args.steps
         if mode == "streamed":
             ps1 = st.pool_stats()
             pool_stats = {k: ps1[k] - ps0[k] for k in ps1}
@@ -279,11 +293,20 @@ def run_ours(args):
     dq = kernel["dequant"]
     h2d_gbs = (pool_stats["bytes_copied"] / (pool_stats["copy_ms"] / 1e3) / 1e9
                if pool_stats and pool_stats["copy_ms"] > 0 else None)
+    def mode_flop_per_step(m):
+        f = flop_step * mode_tokens[m] / T
+        if m == "dpo":
+            f += base_flop
+        elif m == "recompute":
+            f += fwd_flop
+        return f
+
     extra_modes = {m: {"ms_per_step": results[m], "host_issue_ms_per_step": host_issue.get(m),
                        "tokens": mode_tokens[m],
                        "tok_s": world * mode_tokens[m] / (results[m] / 1e3),
-                       "pct_bf16_peak": 100 * flop_step * mode_tokens[m] / T / (results[m] / 1e3) / 1e12
-                       / peaks["bf16_tflops"]}
+                       "flop_per_step": mode_flop_per_step(m),
+                       "pct_bf16_peak": 100 * mode_flop_per_step(m) / (results[m] / 1e3) / 1e12 / peaks["bf16_tflops"],
+                       "layer_copies_per_step": mode_copies.get(m)}
                    for m in results}
     traffic = _traffic_from_profile()
     line = {
@@ -463,7 +486,7 @@ def main():
     ap.add_argument("--tokens", type=int, default=0, help="override T (default: the workload's 2048)")
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (default 32)")
     ap.add_argument("--slots", type=int, default=2)
-    ap.add_argument("--modes", default="no_h2d,resident,proj,streamed_T8192",
+    ap.add_argument("--modes", default="no_h2d,resident,proj,streamed_T8192,dpo,recompute",
                     help="extra modes timed after the streamed one (streamed_T<n>: streamed with n tokens)")
     ap.add_argument("--api", choices=["layer", "proj"], default="layer",
                     help="one library call per layer, or one per projection")

@@ -208,7 +208,11 @@ lsn_status lora_linear_bwd(const lsn_base* W, const uint16_t* x, const uint16_t*
  * kernel, their rank-r down projections one kernel, their dA/dB token
  * reductions one kernel.  The forward can keep u = x A^T, the low-rank
  * activation a LoRA layer saves for its backward pass, so the backward does
- * not read x again to rebuild it.
+ * not read x again to rebuild it.  A projection whose A and B are NULL runs
+ * with the adapter off: the streamed base alone, the reference model of
+ * preference training ("An 8B Fine-Tune Now Fits in 4 GB of VRAM": the
+ * streamed base with the adapters switched off is the reference); its
+ * output is bit for bit the base term of the adapter-on call.
  *
  * p is a HOST array of n descriptors, read during the call only; the
  * pointers inside are device pointers that must stay valid until the
@@ -221,8 +225,8 @@ lsn_status lora_linear_bwd(const lsn_base* W, const uint16_t* x, const uint16_t*
 typedef struct {
     lsn_base W;          /* frozen base [N, K] */
     const uint16_t* x;   /* [T, K] input */
-    const uint16_t* A;   /* [r, K] */
-    const uint16_t* B;   /* [N, r] */
+    const uint16_t* A;   /* [r, K]; A and B both NULL: the adapter is off for this projection */
+    const uint16_t* B;   /* [N, r]   (the frozen base alone: y = x W^T, dX = dY W; dA, dB, u unused) */
     uint16_t* y;         /* forward: output [T, N]; unused by the backward */
     const uint16_t* dY;  /* backward: output gradient [T, N]; unused by the forward */
     uint16_t* dX;        /* backward: input gradient [T, K], or NULL */

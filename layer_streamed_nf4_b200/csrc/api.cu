@@ -121,7 +121,7 @@ LoraWs carve(void* ws, int64_t T, int64_t K, int64_t N, int r, int kind) {
 }
 
 lsn_status check_proj(const lsn_base* W, const uint16_t* x, int64_t T, const uint16_t* A, const uint16_t* B, int r,
-                      const std::string& f) {
+                      const std::string& f, bool adapter_may_be_off = false) {
     LSN_CHECK_ARG(W != nullptr, f + ": base is NULL");
     LSN_CHECK_ARG(W->kind == LSN_BASE_NF4 || W->kind == LSN_BASE_BF16, f + ": unknown base kind");
     LSN_CHECK_ARG(T >= 0, f + ": T must be >= 0");
@@ -137,7 +137,8 @@ lsn_status check_proj(const lsn_base* W, const uint16_t* x, int64_t T, const uin
     } else {
         LSN_CHECK_ARG(W->bf16 != nullptr && aligned16(W->bf16), f + ": bf16 base must be a 16-byte aligned pointer");
     }
-    LSN_CHECK_ARG((x || T == 0) && A && B, f + ": NULL tensor");
+    const bool off = adapter_may_be_off && A == nullptr && B == nullptr;
+    LSN_CHECK_ARG((x || T == 0) && ((A && B) || off), f + ": NULL tensor");
     LSN_CHECK_ARG(aligned16(x) && aligned16(A) && aligned16(B), f + ": tensors must be 16-byte aligned");
     return LSN_OK;
 }
@@ -189,6 +190,8 @@ LayerWs carve_layer(void* ws, int n, const lsn_lora_proj* p, int64_t T, int r) {
     return w;
 }
 
+bool adapter_off(const lsn_lora_proj& q) { return q.A == nullptr && q.B == nullptr; }
+
 lsn_status check_layer(int n, const lsn_lora_proj* p, int64_t T, int r, void* ws, size_t ws_bytes, bool bwd,
                        const char* who) {
     const std::string f(who);
@@ -196,14 +199,14 @@ lsn_status check_layer(int n, const lsn_lora_proj* p, int64_t T, int r, void* ws
     LSN_CHECK_ARG(p != nullptr, f + ": projection array is NULL");
     for (int i = 0; i < n; ++i) {
         const std::string fi = f + ": projection " + std::to_string(i);
-        lsn_status s = check_proj(&p[i].W, p[i].x, T, p[i].A, p[i].B, r, fi);
+        lsn_status s = check_proj(&p[i].W, p[i].x, T, p[i].A, p[i].B, r, fi, true);
         if (s != LSN_OK) return s;
         LSN_CHECK_ARG(aligned16(p[i].u), fi + ": u must be 16-byte aligned");
         if (!bwd) {
             LSN_CHECK_ARG((p[i].y != nullptr || T == 0) && aligned16(p[i].y), fi + ": y must be a 16-byte aligned device pointer");
         } else {
             LSN_CHECK_ARG((p[i].dY != nullptr || T == 0) && aligned16(p[i].dY), fi + ": dY must be a 16-byte aligned device pointer");
-            LSN_CHECK_ARG(p[i].dA && p[i].dB && aligned16(p[i].dA) && aligned16(p[i].dB),
+            LSN_CHECK_ARG(adapter_off(p[i]) || (p[i].dA && p[i].dB && aligned16(p[i].dA) && aligned16(p[i].dB)),
                           fi + ": dA/dB must be 16-byte aligned device pointers");
             LSN_CHECK_ARG(aligned16(p[i].dX), fi + ": dX must be 16-byte aligned");
         }
@@ -466,23 +469,26 @@ lsn_status lora_layer_fwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
     const LayerWs w = carve_layer(ws, n, p, T, r);
     bool deq[LSN_LAYER_MAX_PROJ];
     DownSpec dn[LSN_LAYER_MAX_PROJ];
+    int nd = 0;
     for (int i = 0; i < n; ++i) {
         deq[i] = p[i].W.kind == LSN_BASE_NF4 && !fused_here(p[i].W, T, p[i].W.rows);
-        dn[i] = DownSpec{p[i].x, p[i].A, p[i].u, w.s16[i], T, p[i].W.cols, scale};
+        if (!adapter_off(p[i])) dn[nd++] = DownSpec{p[i].x, p[i].A, p[i].u, w.s16[i], T, p[i].W.cols, scale};
     }
     if ((s = layer_dequant(n, p, deq, w, st)) != LSN_OK) return s;
-    if ((s = timed_down_batch(n, dn, true, r, st)) != LSN_OK) return s;
+    if ((s = timed_down_batch(nd, dn, true, r, st)) != LSN_OK) return s;
     // The GEMMs of the projections are independent: alternate them over two lanes.
     LaneScope lanes(st, n > 1 && g_layer_lanes.load() == 2);
     for (int i = 0; i < n; ++i) {
         const int64_t N = p[i].W.rows, K = p[i].W.cols;
         const cudaStream_t gs = (i & 1) ? lanes.side() : lanes.main();
+        const int ri = adapter_off(p[i]) ? 0 : r;       // no LoRA K-block with the adapter off
         if (fused_here(p[i].W, T, N)) {
-            TimingScope ts(LSN_K_GEMM_FWD, 2.0 * T * N * (double)(K + r), gs);
-            s = launch_gemm_nf4(p[i].x, K, &p[i].W.nf4, false, w.s16[i], p[i].B, r, T, N, K, p[i].y, N, w.err, gs);
+            TimingScope ts(LSN_K_GEMM_FWD, 2.0 * T * N * (double)(K + ri), gs);
+            s = launch_gemm_nf4(p[i].x, K, &p[i].W.nf4, false, w.s16[i], p[i].B, ri, T, N, K, p[i].y, N, w.err, gs);
         } else {
             const uint16_t* Wb = p[i].W.kind == LSN_BASE_NF4 ? w.w16[i] : p[i].W.bf16;
-            s = timed_gemm(LSN_K_GEMM_FWD, p[i].x, K, Wb, K, false, w.s16[i], p[i].B, r, T, N, K, p[i].y, N, w.err, gs);
+            s = timed_gemm(LSN_K_GEMM_FWD, p[i].x, K, Wb, K, false, w.s16[i], p[i].B, ri, T, N, K, p[i].y, N, w.err,
+                           gs);
         }
         if (s != LSN_OK) return s;
     }
@@ -499,39 +505,44 @@ lsn_status lora_layer_bwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
     if (T > 0) {
         bool deq[LSN_LAYER_MAX_PROJ];
         DownSpec dg[LSN_LAYER_MAX_PROJ], du[LSN_LAYER_MAX_PROJ];
-        int nu = 0;
+        int ng = 0, nu = 0;
         for (int i = 0; i < n; ++i) {
             const int64_t N = p[i].W.rows, K = p[i].W.cols;
             deq[i] = p[i].dX && p[i].W.kind == LSN_BASE_NF4 && !fused_here(p[i].W, T, K);
-            dg[i] = DownSpec{p[i].dY, p[i].B, w.g32[i], w.s16[i], T, N, scale};
+            if (adapter_off(p[i])) continue;
+            dg[ng++] = DownSpec{p[i].dY, p[i].B, w.g32[i], w.s16[i], T, N, scale};
             if (!p[i].u) du[nu++] = DownSpec{p[i].x, p[i].A, w.u32[i], nullptr, T, K, scale};
         }
         if ((s = layer_dequant(n, p, deq, w, st)) != LSN_OK) return s;
-        if ((s = timed_down_batch(n, dg, false, r, st)) != LSN_OK) return s;
+        if ((s = timed_down_batch(ng, dg, false, r, st)) != LSN_OK) return s;
         if ((s = timed_down_batch(nu, du, true, r, st)) != LSN_OK) return s;
     }
     // dA and dB of every projection in one launch (with T == 0: zeros, or the
     // accumulators left as they are).  They need only g and u, so with two
     // lanes they run on the side stream beside the input-gradient GEMMs.
     TgSpec tg[2 * LSN_LAYER_MAX_PROJ];
+    int nt = 0;
     for (int i = 0; i < n; ++i) {
+        if (adapter_off(p[i])) continue;                // no adapter, no adapter gradients
         const int64_t N = p[i].W.rows, K = p[i].W.cols;
-        tg[2 * i] = TgSpec{w.g32[i], p[i].x, p[i].dA, T, K, true, accumulate, scale};
-        tg[2 * i + 1] = TgSpec{p[i].u ? p[i].u : w.u32[i], p[i].dY, p[i].dB, T, N, false, accumulate, scale};
+        tg[nt++] = TgSpec{w.g32[i], p[i].x, p[i].dA, T, K, true, accumulate, scale};
+        tg[nt++] = TgSpec{p[i].u ? p[i].u : w.u32[i], p[i].dY, p[i].dB, T, N, false, accumulate, scale};
     }
     LaneScope lanes(st, T > 0 && g_layer_lanes.load() == 2);
-    if ((s = timed_tgrad_batch(2 * n, tg, r, lanes.side())) != LSN_OK) return s;
+    if ((s = timed_tgrad_batch(nt, tg, r, lanes.side())) != LSN_OK) return s;
     if (T > 0) {
         for (int i = 0, j = 0; i < n; ++i) {
             if (!p[i].dX) continue;
             const int64_t N = p[i].W.rows, K = p[i].W.cols;
             const cudaStream_t gs = (j++ & 1) ? lanes.side() : lanes.main();
+            const int ri = adapter_off(p[i]) ? 0 : r;
             if (fused_here(p[i].W, T, K)) {
-                TimingScope ts(LSN_K_GEMM_BWD, 2.0 * T * K * (double)(N + r), gs);
-                s = launch_gemm_nf4(p[i].dY, N, &p[i].W.nf4, true, w.s16[i], p[i].A, r, T, K, N, p[i].dX, K, w.err, gs);
+                TimingScope ts(LSN_K_GEMM_BWD, 2.0 * T * K * (double)(N + ri), gs);
+                s = launch_gemm_nf4(p[i].dY, N, &p[i].W.nf4, true, w.s16[i], p[i].A, ri, T, K, N, p[i].dX, K, w.err,
+                                    gs);
             } else {
                 const uint16_t* Wb = p[i].W.kind == LSN_BASE_NF4 ? w.w16[i] : p[i].W.bf16;
-                s = timed_gemm(LSN_K_GEMM_BWD, p[i].dY, N, Wb, K, true, w.s16[i], p[i].A, r, T, K, N, p[i].dX, K,
+                s = timed_gemm(LSN_K_GEMM_BWD, p[i].dY, N, Wb, K, true, w.s16[i], p[i].A, ri, T, K, N, p[i].dX, K,
                                w.err, gs);
             }
             if (s != LSN_OK) return s;

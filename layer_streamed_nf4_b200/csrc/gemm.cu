@@ -826,7 +826,11 @@ lsn_status launch_gemm_nf4(const uint16_t* A, int64_t lda, const lsn_nf4_weight*
     if ((s = make_map(&ma, A, Kc, M, lda, SUB, BM)) != LSN_OK) return s;
     // packed [wrows, wcols/2] bytes, boxes of 64 bytes x 128 rows
     if ((s = make_map(&mp, w->packed, w->cols / 2, w->rows, w->cols / 2, 64, 128, true)) != LSN_OK) return s;
-    if ((s = make_map(&mla, LA, r, M, r, SUB, BM)) != LSN_OK) return s;
+    if (r > 0) {
+        if ((s = make_map(&mla, LA, r, M, r, SUB, BM)) != LSN_OK) return s;
+    } else {
+        mla = ma;                                   // no LoRA term: never read
+    }
     GemmArgs args{};
     args.M = (int)M;
     args.N = (int)N;
@@ -895,11 +899,16 @@ lsn_status launch_gemm(const uint16_t* A, int64_t lda, const uint16_t* B, int64_
     } else {
         if ((s = make_map(&mb, B, N, Kc, ldb, 64, BK)) != LSN_OK) return s;
     }
-    if ((s = make_map(&mla, LA, r, M, r, SUB, BM)) != LSN_OK) return s;
-    if (!b_mn) {
-        if ((s = make_map(&mlb, LB, r, N, r, SUB, b_rows)) != LSN_OK) return s;
-    } else {
-        if ((s = make_map(&mlb, LB, N, r, N, 64, BK)) != LSN_OK) return s;
+    if (r > 0) {
+        if ((s = make_map(&mla, LA, r, M, r, SUB, BM)) != LSN_OK) return s;
+        if (!b_mn) {
+            if ((s = make_map(&mlb, LB, r, N, r, SUB, b_rows)) != LSN_OK) return s;
+        } else {
+            if ((s = make_map(&mlb, LB, N, r, N, 64, BK)) != LSN_OK) return s;
+        }
+    } else {                                        // no LoRA term: the maps are never read
+        mla = ma;
+        mlb = mb;
     }
     GemmArgs args{};
     args.M = (int)M;

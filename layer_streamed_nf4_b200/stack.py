@@ -142,6 +142,8 @@ class Stack:
                   for l in range(nl) for pi, p in enumerate(self.proj)}
         self.dX = {(l, pi): torch.empty((T, p.K), dtype=torch.bfloat16, device=dev)
                    for l in range(nl) for pi, p in enumerate(self.proj)}
+        self.y_ref = {(l, pi): torch.empty((T, p.N), dtype=torch.bfloat16, device=dev)
+                      for l in range(nl) for pi, p in enumerate(self.proj)}
         if self.api == "layer":
             # u = x A^T kept from the forward for the backward, per (layer, projection)
             self.u = {(l, pi): torch.zeros((T, r), dtype=torch.float32, device=dev)
@@ -281,46 +283,54 @@ class Stack:
             self._calls[key] = a
         return a
 
-    def _layer_projs(self, addr: int, l: int):
-        """The lsn_lora_proj array of layer l whose blob sits at addr (cached: it depends on nothing else)."""
-        key = ("L", addr, l)
+    def _layer_projs(self, addr: int, l: int, adapter: bool = True):
+        """The lsn_lora_proj array of layer l whose blob sits at addr (cached: it depends on nothing else).
+        adapter=False: A and B NULL, the frozen base alone (the reference model of preference training)."""
+        key = ("L", addr, l, adapter)
         a = self._calls.get(key)
         if a is None:
-            projs = [lsnf4.lora_proj(self._base(addr, p), self.x[l, pi], self.A[l, pi], self.B[l, pi],
-                                     y=self._out(self.y, l, pi), dY=self.dY[l, pi], dX=self._out(self.dX, l, pi),
-                                     dA=self.dA[l, pi], dB=self.dB[l, pi],
-                                     u=self.u[l, pi] if hasattr(self, "u") else None)
+            projs = [lsnf4.lora_proj(self._base(addr, p), self.x[l, pi],
+                                     self.A[l, pi] if adapter else None, self.B[l, pi] if adapter else None,
+                                     y=self._out(self.y if adapter else self.y_ref, l, pi), dY=self.dY[l, pi],
+                                     dX=self._out(self.dX, l, pi), dA=self.dA[l, pi], dB=self.dB[l, pi],
+                                     u=self.u[l, pi] if (adapter and hasattr(self, "u")) else None)
                      for pi, p in enumerate(self.proj)]
             a = lsnf4.proj_array(projs)
             if addr:
                 self._calls[key] = a
         return a
 
-    def _forward_layers(self):
+    def _forward_layers(self, adapter: bool = True):
         fwd = lsnf4._lib.lora_layer_fwd
         n, ws, nb, sp = len(self.proj), self.ws[0].data_ptr(), self.ws_bytes, self.stream.cuda_stream
         for l in range(self.L):
             addr = self._acquire(l)
             self._prefetch(l + 1)
-            st = fwd(n, self._layer_projs(addr, l), self.T, self.r, self.scale, ws, nb, sp)
+            st = fwd(n, self._layer_projs(addr, l, adapter), self.T, self.r, self.scale, ws, nb, sp)
             if st:
                 lsnf4._check(st, "lora_layer_fwd")
             self._release(l)
 
-    def _backward_layers(self, accumulate: bool):
-        bwd = lsnf4._lib.lora_layer_bwd
+    def _backward_layers(self, accumulate: bool, recompute: bool = False):
+        fwd, bwd = lsnf4._lib.lora_layer_fwd, lsnf4._lib.lora_layer_bwd
         n, ws, nb, sp = len(self.proj), self.ws[0].data_ptr(), self.ws_bytes, self.stream.cuda_stream
         for l in reversed(range(self.L)):
             addr = self._acquire(l)
             self._prefetch(l - 1)
-            st = bwd(n, self._layer_projs(addr, l), self.T, self.r, self.scale, int(accumulate), ws, nb, sp)
+            projs = self._layer_projs(addr, l)
+            if recompute:     # the layer's forward again, inside the backward sweep (activation checkpointing)
+                st = fwd(n, projs, self.T, self.r, self.scale, ws, nb, sp)
+                if st:
+                    lsnf4._check(st, "lora_layer_fwd")
+            st = bwd(n, projs, self.T, self.r, self.scale, int(accumulate), ws, nb, sp)
             if st:
                 lsnf4._check(st, "lora_layer_bwd")
             self._release(l)
 
-    def forward(self):
+    def forward(self, adapter: bool = True):
         if self.api == "layer":
-            return self._forward_layers()
+            return self._forward_layers(adapter)
+        assert adapter, "the adapter-off forward runs through the layer calls"
         fwd = lsnf4._lib.lora_linear_fwd
         for l in range(self.L):
             addr = self._acquire(l)
@@ -333,9 +343,10 @@ class Stack:
             self._join_lanes()
             self._release(l)
 
-    def backward(self, accumulate: bool = False):
+    def backward(self, accumulate: bool = False, recompute: bool = False):
         if self.api == "layer":
-            return self._backward_layers(accumulate)
+            return self._backward_layers(accumulate, recompute)
+        assert not recompute, "the recomputing backward runs through the layer calls"
         bwd = lsnf4._lib.lora_linear_bwd
         for l in reversed(range(self.L)):
             addr = self._acquire(l)
@@ -348,9 +359,14 @@ class Stack:
             self._join_lanes()
             self._release(l)
 
-    def step(self, accumulate: bool = False):
+    def step(self, accumulate: bool = False, reference: bool = False, recompute: bool = False):
+        """One training step.  reference: first a forward sweep with the adapters off (the reference model
+        of preference training, read from the same stream of layers); recompute: every layer's forward runs
+        again inside the backward sweep, as with activation checkpointing."""
+        if reference:
+            self.forward(adapter=False)
         self.forward()
-        self.backward(accumulate)
+        self.backward(accumulate, recompute)
 
     # ------------------------------------------------------------ facts ---
 

@@ -185,3 +185,34 @@ def test_dependent_launch_option_gives_the_same_bits(lib):
         lib.set_option(lib.LSN_OPT_PDL, 1)
     _equal(a, b)
     _equal(a, c)
+
+
+def test_adapter_off_is_the_base_term(lib, orc):
+    """A projection with A = B = NULL gives exactly the base term: the adapter-on call with B = 0 (whose
+    LoRA K-block adds exact zeros) and, within tolerance, the oracle's x W^T."""
+    import torch
+    L = Layer(lib, SMALL[:4], 150, 16, "nf4", seed=6)
+    ref = L.outputs()
+    off = L.outputs()
+    for d in L.p:
+        d["B"].zero_()
+    projs_on = [lib.lora_proj(d["base"], d["x"], d["A"], d["B"], y=o["y"], dY=d["dY"], dX=o["dX"], dA=o["dA"],
+                              dB=o["dB"]) for d, o in zip(L.p, ref)]
+    projs_off = [lib.lora_proj(d["base"], d["x"], None, None, y=o["y"], dY=d["dY"], dX=o["dX"])
+                 for d, o in zip(L.p, off)]
+    for projs in (projs_on, projs_off):
+        arr = lib.proj_array(projs)
+        n = lib.layer_ws_bytes(arr, L.T, L.r)
+        ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
+        lib.lora_layer_fwd(arr, L.T, L.r, L.scale, ws, n)
+        lib.lora_layer_bwd(arr, L.T, L.r, L.scale, False, ws, n)
+        torch.cuda.synchronize()
+        lib.ws_status(ws)
+    # dX of the adapter-on call with B = 0 is dY W + s (dY 0) A: the base term again
+    _equal(off, ref, ("y", "dX"))
+    for d, o in zip(L.p, off):
+        c = d["case"]
+        q = orc.nf4_quantize(c.W)
+        Wb = orc.nf4_dequant(q["packed"], q["absmax_q"], q["s2"], q["offset"], c.W.size).reshape(c.W.shape)
+        zeroB = np.zeros_like(c.B)
+        assert_close(bf16_tensor_to_f64(o["y"]), orc.lora_fwd(c.x, Wb, c.A, zeroB, L.scale), "y (adapter off)")

@@ -88,6 +88,29 @@ def test_lane_count_does_not_change_results(lib, name, layers, tokens):
     one.close()
 
 
+def test_recompute_and_reference_steps(lib):
+    """A backward that recomputes each layer's forward, and a step that first runs the adapter-off
+    reference forward, give the same y, dX, dA, dB as the plain step; the reference outputs are the
+    base term (equal to an adapter-on forward with B = 0)."""
+    import torch
+    cfg = synth.STACKS["8b"]
+    plain = _run(cfg, 3, 256, "streamed")
+    from layer_streamed_nf4_b200.stack import Stack
+    st = Stack(cfg, layers=3, tokens=256, mode="streamed", keep_outputs=True)
+    st.step(reference=True, recompute=True)
+    torch.cuda.synchronize()
+    st.check_status()
+    fwd, bwd, bad = _compare(st, plain)
+    assert fwd and bwd, bad
+    for k in st.B:
+        st.B[k].zero_()
+    st.forward()
+    torch.cuda.synchronize()
+    assert all(torch.equal(st.y[k], st.y_ref[k]) for k in st.y)
+    st.close()
+    plain.close()
+
+
 def test_no_h2d_equals_resident(lib):
     cfg = synth.STACKS["8b"]
     res = _run(cfg, 3, 512, "resident")
