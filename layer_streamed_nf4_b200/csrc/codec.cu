@@ -212,11 +212,19 @@ struct DqBatch {
 // 128-bit words of packed codes (coalesced across the warp, all four in
 // flight at once), builds the block's 16 scaled levels bf16(level *
 // absmax_hat) in registers and maps the 32 codes of a word onto them with
-// byte permutes (no shared-memory lookup per element), writing 64 bytes of
-// bf16 per word.  A block covers 1024 consecutive words of one weight.
+// byte permutes (no shared-memory lookup per element).  The 64 bytes of bf16
+// a thread makes for one word are passed through a per-warp staging buffer
+// in shared memory (16-byte chunks XOR-swizzled, conflict-free both ways) so
+// that every global store instruction of the warp writes 512 contiguous
+// bytes.  A block covers 1024 consecutive words of one weight.
+constexpr int kDqWarps = kDqThreads / 32;
+
+__device__ __forceinline__ int dq_stage_chunk(int c) { return c ^ ((c >> 3) & 7); }
+
 __global__ void __launch_bounds__(kDqThreads) nf4_dequant_kernel(const __grid_constant__ DqBatch bt,
                                                                  const __grid_constant__ DequantParams P) {
     __shared__ float dq[256];
+    __shared__ uint4 stage[kDqWarps][128];                 // 2 KB per warp: 32 lanes x 64 bytes
     for (int i = threadIdx.x; i < 256; i += blockDim.x) dq[i] = P.dq[i];
     int ii = 0;
     while (ii + 1 < bt.n && (int64_t)blockIdx.x >= bt.it[ii + 1].first) ++ii;
@@ -228,6 +236,7 @@ __global__ void __launch_bounds__(kDqThreads) nf4_dequant_kernel(const __grid_co
     const float* __restrict__ s2 = it.s2;
     uint4* __restrict__ out = it.out;
     const float off = *it.offset;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int64_t v0 = ((int64_t)blockIdx.x - it.first) * kDqVecPerBlock + threadIdx.x;
     uint4 p[kDqUnroll];
     uint32_t code[kDqUnroll];
@@ -242,17 +251,26 @@ __global__ void __launch_bounds__(kDqThreads) nf4_dequant_kernel(const __grid_co
         sc[u] = __ldg(s2 + (b >> 8));
     }
     __syncthreads();                                     // the code table is in shared memory
+    uint4* st = stage[warp];
     #pragma unroll
     for (int u = 0; u < kDqUnroll; ++u) {
-        const int64_t v = v0 + u * kDqThreads;
-        if (v >= it.nvec) break;
         const float ah = __fadd_rn(__fmul_rn(dq[code[u]], sc[u]), off);
         uint32_t lo[4], hi[4];
         nf4_scaled_table(P.level, ah, lo, hi);
-        out[v * 4 + 0] = nf4x8_to_bf16(p[u].x, lo, hi);
-        out[v * 4 + 1] = nf4x8_to_bf16(p[u].y, lo, hi);
-        out[v * 4 + 2] = nf4x8_to_bf16(p[u].z, lo, hi);
-        out[v * 4 + 3] = nf4x8_to_bf16(p[u].w, lo, hi);
+        st[dq_stage_chunk(4 * lane + 0)] = nf4x8_to_bf16(p[u].x, lo, hi);
+        st[dq_stage_chunk(4 * lane + 1)] = nf4x8_to_bf16(p[u].y, lo, hi);
+        st[dq_stage_chunk(4 * lane + 2)] = nf4x8_to_bf16(p[u].z, lo, hi);
+        st[dq_stage_chunk(4 * lane + 3)] = nf4x8_to_bf16(p[u].w, lo, hi);
+        __syncwarp();
+        // The warp's 32 consecutive words start at word w0; their output is
+        // 2 KB at out + 4 * w0, written as four 512-byte rows.
+        const int64_t w0 = v0 - lane + u * kDqThreads;
+        #pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int c = 32 * i + lane;                 // output chunk of the warp, in 16-byte units
+            if (w0 + (c >> 2) < it.nvec) out[4 * w0 + c] = st[dq_stage_chunk(c)];
+        }
+        __syncwarp();
     }
 }
 
