@@ -290,6 +290,15 @@ class LaneScope {
     }
     cudaStream_t main() const { return st_; }
     cudaStream_t side() const { return lane_ ? lane_->side : st_; }
+    // Both lanes continue only after everything enqueued so far on either.
+    lsn_status barrier() {
+        if (!lane_) return LSN_OK;
+        LSN_CUDA_TRY(cudaEventRecord(lane_->fork, st_));
+        LSN_CUDA_TRY(cudaEventRecord(lane_->join, lane_->side));
+        LSN_CUDA_TRY(cudaStreamWaitEvent(st_, lane_->join, 0));
+        LSN_CUDA_TRY(cudaStreamWaitEvent(lane_->side, lane_->fork, 0));
+        return LSN_OK;
+    }
     // Join: the caller's stream waits for everything enqueued on the side stream.
     lsn_status join() {
         if (!lane_) return LSN_OK;
@@ -474,10 +483,13 @@ lsn_status lora_layer_fwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
         deq[i] = p[i].W.kind == LSN_BASE_NF4 && !fused_here(p[i].W, T, p[i].W.rows);
         if (!adapter_off(p[i])) dn[nd++] = DownSpec{p[i].x, p[i].A, p[i].u, w.s16[i], T, p[i].W.cols, scale};
     }
-    if ((s = layer_dequant(n, p, deq, w, st)) != LSN_OK) return s;
-    if ((s = timed_down_batch(nd, dn, true, r, st)) != LSN_OK) return s;
-    // The GEMMs of the projections are independent: alternate them over two lanes.
-    LaneScope lanes(st, n > 1 && g_layer_lanes.load() == 2);
+    // Two lanes: the down projections (bound by reading x) run beside the
+    // dequantisation (bound by writing W); then the GEMMs, which are
+    // independent of each other, alternate over the lanes.
+    LaneScope lanes(st, g_layer_lanes.load() == 2);
+    if ((s = timed_down_batch(nd, dn, true, r, lanes.side())) != LSN_OK) return s;
+    if ((s = layer_dequant(n, p, deq, w, lanes.main())) != LSN_OK) return s;
+    if ((s = lanes.barrier()) != LSN_OK) return s;
     for (int i = 0; i < n; ++i) {
         const int64_t N = p[i].W.rows, K = p[i].W.cols;
         const cudaStream_t gs = (i & 1) ? lanes.side() : lanes.main();
@@ -502,6 +514,10 @@ lsn_status lora_layer_bwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
     if ((s = check_device()) != LSN_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const LayerWs w = carve_layer(ws, n, p, T, r);
+    // Two lanes: the down projections (reading dY, and x when no u was kept)
+    // run beside the dequantisation; then the token reductions run on the
+    // side lane beside the input-gradient GEMMs, which alternate over both.
+    LaneScope lanes(st, T > 0 && g_layer_lanes.load() == 2);
     if (T > 0) {
         bool deq[LSN_LAYER_MAX_PROJ];
         DownSpec dg[LSN_LAYER_MAX_PROJ], du[LSN_LAYER_MAX_PROJ];
@@ -513,13 +529,13 @@ lsn_status lora_layer_bwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
             dg[ng++] = DownSpec{p[i].dY, p[i].B, w.g32[i], w.s16[i], T, N, scale};
             if (!p[i].u) du[nu++] = DownSpec{p[i].x, p[i].A, w.u32[i], nullptr, T, K, scale};
         }
-        if ((s = layer_dequant(n, p, deq, w, st)) != LSN_OK) return s;
-        if ((s = timed_down_batch(ng, dg, false, r, st)) != LSN_OK) return s;
-        if ((s = timed_down_batch(nu, du, true, r, st)) != LSN_OK) return s;
+        if ((s = timed_down_batch(ng, dg, false, r, lanes.side())) != LSN_OK) return s;
+        if ((s = timed_down_batch(nu, du, true, r, lanes.side())) != LSN_OK) return s;
+        if ((s = layer_dequant(n, p, deq, w, lanes.main())) != LSN_OK) return s;
+        if ((s = lanes.barrier()) != LSN_OK) return s;
     }
     // dA and dB of every projection in one launch (with T == 0: zeros, or the
-    // accumulators left as they are).  They need only g and u, so with two
-    // lanes they run on the side stream beside the input-gradient GEMMs.
+    // accumulators left as they are); they need only g and u.
     TgSpec tg[2 * LSN_LAYER_MAX_PROJ];
     int nt = 0;
     for (int i = 0; i < n; ++i) {
@@ -528,7 +544,6 @@ lsn_status lora_layer_bwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
         tg[nt++] = TgSpec{w.g32[i], p[i].x, p[i].dA, T, K, true, accumulate, scale};
         tg[nt++] = TgSpec{p[i].u ? p[i].u : w.u32[i], p[i].dY, p[i].dB, T, N, false, accumulate, scale};
     }
-    LaneScope lanes(st, T > 0 && g_layer_lanes.load() == 2);
     if ((s = timed_tgrad_batch(nt, tg, r, lanes.side())) != LSN_OK) return s;
     if (T > 0) {
         for (int i = 0, j = 0; i < n; ++i) {
