@@ -146,7 +146,8 @@ def run_ours(args):
                     stream=stream, lanes=args.lanes, api=args.api)
     wanted = [m for m in args.modes.split(",") if m]
     modes = ["streamed"] + [m for m in wanted
-                            if m in ("no_h2d", "resident", "proj", "dpo", "recompute") or m.startswith("streamed_T")]
+                            if m in ("no_h2d", "resident", "proj", "dpo", "recompute", "shared", "grouped")
+                            or m.startswith("streamed_T")]
     mode_tokens = {m: T for m in modes}
     mode_copies = {}
     # Extra work of the step variants: the reference forward of preference
@@ -165,6 +166,8 @@ def run_ours(args):
             st = st_main.with_tokens(mode_tokens[mode], "streamed", n_slots=args.slots)
         elif mode in ("dpo", "recompute"):    # step variants over the same streamed pool
             st = st_main.with_mode("streamed", n_slots=args.slots)
+        elif mode in ("shared", "grouped"):   # q|k|v and gate|up read one input each (no_h2d pool)
+            st = st_main.with_inputs(shared_inputs=True, grouped=(mode == "grouped"))
         else:
             st = st_main.with_mode(mode)
         with torch.cuda.stream(stream):
@@ -486,7 +489,7 @@ def main():
     ap.add_argument("--tokens", type=int, default=0, help="override T (default: the workload's 2048)")
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (default 32)")
     ap.add_argument("--slots", type=int, default=2)
-    ap.add_argument("--modes", default="no_h2d,resident,proj,streamed_T8192,dpo,recompute",
+    ap.add_argument("--modes", default="no_h2d,resident,proj,streamed_T8192,dpo,recompute,shared,grouped",
                     help="extra modes timed after the streamed one (streamed_T<n>: streamed with n tokens)")
     ap.add_argument("--api", choices=["layer", "proj"], default="layer",
                     help="one library call per layer, or one per projection")

@@ -214,6 +214,17 @@ lsn_status lora_linear_bwd(const lsn_base* W, const uint16_t* x, const uint16_t*
  * streamed base with the adapters switched off is the reference); its
  * output is bit for bit the base term of the adapter-on call.
  *
+ * Groups.  Projections that read the same input (q, k, v of attention; gate
+ * and up of the MLP) can be marked as a group: consecutive entries with the
+ * same positive `group`, at most 4, sharing the x pointer, K, base kind and
+ * adapter state, with group size x r <= 64; bf16 bases of a group must lie
+ * back to back in memory (as in a layer blob).  The forward computes the
+ * group as one GEMM over the stacked weights (outputs routed to each y; the
+ * same bits as ungrouped).  The backward computes the group's input gradient
+ * sum_j (dY_j W_j + s (dY_j B_j) A_j) as one GEMM and writes it to the first
+ * member's dX (the other members' dX must be NULL); dA and dB are per member
+ * and the same bits as ungrouped.
+ *
  * p is a HOST array of n descriptors, read during the call only; the
  * pointers inside are device pointers that must stay valid until the
  * enqueued work has finished.  Projections may have different K and N but
@@ -235,6 +246,8 @@ typedef struct {
     float* u;            /* fp32 [T, r] = x A^T, or NULL.  Forward: written when non-NULL.
                             Backward: read when non-NULL (it must hold what the forward
                             wrote for the same x and A), recomputed when NULL. */
+    int group;           /* 0, or a group id: consecutive projections with the same positive id
+                            form a group (see below) */
 } lsn_lora_proj;
 
 /* Workspace bytes of lora_layer_fwd / lora_layer_bwd for these projections

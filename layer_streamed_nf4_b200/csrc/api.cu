@@ -163,13 +163,43 @@ double dequant_bytes(int64_t N, int64_t K) {
 //   s16 bf16 [T, r]  bf16(s u_i) (forward) or bf16(s g_i) (backward)
 //   g32 fp32 [T, r]  dY_i B_i
 //   u32 fp32 [T, r]  x_i A_i^T when the caller keeps no u
+// then per group (led by its first member g):
+//   la  bf16 [T, m r]        the members' bf16(s u) or bf16(s g), side by side
+//   lb  bf16 [N_sum, m r]    forward: block-diagonal of the members' B
+//       bf16 [m r, K]        backward: the members' A stacked
+// and last, back to back in projection order (so a group's stack is one
+// matrix):
 //   w16 bf16 [N, K]  dequantised base (NF4 bases only)
+
+// The groups of a layer call: group k spans projections first[k] ..
+// first[k] + count[k] - 1 (ungrouped projections are groups of one).
+struct Groups {
+    int n = 0;
+    int first[LSN_LAYER_MAX_PROJ];
+    int count[LSN_LAYER_MAX_PROJ];
+};
+
+Groups find_groups(int n, const lsn_lora_proj* p) {
+    Groups g;
+    for (int i = 0; i < n;) {
+        int j = i + 1;
+        if (p[i].group > 0)
+            while (j < n && p[j].group == p[i].group && j - i < kGemmMaxSeg) ++j;
+        g.first[g.n] = i;
+        g.count[g.n++] = j - i;
+        i = j;
+    }
+    return g;
+}
+
 struct LayerWs {
     int* err;
     uint16_t* s16[LSN_LAYER_MAX_PROJ];
     float* g32[LSN_LAYER_MAX_PROJ];
     float* u32[LSN_LAYER_MAX_PROJ];
     uint16_t* w16[LSN_LAYER_MAX_PROJ];
+    uint16_t* la[LSN_LAYER_MAX_PROJ];   // per group leader
+    uint16_t* lb[LSN_LAYER_MAX_PROJ];   // per group leader
     size_t total;
 };
 
@@ -183,6 +213,19 @@ LayerWs carve_layer(void* ws, int n, const lsn_lora_proj* p, int64_t T, int r) {
         w.s16[i] = reinterpret_cast<uint16_t*>(take((size_t)T * r * 2));
         w.g32[i] = reinterpret_cast<float*>(take((size_t)T * r * 4));
         w.u32[i] = reinterpret_cast<float*>(take((size_t)T * r * 4));
+    }
+    const Groups g = find_groups(n, p);
+    for (int k = 0; k < g.n; ++k) {
+        if (g.count[k] < 2) continue;
+        const int i0 = g.first[k], m = g.count[k];
+        int64_t nsum = 0;
+        for (int j = 0; j < m; ++j) nsum += p[i0 + j].W.rows;
+        const int64_t K = p[i0].W.cols;
+        w.la[i0] = reinterpret_cast<uint16_t*>(take((size_t)T * m * r * 2));
+        const int64_t lb_elems = nsum * m * r > (int64_t)m * r * K ? nsum * m * r : (int64_t)m * r * K;
+        w.lb[i0] = reinterpret_cast<uint16_t*>(take((size_t)lb_elems * 2));
+    }
+    for (int i = 0; i < n; ++i) {
         const bool nf4 = p[i].W.kind == LSN_BASE_NF4;
         w.w16[i] = reinterpret_cast<uint16_t*>(take(nf4 ? (size_t)p[i].W.rows * p[i].W.cols * 2 : 0));
     }
@@ -210,6 +253,26 @@ lsn_status check_layer(int n, const lsn_lora_proj* p, int64_t T, int r, void* ws
                           fi + ": dA/dB must be 16-byte aligned device pointers");
             LSN_CHECK_ARG(aligned16(p[i].dX), fi + ": dX must be 16-byte aligned");
         }
+    }
+    const Groups g = find_groups(n, p);
+    for (int k = 0; k < g.n; ++k) {
+        const int i0 = g.first[k], m = g.count[k];
+        if (m < 2) continue;
+        const std::string fg = f + ": group of projections " + std::to_string(i0) + ".." + std::to_string(i0 + m - 1);
+        LSN_CHECK_ARG(m * r <= 64, fg + ": group size x rank must be <= 64");
+        for (int j = 1; j < m; ++j) {
+            const lsn_lora_proj& a = p[i0 + j - 1];
+            const lsn_lora_proj& q = p[i0 + j];
+            LSN_CHECK_ARG(q.x == p[i0].x && q.W.cols == p[i0].W.cols && q.W.kind == p[i0].W.kind &&
+                              adapter_off(q) == adapter_off(p[i0]),
+                          fg + ": members must share x, K, base kind and adapter state");
+            if (q.W.kind == LSN_BASE_BF16)
+                LSN_CHECK_ARG(q.W.bf16 == a.W.bf16 + a.W.rows * a.W.cols,
+                              fg + ": bf16 bases of a group must lie back to back");
+            if (bwd) LSN_CHECK_ARG(q.dX == nullptr, fg + ": only the first member has a dX (the group's sum)");
+        }
+        for (int j = 0; j + 1 < m && bwd; ++j)
+            LSN_CHECK_ARG(p[i0 + j].W.rows % 128 == 0, fg + ": N of all but the last member must be a multiple of 128");
     }
     LSN_CHECK_ARG(ws != nullptr && aligned16(ws), f + ": workspace must be a 16-byte aligned device pointer");
     const size_t need = carve_layer(nullptr, n, p, T, r).total;
@@ -468,6 +531,32 @@ size_t lsn_layer_ws_bytes(int n, const lsn_lora_proj* p, int64_t T, int r) {
     return carve_layer(nullptr, n, p, T, r).total;
 }
 
+// The LoRA operand of a group's extra K-block, built on stream st:
+// forward, the block-diagonal [N_sum, m r] of the members' B (member j's B in
+// rows of its outputs, columns j r .. j r + r - 1, zeros elsewhere, so every
+// output column gets exactly its own projection's s u B^T); backward, the
+// members' A stacked into [m r, K].
+lsn_status build_group_lb(const lsn_lora_proj* p, int i0, int m, int r, bool bwd, uint16_t* lb, cudaStream_t st) {
+    const int64_t K = p[i0].W.cols;
+    if (!bwd) {
+        int64_t nsum = 0;
+        for (int j = 0; j < m; ++j) nsum += p[i0 + j].W.rows;
+        LSN_CUDA_TRY(cudaMemsetAsync(lb, 0, (size_t)nsum * m * r * 2, st));
+        int64_t row = 0;
+        for (int j = 0; j < m; ++j) {
+            const int64_t N = p[i0 + j].W.rows;
+            LSN_CUDA_TRY(cudaMemcpy2DAsync(lb + row * m * r + j * r, (size_t)m * r * 2, p[i0 + j].B, (size_t)r * 2,
+                                           (size_t)r * 2, (size_t)N, cudaMemcpyDeviceToDevice, st));
+            row += N;
+        }
+    } else {
+        for (int j = 0; j < m; ++j)
+            LSN_CUDA_TRY(cudaMemcpyAsync(lb + (int64_t)j * r * K, p[i0 + j].A, (size_t)r * K * 2,
+                                         cudaMemcpyDeviceToDevice, st));
+    }
+    return LSN_OK;
+}
+
 lsn_status lora_layer_fwd(int n, const lsn_lora_proj* p, int64_t T, int r, float scale, void* ws, size_t ws_bytes,
                           lsn_stream_t stream) {
     lsn_status s = check_layer(n, p, T, r, ws, ws_bytes, false, "lora_layer_fwd");
@@ -476,29 +565,60 @@ lsn_status lora_layer_fwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
     if ((s = check_device()) != LSN_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const LayerWs w = carve_layer(ws, n, p, T, r);
+    const Groups g = find_groups(n, p);
     bool deq[LSN_LAYER_MAX_PROJ];
     DownSpec dn[LSN_LAYER_MAX_PROJ];
     int nd = 0;
-    for (int i = 0; i < n; ++i) {
-        deq[i] = p[i].W.kind == LSN_BASE_NF4 && !fused_here(p[i].W, T, p[i].W.rows);
-        if (!adapter_off(p[i])) dn[nd++] = DownSpec{p[i].x, p[i].A, p[i].u, w.s16[i], T, p[i].W.cols, scale};
+    for (int k = 0; k < g.n; ++k) {
+        const int i0 = g.first[k], m = g.count[k];
+        for (int j = 0; j < m; ++j) {
+            const int i = i0 + j;
+            deq[i] = p[i].W.kind == LSN_BASE_NF4 && (m > 1 || !fused_here(p[i].W, T, p[i].W.rows));
+            if (adapter_off(p[i])) continue;
+            // a group's bf16(s u) go side by side into its LoRA operand
+            dn[nd++] = m > 1 ? DownSpec{p[i].x, p[i].A, p[i].u, w.la[i0] + j * r, T, p[i].W.cols, scale, m * r}
+                             : DownSpec{p[i].x, p[i].A, p[i].u, w.s16[i], T, p[i].W.cols, scale};
+        }
     }
     // Two lanes: the down projections (bound by reading x) run beside the
     // dequantisation (bound by writing W); then the GEMMs, which are
     // independent of each other, alternate over the lanes.
     LaneScope lanes(st, g_layer_lanes.load() == 2);
+    for (int k = 0; k < g.n; ++k)
+        if (g.count[k] > 1 && !adapter_off(p[g.first[k]]))
+            if ((s = build_group_lb(p, g.first[k], g.count[k], r, false, w.lb[g.first[k]], lanes.side())) != LSN_OK)
+                return s;
     if ((s = timed_down_batch(nd, dn, true, r, lanes.side())) != LSN_OK) return s;
     if ((s = layer_dequant(n, p, deq, w, lanes.main())) != LSN_OK) return s;
     if ((s = lanes.barrier()) != LSN_OK) return s;
-    for (int i = 0; i < n; ++i) {
-        const int64_t N = p[i].W.rows, K = p[i].W.cols;
-        const cudaStream_t gs = (i & 1) ? lanes.side() : lanes.main();
+    for (int k = 0; k < g.n; ++k) {
+        const int i = g.first[k], m = g.count[k];
+        const int64_t K = p[i].W.cols;
+        const cudaStream_t gs = (k & 1) ? lanes.side() : lanes.main();
         const int ri = adapter_off(p[i]) ? 0 : r;       // no LoRA K-block with the adapter off
-        if (fused_here(p[i].W, T, N)) {
+        const uint16_t* Wb = p[i].W.kind == LSN_BASE_NF4 ? w.w16[i] : p[i].W.bf16;
+        if (m > 1) {
+            // one GEMM over the stacked weights, each projection's columns to its own y
+            GemmGroup gg;
+            gg.A[0] = p[i].x;
+            gg.lda[0] = K;
+            gg.a_kc[0] = K;
+            gg.nseg = m;
+            int64_t nsum = 0;
+            for (int j = 0; j < m; ++j) {
+                gg.seg_cols[j] = p[i + j].W.rows;
+                gg.seg_D[j] = p[i + j].y;
+                gg.seg_ld[j] = p[i + j].W.rows;
+                nsum += p[i + j].W.rows;
+            }
+            TimingScope ts(LSN_K_GEMM_FWD, 2.0 * T * nsum * (double)(K + m * ri), gs);
+            s = launch_gemm_grouped(gg, Wb, K, false, w.la[i], w.lb[i], m * ri, T, nsum, K, nullptr, 0, w.err, gs);
+        } else if (fused_here(p[i].W, T, p[i].W.rows)) {
+            const int64_t N = p[i].W.rows;
             TimingScope ts(LSN_K_GEMM_FWD, 2.0 * T * N * (double)(K + ri), gs);
             s = launch_gemm_nf4(p[i].x, K, &p[i].W.nf4, false, w.s16[i], p[i].B, ri, T, N, K, p[i].y, N, w.err, gs);
         } else {
-            const uint16_t* Wb = p[i].W.kind == LSN_BASE_NF4 ? w.w16[i] : p[i].W.bf16;
+            const int64_t N = p[i].W.rows;
             s = timed_gemm(LSN_K_GEMM_FWD, p[i].x, K, Wb, K, false, w.s16[i], p[i].B, ri, T, N, K, p[i].y, N, w.err,
                            gs);
         }
@@ -514,6 +634,7 @@ lsn_status lora_layer_bwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
     if ((s = check_device()) != LSN_OK) return s;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const LayerWs w = carve_layer(ws, n, p, T, r);
+    const Groups g = find_groups(n, p);
     // Two lanes: the down projections (reading dY, and x when no u was kept)
     // run beside the dequantisation; then the token reductions run on the
     // side lane beside the input-gradient GEMMs, which alternate over both.
@@ -522,13 +643,23 @@ lsn_status lora_layer_bwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
         bool deq[LSN_LAYER_MAX_PROJ];
         DownSpec dg[LSN_LAYER_MAX_PROJ], du[LSN_LAYER_MAX_PROJ];
         int ng = 0, nu = 0;
-        for (int i = 0; i < n; ++i) {
-            const int64_t N = p[i].W.rows, K = p[i].W.cols;
-            deq[i] = p[i].dX && p[i].W.kind == LSN_BASE_NF4 && !fused_here(p[i].W, T, K);
-            if (adapter_off(p[i])) continue;
-            dg[ng++] = DownSpec{p[i].dY, p[i].B, w.g32[i], w.s16[i], T, N, scale};
-            if (!p[i].u) du[nu++] = DownSpec{p[i].x, p[i].A, w.u32[i], nullptr, T, K, scale};
+        for (int k = 0; k < g.n; ++k) {
+            const int i0 = g.first[k], m = g.count[k];
+            const bool want_dx = p[i0].dX != nullptr;    // a group's dX is its first member's
+            for (int j = 0; j < m; ++j) {
+                const int i = i0 + j;
+                const int64_t N = p[i].W.rows, K = p[i].W.cols;
+                deq[i] = want_dx && p[i].W.kind == LSN_BASE_NF4 && (m > 1 || !fused_here(p[i].W, T, K));
+                if (adapter_off(p[i])) continue;
+                dg[ng++] = m > 1 ? DownSpec{p[i].dY, p[i].B, w.g32[i], w.la[i0] + j * r, T, N, scale, m * r}
+                                 : DownSpec{p[i].dY, p[i].B, w.g32[i], w.s16[i], T, N, scale};
+                if (!p[i].u) du[nu++] = DownSpec{p[i].x, p[i].A, w.u32[i], nullptr, T, K, scale};
+            }
         }
+        for (int k = 0; k < g.n; ++k)
+            if (g.count[k] > 1 && p[g.first[k]].dX && !adapter_off(p[g.first[k]]))
+                if ((s = build_group_lb(p, g.first[k], g.count[k], r, true, w.lb[g.first[k]], lanes.side())) != LSN_OK)
+                    return s;
         if ((s = timed_down_batch(ng, dg, false, r, lanes.side())) != LSN_OK) return s;
         if ((s = timed_down_batch(nu, du, true, r, lanes.side())) != LSN_OK) return s;
         if ((s = layer_dequant(n, p, deq, w, lanes.main())) != LSN_OK) return s;
@@ -546,17 +677,33 @@ lsn_status lora_layer_bwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
     }
     if ((s = timed_tgrad_batch(nt, tg, r, lanes.side())) != LSN_OK) return s;
     if (T > 0) {
-        for (int i = 0, j = 0; i < n; ++i) {
+        for (int k = 0, j = 0; k < g.n; ++k) {
+            const int i = g.first[k], m = g.count[k];
             if (!p[i].dX) continue;
-            const int64_t N = p[i].W.rows, K = p[i].W.cols;
+            const int64_t K = p[i].W.cols;
             const cudaStream_t gs = (j++ & 1) ? lanes.side() : lanes.main();
             const int ri = adapter_off(p[i]) ? 0 : r;
-            if (fused_here(p[i].W, T, K)) {
+            const uint16_t* Wb = p[i].W.kind == LSN_BASE_NF4 ? w.w16[i] : p[i].W.bf16;
+            if (m > 1) {
+                // dX = [dY_1 .. dY_m] [W_1; ..; W_m] + [s g_1 .. s g_m] [A_1; ..; A_m]
+                GemmGroup gg;
+                gg.na = m;
+                int64_t nsum = 0;
+                for (int q = 0; q < m; ++q) {
+                    gg.A[q] = p[i + q].dY;
+                    gg.lda[q] = p[i + q].W.rows;
+                    gg.a_kc[q] = p[i + q].W.rows;
+                    nsum += p[i + q].W.rows;
+                }
+                TimingScope ts(LSN_K_GEMM_BWD, 2.0 * T * K * (double)(nsum + m * ri), gs);
+                s = launch_gemm_grouped(gg, Wb, K, true, w.la[i], w.lb[i], m * ri, T, K, nsum, p[i].dX, K, w.err, gs);
+            } else if (fused_here(p[i].W, T, K)) {
+                const int64_t N = p[i].W.rows;
                 TimingScope ts(LSN_K_GEMM_BWD, 2.0 * T * K * (double)(N + ri), gs);
                 s = launch_gemm_nf4(p[i].dY, N, &p[i].W.nf4, true, w.s16[i], p[i].A, ri, T, K, N, p[i].dX, K, w.err,
                                     gs);
             } else {
-                const uint16_t* Wb = p[i].W.kind == LSN_BASE_NF4 ? w.w16[i] : p[i].W.bf16;
+                const int64_t N = p[i].W.rows;
                 s = timed_gemm(LSN_K_GEMM_BWD, p[i].dY, N, Wb, K, true, w.s16[i], p[i].A, ri, T, K, N, p[i].dX, K,
                                w.err, gs);
             }

@@ -11,12 +11,24 @@
 // Laptop? (I Did the Math)", 1:47-1:58: the adapter rides alongside the
 // frozen weights).
 //
-// Structure (one persistent CTA per SM, 192 threads):
-//   warp 0     TMA producer: one elected lane streams 128x64 A tiles and
-//              64xBN B tiles (128-byte swizzle) into a 4-stage ring;
-//   warp 1     allocates 2*BN TMEM columns; one lane issues tcgen05.mma
-//              (M=128, N=BN, K=16) and commits each stage back to the
-//              producer and each finished accumulator to the epilogue;
+// Grouped projections (several linears reading the same x, e.g. q, k, v):
+// the forward is one GEMM over their stacked weights whose output columns are
+// routed to each projection's y (up to kMaxSeg segments); the backward is one
+// GEMM whose contraction runs over the projections' dY side by side (one A
+// tensor map per projection, chosen per 128-wide K-block), giving the summed
+// input gradient.
+//
+// Structure (one persistent CTA per SM, or one CTA pair per two SMs, 192
+// threads):
+//   warp 0     TMA producer: one elected lane streams 128-wide contraction
+//              stages (two 64-wide 128-byte-swizzled sub-tiles per operand)
+//              into a 3-stage ring; with CTA pairs each CTA loads its own
+//              128 rows of A and half of B, completing on the leader's
+//              barrier;
+//   warp 1     allocates 2*BN TMEM columns; one lane of the leader issues
+//              tcgen05.mma (M = 128, or 256 across a pair with
+//              cta_group::2; N = BN; K = 16) and commits each stage back to
+//              the producers and each finished accumulator to the epilogue;
 //   warps 2-5  epilogue: tcgen05.ld 32 columns at a time from their TMEM lane
 //              quadrant, round to bf16, store; the two accumulator buffers
 //              let the epilogue of tile i overlap the main loop of tile i+1.
@@ -30,6 +42,8 @@
 
 namespace lsn {
 
+constexpr int kMaxSeg = kGemmMaxSeg;   // output segments / A tensor maps of a grouped GEMM
+
 struct GemmArgs {
     int M, N;            // output rows (tokens) and columns
     int num_kb;          // 128-wide contraction blocks of the base term
@@ -37,6 +51,18 @@ struct GemmArgs {
     uint16_t* D;         // bf16 output, row-major
     int64_t ldd;         // elements
     int* err;            // device error flag (set on a timed-out wait)
+    // Output segments: columns [seg_col[i], seg_col[i+1]) go to seg_D[i] with
+    // row stride seg_ld[i] (column 0 of the segment at seg_D[i]); nseg == 0
+    // means the single output D.
+    int nseg;
+    int seg_col[kMaxSeg + 1];
+    uint16_t* seg_D[kMaxSeg];
+    int64_t seg_ld[kMaxSeg];
+    // A operand split along the contraction: K-blocks [a_kb[i], a_kb[i+1])
+    // come from A tensor map i at contraction coordinate (kb - a_kb[i]) * 128;
+    // na == 1 means the single map.
+    int na;
+    int a_kb[kMaxSeg + 1];
     // NF4 base converted in the kernel (fused variant only):
     const uint8_t* absmax_q;   // [wrows * wcols / 64] second-level codes
     const float* absmax_s2;    // [ceil(nblk / 256)]
@@ -64,27 +90,21 @@ constexpr int CONV_WARPS = 8;    // NF4 converter warps (fused variant)
 // PAIR = false: one CTA per SM, tile 128 x BN.
 // PAIR = true : a CTA pair (cluster of 2) issues the 2-SM MMA, tile 256 x BN,
 //               each CTA staging its 128 rows of A and BN/2 rows of B.
-// NF4  = true : B is the NF4 weight, converted to bf16 in shared memory by
-//               converter warps from a TMA-staged packed tile (PAIR only).
-template <bool PAIR, int BN, bool B_MN, bool NF4 = false>
+template <bool PAIR, int BN, bool B_MN>
 struct Cfg {
     static constexpr int B_ROWS = PAIR ? BN / 2 : BN;     // B rows (N extent) staged per CTA
     static constexpr int A_SUB = BM * SUB * 2;             // bytes of one A sub-tile
     static constexpr int A_BYTES = 2 * A_SUB;
     static constexpr int B_SUB = B_ROWS * SUB * 2;         // K-major: bytes of one B sub-tile
     static constexpr int B_BYTES = 2 * B_SUB;              // MN-major: B_ROWS/64 atom columns of 128 x 64
-    static constexpr int P_BYTES = NF4 ? 128 * 64 : 0;     // packed NF4 tile: 128 rows x 64 bytes
-    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + P_BYTES;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int BAR_BYTES = 256;
-    static constexpr int DQ_BYTES = NF4 ? 1024 : 0;
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + DQ_BYTES + 1024;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
     static constexpr uint32_t IDESC = idesc_bf16(PAIR ? 2 * BM : BM, BN, 0, B_MN ? 1 : 0);
     static constexpr uint32_t TMEM_COLS = 2 * BN;
     static constexpr int TILE_M = PAIR ? 2 * BM : BM;
     static constexpr uint32_t ACC_EMPTY_ARRIVALS = (PAIR ? 2 : 1) * 4;
-    static constexpr uint32_t READY_ARRIVALS = (PAIR ? 2 : 1) * CONV_WARPS;
-    static constexpr int THREADS = 192 + (NF4 ? 32 * CONV_WARPS : 0);
-    static_assert(!NF4 || (PAIR && B_ROWS == 128), "the fused NF4 path runs on the pair kernel");
+    static constexpr int THREADS = 192;
 };
 
 __device__ __forceinline__ void raise_error(volatile int* abort_flag, int* err, int code) {
@@ -92,24 +112,27 @@ __device__ __forceinline__ void raise_error(volatile int* abort_flag, int* err, 
     if (err) atomicExch(err, code);
 }
 
-template <bool PAIR, int BN, bool B_MN, bool NF4>
-__global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN, NF4>::THREADS, 1)
-    lsn_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+// The A tensor maps of a grouped GEMM (the caller's separate dY tensors).
+struct AMaps {
+    CUtensorMap m[kMaxSeg];
+};
+
+template <bool PAIR, int BN, bool B_MN>
+__global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
+    lsn_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmLA, const __grid_constant__ CUtensorMap tmLB,
                     const __grid_constant__ GemmArgs p) {
-    using C = Cfg<PAIR, BN, B_MN, NF4>;
+    using C = Cfg<PAIR, BN, B_MN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
-    uint64_t* full = bars;                    // TMA landed (bf16 path: A and B; NF4: this CTA's A + packed)
+    uint64_t* full = bars;                    // TMA landed (A and B of the stage, both CTAs of a pair)
     uint64_t* empty = bars + STAGES;          // MMAs done reading the stage
-    uint64_t* ready = bars + 2 * STAGES;      // NF4: converted B written (counted on the leader)
-    uint64_t* acc_full = bars + 3 * STAGES;
+    uint64_t* acc_full = bars + 2 * STAGES;
     uint64_t* acc_empty = acc_full + 2;
     uint64_t* drain = acc_empty + 2;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-    float* dq_s = reinterpret_cast<float*>(smem + STAGES * C::STAGE_BYTES + C::BAR_BYTES);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint32_t rank = 0;
@@ -126,18 +149,15 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN, NF4>::THREADS, 1)
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
-            mbar_init(&ready[s], C::READY_ARRIVALS);
         }
         for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], C::ACC_EMPTY_ARRIVALS); }
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if constexpr (NF4) {
-        for (int i = threadIdx.x; i < 256; i += blockDim.x) dq_s[i] = p.dq[i];
-    }
     if (warp == 0 && lane == 0) {
-        tma_prefetch_desc(&tmA); tma_prefetch_desc(&tmB);
+        for (int i = 0; i < p.na; ++i) tma_prefetch_desc(&tmA.m[i]);
+        tma_prefetch_desc(&tmB);
         if (p.lora_k16 > 0) { tma_prefetch_desc(&tmLA); tma_prefetch_desc(&tmLB); }
     }
     if (warp == 1) {
@@ -162,52 +182,32 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN, NF4>::THREADS, 1)
                 const int mb = tile % num_m, nb = tile / num_m;
                 const int m_row = mb * C::TILE_M + (int)rank * BM;
                 const int n_off = nb * BN + (int)rank * C::B_ROWS;
+                int ai = 0;                                   // A map of the current K-block
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
                     uint8_t* sA = smem + stage * C::STAGE_BYTES;
                     uint8_t* sB = sA + C::A_BYTES;
-                    uint8_t* sP = sB + C::B_BYTES;
                     const bool lora = kb >= p.num_kb;
-                    const CUtensorMap* ma = lora ? &tmLA : &tmA;
+                    while (!lora && ai + 1 < p.na && kb >= p.a_kb[ai + 1]) ++ai;
+                    const CUtensorMap* ma = lora ? &tmLA : &tmA.m[ai];
                     const CUtensorMap* mbp = lora ? &tmLB : &tmB;
-                    const int kc = lora ? 0 : kb * BK;
-                    if constexpr (NF4) {
-                        // Each CTA counts its own bytes on its own barrier; the
-                        // converters release the stage to the MMA.
-                        mbar_arrive_expect_tx(&full[stage], C::A_BYTES + (lora ? C::B_BYTES : C::P_BYTES));
-                        tma_load_2d(sA, ma, kc, m_row, &full[stage]);
-                        tma_load_2d(sA + C::A_SUB, ma, kc + SUB, m_row, &full[stage]);
-                        if (lora) {
-                            if (!B_MN) {
-                                tma_load_2d(sB, mbp, 0, n_off, &full[stage]);
-                                tma_load_2d(sB + C::B_SUB, mbp, SUB, n_off, &full[stage]);
-                            } else {
-                                #pragma unroll
-                                for (int a = 0; a < C::B_ROWS / 64; ++a)
-                                    tma_load_2d(sB + a * (BK * 128), mbp, n_off + a * 64, 0, &full[stage]);
-                            }
-                        } else {
-                            // packed bytes: fwd rows n_off.., bytes kb*64..; bwd rows kb*128.., bytes n_off/2..
-                            if (!B_MN) tma_load_2d(sP, &tmB, kb * 64, n_off, &full[stage]);
-                            else       tma_load_2d(sP, &tmB, n_off / 2, kb * BK, &full[stage]);
-                        }
+                    const int kc = lora ? 0 : kb * BK;                       // contraction coordinate of B
+                    const int ka = lora ? 0 : (kb - p.a_kb[ai]) * BK;        // ... and of the A map
+                    uint32_t fbar = smem_u32(&full[stage]);
+                    if constexpr (PAIR) fbar = mapa_shared(fbar, 0);
+                    if (leader) mbar_arrive_expect_tx(&full[stage], (PAIR ? 2 : 1) * (C::A_BYTES + C::B_BYTES));
+                    auto load = [&](void* dst, const CUtensorMap* m, int x, int y) {
+                        if constexpr (PAIR) tma_load_2d_pair(dst, m, x, y, fbar);
+                        else                tma_load_2d(dst, m, x, y, &full[stage]);
+                    };
+                    load(sA, ma, ka, m_row);
+                    load(sA + C::A_SUB, ma, ka + SUB, m_row);
+                    if (!B_MN) {
+                        load(sB, mbp, kc, n_off);
+                        load(sB + C::B_SUB, mbp, kc + SUB, n_off);
                     } else {
-                        uint32_t fbar = smem_u32(&full[stage]);
-                        if constexpr (PAIR) fbar = mapa_shared(fbar, 0);
-                        if (leader) mbar_arrive_expect_tx(&full[stage], (PAIR ? 2 : 1) * (C::A_BYTES + C::B_BYTES));
-                        auto load = [&](void* dst, const CUtensorMap* m, int x, int y) {
-                            if constexpr (PAIR) tma_load_2d_pair(dst, m, x, y, fbar);
-                            else                tma_load_2d(dst, m, x, y, &full[stage]);
-                        };
-                        load(sA, ma, kc, m_row);
-                        load(sA + C::A_SUB, ma, kc + SUB, m_row);
-                        if (!B_MN) {
-                            load(sB, mbp, kc, n_off);
-                            load(sB + C::B_SUB, mbp, kc + SUB, n_off);
-                        } else {
-                            #pragma unroll
-                            for (int a = 0; a < C::B_ROWS / 64; ++a) load(sB + a * (BK * 128), mbp, n_off + a * 64, kc);
-                        }
+                        #pragma unroll
+                        for (int a = 0; a < C::B_ROWS / 64; ++a) load(sB + a * (BK * 128), mbp, n_off + a * 64, kc);
                     }
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
@@ -225,9 +225,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN, NF4>::THREADS, 1)
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
                 for (int kb = 0; kb < nkb; ++kb) {
-                    const bool got = NF4 ? mbar_wait_cluster(&ready[stage], phase, abort_flag)
-                                         : mbar_wait(&full[stage], phase, abort_flag);
-                    if (!got) { ok = false; break; }
+                    if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(smem + stage * C::STAGE_BYTES);
                     const uint32_t b0 = a0 + C::A_BYTES;
@@ -256,7 +254,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN, NF4>::THREADS, 1)
             else                umma_commit(drain);
             mbar_wait(drain, 0, nullptr);
         }
-    } else if (warp < 6) {
+    } else {
         // -------------------------------------------------------- epilogue --
         const int q = warp & 3;                    // TMEM lanes 32q .. 32q+31
         int acc = 0;
@@ -275,7 +273,18 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN, NF4>::THREADS, 1)
                 tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c * 32), v);
                 tmem_ld_wait();
                 if (row < p.M) {
-                    uint4* dst = reinterpret_cast<uint4*>(p.D + (int64_t)row * p.ldd + col);
+                    // Output segment of these 32 columns (segment widths are multiples of 64).
+                    uint16_t* base = p.D;
+                    int64_t ld = p.ldd;
+                    int lc = col;
+                    for (int sgi = 0; sgi < p.nseg; ++sgi) {
+                        if (col >= p.seg_col[sgi] && col < p.seg_col[sgi + 1]) {
+                            base = p.seg_D[sgi];
+                            ld = p.seg_ld[sgi];
+                            lc = col - p.seg_col[sgi];
+                        }
+                    }
+                    uint4* dst = reinterpret_cast<uint4*>(base + (int64_t)row * ld + lc);
                     #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         uint4 o;
@@ -295,92 +304,6 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN, NF4>::THREADS, 1)
             }
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1;
-        }
-    } else if constexpr (NF4) {
-        // ------------------------------------------------------- converters --
-        // Thread t of the 256 converters owns one (row, 64-block) of the
-        // CTA's 128 x 128 B tile per stage: row = t % 128, block = t / 128.
-        // Rows are B rows (forward: W rows n; backward: the contraction rows n
-        // of W read MN-major); the block is 64 consecutive W columns.  In both
-        // majors the 64 bf16 go to one 128-byte row of a 128-byte-swizzled
-        // atom: block b's atom at b * 16 KB, row at (row/8)*1024 + (row%8)*128.
-        const int t = threadIdx.x - 192;
-        const int row = t & 127, blk = t >> 7;
-        const int64_t nblk_row = p.wcols / 64;          // 64-blocks per W row
-        const float off = *p.absmax_off;
-        // The unit's second-level code and s2 are fetched two k-blocks ahead,
-        // so their global-load latency overlaps earlier conversions.
-        struct Meta { uint32_t code; float s2; bool ok; };
-        auto fetch = [&](int tl, int k) -> Meta {
-            Meta m{0u, 0.0f, false};
-            if (tl >= num_tiles || k >= p.num_kb) return m;
-            const int n_off = (tl / num_m) * BN + (int)rank * C::B_ROWS;
-            const int64_t wr = B_MN ? (int64_t)k * BK + row : (int64_t)n_off + row;
-            const int64_t wb = B_MN ? (int64_t)(n_off / 64) + blk : (int64_t)k * 2 + blk;
-            if (wr < p.wrows && wb < nblk_row) {
-                const int64_t bi = wr * nblk_row + wb;
-                m.code = __ldg(p.absmax_q + bi);
-                m.s2 = __ldg(p.absmax_s2 + (bi >> 8));
-                m.ok = true;
-            }
-            return m;
-        };
-        int ft = unit, fk = 0;
-        auto step = [&]() { if (++fk == nkb) { fk = 0; ft += nunits; } };
-        Meta m0 = fetch(ft, fk);
-        step();
-        Meta m1 = fetch(ft, fk);
-        step();
-        int stage = 0;
-        uint32_t phase = 0;
-        bool bad = false;
-        for (int tile = unit; tile < num_tiles && !bad; tile += nunits) {
-            for (int kb = 0; kb < nkb; ++kb) {
-                const Meta cur = m0;
-                m0 = m1;
-                m1 = fetch(ft, fk);
-                step();
-                const bool got = mbar_wait(&full[stage], phase, abort_flag);
-                if (!__all_sync(0xffffffffu, got)) { if (lane == 0) raise_error(abort_flag, p.err, 4); bad = true; break; }
-                if (kb < p.num_kb) {
-                    uint8_t* sB = smem + stage * C::STAGE_BYTES + C::A_BYTES;
-                    const uint8_t* sP = sB + C::B_BYTES;
-                    uint8_t* dst = sB + blk * (BK * 128) + (row >> 3) * 1024 + (row & 7) * 128;
-                    if (cur.ok) {
-                        const float ah = __fadd_rn(__fmul_rn(dq_s[cur.code], cur.s2), off);
-                        // Scaled table: entry q = bf16(level[q] * absmax_hat), packed in pairs.
-                        uint32_t e[8];
-                        #pragma unroll
-                        for (int i = 0; i < 8; ++i) e[i] = pack_bf16x2(__fmul_rn(p.level[2 * i], ah), __fmul_rn(p.level[2 * i + 1], ah));
-                        uint32_t lo[4], hi[4];
-                        #pragma unroll
-                        for (int i = 0; i < 4; ++i) { lo[i] = prmt(e[2 * i], e[2 * i + 1], 0x6420u); hi[i] = prmt(e[2 * i], e[2 * i + 1], 0x7531u); }
-                        // Packed tile row: 64 bytes, 64-byte swizzle (16-byte chunk c stored at c ^ ((row >> 1) & 3)).
-                        const uint8_t* prow = sP + row * 64;
-                        #pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const int ch = (2 * blk + h) ^ ((row >> 1) & 3);
-                            const uint4 pk = *reinterpret_cast<const uint4*>(prow + ch * 16);
-                            const uint32_t w[4] = {pk.x, pk.y, pk.z, pk.w};
-                            #pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const int c = h * 4 + i;                 // 8-element chunk of the 64
-                                *reinterpret_cast<uint4*>(dst + ((c ^ (row & 7)) << 4)) = nf4x8_to_bf16(w[i], lo, hi);
-                            }
-                        }
-                    } else {
-                        #pragma unroll
-                        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(dst + (c << 4)) = make_uint4(0, 0, 0, 0);
-                    }
-                    fence_proxy_async_smem();
-                }
-                __syncwarp();
-                if (lane == 0) {
-                    if constexpr (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&ready[stage]), 0));
-                    else                mbar_arrive(&ready[stage]);
-                }
-                if (++stage == STAGES) { stage = 0; phase ^= 1; }
-            }
         }
     }
     __syncwarp();
@@ -767,14 +690,14 @@ lsn_status make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t out
     return LSN_OK;
 }
 
-template <bool PAIR, int BN, bool B_MN, bool NF4 = false>
-lsn_status launch_cfg(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& la, const CUtensorMap& lb,
+template <bool PAIR, int BN, bool B_MN>
+lsn_status launch_cfg(const AMaps& a, const CUtensorMap& b, const CUtensorMap& la, const CUtensorMap& lb,
                       const GemmArgs& args, cudaStream_t st) {
-    using C = Cfg<PAIR, BN, B_MN, NF4>;
+    using C = Cfg<PAIR, BN, B_MN>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(lsn_gemm_kernel<PAIR, BN, B_MN, NF4>,
+        attr_err = cudaFuncSetAttribute(lsn_gemm_kernel<PAIR, BN, B_MN>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     });
     if (attr_err != cudaSuccess) return fail_cuda(attr_err, "cudaFuncSetAttribute(gemm smem)");
@@ -798,7 +721,7 @@ lsn_status launch_cfg(const CUtensorMap& a, const CUtensorMap& b, const CUtensor
     na += pdl_attr(&attr[na]);
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    LSN_CUDA_TRY(cudaLaunchKernelEx(&cfg, lsn_gemm_kernel<PAIR, BN, B_MN, NF4>, a, b, la, lb, args));
+    LSN_CUDA_TRY(cudaLaunchKernelEx(&cfg, lsn_gemm_kernel<PAIR, BN, B_MN>, a, b, la, lb, args));
     return LSN_OK;
 }
 
@@ -886,14 +809,28 @@ lsn_status launch_gemm_nf4(const uint16_t* A, int64_t lda, const lsn_nf4_weight*
 //   b_mn == false: B is [N, Kc] (ldb), LB is [N, r]   (forward: W, B_lora)
 //   b_mn == true : B is [Kc, N] (ldb), LB is [r, N]   (backward: W, A_lora)
 //   LA [M, r] (bf16(s u) or bf16(s g)); r == 0 disables the LoRA term.
-lsn_status launch_gemm(const uint16_t* A, int64_t lda, const uint16_t* B, int64_t ldb, bool b_mn, const uint16_t* LA,
-                       const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D, int64_t ldd,
-                       int* err, cudaStream_t st) {
+lsn_status launch_gemm_grouped(const GemmGroup& g, const uint16_t* B, int64_t ldb, bool b_mn, const uint16_t* LA,
+                               const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D,
+                               int64_t ldd, int* err, cudaStream_t st) {
+    if (g.na < 1 || g.na > kMaxSeg || g.nseg < 0 || g.nseg > kMaxSeg)
+        return fail(LSN_ERR_INVALID_ARG, "grouped GEMM: bad operand or segment count");
     const bool pair = gemm_use_pairs(M, N);
-    const int b_rows = pair ? 128 : 128;           // B rows staged per CTA: BN/2 = 128 (pair) or BN = 128
-    CUtensorMap ma, mb, mla, mlb;
+    const int b_rows = 128;                         // B rows staged per CTA: BN/2 = 128 (pair) or BN = 128
+    AMaps ma;
+    CUtensorMap mb, mla, mlb;
     lsn_status s;
-    if ((s = make_map(&ma, A, Kc, M, lda, SUB, BM)) != LSN_OK) return s;
+    GemmArgs args{};
+    int64_t kb_acc = 0;
+    for (int i = 0; i < g.na; ++i) {
+        if ((s = make_map(&ma.m[i], g.A[i], g.a_kc[i], M, g.lda[i], SUB, BM)) != LSN_OK) return s;
+        args.a_kb[i] = (int)kb_acc;
+        if (i + 1 < g.na && g.a_kc[i] % BK != 0)
+            return fail(LSN_ERR_INVALID_ARG, "grouped GEMM: inner A extents must be multiples of 128");
+        kb_acc += (g.a_kc[i] + BK - 1) / BK;
+    }
+    args.a_kb[g.na] = (int)kb_acc;
+    args.na = g.na;
+    for (int i = g.na; i < kMaxSeg; ++i) ma.m[i] = ma.m[0];
     if (!b_mn) {
         if ((s = make_map(&mb, B, Kc, N, ldb, SUB, b_rows)) != LSN_OK) return s;
     } else {
@@ -907,21 +844,42 @@ lsn_status launch_gemm(const uint16_t* A, int64_t lda, const uint16_t* B, int64_
             if ((s = make_map(&mlb, LB, N, r, N, 64, BK)) != LSN_OK) return s;
         }
     } else {                                        // no LoRA term: the maps are never read
-        mla = ma;
+        mla = ma.m[0];
         mlb = mb;
     }
-    GemmArgs args{};
     args.M = (int)M;
     args.N = (int)N;
     args.num_kb = (int)((Kc + BK - 1) / BK);
+    if (args.num_kb != args.a_kb[g.na]) return fail(LSN_ERR_INVALID_ARG, "grouped GEMM: A extents do not add up to Kc");
     args.lora_k16 = (r + 15) / 16;
     args.D = D;
     args.ldd = ldd;
     args.err = err;
+    args.nseg = g.nseg;
+    int64_t c0 = 0;
+    for (int i = 0; i < g.nseg; ++i) {
+        args.seg_col[i] = (int)c0;
+        args.seg_D[i] = g.seg_D[i];
+        args.seg_ld[i] = g.seg_ld[i];
+        c0 += g.seg_cols[i];
+    }
+    args.seg_col[g.nseg] = (int)c0;
+    if (g.nseg > 0 && c0 != N) return fail(LSN_ERR_INVALID_ARG, "grouped GEMM: segments do not add up to N");
     if (pair) return b_mn ? launch_cfg<true, 256, true>(ma, mb, mla, mlb, args, st)
                           : launch_cfg<true, 256, false>(ma, mb, mla, mlb, args, st);
     return b_mn ? launch_cfg<false, 128, true>(ma, mb, mla, mlb, args, st)
                 : launch_cfg<false, 128, false>(ma, mb, mla, mlb, args, st);
+}
+
+lsn_status launch_gemm(const uint16_t* A, int64_t lda, const uint16_t* B, int64_t ldb, bool b_mn, const uint16_t* LA,
+                       const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D, int64_t ldd,
+                       int* err, cudaStream_t st) {
+    GemmGroup g;
+    g.na = 1;
+    g.A[0] = A;
+    g.lda[0] = lda;
+    g.a_kc[0] = Kc;
+    return launch_gemm_grouped(g, B, ldb, b_mn, LA, LB, r, M, N, Kc, D, ldd, err, st);
 }
 
 }  // namespace lsn

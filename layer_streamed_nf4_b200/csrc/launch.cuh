@@ -7,8 +7,8 @@
 namespace lsn {
 
 // One rank-r down projection: out[t, j] = sum_k X[t, k] W(j, k) for j < r,
-// W either A [r, Kd] or B [Kd, r]; written as fp32 (u32) and/or as
-// bf16(scale * out) (u16), either may be NULL.
+// W either A [r, Kd] or B [Kd, r]; written as fp32 (u32, row stride r) and/or
+// as bf16(scale * out) (u16, row stride ld16, r when 0), either may be NULL.
 struct DownSpec {
     const uint16_t* X;
     const uint16_t* W;
@@ -16,6 +16,7 @@ struct DownSpec {
     uint16_t* u16;
     int64_t T, Kd;
     float scale;
+    int ld16 = 0;
 };
 
 // One token reduction: R[j, k] = sum_t G[t, j] X[t, k], written (or, with
@@ -47,6 +48,25 @@ lsn_status launch_dequant(const lsn_nf4_weight* w, uint16_t* out, cudaStream_t s
 // Several NF4 weights dequantised by one launch (at most 16 per launch; more take several).
 lsn_status launch_dequant_batch(int n, const lsn_nf4_weight* const* w, uint16_t* const* out, cudaStream_t st);
 
+// Grouped GEMM operands: the A operand as na tensors side by side along the
+// contraction (tensor i: [M, a_kc[i]] row-major with row stride lda[i]; every
+// a_kc but the last a multiple of 128), and the output columns split into
+// nseg segments (segment i: seg_cols[i] columns, a multiple of 64, written at
+// seg_D[i] with row stride seg_ld[i]); nseg == 0: the single output D.
+constexpr int kGemmMaxSeg = 4;
+struct GemmGroup {
+    int na = 1;
+    const uint16_t* A[kGemmMaxSeg] = {};
+    int64_t lda[kGemmMaxSeg] = {};
+    int64_t a_kc[kGemmMaxSeg] = {};
+    int nseg = 0;
+    int64_t seg_cols[kGemmMaxSeg] = {};
+    uint16_t* seg_D[kGemmMaxSeg] = {};
+    int64_t seg_ld[kGemmMaxSeg] = {};
+};
+lsn_status launch_gemm_grouped(const GemmGroup& g, const uint16_t* B, int64_t ldb, bool b_mn, const uint16_t* LA,
+                               const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D,
+                               int64_t ldd, int* err, cudaStream_t st);
 lsn_status launch_gemm(const uint16_t* A, int64_t lda, const uint16_t* B, int64_t ldb, bool b_mn, const uint16_t* LA,
                        const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D, int64_t ldd,
                        int* err, cudaStream_t st);

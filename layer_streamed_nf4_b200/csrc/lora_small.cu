@@ -96,6 +96,7 @@ struct DownProb {
     int64_t T, Kd;
     int cps, ns;         // 64-wide K chunks per split, splits
     int first;           // first blockIdx.x of the problem
+    int ld16;            // row stride of u16
     float scale;
 };
 struct DownBatch {
@@ -142,7 +143,7 @@ __global__ void __launch_bounds__(128) lora_down_kernel(const __grid_constant__ 
     float* __restrict__ u32 = pb.u32;
     uint16_t* __restrict__ u16 = pb.u16;
     const int64_t T = pb.T, Kd = pb.Kd;
-    const int chunks_per_split = pb.cps, nsplit = pb.ns;
+    const int chunks_per_split = pb.cps, nsplit = pb.ns, ld16 = pb.ld16;
     const float scale = pb.scale;
     pdl_launch_dependents();
     pdl_wait();
@@ -230,7 +231,7 @@ __global__ void __launch_bounds__(128) lora_down_kernel(const __grid_constant__ 
     const bool ok0 = row0 < T, ok1 = row1 < T;
     auto emit = [&](int64_t row, int j, float v) {
         if (u32) u32[row * R + j] = v;
-        if (u16) u16[row * R + j] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(scale, v)));
+        if (u16) u16[row * ld16 + j] = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(scale, v)));
     };
     if (nsplit == 1) {                  // every CTA of the cluster takes this branch
         if (blockIdx.y != 0) return;
@@ -606,6 +607,7 @@ lsn_status launch_lora_down_batch(int n, const DownSpec* specs, bool w_rk, int r
         pb.ns = down_splits(d.T, d.Kd);
         pb.cps = (int)((d.Kd / 64 + pb.ns - 1) / pb.ns);
         pb.first = blocks;
+        pb.ld16 = d.ld16 > 0 ? d.ld16 : r;
         pb.scale = d.scale;
         blocks += (int)((d.T + kDnRows - 1) / kDnRows);
         smax = pb.ns > smax ? pb.ns : smax;

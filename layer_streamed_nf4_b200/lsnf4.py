@@ -67,7 +67,7 @@ class LoraProj(ctypes.Structure):
     """One projection of a layer call (lsn_lora_proj)."""
     _fields_ = [("W", Base), ("x", ctypes.c_void_p), ("A", ctypes.c_void_p), ("B", ctypes.c_void_p),
                 ("y", ctypes.c_void_p), ("dY", ctypes.c_void_p), ("dX", ctypes.c_void_p), ("dA", ctypes.c_void_p),
-                ("dB", ctypes.c_void_p), ("u", ctypes.c_void_p)]
+                ("dB", ctypes.c_void_p), ("u", ctypes.c_void_p), ("group", ctypes.c_int)]
 
 
 LSN_LAYER_MAX_PROJ = 16
@@ -245,8 +245,8 @@ def lora_linear_bwd(W: Base, x, dY, T: int, A, B, r: int, scale: float, dX, dA, 
 
 # ------------------------------------------------------------ whole layer ---
 
-def lora_proj(W: Base, x, A, B, y=None, dY=None, dX=None, dA=None, dB=None, u=None) -> LoraProj:
-    return LoraProj(W, _ptr(x), _ptr(A), _ptr(B), _ptr(y), _ptr(dY), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(u))
+def lora_proj(W: Base, x, A, B, y=None, dY=None, dX=None, dA=None, dB=None, u=None, group: int = 0) -> LoraProj:
+    return LoraProj(W, _ptr(x), _ptr(A), _ptr(B), _ptr(y), _ptr(dY), _ptr(dX), _ptr(dA), _ptr(dB), _ptr(u), group)
 
 
 def proj_array(projs) -> ctypes.Array:

@@ -18,6 +18,13 @@ Two ways to drive a layer (api=...):
   "proj"   seven lora_linear_fwd / lora_linear_bwd calls per layer and sweep.
 Both give the same bits.
 
+Inputs: by default every (layer, projection) has its own x.  With
+shared_inputs, q, k and v read one x and gate and up read one x, as in a
+decoder layer; with grouped (which implies shared_inputs) those projections
+are passed to the layer calls as groups, so each group's forward is one GEMM
+over its stacked weights and its backward one GEMM producing the group's
+summed input gradient (written to the first member's dX).
+
 Lanes ("proj" only): the seven projections of a layer are independent calls, so they are
 issued round-robin on `lanes` streams (default 2), each with its own
 workspace.  The side kernels and the dequantisation of one projection then
@@ -62,10 +69,13 @@ class Stack:
     def __init__(self, cfg: synth.StackConfig, layers: int | None = None, tokens: int | None = None,
                  mode: str = "streamed", n_slots: int = 2, seed: int = synth.SEED, keep_outputs: bool = False,
                  distinct_activations: bool = True, device: int = 0, stream: torch.cuda.Stream | None = None,
-                 lanes: int = 2, api: str = "layer"):
+                 lanes: int = 2, api: str = "layer", shared_inputs: bool = False, grouped: bool = False):
         assert mode in ("resident", "streamed", "no_h2d")
         assert api in ("layer", "proj")
+        assert not grouped or api == "layer", "groups are a feature of the layer calls"
         self.api = api
+        self.grouped = grouped
+        self.shared_inputs = shared_inputs or grouped
         self.cfg, self.mode, self.seed = cfg, mode, seed
         self.L = layers if layers is not None else cfg.layers
         self.T = tokens if tokens is not None else cfg.tokens
@@ -127,8 +137,12 @@ class Stack:
         for l in range(self.L):
             for pi, p in enumerate(self.proj):
                 la = l if distinct else 0
-                self.x[l, pi] = synth.device_normal((T, p.K), 1.0, self.seed, la, pi, synth.T_X, device=dev,
-                                                    dtype=torch.bfloat16) if (distinct or l == 0) else self.x[0, pi]
+                src = self._input_of(pi)
+                if src != pi:                                   # shares the x of an earlier projection
+                    self.x[l, pi] = self.x[l, src]
+                else:
+                    self.x[l, pi] = synth.device_normal((T, p.K), 1.0, self.seed, la, pi, synth.T_X, device=dev,
+                                                        dtype=torch.bfloat16) if (distinct or l == 0) else self.x[0, pi]
                 self.dY[l, pi] = synth.device_normal((T, p.N), 1.0, self.seed, la, pi, synth.T_DY, device=dev,
                                                      dtype=torch.bfloat16) if (distinct or l == 0) else self.dY[0, pi]
                 self.A[l, pi] = synth.device_uniform((r, p.K), 1.0 / p.K ** 0.5, self.seed, l, pi, synth.T_A,
@@ -283,6 +297,36 @@ class Stack:
             self._calls[key] = a
         return a
 
+    # q, k, v read the input of q; gate and up the input of gate (index into the projection list)
+    _GROUP_OF = {"q": 1, "k": 1, "v": 1, "gate": 2, "up": 2}
+    _INPUT_OF = {"k": "q", "v": "q", "up": "gate"}
+
+    def _input_of(self, pi: int) -> int:
+        if not self.shared_inputs:
+            return pi
+        names = [p.name for p in self.proj]
+        src = self._INPUT_OF.get(names[pi])
+        return names.index(src) if src in names else pi
+
+    def _group_of(self, pi: int) -> int:
+        return self._GROUP_OF.get(self.proj[pi].name, 0) if self.grouped else 0
+
+    def _leads(self, pi: int) -> bool:
+        g = self._group_of(pi)
+        return g == 0 or pi == 0 or self._group_of(pi - 1) != g
+
+    def with_inputs(self, shared_inputs: bool = True, grouped: bool = False, mode: str = "no_h2d",
+                    n_slots: int = 2) -> "Stack":
+        """A stack sharing this one's host blobs, with its own activations: shared inputs per group of
+        projections, and (grouped) the groups passed to the layer calls."""
+        import copy
+        other = copy.copy(self)
+        other.shared_inputs, other.grouped = shared_inputs or grouped, grouped
+        other.mode, other.pool, other.resident, other._calls = mode, None, None, {}
+        other._build_tensors(self._distinct)
+        other._setup_mode(n_slots)
+        return other
+
     def _layer_projs(self, addr: int, l: int, adapter: bool = True):
         """The lsn_lora_proj array of layer l whose blob sits at addr (cached: it depends on nothing else).
         adapter=False: A and B NULL, the frozen base alone (the reference model of preference training)."""
@@ -292,8 +336,10 @@ class Stack:
             projs = [lsnf4.lora_proj(self._base(addr, p), self.x[l, pi],
                                      self.A[l, pi] if adapter else None, self.B[l, pi] if adapter else None,
                                      y=self._out(self.y if adapter else self.y_ref, l, pi), dY=self.dY[l, pi],
-                                     dX=self._out(self.dX, l, pi), dA=self.dA[l, pi], dB=self.dB[l, pi],
-                                     u=self.u[l, pi] if (adapter and hasattr(self, "u")) else None)
+                                     dX=self._out(self.dX, l, pi) if self._leads(pi) else None,
+                                     dA=self.dA[l, pi], dB=self.dB[l, pi],
+                                     u=self.u[l, pi] if (adapter and hasattr(self, "u")) else None,
+                                     group=self._group_of(pi))
                      for pi, p in enumerate(self.proj)]
             a = lsnf4.proj_array(projs)
             if addr:

@@ -127,14 +127,15 @@ def test_struct_layouts_match_the_header(lib, tmp_path):
     src.write_text(
         '#include <stdio.h>\n#include <stddef.h>\n#include "lsnf4.h"\n'
         "int main(void) {\n"
-        '  printf("%zu %zu %zu %zu %zu %zu\\n", sizeof(lsn_nf4_weight), sizeof(lsn_base), sizeof(lsn_lora_proj),\n'
-        "         offsetof(lsn_base, nf4), offsetof(lsn_lora_proj, x), offsetof(lsn_lora_proj, u));\n"
+        '  printf("%zu %zu %zu %zu %zu %zu %zu\\n", sizeof(lsn_nf4_weight), sizeof(lsn_base), sizeof(lsn_lora_proj),\n'
+        "         offsetof(lsn_base, nf4), offsetof(lsn_lora_proj, x), offsetof(lsn_lora_proj, u),\n"
+        "         offsetof(lsn_lora_proj, group));\n"
         "  return 0;\n}\n")
     exe = tmp_path / "layout"
     subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
     got = [int(v) for v in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()]
     want = [ctypes.sizeof(lib.NF4Weight), ctypes.sizeof(lib.Base), ctypes.sizeof(lib.LoraProj),
-            lib.Base.nf4.offset, lib.LoraProj.x.offset, lib.LoraProj.u.offset]
+            lib.Base.nf4.offset, lib.LoraProj.x.offset, lib.LoraProj.u.offset, lib.LoraProj.group.offset]
     assert got == want
 
 

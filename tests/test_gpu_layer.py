@@ -216,3 +216,94 @@ def test_adapter_off_is_the_base_term(lib, orc):
         Wb = orc.nf4_dequant(q["packed"], q["absmax_q"], q["s2"], q["offset"], c.W.size).reshape(c.W.shape)
         zeroB = np.zeros_like(c.B)
         assert_close(bf16_tensor_to_f64(o["y"]), orc.lora_fwd(c.x, Wb, c.A, zeroB, L.scale), "y (adapter off)")
+
+
+# ------------------------------------------------------------------ groups --
+
+GROUPS = (1, 1, 1, 0, 2, 2, 0)       # q|k|v and gate|up read the same input
+SMALL_G = [(256, 256), (256, 128), (256, 64), (256, 256), (256, 512), (256, 384), (512, 256)]
+
+
+def _grouped_setup(lib, shapes, T, kind, seed):
+    """One x per group (q, k, v share x_attn; gate, up share x_mlp), bases laid out back to back
+    (one buffer per layer, like a pool slot)."""
+    import torch
+    L = Layer(lib, shapes, T, 16, kind, seed=seed)
+    for pi in (1, 2):
+        L.p[pi]["x"] = L.p[0]["x"]
+        L.p[pi]["case"].x = L.p[0]["case"].x
+    L.p[5]["x"] = L.p[4]["x"]
+    L.p[5]["case"].x = L.p[4]["case"].x
+    if kind == "bf16":
+        total = sum(d["N"] * d["K"] for d in L.p)
+        L.wbuf = torch.empty(total, dtype=torch.bfloat16, device="cuda")
+        off = 0
+        for d in L.p:
+            n = d["N"] * d["K"]
+            L.wbuf[off:off + n].copy_(d["Wb"].reshape(-1))
+            d["Wb"] = L.wbuf[off:off + n].view(d["N"], d["K"])
+            d["base"] = lib.base_bf16(d["Wb"], d["N"], d["K"])
+            off += n
+    return L
+
+
+def _run_layer(lib, L, out, groups):
+    import torch
+    projs = []
+    for pi, (d, o) in enumerate(zip(L.p, out)):
+        lead = groups[pi] == 0 or pi == 0 or groups[pi - 1] != groups[pi]
+        projs.append(lib.lora_proj(d["base"], d["x"], d["A"], d["B"], y=o["y"], dY=d["dY"],
+                                   dX=o["dX"] if lead else None, dA=o["dA"], dB=o["dB"], u=o["u"],
+                                   group=groups[pi]))
+    arr = lib.proj_array(projs)
+    n = lib.layer_ws_bytes(arr, L.T, L.r)
+    ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
+    lib.lora_layer_fwd(arr, L.T, L.r, L.scale, ws, n)
+    lib.lora_layer_bwd(arr, L.T, L.r, L.scale, False, ws, n)
+    torch.cuda.synchronize()
+    lib.ws_status(ws)
+    return out
+
+
+@pytest.mark.parametrize("shapes,T,kind", [(SHAPES_8B, 2048, "nf4"), (SMALL_G, 300, "bf16"), (SMALL_G, 77, "nf4"),
+                                          ([(896, 896), (896, 128), (896, 128), (896, 896), (896, 4864),
+                                            (896, 4864), (4864, 896)], 512, "bf16")])
+def test_grouped_projections(lib, orc, shapes, T, kind):
+    """Grouped forward: the same bits as ungrouped.  Grouped backward: the group's dX is the sum of the
+    members' input gradients (checked against the oracle's sum on sampled rows); dA, dB the same bits."""
+    L = _grouped_setup(lib, shapes, T, kind, seed=21)
+    plain = _run_layer(lib, L, L.outputs(), (0,) * 7)
+    grp = _run_layer(lib, L, L.outputs(), GROUPS)
+    _equal(grp, plain, ("y", "dA", "dB", "u"))
+    _equal([grp[3], grp[6]], [plain[3], plain[6]], ("dX",))          # ungrouped projections
+    rows = np.sort(np.random.default_rng(3).choice(T, size=min(T, 48), replace=False))
+    for members in ((0, 1, 2), (4, 5)):
+        ref = 0.0
+        for pi in members:
+            c = L.p[pi]["case"]
+            if kind == "nf4":
+                q = orc.nf4_quantize(c.W)
+                Wb = orc.nf4_dequant(q["packed"], q["absmax_q"], q["s2"], q["offset"], c.W.size).reshape(c.W.shape)
+            else:
+                Wb = synth.to_bf16_bits(c.W)
+            ref = ref + orc.lora_bwd_dx(c.dY, Wb, c.A, c.B, L.scale, rows=rows)
+        assert_close(bf16_tensor_to_f64(grp[members[0]]["dX"])[rows], ref, f"group {members} dX")
+
+
+def test_group_arguments_are_checked(lib):
+    import torch
+    L = _grouped_setup(lib, SMALL_G, 64, "nf4", seed=2)
+    out = L.outputs()
+    projs = [lib.lora_proj(d["base"], d["x"], d["A"], d["B"], y=o["y"], dY=d["dY"], dX=o["dX"], dA=o["dA"],
+                           dB=o["dB"], group=GROUPS[pi]) for pi, (d, o) in enumerate(zip(L.p, out))]
+    arr = lib.proj_array(projs)
+    n = lib.layer_ws_bytes(arr, L.T, L.r)
+    ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
+    with pytest.raises(lib.LsnError) as e:           # members 1, 2, 5 carry a dX
+        lib.lora_layer_bwd(arr, L.T, L.r, L.scale, False, ws, n)
+    assert e.value.status == lib.LSN_ERR_INVALID_ARG
+    projs[3].group = 1                               # o has its own x: cannot join q, k, v
+    projs[3].dX = None
+    with pytest.raises(lib.LsnError) as e:
+        lib.lora_layer_fwd(lib.proj_array(projs), L.T, L.r, L.scale, ws, n)
+    assert e.value.status == lib.LSN_ERR_INVALID_ARG

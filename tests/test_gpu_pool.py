@@ -182,3 +182,26 @@ def test_pool_rules(lib):
         assert st["copies"] == 2 and st["bytes_copied"] == 2 * n and st["misses"] == 2
     finally:
         lib.layer_pool_destroy(pool)
+
+
+def test_grouped_stack_matches_shared_inputs(lib):
+    """A stack whose q|k|v and gate|up run as groups gives the same y, dA and dB as the same stack run
+    ungrouped, streamed or resident; the grouped dX equals the ungrouped sum within bf16 rounding."""
+    import torch
+    from layer_streamed_nf4_b200.stack import Stack
+    cfg = synth.STACKS["8b"]
+    shared = Stack(cfg, layers=2, tokens=512, mode="resident", keep_outputs=True, shared_inputs=True)
+    shared.step()
+    grouped = shared.with_inputs(shared_inputs=True, grouped=True, mode="streamed")
+    grouped.step()
+    torch.cuda.synchronize()
+    grouped.check_status()
+    assert all(torch.equal(shared.y[k], grouped.y[k]) for k in shared.y)
+    assert all(torch.equal(shared.dA[k], grouped.dA[k]) and torch.equal(shared.dB[k], grouped.dB[k]) for k in shared.dA)
+    for l in range(2):
+        for members in ((0, 1, 2), (4, 5)):
+            ref = sum(shared.dX[l, pi].double() for pi in members)
+            got = grouped.dX[l, members[0]].double()
+            err = float((got - ref).norm() / ref.norm())
+            assert err < 5e-3, (l, members, err)
+    grouped.close()
