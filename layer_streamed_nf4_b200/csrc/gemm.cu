@@ -257,6 +257,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
     } else {
         // -------------------------------------------------------- epilogue --
         const int q = warp & 3;                    // TMEM lanes 32q .. 32q+31
+        const int nseg = p.nseg;
         int acc = 0;
         uint32_t acc_phase = 0;
         for (int tile = unit; tile < num_tiles; tile += nunits) {
@@ -273,16 +274,15 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
                 tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c * 32), v);
                 tmem_ld_wait();
                 if (row < p.M) {
-                    // Output segment of these 32 columns (segment widths are multiples of 64).
                     uint16_t* base = p.D;
                     int64_t ld = p.ldd;
                     int lc = col;
-                    for (int sgi = 0; sgi < p.nseg; ++sgi) {
-                        if (col >= p.seg_col[sgi] && col < p.seg_col[sgi + 1]) {
-                            base = p.seg_D[sgi];
-                            ld = p.seg_ld[sgi];
-                            lc = col - p.seg_col[sgi];
-                        }
+                    if (nseg > 0) {                // the segment of these 32 columns (widths: multiples of 64)
+                        int sgi = 0;
+                        while (sgi + 1 < nseg && col >= p.seg_col[sgi + 1]) ++sgi;
+                        base = p.seg_D[sgi];
+                        ld = p.seg_ld[sgi];
+                        lc = col - p.seg_col[sgi];
                     }
                     uint4* dst = reinterpret_cast<uint4*>(base + (int64_t)row * ld + lc);
                     #pragma unroll
