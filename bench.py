@@ -370,36 +370,49 @@ def _traffic_from_profile():
 
 # ------------------------------------------------------------ reference ---
 
+_ORACLE_CASES = {}
+
+
+def _oracle_cases(sample_rows: int):
+    """Inputs of the oracle sample: `sample_rows` token rows of the workload's distributions for each of the
+    seven projections of one layer, weights NF4 through the oracle's own quantiser (built once, untimed)."""
+    import oracle
+    from layer_streamed_nf4_b200 import synth
+    if sample_rows not in _ORACLE_CASES:
+        cfg = synth.STACKS[WORKLOAD]
+        cases = []
+        for pi, (name, K, N) in enumerate(cfg.projections):
+            c = synth.linear_case(sample_rows, K, N, cfg.rank, cfg.alpha, seed=synth.SEED, layer=0, proj=pi)
+            q = oracle.nf4_quantize(c.W)
+            Wb = oracle.nf4_dequant(q["packed"], q["absmax_q"], q["s2"], q["offset"], c.W.size).reshape(N, K)
+            cases.append((c, Wb))
+        _ORACLE_CASES[sample_rows] = cases
+    return _ORACLE_CASES[sample_rows]
+
+
 def cpu_baseline(args, sample_rows: int, budget_s: float):
     """The oracle (fp64, plain loops, OpenMP over rows) on a bounded sample: `sample_rows` token rows through
     the seven projections of one 8B-shaped layer, fwd + bwd.  Step time per token is scaled by the layer count
     (derived, arithmetic)."""
-    import numpy as np
-
     import oracle
     from layer_streamed_nf4_b200 import synth
     cfg = synth.STACKS[WORKLOAD]
     L = cfg.layers
     cores = os.cpu_count() or 1
-    # Inputs: a few rows of the same distributions; weights NF4 via the oracle.
-    t_total = 0.0
-    rows_done = 0
-    cases = []
-    for pi, (name, K, N) in enumerate(cfg.projections):
-        c = synth.linear_case(sample_rows, K, N, cfg.rank, cfg.alpha, seed=synth.SEED, layer=0, proj=pi)
-        q = oracle.nf4_quantize(c.W)
-        Wb = oracle.nf4_dequant(q["packed"], q["absmax_q"], q["s2"], q["offset"], c.W.size).reshape(N, K)
-        cases.append((c, Wb))
+    cases = _oracle_cases(sample_rows)
+    work_all = sum(c.K * c.N for c, _ in cases)
+    work_done = 0
     t0 = time.perf_counter()
     for c, Wb in cases:
         oracle.lora_fwd(c.x, Wb, c.A, c.B, c.scale)
         oracle.lora_bwd_dx(c.dY, Wb, c.A, c.B, c.scale)
         oracle.lora_bwd_dadb(c.x, c.dY, c.A, c.B, c.scale)
-        if time.perf_counter() - t0 > budget_s:
+        work_done += c.K * c.N
+        if time.perf_counter() - t0 > budget_s:     # out of budget: scale by the share of the layer done
             break
     t_total = time.perf_counter() - t0
     rows_done = sample_rows
-    s_per_token_step = t_total / rows_done * L
+    s_per_token_step = t_total / rows_done * L * (work_all / work_done)
     return {"value": 1.0 / s_per_token_step, "unit": UNIT, "cores": cores, "kind": "oracle",
             "sample": f"{rows_done} token rows through the 7 projections of one {cfg.name} layer (fwd+bwd, "
                       f"fp64 oracle, OpenMP); per-step time = layer time x {L} layers (derived, arithmetic)",
@@ -414,7 +427,7 @@ def run_reference(args):
     cfg = synth.STACKS[WORKLOAD]
     vals = []
     for i in range(args.warmup + args.steps):
-        cb = cpu_baseline(args, sample_rows=args.ref_rows, budget_s=1e9)
+        cb = cpu_baseline(args, sample_rows=max(args.ref_rows, os.cpu_count() or 1), budget_s=1e9)
         if i >= args.warmup:
             vals.append(cb)
     v = statistics.median(c["value"] for c in vals)
@@ -496,9 +509,9 @@ def main():
     ap.add_argument("--lanes", type=int, default=2, help="streams the seven projections of a layer are spread over")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-rows", type=int, default=32)
+    ap.add_argument("--cpu-rows", type=int, default=768, help="token rows of the timed oracle sample")
     ap.add_argument("--cpu-budget", type=float, default=60.0)
-    ap.add_argument("--ref-rows", type=int, default=4)
+    ap.add_argument("--ref-rows", type=int, default=64, help="token rows per step of the reference arm")
     ap.add_argument("--fused-nf4", action="store_true", help="convert NF4 inside the GEMM (no bf16 copy of W)")
     ap.add_argument("--no-pdl", action="store_true", help="ordinary launches instead of programmatic dependent ones")
     ap.add_argument("--case", default="", help="profile one 8B projection (q,k,v,o,gate,up,down) instead of the stack")
