@@ -111,6 +111,31 @@ def test_recompute_and_reference_steps(lib):
     plain.close()
 
 
+@pytest.mark.parametrize("mode", ["streamed", "no_h2d"])
+def test_dequant_ahead_gives_the_same_bits(lib, mode):
+    """Dequantising each layer on a side stream one layer ahead (bf16 bases into the layer calls) and
+    dequantising inside the layer calls give the same bits."""
+    import torch
+    from layer_streamed_nf4_b200.stack import Stack
+    cfg = synth.STACKS["8b"]
+    inside = Stack(cfg, layers=3, tokens=256, mode=mode, keep_outputs=True, dequant_ahead=False)
+    ahead = Stack(cfg, layers=3, tokens=256, mode=mode, keep_outputs=True, dequant_ahead=True)
+    assert ahead.ahead and not inside.ahead
+    auto = Stack(cfg, layers=2, tokens=64, mode=mode)
+    assert auto.ahead == (mode == "streamed") and not auto.with_mode("resident").ahead
+    auto.close()
+    for st in (inside, ahead):
+        st.step()
+        st.step(reference=True, recompute=True)
+    torch.cuda.synchronize()
+    ahead.check_status()
+    fwd, bwd, bad = _compare(ahead, inside)
+    assert fwd and bwd, bad
+    assert all(torch.equal(ahead.y_ref[k], inside.y_ref[k]) for k in ahead.y_ref)
+    inside.close()
+    ahead.close()
+
+
 def test_no_h2d_equals_resident(lib):
     cfg = synth.STACKS["8b"]
     res = _run(cfg, 3, 512, "resident")
