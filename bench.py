@@ -107,35 +107,59 @@ def _dist():
     return n, rank, local
 
 
+class Replicas:
+    """The N > 1 plumbing: one process per GPU (launched by torchrun), each an independent replica of the
+    path (no collective on the data path: the method does not shard).  Timed regions are bracketed by
+    barriers, every timed figure is the max over ranks, and throughput counts the tokens of all ranks."""
+
+    def __init__(self, backend: str, device):
+        import torch.distributed as dist
+        self.world, self.rank, self.local = _dist()
+        self.device = device
+        self.dist = dist
+        if self.world > 1 and not dist.is_initialized():
+            from datetime import timedelta
+            kw = {"device_id": device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=timedelta(seconds=300), **kw)
+
+    def barrier(self):
+        if self.world > 1:
+            self.dist.barrier()
+
+    def max(self, v: float) -> float:
+        if self.world == 1:
+            return v
+        import torch
+        t = torch.tensor([v], dtype=torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def throughput(self, tokens_per_rank: int, ms: float) -> float:
+        return self.world * tokens_per_rank / (ms / 1e3)
+
+    def close(self):
+        if self.world > 1 and self.dist.is_initialized():
+            self.dist.destroy_process_group()
+
+
 # ----------------------------------------------------------------- ours ---
 
 def run_ours(args):
     import torch
-    import torch.distributed as dist
     from layer_streamed_nf4_b200 import lsnf4, synth
     from layer_streamed_nf4_b200.stack import Stack
 
     world, rank, local = _dist()
     torch.cuda.set_device(local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+    reps = Replicas("nccl", torch.device("cuda", local))
     cfg = synth.STACKS[WORKLOAD]
     T = args.tokens or cfg.tokens
     L = args.layers or cfg.layers
     stream = torch.cuda.Stream()
     peaks = _peaks()
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    barrier = reps.barrier
+    max_over_ranks = reps.max
 
     results = {}
     host_issue = {}
@@ -271,20 +295,19 @@ def run_ours(args):
         barrier()
         ems = max_over_ranks(e0.elapsed_time(e1) / args.steps)
         ps = st.pool_stats() or {"bytes_copied": 0}
-        e2e = {"value": world * T / (ems / 1e3), "unit": UNIT,
+        e2e = {"value": reps.throughput(T, ems), "unit": UNIT,
                "h2d_bytes_per_step": int(bi + (ps["bytes_copied"] - ps0["bytes_copied"]) / max(args.steps, 1)),
                "d2h_bytes_per_step": int(bo), "ms_per_step": ems}
 
     st_main.check_status()
-    if world > 1:
-        dist.destroy_process_group()
+    reps.close()
     if rank != 0:
         st_main.close()
         return
 
     ms = results["streamed"]
     flop_step = st_main.flop_per_step()
-    value = world * T / (ms / 1e3)
+    value = reps.throughput(T, ms)
 
     g = {k: kernel[k] for k in ("gemm_fwd", "gemm_bwd")}
     g_ms = sum(v["ms"] for v in g.values())
