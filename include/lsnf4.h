@@ -179,9 +179,9 @@ typedef struct {
 } lsn_base;
 
 /* Workspace bytes lora_linear_fwd / lora_linear_bwd need (the larger of the two).
- * The workspace holds a status word and the tickets of the deterministic split
- * reductions, which must start at zero: fill a new workspace with zeros once
- * (they return to zero at the end of every call). */
+ * The workspace starts with the kernels' status word, which must start at
+ * zero: fill a new workspace with zeros once (lsn_ws_status clears it after
+ * reporting a timeout). */
 size_t lsn_lora_ws_bytes(int64_t T, int64_t K, int64_t N, int r, int kind);
 
 /* Forward.  y may not alias x.  ws: device scratch of lsn_lora_ws_bytes bytes,

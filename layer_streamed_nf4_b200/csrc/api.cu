@@ -82,22 +82,17 @@ lsn_status check_nf4(const lsn_nf4_weight* w, const char* who) {
 
 // Workspace layout of the LoRA calls (each region 256-byte aligned):
 //   [0, 256)  status word of the GEMM kernels
-//   cnt  int32           tickets of the split reductions (self-resetting)
 //   u32  fp32 [T, r]     x A^T
 //   g32  fp32 [T, r]     dY B
 //   s16  bf16 [T, r]     bf16(s u) or bf16(s g)
-//   part fp32 split partials (down projections and token reductions, used
-//        one after the other on the stream)
 //   w16  bf16 [N, K]     dequantised base (NF4 base only)
-// The status word and the tickets must be zero when the workspace is first
-// used: fill the workspace with zeros once, when it is allocated.
+// The status word must be zero when the workspace is first used: fill the
+// workspace with zeros once, when it is allocated.
 struct LoraWs {
     int* err;
-    int* cnt;
     float* u32;
     float* g32;
     uint16_t* s16;
-    float* part;
     uint16_t* w16;
     size_t total;
 };
@@ -108,13 +103,9 @@ LoraWs carve(void* ws, int64_t T, int64_t K, int64_t N, int r, int kind) {
     char* b = reinterpret_cast<char*>(ws);
     auto take = [&](size_t bytes) { char* p = b ? b + off : nullptr; off += round_up(bytes, 256); return p; };
     w.err = reinterpret_cast<int*>(take(256));
-    w.cnt = reinterpret_cast<int*>(take(split_counter_count(T, K, N) * sizeof(int)));
     w.u32 = reinterpret_cast<float*>(take((size_t)T * r * 4));
     w.g32 = reinterpret_cast<float*>(take((size_t)T * r * 4));
     w.s16 = reinterpret_cast<uint16_t*>(take((size_t)T * r * 2));
-    size_t part = tgrad_ws_bytes(T, K, r);
-    for (size_t v : {tgrad_ws_bytes(T, N, r), down_ws_bytes(T, K, r), down_ws_bytes(T, N, r)}) part = v > part ? v : part;
-    w.part = reinterpret_cast<float*>(take(part));
     w.w16 = reinterpret_cast<uint16_t*>(take(kind == LSN_BASE_NF4 ? (size_t)N * K * 2 : 0));
     w.total = off;
     return w;
@@ -388,14 +379,14 @@ lsn_status timed_down(const uint16_t* X, const uint16_t* W, bool w_rk, int64_t T
                       float* u32, uint16_t* u16, const LoraWs& w, cudaStream_t st) {
     const double bytes = 2.0 * T * Kd + 2.0 * r * Kd + (u32 ? 4.0 * T * r : 0.0) + (u16 ? 2.0 * T * r : 0.0);
     TimingScope ts(LSN_K_LORA_DOWN, bytes, st, 1);
-    return launch_lora_down(X, W, w_rk, T, Kd, r, scale, u32, u16, w.part, w.cnt, st);
+    return launch_lora_down(X, W, w_rk, T, Kd, r, scale, u32, u16, st);
 }
 
 lsn_status timed_tgrad(const float* G, const uint16_t* X, bool out_rk, int64_t T, int64_t Kd, int r, float scale,
                        int accumulate, float* out, const LoraWs& w, cudaStream_t st) {
     const double bytes = 2.0 * T * Kd + 4.0 * T * r + 4.0 * r * Kd * (accumulate ? 2.0 : 1.0);
     TimingScope ts(LSN_K_LORA_TGRAD, bytes, st, 1);
-    return launch_lora_tgrad(G, X, out_rk, T, Kd, r, scale, accumulate, out, w.part, w.cnt, st);
+    return launch_lora_tgrad(G, X, out_rk, T, Kd, r, scale, accumulate, out, st);
 }
 
 lsn_status timed_gemm(int kind, const uint16_t* A, int64_t lda, const uint16_t* B, int64_t ldb, bool b_mn,

@@ -76,14 +76,11 @@ lsn_status launch_gemm_nf4(const uint16_t* A, int64_t lda, const lsn_nf4_weight*
 bool gemm_use_pairs(int64_t M, int64_t N);
 
 lsn_status launch_lora_down(const uint16_t* X, const uint16_t* W, bool w_rk, int64_t T, int64_t Kd, int r,
-                            float scale, float* u32, uint16_t* u16, float* partial, int* counters, cudaStream_t st);
+                            float scale, float* u32, uint16_t* u16, cudaStream_t st);
 lsn_status launch_lora_down_batch(int n, const DownSpec* specs, bool w_rk, int r, cudaStream_t st);
 lsn_status launch_lora_tgrad(const float* G, const uint16_t* X, bool out_rk, int64_t T, int64_t Kd, int r,
-                             float scale, int accumulate, float* out, float* partial, int* counters, cudaStream_t st);
+                             float scale, int accumulate, float* out, cudaStream_t st);
 lsn_status launch_lora_tgrad_batch(int n, const TgSpec* specs, int r, cudaStream_t st);
-size_t down_ws_bytes(int64_t T, int64_t Kd, int r);
-size_t tgrad_ws_bytes(int64_t T, int64_t Kd, int r);
-size_t split_counter_count(int64_t T, int64_t K, int64_t N);
 int down_splits(int64_t T, int64_t Kd);
 int tgrad_splits(int64_t T, int64_t Kd);
 

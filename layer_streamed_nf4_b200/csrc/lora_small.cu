@@ -556,7 +556,6 @@ int down_splits(int64_t T, int64_t Kd) {
     return (int)s;
 }
 
-size_t down_ws_bytes(int64_t, int64_t, int) { return 0; }
 
 // Token splits of a reduction: up to 8 (one cluster), aiming at about four
 // 128-thread CTAs per SM, at least 64 tokens per split.
@@ -571,9 +570,6 @@ int tgrad_splits(int64_t T, int64_t Kd) {
     return (int)s;
 }
 
-size_t tgrad_ws_bytes(int64_t, int64_t, int) { return 0; }
-
-size_t split_counter_count(int64_t, int64_t, int64_t) { return 0; }
 
 // Down projections of a batch of problems, all with W in the same layout
 // (w_rk: A [r, Kd]; otherwise B [Kd, r]) and the same rank.  Problems with
@@ -654,13 +650,13 @@ lsn_status launch_lora_tgrad_batch(int n, const TgSpec* specs, int r, cudaStream
 
 // X [T, Kd] times W: w_rk ? W is A [r, Kd] : W is B [Kd, r].
 lsn_status launch_lora_down(const uint16_t* X, const uint16_t* W, bool w_rk, int64_t T, int64_t Kd, int r,
-                            float scale, float* u32, uint16_t* u16, float*, int*, cudaStream_t st) {
+                            float scale, float* u32, uint16_t* u16, cudaStream_t st) {
     const DownSpec d{X, W, u32, u16, T, Kd, scale};
     return launch_lora_down_batch(1, &d, w_rk, r, st);
 }
 
 lsn_status launch_lora_tgrad(const float* G, const uint16_t* X, bool out_rk, int64_t T, int64_t Kd, int r,
-                             float scale, int accumulate, float* out, float*, int*, cudaStream_t st) {
+                             float scale, int accumulate, float* out, cudaStream_t st) {
     const TgSpec d{G, X, out, T, Kd, out_rk, accumulate, scale};
     return launch_lora_tgrad_batch(1, &d, r, st);
 }
