@@ -238,6 +238,7 @@ def run_ours(args):
             # without them.)  It runs with one lane, so that no launch waits
             # for SMs held by another lane's kernel inside its events.
             st_k = st.with_mode("streamed", n_slots=args.slots, lanes=1)
+            st_k.ahead = False                    # no dequantisation on a side stream either
             lanes_opt = lsnf4.get_option(lsnf4.LSN_OPT_LAYER_LANES)
             lsnf4.set_option(lsnf4.LSN_OPT_LAYER_LANES, 1)
             try:

@@ -154,6 +154,17 @@ lsn_status nf4_quantize_noalloc(const float* W, const lsn_nf4_weight* out, lsn_s
 /* Dequantise *w into bf16 W_out [rows, cols] (device).  HBM-bound. */
 lsn_status nf4_dequant(const lsn_nf4_weight* w, uint16_t* W_out, lsn_stream_t stream);
 
+/* Dequantise n weights with one launch (e.g. the projections of a layer):
+ * w is a HOST array of n weights, W_out a HOST array of n device pointers
+ * (bf16 [rows_i, cols_i] each, 16-byte aligned, not overlapping), both read
+ * during the call only.  Same bits as n nf4_dequant calls.  Any n >= 0; more
+ * than 16 weights take several launches.  blocks_per_sm: 0 = as many blocks
+ * as the work has (fastest on an idle GPU); k > 0 = at most k blocks per SM,
+ * looping over the work, for a dequantisation that runs beside other
+ * kernels (e.g. the next layer's weights under the current layer's GEMMs). */
+lsn_status nf4_dequant_batch(int n, const lsn_nf4_weight* w, uint16_t* const* W_out, int blocks_per_sm,
+                             lsn_stream_t stream);
+
 /* ------------------------------------------------------------ LoRA linear --
  *
  * y  = x W^T + s (x A^T) B^T                        (forward)

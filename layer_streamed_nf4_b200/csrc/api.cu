@@ -454,6 +454,38 @@ lsn_status nf4_dequant(const lsn_nf4_weight* w, uint16_t* W_out, lsn_stream_t st
     return timed_dequant(w, W_out, reinterpret_cast<cudaStream_t>(stream));
 }
 
+lsn_status nf4_dequant_batch(int n, const lsn_nf4_weight* w, uint16_t* const* W_out, int blocks_per_sm,
+                             lsn_stream_t stream) {
+    LSN_CHECK_ARG(n >= 0 && blocks_per_sm >= 0, "nf4_dequant_batch: n and blocks_per_sm must be >= 0");
+    if (n == 0) return LSN_OK;
+    LSN_CHECK_ARG(w != nullptr && W_out != nullptr, "nf4_dequant_batch: NULL array");
+    const lsn_nf4_weight* ws[16];
+    uint16_t* outs[16];
+    double bytes = 0.0;
+    for (int i = 0; i < n; ++i) {
+        lsn_status s = check_nf4(&w[i], "nf4_dequant_batch");
+        if (s != LSN_OK) return s;
+        if (w[i].rows * w[i].cols != 0)
+            LSN_CHECK_ARG(W_out[i] != nullptr && aligned16(W_out[i]),
+                          "nf4_dequant_batch: outputs must be 16-byte aligned device pointers");
+    }
+    lsn_status s = check_device();
+    if (s != LSN_OK) return s;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    for (int i0 = 0; i0 < n; i0 += 16) {
+        const int m = n - i0 < 16 ? n - i0 : 16;
+        bytes = 0.0;
+        for (int j = 0; j < m; ++j) {
+            ws[j] = &w[i0 + j];
+            outs[j] = W_out[i0 + j];
+            bytes += dequant_bytes(w[i0 + j].rows, w[i0 + j].cols);
+        }
+        TimingScope ts(LSN_K_DEQUANT, bytes, st);
+        if ((s = launch_dequant_batch(m, ws, outs, st, blocks_per_sm)) != LSN_OK) return s;
+    }
+    return LSN_OK;
+}
+
 size_t lsn_lora_ws_bytes(int64_t T, int64_t K, int64_t N, int r, int kind) {
     return carve(nullptr, T, K, N, r, kind).total;
 }

@@ -222,55 +222,60 @@ constexpr int kDqWarps = kDqThreads / 32;
 __device__ __forceinline__ int dq_stage_chunk(int c) { return c ^ ((c >> 3) & 7); }
 
 __global__ void __launch_bounds__(kDqThreads) nf4_dequant_kernel(const __grid_constant__ DqBatch bt,
-                                                                 const __grid_constant__ DequantParams P) {
+                                                                 const __grid_constant__ DequantParams P,
+                                                                 int64_t units) {
     __shared__ float dq[256];
     __shared__ uint4 stage[kDqWarps][128];                 // 2 KB per warp: 32 lanes x 64 bytes
     for (int i = threadIdx.x; i < 256; i += blockDim.x) dq[i] = P.dq[i];
-    int ii = 0;
-    while (ii + 1 < bt.n && (int64_t)blockIdx.x >= bt.it[ii + 1].first) ++ii;
-    const DqItem& it = bt.it[ii];
     pdl_launch_dependents();
     pdl_wait();
-    const uint4* __restrict__ packed = it.packed;
-    const uint8_t* __restrict__ absmax_q = it.absmax_q;
-    const float* __restrict__ s2 = it.s2;
-    uint4* __restrict__ out = it.out;
-    const float off = *it.offset;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t v0 = ((int64_t)blockIdx.x - it.first) * kDqVecPerBlock + threadIdx.x;
-    uint4 p[kDqUnroll];
-    uint32_t code[kDqUnroll];
-    float sc[kDqUnroll];
-    #pragma unroll
-    for (int u = 0; u < kDqUnroll; ++u) {
-        const int64_t v = v0 + u * kDqThreads;
-        const bool ok = v < it.nvec;
-        const int64_t b = (ok ? v : 0) >> 1;             // absmax block of the vector
-        p[u] = ok ? __ldg(packed + v) : make_uint4(0, 0, 0, 0);
-        code[u] = __ldg(absmax_q + b);
-        sc[u] = __ldg(s2 + (b >> 8));
-    }
     __syncthreads();                                     // the code table is in shared memory
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint4* st = stage[warp];
-    #pragma unroll
-    for (int u = 0; u < kDqUnroll; ++u) {
-        const float ah = __fadd_rn(__fmul_rn(dq[code[u]], sc[u]), off);
-        uint32_t lo[4], hi[4];
-        nf4_scaled_table(P.level, ah, lo, hi);
-        st[dq_stage_chunk(4 * lane + 0)] = nf4x8_to_bf16(p[u].x, lo, hi);
-        st[dq_stage_chunk(4 * lane + 1)] = nf4x8_to_bf16(p[u].y, lo, hi);
-        st[dq_stage_chunk(4 * lane + 2)] = nf4x8_to_bf16(p[u].z, lo, hi);
-        st[dq_stage_chunk(4 * lane + 3)] = nf4x8_to_bf16(p[u].w, lo, hi);
-        __syncwarp();
-        // The warp's 32 consecutive words start at word w0; their output is
-        // 2 KB at out + 4 * w0, written as four 512-byte rows.
-        const int64_t w0 = v0 - lane + u * kDqThreads;
+    // One unit = 1024 consecutive words of one weight; a full grid has one
+    // block per unit, a smaller one loops over them with the grid's stride.
+    for (int64_t unit = blockIdx.x; unit < units; unit += gridDim.x) {
+        int ii = 0;
+        while (ii + 1 < bt.n && unit >= bt.it[ii + 1].first) ++ii;
+        const DqItem& it = bt.it[ii];
+        const uint4* __restrict__ packed = it.packed;
+        const uint8_t* __restrict__ absmax_q = it.absmax_q;
+        const float* __restrict__ s2 = it.s2;
+        uint4* __restrict__ out = it.out;
+        const float off = *it.offset;
+        const int64_t v0 = (unit - it.first) * kDqVecPerBlock + threadIdx.x;
+        uint4 p[kDqUnroll];
+        uint32_t code[kDqUnroll];
+        float sc[kDqUnroll];
         #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int c = 32 * i + lane;                 // output chunk of the warp, in 16-byte units
-            if (w0 + (c >> 2) < it.nvec) out[4 * w0 + c] = st[dq_stage_chunk(c)];
+        for (int u = 0; u < kDqUnroll; ++u) {
+            const int64_t v = v0 + u * kDqThreads;
+            const bool ok = v < it.nvec;
+            const int64_t b = (ok ? v : 0) >> 1;         // absmax block of the vector
+            p[u] = ok ? __ldg(packed + v) : make_uint4(0, 0, 0, 0);
+            code[u] = __ldg(absmax_q + b);
+            sc[u] = __ldg(s2 + (b >> 8));
         }
-        __syncwarp();
+        #pragma unroll
+        for (int u = 0; u < kDqUnroll; ++u) {
+            const float ah = __fadd_rn(__fmul_rn(dq[code[u]], sc[u]), off);
+            uint32_t lo[4], hi[4];
+            nf4_scaled_table(P.level, ah, lo, hi);
+            st[dq_stage_chunk(4 * lane + 0)] = nf4x8_to_bf16(p[u].x, lo, hi);
+            st[dq_stage_chunk(4 * lane + 1)] = nf4x8_to_bf16(p[u].y, lo, hi);
+            st[dq_stage_chunk(4 * lane + 2)] = nf4x8_to_bf16(p[u].z, lo, hi);
+            st[dq_stage_chunk(4 * lane + 3)] = nf4x8_to_bf16(p[u].w, lo, hi);
+            __syncwarp();
+            // The warp's 32 consecutive words start at word w0; their output is
+            // 2 KB at out + 4 * w0, written as four 512-byte rows.
+            const int64_t w0 = v0 - lane + u * kDqThreads;
+            #pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int c = 32 * i + lane;             // output chunk of the warp, in 16-byte units
+                if (w0 + (c >> 2) < it.nvec) out[4 * w0 + c] = st[dq_stage_chunk(c)];
+            }
+            __syncwarp();
+        }
     }
 }
 
@@ -315,7 +320,8 @@ lsn_status launch_quantize(const float* W, const lsn_nf4_weight* out, void* ws, 
     return LSN_OK;
 }
 
-lsn_status launch_dequant_batch(int n, const lsn_nf4_weight* const* w, uint16_t* const* out, cudaStream_t st) {
+lsn_status launch_dequant_batch(int n, const lsn_nf4_weight* const* w, uint16_t* const* out, cudaStream_t st,
+                                int blocks_per_sm) {
     const Nf4Tables& T = nf4_tables();
     DequantParams P;
     std::memcpy(P.level, T.level, sizeof(P.level));
@@ -325,13 +331,15 @@ lsn_status launch_dequant_batch(int n, const lsn_nf4_weight* const* w, uint16_t*
     auto flush = [&]() -> lsn_status {
         if (bt.n == 0) return LSN_OK;
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)blocks);
+        int64_t grid = blocks;
+        if (blocks_per_sm > 0 && grid > (int64_t)sm_count() * blocks_per_sm) grid = (int64_t)sm_count() * blocks_per_sm;
+        cfg.gridDim = dim3((unsigned)grid);
         cfg.blockDim = dim3(kDqThreads);
         cfg.stream = st;
         cudaLaunchAttribute attr[1];
         cfg.attrs = attr;
         cfg.numAttrs = pdl_attr(&attr[0]);
-        LSN_CUDA_TRY(cudaLaunchKernelEx(&cfg, nf4_dequant_kernel, bt, P));
+        LSN_CUDA_TRY(cudaLaunchKernelEx(&cfg, nf4_dequant_kernel, bt, P, blocks));
         bt = DqBatch{};
         blocks = 0;
         return LSN_OK;

@@ -46,7 +46,10 @@ size_t quantize_ws_bytes(int64_t rows, int64_t cols);
 lsn_status launch_quantize(const float* W, const lsn_nf4_weight* out, void* ws, size_t ws_bytes, cudaStream_t st);
 lsn_status launch_dequant(const lsn_nf4_weight* w, uint16_t* out, cudaStream_t st);
 // Several NF4 weights dequantised by one launch (at most 16 per launch; more take several).
-lsn_status launch_dequant_batch(int n, const lsn_nf4_weight* const* w, uint16_t* const* out, cudaStream_t st);
+// blocks_per_sm > 0 caps the grid at that many blocks per SM (which then loop
+// over the work), for a dequantisation meant to run beside other kernels.
+lsn_status launch_dequant_batch(int n, const lsn_nf4_weight* const* w, uint16_t* const* out, cudaStream_t st,
+                                int blocks_per_sm = 0);
 
 // Grouped GEMM operands: the A operand as na tensors side by side along the
 // contraction (tensor i: [M, a_kc[i]] row-major with row stride lda[i]; every

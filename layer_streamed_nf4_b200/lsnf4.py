@@ -43,7 +43,7 @@ EXPORTS = (
     "layer_pool_release", "layer_pool_wait_idle", "layer_pool_stats", "layer_pool_reset",
     "layer_pool_inject_fault", "layer_pool_destroy", "lsn_timing_enable", "lsn_timing_read",
     "nf4_quantize_noalloc", "lsn_set_option", "lsn_get_option",
-    "lsn_layer_ws_bytes", "lora_layer_fwd", "lora_layer_bwd",
+    "lsn_layer_ws_bytes", "lora_layer_fwd", "lora_layer_bwd", "nf4_dequant_batch",
 )
 
 
@@ -105,6 +105,7 @@ for _n in ("lsn_nf4_packed_bytes", "lsn_nf4_absmax_bytes", "lsn_nf4_s2_bytes", "
 _sig("lsn_nf4_blob_layout", None, [_i64, _i64, ctypes.POINTER(_sz)])
 _sig("nf4_quantize", _i, [_vp, ctypes.POINTER(NF4Weight), _vp, _sz, _vp])
 _sig("nf4_dequant", _i, [ctypes.POINTER(NF4Weight), _vp, _vp])
+_sig("nf4_dequant_batch", _i, [_i, ctypes.POINTER(NF4Weight), ctypes.POINTER(_vp), _i, _vp])
 _sig("nf4_quantize_noalloc", _i, [_vp, ctypes.POINTER(NF4Weight), _vp])
 _sig("lsn_lora_ws_bytes", _sz, [_i64, _i64, _i64, _i, _i])
 _sig("lora_linear_fwd", _i, [ctypes.POINTER(Base), _vp, _i64, _vp, _vp, _i, ctypes.c_float, _vp, _vp, _sz, _vp])
@@ -215,6 +216,17 @@ NF4_NOALLOC_MAX_ELEMS = 1 << 26
 
 def nf4_dequant(w: NF4Weight, W_out, stream=None):
     _check(_lib.nf4_dequant(ctypes.byref(w), _ptr(W_out), _stream(stream)), "nf4_dequant")
+
+
+def dequant_batch_args(weights, outs):
+    """(n, weight array, output-pointer array) for nf4_dequant_batch; keep the arrays alive while used."""
+    n = len(weights)
+    return n, (NF4Weight * n)(*weights), (ctypes.c_void_p * n)(*[_ptr(o) for o in outs])
+
+
+def nf4_dequant_batch(weights, outs, blocks_per_sm: int = 0, stream=None):
+    n, wa, oa = dequant_batch_args(weights, outs)
+    _check(_lib.nf4_dequant_batch(n, wa, oa, blocks_per_sm, _stream(stream)), "nf4_dequant_batch")
 
 
 # --------------------------------------------------------- LoRA linear ---

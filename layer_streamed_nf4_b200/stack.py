@@ -394,15 +394,16 @@ class Stack:
         ps = self._prep
         ps.wait_event(self._ev_done[b])
         addr = self._acquire(l, ps)
-        deq = lsnf4._lib.nf4_dequant
-        for pi, p in enumerate(self.proj):
-            key = ("W", addr, pi)
-            w = self._calls.get(key)
-            if w is None:
-                w = self._calls[key] = lsnf4.nf4_weight_in_blob(p.N, p.K, addr + p.offset)
-            st = deq(ctypes.byref(w), self._wbuf[b].data_ptr() + 2 * self._woff[pi], ps.cuda_stream)
-            if st:
-                lsnf4._check(st, "nf4_dequant")
+        key = ("D", addr, b)
+        args = self._calls.get(key)
+        if args is None:                          # one launch for the layer's projections
+            ws = [lsnf4.nf4_weight_in_blob(p.N, p.K, addr + p.offset) for p in self.proj]
+            outs = [self._wbuf[b].data_ptr() + 2 * self._woff[pi] for pi in range(len(self.proj))]
+            args = self._calls[key] = lsnf4.dequant_batch_args(ws, outs)
+        # two blocks per SM: the dequantisation trickles along beside the current layer's GEMMs
+        st = lsnf4._lib.nf4_dequant_batch(*args, 2, ps.cuda_stream)
+        if st:
+            lsnf4._check(st, "nf4_dequant_batch")
         self._release(l, ps)
         self._ev_ready[b].record(ps)
 

@@ -195,3 +195,15 @@ def test_options(lib):
     assert lib.get_option(lib.LSN_OPT_PDL) == 0
     lib.set_option(lib.LSN_OPT_PDL, 1)
     assert lib.get_option(12345) == -1
+
+
+def test_dequant_batch_rejects_bad_arguments(lib):
+    w = lib.make_nf4_weight(64, 128, 1 << 20, 1 << 20, 1 << 20, 1 << 20)
+    with pytest.raises(lib.LsnError) as e:                       # misaligned output
+        lib.nf4_dequant_batch([w], [(1 << 20) + 2], stream=0)
+    assert e.value.status == lib.LSN_ERR_INVALID_ARG
+    bad = lib.make_nf4_weight(64, 100, 1 << 20, 1 << 20, 1 << 20, 1 << 20)
+    with pytest.raises(lib.LsnError) as e:                       # cols % 64 != 0
+        lib.nf4_dequant_batch([w, bad], [1 << 20, 1 << 21], stream=0)
+    assert e.value.status == lib.LSN_ERR_INVALID_ARG
+    lib.nf4_dequant_batch([], [], stream=0)                      # nothing to do

@@ -72,3 +72,26 @@ def test_quantize_is_deterministic(lib):
     b = DeviceNF4(512, 512).quantize(W)
     torch.cuda.synchronize()
     assert torch.equal(a.blob, b.blob)
+
+
+def test_dequant_batch_equals_single_calls():
+    """nf4_dequant_batch over weights of several shapes (more than one launch's worth) gives the bits of
+    one nf4_dequant per weight."""
+    import torch
+    from layer_streamed_nf4_b200 import lsnf4
+    shapes = [(64, 64), (128, 4096), (1024, 4096), (4096, 1024), (192, 320)] * 4
+    ws, singles, outs = [], [], []
+    for i, (r, c) in enumerate(shapes):
+        d = DeviceNF4(r, c).quantize(torch.randn((r, c), generator=torch.Generator().manual_seed(i)).numpy() * 0.02)
+        ws.append(d)
+        a = torch.empty((r, c), dtype=torch.bfloat16, device="cuda")
+        lsnf4.nf4_dequant(d.w, a)
+        singles.append(a)
+        outs.append(torch.empty((r, c), dtype=torch.bfloat16, device="cuda"))
+    for bps in (0, 1, 3):
+        for o in outs:
+            o.zero_()
+        lsnf4.nf4_dequant_batch([d.w for d in ws], outs, blocks_per_sm=bps)
+        torch.cuda.synchronize()
+        for a, b in zip(singles, outs):
+            assert torch.equal(a, b), bps
