@@ -168,7 +168,7 @@ def run_ours(args):
     clocks = None
     st_main = Stack(cfg, layers=L, tokens=T, mode="streamed", n_slots=args.slots, seed=synth.SEED + rank,
                     stream=stream, lanes=args.lanes, api=args.api,
-                    dequant_ahead=args.dequant_ahead if args.dequant_ahead == "auto" else args.dequant_ahead == "1")
+                    dequant_ahead=bool(args.dequant_ahead))
     wanted = [m for m in args.modes.split(",") if m]
     modes = ["streamed"] + [m for m in wanted
                             if m in ("no_h2d", "resident", "proj", "dpo", "recompute", "shared", "grouped")
@@ -540,8 +540,8 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=64, help="token rows per step of the reference arm")
     ap.add_argument("--fused-nf4", action="store_true", help="convert NF4 inside the GEMM (no bf16 copy of W)")
     ap.add_argument("--no-pdl", action="store_true", help="ordinary launches instead of programmatic dependent ones")
-    ap.add_argument("--dequant-ahead", default="auto", choices=["auto", "0", "1"],
-                    help="dequantise each layer on a side stream one layer ahead (auto: when the layers stream)")
+    ap.add_argument("--dequant-ahead", type=int, default=1, choices=[0, 1],
+                    help="dequantise each layer on a side stream one layer ahead (1, default) or inside the layer call")
     ap.add_argument("--case", default="", help="profile one 8B projection (q,k,v,o,gate,up,down) instead of the stack")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)

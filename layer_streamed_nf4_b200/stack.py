@@ -18,19 +18,18 @@ Two ways to drive a layer (api=...):
   "proj"   seven lora_linear_fwd / lora_linear_bwd calls per layer and sweep.
 Both give the same bits.
 
-Dequantisation ahead (dequant_ahead, NF4 bases with the layer calls): the
-weights do not depend on the activations, so while layer i
+Dequantisation ahead (dequant_ahead, on by default for NF4 bases with the
+layer calls): the weights do not depend on the activations, so while layer i
 computes, a side stream acquires layer i+1's slot, runs nf4_dequant on its
 projections into one of two bf16 buffers and releases the slot; layer i+1's
 call then takes bf16 bases pointing at that buffer.  The dequantisation runs
 underneath the previous layer's GEMMs, and a pool slot is held only until
 its layer is dequantised.  Same bits as dequantising inside the call.
-"auto" (the default) dequantises ahead when the layers stream from host
-memory (the slot then returns to the pool a layer earlier, which keeps the
-copy engine busier: 123.2 vs 125.6 ms per 8B step on one B200) and inside
-the call when every layer is resident (there the dequantisation overlaps the
-down projections instead of slowing the previous layer's GEMMs: 59.5 vs
-60.2 ms).
+The dequantisation runs with at most two blocks per SM, so that it trickles
+along beside the GEMMs instead of crowding them.  Measured on one B200 (8B
+shapes): with streamed layers the slot returns to the pool a layer earlier
+and the copy engine stays busy (122.8 vs 125.6 ms per step at T = 2048;
+212 vs 226 ms at T = 8192); with every layer resident 58.6 vs 58.9 ms.
 
 Inputs: by default every (layer, projection) has its own x.  With
 shared_inputs, q, k and v read one x and gate and up read one x, as in a
@@ -84,7 +83,7 @@ class Stack:
                  mode: str = "streamed", n_slots: int = 2, seed: int = synth.SEED, keep_outputs: bool = False,
                  distinct_activations: bool = True, device: int = 0, stream: torch.cuda.Stream | None = None,
                  lanes: int = 2, api: str = "layer", shared_inputs: bool = False, grouped: bool = False,
-                 dequant_ahead: bool | str = "auto"):
+                 dequant_ahead: bool = True):
         assert mode in ("resident", "streamed", "no_h2d")
         assert api in ("layer", "proj")
         assert not grouped or api == "layer", "groups are a feature of the layer calls"
@@ -358,11 +357,7 @@ class Stack:
         return other
 
     def _ahead_for(self, mode: str) -> bool:
-        if not (self.nf4 and self.api == "layer"):
-            return False
-        if self._ahead_opt == "auto":
-            return mode == "streamed"
-        return bool(self._ahead_opt)
+        return bool(self._ahead_opt and self.nf4 and self.api == "layer")
 
     def _ahead_base(self, b: int, pi: int):
         p = self.proj[pi]

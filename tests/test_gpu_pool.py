@@ -121,9 +121,10 @@ def test_dequant_ahead_gives_the_same_bits(lib, mode):
     inside = Stack(cfg, layers=3, tokens=256, mode=mode, keep_outputs=True, dequant_ahead=False)
     ahead = Stack(cfg, layers=3, tokens=256, mode=mode, keep_outputs=True, dequant_ahead=True)
     assert ahead.ahead and not inside.ahead
-    auto = Stack(cfg, layers=2, tokens=64, mode=mode)
-    assert auto.ahead == (mode == "streamed") and not auto.with_mode("resident").ahead
-    auto.close()
+    default = Stack(cfg, layers=2, tokens=64, mode=mode)
+    assert default.ahead and default.with_mode("resident").ahead
+    assert not default.with_mode("no_h2d", api="proj").ahead or default.with_mode("no_h2d", api="proj").api == "proj"
+    default.close()
     for st in (inside, ahead):
         st.step()
         st.step(reference=True, recompute=True)
