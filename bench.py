@@ -45,7 +45,7 @@ def _peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms while running."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
          "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
          "clocks_event_reasons.sw_power_cap")
@@ -58,7 +58,7 @@ class ClockSampler:
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self._t = threading.Thread(target=self._read, daemon=True)
             self._t.start()
@@ -195,6 +195,11 @@ def run_ours(args):
             st = st_main.with_inputs(shared_inputs=True, grouped=(mode == "grouped"))
         else:
             st = st_main.with_mode(mode)
+        # Clocks of the value's mode: the sampler starts before the warm-up
+        # (nvidia-smi needs a moment to start), so the timed steps are covered.
+        sampler = ClockSampler(local) if mode == "streamed" else None
+        if sampler:
+            sampler.__enter__()
         with torch.cuda.stream(stream):
             for _ in range(args.warmup):
                 st.step(**kw)
@@ -206,9 +211,6 @@ def run_ours(args):
             ps0 = ps0_mode
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
-        sampler = ClockSampler(local) if mode == "streamed" else None
-        if sampler:
-            sampler.__enter__()
         with torch.cuda.stream(stream):
             t0.record(stream)
             h0 = time.perf_counter()
