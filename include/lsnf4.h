@@ -281,6 +281,13 @@ lsn_status lora_layer_bwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
  * The workspace must have been zero-filled once when it was allocated. */
 lsn_status lsn_ws_status(void* ws, lsn_stream_t stream);
 
+/* Self-test of the bounded wait the tensor-core kernels use: one thread waits
+ * on an mbarrier that nothing arrives on, giving up after about limit_us
+ * microseconds (1 .. 1e6) of SM clock.  Synchronises `stream`.  Returns
+ * LSN_ERR_TIMEOUT when the wait gave up as designed (the expected outcome;
+ * the context stays usable), LSN_ERR_STATE if it did not. */
+lsn_status lsn_selftest_wait_timeout(int limit_us, lsn_stream_t stream);
+
 /* ------------------------------------------------------- kernel timing --
  *
  * Optional per-launch timing of the library's own kernels: while enabled,

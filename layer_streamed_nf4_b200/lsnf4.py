@@ -44,6 +44,7 @@ EXPORTS = (
     "layer_pool_inject_fault", "layer_pool_destroy", "lsn_timing_enable", "lsn_timing_read",
     "nf4_quantize_noalloc", "lsn_set_option", "lsn_get_option",
     "lsn_layer_ws_bytes", "lora_layer_fwd", "lora_layer_bwd", "nf4_dequant_batch",
+    "lsn_selftest_wait_timeout",
 )
 
 
@@ -112,6 +113,7 @@ _sig("lora_linear_fwd", _i, [ctypes.POINTER(Base), _vp, _i64, _vp, _vp, _i, ctyp
 _sig("lora_linear_bwd", _i, [ctypes.POINTER(Base), _vp, _vp, _i64, _vp, _vp, _i, ctypes.c_float, _vp, _vp, _vp, _i,
                              _vp, _sz, _vp])
 _sig("lsn_ws_status", _i, [_vp, _vp])
+_sig("lsn_selftest_wait_timeout", _i, [_i, _vp])
 _sig("lsn_layer_ws_bytes", _sz, [_i, ctypes.POINTER(LoraProj), _i64, _i])
 _sig("lora_layer_fwd", _i, [_i, ctypes.POINTER(LoraProj), _i64, _i, ctypes.c_float, _vp, _sz, _vp])
 _sig("lora_layer_bwd", _i, [_i, ctypes.POINTER(LoraProj), _i64, _i, ctypes.c_float, _i, _vp, _sz, _vp])
@@ -279,6 +281,11 @@ def lora_layer_bwd(projs, T: int, r: int, scale: float, accumulate: bool, ws, ws
     arr = projs if isinstance(projs, ctypes.Array) else proj_array(projs)
     _check(_lib.lora_layer_bwd(len(arr), arr, T, r, scale, int(bool(accumulate)), _ptr(ws), ws_bytes,
                                _stream(stream)), "lora_layer_bwd")
+
+
+def selftest_wait_timeout(limit_us: int = 1000, stream=None) -> int:
+    """Status of the bounded-wait self-test: LSN_ERR_TIMEOUT is the expected outcome."""
+    return _lib.lsn_selftest_wait_timeout(limit_us, _stream(stream))
 
 
 def ws_status(ws, stream=None):

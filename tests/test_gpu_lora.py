@@ -213,3 +213,13 @@ def test_full_size_sampled_rows(lib, orc, name, T, K, N):
     rA, rB = orc.lora_bwd_dadb(c.x, c.dY, c.A, c.B, c.scale)
     assert_close(dA.cpu().numpy(), rA, f"{name} dA")
     assert_close(dB.cpu().numpy(), rB, f"{name} dB")
+
+
+def test_bounded_wait_gives_up_and_the_context_stays_usable(lib, orc):
+    """A wait on an mbarrier that nothing arrives on ends after its limit with a timeout status (no
+    hang), and kernels launched afterwards still compute correct results."""
+    import time
+    t0 = time.perf_counter()
+    assert lib.selftest_wait_timeout(2000) == lib.LSN_ERR_TIMEOUT
+    assert time.perf_counter() - t0 < 30.0
+    test_single_linear_config(lib, orc, "nf4")
