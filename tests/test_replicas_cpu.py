@@ -9,7 +9,6 @@ import socket
 import sys
 from contextlib import redirect_stdout
 
-import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
