@@ -53,7 +53,7 @@ def build(force: bool = False) -> str:
             return _SO
         os.makedirs(_OUT_DIR, exist_ok=True)
         tmp = _SO + f".tmp{os.getpid()}"
-        subprocess.check_call(["g++", "-O2", "-std=c++17", "-fopenmp", "-fPIC", "-shared",
+        subprocess.check_call(["g++", "-O2", "-std=c++17", "-ffp-contract=off", "-fopenmp", "-fPIC", "-shared",
                                "-o", tmp, _SRC])
         os.replace(tmp, _SO)
         return _SO
