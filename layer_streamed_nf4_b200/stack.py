@@ -48,6 +48,13 @@ acquire and join it before the layer's release, so the pool's ordering
 is independent of the lane it runs on, so results are bitwise the same for
 any lane count.
 
+Resident constants (resident_constants, on by default for NF4 bases): a
+layer's blob in host RAM holds only the packed codes of its projections;
+their double-quantised constants (absmax_q, s2, offset: about 1/32 of the
+codes' bytes) stay in device memory for the whole run, so every copy moves codes
+only.  The kernels see the same arrays either way (an NF4 weight is four
+pointers), so the results are the same bits.
+
 Modes with identical kernels and launch shapes, for the bit-exactness gate
 ("Exact Layer Streaming", abstract: streamed compared with a resident run of
 the same numerics):
@@ -74,8 +81,10 @@ class ProjLayout:
     name: str
     K: int
     N: int
-    offset: int      # byte offset of this projection in the layer blob
+    offset: int      # byte offset of this projection's streamed bytes in the layer blob
     nbytes: int
+    coffset: int = 0  # NF4 with resident constants: byte offset of its constants in the layer's constant block
+    cbytes: int = 0
 
 
 class Stack:
@@ -83,7 +92,7 @@ class Stack:
                  mode: str = "streamed", n_slots: int = 2, seed: int = synth.SEED, keep_outputs: bool = False,
                  distinct_activations: bool = True, device: int = 0, stream: torch.cuda.Stream | None = None,
                  lanes: int = 2, api: str = "layer", shared_inputs: bool = False, grouped: bool = False,
-                 dequant_ahead: bool = True):
+                 dequant_ahead: bool = True, resident_constants: bool = True):
         assert mode in ("resident", "streamed", "no_h2d")
         assert api in ("layer", "proj")
         assert not grouped or api == "layer", "groups are a feature of the layer calls"
@@ -105,13 +114,19 @@ class Stack:
         self.lanes = [self.stream] + [torch.cuda.Stream(self.dev) for _ in range(lanes - 1)]
         self._fork = [torch.cuda.Event() for _ in range(lanes)]
         self._join = [torch.cuda.Event() for _ in range(lanes)]
-        off = 0
+        off = coff = 0
         self.proj: list[ProjLayout] = []
         for name, K, N in cfg.projections:
-            nb = lsnf4.nf4_blob_bytes(N, K) if self.nf4 else _round_up(N * K * 2, 1024)
-            self.proj.append(ProjLayout(name, K, N, off, nb))
+            nb, cb = (lsnf4.nf4_blob_bytes(N, K) if self.nf4 else _round_up(N * K * 2, 1024)), 0
+            if self.nf4 and resident_constants:         # stream the packed codes, keep the constants on the device
+                cb = nb - lsnf4.nf4_blob_layout(N, K)[1]
+                nb -= cb
+            self.proj.append(ProjLayout(name, K, N, off, nb, coff, cb))
             off += nb
+            coff += cb
         self.layer_bytes = off
+        self.const_bytes = coff
+        self.consts = None
         self.pool = None
         self.host = None
         self.resident = None
@@ -136,9 +151,13 @@ class Stack:
     # ------------------------------------------------------------ set-up --
 
     def _build_weights(self):
-        """W ~ N(0, 0.02) per projection, quantised on the device, stored per layer in pinned host RAM."""
+        """W ~ N(0, 0.02) per projection, quantised on the device, stored per layer in pinned host RAM
+        (with resident constants: the packed codes there, absmax_q / s2 / offset in device memory)."""
         self.host = torch.empty((self.L, self.layer_bytes), dtype=torch.uint8, pin_memory=True)
         dblob = torch.zeros(self.layer_bytes, dtype=torch.uint8, device=self.dev)
+        if self.const_bytes:
+            self.consts = torch.zeros((self.L, self.const_bytes), dtype=torch.uint8, device=self.dev)
+            full = torch.zeros(max(p.nbytes + p.cbytes for p in self.proj), dtype=torch.uint8, device=self.dev)
         maxnk = max(p.N * p.K for p in self.proj)
         qws_bytes = lsnf4.nf4_quantize_ws_bytes(1, maxnk) if self.nf4 else 0
         qws = torch.zeros(max(qws_bytes, 16), dtype=torch.uint8, device=self.dev)
@@ -146,9 +165,13 @@ class Stack:
             for l in range(self.L):
                 for pi, p in enumerate(self.proj):
                     W = synth.device_normal((p.N, p.K), 0.02, self.seed, l, pi, synth.T_W, device=self.dev)
-                    addr = dblob.data_ptr() + p.offset
-                    if self.nf4:
-                        w = lsnf4.nf4_weight_in_blob(p.N, p.K, addr)
+                    if self.nf4 and p.cbytes:           # quantise into one full blob, then split it
+                        w = lsnf4.nf4_weight_in_blob(p.N, p.K, full.data_ptr())
+                        lsnf4.nf4_quantize(W, w, qws, qws_bytes, self.stream)
+                        dblob[p.offset:p.offset + p.nbytes].copy_(full[:p.nbytes])
+                        self.consts[l, p.coffset:p.coffset + p.cbytes].copy_(full[p.nbytes:p.nbytes + p.cbytes])
+                    elif self.nf4:
+                        w = lsnf4.nf4_weight_in_blob(p.N, p.K, dblob.data_ptr() + p.offset)
                         lsnf4.nf4_quantize(W, w, qws, qws_bytes, self.stream)
                     else:
                         dst = dblob[p.offset:p.offset + p.N * p.K * 2].view(torch.bfloat16)
@@ -274,9 +297,17 @@ class Stack:
         if self.mode != "resident":
             lsnf4.layer_pool_release(self.pool, l, stream or self.stream)
 
-    def _base(self, addr: int, p: ProjLayout):
+    def _nf4_view(self, addr: int, l: int, p: ProjLayout) -> lsnf4.NF4Weight:
+        """Projection p of layer l, its blob bytes at addr (and its constants in the resident block)."""
+        if not p.cbytes:
+            return lsnf4.nf4_weight_in_blob(p.N, p.K, addr + p.offset)
+        o = lsnf4.nf4_blob_layout(p.N, p.K)
+        c = self.consts[l].data_ptr() + p.coffset - o[1]
+        return lsnf4.NF4Weight(p.N, p.K, addr + p.offset, c + o[1], c + o[2], c + o[3])
+
+    def _base(self, addr: int, l: int, p: ProjLayout):
         if self.nf4:
-            return lsnf4.base_nf4(lsnf4.nf4_weight_in_blob(p.N, p.K, addr + p.offset))
+            return lsnf4.base_nf4(self._nf4_view(addr, l, p))
         return lsnf4.base_bf16(addr + p.offset, p.N, p.K)
 
     def _out(self, d, l, pi):
@@ -303,7 +334,7 @@ class Stack:
         a = self._calls.get(key)
         if a is None:
             p = self.proj[pi]
-            base = self._base(addr, p)
+            base = self._base(addr, l, p)
             lane = pi % self.n_lanes
             a = (ctypes.byref(base), self.x[l, pi].data_ptr(), self.T, self.A[l, pi].data_ptr(),
                  self.B[l, pi].data_ptr(), self.r, self.scale, self._out(self.y, l, pi).data_ptr(),
@@ -316,7 +347,7 @@ class Stack:
         a = self._calls.get(key)
         if a is None:
             p = self.proj[pi]
-            base = self._base(addr, p)
+            base = self._base(addr, l, p)
             lane = (len(self.proj) - 1 - pi) % self.n_lanes
             a = (ctypes.byref(base), self.x[l, pi].data_ptr(), self.dY[l, pi].data_ptr(), self.T,
                  self.A[l, pi].data_ptr(), self.B[l, pi].data_ptr(), self.r, self.scale,
@@ -370,7 +401,7 @@ class Stack:
         key = ("L", addr, l, adapter, wb)
         a = self._calls.get(key)
         if a is None:
-            projs = [lsnf4.lora_proj(self._base(addr, p) if wb is None else self._ahead_base(wb, pi), self.x[l, pi],
+            projs = [lsnf4.lora_proj(self._base(addr, l, p) if wb is None else self._ahead_base(wb, pi), self.x[l, pi],
                                      self.A[l, pi] if adapter else None, self.B[l, pi] if adapter else None,
                                      y=self._out(self.y if adapter else self.y_ref, l, pi), dY=self.dY[l, pi],
                                      dX=self._out(self.dX, l, pi) if self._leads(pi) else None,
@@ -389,10 +420,10 @@ class Stack:
         ps = self._prep
         ps.wait_event(self._ev_done[b])
         addr = self._acquire(l, ps)
-        key = ("D", addr, b)
+        key = ("D", addr, l, b)
         args = self._calls.get(key)
         if args is None:                          # one launch for the layer's projections
-            ws = [lsnf4.nf4_weight_in_blob(p.N, p.K, addr + p.offset) for p in self.proj]
+            ws = [self._nf4_view(addr, l, p) for p in self.proj]
             outs = [self._wbuf[b].data_ptr() + 2 * self._woff[pi] for pi in range(len(self.proj))]
             args = self._calls[key] = lsnf4.dequant_batch_args(ws, outs)
         # two blocks per SM: the dequantisation trickles along beside the current layer's GEMMs

@@ -137,6 +137,31 @@ def test_dequant_ahead_gives_the_same_bits(lib, mode):
     ahead.close()
 
 
+def test_resident_constants_give_the_same_bits(lib):
+    """Streaming only the packed codes (constants kept in device memory) and streaming whole NF4 blobs give
+    the same bits; the pool then copies the codes alone."""
+    cfg = synth.STACKS["8b"]
+    import torch
+    from layer_streamed_nf4_b200.stack import Stack
+    runs = []
+    for rc in (False, True):
+        st = Stack(cfg, layers=3, tokens=256, mode="streamed", keep_outputs=True, resident_constants=rc)
+        st.step()
+        torch.cuda.synchronize()
+        st.check_status()
+        runs.append(st)
+    whole, codes = runs
+    fwd, bwd, bad = _compare(codes, whole)
+    assert fwd and bwd, bad
+    assert codes.const_bytes > 0 and whole.const_bytes == 0
+    assert codes.layer_bytes + codes.const_bytes == whole.layer_bytes
+    assert codes.layer_bytes == sum(p.N * p.K // 2 for p in codes.proj)       # 8B shapes: no padding
+    for st in runs:
+        s = st.pool_stats()
+        assert s["bytes_copied"] == s["copies"] * st.layer_bytes, s
+        st.close()
+
+
 def test_no_h2d_equals_resident(lib):
     cfg = synth.STACKS["8b"]
     res = _run(cfg, 3, 512, "resident")
