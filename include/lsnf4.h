@@ -94,10 +94,13 @@ void lsn_dq_codebook(float out[256]);
 
 /* A quantised weight of rows x cols (N x K), cols % 64 == 0.  All pointers are
  * caller-owned device memory:
- *   packed     [rows*cols/2]      uint8, two 4-bit codes per byte
+ *   packed     [rows*cols/2]      uint8, two 4-bit codes per byte (16-byte aligned)
  *   absmax_q   [rows*cols/64]     uint8 second-level codes
- *   absmax_s2  [ceil(nblk/256)]   fp32 per group of 256 blocks
- *   offset     [1]                fp32 (device, so quantisation never syncs) */
+ *   absmax_s2  [ceil(nblk/256)]   fp32 per group of 256 blocks (4-byte aligned)
+ *   offset     [1]                fp32 (device, so quantisation never syncs; 4-byte aligned)
+ * The four arrays are independent: they may sit in one blob
+ * (lsn_nf4_blob_layout) or apart, e.g. the codes in a layer-pool slot and the
+ * constants in memory that stays resident. */
 typedef struct {
     int64_t rows, cols;
     uint8_t* packed;
