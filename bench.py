@@ -1,6 +1,8 @@
 """Benchmark: layer-streamed NF4 LoRA linears, fwd + bwd, on the Llama-3.1-8B
 shaped stack (32 layers x 7 projections, T = 2048 tokens, r = 16, alpha = 32,
-NF4 base streamed from pinned host RAM through a 2-slot VRAM pool).
+NF4 codes streamed from pinned host RAM through a VRAM pool of 20 layer
+slots, which at 2048 tokens hides the PCIe copies behind compute; the
+two-slot pool is timed beside it as mode streamed_S2).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -155,6 +157,7 @@ def run_ours(args):
     cfg = synth.STACKS[WORKLOAD]
     T = args.tokens or cfg.tokens
     L = args.layers or cfg.layers
+    args.slots = max(1, min(args.slots, L))
     stream = torch.cuda.Stream()
     peaks = _peaks()
 
@@ -172,7 +175,7 @@ def run_ours(args):
     wanted = [m for m in args.modes.split(",") if m]
     modes = ["streamed"] + [m for m in wanted
                             if m in ("no_h2d", "resident", "proj", "dpo", "recompute", "shared", "grouped")
-                            or m.startswith("streamed_T")]
+                            or m.startswith("streamed_T") or m.startswith("streamed_S")]
     mode_tokens = {m: T for m in modes}
     mode_copies = {}
     # Extra work of the step variants: the reference forward of preference
@@ -189,6 +192,8 @@ def run_ours(args):
         elif mode.startswith("streamed_T"):   # the same stream of weights under a larger batch
             mode_tokens[mode] = int(mode[len("streamed_T"):])
             st = st_main.with_tokens(mode_tokens[mode], "streamed", n_slots=args.slots)
+        elif mode.startswith("streamed_S"):   # the same stream of weights through a pool of n slots
+            st = st_main.with_mode("streamed", n_slots=int(mode[len("streamed_S"):]))
         elif mode in ("dpo", "recompute"):    # step variants over the same streamed pool
             st = st_main.with_mode("streamed", n_slots=args.slots)
         elif mode in ("shared", "grouped"):   # q|k|v and gate|up read one input each (no_h2d pool)
@@ -346,7 +351,7 @@ def run_ours(args):
         "config": {"workload": f"{cfg.name} NF4 LoRA stack: {L} layers x 7 projections (q,k,v,o,gate,up,down), "
                                f"T={T} tokens (batch 1 x seq {T}), r={cfg.rank}, alpha={cfg.alpha:g}, "
                                f"base NF4 blk-64 + double quant streamed from pinned host RAM, "
-                               f"{args.slots}-slot VRAM pool",
+                               f"{args.slots}-slot VRAM pool ({L} layers)",
                    "tokens": T, "layers": L, "rank": cfg.rank, "pool_slots": args.slots, "base": cfg.base,
                    "parallelism": f"replicas x{world}",
                    "api": args.api,
@@ -354,7 +359,7 @@ def run_ours(args):
                    "nf4_conversion": "inside the GEMM" if args.fused_nf4 else "nf4_dequant then bf16 GEMM",
                    "programmatic_dependent_launch": not args.no_pdl,
                    "dequant_ahead": st_main.ahead,
-                   "l2": "inputs larger than L2 (per step ~11 GB of activations, ~3.6 GB of streamed weights)"},
+                   "l2": "inputs larger than L2 (per step ~11 GB of activations; every layer's NF4 codes read twice)"},
         "pct_bf16_peak": 100 * flop_step / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
         "flop_per_step": flop_step,
         "modes": extra_modes,
@@ -529,9 +534,12 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--tokens", type=int, default=0, help="override T (default: the workload's 2048)")
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (default 32)")
-    ap.add_argument("--slots", type=int, default=2)
-    ap.add_argument("--modes", default="no_h2d,resident,proj,streamed_T8192,dpo,recompute,shared,grouped",
-                    help="extra modes timed after the streamed one (streamed_T<n>: streamed with n tokens)")
+    ap.add_argument("--slots", type=int, default=20,
+                    help="VRAM pool slots of the timed stream (default 20 of 32 layers: the smallest measured "
+                         "window that hides the copies behind compute at 2048 tokens on one B200)")
+    ap.add_argument("--modes", default="no_h2d,resident,proj,streamed_S2,streamed_T8192,dpo,recompute,shared,grouped",
+                    help="extra modes timed after the streamed one (streamed_T<n>: streamed with n tokens; "
+                         "streamed_S<n>: streamed through n pool slots)")
     ap.add_argument("--api", choices=["layer", "proj"], default="layer",
                     help="one library call per layer, or one per projection")
     ap.add_argument("--lanes", type=int, default=2, help="streams the seven projections of a layer are spread over")

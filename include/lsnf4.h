@@ -359,8 +359,11 @@ int lsn_get_option(int option);
  * A copy into a slot always waits for that slot's released event, so a slot is
  * never overwritten while compute may still read it.  Forward sweeps prefetch
  * layer i+1 while layer i computes, backward sweeps layer i-1; with 2 slots a
- * fwd+bwd step reads 2L-2 layers (each layer twice, minus the two still
- * resident at the turn).
+ * fwd+bwd step reads 2L-4 layers in steady state (each layer twice, minus the
+ * two still resident at each turn).  With S slots a sweep can keep S layers
+ * in flight: prefetch the next S layers of the sweep at its start and one
+ * more each time a layer is released; at each turn the S layers used last are
+ * the S used first, so a step reads 2L-2S layers.
  */
 typedef struct lsn_pool lsn_pool;
 
@@ -383,9 +386,12 @@ lsn_status layer_pool_create(int n_slots, size_t slot_bytes, int device, lsn_poo
  * any resident copy. */
 lsn_status layer_pool_register(lsn_pool* pool, int layer, const void* host_pinned, size_t bytes);
 
-/* Start copying `layer` into a free slot (no-op if resident or in flight).
- * Takes the least recently released slot that is neither acquired nor holding
- * a prefetched, not yet acquired layer; LSN_ERR_STATE if there is none. */
+/* Start copying `layer` into a free slot.  Takes the least recently released
+ * slot that is neither acquired nor holding a prefetched, not yet acquired
+ * layer; LSN_ERR_STATE if there is none.  If `layer` is resident or in flight
+ * nothing is copied, and a resident layer that is not acquired counts as
+ * prefetched again: its slot is not taken for another layer until it has been
+ * acquired. */
 lsn_status layer_pool_prefetch(lsn_pool* pool, int layer);
 
 /* Make `compute` wait until `layer` is in VRAM (copying it first if needed)

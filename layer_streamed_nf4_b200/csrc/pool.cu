@@ -204,7 +204,12 @@ lsn_status layer_pool_register(lsn_pool* p, int layer, const void* host, size_t 
 lsn_status layer_pool_prefetch(lsn_pool* p, int layer) {
     LSN_CHECK_ARG(p != nullptr, "layer_pool_prefetch: pool is NULL");
     std::lock_guard<std::mutex> lk(p->mu);
-    if (find_slot(p, layer) >= 0) { p->stats.hits += 1; return LSN_OK; }
+    const int s = find_slot(p, layer);
+    if (s >= 0) {                        // resident: keep it there until it is acquired
+        p->stats.hits += 1;
+        if (p->slots[s].refs == 0) p->slots[s].pending = true;
+        return LSN_OK;
+    }
     DeviceGuard g(p->device);
     int slot;
     return start_copy(p, layer, &slot);

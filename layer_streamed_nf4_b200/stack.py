@@ -10,6 +10,14 @@ backward sweep over L-1..0 (acquire i, prefetch i-1, seven lora_linear_bwd
 calls, release i).  All compute and all copies are library calls; this file
 only sequences them and owns the (synthetic) tensors.
 
+With S pool slots (n_slots) a sweep keeps S layers in flight instead of one:
+it prefetches its first S layers at its start and the layer S positions
+ahead whenever one is released.  At each turn of the step the S layers the
+last sweep used are the first S the next one needs, still resident, so a
+step copies 2L-2S layers (2L-4 with the pages' two slots).  S sets how much
+of the copy time hides behind compute: on B200 at 2048 tokens a layer's
+codes take about twice as long to cross PCIe as its compute.
+
 Two ways to drive a layer (api=...):
   "layer"  one lora_layer_fwd / lora_layer_bwd call per layer and sweep: the
            library launches the seven projections together (one dequant, one
@@ -220,8 +228,10 @@ class Stack:
     def _setup_mode(self, n_slots: int):
         if self.mode == "resident":
             self.resident = self.host.to(self.dev)
+            self.n_slots = self.L
             return
         slots = self.L if self.mode == "no_h2d" else n_slots
+        self.n_slots = slots
         self.pool = lsnf4.layer_pool_create(slots, self.layer_bytes, self.dev.index or 0)
         for l in range(self.L):
             lsnf4.layer_pool_register(self.pool, l, self.host[l].data_ptr(), self.layer_bytes)
@@ -292,6 +302,19 @@ class Stack:
     def _prefetch(self, l: int):
         if self.mode != "resident" and 0 <= l < self.L:
             lsnf4.layer_pool_prefetch(self.pool, l)
+
+    def _window(self, order):
+        """fill(pos): prefetch the layers at positions <= pos of a sweep, each once.  A sweep keeps
+        the pool's S slots busy: its first S layers at the start (at a turn these are the S layers the
+        previous sweep used last, still resident), then one more whenever a layer has been released."""
+        nxt = 0
+
+        def fill(pos):
+            nonlocal nxt
+            while nxt < len(order) and nxt <= pos:
+                self._prefetch(order[nxt])
+                nxt += 1
+        return fill
 
     def _release(self, l: int, stream=None):
         if self.mode != "resident":
@@ -434,20 +457,21 @@ class Stack:
         self._ev_ready[b].record(ps)
 
     def _sweep_ahead(self, order, call):
-        """Run call(l, projs) over the layers in `order`, each layer dequantised one layer ahead."""
+        """Run call(l, projs) over the layers in `order`, each layer dequantised one layer ahead.
+        The slot of position j is released once j is dequantised, so position j + S may be prefetched."""
         order = list(order)
         if not order:
             return
-        self._prefetch(order[0])
+        S = self.n_slots
+        fill = self._window(order)
+        fill(S - 1)
         self._prep_layer(order[0], 0)
-        if len(order) > 1:
-            self._prefetch(order[1])
+        fill(S)
         for idx, l in enumerate(order):
             b = idx % 2
             if idx + 1 < len(order):
                 self._prep_layer(order[idx + 1], (idx + 1) % 2)
-            if idx + 2 < len(order):
-                self._prefetch(order[idx + 2])
+                fill(idx + 1 + S)
             self.stream.wait_event(self._ev_ready[b])
             call(l, b)
             self._ev_done[b].record(self.stream)
@@ -461,9 +485,12 @@ class Stack:
                 if st:
                     lsnf4._check(st, "lora_layer_fwd")
             return self._sweep_ahead(range(self.L), call)
-        for l in range(self.L):
+        order = list(range(self.L))
+        fill = self._window(order)
+        fill(self.n_slots - 1)
+        for j, l in enumerate(order):
             addr = self._acquire(l)
-            self._prefetch(l + 1)
+            fill(j + self.n_slots - 1)
             st = fwd(n, self._layer_projs(addr, l, adapter), self.T, self.r, self.scale, ws, nb, sp)
             if st:
                 lsnf4._check(st, "lora_layer_fwd")
@@ -483,9 +510,12 @@ class Stack:
                 if st:
                     lsnf4._check(st, "lora_layer_bwd")
             return self._sweep_ahead(reversed(range(self.L)), call)
-        for l in reversed(range(self.L)):
+        order = list(reversed(range(self.L)))
+        fill = self._window(order)
+        fill(self.n_slots - 1)
+        for j, l in enumerate(order):
             addr = self._acquire(l)
-            self._prefetch(l - 1)
+            fill(j + self.n_slots - 1)
             projs = self._layer_projs(addr, l)
             if recompute:     # the layer's forward again, inside the backward sweep (activation checkpointing)
                 st = fwd(n, projs, self.T, self.r, self.scale, ws, nb, sp)
@@ -501,9 +531,12 @@ class Stack:
             return self._forward_layers(adapter)
         assert adapter, "the adapter-off forward runs through the layer calls"
         fwd = lsnf4._lib.lora_linear_fwd
-        for l in range(self.L):
+        order = list(range(self.L))
+        fill = self._window(order)
+        fill(self.n_slots - 1)
+        for j, l in enumerate(order):
             addr = self._acquire(l)
-            self._prefetch(l + 1)
+            fill(j + self.n_slots - 1)
             self._fork_lanes()
             for pi in range(len(self.proj)):
                 st = fwd(*self._fwd_args(addr, l, pi)[:-1])
@@ -517,9 +550,12 @@ class Stack:
             return self._backward_layers(accumulate, recompute)
         assert not recompute, "the recomputing backward runs through the layer calls"
         bwd = lsnf4._lib.lora_linear_bwd
-        for l in reversed(range(self.L)):
+        order = list(reversed(range(self.L)))
+        fill = self._window(order)
+        fill(self.n_slots - 1)
+        for j, l in enumerate(order):
             addr = self._acquire(l)
-            self._prefetch(l - 1)
+            fill(j + self.n_slots - 1)
             self._fork_lanes()
             for pi in reversed(range(len(self.proj))):
                 st = bwd(*self._bwd_args(addr, l, pi, accumulate)[:-1])

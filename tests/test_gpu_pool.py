@@ -235,6 +235,61 @@ def test_pool_rules(lib):
         lib.layer_pool_destroy(pool)
 
 
+def test_prefetch_keeps_a_resident_layer(lib):
+    """Prefetching a layer that is already in a slot protects that slot: the next copy takes another
+    slot even where the protected one was released longer ago, and the later acquire copies nothing."""
+    import torch
+    n = 1 << 20
+    hosts = [torch.full((n,), i + 1, dtype=torch.uint8, pin_memory=True) for i in range(3)]
+    pool = lib.layer_pool_create(2, n, 0)
+    try:
+        for i, h in enumerate(hosts):
+            lib.layer_pool_register(pool, i, h.data_ptr(), n)
+        s = torch.cuda.current_stream()
+        p0 = lib.layer_pool_acquire(pool, 0, s)
+        lib.layer_pool_release(pool, 0, s)
+        p1 = lib.layer_pool_acquire(pool, 1, s)
+        lib.layer_pool_release(pool, 1, s)
+        assert p0 != p1
+        lib.layer_pool_prefetch(pool, 0)              # resident, released first: now protected
+        lib.layer_pool_prefetch(pool, 2)              # must take layer 1's slot
+        c = lib.layer_pool_stats(pool)["copies"]
+        assert lib.layer_pool_acquire(pool, 0, s) == p0
+        assert lib.layer_pool_acquire(pool, 2, s) == p1
+        assert lib.layer_pool_stats(pool)["copies"] == c == 3
+        lib.layer_pool_release(pool, 0, s)
+        lib.layer_pool_release(pool, 2, s)
+        lib.layer_pool_wait_idle(pool, 10000)
+    finally:
+        lib.layer_pool_destroy(pool)
+
+
+@pytest.mark.parametrize("slots,ahead,api", [(3, True, "layer"), (5, True, "layer"), (5, False, "layer"),
+                                             (4, False, "proj"), (8, True, "layer")])
+def test_slot_window_copies_and_bits(lib, slots, ahead, api):
+    """With S slots each sweep keeps S layers in flight; a step copies 2L-2S layers in steady state
+    (2L-S in the first), and the results equal the resident run bit for bit."""
+    import torch
+    from layer_streamed_nf4_b200.stack import Stack
+    cfg = synth.STACKS["8b"]
+    L = 8
+    res = _run(cfg, L, 256, "resident", lanes=1, api="proj")
+    st = Stack(cfg, layers=L, tokens=256, mode="streamed", n_slots=slots, keep_outputs=True, api=api,
+               dequant_ahead=ahead)
+    assert st.ahead == ahead and st.n_slots == slots
+    counts = []
+    for _ in range(3):
+        c0 = st.pool_stats()["copies"]
+        st.step()
+        counts.append(st.pool_stats()["copies"] - c0)
+    torch.cuda.synchronize()
+    st.check_status()
+    assert counts == [2 * L - slots, 2 * L - 2 * slots, 2 * L - 2 * slots], counts
+    fwd, bwd, bad = _compare(st, res)
+    assert fwd and bwd, bad
+    st.close()
+
+
 def test_grouped_stack_matches_shared_inputs(lib):
     """A stack whose q|k|v and gate|up run as groups gives the same y, dA and dB as the same stack run
     ungrouped, streamed or resident; the grouped dX equals the ungrouped sum within bf16 rounding."""
