@@ -35,9 +35,10 @@ underneath the previous layer's GEMMs, and a pool slot is held only until
 its layer is dequantised.  Same bits as dequantising inside the call.
 The dequantisation runs with at most two blocks per SM, so that it trickles
 along beside the GEMMs instead of crowding them.  Measured on one B200 (8B
-shapes): with streamed layers the slot returns to the pool a layer earlier
-and the copy engine stays busy (122.8 vs 125.6 ms per step at T = 2048;
-212 vs 226 ms at T = 8192); with every layer resident 58.6 vs 58.9 ms.
+shapes, two slots, whole blobs streamed): with streamed layers the slot
+returns to the pool a layer earlier and the copy engine stays busy (122.8 vs
+125.6 ms per step at T = 2048; 212 vs 226 ms at T = 8192); with every layer
+resident 58.6 vs 58.9 ms.
 
 Inputs: by default every (layer, projection) has its own x.  With
 shared_inputs, q, k and v read one x and gate and up read one x, as in a
