@@ -192,12 +192,23 @@ class Stack:
     def _build_tensors(self, distinct: bool):
         T, r, dev = self.T, self.r, self.dev
         self.x, self.dY, self.A, self.B, self.dA, self.dB = {}, {}, {}, {}, {}, {}
+        h0 = None
+        if self.cfg.vocab:
+            # Layer 0 reads token embeddings: rows of a resident N(0, 1) bf16 table [vocab, hidden] picked by T
+            # token ids uniform over the vocabulary.  q, k and v take them as their input (the layer's input
+            # norm is not part of the linears).
+            self.token_ids = synth.device_token_ids(T, self.cfg.vocab, self.seed, device=dev)
+            self.embedding = synth.device_normal((self.cfg.vocab, self.cfg.hidden), 1.0, self.seed, synth.T_EMB,
+                                                 device=dev, dtype=torch.bfloat16)
+            h0 = self.embedding.index_select(0, self.token_ids)
         for l in range(self.L):
             for pi, p in enumerate(self.proj):
                 la = l if distinct else 0
                 src = self._input_of(pi)
                 if src != pi:                                   # shares the x of an earlier projection
                     self.x[l, pi] = self.x[l, src]
+                elif l == 0 and h0 is not None and p.name in ("q", "k", "v"):
+                    self.x[l, pi] = h0
                 else:
                     self.x[l, pi] = synth.device_normal((T, p.K), 1.0, self.seed, la, pi, synth.T_X, device=dev,
                                                         dtype=torch.bfloat16) if (distinct or l == 0) else self.x[0, pi]

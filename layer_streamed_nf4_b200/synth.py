@@ -162,3 +162,11 @@ def device_uniform(shape, bound: float, seed: int, *ids, device="cuda", dtype=No
     t = torch.rand(shape, generator=g, device=device, dtype=torch.float32)
     t.mul_(2.0).sub_(1.0).mul_(bound)
     return t if dtype is None else t.to(dtype)
+
+
+def device_token_ids(T: int, vocab: int, seed: int, device="cuda"):
+    """T token ids uniform over [0, vocab) (torch's Philox generator on the device)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(stream_seed(seed, T_TOK))
+    return torch.randint(0, vocab, (T,), generator=g, device=device, dtype=torch.int64)

@@ -162,6 +162,27 @@ def test_resident_constants_give_the_same_bits(lib):
         st.close()
 
 
+def test_first_layer_reads_token_embeddings(lib):
+    """0.5B workload: the layer-0 inputs of q, k and v are the rows of the resident embedding table that
+    the token ids pick; the ids cover the vocabulary uniformly."""
+    import torch
+    from layer_streamed_nf4_b200.stack import Stack
+    cfg = synth.STACKS["0.5b"]
+    st = Stack(cfg, layers=2, tokens=512, mode="streamed")
+    ids = st.token_ids
+    assert ids.shape == (512,) and int(ids.min()) >= 0 and int(ids.max()) < cfg.vocab
+    assert abs(float(ids.double().mean()) / cfg.vocab - 0.5) < 0.05
+    assert st.embedding.shape == (cfg.vocab, cfg.hidden) and st.embedding.dtype == torch.bfloat16
+    rows = st.embedding[ids]
+    for pi in range(3):                              # q, k, v
+        assert torch.equal(st.x[0, pi], rows)
+    assert not torch.equal(st.x[1, 0], rows)         # later layers: their own synthetic inputs
+    st.step()
+    torch.cuda.synchronize()
+    st.check_status()
+    st.close()
+
+
 def test_no_h2d_equals_resident(lib):
     cfg = synth.STACKS["8b"]
     res = _run(cfg, 3, 512, "resident")
