@@ -110,9 +110,11 @@ def _dist():
 
 
 class Replicas:
-    """The N > 1 plumbing: one process per GPU (launched by torchrun), each an independent replica of the
-    path (no collective on the data path: the method does not shard).  Timed regions are bracketed by
-    barriers, every timed figure is the max over ranks, and throughput counts the tokens of all ranks."""
+    """The N > 1 plumbing: one process per GPU (launched by torchrun), each a data-parallel replica of the
+    path on its own tokens.  The one exchange of data-parallel training is the sum of the adapter gradients
+    over ranks, once per step (allreduce_sum); the layer stream and the linears do not shard.  Timed regions
+    are bracketed by barriers, every timed figure is the max over ranks, and throughput counts the tokens
+    of all ranks."""
 
     def __init__(self, backend: str, device):
         import torch.distributed as dist
@@ -135,6 +137,11 @@ class Replicas:
         t = torch.tensor([v], dtype=torch.float64, device=self.device)
         self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
         return float(t.item())
+
+    def allreduce_sum(self, t):
+        """t summed over the ranks in place (enqueued on the current stream); nothing with one rank."""
+        if self.world > 1:
+            self.dist.all_reduce(t, op=self.dist.ReduceOp.SUM)
 
     def throughput(self, tokens_per_rank: int, ms: float) -> float:
         return self.world * tokens_per_rank / (ms / 1e3)
@@ -164,6 +171,13 @@ def run_ours(args):
     barrier = reps.barrier
     max_over_ranks = reps.max
 
+    def train_step(st, micro=1, **kw):
+        """One step of the path (micro > 1: that many micro-batches, the adapter gradients accumulated over
+        them), then (N > 1) the adapter gradients summed over the replicas."""
+        for i in range(micro):
+            st.step(accumulate=i > 0, **kw)
+        reps.allreduce_sum(st.grads)
+
     results = {}
     host_issue = {}
     kernel = None
@@ -175,7 +189,7 @@ def run_ours(args):
     wanted = [m for m in args.modes.split(",") if m]
     modes = ["streamed"] + [m for m in wanted
                             if m in ("no_h2d", "resident", "proj", "dpo", "recompute", "shared", "grouped")
-                            or m.startswith("streamed_T") or m.startswith("streamed_S")]
+                            or m.startswith("streamed_T") or m.startswith("streamed_S") or m.startswith("accum")]
     mode_tokens = {m: T for m in modes}
     mode_copies = {}
     # Extra work of the step variants: the reference forward of preference
@@ -192,6 +206,10 @@ def run_ours(args):
         elif mode.startswith("streamed_T"):   # the same stream of weights under a larger batch
             mode_tokens[mode] = int(mode[len("streamed_T"):])
             st = st_main.with_tokens(mode_tokens[mode], "streamed", n_slots=args.slots)
+        elif mode.startswith("accum"):        # n micro-batches of T tokens per step, gradients accumulated
+            kw = {"micro": int(mode[len("accum"):])}
+            mode_tokens[mode] = kw["micro"] * T
+            st = st_main.with_mode("streamed", n_slots=args.slots)
         elif mode.startswith("streamed_S"):   # the same stream of weights through a pool of n slots
             st = st_main.with_mode("streamed", n_slots=int(mode[len("streamed_S"):]))
         elif mode in ("dpo", "recompute"):    # step variants over the same streamed pool
@@ -207,7 +225,7 @@ def run_ours(args):
             sampler.__enter__()
         with torch.cuda.stream(stream):
             for _ in range(args.warmup):
-                st.step(**kw)
+                train_step(st, **kw)
         stream.synchronize()
         barrier()
         torch.cuda.synchronize()
@@ -220,7 +238,7 @@ def run_ours(args):
             t0.record(stream)
             h0 = time.perf_counter()
             for _ in range(args.steps):
-                st.step(**kw)
+                train_step(st, **kw)
             host_ms = (time.perf_counter() - h0) * 1e3 / args.steps
             t1.record(stream)
         t1.synchronize()
@@ -250,13 +268,13 @@ def run_ours(args):
             lsnf4.set_option(lsnf4.LSN_OPT_LAYER_LANES, 1)
             try:
                 with torch.cuda.stream(stream):
-                    st_k.step()
+                    train_step(st_k)
                 stream.synchronize()
                 barrier()
                 lsnf4.timing_enable(True)
                 with torch.cuda.stream(stream):
                     for _ in range(args.steps):
-                        st_k.step()
+                        train_step(st_k)
                 stream.synchronize()
                 kernel = lsnf4.timing_read()
                 lsnf4.timing_enable(False)
@@ -295,7 +313,7 @@ def run_ours(args):
             for _ in range(args.steps):
                 for h, t in zip(h_in, ins):
                     t.copy_(h, non_blocking=True)
-                st.step()
+                train_step(st)
                 for h, t in zip(h_out, outs):
                     h.copy_(t, non_blocking=True)
             e1.record(stream)
@@ -353,7 +371,7 @@ def run_ours(args):
                                f"base NF4 blk-64 + double quant streamed from pinned host RAM, "
                                f"{args.slots}-slot VRAM pool ({L} layers)",
                    "tokens": T, "layers": L, "rank": cfg.rank, "pool_slots": args.slots, "base": cfg.base,
-                   "parallelism": f"replicas x{world}",
+                   "parallelism": f"dp{world}" + (" (adapter gradients summed over ranks each step)" if world > 1 else ""),
                    "api": args.api,
                    "lanes": args.lanes if args.api == "proj" else 1,
                    "nf4_conversion": "inside the GEMM" if args.fused_nf4 else "nf4_dequant then bf16 GEMM",
@@ -537,9 +555,11 @@ def main():
     ap.add_argument("--slots", type=int, default=20,
                     help="VRAM pool slots of the timed stream (default 20 of 32 layers: the smallest measured "
                          "window that hides the copies behind compute at 2048 tokens on one B200)")
-    ap.add_argument("--modes", default="no_h2d,resident,proj,streamed_S2,streamed_T8192,dpo,recompute,shared,grouped",
+    ap.add_argument("--modes", default="no_h2d,resident,proj,streamed_S2,streamed_T8192,accum4,dpo,recompute,shared,"
+                                       "grouped",
                     help="extra modes timed after the streamed one (streamed_T<n>: streamed with n tokens; "
-                         "streamed_S<n>: streamed through n pool slots)")
+                         "streamed_S<n>: streamed through n pool slots; accum<n>: n micro-batches per step, "
+                         "gradients accumulated)")
     ap.add_argument("--api", choices=["layer", "proj"], default="layer",
                     help="one library call per layer, or one per projection")
     ap.add_argument("--lanes", type=int, default=2, help="streams the seven projections of a layer are spread over")

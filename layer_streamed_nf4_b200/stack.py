@@ -85,6 +85,18 @@ def _round_up(a: int, b: int) -> int:
     return (a + b - 1) // b * b
 
 
+def grad_layout(projs, layers: int, r: int):
+    """Element offsets of (dA, dB) of every (layer, projection) in one flat fp32 buffer, and its size:
+    per (layer, projection) dA [r, K] then dB [N, r], each starting on a 16-byte boundary."""
+    off, n = {}, 0
+    for l in range(layers):
+        for pi, p in enumerate(projs):
+            off[l, pi] = n
+            n += r * (p.K + p.N)
+            n = _round_up(n, 4)
+    return off, n
+
+
 @dataclass
 class ProjLayout:
     name: str
@@ -192,6 +204,10 @@ class Stack:
     def _build_tensors(self, distinct: bool):
         T, r, dev = self.T, self.r, self.dev
         self.x, self.dY, self.A, self.B, self.dA, self.dB = {}, {}, {}, {}, {}, {}
+        # every dA [r, K] and dB [N, r] of the stack in one fp32 buffer, so that data-parallel
+        # replicas sum them with one collective
+        self.grad_offsets, n = grad_layout(self.proj, self.L, r)
+        self.grads = torch.zeros(n, dtype=torch.float32, device=dev)
         h0 = None
         if self.cfg.vocab:
             # Layer 0 reads token embeddings: rows of a resident N(0, 1) bf16 table [vocab, hidden] picked by T
@@ -218,8 +234,9 @@ class Stack:
                                                      device=dev, dtype=torch.bfloat16)
                 self.B[l, pi] = synth.device_normal((p.N, r), 0.01, self.seed, l, pi, synth.T_B, device=dev,
                                                     dtype=torch.bfloat16)
-                self.dA[l, pi] = torch.zeros((r, p.K), dtype=torch.float32, device=dev)
-                self.dB[l, pi] = torch.zeros((p.N, r), dtype=torch.float32, device=dev)
+                o = self.grad_offsets[l, pi]
+                self.dA[l, pi] = self.grads[o:o + r * p.K].view(r, p.K)
+                self.dB[l, pi] = self.grads[o + r * p.K:o + r * (p.K + p.N)].view(p.N, r)
         nl = self.L if self.keep_outputs else 1
         self.y = {(l, pi): torch.empty((T, p.N), dtype=torch.bfloat16, device=dev)
                   for l in range(nl) for pi, p in enumerate(self.proj)}
