@@ -366,12 +366,7 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{cfg.name} NF4 LoRA stack: {L} layers x 7 projections (q,k,v,o,gate,up,down), "
-                               f"T={T} tokens (batch 1 x seq {T}), r={cfg.rank}, alpha={cfg.alpha:g}, "
-                               f"base NF4 blk-64 + double quant streamed from pinned host RAM, "
-                               f"{args.slots}-slot VRAM pool ({L} layers)",
-                   "tokens": T, "layers": L, "rank": cfg.rank, "pool_slots": args.slots, "base": cfg.base,
-                   "parallelism": f"dp{world}" + (" (adapter gradients summed over ranks each step)" if world > 1 else ""),
+        "config": {**workload_config(cfg, T, L, args.slots, world),
                    "api": args.api,
                    "lanes": args.lanes if args.api == "proj" else 1,
                    "nf4_conversion": "inside the GEMM" if args.fused_nf4 else "nf4_dequant then bf16 GEMM",
@@ -470,6 +465,17 @@ def cpu_baseline(args, sample_rows: int, budget_s: float):
             "seconds": t_total}
 
 
+def workload_config(cfg, T: int, L: int, slots: int, world: int) -> dict:
+    """The workload both arms report (the reference arm times a bounded sample of it, stated in its
+    cpu_baseline)."""
+    return {"workload": f"{cfg.name} NF4 LoRA stack: {L} layers x 7 projections (q,k,v,o,gate,up,down), "
+                        f"T={T} tokens (batch 1 x seq {T}), r={cfg.rank}, alpha={cfg.alpha:g}, "
+                        f"base NF4 blk-64 + double quant streamed from pinned host RAM, "
+                        f"{slots}-slot VRAM pool ({L} layers)",
+            "tokens": T, "layers": L, "rank": cfg.rank, "pool_slots": slots, "base": cfg.base,
+            "parallelism": f"dp{world}" + (" (adapter gradients summed over ranks each step)" if world > 1 else "")}
+
+
 def run_reference(args):
     world, rank, _ = _dist()
     if rank != 0:
@@ -486,8 +492,7 @@ def run_reference(args):
     line = {"metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": s_step * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": f"{cfg.name} NF4 LoRA stack (oracle sample)", "tokens": cfg.tokens,
-                       "layers": cfg.layers, "rank": cfg.rank},
+            "config": workload_config(cfg, cfg.tokens, cfg.layers, min(getattr(args, "slots", 20), cfg.layers), world),
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": vals[0]["cores"], "kind": "oracle",
                              "sample": vals[0]["sample"]},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
