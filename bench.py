@@ -371,7 +371,6 @@ def run_ours(args):
                    "lanes": args.lanes if args.api == "proj" else 1,
                    "nf4_conversion": "inside the GEMM" if args.fused_nf4 else "nf4_dequant then bf16 GEMM",
                    "programmatic_dependent_launch": not args.no_pdl,
-                   "gemm_tile_order": "dynamic" if lsnf4.get_option(lsnf4.LSN_OPT_DYN_TILES) else "static",
                    "dequant_ahead": st_main.ahead,
                    "l2": "inputs larger than L2 (per step ~11 GB of activations; every layer's NF4 codes read twice)"},
         "pct_bf16_peak": 100 * flop_step / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
@@ -578,19 +577,15 @@ def main():
     ap.add_argument("--no-pdl", action="store_true", help="ordinary launches instead of programmatic dependent ones")
     ap.add_argument("--dequant-ahead", type=int, default=1, choices=[0, 1],
                     help="dequantise each layer on a side stream one layer ahead (1, default) or inside the layer call")
-    ap.add_argument("--dyn-tiles", type=int, default=None, choices=[0, 1],
-                    help="GEMM tiles handed out at run time (1) or fixed by CTA index (0); default: the library's")
     ap.add_argument("--case", default="", help="profile one 8B projection (q,k,v,o,gate,up,down) instead of the stack")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
-    if args.impl == "ours" and (args.fused_nf4 or args.no_pdl or args.dyn_tiles is not None):
+    if args.impl == "ours" and (args.fused_nf4 or args.no_pdl):
         from layer_streamed_nf4_b200 import lsnf4
         if args.fused_nf4:
             lsnf4.set_option(lsnf4.LSN_OPT_FUSED_NF4, 1)
         if args.no_pdl:
             lsnf4.set_option(lsnf4.LSN_OPT_PDL, 0)
-        if args.dyn_tiles is not None:
-            lsnf4.set_option(lsnf4.LSN_OPT_DYN_TILES, args.dyn_tiles)
     if args.impl == "reference":
         run_reference(args)
     elif args.case:

@@ -193,10 +193,9 @@ typedef struct {
 } lsn_base;
 
 /* Workspace bytes lora_linear_fwd / lora_linear_bwd need (the larger of the two).
- * The workspace starts with a 256-byte status region -- the kernels' status
- * word and the GEMMs' tile counters -- which must start at zero: fill a new
- * workspace with zeros once.  The calls leave the counters at zero, and
- * lsn_ws_status clears the status word after reporting a timeout. */
+ * The workspace starts with the kernels' status word, which must start at
+ * zero: fill a new workspace with zeros once (lsn_ws_status clears it after
+ * reporting a timeout). */
 size_t lsn_lora_ws_bytes(int64_t T, int64_t K, int64_t N, int r, int kind);
 
 /* Forward.  y may not alias x.  ws: device scratch of lsn_lora_ws_bytes bytes,
@@ -267,9 +266,8 @@ typedef struct {
 
 /* Workspace bytes of lora_layer_fwd / lora_layer_bwd for these projections
  * (the larger of the two; 0 when an argument is invalid).  Like the
- * single-linear workspace it starts with the 256-byte status region and must
- * be zero-filled once when allocated.  With NF4 bases it holds the
- * dequantised bf16 copy of every projection. */
+ * single-linear workspace it must be zero-filled once when allocated.  With
+ * NF4 bases it holds the dequantised bf16 copy of every projection. */
 size_t lsn_layer_ws_bytes(int n, const lsn_lora_proj* p, int64_t T, int r);
 
 /* Forward of n projections: y_i = x_i W_i^T + s (x_i A_i^T) B_i^T. */
@@ -346,14 +344,8 @@ lsn_status lsn_timing_read(lsn_kernel_timing* out);
  *                      every kernel still waits for its predecessor to finish
  *                      before it reads or writes global memory.  0: ordinary
  *                      stream-ordered launches.
- *   LSN_OPT_DYN_TILES  1: the bf16 GEMMs (base + LoRA, forward and input
- *                      gradient) hand out their output tiles at run time from
- *                      a counter in the workspace's status region, so that
- *                      the GEMMs a layer call runs on its two streams take
- *                      over each other's idle SMs at the end of each GEMM;
- *                      0 (default): each CTA's tiles are fixed by its index.
  */
-typedef enum { LSN_OPT_FUSED_NF4 = 1, LSN_OPT_LAYER_LANES = 2, LSN_OPT_PDL = 3, LSN_OPT_DYN_TILES = 4 } lsn_option;
+typedef enum { LSN_OPT_FUSED_NF4 = 1, LSN_OPT_LAYER_LANES = 2, LSN_OPT_PDL = 3 } lsn_option;
 lsn_status lsn_set_option(int option, int value);
 int lsn_get_option(int option);
 

@@ -17,7 +17,6 @@ thread_local std::string g_last_error = "no error";
 std::atomic<int> g_fused_nf4{0};
 std::atomic<int> g_layer_lanes{2};
 std::atomic<int> g_pdl{1};
-std::atomic<int> g_dyn_tiles{0};
 }
 
 lsn_status fail(lsn_status st, const std::string& msg) {
@@ -31,7 +30,6 @@ lsn_status fail_cuda(cudaError_t e, const char* what) {
 }
 
 bool pdl_enabled() { return g_pdl.load() != 0; }
-bool dyn_tiles_enabled() { return g_dyn_tiles.load() != 0; }
 
 int sm_count() {
     int dev = 0;
@@ -393,9 +391,9 @@ lsn_status timed_tgrad(const float* G, const uint16_t* X, bool out_rk, int64_t T
 
 lsn_status timed_gemm(int kind, const uint16_t* A, int64_t lda, const uint16_t* B, int64_t ldb, bool b_mn,
                       const uint16_t* LA, const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D,
-                      int64_t ldd, int* err, cudaStream_t st, unsigned* sched) {
+                      int64_t ldd, int* err, cudaStream_t st) {
     TimingScope ts(kind, 2.0 * M * N * (double)(Kc + r), st);
-    return launch_gemm(A, lda, B, ldb, b_mn, LA, LB, r, M, N, Kc, D, ldd, err, st, sched);
+    return launch_gemm(A, lda, B, ldb, b_mn, LA, LB, r, M, N, Kc, D, ldd, err, st);
 }
 
 }  // namespace
@@ -513,7 +511,7 @@ lsn_status lora_linear_fwd(const lsn_base* W, const uint16_t* x, int64_t T, cons
         if ((s = timed_dequant(&W->nf4, w.w16, st)) != LSN_OK) return s;
         Wb = w.w16;
     }
-    return timed_gemm(LSN_K_GEMM_FWD, x, K, Wb, K, false, w.s16, B, r, T, N, K, y, N, w.err, st, gemm_sched(w.err, 0));
+    return timed_gemm(LSN_K_GEMM_FWD, x, K, Wb, K, false, w.s16, B, r, T, N, K, y, N, w.err, st);
 }
 
 lsn_status lora_linear_bwd(const lsn_base* W, const uint16_t* x, const uint16_t* dY, int64_t T, const uint16_t* A,
@@ -540,8 +538,7 @@ lsn_status lora_linear_bwd(const lsn_base* W, const uint16_t* x, const uint16_t*
                 if ((s = timed_dequant(&W->nf4, w.w16, st)) != LSN_OK) return s;
                 Wb = w.w16;
             }
-            if ((s = timed_gemm(LSN_K_GEMM_BWD, dY, N, Wb, K, true, w.s16, A, r, T, K, N, dX, K, w.err, st,
-                                gemm_sched(w.err, 0))) != LSN_OK)
+            if ((s = timed_gemm(LSN_K_GEMM_BWD, dY, N, Wb, K, true, w.s16, A, r, T, K, N, dX, K, w.err, st)) != LSN_OK)
                 return s;
         }
     }
@@ -621,7 +618,6 @@ lsn_status lora_layer_fwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
         const int i = g.first[k], m = g.count[k];
         const int64_t K = p[i].W.cols;
         const cudaStream_t gs = (k & 1) ? lanes.side() : lanes.main();
-        unsigned* sched = gemm_sched(w.err, gs == st ? 0 : 1);
         const int ri = adapter_off(p[i]) ? 0 : r;       // no LoRA K-block with the adapter off
         const uint16_t* Wb = p[i].W.kind == LSN_BASE_NF4 ? w.w16[i] : p[i].W.bf16;
         if (m > 1) {
@@ -639,8 +635,7 @@ lsn_status lora_layer_fwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
                 nsum += p[i + j].W.rows;
             }
             TimingScope ts(LSN_K_GEMM_FWD, 2.0 * T * nsum * (double)(K + m * ri), gs);
-            s = launch_gemm_grouped(gg, Wb, K, false, w.la[i], w.lb[i], m * ri, T, nsum, K, nullptr, 0, w.err, gs,
-                                    sched);
+            s = launch_gemm_grouped(gg, Wb, K, false, w.la[i], w.lb[i], m * ri, T, nsum, K, nullptr, 0, w.err, gs);
         } else if (fused_here(p[i].W, T, p[i].W.rows)) {
             const int64_t N = p[i].W.rows;
             TimingScope ts(LSN_K_GEMM_FWD, 2.0 * T * N * (double)(K + ri), gs);
@@ -648,7 +643,7 @@ lsn_status lora_layer_fwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
         } else {
             const int64_t N = p[i].W.rows;
             s = timed_gemm(LSN_K_GEMM_FWD, p[i].x, K, Wb, K, false, w.s16[i], p[i].B, ri, T, N, K, p[i].y, N, w.err,
-                           gs, sched);
+                           gs);
         }
         if (s != LSN_OK) return s;
     }
@@ -710,7 +705,6 @@ lsn_status lora_layer_bwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
             if (!p[i].dX) continue;
             const int64_t K = p[i].W.cols;
             const cudaStream_t gs = (j++ & 1) ? lanes.side() : lanes.main();
-            unsigned* sched = gemm_sched(w.err, gs == st ? 0 : 1);
             const int ri = adapter_off(p[i]) ? 0 : r;
             const uint16_t* Wb = p[i].W.kind == LSN_BASE_NF4 ? w.w16[i] : p[i].W.bf16;
             if (m > 1) {
@@ -725,8 +719,7 @@ lsn_status lora_layer_bwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
                     nsum += p[i + q].W.rows;
                 }
                 TimingScope ts(LSN_K_GEMM_BWD, 2.0 * T * K * (double)(nsum + m * ri), gs);
-                s = launch_gemm_grouped(gg, Wb, K, true, w.la[i], w.lb[i], m * ri, T, K, nsum, p[i].dX, K, w.err, gs,
-                                        sched);
+                s = launch_gemm_grouped(gg, Wb, K, true, w.la[i], w.lb[i], m * ri, T, K, nsum, p[i].dX, K, w.err, gs);
             } else if (fused_here(p[i].W, T, K)) {
                 const int64_t N = p[i].W.rows;
                 TimingScope ts(LSN_K_GEMM_BWD, 2.0 * T * K * (double)(N + ri), gs);
@@ -735,7 +728,7 @@ lsn_status lora_layer_bwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
             } else {
                 const int64_t N = p[i].W.rows;
                 s = timed_gemm(LSN_K_GEMM_BWD, p[i].dY, N, Wb, K, true, w.s16[i], p[i].A, ri, T, K, N, p[i].dX, K,
-                               w.err, gs, sched);
+                               w.err, gs);
             }
             if (s != LSN_OK) return s;
         }
@@ -757,10 +750,6 @@ lsn_status lsn_set_option(int option, int value) {
         g_fused_nf4.store(value != 0 ? 1 : 0);
         return LSN_OK;
     }
-    if (option == LSN_OPT_DYN_TILES) {
-        g_dyn_tiles.store(value != 0 ? 1 : 0);
-        return LSN_OK;
-    }
     return fail(LSN_ERR_INVALID_ARG, "lsn_set_option: unknown option");
 }
 
@@ -768,7 +757,6 @@ int lsn_get_option(int option) {
     if (option == LSN_OPT_FUSED_NF4) return g_fused_nf4.load();
     if (option == LSN_OPT_LAYER_LANES) return g_layer_lanes.load();
     if (option == LSN_OPT_PDL) return g_pdl.load();
-    if (option == LSN_OPT_DYN_TILES) return g_dyn_tiles.load();
     return -1;
 }
 

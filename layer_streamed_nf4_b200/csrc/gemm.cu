@@ -72,9 +72,6 @@ struct GemmArgs {
     float dq[256];             // second-level table
     const uint16_t* lora_b;    // LoRA operand of the last K-block (fwd: B [N, r]; bwd: A [r, N])
     int lora_r;
-    // Dynamic tile order (the DYN kernels): [0] ticket counter, [1] CTAs
-    // finished; both zero at launch, and the last CTA to finish zeroes them.
-    unsigned* sched;
 };
 
 namespace {
@@ -93,9 +90,6 @@ constexpr int CONV_WARPS = 8;    // NF4 converter warps (fused variant)
 // PAIR = false: one CTA per SM, tile 128 x BN.
 // PAIR = true : a CTA pair (cluster of 2) issues the 2-SM MMA, tile 256 x BN,
 //               each CTA staging its 128 rows of A and BN/2 rows of B.
-// Ring of tile indices between the tile fetcher and the other roles (DYN).
-constexpr int SCHED_SLOTS = 8;
-
 template <bool PAIR, int BN, bool B_MN>
 struct Cfg {
     static constexpr int B_ROWS = PAIR ? BN / 2 : BN;     // B rows (N extent) staged per CTA
@@ -104,11 +98,8 @@ struct Cfg {
     static constexpr int B_SUB = B_ROWS * SUB * 2;         // K-major: bytes of one B sub-tile
     static constexpr int B_BYTES = 2 * B_SUB;              // MN-major: B_ROWS/64 atom columns of 128 x 64
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int BAR_BYTES = 512;
+    static constexpr int BAR_BYTES = 256;
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
-    // Readers of each tile index (DYN): the MMA issuer and 4 epilogue warps,
-    // plus, on a pair, the peer CTA's producer and 4 epilogue warps.
-    static constexpr uint32_t SCHED_READERS = PAIR ? 10 : 5;
     static constexpr uint32_t IDESC = idesc_bf16(PAIR ? 2 * BM : BM, BN, 0, B_MN ? 1 : 0);
     static constexpr uint32_t TMEM_COLS = 2 * BN;
     static constexpr int TILE_M = PAIR ? 2 * BM : BM;
@@ -121,70 +112,12 @@ __device__ __forceinline__ void raise_error(volatile int* abort_flag, int* err, 
     if (err) atomicExch(err, code);
 }
 
-// The sequence of output tiles one role of a CTA works through.
-//
-// Static (DYN = false): unit, unit + nunits, unit + 2 nunits, ... .
-// Dynamic (DYN = true): the producer of the CTA (pair leader) takes tickets
-// from a counter in global memory, one per tile, and hands each tile index to
-// the other roles of its CTA (and of the peer CTA) through a ring of slots in
-// shared memory: index, "full" barrier (one arrival: the fetcher) and "empty"
-// barrier (one arrival per reader).  A ticket past the last tile is handed on
-// as -1, which ends every role's loop.  Units that start early (on SMs another
-// grid has left) take more tiles, so two grids on different streams fill each
-// other's last waves.  Which unit computes a tile does not change its
-// arithmetic, so results are the same bits in both orders.
-template <bool PAIR, bool DYN>
-struct TileSeq {
-    uint64_t* full;
-    uint64_t* empty;
-    int* slot_tile;
-    volatile int* abort;
-    int num_tiles, unit, nunits;
-    int i = 0;
-
-    // Static order, every role.
-    __device__ bool next_static(int& t) {
-        t = unit + i * nunits;
-        ++i;
-        return t < num_tiles;
-    }
-    // Dynamic order, the fetcher (producer of the leader CTA).  `ticket` is
-    // the ticket taken for this tile; ok turns false when a wait ran out.
-    __device__ bool fetch(int& t, unsigned ticket, bool& ok) {
-        const int s = i % SCHED_SLOTS;
-        const uint32_t ph = (uint32_t)(i / SCHED_SLOTS) & 1u;
-        if (!mbar_wait_cluster(&empty[s], ph ^ 1u, abort)) { ok = false; return false; }
-        t = ticket < (unsigned)num_tiles ? (int)ticket : -1;
-        slot_tile[s] = t;
-        if constexpr (PAIR) {
-            st_cluster_u32(mapa_shared(smem_u32(&slot_tile[s]), 1), (uint32_t)t);
-            mbar_arrive_cluster(mapa_shared(smem_u32(&full[s]), 1));
-        }
-        mbar_arrive(&full[s]);
-        ++i;
-        return t >= 0;
-    }
-    // Dynamic order, every other reader (one thread per reader).
-    __device__ bool take(int& t, bool releaser, bool& ok) {
-        const int s = i % SCHED_SLOTS;
-        const uint32_t ph = (uint32_t)(i / SCHED_SLOTS) & 1u;
-        if (!mbar_wait_cluster(&full[s], ph, abort)) { ok = false; return false; }
-        t = *reinterpret_cast<volatile int*>(&slot_tile[s]);
-        if (releaser) {
-            if constexpr (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&empty[s]), 0));
-            else                mbar_arrive(&empty[s]);
-        }
-        ++i;
-        return t >= 0;
-    }
-};
-
 // The A tensor maps of a grouped GEMM (the caller's separate dY tensors).
 struct AMaps {
     CUtensorMap m[kMaxSeg];
 };
 
-template <bool PAIR, int BN, bool B_MN, bool DYN>
+template <bool PAIR, int BN, bool B_MN>
 __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
     lsn_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmLA, const __grid_constant__ CUtensorMap tmLB,
@@ -200,9 +133,6 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
     uint64_t* drain = acc_empty + 2;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-    uint64_t* sched_full = bars + 16;                       // DYN: tile-index ring (bytes 128..)
-    uint64_t* sched_empty = sched_full + SCHED_SLOTS;
-    int* sched_tile = reinterpret_cast<int*>(sched_empty + SCHED_SLOTS);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint32_t rank = 0;
@@ -214,7 +144,6 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
     const int num_n = (p.N + BN - 1) / BN;
     const int num_tiles = num_m * num_n;
     const int nkb = p.num_kb + (p.lora_k16 > 0 ? 1 : 0);
-    TileSeq<PAIR, DYN> seq{sched_full, sched_empty, sched_tile, abort_flag, num_tiles, unit, nunits};
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -223,12 +152,6 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], C::ACC_EMPTY_ARRIVALS); }
         mbar_init(drain, 1);
-        if constexpr (DYN) {
-            for (int s = 0; s < SCHED_SLOTS; ++s) {
-                mbar_init(&sched_full[s], 1);
-                mbar_init(&sched_empty[s], C::SCHED_READERS);
-            }
-        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -255,11 +178,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            unsigned ticket = 0;
-            if constexpr (DYN) { if (leader) ticket = atomicAdd(p.sched, 1u); }
-            int tile;
-            while (ok && (!DYN ? seq.next_static(tile)
-                               : (leader ? seq.fetch(tile, ticket, ok) : seq.take(tile, true, ok)))) {
+            for (int tile = unit; tile < num_tiles && ok; tile += nunits) {
                 const int mb = tile % num_m, nb = tile / num_m;
                 const int m_row = mb * C::TILE_M + (int)rank * BM;
                 const int n_off = nb * BN + (int)rank * C::B_ROWS;
@@ -292,8 +211,6 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
                     }
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
-                // the next tile's ticket, taken once this tile's loads are all issued
-                if constexpr (DYN) { if (leader && ok) ticket = atomicAdd(p.sched, 1u); }
             }
             if (!ok) raise_error(abort_flag, p.err, 1);
         }
@@ -303,8 +220,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
-            int tile;
-            while (ok && (!DYN ? seq.next_static(tile) : seq.take(tile, true, ok))) {
+            for (int tile = unit; tile < num_tiles && ok; tile += nunits) {
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
@@ -344,17 +260,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
         const int nseg = p.nseg;
         int acc = 0;
         uint32_t acc_phase = 0;
-        while (true) {
-            int tile = -1;
-            if constexpr (!DYN) {
-                if (!seq.next_static(tile)) break;
-            } else {
-                bool ok = true;
-                if (lane == 0) seq.take(tile, true, ok);
-                tile = __shfl_sync(0xffffffffu, tile, 0);
-                if (!__shfl_sync(0xffffffffu, (int)ok, 0)) { if (lane == 0) raise_error(abort_flag, p.err, 4); break; }
-                if (tile < 0) break;
-            }
+        for (int tile = unit; tile < num_tiles; tile += nunits) {
             const int mb = tile % num_m, nb = tile / num_m;
             const bool got = mbar_wait(&acc_full[acc], acc_phase, abort_flag);
             if (!__all_sync(0xffffffffu, got)) { if (lane == 0) raise_error(abort_flag, p.err, 3); break; }
@@ -408,18 +314,6 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
         tc_fence_after();
         if constexpr (PAIR) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
         else                tmem_dealloc(tmem_base, C::TMEM_COLS);
-    }
-    if constexpr (DYN) {
-        // Every ticket of this grid has been taken once this CTA is here; the
-        // last CTA to arrive leaves the counters at zero for the next grid on
-        // the stream (which reads them only after this grid has finished).
-        if (threadIdx.x == 0) {
-            __threadfence();
-            if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
-                atomicExch(p.sched, 0u);
-                atomicExch(p.sched + 1, 0u);
-            }
-        }
     }
 }
 
@@ -796,14 +690,14 @@ lsn_status make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t out
     return LSN_OK;
 }
 
-template <bool PAIR, int BN, bool B_MN, bool DYN>
+template <bool PAIR, int BN, bool B_MN>
 lsn_status launch_cfg(const AMaps& a, const CUtensorMap& b, const CUtensorMap& la, const CUtensorMap& lb,
                       const GemmArgs& args, cudaStream_t st) {
     using C = Cfg<PAIR, BN, B_MN>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(lsn_gemm_kernel<PAIR, BN, B_MN, DYN>,
+        attr_err = cudaFuncSetAttribute(lsn_gemm_kernel<PAIR, BN, B_MN>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     });
     if (attr_err != cudaSuccess) return fail_cuda(attr_err, "cudaFuncSetAttribute(gemm smem)");
@@ -827,15 +721,8 @@ lsn_status launch_cfg(const AMaps& a, const CUtensorMap& b, const CUtensorMap& l
     na += pdl_attr(&attr[na]);
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    LSN_CUDA_TRY(cudaLaunchKernelEx(&cfg, lsn_gemm_kernel<PAIR, BN, B_MN, DYN>, a, b, la, lb, args));
+    LSN_CUDA_TRY(cudaLaunchKernelEx(&cfg, lsn_gemm_kernel<PAIR, BN, B_MN>, a, b, la, lb, args));
     return LSN_OK;
-}
-
-template <bool PAIR, int BN, bool B_MN>
-lsn_status launch_sched(const AMaps& a, const CUtensorMap& b, const CUtensorMap& la, const CUtensorMap& lb,
-                        const GemmArgs& args, cudaStream_t st) {
-    return args.sched ? launch_cfg<PAIR, BN, B_MN, true>(a, b, la, lb, args, st)
-                      : launch_cfg<PAIR, BN, B_MN, false>(a, b, la, lb, args, st);
 }
 
 }  // namespace
@@ -924,7 +811,7 @@ lsn_status launch_gemm_nf4(const uint16_t* A, int64_t lda, const lsn_nf4_weight*
 //   LA [M, r] (bf16(s u) or bf16(s g)); r == 0 disables the LoRA term.
 lsn_status launch_gemm_grouped(const GemmGroup& g, const uint16_t* B, int64_t ldb, bool b_mn, const uint16_t* LA,
                                const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D,
-                               int64_t ldd, int* err, cudaStream_t st, unsigned* sched) {
+                               int64_t ldd, int* err, cudaStream_t st) {
     if (g.na < 1 || g.na > kMaxSeg || g.nseg < 0 || g.nseg > kMaxSeg)
         return fail(LSN_ERR_INVALID_ARG, "grouped GEMM: bad operand or segment count");
     const bool pair = gemm_use_pairs(M, N);
@@ -968,7 +855,6 @@ lsn_status launch_gemm_grouped(const GemmGroup& g, const uint16_t* B, int64_t ld
     args.D = D;
     args.ldd = ldd;
     args.err = err;
-    args.sched = dyn_tiles_enabled() ? sched : nullptr;
     args.nseg = g.nseg;
     int64_t c0 = 0;
     for (int i = 0; i < g.nseg; ++i) {
@@ -979,21 +865,21 @@ lsn_status launch_gemm_grouped(const GemmGroup& g, const uint16_t* B, int64_t ld
     }
     args.seg_col[g.nseg] = (int)c0;
     if (g.nseg > 0 && c0 != N) return fail(LSN_ERR_INVALID_ARG, "grouped GEMM: segments do not add up to N");
-    if (pair) return b_mn ? launch_sched<true, 256, true>(ma, mb, mla, mlb, args, st)
-                          : launch_sched<true, 256, false>(ma, mb, mla, mlb, args, st);
-    return b_mn ? launch_sched<false, 128, true>(ma, mb, mla, mlb, args, st)
-                : launch_sched<false, 128, false>(ma, mb, mla, mlb, args, st);
+    if (pair) return b_mn ? launch_cfg<true, 256, true>(ma, mb, mla, mlb, args, st)
+                          : launch_cfg<true, 256, false>(ma, mb, mla, mlb, args, st);
+    return b_mn ? launch_cfg<false, 128, true>(ma, mb, mla, mlb, args, st)
+                : launch_cfg<false, 128, false>(ma, mb, mla, mlb, args, st);
 }
 
 lsn_status launch_gemm(const uint16_t* A, int64_t lda, const uint16_t* B, int64_t ldb, bool b_mn, const uint16_t* LA,
                        const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D, int64_t ldd,
-                       int* err, cudaStream_t st, unsigned* sched) {
+                       int* err, cudaStream_t st) {
     GemmGroup g;
     g.na = 1;
     g.A[0] = A;
     g.lda[0] = lda;
     g.a_kc[0] = Kc;
-    return launch_gemm_grouped(g, B, ldb, b_mn, LA, LB, r, M, N, Kc, D, ldd, err, st, sched);
+    return launch_gemm_grouped(g, B, ldb, b_mn, LA, LB, r, M, N, Kc, D, ldd, err, st);
 }
 
 }  // namespace lsn

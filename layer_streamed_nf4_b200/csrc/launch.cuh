@@ -67,21 +67,12 @@ struct GemmGroup {
     uint16_t* seg_D[kGemmMaxSeg] = {};
     int64_t seg_ld[kGemmMaxSeg] = {};
 };
-// sched: two words of device memory for the dynamic tile order (zero before
-// the launch, left zero by it), used when LSN_OPT_DYN_TILES is on; one pair
-// per stream that GEMMs run on, never shared by GEMMs that may overlap.
-// nullptr: the static order.
 lsn_status launch_gemm_grouped(const GemmGroup& g, const uint16_t* B, int64_t ldb, bool b_mn, const uint16_t* LA,
                                const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D,
-                               int64_t ldd, int* err, cudaStream_t st, unsigned* sched = nullptr);
+                               int64_t ldd, int* err, cudaStream_t st);
 lsn_status launch_gemm(const uint16_t* A, int64_t lda, const uint16_t* B, int64_t ldb, bool b_mn, const uint16_t* LA,
                        const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D, int64_t ldd,
-                       int* err, cudaStream_t st, unsigned* sched = nullptr);
-bool dyn_tiles_enabled();
-// The tile counters of lane `lane` (0: the caller's stream, 1: the library's
-// second stream) inside a workspace's 256-byte status region, whose first
-// word is `err`: bytes 64 + 16 lane .. 72 + 16 lane.
-inline unsigned* gemm_sched(int* err, int lane) { return reinterpret_cast<unsigned*>(err) + 16 + 4 * lane; }
+                       int* err, cudaStream_t st);
 lsn_status launch_gemm_nf4(const uint16_t* A, int64_t lda, const lsn_nf4_weight* w, bool b_mn, const uint16_t* LA,
                            const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D, int64_t ldd,
                            int* err, cudaStream_t st);

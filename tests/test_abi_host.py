@@ -194,11 +194,6 @@ def test_options(lib):
     lib.set_option(lib.LSN_OPT_PDL, 0)
     assert lib.get_option(lib.LSN_OPT_PDL) == 0
     lib.set_option(lib.LSN_OPT_PDL, 1)
-    dyn = lib.get_option(lib.LSN_OPT_DYN_TILES)
-    assert dyn == 0
-    lib.set_option(lib.LSN_OPT_DYN_TILES, 1)
-    assert lib.get_option(lib.LSN_OPT_DYN_TILES) == 1
-    lib.set_option(lib.LSN_OPT_DYN_TILES, dyn)
     assert lib.get_option(12345) == -1
 
 

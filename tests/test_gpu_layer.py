@@ -307,55 +307,3 @@ def test_group_arguments_are_checked(lib):
     with pytest.raises(lib.LsnError) as e:
         lib.lora_layer_fwd(lib.proj_array(projs), L.T, L.r, L.scale, ws, n)
     assert e.value.status == lib.LSN_ERR_INVALID_ARG
-
-
-def _layer_keep_ws(lib, L, groups=None):
-    """Layer forward + backward with the outputs and the workspace (to inspect its status region)."""
-    import torch
-    out = L.outputs()
-    groups = groups or (0,) * len(L.p)
-    projs = []
-    for pi, (d, o) in enumerate(zip(L.p, out)):
-        lead = groups[pi] == 0 or pi == 0 or groups[pi - 1] != groups[pi]
-        projs.append(lib.lora_proj(d["base"], d["x"], d["A"], d["B"], y=o["y"], dY=d["dY"],
-                                   dX=o["dX"] if lead else None, dA=o["dA"], dB=o["dB"], u=o["u"],
-                                   group=groups[pi]))
-    arr = lib.proj_array(projs)
-    n = lib.layer_ws_bytes(arr, L.T, L.r)
-    ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
-    for _ in range(2):                                # the second round reuses the tile counters
-        lib.lora_layer_fwd(arr, L.T, L.r, L.scale, ws, n)
-        lib.lora_layer_bwd(arr, L.T, L.r, L.scale, False, ws, n)
-    torch.cuda.synchronize()
-    lib.ws_status(ws)
-    return out, ws
-
-
-@pytest.mark.parametrize("shapes,T,kind", [(SHAPES_8B, 2048, "nf4"), (SMALL, 257, "nf4"), (SMALL_G, 300, "bf16")])
-def test_dynamic_tile_order_gives_the_same_bits(lib, shapes, T, kind):
-    """GEMM output tiles handed out at run time (LSN_OPT_DYN_TILES) instead of fixed by CTA index: the same
-    bits from the layer calls on two lanes and on one, with groups, and from the single-linear calls; the
-    tile counters in the workspace's status region are back at zero after every call."""
-    L = _grouped_setup(lib, shapes, T, kind, seed=8) if shapes is SMALL_G else Layer(lib, shapes, T, 16, kind, seed=8)
-    groups = GROUPS if shapes is SMALL_G else None
-    ref, _ = _layer_keep_ws(lib, L, groups)
-    ref_single = L.single() if groups is None else None
-    lib.set_option(lib.LSN_OPT_DYN_TILES, 1)
-    try:
-        two, ws2 = _layer_keep_ws(lib, L, groups)
-        lib.set_option(lib.LSN_OPT_LAYER_LANES, 1)
-        one, ws1 = _layer_keep_ws(lib, L, groups)
-        lib.set_option(lib.LSN_OPT_LAYER_LANES, 2)
-        single = L.single() if groups is None else None
-    finally:
-        lib.set_option(lib.LSN_OPT_DYN_TILES, 0)
-        lib.set_option(lib.LSN_OPT_LAYER_LANES, 2)
-    names = ("y", "dX", "dA", "dB") if groups is None else ("y", "dA", "dB", "u")
-    _equal(two, ref, names)
-    _equal(one, ref, names)
-    if groups is not None:
-        _equal([two[0], two[3], two[4], two[6]], [ref[0], ref[3], ref[4], ref[6]], ("dX",))
-    else:
-        _equal(single, ref_single)
-    for ws in (ws1, ws2):
-        assert int(ws[64:96].count_nonzero()) == 0, ws[64:96].tolist()

@@ -162,22 +162,6 @@ def test_resident_constants_give_the_same_bits(lib):
         st.close()
 
 
-def test_dynamic_tile_order_in_the_stack(lib):
-    """A streamed 8B stack with the GEMM tiles handed out at run time gives the resident run's bits."""
-    import torch
-    cfg = synth.STACKS["8b"]
-    res = _run(cfg, 3, 512, "resident")
-    lib.set_option(lib.LSN_OPT_DYN_TILES, 1)
-    try:
-        dyn = _run(cfg, 3, 512, "streamed", steps=2)
-    finally:
-        lib.set_option(lib.LSN_OPT_DYN_TILES, 0)
-    fwd, bwd, bad = _compare(dyn, res)
-    assert fwd and bwd, bad
-    assert int(dyn.ws[0][64:96].count_nonzero()) == 0
-    dyn.close()
-
-
 def test_first_layer_reads_token_embeddings(lib):
     """0.5B workload: the layer-0 inputs of q, k and v are the rows of the resident embedding table that
     the token ids pick; the ids cover the vocabulary uniformly."""
