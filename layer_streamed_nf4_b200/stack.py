@@ -108,6 +108,24 @@ class ProjLayout:
     cbytes: int = 0
 
 
+def layer_layout(cfg: synth.StackConfig, resident_constants: bool = True):
+    """(projection layouts, streamed bytes per layer, resident constant bytes per layer).  NF4: per
+    projection the blob of lsn_nf4_blob_layout, split after the packed codes when the constants stay
+    resident; bf16: the row-major matrix.  Every piece starts on a 1 KiB boundary."""
+    nf4 = cfg.base == "nf4"
+    off = coff = 0
+    projs: list[ProjLayout] = []
+    for name, K, N in cfg.projections:
+        nb, cb = (lsnf4.nf4_blob_bytes(N, K) if nf4 else _round_up(N * K * 2, 1024)), 0
+        if nf4 and resident_constants:              # stream the packed codes, keep the constants on the device
+            cb = nb - lsnf4.nf4_blob_layout(N, K)[1]
+            nb -= cb
+        projs.append(ProjLayout(name, K, N, off, nb, coff, cb))
+        off += nb
+        coff += cb
+    return projs, off, coff
+
+
 class Stack:
     def __init__(self, cfg: synth.StackConfig, layers: int | None = None, tokens: int | None = None,
                  mode: str = "streamed", n_slots: int = 2, seed: int = synth.SEED, keep_outputs: bool = False,
@@ -135,18 +153,7 @@ class Stack:
         self.lanes = [self.stream] + [torch.cuda.Stream(self.dev) for _ in range(lanes - 1)]
         self._fork = [torch.cuda.Event() for _ in range(lanes)]
         self._join = [torch.cuda.Event() for _ in range(lanes)]
-        off = coff = 0
-        self.proj: list[ProjLayout] = []
-        for name, K, N in cfg.projections:
-            nb, cb = (lsnf4.nf4_blob_bytes(N, K) if self.nf4 else _round_up(N * K * 2, 1024)), 0
-            if self.nf4 and resident_constants:         # stream the packed codes, keep the constants on the device
-                cb = nb - lsnf4.nf4_blob_layout(N, K)[1]
-                nb -= cb
-            self.proj.append(ProjLayout(name, K, N, off, nb, coff, cb))
-            off += nb
-            coff += cb
-        self.layer_bytes = off
-        self.const_bytes = coff
+        self.proj, self.layer_bytes, self.const_bytes = layer_layout(cfg, resident_constants)
         self.consts = None
         self.pool = None
         self.host = None
