@@ -154,3 +154,22 @@ def test_reference_and_recompute_steps_keep_the_pool_consistent(monkeypatch, L, 
         st.step(reference=True, recompute=True)
         assert pool.acquired[a0:] == list(range(L)) * 2 + list(reversed(range(L)))
         assert sum(pool.refs) == 0
+
+
+def test_layer_layout_splits_codes_and_constants():
+    """With resident constants a layer blob is the packed codes alone (4 bits per weight, 1 KiB aligned);
+    codes plus constants add up to the whole-blob layout, piece by piece."""
+    for name, cfg in synth.STACKS.items():
+        codes, lb, cb = layer_layout(cfg, True)
+        whole, wb, wcb = layer_layout(cfg, False)
+        assert lb + cb == wb and wcb == 0
+        for p, q in zip(codes, whole):
+            assert p.nbytes + p.cbytes == q.nbytes
+            assert p.offset % 1024 == 0 and p.coffset % 1024 == 0
+            if cfg.base == "nf4":
+                assert p.nbytes == -(-p.N * p.K // 2 // 1024) * 1024
+                assert p.cbytes == lsnf4.nf4_blob_bytes(p.N, p.K) - lsnf4.nf4_blob_layout(p.N, p.K)[1]
+            else:
+                assert p.cbytes == 0 and p.nbytes == -(-p.N * p.K * 2 // 1024) * 1024
+    _, lb, cb = layer_layout(synth.STACKS["8b"], True)
+    assert (lb, cb) == (109051904, 3468288)          # 8B layer: 109.05 MB streamed, 3.47 MB resident
