@@ -393,6 +393,7 @@ def run_ours(args):
         "step_kernel_ms": step_kernel_ms,
         "peak_mem_gb": torch.cuda.max_memory_allocated() / 1e9,
         "gpu_launches": launches,
+        "gpu": torch.cuda.get_device_name(local),
         "clocks": clocks,
         "e2e": e2e,
     }

@@ -430,6 +430,17 @@ typedef enum {
 } lsn_pool_fault;
 lsn_status layer_pool_inject_fault(lsn_pool* pool, int fault);
 
+/* Debugging aids (flags, 0 = none):
+ *   LSN_POOL_DEBUG_POISON  before every copy the slot is filled with 0xFF
+ *                          bytes (on the copy stream, after the slot's
+ *                          released event), so a read of a slot outside its
+ *                          acquire..release window sees the sentinel instead
+ *                          of plausible weights: NF4 codes of all 15s, bf16
+ *                          NaNs.  Costs one device-side fill per copy.
+ * LSN_ERR_INVALID_ARG for a NULL pool or unknown flag bits. */
+typedef enum { LSN_POOL_DEBUG_POISON = 1 } lsn_pool_debug_flag;
+lsn_status layer_pool_set_debug(lsn_pool* pool, int flags);
+
 /* Free the slots, events and the copy stream (waits for pending copies). */
 void layer_pool_destroy(lsn_pool* pool);
 

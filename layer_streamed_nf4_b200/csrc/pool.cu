@@ -49,6 +49,7 @@ struct lsn_pool {
     uint64_t tick = 0;
     lsn_pool_stats stats = {};
     int fault = LSN_POOL_FAULT_NONE;
+    int debug = 0;                                    // LSN_POOL_DEBUG_* flags
     std::unordered_map<int, std::vector<int>> held;   // layer -> slots acquired for it
     std::mutex mu;
 };
@@ -107,6 +108,8 @@ lsn_status start_copy(lsn_pool* p, int layer, int* slot_out) {
     if (p->timing_live == kTimingRing) harvest_timing(p, true);
     const int ti = p->timing_next;
     LSN_CUDA_TRY(cudaEventRecord(p->t0[ti], p->copy));
+    // Debugging aid: the slot holds a sentinel from its release until the copy lands.
+    if (p->debug & LSN_POOL_DEBUG_POISON) LSN_CUDA_TRY(cudaMemsetAsync(dst, 0xFF, p->slot_bytes, p->copy));
     // Planted defect (test hook): a reused slot is relabelled without its copy.
     const bool stale = p->fault == LSN_POOL_FAULT_STALE_SLOT && sl.layer >= 0;
     if (!stale)
@@ -299,6 +302,14 @@ lsn_status layer_pool_inject_fault(lsn_pool* p, int fault) {
     LSN_CHECK_ARG(fault >= LSN_POOL_FAULT_NONE && fault <= LSN_POOL_FAULT_COPY_ERROR, "layer_pool_inject_fault: unknown fault");
     std::lock_guard<std::mutex> lk(p->mu);
     p->fault = fault;
+    return LSN_OK;
+}
+
+lsn_status layer_pool_set_debug(lsn_pool* p, int flags) {
+    LSN_CHECK_ARG(p != nullptr, "layer_pool_set_debug: pool is NULL");
+    LSN_CHECK_ARG((flags & ~LSN_POOL_DEBUG_POISON) == 0, "layer_pool_set_debug: unknown flag bits");
+    std::lock_guard<std::mutex> lk(p->mu);
+    p->debug = flags;
     return LSN_OK;
 }
 

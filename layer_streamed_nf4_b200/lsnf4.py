@@ -26,6 +26,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 LSN_OK, LSN_ERR_INVALID_ARG, LSN_ERR_CUDA, LSN_ERR_NO_MEMORY, LSN_ERR_TIMEOUT, LSN_ERR_UNSUPPORTED, LSN_ERR_STATE = range(7)
 LSN_BASE_NF4, LSN_BASE_BF16 = 0, 1
 LSN_POOL_FAULT_NONE, LSN_POOL_FAULT_STALE_SLOT, LSN_POOL_FAULT_COPY_ERROR = 0, 1, 2
+LSN_POOL_DEBUG_POISON = 1
 LSN_OPT_FUSED_NF4 = 1
 LSN_OPT_LAYER_LANES = 2
 LSN_OPT_PDL = 3
@@ -44,7 +45,7 @@ EXPORTS = (
     "layer_pool_inject_fault", "layer_pool_destroy", "lsn_timing_enable", "lsn_timing_read",
     "nf4_quantize_noalloc", "lsn_set_option", "lsn_get_option",
     "lsn_layer_ws_bytes", "lora_layer_fwd", "lora_layer_bwd", "nf4_dequant_batch",
-    "lsn_selftest_wait_timeout",
+    "lsn_selftest_wait_timeout", "layer_pool_set_debug",
 )
 
 
@@ -130,6 +131,7 @@ _sig("layer_pool_wait_idle", _i, [_vp, _i])
 _sig("layer_pool_stats", _i, [_vp, ctypes.POINTER(PoolStats)])
 _sig("layer_pool_reset", _i, [_vp])
 _sig("layer_pool_inject_fault", _i, [_vp, _i])
+_sig("layer_pool_set_debug", _i, [_vp, _i])
 _sig("layer_pool_destroy", None, [_vp])
 
 
@@ -359,6 +361,10 @@ def layer_pool_reset(pool: int):
 
 def layer_pool_inject_fault(pool: int, fault: int):
     _check(_lib.layer_pool_inject_fault(pool, fault), "layer_pool_inject_fault")
+
+
+def layer_pool_set_debug(pool: int, flags: int):
+    _check(_lib.layer_pool_set_debug(pool, flags), "layer_pool_set_debug")
 
 
 def layer_pool_destroy(pool: int):

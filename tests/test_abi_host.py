@@ -197,6 +197,12 @@ def test_options(lib):
     assert lib.get_option(12345) == -1
 
 
+def test_pool_debug_rejects_a_null_pool(lib):
+    with pytest.raises(lib.LsnError) as e:
+        lib.layer_pool_set_debug(None, lib.LSN_POOL_DEBUG_POISON)
+    assert e.value.status == lib.LSN_ERR_INVALID_ARG
+
+
 def test_dequant_batch_rejects_bad_arguments(lib):
     w = lib.make_nf4_weight(64, 128, 1 << 20, 1 << 20, 1 << 20, 1 << 20)
     with pytest.raises(lib.LsnError) as e:                       # misaligned output

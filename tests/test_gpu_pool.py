@@ -183,6 +183,30 @@ def test_first_layer_reads_token_embeddings(lib):
     st.close()
 
 
+def test_slot_poisoning(lib):
+    """With every slot filled with 0xFF bytes before each copy, a correct pool still gives the resident
+    bits (no kernel reads a slot outside its acquire..release window), and the planted stale slot, now
+    holding the sentinel instead of an older layer, is caught as before."""
+    import torch
+    from layer_streamed_nf4_b200.stack import Stack
+    cfg = synth.STACKS["8b"]
+    res = _run(cfg, 4, 256, "resident")
+    for fault, equal in ((None, True), (lib.LSN_POOL_FAULT_STALE_SLOT, False)):
+        st = Stack(cfg, layers=4, tokens=256, mode="streamed", keep_outputs=True)
+        lib.layer_pool_set_debug(st.pool, lib.LSN_POOL_DEBUG_POISON)
+        with pytest.raises(lib.LsnError) as e:        # unknown flag bits: refused, the setting stays
+            lib.layer_pool_set_debug(st.pool, 4)
+        assert e.value.status == lib.LSN_ERR_INVALID_ARG
+        if fault is not None:
+            lib.layer_pool_inject_fault(st.pool, fault)
+        st.step()
+        st.step()
+        torch.cuda.synchronize()
+        fwd, bwd, bad = _compare(st, res)
+        assert (fwd and bwd) == equal, (fault, bad)
+        st.close()
+
+
 def test_no_h2d_equals_resident(lib):
     cfg = synth.STACKS["8b"]
     res = _run(cfg, 3, 512, "resident")
