@@ -432,6 +432,7 @@ size_t lsn_nf4_blob_bytes(int64_t rows, int64_t cols) {
 size_t lsn_nf4_quantize_ws_bytes(int64_t rows, int64_t cols) { return quantize_ws_bytes(rows, cols); }
 
 lsn_status nf4_quantize(const float* W, const lsn_nf4_weight* out, void* ws, size_t ws_bytes, lsn_stream_t stream) {
+    NvtxRange nvtx("nf4_quantize");
     lsn_status s = check_nf4(out, "nf4_quantize");
     if (s != LSN_OK) return s;
     if (out->rows * out->cols == 0) return LSN_OK;
@@ -446,6 +447,7 @@ lsn_status nf4_quantize(const float* W, const lsn_nf4_weight* out, void* ws, siz
 }
 
 lsn_status nf4_dequant(const lsn_nf4_weight* w, uint16_t* W_out, lsn_stream_t stream) {
+    NvtxRange nvtx("nf4_dequant");
     lsn_status s = check_nf4(w, "nf4_dequant");
     if (s != LSN_OK) return s;
     if (w->rows * w->cols == 0) return LSN_OK;
@@ -456,6 +458,7 @@ lsn_status nf4_dequant(const lsn_nf4_weight* w, uint16_t* W_out, lsn_stream_t st
 
 lsn_status nf4_dequant_batch(int n, const lsn_nf4_weight* w, uint16_t* const* W_out, int blocks_per_sm,
                              lsn_stream_t stream) {
+    NvtxRange nvtx("nf4_dequant_batch");
     LSN_CHECK_ARG(n >= 0 && blocks_per_sm >= 0, "nf4_dequant_batch: n and blocks_per_sm must be >= 0");
     if (n == 0) return LSN_OK;
     LSN_CHECK_ARG(w != nullptr && W_out != nullptr, "nf4_dequant_batch: NULL array");
@@ -492,6 +495,7 @@ size_t lsn_lora_ws_bytes(int64_t T, int64_t K, int64_t N, int r, int kind) {
 
 lsn_status lora_linear_fwd(const lsn_base* W, const uint16_t* x, int64_t T, const uint16_t* A, const uint16_t* B, int r,
                            float scale, uint16_t* y, void* ws, size_t ws_bytes, lsn_stream_t stream) {
+    NvtxRange nvtx("lora_linear_fwd");
     lsn_status s = check_lora(W, x, T, A, B, r, ws, ws_bytes, "lora_linear_fwd");
     if (s != LSN_OK) return s;
     LSN_CHECK_ARG((y != nullptr || T == 0) && aligned16(y), "lora_linear_fwd: y must be a 16-byte aligned device pointer");
@@ -517,6 +521,7 @@ lsn_status lora_linear_fwd(const lsn_base* W, const uint16_t* x, int64_t T, cons
 lsn_status lora_linear_bwd(const lsn_base* W, const uint16_t* x, const uint16_t* dY, int64_t T, const uint16_t* A,
                            const uint16_t* B, int r, float scale, uint16_t* dX, float* dA, float* dB, int accumulate,
                            void* ws, size_t ws_bytes, lsn_stream_t stream) {
+    NvtxRange nvtx("lora_linear_bwd");
     lsn_status s = check_lora(W, x, T, A, B, r, ws, ws_bytes, "lora_linear_bwd");
     if (s != LSN_OK) return s;
     LSN_CHECK_ARG((dY != nullptr || T == 0) && aligned16(dY), "lora_linear_bwd: dY must be a 16-byte aligned device pointer");
@@ -582,6 +587,7 @@ lsn_status build_group_lb(const lsn_lora_proj* p, int i0, int m, int r, bool bwd
 
 lsn_status lora_layer_fwd(int n, const lsn_lora_proj* p, int64_t T, int r, float scale, void* ws, size_t ws_bytes,
                           lsn_stream_t stream) {
+    NvtxRange nvtx("lora_layer_fwd");
     lsn_status s = check_layer(n, p, T, r, ws, ws_bytes, false, "lora_layer_fwd");
     if (s != LSN_OK) return s;
     if (T == 0) return LSN_OK;
@@ -652,6 +658,7 @@ lsn_status lora_layer_fwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
 
 lsn_status lora_layer_bwd(int n, const lsn_lora_proj* p, int64_t T, int r, float scale, int accumulate, void* ws,
                           size_t ws_bytes, lsn_stream_t stream) {
+    NvtxRange nvtx("lora_layer_bwd");
     lsn_status s = check_layer(n, p, T, r, ws, ws_bytes, true, "lora_layer_bwd");
     if (s != LSN_OK) return s;
     if ((s = check_device()) != LSN_OK) return s;

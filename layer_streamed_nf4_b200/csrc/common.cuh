@@ -4,6 +4,7 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
 #include <string>
@@ -11,6 +12,16 @@
 #include "../../include/lsnf4.h"
 
 namespace lsn {
+
+// A named span on a profiler's timeline (NVTX), around a library call's
+// host-side work (argument checks and the launches it enqueues); nothing
+// happens unless a profiling tool is attached.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // ------------------------------------------------------------ host side ---
 

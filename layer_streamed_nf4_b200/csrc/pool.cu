@@ -87,6 +87,7 @@ int find_slot(lsn_pool* p, int layer) {
 }
 
 lsn_status start_copy(lsn_pool* p, int layer, int* slot_out) {
+    lsn::NvtxRange nvtx("layer_pool copy");
     auto it = p->blobs.find(layer);
     if (it == p->blobs.end()) return lsn::fail(LSN_ERR_INVALID_ARG, "layer " + std::to_string(layer) + " is not registered");
     int best = -1;
