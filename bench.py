@@ -445,7 +445,7 @@ def cpu_baseline(args, sample_rows: int, budget_s: float):
     from layer_streamed_nf4_b200 import synth
     cfg = synth.STACKS[WORKLOAD]
     L = cfg.layers
-    cores = os.cpu_count() or 1
+    cores = oracle.threads()                          # the threads its OpenMP loops actually use
     cases = _oracle_cases(sample_rows)
     work_all = sum(c.K * c.N for c, _ in cases)
     work_done = 0

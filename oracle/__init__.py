@@ -84,6 +84,8 @@ def _load():
     lib.orc_lora_fwd.argtypes = common + [_i64p, ctypes.c_int64, _f64p]
     lib.orc_lora_bwd_dx.argtypes = common + [_i64p, ctypes.c_int64, _f64p]
     lib.orc_lora_bwd_dadb.argtypes = common + [_f64p, _f64p]
+    lib.orc_threads.restype = ctypes.c_int
+    lib.orc_threads.argtypes = []
     _lib = lib
     return lib
 
@@ -94,6 +96,11 @@ def _p(a: np.ndarray, typ):
 
 
 # ----------------------------------------------------------------- codec ---
+
+def threads() -> int:
+    """Threads the oracle's OpenMP loops run on in this process."""
+    return int(_load().orc_threads())
+
 
 def ppnd16(p: float) -> float:
     return float(_load().orc_ppnd16(float(p)))

@@ -34,6 +34,8 @@
 // or sum, obtained here by computing in fp64 and rounding once, which is exact
 // for a single operation on fp32 operands); every matmul is accumulated in
 // fp64 from the exact bf16/fp32 input values.
+#include <omp.h>
+
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
@@ -344,5 +346,8 @@ void orc_lora_bwd_dadb(const uint16_t* x, const uint16_t* dY, const uint16_t* A,
             dB[n * r + j] = s * acc;
         }
 }
+
+// Threads the parallel loops above use (OpenMP's count for this process).
+int orc_threads() { return omp_get_max_threads(); }
 
 }  // extern "C"
