@@ -139,6 +139,35 @@ def test_struct_layouts_match_the_header(lib, tmp_path):
     assert got == want
 
 
+def test_a_c_program_links_and_calls_the_library(lib, tmp_path):
+    """The ABI from C alone: a program built against the header and linked to the .so calls the host-side
+    entry points (version, the NF4 levels, the blob layout, an argument error with its message)."""
+    import subprocess
+    src = tmp_path / "use.c"
+    src.write_text(
+        '#include <stdio.h>\n#include <stdlib.h>\n#include "lsnf4.h"\n'
+        "int main(void) {\n"
+        "  float lv[16]; size_t o[4];\n"
+        "  lsn_nf4_codebook(lv);\n"
+        "  lsn_nf4_blob_layout(4096, 14336, o);\n"
+        "  lsn_nf4_weight w = {64, 100, 0, 0, 0, 0};\n"
+        "  lsn_status st = nf4_dequant(&w, 0, 0);\n"
+        '  printf("%d %.9g %.9g %.9g %zu %zu %zu %zu %zu %d %s\\n", lsn_version(), lv[0], lv[7], lv[15],\n'
+        "         o[0], o[1], o[2], o[3], lsn_nf4_blob_bytes(4096, 14336), (int)st,\n"
+        '         lsn_last_error()[0] ? "message" : "empty");\n'
+        "  return 0;\n}\n")
+    exe = tmp_path / "use"
+    libdir = os.path.dirname(lib.lib_path())
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe), "-L", libdir, "-llsnf4",
+                    "-Wl,-rpath," + libdir], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
+    assert int(out[0]) == lib.version()
+    assert [float(v) for v in out[1:4]] == [-1.0, 0.0, 1.0]
+    assert [int(v) for v in out[4:8]] == lib.nf4_blob_layout(4096, 14336)
+    assert int(out[8]) == lib.nf4_blob_bytes(4096, 14336)
+    assert int(out[9]) == lib.LSN_ERR_INVALID_ARG and out[10] == "message"
+
+
 def _fake_projs(lib, shapes, kind):
     projs = []
     for K, N in shapes:
