@@ -19,6 +19,7 @@ from __future__ import annotations
 import argparse
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -153,6 +154,9 @@ class Replicas:
 
 # ----------------------------------------------------------------- ours ---
 
+# streamed[_S<slots>][_T<tokens>] and no_h2d_T<tokens>
+_POOL_MODE = re.compile(r"^(streamed|no_h2d)(?:_S(\d+))?(?:_T(\d+))?$")
+
 def run_ours(args):
     import torch
     from layer_streamed_nf4_b200 import lsnf4, synth
@@ -189,7 +193,7 @@ def run_ours(args):
     wanted = [m for m in args.modes.split(",") if m]
     modes = ["streamed"] + [m for m in wanted
                             if m in ("no_h2d", "resident", "proj", "dpo", "recompute", "shared", "grouped")
-                            or m.startswith("streamed_T") or m.startswith("streamed_S") or m.startswith("accum")]
+                            or _POOL_MODE.match(m) or m.startswith("accum")]
     mode_tokens = {m: T for m in modes}
     mode_copies = {}
     # Extra work of the step variants: the reference forward of preference
@@ -203,15 +207,21 @@ def run_ours(args):
             st = st_main
         elif mode == "proj":            # no_h2d through the per-projection calls on two lanes
             st = st_main.with_mode("no_h2d", lanes=2, api="proj")
-        elif mode.startswith("streamed_T"):   # the same stream of weights under a larger batch
-            mode_tokens[mode] = int(mode[len("streamed_T"):])
-            st = st_main.with_tokens(mode_tokens[mode], "streamed", n_slots=args.slots)
+        elif _POOL_MODE.match(mode) and mode not in ("no_h2d",):
+            # streamed_S<n>: the same stream of weights through a pool of n slots; _T<n>: under a batch of
+            # n tokens (its own activations); no_h2d_T<n>: the pre-filled pool under that batch
+            m = _POOL_MODE.match(mode)
+            pool_mode = m.group(1)
+            slots = int(m.group(2)) if m.group(2) else args.slots
+            if m.group(3):
+                mode_tokens[mode] = int(m.group(3))
+                st = st_main.with_tokens(mode_tokens[mode], pool_mode, n_slots=slots)
+            else:
+                st = st_main.with_mode(pool_mode, n_slots=slots)
         elif mode.startswith("accum"):        # n micro-batches of T tokens per step, gradients accumulated
             kw = {"micro": int(mode[len("accum"):])}
             mode_tokens[mode] = kw["micro"] * T
             st = st_main.with_mode("streamed", n_slots=args.slots)
-        elif mode.startswith("streamed_S"):   # the same stream of weights through a pool of n slots
-            st = st_main.with_mode("streamed", n_slots=int(mode[len("streamed_S"):]))
         elif mode in ("dpo", "recompute"):    # step variants over the same streamed pool
             st = st_main.with_mode("streamed", n_slots=args.slots)
         elif mode in ("shared", "grouped"):   # q|k|v and gate|up read one input each (no_h2d pool)
@@ -561,11 +571,12 @@ def main():
     ap.add_argument("--slots", type=int, default=20,
                     help="VRAM pool slots of the timed stream (default 20 of 32 layers: the smallest measured "
                          "window that hides the copies behind compute at 2048 tokens on one B200)")
-    ap.add_argument("--modes", default="no_h2d,resident,proj,streamed_S2,streamed_T8192,accum4,dpo,recompute,shared,"
-                                       "grouped",
+    ap.add_argument("--modes", default="no_h2d,resident,proj,streamed_S2,streamed_T8192,streamed_S2_T8192,"
+                                       "no_h2d_T8192,accum4,dpo,recompute,shared,grouped",
                     help="extra modes timed after the streamed one (streamed_T<n>: streamed with n tokens; "
-                         "streamed_S<n>: streamed through n pool slots; accum<n>: n micro-batches per step, "
-                         "gradients accumulated)")
+                         "streamed_S<n>: streamed through n pool slots; streamed_S<n>_T<m>: both; no_h2d_T<n>: "
+                         "the pre-filled pool with n tokens; accum<n>: n micro-batches per step, gradients "
+                         "accumulated)")
     ap.add_argument("--api", choices=["layer", "proj"], default="layer",
                     help="one library call per layer, or one per projection")
     ap.add_argument("--lanes", type=int, default=2, help="streams the seven projections of a layer are spread over")

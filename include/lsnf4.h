@@ -147,8 +147,10 @@ lsn_status nf4_quantize(const float* W, const lsn_nf4_weight* out, void* ws, siz
  * to nf4_quantize.
  *
  * The first call on a device looks up the array's device address (once per
- * device, with that device current); make that first call before any stream
- * capture.  All calls share the one array: calls whose work overlaps on the
+ * device, with that device current) and keeps it for the life of the process;
+ * make that first call before any stream capture.  A device reset
+ * (cudaDeviceReset) after that first call is not supported: the kept address
+ * would no longer name the array.  All calls share the one array: calls whose work overlaps on the
  * GPU (different streams without ordering between them) race and corrupt
  * each other's results -- order them on one stream or with events.  It calls
  * no cudaMalloc, cudaFree or allocating library routine. */
@@ -355,9 +357,12 @@ int lsn_get_option(int option);
  * pool copies registered host blobs (one per layer) into slots on its own copy
  * stream and orders copy and compute with events:
  *   ready[slot]     recorded on the copy stream after a layer's copy;
- *   released[slot]  recorded on the compute stream by layer_pool_release.
- * A copy into a slot always waits for that slot's released event, so a slot is
- * never overwritten while compute may still read it.  Forward sweeps prefetch
+ *   released        one event per layer_pool_release, recorded on the
+ *                   releasing stream.
+ * A copy into a slot waits for every release event of that slot recorded
+ * since its last fill, so a slot is never overwritten while any holder's
+ * compute may still read it (a layer acquired on two streams stays intact
+ * until both have released it, whichever releases first).  Forward sweeps prefetch
  * layer i+1 while layer i computes, backward sweeps layer i-1; with 2 slots a
  * fwd+bwd step reads 2L-4 layers in steady state (each layer twice, minus the
  * two still resident at each turn).  With S slots a sweep can keep S layers
@@ -399,8 +404,9 @@ lsn_status layer_pool_prefetch(lsn_pool* pool, int layer);
  * enqueued on `compute` until layer_pool_release. */
 lsn_status layer_pool_acquire(lsn_pool* pool, int layer, lsn_stream_t compute, void** dev_ptr);
 
-/* Record released[slot] on `compute`: the slot may be reused once the work
- * enqueued on `compute` before this call has finished. */
+/* Record a release event of the layer's slot on `compute`: this holder's
+ * claim ends once the work enqueued on `compute` before this call has
+ * finished; the slot may be reused when every holder's claim has ended. */
 lsn_status layer_pool_release(lsn_pool* pool, int layer, lsn_stream_t compute);
 
 /* Host-side bounded wait for every enqueued copy; LSN_ERR_TIMEOUT after

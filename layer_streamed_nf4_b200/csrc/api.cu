@@ -57,7 +57,7 @@ bool device_is_sm100() {
 
 using namespace lsn;
 
-namespace {
+namespace lsn {
 
 lsn_status check_device() {
     int dev = 0;
@@ -72,6 +72,8 @@ lsn_status check_nf4(const lsn_nf4_weight* w, const char* who) {
     LSN_CHECK_ARG(w != nullptr, f + ": weight is NULL");
     LSN_CHECK_ARG(w->rows >= 0 && w->cols >= 0, f + ": negative shape");
     LSN_CHECK_ARG(w->cols % 64 == 0, f + ": cols must be a multiple of 64");
+    // rows * cols is formed only once it is known to fit (at most 2^46 elements).
+    LSN_CHECK_ARG(w->cols == 0 || w->rows <= kMaxNf4Elems / w->cols, f + ": rows * cols too large");
     if (w->rows * w->cols == 0) return LSN_OK;
     LSN_CHECK_ARG(w->packed && w->absmax_q && w->absmax_s2 && w->offset, f + ": NULL array in the NF4 weight");
     LSN_CHECK_ARG(aligned16(w->packed), f + ": packed must be 16-byte aligned");
@@ -79,6 +81,10 @@ lsn_status check_nf4(const lsn_nf4_weight* w, const char* who) {
                   f + ": absmax_s2/offset must be 4-byte aligned");
     return LSN_OK;
 }
+
+}  // namespace lsn
+
+namespace {
 
 // Workspace layout of the LoRA calls (each region 256-byte aligned):
 //   [0, 256)  status word of the GEMM kernels

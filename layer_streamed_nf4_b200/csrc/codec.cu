@@ -21,6 +21,7 @@
 
 #include "common.cuh"
 #include "launch.cuh"
+#include "timing.cuh"
 
 namespace lsn {
 
@@ -425,22 +426,21 @@ lsn_status noalloc_scratch(void** out) {
 
 extern "C" lsn_status nf4_quantize_noalloc(const float* W, const lsn_nf4_weight* out, lsn_stream_t stream) {
     using namespace lsn;
-    LSN_CHECK_ARG(out != nullptr, "nf4_quantize_noalloc: weight is NULL");
-    LSN_CHECK_ARG(out->rows >= 0 && out->cols >= 0, "nf4_quantize_noalloc: negative shape");
-    LSN_CHECK_ARG(out->cols % 64 == 0, "nf4_quantize_noalloc: cols must be a multiple of 64");
+    NvtxRange nvtx("nf4_quantize_noalloc");
+    lsn_status s = check_nf4(out, "nf4_quantize_noalloc");
+    if (s != LSN_OK) return s;
+    // The limit is tested by division, before rows * cols is formed.
+    LSN_CHECK_ARG(out->cols == 0 || out->rows <= kNoAllocMaxElems / out->cols,
+                  "nf4_quantize_noalloc: rows*cols = " + std::to_string(out->rows) + "*" + std::to_string(out->cols) +
+                      " exceeds the fixed scratch limit of " + std::to_string(kNoAllocMaxElems) +
+                      " elements; use nf4_quantize with a caller workspace");
     const int64_t numel = out->rows * out->cols;
     if (numel == 0) return LSN_OK;
-    LSN_CHECK_ARG(numel <= kNoAllocMaxElems,
-                  "nf4_quantize_noalloc: rows*cols = " + std::to_string(numel) + " exceeds the fixed scratch limit of " +
-                      std::to_string(kNoAllocMaxElems) + " elements; use nf4_quantize with a caller workspace");
     LSN_CHECK_ARG(W != nullptr && aligned16(W), "nf4_quantize_noalloc: W must be a 16-byte aligned device pointer");
-    LSN_CHECK_ARG(out->packed && out->absmax_q && out->absmax_s2 && out->offset,
-                  "nf4_quantize_noalloc: NULL array in the NF4 weight");
-    LSN_CHECK_ARG(aligned16(out->packed), "nf4_quantize_noalloc: packed must be 16-byte aligned");
-    if (!device_is_sm100()) return fail(LSN_ERR_UNSUPPORTED, "liblsnf4 is built for sm_100a (B200) only");
+    if ((s = check_device()) != LSN_OK) return s;
     void* scratch = nullptr;
-    lsn_status s = noalloc_scratch(&scratch);
-    if (s != LSN_OK) return s;
+    if ((s = noalloc_scratch(&scratch)) != LSN_OK) return s;
+    const double n = (double)numel;
+    TimingScope ts(LSN_K_QUANTIZE, n * 4.0 + n / 2.0 + n / 64.0 * 6.0, reinterpret_cast<cudaStream_t>(stream), 4);
     return launch_quantize(W, out, scratch, kNoAllocScratchBytes, reinterpret_cast<cudaStream_t>(stream));
 }
-

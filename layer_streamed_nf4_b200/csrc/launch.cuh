@@ -42,6 +42,13 @@ inline int pdl_attr(cudaLaunchAttribute* a) {
     return 1;
 }
 
+// Argument checks shared by the entry points (api.cu): the current device is
+// an sm_100 part; an NF4 weight descriptor is well formed (shape, arrays,
+// alignment, rows * cols <= kMaxNf4Elems checked without overflow).
+constexpr int64_t kMaxNf4Elems = (int64_t)1 << 46;
+lsn_status check_device();
+lsn_status check_nf4(const lsn_nf4_weight* w, const char* who);
+
 size_t quantize_ws_bytes(int64_t rows, int64_t cols);
 lsn_status launch_quantize(const float* W, const lsn_nf4_weight* out, void* ws, size_t ws_bytes, cudaStream_t st);
 lsn_status launch_dequant(const lsn_nf4_weight* w, uint16_t* out, cudaStream_t st);

@@ -10,8 +10,11 @@
 // frozen weights are just data") adds that the buffers are pre-allocated.
 // The abstract of "Exact Layer Streaming" reports the failure mode this
 // design rules out: gradients silently wrong through aliasing.  Here a slot
-// is only ever overwritten after the compute stream has recorded its release
-// event, and the copy stream waits on that event before the copy.
+// is only ever overwritten after every holder has released it: each release
+// records an event of its own on the releasing stream, and the copy stream
+// waits on all the events recorded since the slot's last fill before the
+// copy (a layer acquired on two streams is safe from the reader that releases
+// first).
 #include <chrono>
 #include <mutex>
 #include <thread>
@@ -28,7 +31,7 @@ struct Slot {
     int layer = -1;          // layer held (or being copied), -1 if none
     int refs = 0;            // acquire count not yet released
     bool pending = false;    // prefetched, not yet acquired: not evictable
-    bool released_once = false;
+    int n_rel = 0;           // release events recorded since the slot's last fill
     uint64_t last_release = 0;
     uint64_t last_fill = 0;
 };
@@ -41,7 +44,10 @@ struct lsn_pool {
     size_t slot_bytes = 0, slot_stride = 0;
     uint8_t* dev = nullptr;
     cudaStream_t copy = nullptr;
-    std::vector<cudaEvent_t> ready, released;
+    std::vector<cudaEvent_t> ready;
+    // Per slot, one event per release since the slot's last fill (the vector
+    // grows to the largest number of holders a slot has had at once).
+    std::vector<std::vector<cudaEvent_t>> released;
     std::vector<Slot> slots;
     std::unordered_map<int, std::pair<const void*, size_t>> blobs;
     cudaEvent_t t0[kTimingRing] = {}, t1[kTimingRing] = {};
@@ -105,7 +111,8 @@ lsn_status start_copy(lsn_pool* p, int layer, int* slot_out) {
     }
     Slot& sl = p->slots[best];
     uint8_t* dst = p->dev + (size_t)best * p->slot_stride;
-    if (sl.released_once) LSN_CUDA_TRY(cudaStreamWaitEvent(p->copy, p->released[best], 0));
+    for (int i = 0; i < sl.n_rel; ++i) LSN_CUDA_TRY(cudaStreamWaitEvent(p->copy, p->released[best][i], 0));
+    sl.n_rel = 0;
     if (p->timing_live == kTimingRing) harvest_timing(p, true);
     const int ti = p->timing_next;
     LSN_CUDA_TRY(cudaEventRecord(p->t0[ti], p->copy));
@@ -131,7 +138,8 @@ lsn_status start_copy(lsn_pool* p, int layer, int* slot_out) {
 void destroy_resources(lsn_pool* p) {
     if (p->copy) cudaStreamSynchronize(p->copy);
     for (auto e : p->ready) if (e) cudaEventDestroy(e);
-    for (auto e : p->released) if (e) cudaEventDestroy(e);
+    for (auto& v : p->released)
+        for (auto e : v) if (e) cudaEventDestroy(e);
     for (int i = 0; i < kTimingRing; ++i) {
         if (p->t0[i]) cudaEventDestroy(p->t0[i]);
         if (p->t1[i]) cudaEventDestroy(p->t1[i]);
@@ -168,10 +176,12 @@ lsn_status layer_pool_create(int n_slots, size_t slot_bytes, int device, lsn_poo
     }
     bool ok = cudaStreamCreateWithFlags(&p->copy, cudaStreamNonBlocking) == cudaSuccess;
     p->ready.assign(n_slots, nullptr);
-    p->released.assign(n_slots, nullptr);
-    for (int s = 0; ok && s < n_slots; ++s)
+    p->released.assign(n_slots, {});
+    for (int s = 0; ok && s < n_slots; ++s) {
+        p->released[s].push_back(nullptr);
         ok = cudaEventCreateWithFlags(&p->ready[s], cudaEventDisableTiming) == cudaSuccess &&
-             cudaEventCreateWithFlags(&p->released[s], cudaEventDisableTiming) == cudaSuccess;
+             cudaEventCreateWithFlags(&p->released[s][0], cudaEventDisableTiming) == cudaSuccess;
+    }
     for (int i = 0; ok && i < kTimingRing; ++i)
         ok = cudaEventCreate(&p->t0[i]) == cudaSuccess && cudaEventCreate(&p->t1[i]) == cudaSuccess;
     if (!ok) {
@@ -249,12 +259,18 @@ lsn_status layer_pool_release(lsn_pool* p, int layer, lsn_stream_t compute) {
     if (it == p->held.end() || it->second.empty())
         return lsn::fail(LSN_ERR_STATE, "layer_pool_release: layer " + std::to_string(layer) + " is not acquired");
     const int s = it->second.back();
-    it->second.pop_back();
     DeviceGuard g(p->device);
-    LSN_CUDA_TRY(cudaEventRecord(p->released[s], reinterpret_cast<cudaStream_t>(compute)));
     Slot& sl = p->slots[s];
+    std::vector<cudaEvent_t>& ev = p->released[s];
+    if (sl.n_rel == (int)ev.size()) {               // more holders than ever before: one more event
+        cudaEvent_t e = nullptr;
+        LSN_CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+        ev.push_back(e);
+    }
+    LSN_CUDA_TRY(cudaEventRecord(ev[sl.n_rel], reinterpret_cast<cudaStream_t>(compute)));
+    it->second.pop_back();
+    sl.n_rel += 1;
     sl.refs -= 1;
-    sl.released_once = true;
     sl.last_release = ++p->tick;
     return LSN_OK;
 }

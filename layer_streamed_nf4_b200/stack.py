@@ -512,14 +512,19 @@ class Stack:
             call(l, b)
             self._ev_done[b].record(self.stream)
 
-    def _forward_layers(self, adapter: bool = True):
+    def _forward_layers(self, adapter: bool = True, reference: bool = False):
+        """Forward sweep through the layer calls.  reference: each layer runs twice while it is held, first
+        with the adapters off (the reference model's forward, into y_ref), then with them on: two
+        independent forward passes sharing one read of the layer stream."""
         fwd = lsnf4._lib.lora_layer_fwd
         n, ws, nb, sp = len(self.proj), self.ws[0].data_ptr(), self.ws_bytes, self.stream.cuda_stream
+        passes = (False, True) if reference else (adapter,)
         if self.ahead:
             def call(l, b):
-                st = fwd(n, self._layer_projs(0, l, adapter, wb=b), self.T, self.r, self.scale, ws, nb, sp)
-                if st:
-                    lsnf4._check(st, "lora_layer_fwd")
+                for ad in passes:
+                    st = fwd(n, self._layer_projs(0, l, ad, wb=b), self.T, self.r, self.scale, ws, nb, sp)
+                    if st:
+                        lsnf4._check(st, "lora_layer_fwd")
             return self._sweep_ahead(range(self.L), call)
         order = list(range(self.L))
         fill = self._window(order)
@@ -527,9 +532,10 @@ class Stack:
         for j, l in enumerate(order):
             addr = self._acquire(l)
             fill(j + self.n_slots - 1)
-            st = fwd(n, self._layer_projs(addr, l, adapter), self.T, self.r, self.scale, ws, nb, sp)
-            if st:
-                lsnf4._check(st, "lora_layer_fwd")
+            for ad in passes:
+                st = fwd(n, self._layer_projs(addr, l, ad), self.T, self.r, self.scale, ws, nb, sp)
+                if st:
+                    lsnf4._check(st, "lora_layer_fwd")
             self._release(l)
 
     def _backward_layers(self, accumulate: bool, recompute: bool = False):
@@ -562,10 +568,10 @@ class Stack:
                 lsnf4._check(st, "lora_layer_bwd")
             self._release(l)
 
-    def forward(self, adapter: bool = True):
+    def forward(self, adapter: bool = True, reference: bool = False):
         if self.api == "layer":
-            return self._forward_layers(adapter)
-        assert adapter, "the adapter-off forward runs through the layer calls"
+            return self._forward_layers(adapter, reference)
+        assert adapter and not reference, "the adapter-off forward runs through the layer calls"
         fwd = lsnf4._lib.lora_linear_fwd
         order = list(range(self.L))
         fill = self._window(order)
@@ -601,12 +607,11 @@ class Stack:
             self._release(l)
 
     def step(self, accumulate: bool = False, reference: bool = False, recompute: bool = False):
-        """One training step.  reference: first a forward sweep with the adapters off (the reference model
-        of preference training, read from the same stream of layers); recompute: every layer's forward runs
-        again inside the backward sweep, as with activation checkpointing."""
-        if reference:
-            self.forward(adapter=False)
-        self.forward()
+        """One training step.  reference: the forward sweep also runs every layer with the adapters off (the
+        reference model of preference training, on the same stream of layers: each layer is read once for
+        both forwards, so the step copies as many layers as a plain one); recompute: every layer's forward
+        runs again inside the backward sweep, as with activation checkpointing."""
+        self.forward(reference=reference)
         self.backward(accumulate, recompute)
 
     # ------------------------------------------------------------ facts ---

@@ -242,3 +242,38 @@ def test_dequant_batch_rejects_bad_arguments(lib):
         lib.nf4_dequant_batch([w, bad], [1 << 20, 1 << 21], stream=0)
     assert e.value.status == lib.LSN_ERR_INVALID_ARG
     lib.nf4_dequant_batch([], [], stream=0)                      # nothing to do
+
+
+def test_huge_nf4_shapes_are_rejected_without_overflow(lib):
+    """rows * cols is never formed before it is known to fit: shapes whose product overflows int64 (or
+    exceeds the library's element limit) are argument errors for the codec calls, the allocation-free one
+    included, and nothing is launched."""
+    for rows, cols in ((1 << 40, 1 << 40), ((1 << 62) // 64, 128), ((1 << 46) // 64 + 1, 64)):
+        w = lib.make_nf4_weight(rows, cols, 1 << 20, 1 << 20, 1 << 20, 1 << 20)
+        for call in (lambda: lib.nf4_dequant(w, 1 << 20, stream=0),
+                     lambda: lib.nf4_quantize(1 << 20, w, 1 << 20, 1 << 40, stream=0),
+                     lambda: lib.nf4_quantize_noalloc(1 << 20, w, stream=0)):
+            with pytest.raises(lib.LsnError) as e:
+                call()
+            assert e.value.status == lib.LSN_ERR_INVALID_ARG
+            assert "too large" in str(e.value)
+
+
+def test_noalloc_checks_its_arguments_like_the_workspace_version(lib):
+    """nf4_quantize_noalloc applies the same descriptor checks as nf4_quantize (NULL arrays, 16-byte packed,
+    4-byte constants) and its element limit, all before any device work."""
+    bad = [lib.make_nf4_weight(64, 128, None, 1 << 20, 1 << 20, 1 << 20),          # NULL packed
+           lib.make_nf4_weight(64, 128, (1 << 20) + 8, 1 << 20, 1 << 20, 1 << 20),  # packed not 16-byte aligned
+           lib.make_nf4_weight(64, 128, 1 << 20, 1 << 20, (1 << 20) + 2, 1 << 20),  # s2 not 4-byte aligned
+           lib.make_nf4_weight(64, 128, 1 << 20, 1 << 20, 1 << 20, (1 << 20) + 1),  # offset not 4-byte aligned
+           lib.make_nf4_weight(64, 100, 1 << 20, 1 << 20, 1 << 20, 1 << 20)]        # cols % 64 != 0
+    for w in bad:
+        for call in (lambda: lib.nf4_quantize(1 << 20, w, 1 << 20, 1 << 30, stream=0),
+                     lambda: lib.nf4_quantize_noalloc(1 << 20, w, stream=0)):
+            with pytest.raises(lib.LsnError) as e:
+                call()
+            assert e.value.status == lib.LSN_ERR_INVALID_ARG
+    over = lib.make_nf4_weight(lib.NF4_NOALLOC_MAX_ELEMS // 4096 + 1, 4096, 1 << 20, 1 << 20, 1 << 20, 1 << 20)
+    with pytest.raises(lib.LsnError) as e:
+        lib.nf4_quantize_noalloc(1 << 20, over, stream=0)
+    assert e.value.status == lib.LSN_ERR_INVALID_ARG and "limit" in str(e.value)

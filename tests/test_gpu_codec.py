@@ -95,3 +95,23 @@ def test_dequant_batch_equals_single_calls():
         torch.cuda.synchronize()
         for a, b in zip(singles, outs):
             assert torch.equal(a, b), bps
+
+
+def test_codec_bit_exact_at_first_level_ties(lib, orc):
+    """Blocks whose w / absmax fall exactly on the midpoints between adjacent levels (absmax a power of two)
+    and one or two fp32 steps either side, at four scales: the GPU's thresholds decide every one of them
+    as the oracle's exact nearest-level rule does (ties to the lower index)."""
+    from tests.helpers import first_level_tie_weights
+    W = first_level_tie_weights(orc.nf4_codebook())
+    assert W.shape[0] % 2 == 0
+    _check_codec(lib, orc, W.reshape(-1, 128))          # blocks run along the flattened rows
+
+
+@pytest.mark.parametrize("off_exp,s2_exp,m_lo,m_hi", [(-12, -5, -1.0 / 128, 1.0), (-5, -5, -1.0, -0.5)])
+def test_codec_bit_exact_at_second_level_ties(lib, orc, off_exp, s2_exp, m_lo, m_hi):
+    """Weights whose second-level values (absmax - offset) / s2 fall exactly on the midpoints of adjacent
+    entries of the k/127 table, and one or two fp32 steps either side (over a hundred exact ties on the
+    positive side, sixty on the negative): codes, s2, offset and dequantised bf16 equal the oracle's."""
+    from tests.helpers import second_level_tie_weights
+    W, _, _ = second_level_tie_weights(orc.dq_table()[:255], off_exp, s2_exp, m_lo, m_hi)
+    _check_codec(lib, orc, W.reshape(-1, 256))

@@ -48,8 +48,8 @@ def _compare(a, b):
     return fwd, bwd, bad
 
 
-@pytest.mark.parametrize("name,layers,tokens,fused", [("0.5b", 24, 512, 0), ("3b", 4, 1024, 0), ("8b", 4, 2048, 0),
-                                                     ("8b", 3, 2048, 1), ("72b", 3, 1024, 0)])
+@pytest.mark.parametrize("name,layers,tokens,fused", [("0.5b", 24, 512, 0), ("8b", 4, 2048, 0), ("8b", 3, 2048, 1),
+                                                     ("72b", 3, 1024, 0)])
 def test_streamed_equals_resident(lib, name, layers, tokens, fused):
     lib.set_option(lib.LSN_OPT_FUSED_NF4, fused)
     try:
@@ -88,11 +88,30 @@ def test_lane_count_does_not_change_results(lib, name, layers, tokens):
     one.close()
 
 
-def test_recompute_and_reference_steps(lib):
-    """A backward that recomputes each layer's forward, and a step that first runs the adapter-off
-    reference forward, give the same y, dX, dA, dB as the plain step; the reference outputs are the
-    base term (equal to an adapter-on forward with B = 0)."""
+def _oracle_weight(orc, st, l, pi):
+    """The oracle's dequantised bf16 bits of projection pi of layer l: the stack's fp32 weight regenerated
+    from its seed, quantised and dequantised by the oracle itself."""
+    p = st.proj[pi]
+    W = synth.device_normal((p.N, p.K), 0.02, st.seed, l, pi, synth.T_W, device=st.dev).cpu().numpy()
+    q = orc.nf4_quantize(W)
+    return orc.nf4_dequant(q["packed"], q["absmax_q"], q["s2"], q["offset"], W.size).reshape(W.shape)
+
+
+def _bits(t):
+    import numpy as np
     import torch
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def test_recompute_and_reference_steps(lib, orc):
+    """A backward that recomputes each layer's forward, and a step that first runs the adapter-off
+    reference forward, give the same y, dX, dA, dB as the plain step, and match the oracle: the
+    recomputing step's dA, dB (in full) and dX (sampled token rows), and the reference forward's y
+    against the oracle's plain x W^T.  The reference outputs are also the base term bit for bit (equal to
+    an adapter-on forward with B = 0)."""
+    import numpy as np
+    import torch
+    from tests.helpers import assert_close, bf16_tensor_to_f64
     cfg = synth.STACKS["8b"]
     plain = _run(cfg, 3, 256, "streamed")
     from layer_streamed_nf4_b200.stack import Stack
@@ -100,8 +119,21 @@ def test_recompute_and_reference_steps(lib):
     st.step(reference=True, recompute=True)
     torch.cuda.synchronize()
     st.check_status()
+    assert st.pool_stats()["copies"] == 2 * 3 - 2        # the reference forward reads no layer of its own
     fwd, bwd, bad = _compare(st, plain)
     assert fwd and bwd, bad
+    rows = np.sort(np.random.default_rng(31).choice(256, size=24, replace=False))
+    for l in range(3):
+        for pi in (0, 2, 6):                                  # q, v, down
+            Wb = _oracle_weight(orc, st, l, pi)
+            x, dY, A, B = _bits(st.x[l, pi]), _bits(st.dY[l, pi]), _bits(st.A[l, pi]), _bits(st.B[l, pi])
+            rA, rB = orc.lora_bwd_dadb(x, dY, A, B, st.scale)
+            assert_close(st.dA[l, pi].cpu().numpy(), rA, f"recompute dA {l},{pi}")
+            assert_close(st.dB[l, pi].cpu().numpy(), rB, f"recompute dB {l},{pi}")
+            assert_close(bf16_tensor_to_f64(st.dX[l, pi])[rows], orc.lora_bwd_dx(dY, Wb, A, B, st.scale, rows=rows),
+                         f"recompute dX {l},{pi}")
+            base = orc.lora_fwd(x, Wb, A, np.zeros_like(B), st.scale, rows=rows)      # x W^T alone
+            assert_close(bf16_tensor_to_f64(st.y_ref[l, pi])[rows], base, f"reference y {l},{pi}")
     for k in st.B:
         st.B[k].zero_()
     st.forward()
@@ -335,11 +367,14 @@ def test_slot_window_copies_and_bits(lib, slots, ahead, api):
     st.close()
 
 
-def test_grouped_stack_matches_shared_inputs(lib):
+def test_grouped_stack_matches_shared_inputs(lib, orc):
     """A stack whose q|k|v and gate|up run as groups gives the same y, dA and dB as the same stack run
-    ungrouped, streamed or resident; the grouped dX equals the ungrouped sum within bf16 rounding."""
+    ungrouped, streamed or resident; the grouped dX (the group's summed input gradient) equals the
+    ungrouped sum within bf16 rounding and the oracle's sum of the members' dX on sampled token rows."""
+    import numpy as np
     import torch
     from layer_streamed_nf4_b200.stack import Stack
+    from tests.helpers import assert_close, bf16_tensor_to_f64
     cfg = synth.STACKS["8b"]
     shared = Stack(cfg, layers=2, tokens=512, mode="resident", keep_outputs=True, shared_inputs=True)
     shared.step()
@@ -349,12 +384,17 @@ def test_grouped_stack_matches_shared_inputs(lib):
     grouped.check_status()
     assert all(torch.equal(shared.y[k], grouped.y[k]) for k in shared.y)
     assert all(torch.equal(shared.dA[k], grouped.dA[k]) and torch.equal(shared.dB[k], grouped.dB[k]) for k in shared.dA)
+    rows = np.sort(np.random.default_rng(32).choice(512, size=16, replace=False))
     for l in range(2):
         for members in ((0, 1, 2), (4, 5)):
             ref = sum(shared.dX[l, pi].double() for pi in members)
             got = grouped.dX[l, members[0]].double()
             err = float((got - ref).norm() / ref.norm())
             assert err < 5e-3, (l, members, err)
+            want = sum(orc.lora_bwd_dx(_bits(grouped.dY[l, pi]), _oracle_weight(orc, grouped, l, pi),
+                                       _bits(grouped.A[l, pi]), _bits(grouped.B[l, pi]), grouped.scale, rows=rows)
+                       for pi in members)
+            assert_close(bf16_tensor_to_f64(grouped.dX[l, members[0]])[rows], want, f"grouped dX {l},{members}")
     grouped.close()
 
 
@@ -388,3 +428,50 @@ def test_full_size_stack_against_oracle(lib, orc):
         assert_close(st.dA[0, pi].cpu().numpy(), rA, f"{p.name} dA")
         assert_close(st.dB[0, pi].cpu().numpy(), rB, f"{p.name} dB")
     st.close()
+
+
+def test_two_holders_keep_the_slot_until_both_release(lib):
+    """A layer acquired on two streams: the reader with the long queue releases first, the other second,
+    then a copy of another layer is started into the (only) slot.  The copy must wait for both releases,
+    so the long reader still sees the first layer's codes (poison mode on: a premature copy would show
+    the 0xFF sentinel or the second layer)."""
+    import torch
+    from tests.helpers import DeviceNF4
+    rows, cols = 256, 4096
+    ws = [DeviceNF4(rows, cols).quantize(synth.normal_f32((rows, cols), 0.02, synth.SEED, 500, i, synth.T_W))
+          for i in range(2)]
+    torch.cuda.synchronize()
+    nbytes = ws[0].blob.numel()
+    hosts = [d.blob.cpu().pin_memory() for d in ws]
+    ref = torch.empty((rows, cols), dtype=torch.bfloat16, device="cuda")
+    lib.nf4_dequant(ws[0].w, ref)
+    pool = lib.layer_pool_create(1, nbytes, 0)
+    try:
+        lib.layer_pool_set_debug(pool, lib.LSN_POOL_DEBUG_POISON)
+        for i, h in enumerate(hosts):
+            lib.layer_pool_register(pool, i, h.data_ptr(), nbytes)
+        a, b = torch.cuda.Stream(), torch.cuda.Stream()
+        out = torch.zeros((rows, cols), dtype=torch.bfloat16, device="cuda")
+        pa = lib.layer_pool_acquire(pool, 0, a)
+        pb = lib.layer_pool_acquire(pool, 0, b)
+        assert pa == pb                                   # one slot, two holders
+        with torch.cuda.stream(a):
+            torch.cuda._sleep(200_000_000)                # a long queue ahead of the reader (bounded spin)
+        w = lib.nf4_weight_in_blob(rows, cols, pa)
+        lib.nf4_dequant(w, out, a)                        # reads the slot after the spin
+        lib.layer_pool_release(pool, 0, a)                # the long reader releases first
+        lib.layer_pool_release(pool, 0, b)                # the idle holder second
+        lib.layer_pool_prefetch(pool, 1)                  # takes the slot: must wait for both
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref), "the slot was overwritten while a holder still read it"
+        p1 = lib.layer_pool_acquire(pool, 1, b)
+        w1 = lib.nf4_weight_in_blob(rows, cols, p1)
+        lib.nf4_dequant(w1, out, b)
+        lib.layer_pool_release(pool, 1, b)
+        want = torch.empty_like(ref)
+        lib.nf4_dequant(ws[1].w, want)
+        torch.cuda.synchronize()
+        assert torch.equal(out, want)                     # and the copy did land afterwards
+        lib.layer_pool_wait_idle(pool, 10000)
+    finally:
+        lib.layer_pool_destroy(pool)

@@ -243,3 +243,118 @@ def test_quantize_brute_force_tiny(orc):
         for j in range(0, cb.size, 9):
             v = np.float32(cb[j] / s2)
             assert q["absmax_q"][g * 256 + j] == _exact_nearest(v, t)
+
+
+def _bf16_rne_torch(x32: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns of fp32 values, rounded to nearest even by torch (a library conversion)."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(x32, np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def test_dequant_exact_at_second_level_points(orc):
+    """Second level with s2 != 0, closed form: every block is level points times its absmax, the absmax
+    values of a group sit at offset - d, offset and offset + d (d differs per group, one group is ragged),
+    so the second-level values are exactly -1, 0, +1 (codes 0, 127, 254) and absmax_hat equals the absmax.
+    Then dequantisation must give bf16(w) for every element, whatever the group: a wrong s2 index, a
+    wrong table entry or a dropped offset changes absmax_hat and breaks the equality."""
+    c = orc.nf4_codebook()
+    rng = np.random.default_rng(21)
+    off = 2.0 ** -5
+    ds = [2.0 ** -7, 2.0 ** -6, 3 * 2.0 ** -8, 2.0 ** -8]
+    sizes = [256, 256, 256, 100]                         # the last group is ragged
+    absmax = []
+    for d, n in zip(ds, sizes):
+        pattern = np.resize([off - d, off + d, off, off + d, off - d, off], n)
+        if pattern.sum() != n * off:                     # keep each group's mean exactly off
+            pattern[-1] = off
+        absmax += list(pattern)
+    absmax = np.array(absmax, np.float32)
+    assert float(np.sum(absmax.astype(np.float64))) == off * absmax.size
+    nblk = absmax.size
+    idx = rng.integers(0, 16, size=(nblk, 64))
+    idx[np.arange(nblk), rng.integers(0, 64, size=nblk)] = rng.choice([0, 15], size=nblk)
+    W = (c[idx].astype(np.float32) * absmax[:, None]).astype(np.float32)
+    q = orc.nf4_quantize(W, want_absmax=True)
+    assert q["offset"] == np.float32(off)
+    assert np.array_equal(q["s2"], np.array(ds, np.float32))
+    assert set(np.unique(q["absmax_q"])) <= {0, 127, 254} and len(set(np.unique(q["absmax_q"]))) == 3
+    codes = np.stack([q["packed"] >> 4, q["packed"] & 15], axis=1).reshape(-1)
+    assert np.array_equal(codes, idx.reshape(-1))
+    deq = orc.nf4_dequant(q["packed"], q["absmax_q"], q["s2"], q["offset"], W.size)
+    assert np.array_equal(deq, _bf16_rne_torch(W.reshape(-1)))
+
+
+def test_dequant_second_level_random_groups(orc):
+    """Second level with s2 != 0 on N(0, 0.02) weights whose groups have very different absmax spreads:
+    (i) every element equals bf16(level[q] * absmax_hat) with absmax_hat rebuilt in numpy fp32 from the
+    stored code, its group's s2 and the offset; (ii) every element lies within the format's error bound of
+    the original weight: half the widest gap between adjacent levels times the block absmax, plus the
+    level times half a second-level step (s2/254), plus bf16 rounding."""
+    c = orc.nf4_codebook()
+    tab = orc.dq_table()
+    rng = np.random.default_rng(22)
+    spreads = [1.0, 6.0, 0.2, 2.5, 1.0]
+    W = np.concatenate([rng.normal(0, 0.02, size=(256 * 64,)) * s for s in spreads]).astype(np.float32)
+    W = W[:W.size - 64 * 37]                             # a ragged last group
+    q = orc.nf4_quantize(W, want_absmax=True)
+    assert np.all(q["s2"] > 0) and q["s2"].max() > 3 * q["s2"].min() and len(set(q["s2"].tolist())) == q["s2"].size
+    deq = orc.nf4_dequant(q["packed"], q["absmax_q"], q["s2"], q["offset"], W.size)
+    nblk = W.size // 64
+    blk = np.arange(nblk)
+    ah = (tab[q["absmax_q"]] * q["s2"][blk // 256]).astype(np.float32) + np.float32(q["offset"])
+    ah = ah.astype(np.float32)
+    codes = np.stack([q["packed"] >> 4, q["packed"] & 15], axis=1).reshape(-1)
+    want = _bf16_rne_torch((c[codes].reshape(nblk, 64) * ah[:, None]).astype(np.float32).reshape(-1))
+    assert np.array_equal(deq, want)
+    got = (deq.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    half_gap = float(np.max(np.diff(c.astype(np.float64)))) / 2
+    a = np.repeat(q["absmax"].astype(np.float64), 64)
+    s2 = np.repeat(q["s2"][blk // 256].astype(np.float64), 64)
+    bound = half_gap * a + np.abs(c[codes].astype(np.float64)) * s2 / 254 * (1 + 1e-5) + 2.0 ** -8 * np.abs(got) + 1e-9
+    assert np.all(np.abs(got - W.astype(np.float64)) <= bound)
+
+
+def test_first_level_ties_constructed(orc):
+    """Weights built on the exact midpoints between adjacent levels (absmax a power of two, so w / absmax is
+    the midpoint itself) and one or two fp32 steps either side: the oracle's codes equal the exact nearest
+    level with ties to the lower index."""
+    from tests.helpers import first_level_tie_weights
+    c = orc.nf4_codebook()
+    W = first_level_tie_weights(c)
+    q = orc.nf4_quantize(W, want_absmax=True)
+    codes = np.stack([q["packed"] >> 4, q["packed"] & 15], axis=1).reshape(W.shape)
+    ties = 0
+    for b in range(W.shape[0]):
+        a = q["absmax"][b]
+        assert a == np.abs(W[b]).max() and np.log2(a) == int(np.log2(a))
+        for i in range(64):
+            v = np.float32(W[b, i] / a)
+            assert codes[b, i] == _exact_nearest(v, c), (b, i, float(v))
+            for k in range(15):
+                if Fraction(float(v)) == (Fraction(float(c[k])) + Fraction(float(c[k + 1]))) / 2:
+                    ties += 1
+                    assert codes[b, i] == k
+    assert ties > 0
+
+
+@pytest.mark.parametrize("off_exp,s2_exp,m_lo,m_hi", [(-12, -5, -1.0 / 128, 1.0), (-5, -5, -1.0, -0.5)])
+def test_second_level_ties_constructed(orc, off_exp, s2_exp, m_lo, m_hi):
+    """Weights whose second-level values land exactly on the midpoints of adjacent entries of the k/127
+    table (and one or two fp32 steps either side): the offset comes out exactly 2^off_exp, every tie group
+    has s2 = 2^s2_exp, and each block's code is the exact nearest entry with ties to the lower index."""
+    from tests.helpers import second_level_tie_weights
+    tab = orc.dq_table()[:255]
+    W, n_groups, where = second_level_tie_weights(tab, off_exp, s2_exp, m_lo, m_hi)
+    q = orc.nf4_quantize(W, want_absmax=True)
+    assert q["offset"] == np.float32(2.0 ** off_exp)
+    assert np.all(q["s2"][:n_groups] == np.float32(2.0 ** s2_exp))
+    ties = 0
+    for b, v in where:
+        got_v = np.float32((np.float32(q["absmax"][b]) - q["offset"]) / q["s2"][b // 256])
+        assert got_v == v
+        assert q["absmax_q"][b] == _exact_nearest(v, tab), (b, float(v))
+        k = int(q["absmax_q"][b])
+        if k < 254 and Fraction(float(v)) == (Fraction(float(tab[k])) + Fraction(float(tab[k + 1]))) / 2:
+            ties += 1
+    assert ties >= 3 and len(where) > 100

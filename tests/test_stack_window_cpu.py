@@ -144,16 +144,22 @@ def test_sweeps_copy_2L_minus_2S_layers(monkeypatch, L, S, ahead, api):
         assert counts == [2 * L - S, 2 * L - 2 * S, 2 * L - 2 * S], counts
 
 
-@pytest.mark.parametrize("L,S", [(6, 2), (6, 4), (32, 20)])
-def test_reference_and_recompute_steps_keep_the_pool_consistent(monkeypatch, L, S):
-    """Three sweeps per step (adapter-off reference forward, forward, backward with the forward again inside):
-    no sweep runs out of slots and every acquire is released."""
-    st, pool = _cpu_stack(monkeypatch, L, S, True)
+@pytest.mark.parametrize("ahead", [True, False])
+@pytest.mark.parametrize("L,S", [(6, 2), (6, 4), (32, 20), (32, 2)])
+def test_reference_and_recompute_steps_keep_the_pool_consistent(monkeypatch, L, S, ahead):
+    """A step with the adapter-off reference forward and the recomputing backward: the reference and the
+    policy forward of a layer share one acquisition, so the sweeps acquire each layer once per direction
+    and copy as many layers as a plain step (2L - S, then 2L - 2S); no sweep runs out of slots and every
+    acquire is released."""
+    st, pool = _cpu_stack(monkeypatch, L, S, ahead)
+    counts = []
     for _ in range(3):
-        a0 = len(pool.acquired)
+        a0, c0 = len(pool.acquired), pool.copies
         st.step(reference=True, recompute=True)
-        assert pool.acquired[a0:] == list(range(L)) * 2 + list(reversed(range(L)))
+        counts.append(pool.copies - c0)
+        assert pool.acquired[a0:] == list(range(L)) + list(reversed(range(L)))
         assert sum(pool.refs) == 0
+    assert counts == [2 * L - S, 2 * L - 2 * S, 2 * L - 2 * S], counts
 
 
 def test_layer_layout_splits_codes_and_constants():

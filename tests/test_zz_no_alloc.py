@@ -28,7 +28,7 @@ def _pair(lib, W):
     """(blob from nf4_quantize with a workspace, blob from nf4_quantize_noalloc)."""
     import torch
     rows, cols = W.shape
-    Wd = torch.from_numpy(np.ascontiguousarray(W, np.float32)).cuda()
+    Wd = W if isinstance(W, torch.Tensor) else torch.from_numpy(np.ascontiguousarray(W, np.float32)).cuda()
     ref = DeviceNF4(rows, cols).quantize(Wd)
     got = DeviceNF4(rows, cols)
     got.blob.fill_(0xA5)                      # garbage where the result must land
@@ -54,6 +54,18 @@ def test_noalloc_matches_workspace_version_twice_in_a_row(lib):
     for W in (W1, W2, W1):                   # consecutive calls share the scratch array
         ref, got = _pair(lib, W)
         _same(ref, got)
+
+
+def test_noalloc_at_exactly_the_limit(lib):
+    """A weight of exactly LSN_NF4_NOALLOC_MAX_ELEMS elements (16384 x 4096) fills the scratch array to its
+    last absmax and partial sum; the result still equals nf4_quantize's bit for bit."""
+    import torch
+    rows, cols = 16384, 4096
+    assert rows * cols == lib.NF4_NOALLOC_MAX_ELEMS
+    W = synth.device_normal((rows, cols), 0.02, synth.SEED, 79, 0, synth.T_W, device=torch.device("cuda", 0))
+    W[-1, -64:] *= 40.0                      # the last block and group carry the largest absmax
+    ref, got = _pair(lib, W)
+    _same(ref, got)
 
 
 def test_noalloc_leaves_free_memory_unchanged(lib):
