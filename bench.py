@@ -192,7 +192,8 @@ def run_ours(args):
                     dequant_ahead=bool(args.dequant_ahead))
     wanted = [m for m in args.modes.split(",") if m]
     modes = ["streamed"] + [m for m in wanted
-                            if m in ("no_h2d", "resident", "proj", "dpo", "recompute", "shared", "grouped")
+                            if m in ("no_h2d", "resident", "proj", "dpo", "recompute", "shared", "grouped",
+                                     "bf16_base")
                             or _POOL_MODE.match(m) or m.startswith("accum")]
     mode_tokens = {m: T for m in modes}
     mode_copies = {}
@@ -226,6 +227,10 @@ def run_ours(args):
             st = st_main.with_mode("streamed", n_slots=args.slots)
         elif mode in ("shared", "grouped"):   # q|k|v and gate|up read one input each (no_h2d pool)
             st = st_main.with_inputs(shared_inputs=True, grouped=(mode == "grouped"))
+        elif mode == "bf16_base":             # the same shapes with a bf16 base: no NF4 conversion at all (no_h2d)
+            import dataclasses
+            st = Stack(dataclasses.replace(cfg, base="bf16"), layers=L, tokens=T, mode="no_h2d",
+                       seed=synth.SEED + rank, stream=stream, lanes=args.lanes, api=args.api)
         else:
             st = st_main.with_mode(mode)
         # Clocks of the value's mode: the sampler starts before the warm-up
@@ -379,8 +384,13 @@ def run_ours(args):
         "config": {**workload_config(cfg, T, L, args.slots, world),
                    "api": args.api,
                    "lanes": args.lanes if args.api == "proj" else 1,
-                   "nf4_conversion": "inside the GEMM" if args.fused_nf4 else "nf4_dequant then bf16 GEMM",
+                   "nf4_conversion": {0: "nf4_dequant then bf16 GEMM",
+                                      1: "inside the GEMM (shared memory), both directions",
+                                      2: "forward: inside the GEMM (tensor memory); backward: nf4_dequant then "
+                                         "bf16 GEMM"}[args.fused_nf4],
                    "programmatic_dependent_launch": not args.no_pdl,
+                   "gemm_schedule": "stream-K where tiles leave the last wave partly empty" if args.stream_k
+                                    else "whole tiles round robin",
                    "dequant_ahead": st_main.ahead,
                    "l2": "inputs larger than L2 (per step ~11 GB of activations; every layer's NF4 codes read twice)"},
         "pct_bf16_peak": 100 * flop_step / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
@@ -572,11 +582,12 @@ def main():
                     help="VRAM pool slots of the timed stream (default 20 of 32 layers: the smallest measured "
                          "window that hides the copies behind compute at 2048 tokens on one B200)")
     ap.add_argument("--modes", default="no_h2d,resident,proj,streamed_S2,streamed_T8192,streamed_S2_T8192,"
-                                       "no_h2d_T8192,accum4,dpo,recompute,shared,grouped",
+                                       "no_h2d_T8192,accum4,dpo,recompute,shared,grouped,bf16_base",
                     help="extra modes timed after the streamed one (streamed_T<n>: streamed with n tokens; "
                          "streamed_S<n>: streamed through n pool slots; streamed_S<n>_T<m>: both; no_h2d_T<n>: "
                          "the pre-filled pool with n tokens; accum<n>: n micro-batches per step, gradients "
-                         "accumulated)")
+                         "accumulated; bf16_base: the same shapes with an un-quantised base, the bound on what "
+                         "any NF4 conversion scheme can save)")
     ap.add_argument("--api", choices=["layer", "proj"], default="layer",
                     help="one library call per layer, or one per projection")
     ap.add_argument("--lanes", type=int, default=2, help="streams the seven projections of a layer are spread over")
@@ -585,19 +596,26 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=768, help="token rows of the timed oracle sample")
     ap.add_argument("--cpu-budget", type=float, default=60.0)
     ap.add_argument("--ref-rows", type=int, default=64, help="token rows per step of the reference arm")
-    ap.add_argument("--fused-nf4", action="store_true", help="convert NF4 inside the GEMM (no bf16 copy of W)")
+    ap.add_argument("--fused-nf4", type=int, default=0, choices=[0, 1, 2],
+                    help="NF4 conversion: 0 = nf4_dequant then the bf16 GEMM; 1 = inside the GEMM into shared "
+                         "memory (both directions); 2 = inside the forward GEMM into tensor memory")
     ap.add_argument("--no-pdl", action="store_true", help="ordinary launches instead of programmatic dependent ones")
+    ap.add_argument("--stream-k", type=int, default=0, choices=[0, 1],
+                    help="GEMM schedule: whole tiles round robin (0, default), or stream-K where tiles leave the "
+                         "last wave partly empty (1)")
     ap.add_argument("--dequant-ahead", type=int, default=1, choices=[0, 1],
                     help="dequantise each layer on a side stream one layer ahead (1, default) or inside the layer call")
     ap.add_argument("--case", default="", help="profile one 8B projection (q,k,v,o,gate,up,down) instead of the stack")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
-    if args.impl == "ours" and (args.fused_nf4 or args.no_pdl):
+    if args.impl == "ours" and (args.fused_nf4 or args.no_pdl or args.stream_k):
         from layer_streamed_nf4_b200 import lsnf4
         if args.fused_nf4:
-            lsnf4.set_option(lsnf4.LSN_OPT_FUSED_NF4, 1)
+            lsnf4.set_option(lsnf4.LSN_OPT_FUSED_NF4, args.fused_nf4)
         if args.no_pdl:
             lsnf4.set_option(lsnf4.LSN_OPT_PDL, 0)
+        if args.stream_k:
+            lsnf4.set_option(lsnf4.LSN_OPT_STREAM_K, 1)
     if args.impl == "reference":
         run_reference(args)
     elif args.case:

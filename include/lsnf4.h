@@ -326,12 +326,23 @@ lsn_status lsn_timing_read(lsn_kernel_timing* out);
 
 /* ------------------------------------------------------------- options --
  *
- * Process-wide switches between equivalent implementations (same results bit
- * for bit; only speed differs).
+ * Process-wide switches between equivalent implementations.  Every setting
+ * is deterministic: a given shape always gives the same bits.  LSN_OPT_STREAM_K
+ * changes the last bits of some outputs (it decides where fp32 partial sums
+ * meet); the other switches change only speed.
  *   LSN_OPT_FUSED_NF4  1: NF4 weights on the 2-SM GEMM are converted to bf16
- *                      inside the GEMM by converter warps (no bf16 copy of W);
+ *                      inside the GEMM by converter warps (no bf16 copy of W;
+ *                      whole tiles only: its bits equal the unfused path's
+ *                      with LSN_OPT_STREAM_K 0);
  *                      0 (default): nf4_dequant into the workspace, then the
  *                      bf16 GEMM.  Narrow shapes always use the latter.
+ *   LSN_OPT_STREAM_K   1: when a GEMM's output tiles do not fill whole
+ *                      waves of the SMs, its contraction blocks are shared out
+ *                      evenly over the SMs (stream-K): a tile cut between two
+ *                      SMs is summed in two fp32 pieces that meet in the
+ *                      workspace (in a fixed way, whatever the timing).
+ *                      0 (default): whole tiles, round robin (the last wave
+ *                      partly idle; measured faster on the 8B shapes).
  *   LSN_OPT_LAYER_LANES 2 (default): lora_layer_fwd / _bwd spread the work
  *                      of different projections that does not depend on each
  *                      other (their GEMMs; the backward's token reductions)
@@ -347,7 +358,7 @@ lsn_status lsn_timing_read(lsn_kernel_timing* out);
  *                      before it reads or writes global memory.  0: ordinary
  *                      stream-ordered launches.
  */
-typedef enum { LSN_OPT_FUSED_NF4 = 1, LSN_OPT_LAYER_LANES = 2, LSN_OPT_PDL = 3 } lsn_option;
+typedef enum { LSN_OPT_FUSED_NF4 = 1, LSN_OPT_LAYER_LANES = 2, LSN_OPT_PDL = 3, LSN_OPT_STREAM_K = 4 } lsn_option;
 lsn_status lsn_set_option(int option, int value);
 int lsn_get_option(int option);
 

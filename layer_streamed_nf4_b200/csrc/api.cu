@@ -88,14 +88,16 @@ namespace {
 
 // Workspace layout of the LoRA calls (each region 256-byte aligned):
 //   [0, 256)  status word of the GEMM kernels
+//   split     stream-K scratch of the GEMM (arrival counters, partial tiles)
 //   u32  fp32 [T, r]     x A^T
 //   g32  fp32 [T, r]     dY B
 //   s16  bf16 [T, r]     bf16(s u) or bf16(s g)
 //   w16  bf16 [N, K]     dequantised base (NF4 base only)
-// The status word must be zero when the workspace is first used: fill the
-// workspace with zeros once, when it is allocated.
+// The status word and the stream-K counters must be zero when the workspace
+// is first used: fill the workspace with zeros once, when it is allocated.
 struct LoraWs {
     int* err;
+    GemmSplitWs split;
     float* u32;
     float* g32;
     uint16_t* s16;
@@ -109,6 +111,7 @@ LoraWs carve(void* ws, int64_t T, int64_t K, int64_t N, int r, int kind) {
     char* b = reinterpret_cast<char*>(ws);
     auto take = [&](size_t bytes) { char* p = b ? b + off : nullptr; off += round_up(bytes, 256); return p; };
     w.err = reinterpret_cast<int*>(take(256));
+    w.split = gemm_split_ws(take(gemm_split_ws_bytes()));
     w.u32 = reinterpret_cast<float*>(take((size_t)T * r * 4));
     w.g32 = reinterpret_cast<float*>(take((size_t)T * r * 4));
     w.s16 = reinterpret_cast<uint16_t*>(take((size_t)T * r * 2));
@@ -156,7 +159,8 @@ double dequant_bytes(int64_t N, int64_t K) {
     return n / 2.0 + n / 64.0 + 4.0 * (double)((N * K / 64 + 255) / 256) + 4.0 + 2.0 * n;
 }
 
-// Workspace of the layer calls: the status word, then per projection i
+// Workspace of the layer calls: the status word, the stream-K scratch of the
+// two lanes' GEMMs, then per projection i
 //   s16 bf16 [T, r]  bf16(s u_i) (forward) or bf16(s g_i) (backward)
 //   g32 fp32 [T, r]  dY_i B_i
 //   u32 fp32 [T, r]  x_i A_i^T when the caller keeps no u
@@ -191,6 +195,7 @@ Groups find_groups(int n, const lsn_lora_proj* p) {
 
 struct LayerWs {
     int* err;
+    GemmSplitWs split[2];               // stream-K scratch of the GEMMs on the main and the side lane
     uint16_t* s16[LSN_LAYER_MAX_PROJ];
     float* g32[LSN_LAYER_MAX_PROJ];
     float* u32[LSN_LAYER_MAX_PROJ];
@@ -206,6 +211,7 @@ LayerWs carve_layer(void* ws, int n, const lsn_lora_proj* p, int64_t T, int r) {
     char* b = reinterpret_cast<char*>(ws);
     auto take = [&](size_t bytes) { char* q = b ? b + off : nullptr; off += round_up(bytes, 256); return q; };
     w.err = reinterpret_cast<int*>(take(256));
+    for (auto& sp : w.split) sp = gemm_split_ws(take(gemm_split_ws_bytes()));
     for (int i = 0; i < n; ++i) {
         w.s16[i] = reinterpret_cast<uint16_t*>(take((size_t)T * r * 2));
         w.g32[i] = reinterpret_cast<float*>(take((size_t)T * r * 4));
@@ -277,8 +283,15 @@ lsn_status check_layer(int n, const lsn_lora_proj* p, int64_t T, int r, void* ws
     return LSN_OK;
 }
 
+// NF4 conversion inside the GEMM (LSN_OPT_FUSED_NF4): 1 = converter warps
+// writing the bf16 tile into shared memory (both directions, 2-SM shapes);
+// 2 = converter warps writing W into tensor memory (forward only, shapes
+// with at least a wave of 256 x 256 tiles).
 bool fused_here(const lsn_base& W, int64_t M, int64_t N) {
-    return W.kind == LSN_BASE_NF4 && g_fused_nf4.load() && gemm_use_pairs(M, N);
+    return W.kind == LSN_BASE_NF4 && g_fused_nf4.load() == 1 && gemm_use_pairs(M, N);
+}
+bool fused_tmem_fwd(const lsn_base& W, int64_t T) {
+    return W.kind == LSN_BASE_NF4 && g_fused_nf4.load() == 2 && gemm_nf4t_supported(T, W.rows, W.cols);
 }
 
 // Dequantise the NF4 bases of the listed projections into their workspace copies, one launch.
@@ -324,7 +337,7 @@ lsn_status timed_tgrad_batch(int n, const TgSpec* d, int r, cudaStream_t st) {
 // from several host threads cannot interleave their fork/join events.
 struct SideLane {
     cudaStream_t side = nullptr;
-    cudaEvent_t fork = nullptr, join = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr, mark = nullptr;
 };
 std::mutex g_side_mu;
 SideLane g_side[64];
@@ -340,7 +353,8 @@ class LaneScope {
         if (!L.side) {
             if (cudaStreamCreateWithFlags(&L.side, cudaStreamNonBlocking) != cudaSuccess ||
                 cudaEventCreateWithFlags(&L.fork, cudaEventDisableTiming) != cudaSuccess ||
-                cudaEventCreateWithFlags(&L.join, cudaEventDisableTiming) != cudaSuccess) {
+                cudaEventCreateWithFlags(&L.join, cudaEventDisableTiming) != cudaSuccess ||
+                cudaEventCreateWithFlags(&L.mark, cudaEventDisableTiming) != cudaSuccess) {
                 L = SideLane{};
                 return;
             }
@@ -349,6 +363,7 @@ class LaneScope {
         lane_ = &L;
     }
     cudaStream_t main() const { return st_; }
+    bool two() const { return lane_ != nullptr; }
     cudaStream_t side() const { return lane_ ? lane_->side : st_; }
     // Both lanes continue only after everything enqueued so far on either.
     lsn_status barrier() {
@@ -356,6 +371,30 @@ class LaneScope {
         LSN_CUDA_TRY(cudaEventRecord(lane_->fork, st_));
         LSN_CUDA_TRY(cudaEventRecord(lane_->join, lane_->side));
         LSN_CUDA_TRY(cudaStreamWaitEvent(st_, lane_->join, 0));
+        LSN_CUDA_TRY(cudaStreamWaitEvent(lane_->side, lane_->fork, 0));
+        return LSN_OK;
+    }
+    // One-way orderings: one lane waits for what the other has enqueued so far.
+    lsn_status main_waits_side() {
+        if (!lane_) return LSN_OK;
+        LSN_CUDA_TRY(cudaEventRecord(lane_->join, lane_->side));
+        LSN_CUDA_TRY(cudaStreamWaitEvent(st_, lane_->join, 0));
+        return LSN_OK;
+    }
+    // A point on the side lane that the main lane can wait for later.
+    lsn_status mark_side() {
+        if (!lane_) return LSN_OK;
+        LSN_CUDA_TRY(cudaEventRecord(lane_->mark, lane_->side));
+        return LSN_OK;
+    }
+    lsn_status main_waits_mark() {
+        if (!lane_) return LSN_OK;
+        LSN_CUDA_TRY(cudaStreamWaitEvent(st_, lane_->mark, 0));
+        return LSN_OK;
+    }
+    lsn_status side_waits_main() {
+        if (!lane_) return LSN_OK;
+        LSN_CUDA_TRY(cudaEventRecord(lane_->fork, st_));
         LSN_CUDA_TRY(cudaStreamWaitEvent(lane_->side, lane_->fork, 0));
         return LSN_OK;
     }
@@ -397,9 +436,9 @@ lsn_status timed_tgrad(const float* G, const uint16_t* X, bool out_rk, int64_t T
 
 lsn_status timed_gemm(int kind, const uint16_t* A, int64_t lda, const uint16_t* B, int64_t ldb, bool b_mn,
                       const uint16_t* LA, const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D,
-                      int64_t ldd, int* err, cudaStream_t st) {
+                      int64_t ldd, int* err, cudaStream_t st, const GemmSplitWs* split) {
     TimingScope ts(kind, 2.0 * M * N * (double)(Kc + r), st);
-    return launch_gemm(A, lda, B, ldb, b_mn, LA, LB, r, M, N, Kc, D, ldd, err, st);
+    return launch_gemm(A, lda, B, ldb, b_mn, LA, LB, r, M, N, Kc, D, ldd, err, st, split);
 }
 
 }  // namespace
@@ -511,7 +550,12 @@ lsn_status lora_linear_fwd(const lsn_base* W, const uint16_t* x, int64_t T, cons
     const int64_t N = W->rows, K = W->cols;
     LoraWs w = carve(ws, T, K, N, r, W->kind);
     if ((s = timed_down(x, A, true, T, K, r, scale, nullptr, w.s16, w, st)) != LSN_OK) return s;
-    if (W->kind == LSN_BASE_NF4 && g_fused_nf4.load() && gemm_use_pairs(T, N)) {
+    if (fused_tmem_fwd(*W, T)) {
+        // NF4 converted straight into tensor memory (no bf16 copy of W).
+        TimingScope ts(LSN_K_GEMM_FWD, 2.0 * T * N * (double)(K + r), st);
+        return launch_gemm_nf4t(x, K, &W->nf4, w.s16, B, r, T, N, K, y, N, w.err, st);
+    }
+    if (fused_here(*W, T, N)) {
         // NF4 converted inside the GEMM (no bf16 copy of W).
         TimingScope ts(LSN_K_GEMM_FWD, 2.0 * T * N * (double)(K + r), st);
         return launch_gemm_nf4(x, K, &W->nf4, false, w.s16, B, r, T, N, K, y, N, w.err, st);
@@ -521,7 +565,7 @@ lsn_status lora_linear_fwd(const lsn_base* W, const uint16_t* x, int64_t T, cons
         if ((s = timed_dequant(&W->nf4, w.w16, st)) != LSN_OK) return s;
         Wb = w.w16;
     }
-    return timed_gemm(LSN_K_GEMM_FWD, x, K, Wb, K, false, w.s16, B, r, T, N, K, y, N, w.err, st);
+    return timed_gemm(LSN_K_GEMM_FWD, x, K, Wb, K, false, w.s16, B, r, T, N, K, y, N, w.err, st, &w.split);
 }
 
 lsn_status lora_linear_bwd(const lsn_base* W, const uint16_t* x, const uint16_t* dY, int64_t T, const uint16_t* A,
@@ -540,7 +584,7 @@ lsn_status lora_linear_bwd(const lsn_base* W, const uint16_t* x, const uint16_t*
     if (T > 0) {
         if ((s = timed_down(dY, B, false, T, N, r, scale, w.g32, w.s16, w, st)) != LSN_OK) return s;
         if ((s = timed_down(x, A, true, T, K, r, scale, w.u32, nullptr, w, st)) != LSN_OK) return s;
-        if (dX && W->kind == LSN_BASE_NF4 && g_fused_nf4.load() && gemm_use_pairs(T, K)) {
+        if (dX && fused_here(*W, T, K)) {
             TimingScope ts(LSN_K_GEMM_BWD, 2.0 * T * K * (double)(N + r), st);
             if ((s = launch_gemm_nf4(dY, N, &W->nf4, true, w.s16, A, r, T, K, N, dX, K, w.err, st)) != LSN_OK) return s;
         } else if (dX) {
@@ -549,7 +593,7 @@ lsn_status lora_linear_bwd(const lsn_base* W, const uint16_t* x, const uint16_t*
                 if ((s = timed_dequant(&W->nf4, w.w16, st)) != LSN_OK) return s;
                 Wb = w.w16;
             }
-            if ((s = timed_gemm(LSN_K_GEMM_BWD, dY, N, Wb, K, true, w.s16, A, r, T, K, N, dX, K, w.err, st)) != LSN_OK)
+            if ((s = timed_gemm(LSN_K_GEMM_BWD, dY, N, Wb, K, true, w.s16, A, r, T, K, N, dX, K, w.err, st, &w.split)) != LSN_OK)
                 return s;
         }
     }
@@ -608,7 +652,8 @@ lsn_status lora_layer_fwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
         const int i0 = g.first[k], m = g.count[k];
         for (int j = 0; j < m; ++j) {
             const int i = i0 + j;
-            deq[i] = p[i].W.kind == LSN_BASE_NF4 && (m > 1 || !fused_here(p[i].W, T, p[i].W.rows));
+            deq[i] = p[i].W.kind == LSN_BASE_NF4 &&
+                     (m > 1 || !(fused_here(p[i].W, T, p[i].W.rows) || fused_tmem_fwd(p[i].W, T)));
             if (adapter_off(p[i])) continue;
             // a group's bf16(s u) go side by side into its LoRA operand
             dn[nd++] = m > 1 ? DownSpec{p[i].x, p[i].A, p[i].u, w.la[i0] + j * r, T, p[i].W.cols, scale, m * r}
@@ -617,19 +662,33 @@ lsn_status lora_layer_fwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
     }
     // Two lanes: the down projections (bound by reading x) run beside the
     // dequantisation (bound by writing W); then the GEMMs, which are
-    // independent of each other, alternate over the lanes.
+    // independent of each other, alternate over the lanes.  With nothing to
+    // dequantise and no groups, only the first GEMM's down projection runs
+    // ahead of it: the others run on the side lane beside that GEMM, and the
+    // main lane's later GEMMs wait for them.
     LaneScope lanes(st, g_layer_lanes.load() == 2);
-    for (int k = 0; k < g.n; ++k)
-        if (g.count[k] > 1 && !adapter_off(p[g.first[k]]))
-            if ((s = build_group_lb(p, g.first[k], g.count[k], r, false, w.lb[g.first[k]], lanes.side())) != LSN_OK)
-                return s;
-    if ((s = timed_down_batch(nd, dn, true, r, lanes.side())) != LSN_OK) return s;
-    if ((s = layer_dequant(n, p, deq, w, lanes.main())) != LSN_OK) return s;
-    if ((s = lanes.barrier()) != LSN_OK) return s;
+    bool any_deq = false, any_group = false;
+    for (int i = 0; i < n; ++i) any_deq = any_deq || deq[i];
+    for (int k = 0; k < g.n; ++k) any_group = any_group || g.count[k] > 1;
+    const bool early = lanes.two() && !any_deq && !any_group && nd > 0 && !adapter_off(p[0]);
+    if (early) {
+        if ((s = timed_down_batch(1, dn, true, r, lanes.main())) != LSN_OK) return s;      // dn[0]: projection 0
+        if ((s = timed_down_batch(nd - 1, dn + 1, true, r, lanes.side())) != LSN_OK) return s;
+    } else {
+        for (int k = 0; k < g.n; ++k)
+            if (g.count[k] > 1 && !adapter_off(p[g.first[k]]))
+                if ((s = build_group_lb(p, g.first[k], g.count[k], r, false, w.lb[g.first[k]], lanes.side())) != LSN_OK)
+                    return s;
+        if ((s = timed_down_batch(nd, dn, true, r, lanes.side())) != LSN_OK) return s;
+        if ((s = layer_dequant(n, p, deq, w, lanes.main())) != LSN_OK) return s;
+        if ((s = lanes.barrier()) != LSN_OK) return s;
+    }
     for (int k = 0; k < g.n; ++k) {
+        if (early && k == 1 && (s = lanes.main_waits_side()) != LSN_OK) return s;
         const int i = g.first[k], m = g.count[k];
         const int64_t K = p[i].W.cols;
         const cudaStream_t gs = (k & 1) ? lanes.side() : lanes.main();
+        const GemmSplitWs* sp = &w.split[k & 1];
         const int ri = adapter_off(p[i]) ? 0 : r;       // no LoRA K-block with the adapter off
         const uint16_t* Wb = p[i].W.kind == LSN_BASE_NF4 ? w.w16[i] : p[i].W.bf16;
         if (m > 1) {
@@ -647,7 +706,11 @@ lsn_status lora_layer_fwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
                 nsum += p[i + j].W.rows;
             }
             TimingScope ts(LSN_K_GEMM_FWD, 2.0 * T * nsum * (double)(K + m * ri), gs);
-            s = launch_gemm_grouped(gg, Wb, K, false, w.la[i], w.lb[i], m * ri, T, nsum, K, nullptr, 0, w.err, gs);
+            s = launch_gemm_grouped(gg, Wb, K, false, w.la[i], w.lb[i], m * ri, T, nsum, K, nullptr, 0, w.err, gs, sp);
+        } else if (fused_tmem_fwd(p[i].W, T)) {
+            const int64_t N = p[i].W.rows;
+            TimingScope ts(LSN_K_GEMM_FWD, 2.0 * T * N * (double)(K + ri), gs);
+            s = launch_gemm_nf4t(p[i].x, K, &p[i].W.nf4, w.s16[i], p[i].B, ri, T, N, K, p[i].y, N, w.err, gs);
         } else if (fused_here(p[i].W, T, p[i].W.rows)) {
             const int64_t N = p[i].W.rows;
             TimingScope ts(LSN_K_GEMM_FWD, 2.0 * T * N * (double)(K + ri), gs);
@@ -655,7 +718,7 @@ lsn_status lora_layer_fwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
         } else {
             const int64_t N = p[i].W.rows;
             s = timed_gemm(LSN_K_GEMM_FWD, p[i].x, K, Wb, K, false, w.s16[i], p[i].B, ri, T, N, K, p[i].y, N, w.err,
-                           gs);
+                           gs, sp);
         }
         if (s != LSN_OK) return s;
     }
@@ -675,6 +738,7 @@ lsn_status lora_layer_bwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
     // run beside the dequantisation; then the token reductions run on the
     // side lane beside the input-gradient GEMMs, which alternate over both.
     LaneScope lanes(st, T > 0 && g_layer_lanes.load() == 2);
+    bool early = false;
     if (T > 0) {
         bool deq[LSN_LAYER_MAX_PROJ];
         DownSpec dg[LSN_LAYER_MAX_PROJ], du[LSN_LAYER_MAX_PROJ];
@@ -692,14 +756,29 @@ lsn_status lora_layer_bwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
                 if (!p[i].u) du[nu++] = DownSpec{p[i].x, p[i].A, w.u32[i], nullptr, T, K, scale};
             }
         }
-        for (int k = 0; k < g.n; ++k)
-            if (g.count[k] > 1 && p[g.first[k]].dX && !adapter_off(p[g.first[k]]))
-                if ((s = build_group_lb(p, g.first[k], g.count[k], r, true, w.lb[g.first[k]], lanes.side())) != LSN_OK)
-                    return s;
-        if ((s = timed_down_batch(ng, dg, false, r, lanes.side())) != LSN_OK) return s;
-        if ((s = timed_down_batch(nu, du, true, r, lanes.side())) != LSN_OK) return s;
-        if ((s = layer_dequant(n, p, deq, w, lanes.main())) != LSN_OK) return s;
-        if ((s = lanes.barrier()) != LSN_OK) return s;
+        bool any_deq = false, any_group = false;
+        for (int i = 0; i < n; ++i) any_deq = any_deq || deq[i];
+        for (int k = 0; k < g.n; ++k) any_group = any_group || g.count[k] > 1;
+        // With nothing to dequantise and no groups, only the first input-gradient
+        // GEMM's g = dY B runs ahead of it (on the main lane); the other down
+        // projections and the token reductions run on the side lane beside it.
+        early = lanes.two() && !any_deq && !any_group && ng > 0 && p[0].dX != nullptr && !adapter_off(p[0]);
+        if (early) {
+            if ((s = timed_down_batch(1, dg, false, r, lanes.main())) != LSN_OK) return s;   // dg[0]: projection 0
+            if ((s = timed_down_batch(ng - 1, dg + 1, false, r, lanes.side())) != LSN_OK) return s;
+            if ((s = timed_down_batch(nu, du, true, r, lanes.side())) != LSN_OK) return s;
+            if ((s = lanes.mark_side()) != LSN_OK) return s;            // every g but the first is made
+            if ((s = lanes.side_waits_main()) != LSN_OK) return s;      // the reductions need g of projection 0
+        } else {
+            for (int k = 0; k < g.n; ++k)
+                if (g.count[k] > 1 && p[g.first[k]].dX && !adapter_off(p[g.first[k]]))
+                    if ((s = build_group_lb(p, g.first[k], g.count[k], r, true, w.lb[g.first[k]], lanes.side())) != LSN_OK)
+                        return s;
+            if ((s = timed_down_batch(ng, dg, false, r, lanes.side())) != LSN_OK) return s;
+            if ((s = timed_down_batch(nu, du, true, r, lanes.side())) != LSN_OK) return s;
+            if ((s = layer_dequant(n, p, deq, w, lanes.main())) != LSN_OK) return s;
+            if ((s = lanes.barrier()) != LSN_OK) return s;
+        }
     }
     // dA and dB of every projection in one launch (with T == 0: zeros, or the
     // accumulators left as they are); they need only g and u.
@@ -717,6 +796,8 @@ lsn_status lora_layer_bwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
             const int i = g.first[k], m = g.count[k];
             if (!p[i].dX) continue;
             const int64_t K = p[i].W.cols;
+            if (early && j == 1 && (s = lanes.main_waits_mark()) != LSN_OK) return s;   // the other g
+            const GemmSplitWs* sp = &w.split[j & 1];
             const cudaStream_t gs = (j++ & 1) ? lanes.side() : lanes.main();
             const int ri = adapter_off(p[i]) ? 0 : r;
             const uint16_t* Wb = p[i].W.kind == LSN_BASE_NF4 ? w.w16[i] : p[i].W.bf16;
@@ -732,7 +813,7 @@ lsn_status lora_layer_bwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
                     nsum += p[i + q].W.rows;
                 }
                 TimingScope ts(LSN_K_GEMM_BWD, 2.0 * T * K * (double)(nsum + m * ri), gs);
-                s = launch_gemm_grouped(gg, Wb, K, true, w.la[i], w.lb[i], m * ri, T, K, nsum, p[i].dX, K, w.err, gs);
+                s = launch_gemm_grouped(gg, Wb, K, true, w.la[i], w.lb[i], m * ri, T, K, nsum, p[i].dX, K, w.err, gs, sp);
             } else if (fused_here(p[i].W, T, K)) {
                 const int64_t N = p[i].W.rows;
                 TimingScope ts(LSN_K_GEMM_BWD, 2.0 * T * K * (double)(N + ri), gs);
@@ -741,7 +822,7 @@ lsn_status lora_layer_bwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
             } else {
                 const int64_t N = p[i].W.rows;
                 s = timed_gemm(LSN_K_GEMM_BWD, p[i].dY, N, Wb, K, true, w.s16[i], p[i].A, ri, T, K, N, p[i].dX, K,
-                               w.err, gs);
+                               w.err, gs, sp);
             }
             if (s != LSN_OK) return s;
         }
@@ -760,7 +841,12 @@ lsn_status lsn_set_option(int option, int value) {
         return LSN_OK;
     }
     if (option == LSN_OPT_FUSED_NF4) {
-        g_fused_nf4.store(value != 0 ? 1 : 0);
+        LSN_CHECK_ARG(value >= 0 && value <= 2, "lsn_set_option: LSN_OPT_FUSED_NF4 takes 0, 1 or 2");
+        g_fused_nf4.store(value);
+        return LSN_OK;
+    }
+    if (option == LSN_OPT_STREAM_K) {
+        gemm_set_stream_k(value != 0);
         return LSN_OK;
     }
     return fail(LSN_ERR_INVALID_ARG, "lsn_set_option: unknown option");
@@ -770,6 +856,7 @@ int lsn_get_option(int option) {
     if (option == LSN_OPT_FUSED_NF4) return g_fused_nf4.load();
     if (option == LSN_OPT_LAYER_LANES) return g_layer_lanes.load();
     if (option == LSN_OPT_PDL) return g_pdl.load();
+    if (option == LSN_OPT_STREAM_K) return gemm_stream_k() ? 1 : 0;
     return -1;
 }
 

@@ -34,6 +34,7 @@
 //              let the epilogue of tile i overlap the main loop of tile i+1.
 // Every wait is bounded; a wait that runs out sets *err and the CTA winds
 // down (after letting its issued copies and MMAs finish) instead of hanging.
+#include <atomic>
 #include <cstring>
 #include <mutex>
 
@@ -72,6 +73,21 @@ struct GemmArgs {
     float dq[256];             // second-level table
     const uint16_t* lora_b;    // LoRA operand of the last K-block (fwd: B [N, r]; bwd: A [r, N])
     int lora_r;
+    // Stream-K schedule (sk != 0).  The num_tiles x num_kb contraction blocks
+    // of the base term, tile after tile, are cut into consecutive ranges of
+    // sk_per blocks, one per worker (CTA pair or CTA), so every worker does
+    // the same work (a tile's LoRA block goes with its last piece).  A
+    // tile cut by a range boundary is computed in two pieces (by the workers
+    // on either side of the boundary); each writes its fp32 partial tile to
+    // sk_part and counts itself in sk_cnt (one counter per boundary and CTA
+    // of a pair); the one that counts second adds the two partials and
+    // stores the tile.  fp32 addition is commutative, so the result does not
+    // depend on which piece finishes first.  Counters are zero between
+    // launches (the second piece resets its counter).
+    int sk;
+    int64_t sk_per;
+    float* sk_part;
+    int* sk_cnt;
 };
 
 namespace {
@@ -110,6 +126,150 @@ struct Cfg {
 __device__ __forceinline__ void raise_error(volatile int* abort_flag, int* err, int code) {
     *abort_flag = 1;
     if (err) atomicExch(err, code);
+}
+
+// The work of one worker: (tile, first contraction block, end block) items,
+// either whole tiles round robin (tile = unit, unit + nunits, ...) or the
+// worker's stream-K range.  Stream-K ranges count the base term's blocks
+// only; the LoRA block (the last of a tile's nkb) always goes with the piece
+// that ends the tile, so a tile is cut at the same place with the adapter on
+// or off (its block adds exact zeros when B = 0).
+struct Items {
+    bool sk;
+    int nkb, nbase, num_tiles, nunits, tile;
+    int64_t cur, hi;
+    __device__ Items(const GemmArgs& p, int unit, int nunits_, int num_tiles_, int nkb_)
+        : sk(p.sk != 0), nkb(nkb_), nbase(p.num_kb), num_tiles(num_tiles_), nunits(nunits_), tile(unit) {
+        const int64_t total = (int64_t)num_tiles_ * p.num_kb;
+        cur = (int64_t)unit * p.sk_per;
+        hi = cur + p.sk_per < total ? cur + p.sk_per : total;
+    }
+    __device__ bool next(int& t, int& kb0, int& kb1) {
+        if (!sk) {
+            if (tile >= num_tiles) return false;
+            t = tile;
+            kb0 = 0;
+            kb1 = nkb;
+            tile += nunits;
+            return true;
+        }
+        if (cur >= hi) return false;
+        t = (int)(cur / nbase);
+        kb0 = (int)(cur - (int64_t)t * nbase);
+        const int64_t left = hi - cur;
+        kb1 = (int64_t)(nbase - kb0) <= left ? nbase : kb0 + (int)left;
+        cur += kb1 - kb0;
+        if (kb1 == nbase) kb1 = nkb;           // the tile's end: its LoRA block too
+        return true;
+    }
+};
+
+// Named barrier 1 over the four epilogue warps (128 threads): a plain
+// barrier, and barriers that also reduce a predicate over the 128 threads.
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ bool epi_all(bool v) {
+    uint32_t r;
+    asm volatile("{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, 1, 128, p;\n selp.u32 %0, 1, 0, q;\n}"
+                 : "=r"(r) : "r"((uint32_t)v) : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ bool epi_any(bool v) {
+    uint32_t r;
+    asm volatile("{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, 1, 128, p;\n selp.u32 %0, 1, 0, q;\n}"
+                 : "=r"(r) : "r"((uint32_t)v) : "memory");
+    return r != 0;
+}
+
+// Round 32 fp32 values to bf16 and store them as 4 x 16 bytes.
+__device__ __forceinline__ void store_bf16x32(uint16_t* dst16, const float (&f)[32]) {
+    uint4* dst = reinterpret_cast<uint4*>(dst16);
+    #pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint4 o;
+        o.x = pack_bf16x2(f[8 * i + 0], f[8 * i + 1]);
+        o.y = pack_bf16x2(f[8 * i + 2], f[8 * i + 3]);
+        o.z = pack_bf16x2(f[8 * i + 4], f[8 * i + 5]);
+        o.w = pack_bf16x2(f[8 * i + 6], f[8 * i + 7]);
+        dst[i] = o;
+    }
+}
+
+
+// The bf16 output address of 32 columns starting at `col` of row `row`
+// (routed to its segment's output for a grouped GEMM).
+__device__ __forceinline__ uint16_t* out_ptr(const GemmArgs& p, int row, int col) {
+    uint16_t* base = p.D;
+    int64_t ld = p.ldd;
+    int lc = col;
+    if (p.nseg > 0) {                          // the segment of these 32 columns (widths: multiples of 64)
+        int sgi = 0;
+        while (sgi + 1 < p.nseg && col >= p.seg_col[sgi + 1]) ++sgi;
+        base = p.seg_D[sgi];
+        ld = p.seg_ld[sgi];
+        lc = col - p.seg_col[sgi];
+    }
+    return base + (int64_t)row * ld + lc;
+}
+
+// The epilogue of one of the two pieces of a stream-K tile (see GemmArgs):
+// write this CTA's fp32 partial, free the accumulator, count the piece and,
+// if it is the second, add both partials and store the tile.  Kept out of
+// line so that the common path of the epilogue keeps its few registers.
+template <bool PAIR, int BN>
+__device__ __noinline__ void split_piece(const GemmArgs& p, uint32_t tm, uint64_t* acc_empty, int piece, int unit,
+                                         uint32_t rank, int q, int lane, int row, int col0) {
+    const int bnd = piece == 0 ? unit + 1 : unit;
+    const int64_t tile_floats = (int64_t)BM * BN;
+    constexpr int CTAS = PAIR ? 2 : 1;
+    float* mine = p.sk_part + (((int64_t)bnd * 2 + piece) * CTAS + rank) * tile_floats;
+    const int rl = q * 32 + lane;
+    #pragma unroll 1
+    for (int c = 0; c < BN / 16; ++c) {
+        uint32_t v[16];
+        tmem_ld16(tm + (uint32_t)(c * 16), v);
+        tmem_ld_wait(v);
+        float4* d = reinterpret_cast<float4*>(mine + ((int64_t)(c >> 1) * BM + rl) * 32 + (c & 1) * 16);
+        #pragma unroll
+        for (int i = 0; i < 4; ++i)
+            d[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]), __uint_as_float(v[4 * i + 2]),
+                               __uint_as_float(v[4 * i + 3]));
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) {                    // the accumulator is free again
+        if constexpr (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(acc_empty), 0));
+        else                mbar_arrive(acc_empty);
+    }
+    __threadfence();                    // this thread's partial, visible device-wide ...
+    epi_sync();                         // ... for all 128 threads, before the count
+    int* cnt = p.sk_cnt + bnd * CTAS + rank;
+    int old = 0;
+    if (q == 0 && lane == 0) old = atomicAdd(cnt, 1);
+    if (!epi_any(old == 1)) return;     // the first piece: the second one stores the tile
+    __threadfence();
+    const float* other = p.sk_part + (((int64_t)bnd * 2 + (1 - piece)) * CTAS + rank) * tile_floats;
+    #pragma unroll 1
+    for (int c = 0; c < BN / 32; ++c) {
+        const int col = col0 + c * 32;
+        if (col >= p.N) break;
+        if (row < p.M) {
+            const float4* a = reinterpret_cast<const float4*>(mine + ((int64_t)c * BM + rl) * 32);
+            const float4* b = reinterpret_cast<const float4*>(other + ((int64_t)c * BM + rl) * 32);
+            uint4* dst = reinterpret_cast<uint4*>(out_ptr(p, row, col));
+            #pragma unroll 1
+            for (int i = 0; i < 4; ++i) {           // 8 columns at a time
+                const float4 x0 = __ldcg(a + 2 * i), x1 = __ldcg(a + 2 * i + 1);
+                const float4 y0 = __ldcg(b + 2 * i), y1 = __ldcg(b + 2 * i + 1);
+                uint4 o;
+                o.x = pack_bf16x2(x0.x + y0.x, x0.y + y0.y);
+                o.y = pack_bf16x2(x0.z + y0.z, x0.w + y0.w);
+                o.z = pack_bf16x2(x1.x + y1.x, x1.y + y1.y);
+                o.w = pack_bf16x2(x1.z + y1.z, x1.w + y1.w);
+                dst[i] = o;
+            }
+        }
+    }
+    if (q == 0 && lane == 0) *cnt = 0;      // ready for the next launch on this workspace
 }
 
 // The A tensor maps of a grouped GEMM (the caller's separate dY tensors).
@@ -178,12 +338,14 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int tile = unit; tile < num_tiles && ok; tile += nunits) {
+            Items items(p, unit, nunits, num_tiles, nkb);
+            int tile, kb0, kb1;
+            while (ok && items.next(tile, kb0, kb1)) {
                 const int mb = tile % num_m, nb = tile / num_m;
                 const int m_row = mb * C::TILE_M + (int)rank * BM;
                 const int n_off = nb * BN + (int)rank * C::B_ROWS;
                 int ai = 0;                                   // A map of the current K-block
-                for (int kb = 0; kb < nkb; ++kb) {
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
                     uint8_t* sA = smem + stage * C::STAGE_BYTES;
                     uint8_t* sB = sA + C::A_BYTES;
@@ -220,11 +382,13 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
-            for (int tile = unit; tile < num_tiles && ok; tile += nunits) {
+            Items items(p, unit, nunits, num_tiles, nkb);
+            int tile, kb0, kb1;
+            while (ok && items.next(tile, kb0, kb1)) {
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-                for (int kb = 0; kb < nkb; ++kb) {
+                for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(smem + stage * C::STAGE_BYTES);
@@ -235,8 +399,9 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
                         const uint64_t ad = smem_desc_sw128(a0 + j * C::A_SUB + kk * 32, 16, 1024);
                         const uint64_t bd = B_MN ? smem_desc_sw128(b0 + k * 2048, BK * 128, 1024)
                                                  : smem_desc_sw128(b0 + j * C::B_SUB + kk * 32, 16, 1024);
-                        if constexpr (PAIR) umma_bf16_pair(d_tmem, ad, bd, C::IDESC, (kb | k) ? 1u : 0u);
-                        else                umma_bf16(d_tmem, ad, bd, C::IDESC, (kb | k) ? 1u : 0u);
+                        const uint32_t accum = (kb > kb0 || k > 0) ? 1u : 0u;
+                        if constexpr (PAIR) umma_bf16_pair(d_tmem, ad, bd, C::IDESC, accum);
+                        else                umma_bf16(d_tmem, ad, bd, C::IDESC, accum);
                     }
                     if constexpr (PAIR) umma_commit_pair(&empty[stage]);
                     else                umma_commit(&empty[stage]);
@@ -257,50 +422,47 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
     } else {
         // -------------------------------------------------------- epilogue --
         const int q = warp & 3;                    // TMEM lanes 32q .. 32q+31
-        const int nseg = p.nseg;
+        const int rloc = (int)rank * BM + q * 32 + lane;   // row of the tile this thread drains
         int acc = 0;
         uint32_t acc_phase = 0;
-        for (int tile = unit; tile < num_tiles; tile += nunits) {
+        Items items(p, unit, nunits, num_tiles, nkb);
+        int tile, kb0, kb1;
+        while (items.next(tile, kb0, kb1)) {
             const int mb = tile % num_m, nb = tile / num_m;
             const bool got = mbar_wait(&acc_full[acc], acc_phase, abort_flag);
-            if (!__all_sync(0xffffffffu, got)) { if (lane == 0) raise_error(abort_flag, p.err, 3); break; }
+            // With stream-K every epilogue warp takes the same path through the
+            // named barriers below, so they decide together.
+            if (p.sk ? !epi_all(got) : !__all_sync(0xffffffffu, got)) {
+                if (lane == 0) raise_error(abort_flag, p.err, 3);
+                break;
+            }
             tc_fence_after();
-            const int row = mb * C::TILE_M + (int)rank * BM + q * 32 + lane;
-            #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                const int col = nb * BN + c * 32;
-                if (col >= p.N) break;
-                uint32_t v[32];
-                tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c * 32), v);
-                tmem_ld_wait();
-                if (row < p.M) {
-                    uint16_t* base = p.D;
-                    int64_t ld = p.ldd;
-                    int lc = col;
-                    if (nseg > 0) {                // the segment of these 32 columns (widths: multiples of 64)
-                        int sgi = 0;
-                        while (sgi + 1 < nseg && col >= p.seg_col[sgi + 1]) ++sgi;
-                        base = p.seg_D[sgi];
-                        ld = p.seg_ld[sgi];
-                        lc = col - p.seg_col[sgi];
-                    }
-                    uint4* dst = reinterpret_cast<uint4*>(base + (int64_t)row * ld + lc);
-                    #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        uint4 o;
-                        o.x = pack_bf16x2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
-                        o.y = pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
-                        o.z = pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
-                        o.w = pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
-                        dst[i] = o;
+            const int row = mb * C::TILE_M + rloc;
+            const uint32_t tm = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+            const bool split = p.sk && (kb0 > 0 || kb1 < nkb);
+            if (!split) {
+                #pragma unroll 1
+                for (int c = 0; c < BN / 32; ++c) {
+                    const int col = nb * BN + c * 32;
+                    if (col >= p.N) break;
+                    uint32_t v[32];
+                    tmem_ld32(tm + (uint32_t)(c * 32), v);
+                    tmem_ld_wait(v);
+                    if (row < p.M) {
+                        float f[32];
+                        #pragma unroll
+                        for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
+                        store_bf16x32(out_ptr(p, row, col), f);
                     }
                 }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                if constexpr (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[acc]), 0));
-                else                mbar_arrive(&acc_empty[acc]);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if constexpr (PAIR) mbar_arrive_cluster(mapa_shared(smem_u32(&acc_empty[acc]), 0));
+                    else                mbar_arrive(&acc_empty[acc]);
+                }
+            } else {
+                split_piece<PAIR, BN>(p, tm, &acc_empty[acc], kb0 == 0 ? 0 : 1, unit, rank, q, lane, row, nb * BN);
             }
             acc ^= 1;
             if (acc == 0) acc_phase ^= 1;
@@ -509,7 +671,7 @@ __global__ void __launch_bounds__(CfgN<B_MN>::THREADS, 1)
                 if (col >= p.N) break;
                 uint32_t v[32];
                 tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c * 32), v);
-                tmem_ld_wait();
+                tmem_ld_wait(v);
                 if (row < p.M) {
                     uint4* dst = reinterpret_cast<uint4*>(p.D + (int64_t)row * p.ldd + col);
                     #pragma unroll
@@ -727,6 +889,11 @@ lsn_status launch_cfg(const AMaps& a, const CUtensorMap& b, const CUtensorMap& l
 
 }  // namespace
 
+lsn_status make_tmap_2d(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, int64_t stride_elems,
+                        int box_inner, int box_outer, bool bytes) {
+    return make_map(m, base, inner, outer, stride_elems, box_inner, box_outer, bytes);
+}
+
 // Kernel choice from the shape alone: the 2-SM kernel (256 x 256 tiles on
 // CTA pairs) when it has at least one full wave of pairs on a 148-SM part,
 // else the 1-SM kernel with 128 x 128 tiles.
@@ -809,9 +976,30 @@ lsn_status launch_gemm_nf4(const uint16_t* A, int64_t lda, const lsn_nf4_weight*
 //   b_mn == false: B is [N, Kc] (ldb), LB is [N, r]   (forward: W, B_lora)
 //   b_mn == true : B is [Kc, N] (ldb), LB is [r, N]   (backward: W, A_lora)
 //   LA [M, r] (bf16(s u) or bf16(s g)); r == 0 disables the LoRA term.
+size_t gemm_split_ws_bytes() {
+    const size_t pair = (size_t)(kSplitMaxUnits / 2 + 1) * 2 * 2 * 128 * 256 * sizeof(float);
+    const size_t one = (size_t)(kSplitMaxUnits + 1) * 2 * 1 * 128 * 128 * sizeof(float);
+    return kSplitCntBytes + (pair > one ? pair : one);
+}
+
+GemmSplitWs gemm_split_ws(void* base) {
+    GemmSplitWs w;
+    char* b = reinterpret_cast<char*>(base);
+    w.cnt = reinterpret_cast<int*>(b);
+    w.part = b ? reinterpret_cast<float*>(b + kSplitCntBytes) : nullptr;
+    return w;
+}
+
+namespace {
+std::atomic<int> g_stream_k{0};
+}
+
+void gemm_set_stream_k(bool on) { g_stream_k.store(on ? 1 : 0); }
+bool gemm_stream_k() { return g_stream_k.load() != 0; }
+
 lsn_status launch_gemm_grouped(const GemmGroup& g, const uint16_t* B, int64_t ldb, bool b_mn, const uint16_t* LA,
                                const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D,
-                               int64_t ldd, int* err, cudaStream_t st) {
+                               int64_t ldd, int* err, cudaStream_t st, const GemmSplitWs* split) {
     if (g.na < 1 || g.na > kMaxSeg || g.nseg < 0 || g.nseg > kMaxSeg)
         return fail(LSN_ERR_INVALID_ARG, "grouped GEMM: bad operand or segment count");
     const bool pair = gemm_use_pairs(M, N);
@@ -865,6 +1053,20 @@ lsn_status launch_gemm_grouped(const GemmGroup& g, const uint16_t* B, int64_t ld
     }
     args.seg_col[g.nseg] = (int)c0;
     if (g.nseg > 0 && c0 != N) return fail(LSN_ERR_INVALID_ARG, "grouped GEMM: segments do not add up to N");
+    // Stream-K when the tiles do not fill whole waves of workers (and there are
+    // at least as many tiles as workers, so that a tile has at most two pieces).
+    {
+        const int64_t tile_m = pair ? 256 : 128, tile_n = pair ? 256 : 128;
+        const int64_t tiles = ((M + tile_m - 1) / tile_m) * ((N + tile_n - 1) / tile_n);
+        const int units = pair ? sm_count() / 2 : sm_count();
+        if (split && split->cnt && gemm_stream_k() && units <= (pair ? kSplitMaxUnits / 2 : kSplitMaxUnits) &&
+            tiles >= units && tiles % units != 0) {
+            args.sk = 1;
+            args.sk_per = (tiles * args.num_kb + units - 1) / units;     // base blocks only (see Items)
+            args.sk_part = split->part;
+            args.sk_cnt = split->cnt;
+        }
+    }
     if (pair) return b_mn ? launch_cfg<true, 256, true>(ma, mb, mla, mlb, args, st)
                           : launch_cfg<true, 256, false>(ma, mb, mla, mlb, args, st);
     return b_mn ? launch_cfg<false, 128, true>(ma, mb, mla, mlb, args, st)
@@ -873,13 +1075,13 @@ lsn_status launch_gemm_grouped(const GemmGroup& g, const uint16_t* B, int64_t ld
 
 lsn_status launch_gemm(const uint16_t* A, int64_t lda, const uint16_t* B, int64_t ldb, bool b_mn, const uint16_t* LA,
                        const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D, int64_t ldd,
-                       int* err, cudaStream_t st) {
+                       int* err, cudaStream_t st, const GemmSplitWs* split) {
     GemmGroup g;
     g.na = 1;
     g.A[0] = A;
     g.lda[0] = lda;
     g.a_kc[0] = Kc;
-    return launch_gemm_grouped(g, B, ldb, b_mn, LA, LB, r, M, N, Kc, D, ldd, err, st);
+    return launch_gemm_grouped(g, B, ldb, b_mn, LA, LB, r, M, N, Kc, D, ldd, err, st, split);
 }
 
 }  // namespace lsn

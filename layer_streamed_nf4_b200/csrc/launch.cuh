@@ -74,16 +74,46 @@ struct GemmGroup {
     uint16_t* seg_D[kGemmMaxSeg] = {};
     int64_t seg_ld[kGemmMaxSeg] = {};
 };
+// Scratch of the GEMM's stream-K schedule (one region per stream that runs
+// GEMMs concurrently): arrival counters (zero between launches; the region
+// must be zero-filled once before its first use) and fp32 partial tiles.
+constexpr int kSplitMaxUnits = 160;                // workers the region is sized for (CTAs; pairs: half)
+constexpr size_t kSplitCntBytes = 4096;
+struct GemmSplitWs {
+    int* cnt = nullptr;
+    float* part = nullptr;
+};
+size_t gemm_split_ws_bytes();
+GemmSplitWs gemm_split_ws(void* base);
+void gemm_set_stream_k(bool on);
+bool gemm_stream_k();
+
+// split == NULL: whole tiles round robin (no stream-K scratch).
 lsn_status launch_gemm_grouped(const GemmGroup& g, const uint16_t* B, int64_t ldb, bool b_mn, const uint16_t* LA,
                                const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D,
-                               int64_t ldd, int* err, cudaStream_t st);
+                               int64_t ldd, int* err, cudaStream_t st, const GemmSplitWs* split);
 lsn_status launch_gemm(const uint16_t* A, int64_t lda, const uint16_t* B, int64_t ldb, bool b_mn, const uint16_t* LA,
                        const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D, int64_t ldd,
-                       int* err, cudaStream_t st);
+                       int* err, cudaStream_t st, const GemmSplitWs* split);
 lsn_status launch_gemm_nf4(const uint16_t* A, int64_t lda, const lsn_nf4_weight* w, bool b_mn, const uint16_t* LA,
                            const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D, int64_t ldd,
                            int* err, cudaStream_t st);
 bool gemm_use_pairs(int64_t M, int64_t N);
+
+// A 2-D tensor map of a row-major [outer, inner] tensor with row stride
+// stride_elems, read in boxes of box_inner x box_outer: bf16 with the
+// 128-byte swizzle, or (bytes) uint8 with the 64-byte swizzle.
+lsn_status make_tmap_2d(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, int64_t stride_elems,
+                        int box_inner, int box_outer, bool bytes);
+
+// The forward GEMM of an NF4 base with W converted straight into tensor
+// memory (gemm_nf4t.cu): y [M, N] = x [M, Kc] W^T + LA [M, r] LB^T with
+// W = w [N, Kc] NF4, LB [N, r].  LSN_ERR_UNSUPPORTED when the shape has fewer
+// output tiles than SM pairs (the caller dequantises instead).
+bool gemm_nf4t_supported(int64_t M, int64_t N, int64_t Kc);
+lsn_status launch_gemm_nf4t(const uint16_t* x, int64_t ldx, const lsn_nf4_weight* w, const uint16_t* LA,
+                            const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* y, int64_t ldy,
+                            int* err, cudaStream_t st);
 
 lsn_status launch_lora_down(const uint16_t* X, const uint16_t* W, bool w_rk, int64_t T, int64_t Kd, int r,
                             float scale, float* u32, uint16_t* u16, cudaStream_t st);

@@ -519,7 +519,9 @@ class Stack:
         fwd = lsnf4._lib.lora_layer_fwd
         n, ws, nb, sp = len(self.proj), self.ws[0].data_ptr(), self.ws_bytes, self.stream.cuda_stream
         passes = (False, True) if reference else (adapter,)
-        if self.ahead:
+        # With the forward GEMMs converting NF4 in tensor memory (LSN_OPT_FUSED_NF4 = 2) the forward sweep
+        # hands the layer calls the NF4 codes themselves; only the backward sweep dequantises ahead.
+        if self.ahead and lsnf4.get_option(lsnf4.LSN_OPT_FUSED_NF4) != 2:
             def call(l, b):
                 for ad in passes:
                     st = fwd(n, self._layer_projs(0, l, ad, wb=b), self.T, self.r, self.scale, ws, nb, sp)

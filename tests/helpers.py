@@ -1,6 +1,8 @@
 """Test helpers: tolerance metrics and device-side setup through the C ABI."""
 from __future__ import annotations
 
+import contextlib
+
 import numpy as np
 
 # Tolerances on floating-point outputs (y, dX, dA, dB) against the fp64
@@ -8,6 +10,17 @@ import numpy as np
 # the oracle's RMS.
 REL_FRO = 5e-3
 MAX_ABS_RMS = 2e-2
+
+
+@contextlib.contextmanager
+def lib_option(lib, option: int, value: int):
+    """Set one of the library's process-wide options for the duration of a block."""
+    old = lib.get_option(option)
+    lib.set_option(option, value)
+    try:
+        yield
+    finally:
+        lib.set_option(option, old)
 
 
 def err_metrics(got: np.ndarray, ref: np.ndarray):

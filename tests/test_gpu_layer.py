@@ -146,13 +146,30 @@ def test_layer_against_oracle(lib, orc):
 
 
 def test_layer_with_fused_nf4_equals_unfused(lib):
-    lib.set_option(lib.LSN_OPT_FUSED_NF4, 1)
-    try:
-        L = Layer(lib, [(4096, 9536), (9536, 4096), (4096, 1024)], 512, 16, "nf4")
+    from tests.helpers import lib_option
+    with lib_option(lib, lib.LSN_OPT_STREAM_K, 0):          # the fused kernel runs whole tiles
+        with lib_option(lib, lib.LSN_OPT_FUSED_NF4, 1):
+            L = Layer(lib, [(4096, 9536), (9536, 4096), (4096, 1024)], 512, 16, "nf4")
+            a = L.layer()
+        _equal(a, L.layer())
+
+
+def test_layer_with_tmem_fused_forward(lib, orc):
+    """Layer calls with the forward GEMMs converting NF4 in tensor memory (LSN_OPT_FUSED_NF4 = 2): the same
+    bits as the single-linear calls in that mode, y against the oracle, and the backward unchanged."""
+    from tests.helpers import lib_option
+    with lib_option(lib, lib.LSN_OPT_FUSED_NF4, 2):
+        L = Layer(lib, [(4096, 9536), (4096, 14336), (9536, 4096), (4096, 1024)], 512, 16, "nf4", seed=8)
         a = L.layer()
-    finally:
-        lib.set_option(lib.LSN_OPT_FUSED_NF4, 0)
-    _equal(a, L.layer())
+        _equal(a, L.single())
+    b = L.layer()
+    _equal(a, b, ("dX", "dA", "dB", "u"))
+    rows = np.sort(np.random.default_rng(4).choice(512, size=24, replace=False))
+    for d, o in zip(L.p, a):
+        c = d["case"]
+        q = orc.nf4_quantize(c.W)
+        Wb = orc.nf4_dequant(q["packed"], q["absmax_q"], q["s2"], q["offset"], c.W.size).reshape(c.W.shape)
+        assert_close(bf16_tensor_to_f64(o["y"])[rows], orc.lora_fwd(c.x, Wb, c.A, c.B, L.scale, rows=rows), "y")
 
 
 def test_layer_zero_tokens(lib):
@@ -269,14 +286,31 @@ def _run_layer(lib, L, out, groups):
                                           ([(896, 896), (896, 128), (896, 128), (896, 896), (896, 4864),
                                             (896, 4864), (4864, 896)], 512, "bf16")])
 def test_grouped_projections(lib, orc, shapes, T, kind):
-    """Grouped forward: the same bits as ungrouped.  Grouped backward: the group's dX is the sum of the
-    members' input gradients (checked against the oracle's sum on sampled rows); dA, dB the same bits."""
+    """Grouped forward: with whole-tile GEMMs the same bits as ungrouped; with the stream-K schedule (whose
+    split points depend on the GEMM's shape) within tolerance of the oracle.  Grouped backward: the
+    group's dX is the sum of the members' input gradients (checked against the oracle's sum on sampled
+    rows); dA, dB the same bits."""
+    from tests.helpers import lib_option
     L = _grouped_setup(lib, shapes, T, kind, seed=21)
-    plain = _run_layer(lib, L, L.outputs(), (0,) * 7)
-    grp = _run_layer(lib, L, L.outputs(), GROUPS)
-    _equal(grp, plain, ("y", "dA", "dB", "u"))
+    with lib_option(lib, lib.LSN_OPT_STREAM_K, 0):
+        plain = _run_layer(lib, L, L.outputs(), (0,) * 7)
+        grp = _run_layer(lib, L, L.outputs(), GROUPS)
+        _equal(grp, plain, ("y", "dA", "dB", "u"))
+    with lib_option(lib, lib.LSN_OPT_STREAM_K, 1):
+        plain = _run_layer(lib, L, L.outputs(), (0,) * 7)
+        grp = _run_layer(lib, L, L.outputs(), GROUPS)
+    _equal(grp, plain, ("dA", "dB", "u"))
     _equal([grp[3], grp[6]], [plain[3], plain[6]], ("dX",))          # ungrouped projections
     rows = np.sort(np.random.default_rng(3).choice(T, size=min(T, 48), replace=False))
+    for pi in (0, 2, 5):
+        c = L.p[pi]["case"]
+        if kind == "nf4":
+            q = orc.nf4_quantize(c.W)
+            Wb = orc.nf4_dequant(q["packed"], q["absmax_q"], q["s2"], q["offset"], c.W.size).reshape(c.W.shape)
+        else:
+            Wb = synth.to_bf16_bits(c.W)
+        assert_close(bf16_tensor_to_f64(grp[pi]["y"])[rows], orc.lora_fwd(c.x, Wb, c.A, c.B, L.scale, rows=rows),
+                     f"group member {pi} y")
     for members in ((0, 1, 2), (4, 5)):
         ref = 0.0
         for pi in members:

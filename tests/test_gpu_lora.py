@@ -112,9 +112,16 @@ def test_pair_kernel_with_ragged_rows(lib, orc, T, K, N):
 @pytest.mark.parametrize("T,K,N", [(512, 4096, 9536), (300, 9536, 4096)])
 def test_fused_nf4_equals_bf16_base_of_its_dequant(lib, T, K, N):
     """The NF4 weight converted inside the GEMM gives exactly the bits of the same
-    GEMM run on nf4_dequant's bf16 weight (same values, same MMA order).  The
+    GEMM run on nf4_dequant's bf16 weight (same values, same MMA order; the
+    fused kernel runs whole tiles, so both take the whole-tile schedule).  The
     shapes put one direction on the fused pair kernel, with a partial last
     N tile and, for K % 128 == 64, a half-empty last contraction stage."""
+    from tests.helpers import lib_option
+    with lib_option(lib, lib.LSN_OPT_STREAM_K, 0):
+        _fused_equals_unfused(lib, T, K, N)
+
+
+def _fused_equals_unfused(lib, T, K, N):
     import torch
     lib.set_option(lib.LSN_OPT_FUSED_NF4, 1)
     c = synth.linear_case(T, K, N, 16, 32.0, seed=T + N)
@@ -137,6 +144,34 @@ def test_fused_nf4_equals_bf16_base_of_its_dequant(lib, T, K, N):
         assert torch.equal(u, v), "unfused " + name
     for name, u, v in zip(("y", "dX", "dA", "dB"), a, b):
         assert torch.equal(u, v), name
+
+
+@pytest.mark.parametrize("T,K,N,r", [(2048, 4096, 4096, 16), (300, 4096, 9536, 16), (512, 4096, 14336, 8),
+                                     (257, 14336, 4096, 32)])
+def test_tmem_fused_forward(lib, orc, T, K, N, r):
+    """The forward GEMM that converts the NF4 codes straight into tensor memory (W as the A operand, y^T in
+    the accumulator, transposed in the epilogue): y against the oracle on sampled rows (the last one
+    included), and against the whole-tile GEMM on nf4_dequant's bf16 weight.  The shapes cover full and
+    ragged token tiles, a partial last W tile and ranks 8 to 32."""
+    import torch
+    from tests.helpers import lib_option
+    c = synth.linear_case(T, K, N, r, 2.0 * r, seed=T + K + N + r)
+    L = Linear(lib, c, "nf4")
+    with lib_option(lib, lib.LSN_OPT_STREAM_K, 0):
+        ref = L.fwd()                                  # nf4_dequant, then the bf16 GEMM
+        with lib_option(lib, lib.LSN_OPT_FUSED_NF4, 2):
+            y = L.fwd()
+            y2 = L.fwd()
+    torch.cuda.synchronize()
+    L.status()
+    assert torch.equal(y, y2), "rerun differs"
+    d = (y.float() - ref.float()).abs()
+    assert float(d.max()) <= 2.0 ** -7 * float(ref.float().abs().max()), float(d.max())
+    rows = np.sort(np.random.default_rng(13).choice(T, size=min(T, 40), replace=False))
+    rows[-1] = T - 1
+    Wb = _oracle_w_bits(orc, c.W, "nf4")
+    assert_close(bf16_tensor_to_f64(y)[rows], orc.lora_fwd(c.x, Wb, c.A, c.B, c.scale, rows=rows), "y (tensor-memory NF4)")
+    print("tmem-fused y bit-identical to dequant + GEMM:", bool(torch.equal(y, ref)))
 
 
 def test_b_zero_gives_the_base_product(lib, orc):
@@ -213,6 +248,40 @@ def test_full_size_sampled_rows(lib, orc, name, T, K, N):
     rA, rB = orc.lora_bwd_dadb(c.x, c.dY, c.A, c.B, c.scale)
     assert_close(dA.cpu().numpy(), rA, f"{name} dA")
     assert_close(dB.cpu().numpy(), rB, f"{name} dB")
+
+
+@pytest.mark.parametrize("T,K,N,rows", [(2048, 4096, 4096, 48), (300, 9536, 9536, 32), (300, 6400, 7680, 32)])
+def test_stream_k_schedule(lib, orc, T, K, N, rows):
+    """GEMMs whose tiles leave the last wave partly empty take the stream-K schedule, in both directions
+    here: the 8B q shape (128 pair tiles for 74 pairs), a ragged 2-SM shape (76 pair tiles, a half-empty
+    last contraction stage) and a ragged 1-SM one (180 and 150 tiles for 148 SMs).  Results match the
+    oracle, repeat bit for bit, and differ from the whole-tile schedule only by the rounding of the split
+    sums."""
+    import torch
+    from tests.helpers import lib_option
+    c = synth.linear_case(T, K, N, 16, 32.0, seed=T + K + N)
+    L = Linear(lib, c, "nf4")
+    with lib_option(lib, lib.LSN_OPT_STREAM_K, 1):
+        a = (L.fwd(), *L.bwd())
+        b = (L.fwd(), *L.bwd())
+    with lib_option(lib, lib.LSN_OPT_STREAM_K, 0):
+        w = (L.fwd(), *L.bwd())
+    torch.cuda.synchronize()
+    L.status()
+    for u, v in zip(a, b):
+        assert torch.equal(u, v), "stream-K rerun differs"
+    assert not torch.equal(a[0], w[0]) and not torch.equal(a[1], w[1]), "the stream-K schedule did not run"
+    for u, v in zip(a[:2], w[:2]):
+        d = (u.float() - v.float()).abs()
+        assert float(d.max()) <= 2.0 ** -6 * float(v.float().abs().max()), "beyond the rounding of split sums"
+    assert torch.equal(a[2], w[2]) and torch.equal(a[3], w[3])     # dA, dB do not come from the GEMM
+    Wb = _oracle_w_bits(orc, c.W, "nf4")
+    sel = np.sort(np.random.default_rng(9).choice(T, size=rows, replace=False)) if rows else None
+    y_ref = orc.lora_fwd(c.x, Wb, c.A, c.B, c.scale, rows=sel)
+    dx_ref = orc.lora_bwd_dx(c.dY, Wb, c.A, c.B, c.scale, rows=sel)
+    y, dX = bf16_tensor_to_f64(a[0]), bf16_tensor_to_f64(a[1])
+    assert_close(y if sel is None else y[sel], y_ref, "y")
+    assert_close(dX if sel is None else dX[sel], dx_ref, "dX")
 
 
 def test_bounded_wait_gives_up_and_the_context_stays_usable(lib, orc):

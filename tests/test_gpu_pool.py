@@ -49,13 +49,15 @@ def _compare(a, b):
 
 
 @pytest.mark.parametrize("name,layers,tokens,fused", [("0.5b", 24, 512, 0), ("8b", 4, 2048, 0), ("8b", 3, 2048, 1),
-                                                     ("72b", 3, 1024, 0)])
+                                                     ("8b", 3, 2048, 2), ("72b", 3, 1024, 0)])
 def test_streamed_equals_resident(lib, name, layers, tokens, fused):
-    lib.set_option(lib.LSN_OPT_FUSED_NF4, fused)
-    try:
+    """Resident through the per-projection calls on one stream, streamed through the layer calls (whose
+    bases arrive dequantised one layer ahead).  With the NF4 conversion inside the GEMM (1: in shared
+    memory, both directions; 2: in tensor memory, forward only, the forward sweep then passes the codes
+    themselves) the fused GEMMs run whole tiles: the other GEMMs then take whole tiles too."""
+    from tests.helpers import lib_option
+    with lib_option(lib, lib.LSN_OPT_FUSED_NF4, fused), lib_option(lib, lib.LSN_OPT_STREAM_K, 0 if fused else 1):
         _streamed_equals_resident(lib, name, layers, tokens)
-    finally:
-        lib.set_option(lib.LSN_OPT_FUSED_NF4, 0)
 
 
 def _streamed_equals_resident(lib, name, layers, tokens):
@@ -375,12 +377,14 @@ def test_grouped_stack_matches_shared_inputs(lib, orc):
     import torch
     from layer_streamed_nf4_b200.stack import Stack
     from tests.helpers import assert_close, bf16_tensor_to_f64
+    from tests.helpers import lib_option
     cfg = synth.STACKS["8b"]
-    shared = Stack(cfg, layers=2, tokens=512, mode="resident", keep_outputs=True, shared_inputs=True)
-    shared.step()
-    grouped = shared.with_inputs(shared_inputs=True, grouped=True, mode="streamed")
-    grouped.step()
-    torch.cuda.synchronize()
+    with lib_option(lib, lib.LSN_OPT_STREAM_K, 0):      # whole tiles: y the same bits grouped or not
+        shared = Stack(cfg, layers=2, tokens=512, mode="resident", keep_outputs=True, shared_inputs=True)
+        shared.step()
+        grouped = shared.with_inputs(shared_inputs=True, grouped=True, mode="streamed")
+        grouped.step()
+        torch.cuda.synchronize()
     grouped.check_status()
     assert all(torch.equal(shared.y[k], grouped.y[k]) for k in shared.y)
     assert all(torch.equal(shared.dA[k], grouped.dA[k]) and torch.equal(shared.dB[k], grouped.dB[k]) for k in shared.dA)
