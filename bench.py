@@ -389,8 +389,10 @@ def run_ours(args):
                                       2: "forward: inside the GEMM (tensor memory); backward: nf4_dequant then "
                                          "bf16 GEMM"}[args.fused_nf4],
                    "programmatic_dependent_launch": not args.no_pdl,
-                   "gemm_schedule": "stream-K where tiles leave the last wave partly empty" if args.stream_k
-                                    else "whole tiles round robin",
+                   "gemm_schedule": ("stream-K where tiles leave the last wave partly empty" if args.stream_k
+                                     else "whole tiles round robin") +
+                                    (", on the fewest SMs for the same rounds" if args.gemm_min_units else ""),
+                   "dequant_spare_sms": args.dequant_spare_sms,
                    "dequant_ahead": st_main.ahead,
                    "l2": "inputs larger than L2 (per step ~11 GB of activations; every layer's NF4 codes read twice)"},
         "pct_bf16_peak": 100 * flop_step / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
@@ -600,6 +602,12 @@ def main():
                     help="NF4 conversion: 0 = nf4_dequant then the bf16 GEMM; 1 = inside the GEMM into shared "
                          "memory (both directions); 2 = inside the forward GEMM into tensor memory")
     ap.add_argument("--no-pdl", action="store_true", help="ordinary launches instead of programmatic dependent ones")
+    ap.add_argument("--gemm-min-units", type=int, default=0, choices=[0, 1],
+                    help="persistent GEMMs on every SM (0, default) or on the fewest SMs that finish in the same "
+                         "number of tile rounds (1)")
+    ap.add_argument("--dequant-spare-sms", type=int, default=0,
+                    help="run the dequantisation-ahead on SMs of its own, sized for this many SMs left free by "
+                         "the GEMMs (0: beside the GEMM CTAs, 2 blocks per SM)")
     ap.add_argument("--stream-k", type=int, default=0, choices=[0, 1],
                     help="GEMM schedule: whole tiles round robin (0, default), or stream-K where tiles leave the "
                          "last wave partly empty (1)")
@@ -608,8 +616,11 @@ def main():
     ap.add_argument("--case", default="", help="profile one 8B projection (q,k,v,o,gate,up,down) instead of the stack")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
-    if args.impl == "ours" and (args.fused_nf4 or args.no_pdl or args.stream_k):
+    if args.impl == "ours" and (args.fused_nf4 or args.no_pdl or args.stream_k or args.gemm_min_units
+                                or args.dequant_spare_sms):
         from layer_streamed_nf4_b200 import lsnf4
+        lsnf4.set_option(lsnf4.LSN_OPT_GEMM_MIN_UNITS, args.gemm_min_units)
+        lsnf4.set_option(lsnf4.LSN_OPT_DEQUANT_SPARE_SMS, args.dequant_spare_sms)
         if args.fused_nf4:
             lsnf4.set_option(lsnf4.LSN_OPT_FUSED_NF4, args.fused_nf4)
         if args.no_pdl:

@@ -357,8 +357,25 @@ lsn_status lsn_timing_read(lsn_kernel_timing* out);
  *                      every kernel still waits for its predecessor to finish
  *                      before it reads or writes global memory.  0: ordinary
  *                      stream-ordered launches.
+ *   LSN_OPT_GEMM_MIN_UNITS 1: a GEMM whose tiles take R rounds over all the
+ *                      SMs runs on the fewest SMs that still finish in R
+ *                      rounds (e.g. 128 tiles of 256 x 256: 64 SM pairs
+ *                      instead of 74), leaving the rest free for work on other
+ *                      streams; 0 (default): one CTA (pair) per SM.
+ *   LSN_OPT_DEQUANT_SPARE_SMS 0 (default); n > 0: nf4_dequant_batch calls with
+ *                      blocks_per_sm = k > 0 launch n * k blocks, each
+ *                      reserving enough shared memory that it never shares an
+ *                      SM with a GEMM CTA: a dequantisation beside GEMMs that
+ *                      leave n SMs free runs on those SMs only.
  */
-typedef enum { LSN_OPT_FUSED_NF4 = 1, LSN_OPT_LAYER_LANES = 2, LSN_OPT_PDL = 3, LSN_OPT_STREAM_K = 4 } lsn_option;
+typedef enum {
+    LSN_OPT_FUSED_NF4 = 1,
+    LSN_OPT_LAYER_LANES = 2,
+    LSN_OPT_PDL = 3,
+    LSN_OPT_STREAM_K = 4,
+    LSN_OPT_GEMM_MIN_UNITS = 5,
+    LSN_OPT_DEQUANT_SPARE_SMS = 6
+} lsn_option;
 lsn_status lsn_set_option(int option, int value);
 int lsn_get_option(int option);
 

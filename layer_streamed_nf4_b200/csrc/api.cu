@@ -849,6 +849,15 @@ lsn_status lsn_set_option(int option, int value) {
         gemm_set_stream_k(value != 0);
         return LSN_OK;
     }
+    if (option == LSN_OPT_GEMM_MIN_UNITS) {
+        gemm_set_min_units(value != 0);
+        return LSN_OK;
+    }
+    if (option == LSN_OPT_DEQUANT_SPARE_SMS) {
+        LSN_CHECK_ARG(value >= 0 && value <= 4096, "lsn_set_option: LSN_OPT_DEQUANT_SPARE_SMS out of range");
+        dequant_set_spare_sms(value);
+        return LSN_OK;
+    }
     return fail(LSN_ERR_INVALID_ARG, "lsn_set_option: unknown option");
 }
 
@@ -857,6 +866,8 @@ int lsn_get_option(int option) {
     if (option == LSN_OPT_LAYER_LANES) return g_layer_lanes.load();
     if (option == LSN_OPT_PDL) return g_pdl.load();
     if (option == LSN_OPT_STREAM_K) return gemm_stream_k() ? 1 : 0;
+    if (option == LSN_OPT_GEMM_MIN_UNITS) return gemm_min_units() ? 1 : 0;
+    if (option == LSN_OPT_DEQUANT_SPARE_SMS) return dequant_spare_sms();
     return -1;
 }
 

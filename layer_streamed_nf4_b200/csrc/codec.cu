@@ -15,6 +15,7 @@
 // Every rounding-sensitive operation uses an explicit IEEE intrinsic
 // (__fdiv_rn, __fsub_rn, __fmul_rn, __fadd_rn) so the compiler can neither
 // contract nor approximate it.
+#include <atomic>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -321,8 +322,28 @@ lsn_status launch_quantize(const float* W, const lsn_nf4_weight* out, void* ws, 
     return LSN_OK;
 }
 
+namespace {
+std::atomic<int> g_spare_sms{0};
+// Dynamic shared memory a dequantisation block reserves when it must run on
+// SMs of its own (LSN_OPT_DEQUANT_SPARE_SMS): with it no block fits beside a
+// GEMM CTA, and at most three fit on an SM.
+constexpr int kDqSpareSmem = 56 * 1024;
+}
+
+void dequant_set_spare_sms(int n) { g_spare_sms.store(n < 0 ? 0 : n); }
+int dequant_spare_sms() { return g_spare_sms.load(); }
+
 lsn_status launch_dequant_batch(int n, const lsn_nf4_weight* const* w, uint16_t* const* out, cudaStream_t st,
                                 int blocks_per_sm) {
+    const int spare = blocks_per_sm > 0 ? dequant_spare_sms() : 0;
+    if (spare > 0) {
+        static std::once_flag once;
+        static cudaError_t attr_err = cudaSuccess;
+        std::call_once(once, [] {
+            attr_err = cudaFuncSetAttribute(nf4_dequant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDqSpareSmem);
+        });
+        if (attr_err != cudaSuccess) return fail_cuda(attr_err, "cudaFuncSetAttribute(dequant smem)");
+    }
     const Nf4Tables& T = nf4_tables();
     DequantParams P;
     std::memcpy(P.level, T.level, sizeof(P.level));
@@ -333,9 +354,11 @@ lsn_status launch_dequant_batch(int n, const lsn_nf4_weight* const* w, uint16_t*
         if (bt.n == 0) return LSN_OK;
         cudaLaunchConfig_t cfg = {};
         int64_t grid = blocks;
-        if (blocks_per_sm > 0 && grid > (int64_t)sm_count() * blocks_per_sm) grid = (int64_t)sm_count() * blocks_per_sm;
+        const int64_t sms = spare > 0 ? spare : sm_count();
+        if (blocks_per_sm > 0 && grid > sms * blocks_per_sm) grid = sms * blocks_per_sm;
         cfg.gridDim = dim3((unsigned)grid);
         cfg.blockDim = dim3(kDqThreads);
+        cfg.dynamicSmemBytes = spare > 0 ? kDqSpareSmem : 0;
         cfg.stream = st;
         cudaLaunchAttribute attr[1];
         cfg.attrs = attr;

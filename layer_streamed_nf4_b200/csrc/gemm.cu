@@ -864,8 +864,8 @@ lsn_status launch_cfg(const AMaps& a, const CUtensorMap& b, const CUtensorMap& l
     });
     if (attr_err != cudaSuccess) return fail_cuda(attr_err, "cudaFuncSetAttribute(gemm smem)");
     const int tiles = ((args.M + C::TILE_M - 1) / C::TILE_M) * ((args.N + BN - 1) / BN);
-    const int units = PAIR ? sm_count() / 2 : sm_count();
-    const int grid = (PAIR ? 2 : 1) * (tiles < units ? tiles : units);
+    const int units = args.sk ? (PAIR ? sm_count() / 2 : sm_count()) : gemm_units(tiles, PAIR);
+    const int grid = (PAIR ? 2 : 1) * units;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(C::THREADS);
@@ -940,8 +940,7 @@ lsn_status launch_gemm_nf4(const uint16_t* A, int64_t lda, const lsn_nf4_weight*
     args.lora_r = r;
     auto launch = [&](auto kernel, int smem_bytes, int threads) -> lsn_status {
         const int tiles = ((args.M + 255) / 256) * ((args.N + 255) / 256);
-        const int units = sm_count() / 2;
-        const int grid = 2 * (tiles < units ? tiles : units);
+        const int grid = 2 * gemm_units(tiles, true);
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)grid);
         cfg.blockDim = dim3((unsigned)threads);
@@ -992,10 +991,25 @@ GemmSplitWs gemm_split_ws(void* base) {
 
 namespace {
 std::atomic<int> g_stream_k{0};
+std::atomic<int> g_min_units{0};
 }
 
 void gemm_set_stream_k(bool on) { g_stream_k.store(on ? 1 : 0); }
 bool gemm_stream_k() { return g_stream_k.load() != 0; }
+void gemm_set_min_units(bool on) { g_min_units.store(on ? 1 : 0); }
+bool gemm_min_units() { return g_min_units.load() != 0; }
+
+// Workers (CTA pairs, or CTAs) of a persistent GEMM over `tiles` whole tiles:
+// with LSN_OPT_GEMM_MIN_UNITS the fewest that still finish in the same number
+// of rounds of tiles as all the SMs would (the rest of the SMs stay free for
+// work on other streams, at no cost to this GEMM); else one per SM (pair).
+int gemm_units(int64_t tiles, bool pair) {
+    const int64_t all = pair ? sm_count() / 2 : sm_count();
+    if (tiles <= 0) return 1;
+    if (!gemm_min_units()) return (int)(tiles < all ? tiles : all);
+    const int64_t rounds = (tiles + all - 1) / all;
+    return (int)((tiles + rounds - 1) / rounds);
+}
 
 lsn_status launch_gemm_grouped(const GemmGroup& g, const uint16_t* B, int64_t ldb, bool b_mn, const uint16_t* LA,
                                const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D,

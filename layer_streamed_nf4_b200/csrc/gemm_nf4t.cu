@@ -17,19 +17,21 @@
 // Tensor memory, 512 columns: the fp32 accumulator [128 lanes x 256 tokens]
 // in columns 0-255, four 128-wide contraction stages of bf16 A in 256-511.
 //
-// Warps (384 threads):
+// Warps (640 threads):
 //   0      x producer: TMA of this CTA's 128 token rows of x per stage (both
 //          CTAs' loads complete on the pair leader's barrier);
 //   1      TMEM allocation; one lane of the leader issues the MMAs;
-//   2..9   converters, then epilogue: warp w owns TMEM lane quadrant w % 4
-//          and NF4 block (w - 2) / 4 of the two in a 128-wide stage; its
+//   2..17  converters, then epilogue.  Converter warp c = w - 2 owns TMEM
+//          lane quadrant w % 4, NF4 block (c / 4) % 2 of the two in a
+//          128-wide stage, and every other stage (c / 8 picks which): its
 //          thread i converts row 32 (w % 4) + i of the CTA's W rows (32 bytes
 //          of codes -> 64 bf16) and stores it with one tcgen05.st of 32
-//          columns.  Once the first stages of the next tile are converted,
-//          the same warps drain the accumulator (a quadrant's two warps take
-//          half of the tokens each);
-//   10     codes producer: TMA of this CTA's 128 W rows x 64 bytes per stage;
-//   11     relay: once the CTA's eight converter warps have written a stage
+//          columns.  Two warp sets on alternate stages give each warp two
+//          stages' time for one stage's conversion.  Once the first stages
+//          of the next tile are converted, the same warps drain the
+//          accumulator (a quadrant's four warps take 64 tokens each);
+//   18     codes producer: TMA of this CTA's 128 W rows x 64 bytes per stage;
+//   19     relay: once the eight converter warps writing a stage are done
 //          (a CTA-local barrier), one arrival on the pair leader's barrier.
 //          The cluster-scope release of that arrival is paid by this thread
 //          alone, not by every converter warp for every stage.
@@ -49,9 +51,16 @@ constexpr int NT_BK = 128;                     // contraction per stage
 constexpr int NT_XSUB = 128 * 64 * 2;          // 128 token rows x 64 bf16 (one 128-byte swizzle atom wide)
 constexpr int NT_XBYTES = 2 * NT_XSUB;         // 32 KB per stage
 constexpr int NT_PBYTES = 128 * 64;            // 128 W rows x 64 bytes of codes: 8 KB per stage
-constexpr int NT_EPI_ROW = 80;                 // transpose tile row: 32 bf16 + 16 bytes of padding
-constexpr int NT_EPI_BYTES = 32 * NT_EPI_ROW;  // one warp's 32 x 32 tile
-constexpr int NT_CONV_WARPS = 8;
+// A warp's 32 x 32 bf16 transpose tile: 32 rows (tokens) of 80 bytes (32 bf16
+// + 16 bytes of padding, so that 8 consecutive rows read as 16-byte chunks
+// fall into distinct banks), rows 16..31 shifted by another 64 bytes (so that
+// the two half-warps, writing rows j and 16 + j, hit distinct banks).
+constexpr int NT_EPI_ROW = 80;
+constexpr int NT_EPI_HALF = 16 * NT_EPI_ROW + 64;
+constexpr int NT_EPI_BYTES = NT_EPI_HALF + 16 * NT_EPI_ROW;
+constexpr int NT_PAR = 2;                      // converter warp sets, taking alternate stages
+constexpr int NT_CONV_PER_STAGE = 8;           // converter warps writing one stage (2 per lane quadrant)
+constexpr int NT_CONV_WARPS = NT_CONV_PER_STAGE * NT_PAR;
 constexpr int NT_THREADS = 64 + 32 * NT_CONV_WARPS + 64;
 constexpr int NT_PPRO_WARP = 2 + NT_CONV_WARPS;
 constexpr int NT_RELAY_WARP = NT_PPRO_WARP + 1;
@@ -121,10 +130,10 @@ __global__ void __launch_bounds__(NT_THREADS, 1)
             mbar_init(&fullX[s], 1);
             mbar_init(&emptyX[s], 1);
             mbar_init(&fullP[s], 1);
-            mbar_init(&emptyP[s], NT_CONV_WARPS);
+            mbar_init(&emptyP[s], NT_CONV_PER_STAGE);
             mbar_init(&readyA[s], 2);
             mbar_init(&emptyA[s], 1);
-            mbar_init(&convDone[s], NT_CONV_WARPS);
+            mbar_init(&convDone[s], NT_CONV_PER_STAGE);
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 2 * NT_CONV_WARPS);
@@ -240,19 +249,22 @@ __global__ void __launch_bounds__(NT_THREADS, 1)
         }
     } else {
         // ------------------------------------------ converters + epilogue --
+        const int cw = warp - 2;                             // converter warp 0 .. NT_CONV_WARPS - 1
         const int q = warp & 3;                              // TMEM lane quadrant
-        const int h = (warp - 2) >> 2;                       // NF4 block of the stage / half of the tokens
+        const int h = (cw >> 2) & 1;                         // NF4 block of the stage
+        const int par = cw >> 3;                             // stages g with g % NT_PAR == par
         const int rloc = q * 32 + lane;                      // W row of the CTA = TMEM lane
         const uint32_t lane_addr = (uint32_t)(q * 32) << 16;
         const float off = *p.absmax_off;
-        uint8_t* tp = epi + (warp - 2) * NT_EPI_BYTES;       // this warp's transpose tile
-        int stage = 0;
-        uint32_t phase = 0, acc_phase = 0;
+        uint8_t* tp = epi + cw * NT_EPI_BYTES;               // this warp's transpose tile
+        uint32_t acc_phase = 0;
         bool bad = false;
         const int first_conv = nkb < NT_STAGES ? nkb : NT_STAGES;   // stages converted before draining
+        const int epi_chunk0 = (h + 2 * par) * (8 / (2 * NT_PAR));  // this warp's 32-token chunks
+        constexpr int kEpiChunks = 8 / (2 * NT_PAR);
 
-        // Drain the accumulator of `tile`: 128 of its 256 tokens (half h) for
-        // the 32 W rows of this warp, transposed to y[token, feature].
+        // Drain the accumulator of `tile`: this warp's chunks of 32 of its 256
+        // tokens for the 32 W rows of its quadrant, transposed to y[token, feature].
         auto epilogue = [&](int tile) -> bool {
             const bool got = mbar_wait(acc_full, acc_phase, abort_flag);
             if (!__all_sync(0xffffffffu, got)) return false;
@@ -261,22 +273,31 @@ __global__ void __launch_bounds__(NT_THREADS, 1)
             const int n_base = (tile % num_w) * 256 + (int)rank * 128 + q * 32;
             const int t_tile = (tile / num_w) * 256;
             #pragma unroll 1
-            for (int c = 4 * h; c < 4 * h + 4; ++c) {
+            for (int c = epi_chunk0; c < epi_chunk0 + kEpiChunks; ++c) {
                 uint32_t v[32];
                 tmem_ld32(tmem_base + lane_addr + NT_ACC_COL + (uint32_t)(c * 32), v);
                 tmem_ld_wait(v);
-                // column `lane` of the 32 x 32 tile: feature n_base + lane, tokens 32c .. 32c+31
+                // Lane i holds feature n_base + i for tokens 32c .. 32c+31.  Lanes 2m and
+                // 2m+1 swap halves, so that the even lane holds features (2m, 2m+1) of
+                // tokens 0..15 and the odd lane those of tokens 16..31, each pair one
+                // 32-bit word of its token's row in the transpose tile.
+                const bool odd = lane & 1;
+                const uint32_t col = (uint32_t)(lane >> 1) * 4;
+                const uint32_t half = odd ? NT_EPI_HALF : 0;
                 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const uint32_t b = pack_bf16x2(__uint_as_float(v[j]), 0.0f) & 0xffffu;
-                    asm volatile("st.shared.u16 [%0], %1;" ::"r"(smem_u32(tp + j * NT_EPI_ROW + lane * 2)),
-                                 "h"((uint16_t)b)
+                for (int j = 0; j < 16; ++j) {
+                    const uint32_t mine = odd ? v[16 + j] : v[j];
+                    const uint32_t other = __shfl_xor_sync(0xffffffffu, odd ? v[j] : v[16 + j], 1);
+                    const uint32_t w = odd ? pack_bf16x2(__uint_as_float(other), __uint_as_float(mine))
+                                           : pack_bf16x2(__uint_as_float(mine), __uint_as_float(other));
+                    asm volatile("st.shared.u32 [%0], %1;" ::"r"(smem_u32(tp + half + j * NT_EPI_ROW + col)), "r"(w)
                                  : "memory");
                 }
                 __syncwarp();
                 const int t = t_tile + c * 32 + lane;        // row `lane`: one token, 32 features
                 if (t < p.M && n_base < p.N) {
-                    const uint4* src = reinterpret_cast<const uint4*>(tp + lane * NT_EPI_ROW);
+                    const uint4* src = reinterpret_cast<const uint4*>(
+                        tp + (lane < 16 ? lane * NT_EPI_ROW : NT_EPI_HALF + (lane - 16) * NT_EPI_ROW));
                     uint4* dst = reinterpret_cast<uint4*>(p.y + (int64_t)t * p.ldy + n_base);
                     #pragma unroll
                     for (int i = 0; i < 4; ++i) dst[i] = src[i];
@@ -289,13 +310,16 @@ __global__ void __launch_bounds__(NT_THREADS, 1)
             return true;
         };
 
-        // Second-level constants of this thread's NF4 block in stage (tile, kb),
-        // fetched two stages ahead of their use.
+        // Second-level constants of this thread's NF4 block at position g of the
+        // worker's stage sequence (tile unit + (g / nkb) nunits, block g % nkb),
+        // fetched one own stage (NT_PAR positions) ahead of their use.
         struct Meta { uint32_t code; float s2; bool ok; };
-        auto fetch = [&](int tl, int kb) -> Meta {
+        auto fetch = [&](int64_t g) -> Meta {
             Meta m{0u, 0.0f, false};
+            const int64_t tl = unit + (g / nkb) * nunits;
+            const int kb = (int)(g % nkb);
             if (tl >= num_tiles || kb >= p.num_kb) return m;
-            const int64_t n = (int64_t)(tl % num_w) * 256 + (int)rank * 128 + rloc;
+            const int64_t n = (tl % num_w) * 256 + (int)rank * 128 + rloc;
             const int64_t b = (int64_t)kb * 2 + h;            // block of the row
             if (n < p.N && b < p.kblk) {
                 const int64_t bi = n * p.kblk + b;
@@ -305,74 +329,71 @@ __global__ void __launch_bounds__(NT_THREADS, 1)
             }
             return m;
         };
-        int ft = unit, fk = 0;
-        auto step = [&]() { if (++fk == nkb) { fk = 0; ft += nunits; } };
-        Meta m0 = fetch(ft, fk);
-        step();
-        Meta m1 = fetch(ft, fk);
-        step();
+        Meta nxt = fetch(par);
 
         int pending = -1;                                     // tile whose accumulator awaits draining
+        int64_t g = 0;                                        // position in the worker's stage sequence
         for (int tile = unit; tile < num_tiles && !bad; tile += nunits) {
             const int64_t n_row = (int64_t)(tile % num_w) * 256 + (int)rank * 128 + rloc;
-            for (int kb = 0; kb < nkb; ++kb) {
-                const Meta cur = m0;
-                m0 = m1;
-                m1 = fetch(ft, fk);
-                step();
-                const bool got = mbar_wait(&fullP[stage], phase, abort_flag) &&
-                                 mbar_wait(&emptyA[stage], phase ^ 1, abort_flag);
-                if (!__all_sync(0xffffffffu, got)) { bad = true; break; }
-                uint32_t v[32];
-                if (kb < p.num_kb) {
-                    // this thread's 32 bytes of codes: half h of its row's 64 bytes
-                    // (64-byte swizzle: 16-byte chunk c of row r at c ^ ((r >> 1) & 3))
-                    const uint8_t* prow = ringP + stage * NT_PBYTES + rloc * 64;
-                    uint4 pk[2];
-                    #pragma unroll
-                    for (int e = 0; e < 2; ++e)
-                        pk[e] = *reinterpret_cast<const uint4*>(prow + (((2 * h + e) ^ ((rloc >> 1) & 3)) << 4));
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&emptyP[stage]);
-                    if (cur.ok) {
-                        const float ah = __fadd_rn(__fmul_rn(dq_s[cur.code], cur.s2), off);
-                        uint32_t lo[4], hi[4];
-                        nf4_scaled_table(p.level, ah, lo, hi);
+            for (int kb = 0; kb < nkb; ++kb, ++g) {
+                const int stage = (int)(g % NT_STAGES);
+                const uint32_t phase = (uint32_t)((g / NT_STAGES) & 1);
+                if ((int)(g % NT_PAR) == par) {
+                    const Meta cur = nxt;
+                    nxt = fetch(g + NT_PAR);
+                    const bool got = mbar_wait(&fullP[stage], phase, abort_flag) &&
+                                     mbar_wait(&emptyA[stage], phase ^ 1, abort_flag);
+                    if (!__all_sync(0xffffffffu, got)) { bad = true; break; }
+                    uint32_t v[32];
+                    if (kb < p.num_kb) {
+                        // this thread's 32 bytes of codes: half h of its row's 64 bytes
+                        // (64-byte swizzle: 16-byte chunk c of row r at c ^ ((r >> 1) & 3))
+                        const uint8_t* prow = ringP + stage * NT_PBYTES + rloc * 64;
+                        uint4 pk[2];
                         #pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const uint32_t w4[4] = {pk[e].x, pk[e].y, pk[e].z, pk[e].w};
+                        for (int e = 0; e < 2; ++e)
+                            pk[e] = *reinterpret_cast<const uint4*>(prow + (((2 * h + e) ^ ((rloc >> 1) & 3)) << 4));
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&emptyP[stage]);
+                        if (cur.ok) {
+                            const float ah = __fadd_rn(__fmul_rn(dq_s[cur.code], cur.s2), off);
+                            uint32_t lo[4], hi[4];
+                            nf4_scaled_table(p.level, ah, lo, hi);
                             #pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const uint4 o = nf4x8_to_bf16(w4[i], lo, hi);
-                                v[16 * e + 4 * i + 0] = o.x;
-                                v[16 * e + 4 * i + 1] = o.y;
-                                v[16 * e + 4 * i + 2] = o.z;
-                                v[16 * e + 4 * i + 3] = o.w;
+                            for (int e = 0; e < 2; ++e) {
+                                const uint32_t w4[4] = {pk[e].x, pk[e].y, pk[e].z, pk[e].w};
+                                #pragma unroll
+                                for (int i = 0; i < 4; ++i) {
+                                    const uint4 o = nf4x8_to_bf16(w4[i], lo, hi);
+                                    v[16 * e + 4 * i + 0] = o.x;
+                                    v[16 * e + 4 * i + 1] = o.y;
+                                    v[16 * e + 4 * i + 2] = o.z;
+                                    v[16 * e + 4 * i + 3] = o.w;
+                                }
                             }
+                        } else {
+                            #pragma unroll
+                            for (int i = 0; i < 32; ++i) v[i] = 0u;
                         }
                     } else {
+                        // LoRA stage: row n of B_lora (r <= 64 bf16) as the A operand, zeros beyond r
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&emptyP[stage]);
                         #pragma unroll
                         for (int i = 0; i < 32; ++i) v[i] = 0u;
+                        if (h == 0 && n_row < p.N) {
+                            const uint32_t* src = reinterpret_cast<const uint32_t*>(p.lora_b + n_row * p.lora_r);
+                            #pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (2 * i < p.lora_r) v[i] = __ldg(src + i);
+                        }
                     }
-                } else {
-                    // LoRA stage: row n of B_lora (r <= 64 bf16) as the A operand, zeros beyond r
+                    tmem_st32(tmem_base + lane_addr + NT_A_COL + (uint32_t)(stage * 64 + h * 32), v);
+                    tmem_st_wait(v);
+                    tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&emptyP[stage]);
-                    #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = 0u;
-                    if (h == 0 && n_row < p.N) {
-                        const uint32_t* src = reinterpret_cast<const uint32_t*>(p.lora_b + n_row * p.lora_r);
-                        #pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            if (2 * i < p.lora_r) v[i] = __ldg(src + i);
-                    }
+                    if (lane == 0) mbar_arrive(&convDone[stage]);
                 }
-                tmem_st32(tmem_base + lane_addr + NT_A_COL + (uint32_t)(stage * 64 + h * 32), v);
-                tmem_st_wait(v);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&convDone[stage]);
-                if (++stage == NT_STAGES) { stage = 0; phase ^= 1; }
                 if (kb == first_conv - 1 && pending >= 0) {
                     if (!epilogue(pending)) { bad = true; break; }
                     pending = -1;
@@ -440,8 +461,7 @@ lsn_status launch_gemm_nf4t(const uint16_t* x, int64_t ldx, const lsn_nf4_weight
     });
     if (attr_err != cudaSuccess) return fail_cuda(attr_err, "cudaFuncSetAttribute(gemm nf4t smem)");
     const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
-    const int units = sm_count() / 2;
-    const int grid = 2 * (int)(tiles < units ? tiles : units);
+    const int grid = 2 * gemm_units(tiles, true);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(NT_THREADS);

@@ -87,6 +87,12 @@ size_t gemm_split_ws_bytes();
 GemmSplitWs gemm_split_ws(void* base);
 void gemm_set_stream_k(bool on);
 bool gemm_stream_k();
+void gemm_set_min_units(bool on);
+bool gemm_min_units();
+int gemm_units(int64_t tiles, bool pair);
+// Dequantisation beside other work (LSN_OPT_DEQUANT_SPARE_SMS).
+void dequant_set_spare_sms(int n);
+int dequant_spare_sms();
 
 // split == NULL: whole tiles round robin (no stream-K scratch).
 lsn_status launch_gemm_grouped(const GemmGroup& g, const uint16_t* B, int64_t ldb, bool b_mn, const uint16_t* LA,

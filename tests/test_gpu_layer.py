@@ -172,6 +172,26 @@ def test_layer_with_tmem_fused_forward(lib, orc):
         assert_close(bf16_tensor_to_f64(o["y"])[rows], orc.lora_fwd(c.x, Wb, c.A, c.B, L.scale, rows=rows), "y")
 
 
+def test_scheduling_options_give_the_same_bits(lib):
+    """GEMMs on the fewest SMs for their number of tile rounds (LSN_OPT_GEMM_MIN_UNITS) and a batched
+    dequantisation confined to SMs of its own (LSN_OPT_DEQUANT_SPARE_SMS) change where work runs, not what
+    it computes: the same bits as the defaults."""
+    import torch
+    from tests.helpers import lib_option
+    L = Layer(lib, SHAPES_8B, 2048, 16, "nf4", seed=9)
+    a = L.layer()
+    with lib_option(lib, lib.LSN_OPT_GEMM_MIN_UNITS, 1):
+        _equal(a, L.layer())
+    outs = [torch.empty((d["N"], d["K"]), dtype=torch.bfloat16, device="cuda") for d in L.p]
+    ref = [torch.empty_like(o) for o in outs]
+    for d, r in zip(L.p, ref):
+        lib.nf4_dequant(d["nf4"].w, r)
+    with lib_option(lib, lib.LSN_OPT_DEQUANT_SPARE_SMS, 12):
+        lib.nf4_dequant_batch([d["nf4"].w for d in L.p], outs, blocks_per_sm=2)
+    torch.cuda.synchronize()
+    assert all(torch.equal(o, r) for o, r in zip(outs, ref))
+
+
 def test_layer_zero_tokens(lib):
     import torch
     L = Layer(lib, SMALL[:2], 0, 16, "nf4")
