@@ -218,7 +218,10 @@ struct DqBatch {
 // a thread makes for one word are passed through a per-warp staging buffer
 // in shared memory (16-byte chunks XOR-swizzled, conflict-free both ways) so
 // that every global store instruction of the warp writes 512 contiguous
-// bytes.  A block covers 1024 consecutive words of one weight.
+// bytes.  A block covers 1024 consecutive words of one weight.  Codes are
+// read and bf16 written with the streaming (evict-first) cache hint: each byte
+// is touched once here, and the GEMMs running beside this kernel keep their
+// operand tiles in L2 (measured 0.2-0.5 ms faster per 8B step).
 constexpr int kDqWarps = kDqThreads / 32;
 
 __device__ __forceinline__ int dq_stage_chunk(int c) { return c ^ ((c >> 3) & 7); }
@@ -254,7 +257,7 @@ __global__ void __launch_bounds__(kDqThreads) nf4_dequant_kernel(const __grid_co
             const int64_t v = v0 + u * kDqThreads;
             const bool ok = v < it.nvec;
             const int64_t b = (ok ? v : 0) >> 1;         // absmax block of the vector
-            p[u] = ok ? __ldg(packed + v) : make_uint4(0, 0, 0, 0);
+            p[u] = ok ? __ldcs(packed + v) : make_uint4(0, 0, 0, 0);
             code[u] = __ldg(absmax_q + b);
             sc[u] = __ldg(s2 + (b >> 8));
         }
@@ -274,7 +277,7 @@ __global__ void __launch_bounds__(kDqThreads) nf4_dequant_kernel(const __grid_co
             #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int c = 32 * i + lane;             // output chunk of the warp, in 16-byte units
-                if (w0 + (c >> 2) < it.nvec) out[4 * w0 + c] = st[dq_stage_chunk(c)];
+                if (w0 + (c >> 2) < it.nvec) __stcs(out + 4 * w0 + c, st[dq_stage_chunk(c)]);
             }
             __syncwarp();
         }
