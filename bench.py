@@ -389,9 +389,7 @@ def run_ours(args):
                                       2: "forward: inside the GEMM (tensor memory); backward: nf4_dequant then "
                                          "bf16 GEMM"}[args.fused_nf4],
                    "programmatic_dependent_launch": not args.no_pdl,
-                   "gemm_schedule": ("stream-K where tiles leave the last wave partly empty" if args.stream_k
-                                     else "whole tiles round robin") +
-                                    (", on the fewest SMs for the same rounds" if args.gemm_min_units else ""),
+                   "gemm_schedule": gemm_schedule(args),
                    "dequant_spare_sms": args.dequant_spare_sms,
                    "dequant_ahead": st_main.ahead,
                    "l2": "inputs larger than L2 (per step ~11 GB of activations; every layer's NF4 codes read twice)"},
@@ -486,6 +484,20 @@ def cpu_baseline(args, sample_rows: int, budget_s: float):
             "sample": f"{rows_done} token rows through the 7 projections of one {cfg.name} layer (fwd+bwd, "
                       f"fp64 oracle, OpenMP); per-step time = layer time x {L} layers (derived, arithmetic)",
             "seconds": t_total}
+
+
+def gemm_schedule(args) -> str:
+    """The GEMM schedule in force, as the library reports it."""
+    from layer_streamed_nf4_b200 import lsnf4
+    if lsnf4.get_option(lsnf4.LSN_OPT_STREAM_K):
+        text = "stream-K where tiles leave the last round partly empty"
+    elif lsnf4.get_option(lsnf4.LSN_OPT_GEMM_TAIL_SPLIT):
+        text = "whole tiles round robin, the last partial round cut into 64-column quanta (128 for MN-major W)"
+    else:
+        text = "whole tiles round robin"
+    if lsnf4.get_option(lsnf4.LSN_OPT_GEMM_MIN_UNITS):
+        text += ", on the fewest SMs for the same rounds"
+    return text
 
 
 def workload_config(cfg, T: int, L: int, slots: int, world: int) -> dict:
@@ -608,6 +620,9 @@ def main():
     ap.add_argument("--dequant-spare-sms", type=int, default=0,
                     help="run the dequantisation-ahead on SMs of its own, sized for this many SMs left free by "
                          "the GEMMs (0: beside the GEMM CTAs, 2 blocks per SM)")
+    ap.add_argument("--tail-split", type=int, default=-1, choices=[-1, 0, 1],
+                    help="GEMM schedule: cut the tiles of a partly filled last round into 64-column quanta shared "
+                         "evenly over the SM pairs (1) or not (0); -1 (default): the library's default")
     ap.add_argument("--stream-k", type=int, default=0, choices=[0, 1],
                     help="GEMM schedule: whole tiles round robin (0, default), or stream-K where tiles leave the "
                          "last wave partly empty (1)")
@@ -617,8 +632,10 @@ def main():
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "ours" and (args.fused_nf4 or args.no_pdl or args.stream_k or args.gemm_min_units
-                                or args.dequant_spare_sms):
+                                or args.dequant_spare_sms or args.tail_split >= 0):
         from layer_streamed_nf4_b200 import lsnf4
+        if args.tail_split >= 0:
+            lsnf4.set_option(lsnf4.LSN_OPT_GEMM_TAIL_SPLIT, args.tail_split)
         lsnf4.set_option(lsnf4.LSN_OPT_GEMM_MIN_UNITS, args.gemm_min_units)
         lsnf4.set_option(lsnf4.LSN_OPT_DEQUANT_SPARE_SMS, args.dequant_spare_sms)
         if args.fused_nf4:

@@ -362,6 +362,13 @@ lsn_status lsn_timing_read(lsn_kernel_timing* out);
  *                      rounds (e.g. 128 tiles of 256 x 256: 64 SM pairs
  *                      instead of 74), leaving the rest free for work on other
  *                      streams; 0 (default): one CTA (pair) per SM.
+ *   LSN_OPT_GEMM_TAIL_SPLIT 1: on the 2-SM GEMM, the output tiles of a last,
+ *                      partly filled round are cut along N into quanta of 64
+ *                      columns (128 for the backward's MN-major W) and shared
+ *                      out evenly, so every SM pair gets about the same number
+ *                      of columns; each output element is still summed over
+ *                      the whole contraction by one SM pair, so the bits do
+ *                      not change.  0 (default): whole tiles round robin.
  *   LSN_OPT_DEQUANT_SPARE_SMS 0 (default); n > 0: nf4_dequant_batch calls with
  *                      blocks_per_sm = k > 0 launch n * k blocks, each
  *                      reserving enough shared memory that it never shares an
@@ -374,7 +381,8 @@ typedef enum {
     LSN_OPT_PDL = 3,
     LSN_OPT_STREAM_K = 4,
     LSN_OPT_GEMM_MIN_UNITS = 5,
-    LSN_OPT_DEQUANT_SPARE_SMS = 6
+    LSN_OPT_DEQUANT_SPARE_SMS = 6,
+    LSN_OPT_GEMM_TAIL_SPLIT = 7
 } lsn_option;
 lsn_status lsn_set_option(int option, int value);
 int lsn_get_option(int option);

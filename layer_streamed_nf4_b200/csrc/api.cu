@@ -853,6 +853,10 @@ lsn_status lsn_set_option(int option, int value) {
         gemm_set_min_units(value != 0);
         return LSN_OK;
     }
+    if (option == LSN_OPT_GEMM_TAIL_SPLIT) {
+        gemm_set_tail_split(value != 0);
+        return LSN_OK;
+    }
     if (option == LSN_OPT_DEQUANT_SPARE_SMS) {
         LSN_CHECK_ARG(value >= 0 && value <= 4096, "lsn_set_option: LSN_OPT_DEQUANT_SPARE_SMS out of range");
         dequant_set_spare_sms(value);
@@ -867,6 +871,7 @@ int lsn_get_option(int option) {
     if (option == LSN_OPT_PDL) return g_pdl.load();
     if (option == LSN_OPT_STREAM_K) return gemm_stream_k() ? 1 : 0;
     if (option == LSN_OPT_GEMM_MIN_UNITS) return gemm_min_units() ? 1 : 0;
+    if (option == LSN_OPT_GEMM_TAIL_SPLIT) return gemm_tail_split() ? 1 : 0;
     if (option == LSN_OPT_DEQUANT_SPARE_SMS) return dequant_spare_sms();
     return -1;
 }

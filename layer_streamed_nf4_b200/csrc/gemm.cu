@@ -88,6 +88,14 @@ struct GemmArgs {
     int64_t sk_per;
     float* sk_part;
     int* sk_cnt;
+    // Tail split (tq > 0; whole-tile schedule of the pair kernel only): the
+    // tiles of the last, partial round, [num_tiles - num_tiles % workers,
+    // num_tiles), are cut along N into quanta of tq columns, and every worker
+    // takes a contiguous run of about the same number of quanta (cut at tile
+    // ends into narrower tiles of whole quanta).  Each output element is still
+    // the same chain of MMAs over the whole contraction, so the bits are those
+    // of whole tiles.
+    int tq;
 };
 
 namespace {
@@ -128,8 +136,9 @@ __device__ __forceinline__ void raise_error(volatile int* abort_flag, int* err, 
     if (err) atomicExch(err, code);
 }
 
-// The work of one worker: (tile, first contraction block, end block) items,
-// either whole tiles round robin (tile = unit, unit + nunits, ...) or the
+// The work of one worker: (tile, columns, first contraction block, end block)
+// items: whole tiles round robin (tile = unit, unit + nunits, ...), then, with
+// the tail split, the worker's run of quanta of the last round's tiles; or the
 // worker's stream-K range.  Stream-K ranges count the base term's blocks
 // only; the LoRA block (the last of a tile's nkb) always goes with the piece
 // that ends the tile, so a tile is cut at the same place with the adapter on
@@ -138,20 +147,46 @@ struct Items {
     bool sk;
     int nkb, nbase, num_tiles, nunits, tile;
     int64_t cur, hi;
-    __device__ Items(const GemmArgs& p, int unit, int nunits_, int num_tiles_, int nkb_)
-        : sk(p.sk != 0), nkb(nkb_), nbase(p.num_kb), num_tiles(num_tiles_), nunits(nunits_), tile(unit) {
+    int full_end, tq, qpt, qcur, qhi, num_m, n, bn;
+    __device__ Items(const GemmArgs& p, int unit, int nunits_, int num_tiles_, int nkb_, int num_m_, int bn_)
+        : sk(p.sk != 0), nkb(nkb_), nbase(p.num_kb), num_tiles(num_tiles_), nunits(nunits_), tile(unit),
+          tq(p.tq), num_m(num_m_), n(p.N), bn(bn_) {
         const int64_t total = (int64_t)num_tiles_ * p.num_kb;
         cur = (int64_t)unit * p.sk_per;
         hi = cur + p.sk_per < total ? cur + p.sk_per : total;
+        full_end = num_tiles_;
+        qpt = qcur = qhi = 0;
+        if (tq > 0) {
+            full_end = num_tiles_ - num_tiles_ % nunits_;
+            qpt = bn_ / tq;
+            const int rq = (num_tiles_ - full_end) * qpt;
+            qcur = (int)((int64_t)unit * rq / nunits_);
+            qhi = (int)((int64_t)(unit + 1) * rq / nunits_);
+        }
     }
-    __device__ bool next(int& t, int& kb0, int& kb1) {
+    // t: tile index; c0, nw: the item's first column inside the tile and its
+    // width (a multiple of 32; columns at or beyond N are never stored).
+    __device__ bool next(int& t, int& c0, int& nw, int& kb0, int& kb1) {
         if (!sk) {
-            if (tile >= num_tiles) return false;
-            t = tile;
             kb0 = 0;
             kb1 = nkb;
-            tile += nunits;
-            return true;
+            if (tile < full_end) {
+                t = tile;
+                c0 = 0;
+                nw = bn;
+                tile += nunits;
+                return true;
+            }
+            while (qcur < qhi) {
+                const int ti = qcur / qpt, qi = qcur - ti * qpt;
+                const int w = qpt - qi < qhi - qcur ? qpt - qi : qhi - qcur;
+                qcur += w;
+                t = full_end + ti;
+                c0 = qi * tq;
+                nw = w * tq;
+                if ((t / num_m) * bn + c0 < n) return true;    // else: quanta past N, nothing to do
+            }
+            return false;
         }
         if (cur >= hi) return false;
         t = (int)(cur / nbase);
@@ -160,6 +195,8 @@ struct Items {
         kb1 = (int64_t)(nbase - kb0) <= left ? nbase : kb0 + (int)left;
         cur += kb1 - kb0;
         if (kb1 == nbase) kb1 = nkb;           // the tile's end: its LoRA block too
+        c0 = 0;
+        nw = bn;
         return true;
     }
 };
@@ -338,12 +375,14 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            Items items(p, unit, nunits, num_tiles, nkb);
-            int tile, kb0, kb1;
-            while (ok && items.next(tile, kb0, kb1)) {
+            Items items(p, unit, nunits, num_tiles, nkb, num_m, BN);
+            int tile, c0, nw, kb0, kb1;
+            while (ok && items.next(tile, c0, nw, kb0, kb1)) {
                 const int mb = tile % num_m, nb = tile / num_m;
                 const int m_row = mb * C::TILE_M + (int)rank * BM;
-                const int n_off = nb * BN + (int)rank * C::B_ROWS;
+                // This CTA's share of the item's B rows (a pair splits N in halves);
+                // the stage is always filled with B_ROWS rows, the MMA reads the share.
+                const int n_off = nb * BN + c0 + (int)rank * (PAIR ? nw / 2 : 0);
                 int ai = 0;                                   // A map of the current K-block
                 for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
@@ -382,12 +421,13 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
-            Items items(p, unit, nunits, num_tiles, nkb);
-            int tile, kb0, kb1;
-            while (ok && items.next(tile, kb0, kb1)) {
+            Items items(p, unit, nunits, num_tiles, nkb, num_m, BN);
+            int tile, c0, nw, kb0, kb1;
+            while (ok && items.next(tile, c0, nw, kb0, kb1)) {
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                const uint32_t idesc = nw == BN ? C::IDESC : idesc_bf16(C::TILE_M, nw, 0, B_MN ? 1 : 0);
                 for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
                     tc_fence_after();
@@ -400,8 +440,8 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
                         const uint64_t bd = B_MN ? smem_desc_sw128(b0 + k * 2048, BK * 128, 1024)
                                                  : smem_desc_sw128(b0 + j * C::B_SUB + kk * 32, 16, 1024);
                         const uint32_t accum = (kb > kb0 || k > 0) ? 1u : 0u;
-                        if constexpr (PAIR) umma_bf16_pair(d_tmem, ad, bd, C::IDESC, accum);
-                        else                umma_bf16(d_tmem, ad, bd, C::IDESC, accum);
+                        if constexpr (PAIR) umma_bf16_pair(d_tmem, ad, bd, idesc, accum);
+                        else                umma_bf16(d_tmem, ad, bd, idesc, accum);
                     }
                     if constexpr (PAIR) umma_commit_pair(&empty[stage]);
                     else                umma_commit(&empty[stage]);
@@ -425,9 +465,9 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
         const int rloc = (int)rank * BM + q * 32 + lane;   // row of the tile this thread drains
         int acc = 0;
         uint32_t acc_phase = 0;
-        Items items(p, unit, nunits, num_tiles, nkb);
-        int tile, kb0, kb1;
-        while (items.next(tile, kb0, kb1)) {
+        Items items(p, unit, nunits, num_tiles, nkb, num_m, BN);
+        int tile, c0, nw, kb0, kb1;
+        while (items.next(tile, c0, nw, kb0, kb1)) {
             const int mb = tile % num_m, nb = tile / num_m;
             const bool got = mbar_wait(&acc_full[acc], acc_phase, abort_flag);
             // With stream-K every epilogue warp takes the same path through the
@@ -442,8 +482,8 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
             const bool split = p.sk && (kb0 > 0 || kb1 < nkb);
             if (!split) {
                 #pragma unroll 1
-                for (int c = 0; c < BN / 32; ++c) {
-                    const int col = nb * BN + c * 32;
+                for (int c = 0; c < nw / 32; ++c) {
+                    const int col = nb * BN + c0 + c * 32;
                     if (col >= p.N) break;
                     uint32_t v[32];
                     tmem_ld32(tm + (uint32_t)(c * 32), v);
@@ -992,12 +1032,15 @@ GemmSplitWs gemm_split_ws(void* base) {
 namespace {
 std::atomic<int> g_stream_k{0};
 std::atomic<int> g_min_units{0};
+std::atomic<int> g_tail_split{0};
 }
 
 void gemm_set_stream_k(bool on) { g_stream_k.store(on ? 1 : 0); }
 bool gemm_stream_k() { return g_stream_k.load() != 0; }
 void gemm_set_min_units(bool on) { g_min_units.store(on ? 1 : 0); }
 bool gemm_min_units() { return g_min_units.load() != 0; }
+void gemm_set_tail_split(bool on) { g_tail_split.store(on ? 1 : 0); }
+bool gemm_tail_split() { return g_tail_split.load() != 0; }
 
 // Workers (CTA pairs, or CTAs) of a persistent GEMM over `tiles` whole tiles:
 // with LSN_OPT_GEMM_MIN_UNITS the fewest that still finish in the same number
@@ -1080,6 +1123,16 @@ lsn_status launch_gemm_grouped(const GemmGroup& g, const uint16_t* B, int64_t ld
             args.sk_part = split->part;
             args.sk_cnt = split->cnt;
         }
+    }
+    // Tail split of the whole-tile schedule (see GemmArgs::tq): quanta of 64
+    // columns (32 B rows per CTA of the pair) for a K-major B; 128 for an
+    // MN-major B, whose per-CTA share must stay whole 64-column swizzle atoms.
+    if (pair && !args.sk && gemm_tail_split()) {
+        const int64_t tiles = ((M + 255) / 256) * ((N + 255) / 256);
+        const int64_t units = gemm_units(tiles, true);
+        const int tq = b_mn ? 128 : 64, qpt = 256 / tq;
+        const int64_t rem = tiles % units;
+        if (tiles > units && rem != 0 && (rem * qpt + units - 1) / units < qpt) args.tq = tq;
     }
     if (pair) return b_mn ? launch_cfg<true, 256, true>(ma, mb, mla, mlb, args, st)
                           : launch_cfg<true, 256, false>(ma, mb, mla, mlb, args, st);

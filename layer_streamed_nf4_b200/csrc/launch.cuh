@@ -89,6 +89,8 @@ void gemm_set_stream_k(bool on);
 bool gemm_stream_k();
 void gemm_set_min_units(bool on);
 bool gemm_min_units();
+void gemm_set_tail_split(bool on);
+bool gemm_tail_split();
 int gemm_units(int64_t tiles, bool pair);
 // Dequantisation beside other work (LSN_OPT_DEQUANT_SPARE_SMS).
 void dequant_set_spare_sms(int n);

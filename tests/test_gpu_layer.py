@@ -173,14 +173,18 @@ def test_layer_with_tmem_fused_forward(lib, orc):
 
 
 def test_scheduling_options_give_the_same_bits(lib):
-    """GEMMs on the fewest SMs for their number of tile rounds (LSN_OPT_GEMM_MIN_UNITS) and a batched
-    dequantisation confined to SMs of its own (LSN_OPT_DEQUANT_SPARE_SMS) change where work runs, not what
-    it computes: the same bits as the defaults."""
+    """GEMMs on the fewest SMs for their number of tile rounds (LSN_OPT_GEMM_MIN_UNITS), the last round's
+    tiles cut into column quanta (LSN_OPT_GEMM_TAIL_SPLIT, either setting) and a batched dequantisation
+    confined to SMs of its own (LSN_OPT_DEQUANT_SPARE_SMS) change where work runs, not what it computes:
+    the same bits as the defaults."""
     import torch
     from tests.helpers import lib_option
     L = Layer(lib, SHAPES_8B, 2048, 16, "nf4", seed=9)
     a = L.layer()
     with lib_option(lib, lib.LSN_OPT_GEMM_MIN_UNITS, 1):
+        _equal(a, L.layer())
+    split = lib.get_option(lib.LSN_OPT_GEMM_TAIL_SPLIT)
+    with lib_option(lib, lib.LSN_OPT_GEMM_TAIL_SPLIT, 1 - split):
         _equal(a, L.layer())
     outs = [torch.empty((d["N"], d["K"]), dtype=torch.bfloat16, device="cuda") for d in L.p]
     ref = [torch.empty_like(o) for o in outs]
@@ -306,7 +310,8 @@ def _run_layer(lib, L, out, groups):
                                           ([(896, 896), (896, 128), (896, 128), (896, 896), (896, 4864),
                                             (896, 4864), (4864, 896)], 512, "bf16")])
 def test_grouped_projections(lib, orc, shapes, T, kind):
-    """Grouped forward: with whole-tile GEMMs the same bits as ungrouped; with the stream-K schedule (whose
+    """Grouped forward: with whole-tile GEMMs the same bits as ungrouped (with the last round's tiles cut into
+    column quanta or not); with the stream-K schedule (whose
     split points depend on the GEMM's shape) within tolerance of the oracle.  Grouped backward: the
     group's dX is the sum of the members' input gradients (checked against the oracle's sum on sampled
     rows); dA, dB the same bits."""
@@ -316,6 +321,12 @@ def test_grouped_projections(lib, orc, shapes, T, kind):
         plain = _run_layer(lib, L, L.outputs(), (0,) * 7)
         grp = _run_layer(lib, L, L.outputs(), GROUPS)
         _equal(grp, plain, ("y", "dA", "dB", "u"))
+        # The other tail-split setting cuts the grouped GEMMs' last rounds differently: the same bits.
+        with lib_option(lib, lib.LSN_OPT_GEMM_TAIL_SPLIT, 1 - lib.get_option(lib.LSN_OPT_GEMM_TAIL_SPLIT)):
+            grp2 = _run_layer(lib, L, L.outputs(), GROUPS)
+        _equal(grp2, grp, ("y", "dA", "dB", "u"))
+        leaders = (0, 3, 4, 6)
+        _equal([grp2[i] for i in leaders], [grp[i] for i in leaders], ("dX",))
     with lib_option(lib, lib.LSN_OPT_STREAM_K, 1):
         plain = _run_layer(lib, L, L.outputs(), (0,) * 7)
         grp = _run_layer(lib, L, L.outputs(), GROUPS)

@@ -284,6 +284,34 @@ def test_stream_k_schedule(lib, orc, T, K, N, rows):
     assert_close(dX if sel is None else dX[sel], dx_ref, "dX")
 
 
+@pytest.mark.parametrize("T,K,N,rows", [(2048, 4096, 4096, 48), (2048, 4096, 14336, 32), (300, 9536, 9536, 0)])
+def test_tail_split_schedule(lib, orc, T, K, N, rows):
+    """The tail split (LSN_OPT_GEMM_TAIL_SPLIT) cuts the tiles of a partly filled last round into column
+    quanta: the 8B q shape (128 pair tiles: 54 tiles in the last round), the 8B gate shape (448 tiles
+    forward: 4 in the last round; its backward fills whole rounds of 128-column quanta and stays whole)
+    and a ragged shape whose last-round tiles are the partial last column block (76 tiles, N = 37.25
+    tiles: three of each tile's four quanta lie past N).  Every output element is still one MMA chain
+    over the whole contraction, so the bits equal the whole-tile schedule's; results match the oracle."""
+    import torch
+    from tests.helpers import lib_option
+    c = synth.linear_case(T, K, N, 16, 32.0, seed=T + K + 2 * N)
+    L = Linear(lib, c, "nf4")
+    with lib_option(lib, lib.LSN_OPT_STREAM_K, 0):
+        with lib_option(lib, lib.LSN_OPT_GEMM_TAIL_SPLIT, 1):
+            a = (L.fwd(), *L.bwd())
+        with lib_option(lib, lib.LSN_OPT_GEMM_TAIL_SPLIT, 0):
+            w = (L.fwd(), *L.bwd())
+    torch.cuda.synchronize()
+    L.status()
+    for name, u, v in zip(("y", "dX", "dA", "dB"), a, w):
+        assert torch.equal(u, v), f"tail split changed {name}"
+    Wb = _oracle_w_bits(orc, c.W, "nf4")
+    sel = np.sort(np.random.default_rng(11).choice(T, size=rows, replace=False)) if rows else None
+    y, dX = bf16_tensor_to_f64(a[0]), bf16_tensor_to_f64(a[1])
+    assert_close(y if sel is None else y[sel], orc.lora_fwd(c.x, Wb, c.A, c.B, c.scale, rows=sel), "y")
+    assert_close(dX if sel is None else dX[sel], orc.lora_bwd_dx(c.dY, Wb, c.A, c.B, c.scale, rows=sel), "dX")
+
+
 def test_bounded_wait_gives_up_and_the_context_stays_usable(lib, orc):
     """A wait on an mbarrier that nothing arrives on ends after its limit with a timeout status (no
     hang), and kernels launched afterwards still compute correct results."""
