@@ -630,3 +630,97 @@ class Stack:
     def check_status(self):
         for ws, ln in zip(self.ws, self.lanes):
             lsnf4.ws_status(ws, ln)
+
+
+class HostIO:
+    """Steps whose inputs come from pinned host memory and whose result goes back to it.
+
+    Each step reads its layer-0 projection inputs from the stack's device tensors (x[0, p]) and leaves its
+    layer-0 input gradients in dX[0, p].  Every step's inputs cross PCIe host-to-device and its result
+    device-to-host, on a copy stream of their own and through device staging buffers, so that the
+    transfers overlap the neighbouring steps' compute: while step k runs, the copy stream brings step k+1's
+    inputs into the input staging buffer and sends step k-1's gradients from the output staging buffer to
+    the host.  The compute stream adds only two device-to-device copies per step (staging -> x[0, p] before
+    the step, dX[0, p] -> staging after it).  The first step's inputs and the last step's result are
+    waited for: `run` returns with every transfer ordered before the compute stream's next work.
+    """
+
+    @staticmethod
+    def inputs_of(stack: "Stack") -> list:
+        """The step's input tensors: x[0, p] of each projection that has its own (q, k, v share one with
+        shared inputs)."""
+        return [stack.x[0, pi] for pi in range(len(stack.proj)) if stack._input_of(pi) == pi]
+
+    @staticmethod
+    def outputs_of(stack: "Stack") -> list:
+        """The step's result: dX[0, p] of each projection that writes one (a group's first member)."""
+        return [stack.dX[0, pi] for pi in range(len(stack.proj)) if stack._leads(pi)]
+
+    @staticmethod
+    def host_buffers(stack: "Stack"):
+        """Pinned host buffers for inputs_of (holding the device inputs' current values) and outputs_of."""
+        h_in = [torch.empty_like(t, device="cpu").pin_memory() for t in HostIO.inputs_of(stack)]
+        for h, t in zip(h_in, HostIO.inputs_of(stack)):
+            h.copy_(t)
+        h_out = [torch.empty_like(t, device="cpu").pin_memory() for t in HostIO.outputs_of(stack)]
+        return h_in, h_out
+
+    def __init__(self, stack: "Stack", h_in, h_out, stream=None):
+        """stream: the stream the steps run on (default: the stack's)."""
+        self.stack = stack
+        self.compute = stream or stack.stream
+        self.copy = torch.cuda.Stream(stack.dev)
+        self.ins = self.inputs_of(stack)
+        self.outs = self.outputs_of(stack)
+        if len(h_in) != len(self.ins) or len(h_out) != len(self.outs):
+            raise ValueError("HostIO: one host buffer per input tensor and per result tensor expected")
+        for h, t in list(zip(h_in, self.ins)) + list(zip(h_out, self.outs)):
+            if h.device.type != "cpu" or not h.is_pinned() or h.shape != t.shape or h.dtype != t.dtype:
+                raise ValueError("HostIO: host buffers must be pinned CPU tensors of the device tensors' shape and "
+                                 "dtype")
+        self.h_in, self.h_out = list(h_in), list(h_out)
+        self.stage_in = [torch.empty_like(t) for t in self.ins]
+        self.stage_out = [torch.empty_like(t) for t in self.outs]
+        self.in_ready, self.in_free = torch.cuda.Event(), torch.cuda.Event()
+        self.out_ready, self.out_free = torch.cuda.Event(), torch.cuda.Event()
+
+    def bytes_in(self) -> int:
+        return sum(h.numel() * h.element_size() for h in self.h_in)
+
+    def bytes_out(self) -> int:
+        return sum(h.numel() * h.element_size() for h in self.h_out)
+
+    def _h2d(self):
+        with torch.cuda.stream(self.copy):
+            for h, s in zip(self.h_in, self.stage_in):
+                s.copy_(h, non_blocking=True)
+            self.in_ready.record(self.copy)
+
+    def run(self, steps: int, step_fn):
+        """`steps` calls of step_fn() on the compute stream, each on inputs copied in from the host and each
+        followed by the copy of its result to the host."""
+        c, cp = self.compute, self.copy
+        cp.wait_stream(c)                          # the staging buffers are free of earlier work
+        self._h2d()
+        for k in range(steps):
+            c.wait_event(self.in_ready)
+            with torch.cuda.stream(c):
+                for s, t in zip(self.stage_in, self.ins):
+                    t.copy_(s, non_blocking=True)
+            self.in_free.record(c)
+            if k + 1 < steps:                      # the next step's inputs, beside this step's compute
+                cp.wait_event(self.in_free)
+                self._h2d()
+            with torch.cuda.stream(c):
+                step_fn()
+                if k > 0:
+                    c.wait_event(self.out_free)    # the previous result has left the staging buffer
+                for t, s in zip(self.outs, self.stage_out):
+                    s.copy_(t, non_blocking=True)
+            self.out_ready.record(c)
+            cp.wait_event(self.out_ready)
+            with torch.cuda.stream(cp):
+                for s, h in zip(self.stage_out, self.h_out):
+                    h.copy_(s, non_blocking=True)
+                self.out_free.record(cp)
+        c.wait_event(self.out_free)                # the last result is on the host

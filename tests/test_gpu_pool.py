@@ -479,3 +479,33 @@ def test_two_holders_keep_the_slot_until_both_release(lib):
         lib.layer_pool_wait_idle(pool, 10000)
     finally:
         lib.layer_pool_destroy(pool)
+
+
+@pytest.mark.parametrize("shared,grouped", [(False, False), (True, True)])
+def test_host_io_steps(lib, shared, grouped):
+    """Steps fed from pinned host memory (stack.HostIO, the bench's end-to-end path): every step takes the
+    host's inputs (here different from the stack's own), its result reaches the host, and that result is
+    bit for bit a plain step's on the same inputs.  With grouped projections there is one host buffer per
+    distinct input and one per group's input gradient."""
+    import torch
+    from layer_streamed_nf4_b200.stack import HostIO, Stack
+    cfg = synth.STACKS["8b"]
+    st = Stack(cfg, layers=3, tokens=512, mode="streamed", n_slots=2, keep_outputs=True, shared_inputs=shared)
+    if grouped:
+        st = st.with_inputs(shared_inputs=True, grouped=True, mode="streamed")
+    h_in, h_out = HostIO.host_buffers(st)
+    assert len(h_in) == (4 if shared else 7) and len(h_out) == (4 if grouped else 7)
+    g = torch.Generator().manual_seed(7)
+    for h in h_in:
+        h.copy_(torch.randn(h.shape, generator=g).to(h.dtype))
+    HostIO(st, h_in, h_out).run(3, st.step)
+    torch.cuda.synchronize()
+    st.check_status()
+    for h, t in zip(h_in, HostIO.inputs_of(st)):
+        assert torch.equal(h, t.cpu()), "the step did not take the host's inputs"
+    got = [h.clone() for h in h_out]
+    st.step()
+    torch.cuda.synchronize()
+    for h, t in zip(got, HostIO.outputs_of(st)):
+        assert torch.equal(h, t.cpu()), "the host result differs from a plain step's"
+    st.close()
