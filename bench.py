@@ -490,6 +490,9 @@ def gemm_schedule(args) -> str:
         text = "whole tiles round robin"
     if lsnf4.get_option(lsnf4.LSN_OPT_GEMM_MIN_UNITS):
         text += ", on the fewest SMs for the same rounds"
+    if lsnf4.get_option(lsnf4.LSN_OPT_LAYER_MERGE):
+        text = ("layer calls: projection 0's GEMM, then projections 1..n-1 as one launch with a balanced "
+                "schedule of whole tiles; single GEMMs: " + text)
     return text
 
 
@@ -613,6 +616,9 @@ def main():
     ap.add_argument("--dequant-spare-sms", type=int, default=0,
                     help="run the dequantisation-ahead on SMs of its own, sized for this many SMs left free by "
                          "the GEMMs (0: beside the GEMM CTAs, 2 blocks per SM)")
+    ap.add_argument("--layer-merge", type=int, default=-1, choices=[-1, 0, 1],
+                    help="run projections 1..n-1 of each layer call as one merged GEMM launch (1) or one launch per "
+                         "projection (0); -1 (default): the library's default")
     ap.add_argument("--tail-split", type=int, default=-1, choices=[-1, 0, 1],
                     help="GEMM schedule: cut the tiles of a partly filled last round into 64-column quanta shared "
                          "evenly over the SM pairs (1) or not (0); -1 (default): the library's default")
@@ -625,8 +631,10 @@ def main():
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "ours" and (args.fused_nf4 or args.no_pdl or args.stream_k or args.gemm_min_units
-                                or args.dequant_spare_sms or args.tail_split >= 0):
+                                or args.dequant_spare_sms or args.tail_split >= 0 or args.layer_merge >= 0):
         from layer_streamed_nf4_b200 import lsnf4
+        if args.layer_merge >= 0:
+            lsnf4.set_option(lsnf4.LSN_OPT_LAYER_MERGE, args.layer_merge)
         if args.tail_split >= 0:
             lsnf4.set_option(lsnf4.LSN_OPT_GEMM_TAIL_SPLIT, args.tail_split)
         lsnf4.set_option(lsnf4.LSN_OPT_GEMM_MIN_UNITS, args.gemm_min_units)

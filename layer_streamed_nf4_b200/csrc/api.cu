@@ -635,6 +635,57 @@ lsn_status build_group_lb(const lsn_lora_proj* p, int i0, int m, int r, bool bwd
     return LSN_OK;
 }
 
+// Whether projections 1..n-1 of an ungrouped layer call run as one merged
+// GEMM launch (LSN_OPT_LAYER_MERGE): all with bf16 bases (and, backward, all
+// asking for dX), at least two, and within the launch's problem and tile
+// limits.
+bool merge_rest(int n, const lsn_lora_proj* p, int64_t T, bool bwd) {
+    if (!gemm_multi() || T <= 0 || n - 1 < 2 || n - 1 > gemm_multi_max_problems()) return false;
+    GemmProblem pr[LSN_LAYER_MAX_PROJ];
+    for (int i = 1; i < n; ++i) {
+        if (p[i].W.kind != LSN_BASE_BF16 || (bwd && !p[i].dX)) return false;
+        pr[i - 1].N = p[i].W.rows;
+    }
+    return gemm_multi_fits(pr, n - 1, T);
+}
+
+// The GEMMs of projections 1..n-1 as one launch: forward y = x W^T + (s u) B^T,
+// backward dX = dY W + (s g) A.
+lsn_status merged_gemms(int n, const lsn_lora_proj* p, int64_t T, int r, const LayerWs& w, bool bwd,
+                        cudaStream_t st) {
+    GemmProblem pr[LSN_LAYER_MAX_PROJ];
+    double flop = 0.0;
+    for (int i = 1; i < n; ++i) {
+        GemmProblem& q = pr[i - 1];
+        const int64_t N = p[i].W.rows, K = p[i].W.cols;
+        const bool lora = !adapter_off(p[i]);
+        q.B = p[i].W.bf16;
+        q.ldb = K;
+        q.LA = lora ? w.s16[i] : nullptr;
+        if (!bwd) {
+            q.A = p[i].x;
+            q.lda = K;
+            q.LB = p[i].B;
+            q.N = N;
+            q.Kc = K;
+            q.D = p[i].y;
+            q.ldd = N;
+            flop += 2.0 * T * N * (double)(K + (lora ? r : 0));
+        } else {
+            q.A = p[i].dY;
+            q.lda = N;
+            q.LB = p[i].A;
+            q.N = K;
+            q.Kc = N;
+            q.D = p[i].dX;
+            q.ldd = K;
+            flop += 2.0 * T * K * (double)(N + (lora ? r : 0));
+        }
+    }
+    TimingScope ts(bwd ? LSN_K_GEMM_BWD : LSN_K_GEMM_FWD, flop, st);
+    return launch_gemm_multi(pr, n - 1, bwd, T, r, w.err, st);
+}
+
 lsn_status lora_layer_fwd(int n, const lsn_lora_proj* p, int64_t T, int r, float scale, void* ws, size_t ws_bytes,
                           lsn_stream_t stream) {
     NvtxRange nvtx("lora_layer_fwd");
@@ -683,7 +734,15 @@ lsn_status lora_layer_fwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
         if ((s = layer_dequant(n, p, deq, w, lanes.main())) != LSN_OK) return s;
         if ((s = lanes.barrier()) != LSN_OK) return s;
     }
+    // Merged: after the first GEMM, the other projections' GEMMs as one
+    // launch on the side lane, right behind their down projections (so it
+    // takes the SMs the first GEMM's last round leaves free).
+    const bool merge = early && merge_rest(n, p, T, false);
     for (int k = 0; k < g.n; ++k) {
+        if (merge && k == 1) {
+            if ((s = merged_gemms(n, p, T, r, w, false, lanes.side())) != LSN_OK) return s;
+            break;
+        }
         if (early && k == 1 && (s = lanes.main_waits_side()) != LSN_OK) return s;
         const int i = g.first[k], m = g.count[k];
         const int64_t K = p[i].W.cols;
@@ -792,11 +851,19 @@ lsn_status lora_layer_bwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
     }
     if ((s = timed_tgrad_batch(nt, tg, r, lanes.side())) != LSN_OK) return s;
     if (T > 0) {
+        // Merged: after the first GEMM, the other projections' input-gradient
+        // GEMMs as one launch on the main lane (the token reductions keep the
+        // side lane).
+        const bool merge = early && merge_rest(n, p, T, true);
         for (int k = 0, j = 0; k < g.n; ++k) {
             const int i = g.first[k], m = g.count[k];
             if (!p[i].dX) continue;
             const int64_t K = p[i].W.cols;
             if (early && j == 1 && (s = lanes.main_waits_mark()) != LSN_OK) return s;   // the other g
+            if (merge && j == 1) {
+                if ((s = merged_gemms(n, p, T, r, w, true, lanes.main())) != LSN_OK) return s;
+                break;
+            }
             const GemmSplitWs* sp = &w.split[j & 1];
             const cudaStream_t gs = (j++ & 1) ? lanes.side() : lanes.main();
             const int ri = adapter_off(p[i]) ? 0 : r;
@@ -857,6 +924,10 @@ lsn_status lsn_set_option(int option, int value) {
         gemm_set_tail_split(value != 0);
         return LSN_OK;
     }
+    if (option == LSN_OPT_LAYER_MERGE) {
+        gemm_set_multi(value != 0);
+        return LSN_OK;
+    }
     if (option == LSN_OPT_DEQUANT_SPARE_SMS) {
         LSN_CHECK_ARG(value >= 0 && value <= 4096, "lsn_set_option: LSN_OPT_DEQUANT_SPARE_SMS out of range");
         dequant_set_spare_sms(value);
@@ -872,6 +943,7 @@ int lsn_get_option(int option) {
     if (option == LSN_OPT_STREAM_K) return gemm_stream_k() ? 1 : 0;
     if (option == LSN_OPT_GEMM_MIN_UNITS) return gemm_min_units() ? 1 : 0;
     if (option == LSN_OPT_GEMM_TAIL_SPLIT) return gemm_tail_split() ? 1 : 0;
+    if (option == LSN_OPT_LAYER_MERGE) return gemm_multi() ? 1 : 0;
     if (option == LSN_OPT_DEQUANT_SPARE_SMS) return dequant_spare_sms();
     return -1;
 }

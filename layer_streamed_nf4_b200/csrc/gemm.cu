@@ -34,9 +34,13 @@
 //              let the epilogue of tile i overlap the main loop of tile i+1.
 // Every wait is bounded; a wait that runs out sets *err and the CTA winds
 // down (after letting its issued copies and MMAs finish) instead of hanging.
+#include <algorithm>
 #include <atomic>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <type_traits>
+#include <vector>
 
 #include "common.cuh"
 #include "launch.cuh"
@@ -98,6 +102,35 @@ struct GemmArgs {
     int tq;
 };
 
+// Several independent GEMMs of one shape family (same M and contraction
+// layout, e.g. the projections of a decoder layer) in one persistent launch:
+// problem i has its own A, B, LA and LB tensor maps, N, contraction blocks,
+// LoRA MMAs and output.  The launch's tiles are numbered problem after
+// problem (tile0[i] .. tile0[i+1]-1 belong to problem i, M-fastest inside a
+// problem), and worker (CTA pair) u takes tile[start[u] .. start[u+1]) in
+// that order: a schedule made on the host that balances the workers' summed
+// tile costs (tiles of different problems can differ in contraction length).
+// Every tile is whole and computed by one worker, so each output element is
+// the same chain of MMAs as in a launch of its problem alone.
+constexpr int kMultiMaxProb = 8;
+constexpr int kMultiMaxUnits = 80;
+constexpr int kMultiMaxTiles = 2048;
+struct MultiProbs {
+    CUtensorMap a[kMultiMaxProb], b[kMultiMaxProb], la[kMultiMaxProb], lb[kMultiMaxProb];
+    int nprob;
+    int tile0[kMultiMaxProb + 1];
+    int N[kMultiMaxProb];
+    int num_kb[kMultiMaxProb];
+    int lora_k16[kMultiMaxProb];
+    uint16_t* D[kMultiMaxProb];
+    int64_t ldd[kMultiMaxProb];
+    uint16_t start[kMultiMaxUnits + 1];
+    uint16_t tile[kMultiMaxTiles];
+};
+struct NoMulti {
+    int unused;
+};
+
 namespace {
 
 // Tile geometry.  A stage holds a 128-wide slice of the contraction as two
@@ -148,9 +181,19 @@ struct Items {
     int nkb, nbase, num_tiles, nunits, tile;
     int64_t cur, hi;
     int full_end, tq, qpt, qcur, qhi, num_m, n, bn;
-    __device__ Items(const GemmArgs& p, int unit, int nunits_, int num_tiles_, int nkb_, int num_m_, int bn_)
+    const MultiProbs* mp;      // several problems: the worker's tile list (else nullptr)
+    int prob;                  // problem of the last item (0 with one problem)
+    __device__ Items(const GemmArgs& p, int unit, int nunits_, int num_tiles_, int nkb_, int num_m_, int bn_,
+                     const MultiProbs* mp_ = nullptr)
         : sk(p.sk != 0), nkb(nkb_), nbase(p.num_kb), num_tiles(num_tiles_), nunits(nunits_), tile(unit),
-          tq(p.tq), num_m(num_m_), n(p.N), bn(bn_) {
+          tq(p.tq), num_m(num_m_), n(p.N), bn(bn_), mp(mp_), prob(0) {
+        if (mp) {                              // tile list positions [cur, hi)
+            cur = mp->start[unit];
+            hi = mp->start[unit + 1];
+            full_end = 0;
+            qpt = qcur = qhi = 0;
+            return;
+        }
         const int64_t total = (int64_t)num_tiles_ * p.num_kb;
         cur = (int64_t)unit * p.sk_per;
         hi = cur + p.sk_per < total ? cur + p.sk_per : total;
@@ -167,6 +210,19 @@ struct Items {
     // t: tile index; c0, nw: the item's first column inside the tile and its
     // width (a multiple of 32; columns at or beyond N are never stored).
     __device__ bool next(int& t, int& c0, int& nw, int& kb0, int& kb1) {
+        if (mp) {
+            if (cur >= hi) return false;
+            const int g = mp->tile[cur++];
+            int pi = 0;
+            while (pi + 1 < mp->nprob && g >= mp->tile0[pi + 1]) ++pi;
+            prob = pi;
+            t = g - mp->tile0[pi];
+            c0 = 0;
+            nw = bn;
+            kb0 = 0;
+            kb1 = mp->num_kb[pi] + (mp->lora_k16[pi] > 0 ? 1 : 0);
+            return true;
+        }
         if (!sk) {
             kb0 = 0;
             kb1 = nkb;
@@ -314,12 +370,17 @@ struct AMaps {
     CUtensorMap m[kMaxSeg];
 };
 
-template <bool PAIR, int BN, bool B_MN>
+template <bool MULTI>
+using MultiParam = std::conditional_t<MULTI, MultiProbs, NoMulti>;
+
+template <bool PAIR, int BN, bool B_MN, bool MULTI>
 __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
     lsn_gemm_kernel(const __grid_constant__ AMaps tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmLA, const __grid_constant__ CUtensorMap tmLB,
-                    const __grid_constant__ GemmArgs p) {
+                    const __grid_constant__ GemmArgs p, const __grid_constant__ MultiParam<MULTI> mpar) {
     using C = Cfg<PAIR, BN, B_MN>;
+    const MultiProbs* mp = nullptr;
+    if constexpr (MULTI) mp = &mpar;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::STAGE_BYTES);
@@ -353,9 +414,17 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
         fence_mbar_init();
     }
     if (warp == 0 && lane == 0) {
-        for (int i = 0; i < p.na; ++i) tma_prefetch_desc(&tmA.m[i]);
-        tma_prefetch_desc(&tmB);
-        if (p.lora_k16 > 0) { tma_prefetch_desc(&tmLA); tma_prefetch_desc(&tmLB); }
+        if constexpr (MULTI) {
+            for (int i = 0; i < mp->nprob; ++i) {
+                tma_prefetch_desc(&mp->a[i]);
+                tma_prefetch_desc(&mp->b[i]);
+                if (mp->lora_k16[i] > 0) { tma_prefetch_desc(&mp->la[i]); tma_prefetch_desc(&mp->lb[i]); }
+            }
+        } else {
+            for (int i = 0; i < p.na; ++i) tma_prefetch_desc(&tmA.m[i]);
+            tma_prefetch_desc(&tmB);
+            if (p.lora_k16 > 0) { tma_prefetch_desc(&tmLA); tma_prefetch_desc(&tmLB); }
+        }
     }
     if (warp == 1) {
         if constexpr (PAIR) { tmem_alloc_pair(tmem_holder, C::TMEM_COLS); tmem_relinquish_pair(); }
@@ -375,9 +444,11 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            Items items(p, unit, nunits, num_tiles, nkb, num_m, BN);
+            Items items(p, unit, nunits, num_tiles, nkb, num_m, BN, mp);
             int tile, c0, nw, kb0, kb1;
             while (ok && items.next(tile, c0, nw, kb0, kb1)) {
+                const int pi = items.prob;
+                const int nbase = MULTI ? mp->num_kb[pi] : p.num_kb;
                 const int mb = tile % num_m, nb = tile / num_m;
                 const int m_row = mb * C::TILE_M + (int)rank * BM;
                 // This CTA's share of the item's B rows (a pair splits N in halves);
@@ -388,12 +459,21 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
                     if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag)) { ok = false; break; }
                     uint8_t* sA = smem + stage * C::STAGE_BYTES;
                     uint8_t* sB = sA + C::A_BYTES;
-                    const bool lora = kb >= p.num_kb;
-                    while (!lora && ai + 1 < p.na && kb >= p.a_kb[ai + 1]) ++ai;
-                    const CUtensorMap* ma = lora ? &tmLA : &tmA.m[ai];
-                    const CUtensorMap* mbp = lora ? &tmLB : &tmB;
+                    const bool lora = kb >= nbase;
+                    const CUtensorMap* ma;
+                    const CUtensorMap* mbp;
+                    int ka;
                     const int kc = lora ? 0 : kb * BK;                       // contraction coordinate of B
-                    const int ka = lora ? 0 : (kb - p.a_kb[ai]) * BK;        // ... and of the A map
+                    if constexpr (MULTI) {
+                        ma = lora ? &mp->la[pi] : &mp->a[pi];
+                        mbp = lora ? &mp->lb[pi] : &mp->b[pi];
+                        ka = kc;
+                    } else {
+                        while (!lora && ai + 1 < p.na && kb >= p.a_kb[ai + 1]) ++ai;
+                        ma = lora ? &tmLA : &tmA.m[ai];
+                        mbp = lora ? &tmLB : &tmB;
+                        ka = lora ? 0 : (kb - p.a_kb[ai]) * BK;              // ... and of the A map
+                    }
                     uint32_t fbar = smem_u32(&full[stage]);
                     if constexpr (PAIR) fbar = mapa_shared(fbar, 0);
                     if (leader) mbar_arrive_expect_tx(&full[stage], (PAIR ? 2 : 1) * (C::A_BYTES + C::B_BYTES));
@@ -421,9 +501,11 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
             int stage = 0, acc = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
-            Items items(p, unit, nunits, num_tiles, nkb, num_m, BN);
+            Items items(p, unit, nunits, num_tiles, nkb, num_m, BN, mp);
             int tile, c0, nw, kb0, kb1;
             while (ok && items.next(tile, c0, nw, kb0, kb1)) {
+                const int nbase = MULTI ? mp->num_kb[items.prob] : p.num_kb;
+                const int lk16 = MULTI ? mp->lora_k16[items.prob] : p.lora_k16;
                 if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1, abort_flag)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
@@ -433,7 +515,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(smem + stage * C::STAGE_BYTES);
                     const uint32_t b0 = a0 + C::A_BYTES;
-                    const int nk = (kb < p.num_kb) ? BK / 16 : p.lora_k16;
+                    const int nk = (kb < nbase) ? BK / 16 : lk16;
                     for (int k = 0; k < nk; ++k) {
                         const int j = k >> 2, kk = k & 3;       // sub-tile, step inside it
                         const uint64_t ad = smem_desc_sw128(a0 + j * C::A_SUB + kk * 32, 16, 1024);
@@ -465,10 +547,11 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
         const int rloc = (int)rank * BM + q * 32 + lane;   // row of the tile this thread drains
         int acc = 0;
         uint32_t acc_phase = 0;
-        Items items(p, unit, nunits, num_tiles, nkb, num_m, BN);
+        Items items(p, unit, nunits, num_tiles, nkb, num_m, BN, mp);
         int tile, c0, nw, kb0, kb1;
         while (items.next(tile, c0, nw, kb0, kb1)) {
             const int mb = tile % num_m, nb = tile / num_m;
+            const int n_out = MULTI ? mp->N[items.prob] : p.N;
             const bool got = mbar_wait(&acc_full[acc], acc_phase, abort_flag);
             // With stream-K every epilogue warp takes the same path through the
             // named barriers below, so they decide together.
@@ -484,7 +567,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
                 #pragma unroll 1
                 for (int c = 0; c < nw / 32; ++c) {
                     const int col = nb * BN + c0 + c * 32;
-                    if (col >= p.N) break;
+                    if (col >= n_out) break;
                     uint32_t v[32];
                     tmem_ld32(tm + (uint32_t)(c * 32), v);
                     tmem_ld_wait(v);
@@ -492,7 +575,10 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
                         float f[32];
                         #pragma unroll
                         for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
-                        store_bf16x32(out_ptr(p, row, col), f);
+                        uint16_t* dst;
+                        if constexpr (MULTI) dst = mp->D[items.prob] + (int64_t)row * mp->ldd[items.prob] + col;
+                        else                 dst = out_ptr(p, row, col);
+                        store_bf16x32(dst, f);
                     }
                 }
                 tc_fence_before();
@@ -892,19 +978,20 @@ lsn_status make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t out
     return LSN_OK;
 }
 
-template <bool PAIR, int BN, bool B_MN>
+template <bool PAIR, int BN, bool B_MN, bool MULTI = false>
 lsn_status launch_cfg(const AMaps& a, const CUtensorMap& b, const CUtensorMap& la, const CUtensorMap& lb,
-                      const GemmArgs& args, cudaStream_t st) {
+                      const GemmArgs& args, cudaStream_t st, const MultiParam<MULTI>& mpar = {}, int multi_units = 0) {
     using C = Cfg<PAIR, BN, B_MN>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(lsn_gemm_kernel<PAIR, BN, B_MN>,
+        attr_err = cudaFuncSetAttribute(lsn_gemm_kernel<PAIR, BN, B_MN, MULTI>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     });
     if (attr_err != cudaSuccess) return fail_cuda(attr_err, "cudaFuncSetAttribute(gemm smem)");
     const int tiles = ((args.M + C::TILE_M - 1) / C::TILE_M) * ((args.N + BN - 1) / BN);
-    const int units = args.sk ? (PAIR ? sm_count() / 2 : sm_count()) : gemm_units(tiles, PAIR);
+    const int units = MULTI ? multi_units
+                            : args.sk ? (PAIR ? sm_count() / 2 : sm_count()) : gemm_units(tiles, PAIR);
     const int grid = (PAIR ? 2 : 1) * units;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
@@ -923,7 +1010,7 @@ lsn_status launch_cfg(const AMaps& a, const CUtensorMap& b, const CUtensorMap& l
     na += pdl_attr(&attr[na]);
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    LSN_CUDA_TRY(cudaLaunchKernelEx(&cfg, lsn_gemm_kernel<PAIR, BN, B_MN>, a, b, la, lb, args));
+    LSN_CUDA_TRY(cudaLaunchKernelEx(&cfg, lsn_gemm_kernel<PAIR, BN, B_MN, MULTI>, a, b, la, lb, args, mpar));
     return LSN_OK;
 }
 
@@ -1033,6 +1120,7 @@ namespace {
 std::atomic<int> g_stream_k{0};
 std::atomic<int> g_min_units{0};
 std::atomic<int> g_tail_split{0};
+std::atomic<int> g_multi{0};
 }
 
 void gemm_set_stream_k(bool on) { g_stream_k.store(on ? 1 : 0); }
@@ -1041,6 +1129,8 @@ void gemm_set_min_units(bool on) { g_min_units.store(on ? 1 : 0); }
 bool gemm_min_units() { return g_min_units.load() != 0; }
 void gemm_set_tail_split(bool on) { g_tail_split.store(on ? 1 : 0); }
 bool gemm_tail_split() { return g_tail_split.load() != 0; }
+void gemm_set_multi(bool on) { g_multi.store(on ? 1 : 0); }
+bool gemm_multi() { return g_multi.load() != 0; }
 
 // Workers (CTA pairs, or CTAs) of a persistent GEMM over `tiles` whole tiles:
 // with LSN_OPT_GEMM_MIN_UNITS the fewest that still finish in the same number
@@ -1138,6 +1228,115 @@ lsn_status launch_gemm_grouped(const GemmGroup& g, const uint16_t* B, int64_t ld
                           : launch_cfg<true, 256, false>(ma, mb, mla, mlb, args, st);
     return b_mn ? launch_cfg<false, 128, true>(ma, mb, mla, mlb, args, st)
                 : launch_cfg<false, 128, false>(ma, mb, mla, mlb, args, st);
+}
+
+// ------------------------------------------------------ several problems --
+
+namespace {
+
+// A balanced static schedule of whole tiles: tiles in decreasing cost
+// (contraction blocks, the LoRA block included), each given to the worker with
+// the least summed cost so far (lowest index on ties).  Depends on the shapes
+// only, so it is computed once per shape family and kept.
+struct MultiSched {
+    std::vector<uint16_t> start, tile;
+};
+
+const MultiSched& multi_schedule(int units, int num_m, const int* ntiles, const int* cost, int n) {
+    static std::mutex mu;
+    static std::map<std::vector<int>, MultiSched> cache;
+    std::vector<int> key{units, num_m, n};
+    for (int i = 0; i < n; ++i) { key.push_back(ntiles[i]); key.push_back(cost[i]); }
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+    std::vector<int> order(n), first(n + 1, 0);
+    for (int i = 0; i < n; ++i) { order[i] = i; first[i + 1] = first[i] + ntiles[i]; }
+    std::stable_sort(order.begin(), order.end(), [&](int a, int b) { return cost[a] > cost[b]; });
+    std::vector<int64_t> load(units, 0);
+    std::vector<std::vector<int>> lists(units);
+    for (int i : order) {
+        for (int t = 0; t < ntiles[i]; ++t) {
+            int u = 0;
+            for (int v = 1; v < units; ++v)
+                if (load[v] < load[u]) u = v;
+            load[u] += cost[i];
+            lists[u].push_back(first[i] + t);
+        }
+    }
+    MultiSched s;
+    s.start.push_back(0);
+    for (int u = 0; u < units; ++u) {
+        for (int t : lists[u]) s.tile.push_back((uint16_t)t);
+        s.start.push_back((uint16_t)s.tile.size());
+    }
+    return cache.emplace(std::move(key), std::move(s)).first->second;
+}
+
+}  // namespace
+
+int gemm_multi_max_problems() { return kMultiMaxProb; }
+
+bool gemm_multi_fits(const GemmProblem* pr, int n, int64_t M) {
+    if (n < 1 || n > kMultiMaxProb || M <= 0 || sm_count() / 2 > kMultiMaxUnits) return false;
+    int64_t tiles = 0;
+    const int64_t num_m = (M + 255) / 256;
+    for (int i = 0; i < n; ++i) tiles += num_m * ((pr[i].N + 255) / 256);
+    return tiles <= kMultiMaxTiles;
+}
+
+lsn_status launch_gemm_multi(const GemmProblem* pr, int n, bool b_mn, int64_t M, int r, int* err,
+                             cudaStream_t st) {
+    if (!gemm_multi_fits(pr, n, M)) return fail(LSN_ERR_INVALID_ARG, "multi-problem GEMM: too many problems or tiles");
+    MultiProbs mp{};
+    mp.nprob = n;
+    const int num_m = (int)((M + 255) / 256);
+    int ntiles[kMultiMaxProb], cost[kMultiMaxProb];
+    lsn_status s;
+    for (int i = 0; i < n; ++i) {
+        const GemmProblem& q = pr[i];
+        const int ri = q.LA ? r : 0;
+        if ((s = make_map(&mp.a[i], q.A, q.Kc, M, q.lda, SUB, BM)) != LSN_OK) return s;
+        if (!b_mn) {
+            if ((s = make_map(&mp.b[i], q.B, q.Kc, q.N, q.ldb, SUB, 128)) != LSN_OK) return s;
+        } else {
+            if ((s = make_map(&mp.b[i], q.B, q.N, q.Kc, q.ldb, 64, BK)) != LSN_OK) return s;
+        }
+        if (ri > 0) {
+            if ((s = make_map(&mp.la[i], q.LA, ri, M, ri, SUB, BM)) != LSN_OK) return s;
+            if (!b_mn) {
+                if ((s = make_map(&mp.lb[i], q.LB, ri, q.N, ri, SUB, 128)) != LSN_OK) return s;
+            } else {
+                if ((s = make_map(&mp.lb[i], q.LB, q.N, ri, q.N, 64, BK)) != LSN_OK) return s;
+            }
+        } else {                                        // no LoRA term: never read
+            mp.la[i] = mp.a[i];
+            mp.lb[i] = mp.b[i];
+        }
+        mp.N[i] = (int)q.N;
+        mp.num_kb[i] = (int)((q.Kc + BK - 1) / BK);
+        mp.lora_k16[i] = (ri + 15) / 16;
+        mp.D[i] = q.D;
+        mp.ldd[i] = q.ldd;
+        ntiles[i] = num_m * (int)((q.N + 255) / 256);
+        cost[i] = mp.num_kb[i] + (ri > 0 ? 1 : 0);
+        mp.tile0[i + 1] = mp.tile0[i] + ntiles[i];
+    }
+    int units = sm_count() / 2;
+    if (mp.tile0[n] < units) units = mp.tile0[n];
+    if (units < 1) return LSN_OK;
+    const MultiSched& sc = multi_schedule(units, num_m, ntiles, cost, n);
+    std::copy(sc.start.begin(), sc.start.end(), mp.start);
+    std::copy(sc.tile.begin(), sc.tile.end(), mp.tile);
+    GemmArgs args{};
+    args.M = (int)M;
+    args.N = 0;
+    args.err = err;
+    args.na = 1;
+    AMaps ma;
+    for (int i = 0; i < kMaxSeg; ++i) ma.m[i] = mp.a[0];
+    return b_mn ? launch_cfg<true, 256, true, true>(ma, mp.b[0], mp.la[0], mp.lb[0], args, st, mp, units)
+                : launch_cfg<true, 256, false, true>(ma, mp.b[0], mp.la[0], mp.lb[0], args, st, mp, units);
 }
 
 lsn_status launch_gemm(const uint16_t* A, int64_t lda, const uint16_t* B, int64_t ldb, bool b_mn, const uint16_t* LA,

@@ -96,6 +96,31 @@ int gemm_units(int64_t tiles, bool pair);
 void dequant_set_spare_sms(int n);
 int dequant_spare_sms();
 
+// One of several independent GEMMs launched together (launch_gemm_multi): the
+// arguments of launch_gemm for one problem, on the 2-SM kernel; LA == NULL:
+// no LoRA term.
+struct GemmProblem {
+    const uint16_t* A = nullptr;
+    int64_t lda = 0;
+    const uint16_t* B = nullptr;
+    int64_t ldb = 0;
+    const uint16_t* LA = nullptr;
+    const uint16_t* LB = nullptr;
+    int64_t N = 0, Kc = 0;
+    uint16_t* D = nullptr;
+    int64_t ldd = 0;
+};
+int gemm_multi_max_problems();
+// Whether n problems of M rows fit one launch (problem and tile limits).
+bool gemm_multi_fits(const GemmProblem* pr, int n, int64_t M);
+// D_i = A_i . op(B_i) + LA_i . op(LB_i) for every problem i, one persistent
+// launch with a balanced static tile schedule (b_mn as for launch_gemm; all
+// problems share M and r).
+lsn_status launch_gemm_multi(const GemmProblem* pr, int n, bool b_mn, int64_t M, int r, int* err,
+                             cudaStream_t st);
+void gemm_set_multi(bool on);
+bool gemm_multi();
+
 // split == NULL: whole tiles round robin (no stream-K scratch).
 lsn_status launch_gemm_grouped(const GemmGroup& g, const uint16_t* B, int64_t ldb, bool b_mn, const uint16_t* LA,
                                const uint16_t* LB, int r, int64_t M, int64_t N, int64_t Kc, uint16_t* D,

@@ -34,6 +34,7 @@ LSN_OPT_STREAM_K = 4
 LSN_OPT_GEMM_MIN_UNITS = 5
 LSN_OPT_DEQUANT_SPARE_SMS = 6
 LSN_OPT_GEMM_TAIL_SPLIT = 7
+LSN_OPT_LAYER_MERGE = 8
 
 STATUS_NAMES = {0: "LSN_OK", 1: "LSN_ERR_INVALID_ARG", 2: "LSN_ERR_CUDA", 3: "LSN_ERR_NO_MEMORY",
                 4: "LSN_ERR_TIMEOUT", 5: "LSN_ERR_UNSUPPORTED", 6: "LSN_ERR_STATE"}

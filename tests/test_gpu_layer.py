@@ -72,12 +72,15 @@ class Layer:
             lib.ws_status(ws)
         return out
 
-    def layer(self, keep_u=True, accumulate=False, out=None):
+    def layer(self, keep_u=True, accumulate=False, out=None, off=()):
+        """One lora_layer_fwd + lora_layer_bwd over the projections; those in `off` with the adapter off."""
         import torch
         lib = self.lib
         out = out or self.outputs()
         projs = [lib.lora_proj(d["base"], d["x"], d["A"], d["B"], y=o["y"], dY=d["dY"], dX=o["dX"], dA=o["dA"],
-                               dB=o["dB"], u=o["u"] if keep_u else None) for d, o in zip(self.p, out)]
+                               dB=o["dB"], u=o["u"] if keep_u else None) if i not in off else
+                 lib.lora_proj(d["base"], d["x"], None, None, y=o["y"], dY=d["dY"], dX=o["dX"])
+                 for i, (d, o) in enumerate(zip(self.p, out))]
         arr = lib.proj_array(projs)
         n = lib.layer_ws_bytes(arr, self.T, self.r)
         ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
@@ -194,6 +197,34 @@ def test_scheduling_options_give_the_same_bits(lib):
         lib.nf4_dequant_batch([d["nf4"].w for d in L.p], outs, blocks_per_sm=2)
     torch.cuda.synchronize()
     assert all(torch.equal(o, r) for o, r in zip(outs, ref))
+
+
+@pytest.mark.parametrize("shapes,T,off", [(SHAPES_8B, 2048, ()), (SMALL, 300, (2,)),
+                                          ([(960, 704), (960, 320), (704, 960), (960, 64)], 77, ())])
+def test_merged_layer_gemms(lib, orc, shapes, T, off):
+    """LSN_OPT_LAYER_MERGE: with bf16 bases, projections 1..n-1 of a layer call run as one multi-problem GEMM
+    launch (a balanced static schedule of whole tiles over the SM pairs), forward and backward.  The same
+    bits as one launch per projection, for every y, dX, dA and dB: the 8B layer, a ragged set with one
+    projection's adapter off, and a ragged set with partial column tiles at T = 77; oracle checks on
+    sampled rows."""
+    from tests.helpers import lib_option
+    L = Layer(lib, shapes, T, 16, "bf16", seed=13)
+    with lib_option(lib, lib.LSN_OPT_LAYER_MERGE, 0):
+        a = L.layer(off=off)
+    with lib_option(lib, lib.LSN_OPT_LAYER_MERGE, 1):
+        b = L.layer(off=off)
+        b2 = L.layer(off=off)
+    _equal(b, a)
+    _equal(b2, a)
+    rows = np.sort(np.random.default_rng(4).choice(T, size=min(T, 24), replace=False))
+    for pi in sorted({1, len(shapes) - 1, *off}):
+        c = L.p[pi]["case"]
+        Wb = synth.to_bf16_bits(c.W)
+        Bm = np.zeros_like(c.B) if pi in off else c.B
+        assert_close(bf16_tensor_to_f64(b[pi]["y"])[rows], orc.lora_fwd(c.x, Wb, c.A, Bm, L.scale, rows=rows),
+                     f"merged y {pi}")
+        assert_close(bf16_tensor_to_f64(b[pi]["dX"])[rows], orc.lora_bwd_dx(c.dY, Wb, c.A, Bm, L.scale, rows=rows),
+                     f"merged dX {pi}")
 
 
 def test_layer_zero_tokens(lib):

@@ -509,3 +509,18 @@ def test_host_io_steps(lib, shared, grouped):
     for h, t in zip(got, HostIO.outputs_of(st)):
         assert torch.equal(h, t.cpu()), "the host result differs from a plain step's"
     st.close()
+
+
+@pytest.mark.parametrize("name,tokens", [("8b", 2048), ("0.5b", 512)])
+def test_merged_gemms_in_the_stack(lib, name, tokens):
+    """The stack's layer calls with projections 1..n-1 as one merged GEMM launch (LSN_OPT_LAYER_MERGE; the
+    dequantisation ahead hands the calls bf16 bases): streamed with merging is torch.equal to resident
+    without it, for every y, dX, dA and dB."""
+    from tests.helpers import lib_option
+    cfg = synth.STACKS[name]
+    with lib_option(lib, lib.LSN_OPT_LAYER_MERGE, 0):
+        res = _run(cfg, 3, tokens, "resident")
+    with lib_option(lib, lib.LSN_OPT_LAYER_MERGE, 1):
+        st = _run(cfg, 3, tokens, "streamed", steps=2)
+    fwd, bwd, bad = _compare(st, res)
+    assert fwd and bwd, bad
