@@ -721,7 +721,9 @@ lsn_status lora_layer_fwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
     bool any_deq = false, any_group = false;
     for (int i = 0; i < n; ++i) any_deq = any_deq || deq[i];
     for (int k = 0; k < g.n; ++k) any_group = any_group || g.count[k] > 1;
-    const bool early = lanes.two() && !any_deq && !any_group && nd > 0 && !adapter_off(p[0]);
+    // (One lane: the same order, everything on the caller's stream; taken when
+    // merging, so that the merged launch is the same with one lane or two.)
+    const bool early = (lanes.two() || gemm_multi()) && !any_deq && !any_group && nd > 0 && !adapter_off(p[0]);
     if (early) {
         if ((s = timed_down_batch(1, dn, true, r, lanes.main())) != LSN_OK) return s;      // dn[0]: projection 0
         if ((s = timed_down_batch(nd - 1, dn + 1, true, r, lanes.side())) != LSN_OK) return s;
@@ -821,7 +823,8 @@ lsn_status lora_layer_bwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
         // With nothing to dequantise and no groups, only the first input-gradient
         // GEMM's g = dY B runs ahead of it (on the main lane); the other down
         // projections and the token reductions run on the side lane beside it.
-        early = lanes.two() && !any_deq && !any_group && ng > 0 && p[0].dX != nullptr && !adapter_off(p[0]);
+        early = (lanes.two() || gemm_multi()) && !any_deq && !any_group && ng > 0 && p[0].dX != nullptr &&
+                !adapter_off(p[0]);
         if (early) {
             if ((s = timed_down_batch(1, dg, false, r, lanes.main())) != LSN_OK) return s;   // dg[0]: projection 0
             if ((s = timed_down_batch(ng - 1, dg + 1, false, r, lanes.side())) != LSN_OK) return s;
