@@ -276,9 +276,12 @@ def run_ours(args):
             # by CUDA events on its stream: per-kernel device time and work.
             # (The events cost host time, so the step time above is taken
             # without them.)  It runs with one lane, so that no launch waits
-            # for SMs held by another lane's kernel inside its events.
+            # for SMs held by another lane's kernel inside its events; the
+            # dequantisation one layer ahead runs on that lane too, so the
+            # layer calls get bf16 bases (and launch the same GEMMs) as in the
+            # timed steps.
             st_k = st.with_mode("streamed", n_slots=args.slots, lanes=1)
-            st_k.ahead = False                    # no dequantisation on a side stream either
+            st_k.ahead_on_compute_stream()
             lanes_opt = lsnf4.get_option(lsnf4.LSN_OPT_LAYER_LANES)
             lsnf4.set_option(lsnf4.LSN_OPT_LAYER_LANES, 1)
             try:

@@ -446,6 +446,12 @@ class Stack:
         other._setup_mode(n_slots)
         return other
 
+    def ahead_on_compute_stream(self):
+        """Run the dequantisation ahead on the compute stream, serialised with the layer calls, instead of on
+        its side stream: the same launches on one lane (for per-launch timing)."""
+        if self.ahead:
+            self._prep = self.stream
+
     def _ahead_for(self, mode: str) -> bool:
         return bool(self._ahead_opt and self.nf4 and self.api == "layer")
 
