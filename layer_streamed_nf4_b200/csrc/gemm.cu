@@ -114,7 +114,7 @@ struct GemmArgs {
 // the same chain of MMAs as in a launch of its problem alone.
 constexpr int kMultiMaxProb = 8;
 constexpr int kMultiMaxUnits = 80;
-constexpr int kMultiMaxTiles = 2048;
+constexpr int kMultiMaxTiles = 5120;
 struct MultiProbs {
     CUtensorMap a[kMultiMaxProb], b[kMultiMaxProb], la[kMultiMaxProb], lb[kMultiMaxProb];
     int nprob;
@@ -1120,7 +1120,7 @@ namespace {
 std::atomic<int> g_stream_k{0};
 std::atomic<int> g_min_units{0};
 std::atomic<int> g_tail_split{0};
-std::atomic<int> g_multi{0};
+std::atomic<int> g_multi{1};
 }
 
 void gemm_set_stream_k(bool on) { g_stream_k.store(on ? 1 : 0); }

@@ -225,7 +225,8 @@ def test_options(lib):
     lib.set_option(lib.LSN_OPT_PDL, 1)
     assert lib.get_option(lib.LSN_OPT_STREAM_K) == 0
     assert lib.get_option(lib.LSN_OPT_GEMM_MIN_UNITS) == 0
-    assert lib.get_option(lib.LSN_OPT_GEMM_TAIL_SPLIT) in (0, 1)
+    assert lib.get_option(lib.LSN_OPT_GEMM_TAIL_SPLIT) == 0
+    assert lib.get_option(lib.LSN_OPT_LAYER_MERGE) == 1
     assert lib.get_option(lib.LSN_OPT_DEQUANT_SPARE_SMS) == 0
     for opt, bad in ((lib.LSN_OPT_FUSED_NF4, 3), (lib.LSN_OPT_DEQUANT_SPARE_SMS, -1)):
         with pytest.raises(lib.LsnError) as e:
