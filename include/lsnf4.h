@@ -377,8 +377,9 @@ lsn_status lsn_timing_read(lsn_kernel_timing* out);
  *                      balances the pairs' summed contraction lengths, so the
  *                      last round of one projection's tiles no longer leaves
  *                      SMs idle (up to 8 projections and 5120 tiles; beyond,
- *                      one launch each).  Same bits (each tile is computed as
- *                      in its own launch).  0: one launch per projection.
+ *                      one launch each; and none with LSN_OPT_STREAM_K 1).
+ *                      Same bits (each tile is computed as in its own launch).
+ *                      0: one launch per projection.
  *   LSN_OPT_DEQUANT_SPARE_SMS 0 (default); n > 0: nf4_dequant_batch calls with
  *                      blocks_per_sm = k > 0 launch n * k blocks, each
  *                      reserving enough shared memory that it never shares an

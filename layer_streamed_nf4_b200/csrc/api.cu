@@ -640,7 +640,8 @@ lsn_status build_group_lb(const lsn_lora_proj* p, int i0, int m, int r, bool bwd
 // asking for dX), at least two, and within the launch's problem and tile
 // limits.
 bool merge_rest(int n, const lsn_lora_proj* p, int64_t T, bool bwd) {
-    if (!gemm_multi() || T <= 0 || n - 1 < 2 || n - 1 > gemm_multi_max_problems()) return false;
+    // (The stream-K option asks for its own schedule of every GEMM: no merging.)
+    if (!gemm_multi() || gemm_stream_k() || T <= 0 || n - 1 < 2 || n - 1 > gemm_multi_max_problems()) return false;
     GemmProblem pr[LSN_LAYER_MAX_PROJ];
     for (int i = 1; i < n; ++i) {
         if (p[i].W.kind != LSN_BASE_BF16 || (bwd && !p[i].dX)) return false;
