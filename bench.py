@@ -618,7 +618,7 @@ def main():
                          "number of tile rounds (1)")
     ap.add_argument("--dequant-spare-sms", type=int, default=0,
                     help="run the dequantisation-ahead on SMs of its own, sized for this many SMs left free by "
-                         "the GEMMs (0: beside the GEMM CTAs, 2 blocks per SM)")
+                         "the GEMMs (0: beside the GEMM CTAs, the capped grid of the dequantisation ahead)")
     ap.add_argument("--layer-merge", type=int, default=-1, choices=[-1, 0, 1],
                     help="run projections 1..n-1 of each layer call as one merged GEMM launch (1) or one launch per "
                          "projection (0); -1 (default): the library's default")

@@ -33,12 +33,15 @@ projections into one of two bf16 buffers and releases the slot; layer i+1's
 call then takes bf16 bases pointing at that buffer.  The dequantisation runs
 underneath the previous layer's GEMMs, and a pool slot is held only until
 its layer is dequantised.  Same bits as dequantising inside the call.
-The dequantisation runs with at most two blocks per SM, so that it trickles
-along beside the GEMMs instead of crowding them.  Measured on one B200 (8B
-shapes, two slots, whole blobs streamed): with streamed layers the slot
-returns to the pool a layer earlier and the copy engine stays busy (122.8 vs
-125.6 ms per step at T = 2048; 212 vs 226 ms at T = 8192); with every layer
-resident 58.6 vs 58.9 ms.
+The dequantisation's grid is capped at ahead_blocks_per_sm blocks per SM
+(default 8; a grid-stride loop covers the rest), so that it runs beside the
+GEMMs without taking every free slot.  Measured on one B200 (8B shapes, two
+slots, whole blobs streamed): with streamed layers the slot returns to the
+pool a layer earlier and the copy engine stays busy (122.8 vs 125.6 ms per
+step at T = 2048; 212 vs 226 ms at T = 8192); with every layer resident 58.6
+vs 58.9 ms.  With the merged GEMM launches, 8 or 16 blocks per SM measured
+1-2 ms per step faster than 2 (8B, T = 2048; 1, 4 and an uncapped grid
+slower or no better).
 
 Inputs: by default every (layer, projection) has its own x.  With
 shared_inputs, q, k and v read one x and gate and up read one x, as in a
@@ -131,7 +134,7 @@ class Stack:
                  mode: str = "streamed", n_slots: int = 2, seed: int = synth.SEED, keep_outputs: bool = False,
                  distinct_activations: bool = True, device: int = 0, stream: torch.cuda.Stream | None = None,
                  lanes: int = 2, api: str = "layer", shared_inputs: bool = False, grouped: bool = False,
-                 dequant_ahead: bool = True, resident_constants: bool = True):
+                 dequant_ahead: bool = True, resident_constants: bool = True, ahead_blocks_per_sm: int = 8):
         assert mode in ("resident", "streamed", "no_h2d")
         assert api in ("layer", "proj")
         assert not grouped or api == "layer", "groups are a feature of the layer calls"
@@ -161,6 +164,8 @@ class Stack:
         self._calls = {}
         self._distinct = distinct_activations
         self._ahead_opt = dequant_ahead
+        assert ahead_blocks_per_sm > 0
+        self.ahead_blocks_per_sm = ahead_blocks_per_sm
         self.ahead = self._ahead_for(mode)
         if self.nf4 and api == "layer":
             tot = sum(p.N * p.K for p in self.proj)
@@ -491,8 +496,8 @@ class Stack:
             ws = [self._nf4_view(addr, l, p) for p in self.proj]
             outs = [self._wbuf[b].data_ptr() + 2 * self._woff[pi] for pi in range(len(self.proj))]
             args = self._calls[key] = lsnf4.dequant_batch_args(ws, outs)
-        # two blocks per SM: the dequantisation trickles along beside the current layer's GEMMs
-        st = lsnf4._lib.nf4_dequant_batch(*args, 2, ps.cuda_stream)
+        # a capped grid: the dequantisation runs beside the current layer's GEMMs
+        st = lsnf4._lib.nf4_dequant_batch(*args, self.ahead_blocks_per_sm, ps.cuda_stream)
         if st:
             lsnf4._check(st, "nf4_dequant_batch")
         self._release(l, ps)
