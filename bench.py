@@ -591,8 +591,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--tokens", type=int, default=0, help="override T (default: the workload's 2048)")
     ap.add_argument("--layers", type=int, default=0, help="override the layer count (default 32)")
-    ap.add_argument("--slots", type=int, default=20,
-                    help="VRAM pool slots of the timed stream (default 20 of 32 layers: the smallest measured "
+    ap.add_argument("--slots", type=int, default=24,
+                    help="VRAM pool slots of the timed stream (default 24 of 32 layers: the smallest measured "
                          "window that hides the copies behind compute at 2048 tokens on one B200)")
     ap.add_argument("--modes", default="no_h2d,resident,proj,streamed_S2,streamed_T8192,streamed_S2_T8192,"
                                        "no_h2d_T8192,accum4,dpo,recompute,shared,grouped,bf16_base",

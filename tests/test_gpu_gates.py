@@ -9,7 +9,7 @@ and the repaired gate was re-run over every layer (320/320 at 72B).  Here
 each workload is gated over all of its layers: the Qwen2.5-3B shape (36 bf16
 layers), the Llama-3.1-8B shape in the exact configuration the benchmark
 times (32 NF4 layers, 2048 tokens, whole-layer calls on two lanes,
-dequantisation one layer ahead, a 20-slot pool) and with the pages' two
+dequantisation one layer ahead, a 24-slot pool, and 20 slots) and with the pages' two
 slots, and the Qwen2.5-72B shape (80 NF4 layers of ~432 MiB through a
 2-slot pool, every layer's adapter gradients).  Resident = the same blobs
 copied once into one device buffer and driven by the same launches."""
@@ -86,15 +86,15 @@ def test_gate_3b_every_layer(lib):
 
 def test_gate_8b_benchmark_configuration(lib):
     """The configuration the benchmark times: Llama-3.1-8B shape, NF4, 32 layers, 2048 tokens, whole-layer
-    calls on two lanes, dequantisation one layer ahead, 20 pool slots; and the same with the pages' two
-    slots.  Every y, dX, dA, dB of every layer equals the resident run's."""
+    calls on two lanes, dequantisation one layer ahead, 24 pool slots (and 20); and the same with the pages'
+    two slots.  Every y, dX, dA, dB of every layer equals the resident run's."""
     from layer_streamed_nf4_b200.stack import Stack
     cfg = synth.STACKS["8b"]
     assert cfg.layers == 32 and cfg.tokens == 2048
     probe = Stack(cfg, layers=1, tokens=64, mode="streamed")
     assert probe.ahead and probe.api == "layer" and lib.get_option(lib.LSN_OPT_LAYER_LANES) == 2
     probe.close()
-    _gate(cfg, 2048, (20, 2))
+    _gate(cfg, 2048, (24, 20, 2))
 
 
 def test_gate_72b_every_layer(lib):
