@@ -102,7 +102,7 @@ def _cpu_stack(monkeypatch, L, S, ahead, api="layer"):
     st.n_lanes, st.lanes, st._fork, st._join = 1, [st.stream], [FakeEvent()], [FakeEvent()]
     st.proj, st.layer_bytes, st.const_bytes = layer_layout(cfg, True)
     st.consts = torch.zeros((L, st.const_bytes), dtype=torch.uint8)
-    st._calls, st._distinct, st._ahead_opt = {}, True, ahead
+    st._calls, st._distinct, st._ahead_opt, st.ahead_blocks_per_sm = {}, True, ahead, 8
     st.ahead = st._ahead_for("streamed")
     st._wbuf = [torch.empty(sum(p.N * p.K for p in st.proj), dtype=torch.bfloat16) for _ in range(2)]
     st._woff, o = [], 0
