@@ -222,7 +222,11 @@ lsn_status lora_linear_bwd(const lsn_base* W, const uint16_t* x, const uint16_t*
  * bit for bit those of lora_linear_fwd / lora_linear_bwd on the same inputs;
  * only the launches differ: the NF4 dequantisation of all projections is one
  * kernel, their rank-r down projections one kernel, their dA/dB token
- * reductions one kernel.  The forward can keep u = x A^T, the low-rank
+ * reductions one kernel, and (LSN_OPT_LAYER_MERGE, bf16 bases, no groups)
+ * the GEMMs of projections 1..n-1 one launch after projection 0's own.  The
+ * projections are independent of each other within a call (each reads only
+ * its own x or dY): a caller whose projections depend on each other (o on
+ * attention over q, k, v) makes one call per independent set.  The forward can keep u = x A^T, the low-rank
  * activation a LoRA layer saves for its backward pass, so the backward does
  * not read x again to rebuild it.  A projection whose A and B are NULL runs
  * with the adapter off: the streamed base alone, the reference model of
