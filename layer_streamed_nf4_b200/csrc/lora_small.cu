@@ -271,19 +271,22 @@ __global__ void __launch_bounds__(128) lora_down_kernel(const __grid_constant__ 
 //
 // R[j, k] = sum_{t in split} G[t, j] * X[t, k] (dA with G = g, X = x; dB with
 // G = u, X = dY).  On the warp-level tensor-core instruction with M = k, N = j
-// and the tokens as the contraction: X tiles [32 t x 128 k] are staged by
+// and the tokens as the contraction: X tiles [32 t x 256 k] are staged by
 // cp.async (3 stages, 16-byte chunks XOR-swizzled by token row) and read
 // transposed with ldmatrix.trans; G is fp32, so
 // each element enters as two bf16 MMAs, hi = bf16(G) and lo = bf16(G - hi),
 // which leaves a relative error below 2^-17 per product before fp32
-// accumulation.  A CTA owns 128 columns k (warp w: k0+32w .. +31) and one
-// token split; the splits of a column tile form one thread-block cluster and
-// are added in split order through distributed shared memory.  At r = 16 the
-// ring takes 31.5 KB, small enough to share an SM with a running GEMM CTA.
-// Batched like the down projection: blockIdx.x runs over the column tiles of
-// all problems (dA and dB of several projections), blockIdx.y is the token
-// split.
-constexpr int kTgCols = 128;
+// accumulation.  A CTA owns 256 columns k (warp w: k0+64w .. +63, so each
+// warp's conversion of G feeds four 16-column MMA rows) and one token split;
+// the splits of a column tile form one thread-block cluster and are added in
+// split order through distributed shared memory.  At r = 16 the ring takes
+// 55.5 KB.  (With 128 columns per CTA and the G conversion feeding two MMA
+// rows the kernel was bound by issue slots and barrier waits: the 32 launches
+// of an 8B step at T = 2048 (14 reductions each) took 3.91-4.06 ms against
+// 3.33-3.46 ms with 256, one B200, events on one lane.)  Batched like the down projection: blockIdx.x
+// runs over the column tiles of all problems (dA and dB of several
+// projections), blockIdx.y is the token split.
+constexpr int kTgCols = 256;
 constexpr int kTgTok = 32;          // tokens per staged tile (two MMA k-steps)
 constexpr int kTgStages = 3;
 
@@ -343,8 +346,8 @@ __global__ void __launch_bounds__(128) lora_tgrad_kernel(const __grid_constant__
     auto load = [&](int stage, int64_t tile) {
         const int64_t t0 = tb + tile * kTgTok;
         #pragma unroll
-        for (int i = 0; i < 4; ++i) {                     // X: 32 rows x 16 pieces of 16 bytes
-            const int p = tid + i * 128, row = p >> 4, piece = p & 15;
+        for (int i = 0; i < 8; ++i) {                     // X: 32 rows x 32 pieces of 16 bytes
+            const int p = tid + i * 128, row = p >> 5, piece = p & 31;
             const int64_t t = t0 + row, k = k0 + piece * 8;
             const bool ok = t < te && k < Kd;
             cp_async16(xa(stage, row, piece * 8), X + (ok ? t : 0) * Kd + (ok ? k : 0), ok ? 16u : 0u);
@@ -357,9 +360,9 @@ __global__ void __launch_bounds__(128) lora_tgrad_kernel(const __grid_constant__
         }
     };
 
-    float acc[2][NT][4];
+    float acc[4][NT][4];
     #pragma unroll
-    for (int m = 0; m < 2; ++m)
+    for (int m = 0; m < 4; ++m)
         #pragma unroll
         for (int n = 0; n < NT; ++n) acc[m][n][0] = acc[m][n][1] = acc[m][n][2] = acc[m][n][3] = 0.0f;
 
@@ -396,9 +399,9 @@ __global__ void __launch_bounds__(128) lora_tgrad_kernel(const __grid_constant__
                 }
             }
             #pragma unroll
-            for (int m = 0; m < 2; ++m) {
+            for (int m = 0; m < 4; ++m) {
                 uint32_t a0, a1, a2, a3;
-                ldsm_x4_t(xa(st, kk * 16 + a_t, warp * 32 + m * 16 + a_k), a0, a1, a2, a3);
+                ldsm_x4_t(xa(st, kk * 16 + a_t, warp * 64 + m * 16 + a_k), a0, a1, a2, a3);
                 #pragma unroll
                 for (int n = 0; n < NT; ++n) {
                     mma_bf16_16816(acc[m][n], a0, a1, a2, a3, bh[n][0], bh[n][1]);
@@ -419,10 +422,10 @@ __global__ void __launch_bounds__(128) lora_tgrad_kernel(const __grid_constant__
     if (nsplit == 1) {                  // every CTA of the cluster takes this branch
         if (blockIdx.y != 0) return;
         #pragma unroll
-        for (int m = 0; m < 2; ++m)
+        for (int m = 0; m < 4; ++m)
             #pragma unroll
             for (int n = 0; n < NT; ++n) {
-                const int64_t k = k0 + warp * 32 + m * 16 + g;
+                const int64_t k = k0 + warp * 64 + m * 16 + g;
                 const int j = 8 * n + 2 * q;
                 if (k < Kd) { finish(k, j, acc[m][n][0]); finish(k, j + 1, acc[m][n][1]); }
                 if (k + 8 < Kd) { finish(k + 8, j, acc[m][n][2]); finish(k + 8, j + 1, acc[m][n][3]); }
@@ -433,10 +436,10 @@ __global__ void __launch_bounds__(128) lora_tgrad_kernel(const __grid_constant__
     __syncthreads();
     float* red = reinterpret_cast<float*>(tg_smem);
     #pragma unroll
-    for (int m = 0; m < 2; ++m)
+    for (int m = 0; m < 4; ++m)
         #pragma unroll
         for (int n = 0; n < NT; ++n) {
-            const int c = warp * 32 + m * 16 + g;
+            const int c = warp * 64 + m * 16 + g;
             const int j = 8 * n + 2 * q;
             red[j * kTgCols + c] = acc[m][n][0];
             red[(j + 1) * kTgCols + c] = acc[m][n][1];
