@@ -289,6 +289,7 @@ __global__ void __launch_bounds__(128) lora_down_kernel(const __grid_constant__ 
 constexpr int kTgCols = 256;
 constexpr int kTgTok = 32;          // tokens per staged tile (two MMA k-steps)
 constexpr int kTgStages = 3;
+static_assert(kTgCols == 32 * 8, "a tile row is 32 pieces of 16 bytes, one per lane (the X load's thread map)");
 
 struct TgProb {
     const float* G;      // [T, r] fp32
@@ -343,14 +344,26 @@ __global__ void __launch_bounds__(128) lora_tgrad_kernel(const __grid_constant__
     const int64_t te = (tb + per_split < T) ? tb + per_split : T;
     const int64_t ntiles = te > tb ? (te - tb + kTgTok - 1) / kTgTok : 0;
 
+    // X loads: thread tid copies the 16-byte piece xpc of rows xr0 + 4 i
+    // (i = 0..7) of every tile, so its column offset, its row stride and the
+    // two swizzle patterns of its rows (xr0 < 4: row & 7 = xr0 + 4 (i & 1))
+    // are fixed for the whole kernel.
+    const int xr0 = tid >> 5, xpc = tid & 31;
+    const bool k_ok = k0 + xpc * 8 < Kd;
+    const uint16_t* const xcol = X + (k_ok ? k0 + xpc * 8 : 0);
+    const int64_t xstride4 = 4 * Kd;
+    const uint32_t xoff0 = (uint32_t)(xr0 * kTgCols + ((xpc ^ xr0) << 3)) * 2u;
+    const uint32_t xoff1 = (uint32_t)(xr0 * kTgCols + ((xpc ^ (xr0 + 4)) << 3)) * 2u;
     auto load = [&](int stage, int64_t tile) {
         const int64_t t0 = tb + tile * kTgTok;
+        const uint32_t dst = smem_u32(xs + stage * L::X_TILE);
+        const uint16_t* src = xcol + (t0 + xr0) * Kd;
         #pragma unroll
-        for (int i = 0; i < 8; ++i) {                     // X: 32 rows x 32 pieces of 16 bytes
-            const int p = tid + i * 128, row = p >> 5, piece = p & 31;
-            const int64_t t = t0 + row, k = k0 + piece * 8;
-            const bool ok = t < te && k < Kd;
-            cp_async16(xa(stage, row, piece * 8), X + (ok ? t : 0) * Kd + (ok ? k : 0), ok ? 16u : 0u);
+        for (int i = 0; i < kTgTok / 4; ++i) {            // X: 32 rows x 32 pieces of 16 bytes
+            const bool ok = k_ok && t0 + xr0 + 4 * i < te;
+            const uint32_t off = ((i & 1) ? xoff1 : xoff0) + (uint32_t)(4 * i * kTgCols * 2);
+            cp_async16(dst + off, ok ? src : X, ok ? 16u : 0u);
+            src += xstride4;
         }
         for (int p = tid; p < kTgTok * (R / 4); p += 128) {   // G: 32 rows x R/4 pieces
             const int row = p / (R / 4), piece = p % (R / 4);
