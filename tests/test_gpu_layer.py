@@ -227,6 +227,20 @@ def test_merged_layer_gemms(lib, orc, shapes, T, off):
                      f"merged dX {pi}")
 
 
+def test_merged_launch_limits(lib):
+    """The merged launch takes at most 8 problems: a call with 9 projections (8 after the first) merges
+    them, one with 10 runs one launch per projection; both give the bits of the single-linear calls."""
+    from tests.helpers import lib_option
+    shapes9 = [(256, 256), (256, 64), (256, 128), (256, 256), (256, 512), (256, 512), (512, 256), (256, 192),
+               (320, 256)]
+    for shapes in (shapes9, shapes9 + [(256, 320)]):
+        L = Layer(lib, shapes, 300, 16, "bf16", seed=17)
+        a = L.single()
+        with lib_option(lib, lib.LSN_OPT_LAYER_MERGE, 1):
+            b = L.layer()
+        _equal(b, a)
+
+
 def test_layer_zero_tokens(lib):
     import torch
     L = Layer(lib, SMALL[:2], 0, 16, "nf4")
