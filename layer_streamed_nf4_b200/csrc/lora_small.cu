@@ -162,14 +162,25 @@ __global__ void __launch_bounds__(128) lora_down_kernel(const __grid_constant__ 
     const int64_t c_end = (c_begin + chunks_per_split < nchunks) ? c_begin + chunks_per_split : nchunks;
     const int64_t nc = c_end > c_begin ? c_end - c_begin : 0;
 
+    // X loads: thread tid copies the 16-byte piece xpc of rows xr0 + 16 i
+    // (i = 0..3) of every chunk; those rows share one swizzle pattern
+    // (row & 7 = xr0 & 7), so the shared-memory offsets and the row pointers
+    // are fixed for the whole kernel.
+    const int xr0 = tid >> 3, xpc = tid & 7;
+    const uint32_t xoff = (uint32_t)(xr0 * 64 + ((xpc ^ (xr0 & 7)) << 3)) * 2u;
+    const uint16_t* xsrc[4];
+    bool xok[4];
+    #pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int64_t t = row_base + xr0 + 16 * i;
+        xok[i] = t < T;
+        xsrc[i] = X + (xok[i] ? t : 0) * Kd + xpc * 8;
+    }
     auto load = [&](int stage, int64_t c) {
+        const uint32_t dst = smem_u32(xs + stage * L::X_TILE) + xoff;
         #pragma unroll
-        for (int i = 0; i < 4; ++i) {                     // X: 64 rows x 8 pieces of 16 bytes
-            const int p = tid + i * 128, row = p >> 3, piece = p & 7;
-            const int64_t t = row_base + row;
-            const bool ok = t < T;
-            cp_async16(xa(stage, row, piece * 8), X + (ok ? t : 0) * Kd + c * 64 + piece * 8, ok ? 16u : 0u);
-        }
+        for (int i = 0; i < 4; ++i)                       // X: 64 rows x 8 pieces of 16 bytes
+            cp_async16(dst + (uint32_t)(i * 16 * 64 * 2), xsrc[i] + c * 64, xok[i] ? 16u : 0u);
         if (B_KR) {                                       // W = B [Kd, r]: 64 rows x r/8 pieces
             for (int p = tid; p < 64 * NT; p += 128) {
                 const int row = p / NT, piece = p % NT;
