@@ -710,6 +710,8 @@ class HostIO:
     def run(self, steps: int, step_fn):
         """`steps` calls of step_fn() on the compute stream, each on inputs copied in from the host and each
         followed by the copy of its result to the host."""
+        if steps <= 0:
+            return
         c, cp = self.compute, self.copy
         cp.wait_stream(c)                          # the staging buffers are free of earlier work
         self._h2d()
