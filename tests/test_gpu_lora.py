@@ -227,6 +227,8 @@ SAMPLED = [
     ("8b-kv", 2048, 4096, 1024),
     ("8b-down", 2048, 14336, 4096),
     ("0.5b-up", 512, 896, 4864),
+    ("3b-gate", 1024, 2048, 11008),
+    ("72b-down", 1024, 29568, 8192),
 ]
 
 
@@ -234,7 +236,7 @@ SAMPLED = [
 def test_full_size_sampled_rows(lib, orc, name, T, K, N):
     import torch
     c = synth.linear_case(T, K, N, 16, 32.0, seed=sum(map(ord, name)))
-    kind = "bf16" if name.startswith("0.5b") else "nf4"
+    kind = "bf16" if name.startswith(("0.5b", "3b")) else "nf4"
     L = Linear(lib, c, kind)
     y = L.fwd()
     dX, dA, dB = L.bwd()

@@ -402,28 +402,34 @@ def test_grouped_stack_matches_shared_inputs(lib, orc):
     grouped.close()
 
 
-def test_full_size_stack_against_oracle(lib, orc):
-    """One 8B-shaped layer at the timed size and launch configuration (T = 2048, layer calls, streamed
-    through the pool, weights dequantised one layer ahead): y and dX on sampled token rows and dA, dB in
-    full for the q and down projections, against the oracle.  The oracle quantises the fp32 weights
-    itself; inputs are the seeded generator's, read back from the device."""
+@pytest.mark.parametrize("name,tokens,pis", [("8b", 2048, (0, 6)), ("3b", 1024, (1, 4)), ("72b", 1024, (0, 6))])
+def test_full_size_stack_against_oracle(lib, orc, name, tokens, pis):
+    """One layer of a workload stack at its stated size in the timed launch configuration (layer calls,
+    streamed through the pool, NF4 weights dequantised one layer ahead, projection 0's GEMM then the merged
+    launch of the others): y and dX on sampled token rows and dA, dB in full for two projections (the
+    8B q and down, the 3B bf16 k and gate, the 72B q and down of ~29568 x 8192), against the oracle.  The
+    oracle quantises (or rounds to bf16) the fp32 weights itself; inputs are the seeded generator's, read
+    back from the device."""
     import numpy as np
     import torch
     from layer_streamed_nf4_b200.stack import Stack
     from tests.helpers import assert_close, bf16_tensor_to_f64
-    cfg = synth.STACKS["8b"]
-    st = Stack(cfg, layers=1, tokens=2048, mode="streamed", keep_outputs=True)
-    assert st.ahead
+    cfg = synth.STACKS[name]
+    st = Stack(cfg, layers=1, tokens=tokens, mode="streamed", keep_outputs=True)
+    assert st.ahead == (cfg.base == "nf4")
     st.step()
     torch.cuda.synchronize()
     st.check_status()
     bits = lambda t: t.view(torch.int16).cpu().numpy().view(np.uint16)
-    rows = np.sort(np.random.default_rng(8).choice(2048, size=32, replace=False))
-    for pi in (0, 6):
+    rows = np.sort(np.random.default_rng(8).choice(tokens, size=32, replace=False))
+    for pi in pis:
         p = st.proj[pi]
         W = synth.device_normal((p.N, p.K), 0.02, st.seed, 0, pi, synth.T_W, device=st.dev).cpu().numpy()
-        q = orc.nf4_quantize(W)
-        Wb = orc.nf4_dequant(q["packed"], q["absmax_q"], q["s2"], q["offset"], W.size).reshape(W.shape)
+        if cfg.base == "nf4":
+            q = orc.nf4_quantize(W)
+            Wb = orc.nf4_dequant(q["packed"], q["absmax_q"], q["s2"], q["offset"], W.size).reshape(W.shape)
+        else:
+            Wb = synth.to_bf16_bits(W)
         x, dY, A, B = bits(st.x[0, pi]), bits(st.dY[0, pi]), bits(st.A[0, pi]), bits(st.B[0, pi])
         assert_close(bf16_tensor_to_f64(st.y[0, pi])[rows], orc.lora_fwd(x, Wb, A, B, st.scale, rows=rows), f"{p.name} y")
         assert_close(bf16_tensor_to_f64(st.dX[0, pi])[rows], orc.lora_bwd_dx(dY, Wb, A, B, st.scale, rows=rows),
