@@ -402,12 +402,14 @@ def test_grouped_stack_matches_shared_inputs(lib, orc):
     grouped.close()
 
 
-@pytest.mark.parametrize("name,tokens,pis", [("8b", 2048, (0, 6)), ("3b", 1024, (1, 4)), ("72b", 1024, (0, 6))])
+@pytest.mark.parametrize("name,tokens,pis", [("8b", 2048, (0, 6)), ("8b", 8192, (1, 6)), ("3b", 1024, (1, 4)),
+                                               ("72b", 1024, (0, 6))])
 def test_full_size_stack_against_oracle(lib, orc, name, tokens, pis):
     """One layer of a workload stack at its stated size in the timed launch configuration (layer calls,
     streamed through the pool, NF4 weights dequantised one layer ahead, projection 0's GEMM then the merged
     launch of the others): y and dX on sampled token rows and dA, dB in full for two projections (the
-    8B q and down, the 3B bf16 k and gate, the 72B q and down of ~29568 x 8192), against the oracle.  The
+    8B q and down, the 8B k and down at 8192 tokens (a merged launch of 4864 tiles), the 3B bf16 k and gate,
+    the 72B q and down of ~29568 x 8192), against the oracle.  The
     oracle quantises (or rounds to bf16) the fp32 weights itself; inputs are the seeded generator's, read
     back from the device."""
     import numpy as np
