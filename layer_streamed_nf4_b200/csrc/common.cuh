@@ -163,7 +163,7 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// 2-D tiled TMA load, completion signalled on an mbarrier (no multicast).
+// 2-D tiled TMA load into this CTA's shared memory, completion signalled on an mbarrier.
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int32_t x, int32_t y,
                                             uint64_t* bar) {
     asm volatile(

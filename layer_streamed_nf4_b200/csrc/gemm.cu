@@ -611,7 +611,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
 // rings advance in lockstep, one slot per 128-wide K-block, each with its own
 // barriers so that no stage waits on a chain of the others' latencies:
 //   A ring   TMA of this CTA's 128 A rows (counted on the leader), released
-//            by the MMA (multicast commit);
+//            by the MMA (a commit that arrives on both CTAs' barriers);
 //   P ring   TMA of this CTA's packed NF4 tile (128 rows x 64 bytes, 64-byte
 //            swizzle), issued by its own producer warp and released by the
 //            converters as soon as they have read it;
