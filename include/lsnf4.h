@@ -403,6 +403,19 @@ typedef enum {
 lsn_status lsn_set_option(int option, int value);
 int lsn_get_option(int option);
 
+/* The tile schedule of the merged GEMM launch (LSN_OPT_LAYER_MERGE), computed
+ * on the host from the shapes alone (no device is touched): n problems of
+ * ntiles[i] whole tiles costing cost[i] contraction blocks each, numbered
+ * problem after problem, shared out over `units` workers (SM pairs): tiles in
+ * decreasing cost (problem order among equal costs), each to the worker with
+ * the least summed cost so far (the lowest index on ties).  Worker u takes
+ * tile[start[u] .. start[u+1]).  start holds units + 1 entries (host memory),
+ * tile max_tiles; LSN_ERR_INVALID_ARG when the tiles do not fit or an argument
+ * is out of range.  Exposed for inspection and tests; the launch computes the
+ * same schedule itself. */
+lsn_status lsn_gemm_merged_schedule(int units, int n, const int* ntiles, const int* cost, int* start, int* tile,
+                                    int max_tiles);
+
 /* ------------------------------------------------------------ layer pool --
  *
  * n_slots VRAM buffers of slot_bytes each, allocated once at creation; the

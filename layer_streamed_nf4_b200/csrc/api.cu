@@ -952,6 +952,11 @@ int lsn_get_option(int option) {
     return -1;
 }
 
+lsn_status lsn_gemm_merged_schedule(int units, int n, const int* ntiles, const int* cost, int* start, int* tile,
+                                    int max_tiles) {
+    return gemm_merged_schedule(units, n, ntiles, cost, start, tile, max_tiles);
+}
+
 lsn_status lsn_ws_status(void* ws, lsn_stream_t stream) {
     LSN_CHECK_ARG(ws != nullptr, "lsn_ws_status: workspace is NULL");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

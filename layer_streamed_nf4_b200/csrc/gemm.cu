@@ -1277,6 +1277,22 @@ const MultiSched& multi_schedule(int units, int num_m, const int* ntiles, const 
 
 int gemm_multi_max_problems() { return kMultiMaxProb; }
 
+lsn_status gemm_merged_schedule(int units, int n, const int* ntiles, const int* cost, int* start, int* tile,
+                                int max_tiles) {
+    if (units < 1 || n < 1 || n > 64 || !ntiles || !cost || !start || !tile || max_tiles < 0)
+        return fail(LSN_ERR_INVALID_ARG, "lsn_gemm_merged_schedule: bad arguments");
+    int64_t total = 0;
+    for (int i = 0; i < n; ++i) {
+        if (ntiles[i] < 0 || cost[i] < 1) return fail(LSN_ERR_INVALID_ARG, "lsn_gemm_merged_schedule: bad tile count or cost");
+        total += ntiles[i];
+    }
+    if (total > max_tiles || total > 65535) return fail(LSN_ERR_INVALID_ARG, "lsn_gemm_merged_schedule: too many tiles");
+    const MultiSched& sc = multi_schedule(units, 0, ntiles, cost, n);
+    for (int u = 0; u <= units; ++u) start[u] = sc.start[u];
+    for (size_t t = 0; t < sc.tile.size(); ++t) tile[t] = sc.tile[t];
+    return LSN_OK;
+}
+
 bool gemm_multi_fits(const GemmProblem* pr, int n, int64_t M) {
     if (n < 1 || n > kMultiMaxProb || M <= 0 || sm_count() / 2 > kMultiMaxUnits) return false;
     int64_t tiles = 0;

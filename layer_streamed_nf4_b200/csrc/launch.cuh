@@ -111,6 +111,8 @@ struct GemmProblem {
     int64_t ldd = 0;
 };
 int gemm_multi_max_problems();
+lsn_status gemm_merged_schedule(int units, int n, const int* ntiles, const int* cost, int* start, int* tile,
+                                int max_tiles);
 // Whether n problems of M rows fit one launch (problem and tile limits).
 bool gemm_multi_fits(const GemmProblem* pr, int n, int64_t M);
 // D_i = A_i . op(B_i) + LA_i . op(LB_i) for every problem i, one persistent

@@ -48,7 +48,7 @@ EXPORTS = (
     "layer_pool_create", "layer_pool_register", "layer_pool_prefetch", "layer_pool_acquire",
     "layer_pool_release", "layer_pool_wait_idle", "layer_pool_stats", "layer_pool_reset",
     "layer_pool_inject_fault", "layer_pool_destroy", "lsn_timing_enable", "lsn_timing_read",
-    "nf4_quantize_noalloc", "lsn_set_option", "lsn_get_option",
+    "nf4_quantize_noalloc", "lsn_set_option", "lsn_get_option", "lsn_gemm_merged_schedule",
     "lsn_layer_ws_bytes", "lora_layer_fwd", "lora_layer_bwd", "nf4_dequant_batch",
     "lsn_selftest_wait_timeout", "layer_pool_set_debug",
 )
@@ -125,6 +125,8 @@ _sig("lora_layer_fwd", _i, [_i, ctypes.POINTER(LoraProj), _i64, _i, ctypes.c_flo
 _sig("lora_layer_bwd", _i, [_i, ctypes.POINTER(LoraProj), _i64, _i, ctypes.c_float, _i, _vp, _sz, _vp])
 _sig("lsn_set_option", _i, [_i, _i])
 _sig("lsn_get_option", _i, [_i])
+_IP = ctypes.POINTER(ctypes.c_int)
+_sig("lsn_gemm_merged_schedule", _i, [_i, _i, _IP, _IP, _IP, _IP, _i])
 _sig("lsn_timing_enable", _i, [_i])
 _sig("lsn_timing_read", _i, [ctypes.POINTER(KernelTiming)])
 _sig("layer_pool_create", _i, [_i, _sz, _i, ctypes.POINTER(_vp)])
@@ -307,6 +309,18 @@ def set_option(option: int, value: int):
 
 def get_option(option: int) -> int:
     return int(_lib.lsn_get_option(option))
+
+
+def gemm_merged_schedule(units: int, ntiles, cost):
+    """The merged GEMM launch's tile lists: one list of tile numbers per worker (host-only call)."""
+    n = len(ntiles)
+    total = int(sum(ntiles))
+    nt = (ctypes.c_int * n)(*ntiles)
+    cs = (ctypes.c_int * n)(*cost)
+    start = (ctypes.c_int * (units + 1))()
+    tile = (ctypes.c_int * max(total, 1))()
+    _check(_lib.lsn_gemm_merged_schedule(units, n, nt, cs, start, tile, total), "lsn_gemm_merged_schedule")
+    return [list(tile[start[u]:start[u + 1]]) for u in range(units)]
 
 
 # -------------------------------------------------------- kernel timing ---

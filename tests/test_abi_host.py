@@ -289,3 +289,35 @@ def test_noalloc_checks_its_arguments_like_the_workspace_version(lib):
     with pytest.raises(lib.LsnError) as e:
         lib.nf4_quantize_noalloc(1 << 20, over, stream=0)
     assert e.value.status == lib.LSN_ERR_INVALID_ARG and "limit" in str(e.value)
+
+
+def test_merged_gemm_schedule(lib):
+    """The merged launch's host-made schedule (no device touched): every tile of every problem goes to
+    exactly one worker; each worker's list runs in decreasing cost; the busiest worker's summed cost is
+    within one tile of the ideal share (the greedy bound); for the forward GEMMs of projections 1..6 of
+    the 8B layer at 2048 tokens on 74 SM pairs it is 688 contraction blocks (ideal 687.7, 886 - 66 = 820
+    for separate launches of those six).  Bad arguments are rejected."""
+    ntiles = [32, 32, 128, 448, 448, 128]          # k, v, o, gate, up, down: 256 x 256 pair tiles
+    cost = [33, 33, 33, 33, 33, 113]               # 128-wide contraction blocks + the LoRA block
+    lists = lib.gemm_merged_schedule(74, ntiles, cost)
+    flat = sorted(t for lst in lists for t in lst)
+    assert flat == list(range(sum(ntiles)))
+    first = [0]
+    for n in ntiles:
+        first.append(first[-1] + n)
+    def c(t):
+        i = max(j for j in range(len(ntiles)) if first[j] <= t)
+        return cost[i]
+    loads = [sum(c(t) for t in lst) for lst in lists]
+    ideal = sum(n * k for n, k in zip(ntiles, cost)) / 74
+    assert max(loads) <= ideal + max(cost)
+    assert max(loads) == 688
+    for lst in lists:
+        costs = [c(t) for t in lst]
+        assert costs == sorted(costs, reverse=True)
+    # the backward's six (dX of k, v, o, gate, up, down): contraction 1024, 1024, 4096, 14336, 14336, 4096
+    b = lib.gemm_merged_schedule(74, [128, 128, 128, 128, 128, 448], [9, 9, 33, 113, 113, 33])
+    assert sorted(t for lst in b for t in lst) == list(range(1088))
+    for bad in ((0, [1], [1]), (4, [1], [0]), (4, [-1], [3])):
+        with pytest.raises(lib.LsnError):
+            lib.gemm_merged_schedule(*bad)
