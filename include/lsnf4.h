@@ -373,17 +373,21 @@ lsn_status lsn_timing_read(lsn_kernel_timing* out);
  *                      of columns; each output element is still summed over
  *                      the whole contraction by one SM pair, so the bits do
  *                      not change.  0 (default): whole tiles round robin.
- *   LSN_OPT_LAYER_MERGE 1 (default): in lora_layer_fwd / _bwd calls without
- *                      groups whose bases are all bf16, the GEMMs of
- *                      projections 1..n-1 run as one persistent launch (after
- *                      projection 0's own): whole 256 x 256 tiles of all of
- *                      them, shared out over the SM pairs by a schedule that
- *                      balances the pairs' summed contraction lengths, so the
- *                      last round of one projection's tiles no longer leaves
- *                      SMs idle (up to 8 projections and 5120 tiles; beyond,
- *                      one launch each; and none with LSN_OPT_STREAM_K 1).
- *                      Same bits (each tile is computed as in its own launch).
- *                      0: one launch per projection.
+ *   LSN_OPT_LAYER_MERGE 1 (default): in lora_layer_fwd / _bwd calls whose
+ *                      bases are all bf16, the GEMMs run as one persistent
+ *                      launch: whole 256 x 256 tiles of all of them, shared
+ *                      out over the SM pairs by a schedule that balances the
+ *                      pairs' summed contraction lengths, so the last round of
+ *                      one projection's tiles no longer leaves SMs idle.
+ *                      Without groups, projection 0's GEMM runs first on its
+ *                      own (only its down projection then precedes a GEMM)
+ *                      and projections 1..n-1 are merged; with groups (or the
+ *                      adapter off on projection 0) every GEMM of the call is
+ *                      merged, a group's backward as one problem over its
+ *                      members' dY.  Up to 8 problems and 5120 tiles (beyond,
+ *                      one launch each); none with LSN_OPT_STREAM_K 1.  Same
+ *                      bits (each tile is computed as in its own launch).
+ *                      0: one launch per projection or group.
  *   LSN_OPT_DEQUANT_SPARE_SMS 0 (default); n > 0: nf4_dequant_batch calls with
  *                      blocks_per_sm = k > 0 launch n * k blocks, each
  *                      reserving enough shared memory that it never shares an

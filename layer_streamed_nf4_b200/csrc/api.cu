@@ -664,8 +664,8 @@ lsn_status merged_gemms(int n, const lsn_lora_proj* p, int64_t T, int r, const L
         q.ldb = K;
         q.LA = lora ? w.s16[i] : nullptr;
         if (!bwd) {
-            q.A = p[i].x;
-            q.lda = K;
+            q.A[0] = p[i].x;
+            q.lda[0] = K;
             q.LB = p[i].B;
             q.N = N;
             q.Kc = K;
@@ -673,8 +673,8 @@ lsn_status merged_gemms(int n, const lsn_lora_proj* p, int64_t T, int r, const L
             q.ldd = N;
             flop += 2.0 * T * N * (double)(K + (lora ? r : 0));
         } else {
-            q.A = p[i].dY;
-            q.lda = N;
+            q.A[0] = p[i].dY;
+            q.lda[0] = N;
             q.LB = p[i].A;
             q.N = K;
             q.Kc = N;
@@ -685,6 +685,80 @@ lsn_status merged_gemms(int n, const lsn_lora_proj* p, int64_t T, int r, const L
     }
     TimingScope ts(bwd ? LSN_K_GEMM_BWD : LSN_K_GEMM_FWD, flop, st);
     return launch_gemm_multi(pr, n - 1, bwd, T, r, w.err, st);
+}
+
+// A layer call with groups as one merged GEMM launch (LSN_OPT_LAYER_MERGE):
+// forward, every projection is a problem of its own (a group's members share
+// x; member j's bf16(s u) is column block j of the group's LoRA operand);
+// backward, every group (or ungrouped projection) asking for dX is one
+// problem whose contraction runs over its members' dY side by side, as in the
+// grouped GEMM.  Returns false (nothing launched) when the call does not
+// qualify: a base that is not bf16, the stream-K option, or more problems or
+// tiles than one launch takes.
+bool grouped_problems(int n, const lsn_lora_proj* p, const Groups& g, int64_t T, int r, const LayerWs& w, bool bwd,
+                      GemmProblem* pr, int* np, double* flop) {
+    if (!gemm_multi() || gemm_stream_k() || T <= 0) return false;
+    for (int i = 0; i < n; ++i)
+        if (p[i].W.kind != LSN_BASE_BF16) return false;
+    int k = 0;
+    double f = 0.0;
+    for (int gi = 0; gi < g.n; ++gi) {
+        const int i0 = g.first[gi], m = g.count[gi];
+        const bool lora = !adapter_off(p[i0]);
+        const int64_t K = p[i0].W.cols;
+        if (!bwd) {
+            for (int j = 0; j < m; ++j) {
+                if (k == gemm_multi_max_problems()) return false;
+                const int i = i0 + j;
+                const int64_t N = p[i].W.rows;
+                GemmProblem& q = pr[k++];
+                q.A[0] = p[i].x;
+                q.lda[0] = K;
+                q.B = p[i].W.bf16;
+                q.ldb = K;
+                if (lora) {
+                    q.LA = m > 1 ? w.la[i0] + (int64_t)j * r : w.s16[i];
+                    q.ld_la = m > 1 ? (int64_t)m * r : r;
+                    q.lr = r;
+                    q.LB = p[i].B;
+                }
+                q.N = N;
+                q.Kc = K;
+                q.D = p[i].y;
+                q.ldd = N;
+                f += 2.0 * T * N * (double)(K + (lora ? r : 0));
+            }
+        } else {
+            if (!p[i0].dX) continue;
+            if (k == gemm_multi_max_problems() || m > kGemmMaxSeg) return false;
+            GemmProblem& q = pr[k++];
+            int64_t nsum = 0;
+            q.na = m;
+            for (int j = 0; j < m; ++j) {
+                q.A[j] = p[i0 + j].dY;
+                q.lda[j] = p[i0 + j].W.rows;
+                q.a_kc[j] = p[i0 + j].W.rows;
+                nsum += p[i0 + j].W.rows;
+            }
+            q.B = p[i0].W.bf16;                 // the members' bases back to back: [nsum, K]
+            q.ldb = K;
+            if (lora) {
+                q.LA = m > 1 ? w.la[i0] : w.s16[i0];
+                q.ld_la = (int64_t)m * r;
+                q.lr = m * r;
+                q.LB = m > 1 ? w.lb[i0] : p[i0].A;
+            }
+            q.N = K;
+            q.Kc = nsum;
+            q.D = p[i0].dX;
+            q.ldd = K;
+            f += 2.0 * T * K * (double)(nsum + (lora ? m * r : 0));
+        }
+    }
+    if (k < 2 || !gemm_multi_fits(pr, k, T)) return false;
+    *np = k;
+    *flop = f;
+    return true;
 }
 
 lsn_status lora_layer_fwd(int n, const lsn_lora_proj* p, int64_t T, int r, float scale, void* ws, size_t ws_bytes,
@@ -736,6 +810,14 @@ lsn_status lora_layer_fwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
         if ((s = timed_down_batch(nd, dn, true, r, lanes.side())) != LSN_OK) return s;
         if ((s = layer_dequant(n, p, deq, w, lanes.main())) != LSN_OK) return s;
         if ((s = lanes.barrier()) != LSN_OK) return s;
+        GemmProblem pr[LSN_LAYER_MAX_PROJ];
+        int np = 0;
+        double flop = 0.0;
+        if (grouped_problems(n, p, g, T, r, w, false, pr, &np, &flop)) {
+            TimingScope ts(LSN_K_GEMM_FWD, flop, lanes.main());
+            if ((s = launch_gemm_multi(pr, np, false, T, r, w.err, lanes.main())) != LSN_OK) return s;
+            return lanes.join();
+        }
     }
     // Merged: after the first GEMM, the other projections' GEMMs as one
     // launch on the side lane, right behind their down projections (so it
@@ -854,6 +936,18 @@ lsn_status lora_layer_bwd(int n, const lsn_lora_proj* p, int64_t T, int r, float
         tg[nt++] = TgSpec{p[i].u ? p[i].u : w.u32[i], p[i].dY, p[i].dB, T, N, false, accumulate, scale};
     }
     if ((s = timed_tgrad_batch(nt, tg, r, lanes.side())) != LSN_OK) return s;
+    if (T > 0 && !early) {
+        // Groups (or a call whose first projection runs with the adapter off):
+        // every input-gradient GEMM in one merged launch on the main lane.
+        GemmProblem pr[LSN_LAYER_MAX_PROJ];
+        int np = 0;
+        double flop = 0.0;
+        if (grouped_problems(n, p, g, T, r, w, true, pr, &np, &flop)) {
+            TimingScope ts(LSN_K_GEMM_BWD, flop, lanes.main());
+            if ((s = launch_gemm_multi(pr, np, true, T, r, w.err, lanes.main())) != LSN_OK) return s;
+            return lanes.join();
+        }
+    }
     if (T > 0) {
         // Merged: after the first GEMM, the other projections' input-gradient
         // GEMMs as one launch on the main lane (the token reductions keep the

@@ -116,7 +116,11 @@ constexpr int kMultiMaxProb = 8;
 constexpr int kMultiMaxUnits = 80;
 constexpr int kMultiMaxTiles = 5120;
 struct MultiProbs {
-    CUtensorMap a[kMultiMaxProb], b[kMultiMaxProb], la[kMultiMaxProb], lb[kMultiMaxProb];
+    // Problem i's A operand may be split along the contraction like a grouped
+    // GEMM's: K-blocks [a_kb[i][j], a_kb[i][j+1]) from map a[i * kMaxSeg + j].
+    CUtensorMap a[kMultiMaxProb * kMaxSeg], b[kMultiMaxProb], la[kMultiMaxProb], lb[kMultiMaxProb];
+    int na[kMultiMaxProb];
+    int a_kb[kMultiMaxProb][kMaxSeg + 1];
     int nprob;
     int tile0[kMultiMaxProb + 1];
     int N[kMultiMaxProb];
@@ -416,7 +420,7 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
     if (warp == 0 && lane == 0) {
         if constexpr (MULTI) {
             for (int i = 0; i < mp->nprob; ++i) {
-                tma_prefetch_desc(&mp->a[i]);
+                for (int j = 0; j < mp->na[i]; ++j) tma_prefetch_desc(&mp->a[i * kMaxSeg + j]);
                 tma_prefetch_desc(&mp->b[i]);
                 if (mp->lora_k16[i] > 0) { tma_prefetch_desc(&mp->la[i]); tma_prefetch_desc(&mp->lb[i]); }
             }
@@ -465,9 +469,10 @@ __global__ void __launch_bounds__(Cfg<PAIR, BN, B_MN>::THREADS, 1)
                     int ka;
                     const int kc = lora ? 0 : kb * BK;                       // contraction coordinate of B
                     if constexpr (MULTI) {
-                        ma = lora ? &mp->la[pi] : &mp->a[pi];
+                        while (!lora && ai + 1 < mp->na[pi] && kb >= mp->a_kb[pi][ai + 1]) ++ai;
+                        ma = lora ? &mp->la[pi] : &mp->a[pi * kMaxSeg + ai];
                         mbp = lora ? &mp->lb[pi] : &mp->b[pi];
-                        ka = kc;
+                        ka = lora ? 0 : (kb - mp->a_kb[pi][ai]) * BK;
                     } else {
                         while (!lora && ai + 1 < p.na && kb >= p.a_kb[ai + 1]) ++ai;
                         ma = lora ? &tmLA : &tmA.m[ai];
@@ -1311,26 +1316,41 @@ lsn_status launch_gemm_multi(const GemmProblem* pr, int n, bool b_mn, int64_t M,
     lsn_status s;
     for (int i = 0; i < n; ++i) {
         const GemmProblem& q = pr[i];
-        const int ri = q.LA ? r : 0;
-        if ((s = make_map(&mp.a[i], q.A, q.Kc, M, q.lda, SUB, BM)) != LSN_OK) return s;
+        const int ri = q.LA ? (q.lr > 0 ? q.lr : r) : 0;
+        const int64_t ld_la = q.ld_la > 0 ? q.ld_la : ri;
+        if (q.na < 1 || q.na > kMaxSeg) return fail(LSN_ERR_INVALID_ARG, "multi-problem GEMM: bad A part count");
+        int64_t kb_acc = 0;
+        for (int j = 0; j < q.na; ++j) {
+            const int64_t akc = q.na == 1 ? q.Kc : q.a_kc[j];
+            if ((s = make_map(&mp.a[i * kMaxSeg + j], q.A[j], akc, M, q.lda[j], SUB, BM)) != LSN_OK) return s;
+            if (j + 1 < q.na && akc % BK != 0)
+                return fail(LSN_ERR_INVALID_ARG, "multi-problem GEMM: inner A parts must be multiples of 128 wide");
+            mp.a_kb[i][j] = (int)kb_acc;
+            kb_acc += (akc + BK - 1) / BK;
+        }
+        mp.a_kb[i][q.na] = (int)kb_acc;
+        mp.na[i] = q.na;
+        for (int j = q.na; j < kMaxSeg; ++j) mp.a[i * kMaxSeg + j] = mp.a[i * kMaxSeg];
         if (!b_mn) {
             if ((s = make_map(&mp.b[i], q.B, q.Kc, q.N, q.ldb, SUB, 128)) != LSN_OK) return s;
         } else {
             if ((s = make_map(&mp.b[i], q.B, q.N, q.Kc, q.ldb, 64, BK)) != LSN_OK) return s;
         }
         if (ri > 0) {
-            if ((s = make_map(&mp.la[i], q.LA, ri, M, ri, SUB, BM)) != LSN_OK) return s;
+            if ((s = make_map(&mp.la[i], q.LA, ri, M, ld_la, SUB, BM)) != LSN_OK) return s;
             if (!b_mn) {
                 if ((s = make_map(&mp.lb[i], q.LB, ri, q.N, ri, SUB, 128)) != LSN_OK) return s;
             } else {
                 if ((s = make_map(&mp.lb[i], q.LB, q.N, ri, q.N, 64, BK)) != LSN_OK) return s;
             }
         } else {                                        // no LoRA term: never read
-            mp.la[i] = mp.a[i];
+            mp.la[i] = mp.a[i * kMaxSeg];
             mp.lb[i] = mp.b[i];
         }
         mp.N[i] = (int)q.N;
         mp.num_kb[i] = (int)((q.Kc + BK - 1) / BK);
+        if (mp.num_kb[i] != mp.a_kb[i][q.na])
+            return fail(LSN_ERR_INVALID_ARG, "multi-problem GEMM: A parts do not add up to Kc");
         mp.lora_k16[i] = (ri + 15) / 16;
         mp.D[i] = q.D;
         mp.ldd[i] = q.ldd;

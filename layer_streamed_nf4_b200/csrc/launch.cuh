@@ -97,15 +97,23 @@ void dequant_set_spare_sms(int n);
 int dequant_spare_sms();
 
 // One of several independent GEMMs launched together (launch_gemm_multi): the
-// arguments of launch_gemm for one problem, on the 2-SM kernel; LA == NULL:
-// no LoRA term.
+// arguments of launch_gemm for one problem, on the 2-SM kernel.  A may be
+// split along the contraction into na parts as for a grouped GEMM (part j:
+// A[j] [M, a_kc[j]] with row stride lda[j]; all parts but the last a multiple
+// of 128 wide; na == 1: A[0] covers Kc).  The LoRA term: LA [M, lr] with row
+// stride ld_la (lr = 0 or LA == NULL: none; lr == 0 means the call's r), LB
+// [N, lr] (K-major B) or [lr, N] (MN-major B).
 struct GemmProblem {
-    const uint16_t* A = nullptr;
-    int64_t lda = 0;
+    int na = 1;
+    const uint16_t* A[kGemmMaxSeg] = {};
+    int64_t lda[kGemmMaxSeg] = {};
+    int64_t a_kc[kGemmMaxSeg] = {};
     const uint16_t* B = nullptr;
     int64_t ldb = 0;
     const uint16_t* LA = nullptr;
     const uint16_t* LB = nullptr;
+    int lr = 0;
+    int64_t ld_la = 0;
     int64_t N = 0, Kc = 0;
     uint16_t* D = nullptr;
     int64_t ldd = 0;
